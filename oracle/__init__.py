@@ -1,0 +1,125 @@
+"""Plain fp64 CPU oracle for the Mamba-3 mixer recurrence.
+
+TEST INFRASTRUCTURE ONLY.  The oracle is the slow, obviously correct reference
+that the CUDA path is checked against; it is imported by ``tests/``, by
+``__graft_entry__.smoke()`` and by the CPU-baseline leg of ``bench.py`` and by
+nothing else.  It shares no code with the CUDA library in
+``state_space_model_06_b200``, and neither side imports the other.
+
+The arithmetic lives in ``m3_oracle.c`` (sequential fp64 loop over tokens,
+OpenMP over independent (batch, head) pairs).  This module only builds that
+file with gcc and marshals numpy float64 arrays into it.
+
+Every function here follows the Mamba-3 paper summary, "Technical Approach":
+Proposition 1 (exponential-trapezoidal recurrence), Propositions 2-4 (complex
+transition as a data-dependent rotation of state pairs) and the MIMO
+formulation (rank-R input and readout).  Parity pins for each part live in
+``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "m3_oracle.c")
+_LIB = os.path.join(_HERE, "libm3_oracle.so")
+
+THETA_IS_ANGLE = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile ``m3_oracle.c`` into ``libm3_oracle.so`` next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("batch", "nheads", "ngroups", "headdim", "dstate", "rank")]
+
+
+_libs = {}
+
+
+def _load(path=None):
+    """Load the oracle library (``path`` lets a test load a deliberately broken copy)."""
+    path = path or build()
+    if path not in _libs:
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.m3o_scan.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int64, ctypes.c_uint32] + \
+            [dp] * 12 + [ctypes.c_int]
+        lib.m3o_scan.restype = ctypes.c_int
+        lib.m3o_max_threads.restype = ctypes.c_int
+        _libs[path] = lib
+    return _libs[path]
+
+
+def max_threads() -> int:
+    return int(_load().m3o_max_threads())
+
+
+def _f64(a, shape, name):
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    if tuple(a.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {a.shape}")
+    return a
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double)) if a is not None else None
+
+
+def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
+         theta_is_angle: bool = False, nthreads: int = 0, lib_path=None):
+    """Run the recurrence over T tokens.
+
+    Shapes: x [b,T,H,R,P]; B, C [b,T,G,R,N]; dt, A, lam [b,T,H];
+    theta [b,T,G,N/2]; D [H] or None; h0 [b,H,N,P] or None (zeros);
+    x_prev [b,H,R,P] / B_prev [b,G,R,N] or None (fresh sequence: zeros).
+
+    Returns (y [b,T,H,R,P], h_T, x_prev_out, B_prev_out), all float64.
+    """
+    x = np.asarray(x)
+    b, T, H, R, P = x.shape
+    G, N = np.asarray(B).shape[2], np.asarray(B).shape[4]
+    x = _f64(x, (b, T, H, R, P), "x")
+    B = _f64(B, (b, T, G, R, N), "B")
+    C = _f64(C, (b, T, G, R, N), "C")
+    dt = _f64(dt, (b, T, H), "dt")
+    A = _f64(A, (b, T, H), "A")
+    lam = _f64(lam, (b, T, H), "lam")
+    theta = _f64(theta, (b, T, G, N // 2), "theta")
+    D = None if D is None else _f64(D, (H,), "D")
+    h = np.zeros((b, H, N, P)) if h0 is None else _f64(h0, (b, H, N, P), "h0").copy()
+    xp = np.zeros((b, H, R, P)) if x_prev is None else _f64(x_prev, (b, H, R, P), "x_prev").copy()
+    bp = np.zeros((b, G, R, N)) if B_prev is None else _f64(B_prev, (b, G, R, N), "B_prev").copy()
+    y = np.zeros((b, T, H, R, P))
+    dims = _Dims(b, H, G, P, N, R)
+    rc = _load(lib_path).m3o_scan(ctypes.byref(dims), T, THETA_IS_ANGLE if theta_is_angle else 0,
+                          _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta),
+                          _ptr(D), _ptr(h), _ptr(xp), _ptr(bp), _ptr(y), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"m3o_scan rejected its arguments (code {rc})")
+    return y, h, xp, bp
+
+
+def decode_step(x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev,
+                theta_is_angle: bool = False, nthreads: int = 0):
+    """One decode token: x [b,H,R,P], B/C [b,G,R,N], dt/A/lam [b,H], theta [b,G,N/2].
+
+    Identical to ``scan`` with T = 1; returns (y [b,H,R,P], h, x_prev, B_prev).
+    """
+    ins = [np.asarray(v)[:, None] for v in (x, B, C, dt, A, lam, theta)]
+    y, h, xp, bp = scan(*ins, D=D, h0=h, x_prev=x_prev, B_prev=B_prev,
+                        theta_is_angle=theta_is_angle, nthreads=nthreads)
+    return y[:, 0], h, xp, bp

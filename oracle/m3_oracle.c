@@ -1,0 +1,180 @@
+/*
+ * m3_oracle.c -- plain fp64 CPU oracle for the Mamba-3 mixer recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously correct reference
+ * that the CUDA path is checked against.  It shares no code, header, table or
+ * constant with the CUDA library, and nothing on the product path may call it:
+ * only tests, the smoke check and the bench's CPU-baseline leg load it.
+ *
+ * What it computes (Mamba-3 paper summary, "Technical Approach" section):
+ *
+ *   Exponential-trapezoidal recurrence, Proposition 1:
+ *       h_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}^T + gamma_t B_t x_t^T
+ *       alpha_t = exp(dt_t A_t), beta_t = (1 - lam_t) dt_t alpha_t, gamma_t = lam_t dt_t
+ *
+ *   Complex transition realised as a real block-diagonal rotation, Proposition 2:
+ *       the transition exp(dt (A + i theta)) = alpha_t R_t, where R_t rotates each
+ *       state pair [h_{2i}, h_{2i+1}] by the angle dt_t theta_t[i], with
+ *       R(phi) = [[cos phi, -sin phi], [sin phi, cos phi]].
+ *
+ *   Complex + exponential-trapezoidal, Proposition 4, moved back from the RoPE
+ *   frame to the original frame (Propositions 2 and 3): the left-endpoint
+ *   trapezoid term carries the full transition, so it is rotated as well:
+ *       h_t = R_t (alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}^T) + gamma_t B_t x_t^T
+ *
+ *   MIMO ("Multi-Input, Multi-Output Formulation"): B_t is N x R, x_t is P x R and
+ *   the input term is the rank-R sum  sum_r B_t[:,r] x_t[:,r]^T.  The readout is
+ *   Y_t = H_t^T C_t (P x R), plus the per-head skip D * x_t.
+ *
+ *   Sequence start ("Parallel representation under SSD"): the unrolling starts
+ *   from h_0 = gamma_0 B_0 x_0, i.e. a fresh state has h = 0 and no previous
+ *   token (x_{-1} = 0, B_{-1} = 0).  Across calls the previous token (x, B) is
+ *   carried with the state so that beta_0 of the next call sees it.
+ *
+ * Layouts (row-major, last index contiguous), all fp64:
+ *   x, y      [b][T][H][R][P]          B, C   [b][T][G][R][N]
+ *   dt, A, lam[b][T][H]                theta  [b][T][G][N/2]     D [H] (may be NULL)
+ *   h         [b][H][N][P]   (in: initial state, out: final state, original frame)
+ *   x_prev    [b][H][R][P]   (in/out)  B_prev [b][G][R][N] (in/out)
+ * Head h reads group g = h / (H / G).
+ *
+ * Parallelised over independent (batch, head) pairs with OpenMP only; the time
+ * loop is the plain sequential recurrence.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define M3O_THETA_IS_ANGLE 1u
+
+typedef struct {
+    int32_t batch, nheads, ngroups, headdim, dstate, rank;
+} m3o_dims;
+
+/* One token of the recurrence for one head, in place on h / xp / bp. */
+static void m3o_step(int N, int P, int R, double dt, double a, double lam,
+                     const double* th, const double* X, const double* Bt,
+                     const double* Ct, double Dh, double* h, double* xp, double* bp,
+                     double* Y, unsigned flags)
+{
+    const double alpha = exp(dt * a);
+    const double beta = (1.0 - lam) * dt * alpha;
+    const double gamma = lam * dt;
+
+    /* M = alpha h + beta * sum_r Bp[:,r] Xp[:,r]^T */
+    for (int n = 0; n < N; ++n)
+        for (int p = 0; p < P; ++p) {
+            double v = 0.0;
+            for (int r = 0; r < R; ++r) v += bp[r * N + n] * xp[r * P + p];
+            h[n * P + p] = alpha * h[n * P + p] + beta * v;
+        }
+
+    /* rotate each state pair (2i, 2i+1) by phi_i = dt * theta_i */
+    for (int i = 0; i < N / 2; ++i) {
+        const double phi = (flags & M3O_THETA_IS_ANGLE) ? th[i] : dt * th[i];
+        const double c = cos(phi), s = sin(phi);
+        double* r0 = h + (2 * i) * P;
+        double* r1 = h + (2 * i + 1) * P;
+        for (int p = 0; p < P; ++p) {
+            const double m0 = r0[p], m1 = r1[p];
+            r0[p] = c * m0 - s * m1;
+            r1[p] = s * m0 + c * m1;
+        }
+    }
+
+    /* + gamma * sum_r B_t[:,r] X_t[:,r]^T */
+    for (int n = 0; n < N; ++n)
+        for (int p = 0; p < P; ++p) {
+            double v = 0.0;
+            for (int r = 0; r < R; ++r) v += Bt[r * N + n] * X[r * P + p];
+            h[n * P + p] += gamma * v;
+        }
+
+    /* Y[r][p] = sum_n h[n][p] C_t[n][r] + D x_t[r][p] */
+    for (int r = 0; r < R; ++r)
+        for (int p = 0; p < P; ++p) {
+            double v = 0.0;
+            for (int n = 0; n < N; ++n) v += h[n * P + p] * Ct[r * N + n];
+            Y[r * P + p] = v + Dh * X[r * P + p];
+        }
+
+    memcpy(xp, X, sizeof(double) * (size_t)R * P);
+    memcpy(bp, Bt, sizeof(double) * (size_t)R * N);
+}
+
+static int m3o_check(const m3o_dims* d, int64_t T)
+{
+    if (!d) return 1;
+    if (d->batch < 0 || d->nheads <= 0 || d->ngroups <= 0 || d->headdim <= 0 ||
+        d->dstate <= 0 || d->rank <= 0 || T < 0)
+        return 2;
+    if (d->nheads % d->ngroups) return 2;
+    if (d->dstate % 2) return 2;
+    return 0;
+}
+
+/*
+ * Run T tokens of the recurrence for every (batch, head).  The state (h, x_prev,
+ * B_prev) is updated in place.  Returns 0 on success, non-zero on bad arguments.
+ * nthreads <= 0 uses the OpenMP default.
+ */
+int m3o_scan(const m3o_dims* d, int64_t T, uint32_t flags, const double* x,
+             const double* B, const double* C, const double* dt, const double* A,
+             const double* lam, const double* theta, const double* D, double* h,
+             double* x_prev, double* B_prev, double* y, int nthreads)
+{
+    int rc = m3o_check(d, T);
+    if (rc) return rc;
+    const int Bn = d->batch, H = d->nheads, G = d->ngroups, P = d->headdim,
+              N = d->dstate, R = d->rank;
+    const int hpg = H / G;
+    if (T == 0 || Bn == 0) return 0;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (int64_t bh = 0; bh < (int64_t)Bn * H; ++bh) {
+        const int b = (int)(bh / H), hh = (int)(bh % H), g = hh / hpg;
+        double* bp = (double*)malloc(sizeof(double) * (size_t)R * N);
+        memcpy(bp, B_prev + ((size_t)b * G + g) * R * N, sizeof(double) * (size_t)R * N);
+        double* xp = x_prev + ((size_t)b * H + hh) * R * P;
+        double* hs = h + ((size_t)b * H + hh) * N * P;
+        const double Dh = D ? D[hh] : 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            const size_t bt = (size_t)b * T + t;
+            m3o_step(N, P, R, dt[bt * H + hh], A[bt * H + hh], lam[bt * H + hh],
+                     theta + (bt * G + g) * (N / 2), x + (bt * H + hh) * R * P,
+                     B + (bt * G + g) * R * N, C + (bt * G + g) * R * N, Dh, hs, xp, bp,
+                     y + (bt * H + hh) * R * P, flags);
+        }
+        free(bp);
+    }
+    /* B_prev <- B_{T-1}, once per group (every head of the group read the old value) */
+    for (int b = 0; b < Bn; ++b)
+        memcpy(B_prev + (size_t)b * G * R * N, B + ((size_t)b * T + (T - 1)) * G * R * N,
+               sizeof(double) * (size_t)G * R * N);
+    return 0;
+}
+
+/* A single decode step is the same recurrence for one token (T = 1). */
+int m3o_decode(const m3o_dims* d, uint32_t flags, const double* x, const double* B,
+               const double* C, const double* dt, const double* A, const double* lam,
+               const double* theta, const double* D, double* h, double* x_prev,
+               double* B_prev, double* y, int nthreads)
+{
+    return m3o_scan(d, 1, flags, x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev, y,
+                    nthreads);
+}
+
+int m3o_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,204 @@
+"""Independent numpy restatements of the Mamba-3 recurrence, used to pin the oracle.
+
+Each route below is a different reading of the same statement in the Mamba-3
+paper summary ("Technical Approach"); none shares code with ``oracle/``.  A
+plausible oracle mistake (a dropped beta term, a rotation sign, a transposed
+operand, a pair-index slip) makes at least one of them disagree.
+
+Array layouts match the library: x [b,T,H,R,P], B/C [b,T,G,R,N], dt/A/lam
+[b,T,H], theta [b,T,G,N/2], D [H], h [b,H,N,P], x_prev [b,H,R,P],
+B_prev [b,G,R,N].  Everything is float64 (complex128 for the complex route).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _heads(x, B):
+    b, T, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    return b, T, H, R, P, G, N, H // G
+
+
+def euler_loop(x, B, C, dt, A, D=None, h0=None):
+    """Exponential-Euler (Mamba-2) recurrence, Remark 2 with lam = 1, theta = 0.
+
+    h_t = exp(dt_t A_t) h_{t-1} + dt_t B_t x_t^T;  Y_t = h_t^T C_t + D x_t.
+    """
+    b, T, H, R, P, G, N, hpg = _heads(x, B)
+    y = np.zeros_like(x, dtype=np.float64)
+    hT = np.zeros((b, H, N, P))
+    for bi in range(b):
+        for h in range(H):
+            g = h // hpg
+            st = np.zeros((N, P)) if h0 is None else h0[bi, h].astype(np.float64).copy()
+            Dh = 0.0 if D is None else D[h]
+            for t in range(T):
+                st = np.exp(dt[bi, t, h] * A[bi, t, h]) * st + \
+                    dt[bi, t, h] * B[bi, t, g].T @ x[bi, t, h]
+                y[bi, t, h] = (st.T @ C[bi, t, g].T).T + Dh * x[bi, t, h]
+            hT[bi, h] = st
+    return y, hT
+
+
+def complex_route(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
+                  theta_is_angle=False):
+    """Complex-valued SSM, "Complex-Valued State Space Models" (h in C^{N/2}).
+
+    Transition z_t = exp(dt_t (A_t + i theta_t)); the generalised trapezoid of the
+    state-input integral puts the full transition on the left endpoint:
+        h_t = z_t h_{t-1} + (1 - lam_t) dt_t z_t v_{t-1} + lam_t dt_t v_t,
+    with v_t = (B + i B_hat) x_t.  Readout y = Re((C + i C_hat)^T h).  The real
+    projections stack as B = [B; B_hat], C = [C; -C_hat] (Proposition 2); state
+    pair i is stored interleaved at (2i, 2i+1).
+    """
+    b, T, H, R, P, G, N, hpg = _heads(x, B)
+    y = np.zeros(x.shape)
+    hT = np.zeros((b, H, N, P))
+    for bi in range(b):
+        for h in range(H):
+            g = h // hpg
+            if h0 is None:
+                hc = np.zeros((N // 2, P), dtype=np.complex128)
+            else:
+                hc = h0[bi, h, 0::2] + 1j * h0[bi, h, 1::2]
+            if x_prev is None:
+                v_prev = np.zeros((N // 2, P), dtype=np.complex128)
+            else:
+                bpc = B_prev[bi, g, :, 0::2] + 1j * B_prev[bi, g, :, 1::2]   # [R, N/2]
+                v_prev = bpc.T @ x_prev[bi, h]                                 # [N/2, P]
+            Dh = 0.0 if D is None else D[h]
+            for t in range(T):
+                d, a, l = dt[bi, t, h], A[bi, t, h], lam[bi, t, h]
+                ang = theta[bi, t, g] if theta_is_angle else d * theta[bi, t, g]
+                z = np.exp(d * a + 1j * ang)[:, None]                          # [N/2, 1]
+                bc = B[bi, t, g, :, 0::2] + 1j * B[bi, t, g, :, 1::2]          # [R, N/2]
+                v = bc.T @ x[bi, t, h]
+                hc = z * hc + (1.0 - l) * d * z * v_prev + l * d * v
+                cc = C[bi, t, g, :, 0::2] - 1j * C[bi, t, g, :, 1::2]          # C + i C_hat
+                y[bi, t, h] = np.real(cc @ hc) + Dh * x[bi, t, h]
+                v_prev = v
+            hT[bi, h, 0::2] = hc.real
+            hT[bi, h, 1::2] = hc.imag
+    return y, hT
+
+
+def _rot_pairs(vec, ang):
+    """Rotate interleaved pairs of ``vec`` (..., N) by angles ``ang`` (N/2,)."""
+    c, s = np.cos(ang), np.sin(ang)
+    out = np.empty_like(vec)
+    out[..., 0::2] = c * vec[..., 0::2] - s * vec[..., 1::2]
+    out[..., 1::2] = s * vec[..., 0::2] + c * vec[..., 1::2]
+    return out
+
+
+def rope_route(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
+               theta_is_angle=False):
+    """Proposition 4 read literally, in the rotated (RoPE) frame.
+
+    psi_t = sum_{k<=t} dt_k theta_k (per pair); Q_t = R(psi_t).
+        g_t = alpha_t g_{t-1} + beta_t Q_{t-1}^T B_{t-1} x_{t-1}^T + gamma_t Q_t^T B_t x_t^T
+        y_t = (Q_t^T C_t)^T g_t
+    with g_{-1} = h0 and Q_{-1} = I; the original-frame state is h_T = Q_T g_T.
+    """
+    b, T, H, R, P, G, N, hpg = _heads(x, B)
+    y = np.zeros(x.shape)
+    hT = np.zeros((b, H, N, P))
+    for bi in range(b):
+        for h in range(H):
+            g = h // hpg
+            st = np.zeros((N, P)) if h0 is None else h0[bi, h].copy()
+            psi = np.zeros(N // 2)
+            if x_prev is None:
+                bt_prev = np.zeros((R, N))
+                xprev = np.zeros((R, P))
+            else:
+                bt_prev = B_prev[bi, g].copy()        # rotated by Q_{-1} = I
+                xprev = x_prev[bi, h]
+            Dh = 0.0 if D is None else D[h]
+            for t in range(T):
+                d, a, l = dt[bi, t, h], A[bi, t, h], lam[bi, t, h]
+                ang = theta[bi, t, g] if theta_is_angle else d * theta[bi, t, g]
+                psi = psi + ang
+                al = np.exp(d * a)
+                be = (1.0 - l) * d * al
+                ga = l * d
+                bt = _rot_pairs(B[bi, t, g], -psi)    # Q_t^T B_t
+                ct = _rot_pairs(C[bi, t, g], -psi)    # Q_t^T C_t
+                st = al * st + be * bt_prev.T @ xprev + ga * bt.T @ x[bi, t, h]
+                y[bi, t, h] = (st.T @ ct.T).T + Dh * x[bi, t, h]
+                bt_prev, xprev = bt, x[bi, t, h]
+            # h_T = Q_T g_T: rotate rows of the state by +psi
+            hT[bi, h] = _rot_pairs(st.T, psi).T
+    return y, hT
+
+
+def bruteforce_txt(x, B, C, dt, A, lam, theta, D=None, theta_is_angle=False):
+    """Materialised parallel form, "Parallel representation under SSD".
+
+    Y = (L o C~ B~^T) X with L = L_decay @ L_band, where L_decay[t,s] is the
+    product alpha_{s+1}..alpha_t (1 on the diagonal) and L_band holds gamma_t on
+    the diagonal and beta_t on the first sub-diagonal.  B~, C~ are B, C rotated
+    by the cumulative angle (Proposition 4).  Fresh sequence: h0 = 0, no
+    previous token.  For MIMO the score matrix runs over (token, rank) pairs
+    and L is shared by the R x R blocks.
+    """
+    b, T, H, R, P, G, N, hpg = _heads(x, B)
+    y = np.zeros(x.shape)
+    for bi in range(b):
+        for h in range(H):
+            g = h // hpg
+            d, a, l = dt[bi, :, h], A[bi, :, h], lam[bi, :, h]
+            al = np.exp(d * a)
+            be = (1.0 - l) * d * al
+            ga = l * d
+            Ld = np.zeros((T, T))
+            for t in range(T):
+                for s in range(t + 1):
+                    Ld[t, s] = np.prod(al[s + 1:t + 1])
+            Lb = np.diag(ga)
+            for t in range(1, T):
+                Lb[t, t - 1] = be[t]
+            L = Ld @ Lb
+            ang = theta[bi, :, g] if theta_is_angle else d[:, None] * theta[bi, :, g]
+            psi = np.cumsum(ang, axis=0)                          # [T, N/2]
+            bt = np.stack([_rot_pairs(B[bi, t, g], -psi[t]) for t in range(T)])  # [T,R,N]
+            ct = np.stack([_rot_pairs(C[bi, t, g], -psi[t]) for t in range(T)])
+            S = np.einsum("trn,usn->trus", ct, bt)                # [T,R,T,R]
+            M = S * L[:, None, :, None]
+            Y = np.einsum("trus,usp->trp", M, x[bi, :, h])
+            Dh = 0.0 if D is None else D[h]
+            y[bi, :, h] = Y + Dh * x[bi, :, h]
+    return y
+
+
+def implicit_conv_route(x, B, C, dt, A, lam, D=None, h0=None, x_prev=None, B_prev=None):
+    """Remark 4 (theta = 0): width-2 data-dependent convolution on v_t = B_t x_t^T,
+
+        v~_t = beta_t v_{t-1} + gamma_t v_t,   h_t = alpha_t h_{t-1} + v~_t.
+    """
+    b, T, H, R, P, G, N, hpg = _heads(x, B)
+    y = np.zeros(x.shape)
+    hT = np.zeros((b, H, N, P))
+    for bi in range(b):
+        for h in range(H):
+            g = h // hpg
+            st = np.zeros((N, P)) if h0 is None else h0[bi, h].copy()
+            v_prev = np.zeros((N, P)) if x_prev is None else B_prev[bi, g].T @ x_prev[bi, h]
+            Dh = 0.0 if D is None else D[h]
+            for t in range(T):
+                d, a, l = dt[bi, t, h], A[bi, t, h], lam[bi, t, h]
+                al = np.exp(d * a)
+                v = B[bi, t, g].T @ x[bi, t, h]
+                vt = (1.0 - l) * d * al * v_prev + l * d * v
+                st = al * st + vt
+                y[bi, t, h] = (st.T @ C[bi, t, g].T).T + Dh * x[bi, t, h]
+                v_prev = v
+            hT[bi, h] = st
+    return y, hT
+
+
+def lti_exact(a, b, omega, tau):
+    """Exact solution of h' = a h + b sin(omega tau), h(0) = 0 (variation of constants)."""
+    return b * (omega * np.exp(a * tau) - omega * np.cos(omega * tau) - a * np.sin(omega * tau)) \
+        / (a * a + omega * omega)
