@@ -1,0 +1,157 @@
+/*
+ * m3.h -- C ABI of the Mamba-3 mixer hot path on B200 (sm_100a).
+ *
+ * The library computes the Mamba-3 SSM recurrence (Mamba-3 paper summary,
+ * "Technical Approach"):
+ *
+ *   Proposition 1 (exponential-trapezoidal discretisation):
+ *     h_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}^T + gamma_t B_t x_t^T,
+ *     alpha_t = exp(dt_t A_t), beta_t = (1 - lam_t) dt_t alpha_t, gamma_t = lam_t dt_t
+ *   Propositions 2-4 (complex-valued transition as a data-dependent rotation):
+ *     every state pair (2i, 2i+1) is rotated by dt_t theta_t[i] each step, and the
+ *     left-endpoint (beta) term is rotated with the previous state, so in the
+ *     original frame  h_t = R_t (alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}^T)
+ *                          + gamma_t B_t x_t^T
+ *   MIMO ("Multi-Input, Multi-Output Formulation"): B_t, C_t are N x R and x_t is
+ *     P x R; the input term is a rank-R sum and the readout is P x R:
+ *     Y_t = h_t^T C_t + D x_t   (D is a per-head scalar skip; SISO is R = 1)
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory and never synchronises the stream, except in
+ *     m3_query_status.  Calls are asynchronous and ordered on `stream` (a
+ *     cudaStream_t passed as void*; NULL is the legacy default stream).
+ *   - Row-major layouts, last index contiguous:
+ *       x, y        [batch][T][H][R][P]     io dtype
+ *       B, C        [batch][T][G][R][N]     io dtype   (shared by the H/G heads of a group)
+ *       dt, A, lam  [batch][T][H]           float      (dt after softplus, lam after sigmoid)
+ *       theta       [batch][T][G][N/2]      float      (angle per state pair; see flags)
+ *       D           [H]                     float      (may be NULL: no skip term)
+ *       state.h     [batch][H][N][P]        float      (original frame)
+ *       state.x_prev[batch][H][R][P]        io dtype   (previous token's x)
+ *       state.B_prev[batch][G][R][N]        io dtype   (previous token's B)
+ *     Head h reads group g = h / (H/G).  The decode step drops the T axis.
+ *     State pair i is stored interleaved at rows (2i, 2i+1).
+ *   - Errors: arguments are validated on the host before anything is launched;
+ *     a failed check returns a status code and touches no memory.  Device code
+ *     never traps; a bounded device-side wait that gives up writes
+ *     M3_ERR_TIMEOUT into the workspace status word (see m3_query_status).
+ *   - Value ranges are the caller's contract: dt > 0, A <= 0, lam in [0, 1].
+ */
+#ifndef M3_H
+#define M3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    M3_OK = 0,
+    M3_ERR_NULL = 1,        /* a required pointer is NULL */
+    M3_ERR_SHAPE = 2,       /* dims / seqlen / chunk out of range or inconsistent */
+    M3_ERR_DTYPE = 3,       /* unknown io dtype */
+    M3_ERR_ALIGN = 4,       /* a pointer is not aligned as documented */
+    M3_ERR_UNSUPPORTED = 5, /* valid arguments that no kernel of this build handles */
+    M3_ERR_WORKSPACE = 6,   /* workspace missing or smaller than m3_scan_workspace_bytes */
+    M3_ERR_LAUNCH = 7,      /* a kernel launch failed (cudaGetLastError) */
+    M3_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up (reported by m3_query_status) */
+    M3_ERR_CUDA = 9         /* another CUDA runtime call failed */
+} m3_status;
+
+typedef enum { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
+
+/* Problem dimensions.  batch >= 1, H % G == 0, N even.  io_dtype is an m3_dtype. */
+typedef struct {
+    int32_t batch;     /* b */
+    int32_t nheads;    /* H */
+    int32_t ngroups;   /* G: B, C and theta are shared by H/G heads */
+    int32_t headdim;   /* P */
+    int32_t dstate;    /* N (even: N/2 complex state pairs) */
+    int32_t rank;      /* R: 1 = SISO, > 1 = MIMO */
+    int32_t io_dtype;  /* m3_dtype of x, B, C, y, x_prev, B_prev */
+} m3_dims;
+
+/* Resumable recurrent state (caller-owned device memory, layouts above).
+ * h must be 16-byte aligned; x_prev and B_prev 16-byte aligned. */
+typedef struct {
+    float* h;
+    void* x_prev;
+    void* B_prev;
+} m3_state;
+
+/* Flags (bitwise OR). */
+#define M3_FLAG_THETA_IS_ANGLE 1u  /* theta already holds the per-step angle: the dt multiply is skipped */
+#define M3_FLAG_FORCE_SIMT 2u      /* m3_scan_fwd: run the sequential fp32 CUDA-core kernel */
+
+/* Bytes of each state buffer for `dims`.  Any out-pointer may be NULL. */
+m3_status m3_state_bytes(const m3_dims* dims, size_t* h_bytes, size_t* x_prev_bytes,
+                         size_t* B_prev_bytes);
+
+/* Start a fresh sequence: h <- h0 (or 0 when h0 is NULL), x_prev <- 0, B_prev <- 0.
+ * A fresh sequence has no previous token, so its first step has no beta term
+ * (the unrolling starts from h_0 = gamma_0 B_0 x_0, "Parallel representation
+ * under SSD").  h0, when given, is a device pointer in the state.h layout. */
+m3_status m3_state_init(const m3_dims* dims, m3_state* state, const float* h0, void* stream);
+
+/* Workspace bytes m3_scan_fwd needs for (dims, seqlen, chunk); at least 256
+ * (the status word).  The workspace is caller-owned device memory, 256-byte
+ * aligned, and must not be shared by calls that can overlap on the GPU. */
+m3_status m3_scan_workspace_bytes(const m3_dims* dims, int32_t seqlen, int32_t chunk,
+                                  size_t* bytes);
+
+/*
+ * Prefill: run `seqlen` tokens of the recurrence for every (batch, head),
+ * chunked parallel scan ("Parallel representation under SSD": the parallel
+ * masked form inside a chunk of `chunk` tokens, the recurrence across chunks).
+ *
+ *   in : x, B, C (io dtype), dt, A, lam, theta, D (float), state (h, x_prev, B_prev)
+ *   out: y [b][T][H][R][P] io dtype (rounded to nearest even from fp32);
+ *        state updated in place to the end of the sequence: h = h_T (original
+ *        frame), x_prev = x_{T-1}, B_prev = B_{T-1}.
+ *
+ * chunk must be 16, 32, 64 or 128; it only changes rounding, not the result.
+ * Pointers to x, B, C, y, state buffers and the workspace must be 16-byte
+ * aligned; float arrays 4-byte aligned.  seqlen == 0 is a no-op returning M3_OK
+ * (only dims, chunk and the state are validated; no other pointer is examined).
+ * bf16 io runs on the tcgen05 tensor-core kernel where the shape is supported
+ * (SISO N in {64,128}, P = 64; MIMO Q*R <= 256); other shapes and fp32 io run
+ * the sequential fp32 CUDA-core kernel.
+ */
+m3_status m3_scan_fwd(const m3_dims* dims, int32_t seqlen, int32_t chunk, const void* x,
+                      const void* B, const void* C, const float* dt, const float* A,
+                      const float* lam, const float* theta, const float* D, m3_state* state,
+                      void* y, void* workspace, size_t workspace_bytes, uint32_t flags,
+                      void* stream);
+
+/*
+ * Decode: one token of the recurrence for every (batch, head), fused in one
+ * pass over the fp32 state ("Multi-Input, Multi-Output Formulation", SISO/MIMO
+ * decode step, with the trapezoid and rotation of Propositions 1 and 4).
+ *
+ *   in : x [b][H][R][P], B, C [b][G][R][N] (io dtype), dt, A, lam [b][H],
+ *        theta [b][G][N/2], D [H] (may be NULL), state
+ *   out: y [b][H][R][P] io dtype; state updated in place (h, x_prev <- x,
+ *        B_prev <- B).
+ *
+ * Supported: N even <= 256, P % 4 == 0 and P <= 256, R <= 8.
+ */
+m3_status m3_decode_step(const m3_dims* dims, const void* x, const void* B, const void* C,
+                         const float* dt, const float* A, const float* lam,
+                         const float* theta, const float* D, m3_state* state, void* y,
+                         uint32_t flags, void* stream);
+
+/* Synchronise `stream` and report the device-side status word in `workspace`
+ * (M3_OK, or M3_ERR_TIMEOUT when a bounded wait gave up). */
+m3_status m3_query_status(const void* workspace, void* stream);
+
+/* Static English text for a status code. */
+const char* m3_status_string(m3_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M3_H */

@@ -1,0 +1,222 @@
+// m3_api.cu -- the C ABI (include/m3.h): host-side validation and dispatch.
+//
+// Every argument is checked here before anything is launched; the kernels assume
+// validated input.  Nothing in this file allocates device memory or synchronises,
+// except m3_query_status.
+#include <cstring>
+
+#include "m3_internal.h"
+
+using namespace m3;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;   // status block at the head of the workspace
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t io_bytes(int io_dtype) { return io_dtype == M3_BF16 ? 2 : 4; }
+
+m3_status check_dims(const m3_dims* d) {
+    if (!d) return M3_ERR_NULL;
+    if (d->io_dtype != M3_F32 && d->io_dtype != M3_BF16) return M3_ERR_DTYPE;
+    if (d->batch < 1 || d->nheads < 1 || d->ngroups < 1 || d->headdim < 1 || d->dstate < 2 ||
+        d->rank < 1)
+        return M3_ERR_SHAPE;
+    if (d->nheads % d->ngroups) return M3_ERR_SHAPE;
+    if (d->dstate % 2) return M3_ERR_SHAPE;
+    if (d->dstate > 1024 || d->headdim > 1024 || d->rank > 8) return M3_ERR_UNSUPPORTED;
+    return M3_OK;
+}
+
+m3_status check_state(const m3_state* st) {
+    if (!st || !st->h || !st->x_prev || !st->B_prev) return M3_ERR_NULL;
+    if (!aligned(st->h, 16) || !aligned(st->x_prev, 16) || !aligned(st->B_prev, 16))
+        return M3_ERR_ALIGN;
+    return M3_OK;
+}
+
+bool rank_has_kernel(int R) { return R == 1 || R == 2 || R == 3 || R == 4 || R == 8; }
+
+// SIMT prefill thread shape: ns lanes per state column (a power of two <= 32),
+// ppt pairs per lane; P * ns threads.
+bool simt_shape(int N, int P, int* ppt, int* ns) {
+    const int pairs = N / 2;
+    int n = 1;
+    while ((pairs + n - 1) / n > 8 && n < 32) n *= 2;
+    int p = (pairs + n - 1) / n;
+    while (P * n > 1024 && n > 1) {
+        n /= 2;
+        p = (pairs + n - 1) / n;
+    }
+    if (p > 32 || P * n > 1024) return false;
+    *ppt = p;
+    *ns = n;
+    return true;
+}
+
+// Decode thread shape: P/4 column chunks x (N/2)/ppt row groups.
+bool decode_shape(int N, int P, int* ppt) {
+    if (P % 4 || P > 256 || N > 256) return false;
+    const int pairs = N / 2, cpr = P / 4;
+    for (int c : {4, 2, 1}) {
+        if (pairs % c) continue;
+        const int threads = cpr * (pairs / c);
+        if (threads <= 512 && (threads >= 128 || c == 1)) {
+            *ppt = c;
+            return true;
+        }
+    }
+    return false;
+}
+
+m3_status launch_status(cudaError_t e) {
+    if (e == cudaSuccess) return M3_OK;
+    if (e == cudaErrorNotSupported) return M3_ERR_UNSUPPORTED;
+    return M3_ERR_LAUNCH;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* m3_status_string(m3_status s) {
+    switch (s) {
+        case M3_OK: return "ok";
+        case M3_ERR_NULL: return "a required pointer is NULL";
+        case M3_ERR_SHAPE: return "dimensions, seqlen or chunk out of range";
+        case M3_ERR_DTYPE: return "unknown io dtype";
+        case M3_ERR_ALIGN: return "pointer not aligned as documented";
+        case M3_ERR_UNSUPPORTED: return "shape not supported by any kernel of this build";
+        case M3_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case M3_ERR_LAUNCH: return "kernel launch failed";
+        case M3_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+        case M3_ERR_CUDA: return "CUDA runtime call failed";
+    }
+    return "unknown status";
+}
+
+m3_status m3_state_bytes(const m3_dims* d, size_t* h_bytes, size_t* x_prev_bytes,
+                         size_t* B_prev_bytes) {
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    const size_t e = io_bytes(d->io_dtype);
+    if (h_bytes) *h_bytes = sizeof(float) * (size_t)d->batch * d->nheads * d->dstate * d->headdim;
+    if (x_prev_bytes) *x_prev_bytes = e * (size_t)d->batch * d->nheads * d->rank * d->headdim;
+    if (B_prev_bytes) *B_prev_bytes = e * (size_t)d->batch * d->ngroups * d->rank * d->dstate;
+    return M3_OK;
+}
+
+m3_status m3_state_init(const m3_dims* d, m3_state* state, const float* h0, void* stream) {
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    if ((st = check_state(state)) != M3_OK) return st;
+    size_t hb, xb, bb;
+    m3_state_bytes(d, &hb, &xb, &bb);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = h0 ? cudaMemcpyAsync(state->h, h0, hb, cudaMemcpyDeviceToDevice, s)
+                       : cudaMemsetAsync(state->h, 0, hb, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(state->x_prev, 0, xb, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(state->B_prev, 0, bb, s);
+    return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+m3_status m3_scan_workspace_bytes(const m3_dims* d, int32_t seqlen, int32_t chunk, size_t* bytes) {
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    if (!bytes) return M3_ERR_NULL;
+    if (seqlen < 0) return M3_ERR_SHAPE;
+    if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return M3_ERR_SHAPE;
+    size_t extra = 0;
+    if (d->io_dtype == M3_BF16 && scan_tc_supported(d->dstate, d->headdim, d->rank, chunk))
+        extra = scan_tc_workspace_bytes(d->batch, d->nheads, d->dstate, d->headdim, d->rank,
+                                        seqlen, chunk);
+    *bytes = kStatusBytes + ((extra + 255) / 256) * 256;
+    return M3_OK;
+}
+
+m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
+                      const void* B, const void* C, const float* dt, const float* A,
+                      const float* lam, const float* theta, const float* D, m3_state* state,
+                      void* y, void* workspace, size_t workspace_bytes, uint32_t flags,
+                      void* stream) {
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    if (seqlen < 0) return M3_ERR_SHAPE;
+    if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return M3_ERR_SHAPE;
+    if ((st = check_state(state)) != M3_OK) return st;
+    if (seqlen == 0) return M3_OK;   // no tokens: nothing is read, written or launched
+    if (!x || !B || !C || !dt || !A || !lam || !theta || !y) return M3_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
+        !aligned(dt, 4) || !aligned(A, 4) || !aligned(lam, 4) || !aligned(theta, 4) ||
+        (D && !aligned(D, 4)))
+        return M3_ERR_ALIGN;
+    size_t need = 0;
+    m3_scan_workspace_bytes(d, seqlen, chunk, &need);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return M3_ERR_WORKSPACE;
+
+    const int N = d->dstate, P = d->headdim, R = d->rank;
+    const bool use_tc = !(flags & M3_FLAG_FORCE_SIMT) && d->io_dtype == M3_BF16 &&
+                        scan_tc_supported(N, P, R, chunk);
+    int ppt = 0, ns = 0;
+    if (!use_tc && (!rank_has_kernel(R) || !simt_shape(N, P, &ppt, &ns)))
+        return M3_ERR_UNSUPPORTED;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    ScanArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.x = x; a.B = B; a.C = C; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D;
+    a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y;
+    a.status = static_cast<uint32_t*>(workspace);
+    a.ws = static_cast<char*>(workspace) + kStatusBytes;
+    a.T = seqlen; a.batch = d->batch; a.H = d->nheads; a.G = d->ngroups; a.P = P; a.N = N;
+    a.chunk = chunk; a.ppt = ppt; a.ns = ns; a.flags = flags;
+
+    if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return M3_ERR_CUDA;
+    cudaError_t e = use_tc ? launch_scan_tc(a, R, s) : launch_scan_simt(a, R, d->io_dtype, s);
+    if (e != cudaSuccess) return launch_status(e);
+    const size_t row = io_bytes(d->io_dtype) * (size_t)d->ngroups * R * N;
+    e = launch_copy_prev(state->B_prev, B, seqlen, seqlen - 1, d->batch, row, s);
+    return launch_status(e);
+}
+
+m3_status m3_decode_step(const m3_dims* d, const void* x, const void* B, const void* C,
+                         const float* dt, const float* A, const float* lam,
+                         const float* theta, const float* D, m3_state* state, void* y,
+                         uint32_t flags, void* stream) {
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    if (!x || !B || !C || !dt || !A || !lam || !theta || !y) return M3_ERR_NULL;
+    if ((st = check_state(state)) != M3_OK) return st;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
+        !aligned(dt, 4) || !aligned(A, 4) || !aligned(lam, 4) || !aligned(theta, 4) ||
+        (D && !aligned(D, 4)))
+        return M3_ERR_ALIGN;
+    int ppt = 0;
+    if (!rank_has_kernel(d->rank) || !decode_shape(d->dstate, d->headdim, &ppt))
+        return M3_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.x = x; a.B = B; a.C = C; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D;
+    a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y;
+    a.H = d->nheads; a.G = d->ngroups; a.P = d->headdim; a.N = d->dstate; a.ppt = ppt;
+    a.flags = flags;
+    cudaError_t e = launch_decode(a, d->batch, d->rank, d->io_dtype, s);
+    if (e != cudaSuccess) return launch_status(e);
+    const size_t row = io_bytes(d->io_dtype) * (size_t)d->ngroups * d->rank * d->dstate;
+    e = launch_copy_prev(state->B_prev, B, 1, 0, d->batch, row, s);
+    return launch_status(e);
+}
+
+m3_status m3_query_status(const void* workspace, void* stream) {
+    if (!workspace) return M3_ERR_NULL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return M3_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return M3_ERR_CUDA;
+    return word == 0 ? M3_OK : M3_ERR_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// m3_common.cuh -- small device helpers shared by the CUDA kernels of the library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "m3.h"
+
+namespace m3 {
+
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float v);
+template <>
+__device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// Argument block of one decode step (device pointers, validated on the host).
+struct DecodeArgs {
+    const void* x;       // [b][H][R][P] io
+    const void* B;       // [b][G][R][N] io
+    const void* C;       // [b][G][R][N] io
+    const float* dt;     // [b][H]
+    const float* A;      // [b][H]
+    const float* lam;    // [b][H]
+    const float* theta;  // [b][G][N/2]
+    const float* D;      // [H] or null
+    float* h;            // [b][H][N][P]
+    void* x_prev;        // [b][H][R][P] io
+    const void* B_prev;  // [b][G][R][N] io (read only here; updated by a follow-up copy)
+    void* y;             // [b][H][R][P] io
+    int H, G, P, N;
+    int ppt;             // state pairs per thread
+    uint32_t flags;
+};
+
+// Argument block of one prefill call.
+struct ScanArgs {
+    const void* x;       // [b][T][H][R][P] io
+    const void* B;       // [b][T][G][R][N] io
+    const void* C;       // [b][T][G][R][N] io
+    const float* dt;     // [b][T][H]
+    const float* A;      // [b][T][H]
+    const float* lam;    // [b][T][H]
+    const float* theta;  // [b][T][G][N/2]
+    const float* D;      // [H] or null
+    float* h;            // [b][H][N][P]   in: h0, out: h_T
+    void* x_prev;        // [b][H][R][P]   in/out
+    const void* B_prev;  // [b][G][R][N]   read only here; updated by a follow-up copy
+    void* y;             // [b][T][H][R][P] io
+    uint32_t* status;    // workspace status word (may be null)
+    void* ws;            // workspace (after the status block)
+    long long T;
+    int batch, H, G, P, N;
+    int chunk;
+    int ppt, ns;         // SIMT kernel: pairs per lane, lanes per column
+    uint32_t flags;
+};
+
+}  // namespace m3

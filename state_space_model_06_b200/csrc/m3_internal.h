@@ -1,0 +1,28 @@
+// m3_internal.h -- launchers between the C ABI (m3_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "m3_common.cuh"
+
+namespace m3 {
+
+// decode step: one CTA per (batch, head); template on io type and rank
+cudaError_t launch_decode(const DecodeArgs& a, int batch, int R, int io_dtype, cudaStream_t s);
+
+// sequential fp32 CUDA-core prefill: one CTA per (batch, head)
+cudaError_t launch_scan_simt(const ScanArgs& a, int R, int io_dtype, cudaStream_t s);
+
+// tcgen05 chunked prefill (bf16 io).  Returns cudaErrorNotSupported for shapes
+// the kernel does not cover (the caller then reports M3_ERR_UNSUPPORTED or
+// falls back to the SIMT kernel).
+bool scan_tc_supported(int N, int P, int R, int chunk);
+size_t scan_tc_workspace_bytes(int batch, int H, int N, int P, int R, long long T, int chunk);
+cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s);
+
+// B_prev <- B[:, t] for every (batch, group): the previous-token input of the
+// next call, written after every head of the group has read the old value.
+cudaError_t launch_copy_prev(void* B_prev, const void* B, long long T, long long t, int batch,
+                             size_t row_bytes, cudaStream_t s);
+
+}  // namespace m3

@@ -1,0 +1,188 @@
+"""Thin ctypes binding of the C ABI in ``include/m3.h`` (libm3.so, built in-tree).
+
+The functions keep the C names and only marshal arguments: torch tensors become
+device pointers, dims become an ``m3_dims`` struct, the current torch stream is
+passed as the cudaStream_t.  Every step of the computation runs in the CUDA
+kernels of libm3.so; there is no fallback of any kind -- if the library is
+missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libm3.so")
+
+M3_OK, M3_ERR_NULL, M3_ERR_SHAPE, M3_ERR_DTYPE, M3_ERR_ALIGN, M3_ERR_UNSUPPORTED, \
+    M3_ERR_WORKSPACE, M3_ERR_LAUNCH, M3_ERR_TIMEOUT, M3_ERR_CUDA = range(10)
+M3_F32, M3_BF16 = 0, 1
+M3_FLAG_THETA_IS_ANGLE = 1
+M3_FLAG_FORCE_SIMT = 2
+
+EXPORTED = ("m3_state_bytes", "m3_state_init", "m3_scan_workspace_bytes", "m3_scan_fwd",
+            "m3_decode_step", "m3_query_status", "m3_status_string")
+
+
+class M3Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {m3_status_string(status)} (status {status})")
+
+
+class m3_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("nheads", ctypes.c_int32),
+                ("ngroups", ctypes.c_int32), ("headdim", ctypes.c_int32),
+                ("dstate", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("io_dtype", ctypes.c_int32)]
+
+
+class m3_state(ctypes.Structure):
+    _fields_ = [("h", ctypes.c_void_p), ("x_prev", ctypes.c_void_p), ("B_prev", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libm3.so (raises if it is missing: there is no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library not built: {path} (run __graft_entry__.build())")
+        lib = ctypes.CDLL(path)
+        vp, u32, i32, sz = ctypes.c_void_p, ctypes.c_uint32, ctypes.c_int32, ctypes.c_size_t
+        dp = ctypes.POINTER(m3_dims)
+        sp = ctypes.POINTER(m3_state)
+        szp = ctypes.POINTER(ctypes.c_size_t)
+        lib.m3_state_bytes.argtypes = [dp, szp, szp, szp]
+        lib.m3_state_init.argtypes = [dp, sp, vp, vp]
+        lib.m3_scan_workspace_bytes.argtypes = [dp, i32, i32, szp]
+        lib.m3_scan_fwd.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp, vp, sz,
+                                    u32, vp]
+        lib.m3_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp, u32, vp]
+        lib.m3_query_status.argtypes = [vp, vp]
+        lib.m3_status_string.argtypes = [ctypes.c_int]
+        lib.m3_status_string.restype = ctypes.c_char_p
+        for name in EXPORTED[:-1]:
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+@dataclass
+class Dims:
+    batch: int
+    nheads: int
+    ngroups: int
+    headdim: int
+    dstate: int
+    rank: int = 1
+    io_dtype: int = M3_BF16
+
+    def c(self) -> m3_dims:
+        return m3_dims(self.batch, self.nheads, self.ngroups, self.headdim, self.dstate,
+                       self.rank, self.io_dtype)
+
+
+def io_dtype_of(t: torch.dtype) -> int:
+    return {torch.bfloat16: M3_BF16, torch.float32: M3_F32}[t]
+
+
+def torch_dtype_of(io: int) -> torch.dtype:
+    return {M3_BF16: torch.bfloat16, M3_F32: torch.float32}[io]
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != M3_OK:
+        raise M3Error(status, where)
+
+
+def m3_status_string(status: int) -> str:
+    return load_library().m3_status_string(int(status)).decode()
+
+
+class State:
+    """Caller-owned resumable state (h fp32, previous token's x and B in io dtype)."""
+
+    def __init__(self, dims: Dims, device="cuda"):
+        io = torch_dtype_of(dims.io_dtype)
+        self.dims = dims
+        self.h = torch.zeros(dims.batch, dims.nheads, dims.dstate, dims.headdim,
+                             dtype=torch.float32, device=device)
+        self.x_prev = torch.zeros(dims.batch, dims.nheads, dims.rank, dims.headdim, dtype=io,
+                                  device=device)
+        self.B_prev = torch.zeros(dims.batch, dims.ngroups, dims.rank, dims.dstate, dtype=io,
+                                  device=device)
+
+    def c(self) -> m3_state:
+        return m3_state(self.h.data_ptr(), self.x_prev.data_ptr(), self.B_prev.data_ptr())
+
+
+def m3_state_bytes(dims: Dims):
+    h, x, b = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load_library().m3_state_bytes(ctypes.byref(dims.c()), ctypes.byref(h), ctypes.byref(x),
+                                         ctypes.byref(b)), "m3_state_bytes")
+    return h.value, x.value, b.value
+
+
+def m3_state_init(dims: Dims, state: State, h0=None, stream=None):
+    st = state.c()
+    _check(load_library().m3_state_init(ctypes.byref(dims.c()), ctypes.byref(st), _ptr(h0),
+                                        _stream(stream)), "m3_state_init")
+
+
+def m3_scan_workspace_bytes(dims: Dims, seqlen: int, chunk: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().m3_scan_workspace_bytes(ctypes.byref(dims.c()), int(seqlen), int(chunk),
+                                                  ctypes.byref(n)), "m3_scan_workspace_bytes")
+    return n.value
+
+
+def m3_scan_fwd(dims: Dims, seqlen: int, chunk: int, x, B, C, dt, A, lam, theta, D,
+                state: State, y, workspace, flags: int = 0, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = state.c()
+    _check(load_library().m3_scan_fwd(
+        ctypes.byref(dims.c()), int(seqlen), int(chunk), _ptr(x), _ptr(B), _ptr(C), _ptr(dt),
+        _ptr(A), _ptr(lam), _ptr(theta), _ptr(D), ctypes.byref(st), _ptr(y), _ptr(workspace),
+        ws_bytes, int(flags), _stream(stream)), "m3_scan_fwd")
+
+
+def m3_decode_step(dims: Dims, x, B, C, dt, A, lam, theta, D, state: State, y, flags: int = 0,
+                   stream=None):
+    st = state.c()
+    _check(load_library().m3_decode_step(
+        ctypes.byref(dims.c()), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam),
+        _ptr(theta), _ptr(D), ctypes.byref(st), _ptr(y), int(flags), _stream(stream)),
+        "m3_decode_step")
+
+
+def m3_query_status(workspace, stream=None) -> int:
+    """Synchronise the stream and return the device-side status word (M3_OK or M3_ERR_TIMEOUT)."""
+    return int(load_library().m3_query_status(_ptr(workspace), _stream(stream)))
+
+
+def alloc_workspace(dims: Dims, seqlen: int, chunk: int, device="cuda") -> torch.Tensor:
+    """A workspace tensor of the size m3_scan_fwd needs (256-byte aligned by torch)."""
+    n = m3_scan_workspace_bytes(dims, seqlen, chunk)
+    return torch.zeros(n, dtype=torch.uint8, device=device)

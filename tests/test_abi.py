@@ -1,0 +1,112 @@
+"""The C-ABI library loads and exports every entry point the header declares;
+host-side validation answers with status codes before touching the GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from state_space_model_06_b200 import m3
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "m3.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(m3_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(m3.LIB_PATH):
+        import __graft_entry__
+        __graft_entry__.build()
+    return m3.load_library()
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in ("m3_state_init", "m3_scan_fwd", "m3_decode_step"):
+        assert name in fns
+    assert set(m3.EXPORTED) <= set(fns)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(10):
+        assert m3.m3_status_string(s)
+    assert "timed out" in m3.m3_status_string(m3.M3_ERR_TIMEOUT)
+
+
+def test_state_bytes(lib):
+    d = m3.Dims(8, 64, 1, 64, 128, 1, m3.M3_BF16)
+    assert m3.m3_state_bytes(d) == (8 * 64 * 128 * 64 * 4, 8 * 64 * 64 * 2, 8 * 128 * 2)
+
+
+def test_workspace_bytes_covers_status_block(lib):
+    d = m3.Dims(1, 2, 1, 16, 16, 1, m3.M3_F32)
+    assert m3.m3_scan_workspace_bytes(d, 256, 64) >= 256
+
+
+@pytest.mark.parametrize("dims,status", [
+    (m3.Dims(1, 3, 2, 16, 16, 1, m3.M3_BF16), m3.M3_ERR_SHAPE),     # H % G != 0
+    (m3.Dims(1, 2, 1, 16, 15, 1, m3.M3_BF16), m3.M3_ERR_SHAPE),     # odd N
+    (m3.Dims(0, 2, 1, 16, 16, 1, m3.M3_BF16), m3.M3_ERR_SHAPE),     # empty batch
+    (m3.Dims(1, 2, 1, 16, 16, 1, 7), m3.M3_ERR_DTYPE),
+    (m3.Dims(1, 2, 1, 16, 16, 16, m3.M3_BF16), m3.M3_ERR_UNSUPPORTED),
+])
+def test_bad_dims_rejected(lib, dims, status):
+    with pytest.raises(m3.M3Error) as e:
+        m3.m3_state_bytes(dims)
+    assert e.value.status == status
+
+
+def _raw_scan(lib, dims, T=16, chunk=64, ptr=0x1000, state=None, ws=0x100000, ws_bytes=1 << 20,
+              x=None):
+    st = state if state is not None else m3.m3_state(0x2000, 0x3000, 0x4000)
+    x = ptr if x is None else x
+    return lib.m3_scan_fwd(ctypes.byref(dims.c()), T, chunk, x, ptr, ptr, ptr, ptr, ptr, ptr,
+                           None, ctypes.byref(st), ptr, ws, ws_bytes, 0, None)
+
+
+def test_scan_validation_before_launch(lib):
+    d = m3.Dims(1, 2, 1, 16, 16, 1, m3.M3_BF16)
+    assert _raw_scan(lib, d, x=0) == m3.M3_ERR_NULL
+    assert _raw_scan(lib, d, state=m3.m3_state(0, 0x3000, 0x4000)) == m3.M3_ERR_NULL
+    assert _raw_scan(lib, d, x=0x1008) == m3.M3_ERR_ALIGN
+    assert _raw_scan(lib, d, chunk=48) == m3.M3_ERR_SHAPE
+    assert _raw_scan(lib, d, T=-1) == m3.M3_ERR_SHAPE
+    assert _raw_scan(lib, d, ws=0) == m3.M3_ERR_WORKSPACE
+    assert _raw_scan(lib, d, ws_bytes=16) == m3.M3_ERR_WORKSPACE
+    assert _raw_scan(lib, d, ws=0x100010) == m3.M3_ERR_WORKSPACE
+    # seqlen 0 is a validated no-op: nothing is launched
+    assert _raw_scan(lib, d, T=0) == m3.M3_OK
+
+
+def test_decode_validation_before_launch(lib):
+    d = m3.Dims(1, 2, 1, 16, 16, 1, m3.M3_BF16)
+    st = m3.m3_state(0x2000, 0x3000, 0x4000)
+    p = 0x1000
+    args = lambda x, y, s: (ctypes.byref(d.c()), x, p, p, p, p, p, p, None, ctypes.byref(s), y, 0,
+                            None)
+    assert lib.m3_decode_step(*args(0, p, st)) == m3.M3_ERR_NULL
+    assert lib.m3_decode_step(*args(p, p + 2, st)) == m3.M3_ERR_ALIGN
+    assert lib.m3_decode_step(*args(p, p, m3.m3_state(0x2004, 0x3000, 0x4000))) == m3.M3_ERR_ALIGN
+    d2 = m3.Dims(1, 2, 1, 18, 16, 1, m3.M3_BF16)       # P % 4 != 0: no decode kernel
+    assert lib.m3_decode_step(ctypes.byref(d2.c()), p, p, p, p, p, p, p, None, ctypes.byref(st),
+                              p, 0, None) == m3.M3_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_missing_library(tmp_path):
+    old = m3._lib
+    m3._lib = None
+    try:
+        with pytest.raises(RuntimeError):
+            m3.load_library(str(tmp_path / "missing.so"))
+    finally:
+        m3._lib = old
