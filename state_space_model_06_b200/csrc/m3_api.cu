@@ -128,7 +128,7 @@ m3_status m3_scan_workspace_bytes(const m3_dims* d, int32_t seqlen, int32_t chun
     if (seqlen < 0) return M3_ERR_SHAPE;
     if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return M3_ERR_SHAPE;
     size_t extra = 0;
-    if (d->io_dtype == M3_BF16 && scan_tc_supported(d->dstate, d->headdim, d->rank, chunk))
+    if (d->io_dtype == M3_BF16 && scan_tc_supported(d->dstate, d->headdim, d->rank, chunk, d->nheads))
         extra = scan_tc_workspace_bytes(d->batch, d->nheads, d->dstate, d->headdim, d->rank,
                                         seqlen, chunk);
     *bytes = kStatusBytes + ((extra + 255) / 256) * 256;
@@ -156,8 +156,10 @@ m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const voi
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return M3_ERR_WORKSPACE;
 
     const int N = d->dstate, P = d->headdim, R = d->rank;
+    // the tensor-core kernel reads dt / A / lam / theta with TMA (16-byte aligned rows)
     const bool use_tc = !(flags & M3_FLAG_FORCE_SIMT) && d->io_dtype == M3_BF16 &&
-                        scan_tc_supported(N, P, R, chunk);
+                        scan_tc_supported(N, P, R, chunk, d->nheads) && aligned(dt, 16) &&
+                        aligned(A, 16) && aligned(lam, 16) && aligned(theta, 16);
     int ppt = 0, ns = 0;
     if (!use_tc && (!rank_has_kernel(R) || !simt_shape(N, P, &ppt, &ns)))
         return M3_ERR_UNSUPPORTED;

@@ -1,10 +1,818 @@
-// scan_tc.cu -- tcgen05 chunked prefill (placeholder until the kernel lands).
+// scan_tc.cu -- chunked prefill of the Mamba-3 recurrence on tcgen05 tensor cores.
+//
+// Math (Mamba-3 paper summary, "Technical Approach"):
+//   The exponential-trapezoidal complex recurrence (Propositions 1 and 4) is run in
+//   chunks of Q tokens: inside a chunk the parallel masked form of "Parallel
+//   representation under SSD" (Y = (L o C B^T) X with L = L_decay . L_band), across
+//   chunks the recurrence on the N x P state.  The rotation is absorbed into B and C
+//   (the RoPE trick, Proposition 3/4) with angles accumulated from the chunk start.
+//
+//   For chunk c with tokens t0..t1, chunk-relative log-decay cum_t = sum_{k=t0..t} dt_k A_k,
+//   chunk-relative angle psi_t = sum_{k=t0..t} dt_k theta_k, rotated B~_u = R(-psi_u) B_u,
+//   C~_t = R(-psi_t) C_t and the carried state g (original frame, with the next token's
+//   trapezoid term already folded in):
+//     Y_t   = sum_{u<=t} e^{cum_t-cum_u} (u<t ? w_u : gamma_u) (C~_t . B~_u) X_u
+//             + e^{cum_t} C~_t^T g  +  D X_t
+//     g'    = R(psi_t1) [ e^{cum_t1} g + sum_u e^{cum_t1-cum_u} w_u B~_u X_u^T ]
+//     w_u   = gamma_u + (1 - lam_{u+1}) dt_{u+1}     (the beta term of token u+1)
+//     g_0   = h0 + (1 - lam_0) dt_0 B_prev x_prev^T   (carried previous token)
+//   At the end of the call w_{T-1} = gamma_{T-1}, so the last g' is exactly h_{T-1}.
+//   MIMO: rows are (token, rank) pairs; L is shared by the R x R blocks.
+//
+// Kernel: one CTA per (batch, head), persistent over the chunks of the sequence.
+//   warp 0      TMA producer (x, B, C, theta, dt/A/lam tiles; zero fill past T)
+//   warp 1      tcgen05.mma issuer:  S = C~ B~^T,  dS = B~^T (w-scaled X),
+//               Y_inter = C~ g,  Y_intra = (S o L) X      (fp32 accumulators in TMEM)
+//   warps 2-5   epilogue: mask S -> bf16 (S o L); fp32 state update in registers;
+//               y = Y_intra + e^{cum} Y_inter + D x, TMA store
+//   warps 6-9   rotation: per-token coefficients (warp scan), cumulative angles,
+//               sincos, rotate B and C into swizzled bf16 MMA operands, scale X
+// Every wait is bounded; a timeout raises a CTA-wide abort and records
+// M3_ERR_TIMEOUT in the workspace status word.
+#include <cuda.h>
+
+#include <cstring>
+
 #include "m3_internal.h"
+#include "sm100.cuh"
 
 namespace m3 {
 
-bool scan_tc_supported(int, int, int, int) { return false; }
+using namespace sm100;
+
+namespace {
+
+constexpr int kP = 64;               // head dimension handled by this kernel
+constexpr int kThreads = 320;
+constexpr int kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum Bar {
+    RAW_FULL0, RAW_FULL1, RAW_EMPTY0, RAW_EMPTY1,
+    DT_FULL0, DT_FULL1, DT_EMPTY0, DT_EMPTY1,
+    X_FULL0, X_FULL1, X_EMPTY0, X_EMPTY1,
+    COEF_FULL0, COEF_FULL1, COEF_EMPTY0, COEF_EMPTY1, CUM_READY0, CUM_READY1,
+    OPS_FULL, OPS_EMPTY, S_FULL, S_EMPTY, SL_FULL, DS_FULL, DS_EMPTY,
+    G_FULL, G_EMPTY, Y_FULL, Y_EMPTY, Y_STAGED, DRAIN, NUM_BARS
+};
+
+template <int NST, int Q, int R>
+struct Cfg {
+    static constexpr int L = Q * R;                 // rows of the intra-chunk tiles
+    static constexpr int PAIRS = NST / 2;
+    static constexpr int PBLK = PAIRS / 32;         // rotation warps along the pairs
+    static constexpr int TSPLIT = 4 / PBLK;         // rotation warps along the tokens
+    static_assert(L == 64 || L == 128, "rows per chunk must be 64 or 128");
+    static_assert(NST == 64 || NST == 128, "dstate must be 64 or 128");
+
+    // bytes of the fixed (non-raw) buffers
+    static constexpr int X_BYTES = L * 128;
+    static constexpr int DT_BOX = (Q + 1) * 16;                 // 4 heads x (Q+1) tokens, fp32
+    static constexpr int DT_BYTES = (DT_BOX + 127) / 128 * 128;  // 128-byte aligned tiles
+    static constexpr int CT_BYTES = (NST / 64) * L * 128;
+    static constexpr int XW_BYTES = L * 128;
+    static constexpr int SL_BYTES = (L / 64) * L * 128;
+    static constexpr int G_BYTES = NST * 128;
+    static constexpr int COEF_FLOATS = 3 * Q + PAIRS + 4;
+    static constexpr int fixed_bytes() {
+        return 2 * X_BYTES + 2 * CT_BYTES + XW_BYTES + SL_BYTES + G_BYTES + 2 * 3 * DT_BYTES +
+               2 * COEF_FLOATS * 4 + NUM_BARS * 8 + 64;
+    }
+    static constexpr int raw_bytes(int rt) { return rt * R * NST * 2 * 2 + rt * PAIRS * 4; }
+    static constexpr int kSmemLimit = 232448 - 1024;            // minus base alignment slack
+    static constexpr int pick_rt() {
+        return (fixed_bytes() + 2 * raw_bytes(Q < 32 ? Q : 32) <= kSmemLimit) ? (Q < 32 ? Q : 32)
+               : (fixed_bytes() + 2 * raw_bytes(16) <= kSmemLimit) ? 16 : 8;
+    }
+    static constexpr int RT = pick_rt();                        // tokens per raw sub-chunk
+    static constexpr int NSUB = Q / RT;
+    static constexpr int TPT = RT / TSPLIT;                     // tokens per rotation thread
+    static_assert(RT % TSPLIT == 0 && Q % RT == 0, "bad raw sub-chunk");
+    static constexpr int BRAW_BYTES = RT * R * NST * 2;
+    static constexpr int TH_BYTES = RT * PAIRS * 4;
+    static constexpr int RAW_BYTES = 2 * BRAW_BYTES + TH_BYTES;
+
+    // shared memory offsets (SW128 tiles first, 1024-byte aligned)
+    static constexpr int OFF_X = 0;                                   // [2] x / y staging
+    static constexpr int OFF_CT = OFF_X + 2 * X_BYTES;                // C~
+    static constexpr int OFF_BT = OFF_CT + CT_BYTES;                  // B~
+    static constexpr int OFF_XW = OFF_BT + CT_BYTES;                  // scaled X
+    static constexpr int OFF_SL = OFF_XW + XW_BYTES;                  // S o L
+    static constexpr int OFF_G = OFF_SL + SL_BYTES;                   // g (bf16)
+    static constexpr int OFF_RAW = OFF_G + G_BYTES;                   // [2] B, C, theta
+    static constexpr int OFF_DT = OFF_RAW + 2 * RAW_BYTES;            // [2] dt, A, lam
+    static constexpr int OFF_COEF = OFF_DT + 2 * 3 * DT_BYTES;        // [2] coefficients
+    static constexpr int OFF_BAR = (OFF_COEF + 2 * COEF_FLOATS * 4 + 7) / 8 * 8;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;           // tmem base, abort flag
+    // + alignment slack; at least 120 KB so that only one CTA fits on an SM (each CTA
+    // allocates all 512 TMEM columns)
+    static constexpr int SMEM_USED = OFF_MISC + 16 + 1024;
+    static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
+    static_assert(SMEM <= 232448, "shared memory budget exceeded");
+    static_assert(OFF_RAW % 16 == 0 && OFF_DT % 16 == 0, "TMA destinations must be 16B aligned");
+
+    // TMEM columns
+    static constexpr uint32_t TM_S = 0, TM_DS = 128, TM_YA = 192, TM_YI = 256;
+
+    // instruction descriptors
+    static constexpr uint32_t ID_S = idesc_bf16(L, L, false, false);
+    static constexpr uint32_t ID_DS = idesc_bf16(NST, kP, true, true);
+    static constexpr uint32_t ID_Y = idesc_bf16(L, kP, false, true);
+};
+
+struct TcParams {
+    CUtensorMap tm_x, tm_y, tm_B, tm_C, tm_th, tm_dt, tm_A, tm_lam;
+    ScanArgs a;
+    int nchunks;
+    unsigned long long limit_ns;
+};
+
+// coefficient slot layout (floats): cum2[Q] | gam[Q] | w[Q] | psi_end[N/2] | cum2_end
+template <int NST, int Q, int R>
+struct Coef {
+    float* base;
+    __device__ float* cum2() const { return base; }
+    __device__ float* gam() const { return base + Q; }
+    __device__ float* w() const { return base + 2 * Q; }
+    __device__ float* psi_end() const { return base + 3 * Q; }
+    __device__ float* cum2_end() const { return base + 3 * Q + NST / 2; }
+};
+
+// A wait taken by all 32 lanes of a warp together: the outcome is made warp-uniform so
+// that no lane reaches a .sync.aligned tcgen05 instruction without the others.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
+    const bool r = mbar_wait(bar, parity, ab);
+    return __all_sync(0xffffffffu, r);
+}
+
+// K-major SW128 operand, K step k (16 elements): atoms of 64 K-elements are `rows`*128 B apart.
+__device__ __forceinline__ uint64_t desc_k(uint32_t base, int k, int rows) {
+    return sdesc_sw128(base + (uint32_t)(k >> 2) * rows * 128u + (uint32_t)(k & 3) * 32u, 16u,
+                       1024u);
+}
+// MN-major SW128 operand, K step k (16 rows of 128 B); MN atoms are `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int k, uint32_t lbo) {
+    return sdesc_sw128(base + (uint32_t)k * 2048u, lbo, 1024u);
+}
+
+// ---------------------------------------------------------------------------------
+template <int NST, int Q, int R>
+__device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab);
+
+// ---------------------------------------------------------------------------------
+// ---------------------------------------------------------------------------------
+template <int NST, int Q, int R>
+__device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
+                           const Abort& ab) {
+    using C = Cfg<NST, Q, R>;
+    const uint32_t s_ct = smem_u32(sm + C::OFF_CT), s_bt = smem_u32(sm + C::OFF_BT);
+    const uint32_t s_xw = smem_u32(sm + C::OFF_XW), s_sl = smem_u32(sm + C::OFF_SL);
+    const uint32_t s_g = smem_u32(sm + C::OFF_G);
+    for (int c = 0; c < p.nchunks; ++c) {
+        const uint32_t ph = c & 1;
+        const int st = c & 1;
+        if (!mbar_wait(&bar[OPS_FULL], ph, ab)) return;
+        tc_fence_after();
+        // S = C~ B~^T   (M = L tokens*ranks, N = L, K = NST)
+        if (!mbar_wait(&bar[S_EMPTY], ph ^ 1, ab)) return;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < NST / 16; ++k)
+            mma_bf16(tmem + C::TM_S, desc_k(s_ct, k, C::L), desc_k(s_bt, k, C::L), C::ID_S, k > 0);
+        mma_commit(&bar[S_FULL]);
+        // dS = B~^T Xw  (M = NST, N = P, K = L)
+        if (!mbar_wait(&bar[DS_EMPTY], ph ^ 1, ab)) return;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < C::L / 16; ++k)
+            mma_bf16(tmem + C::TM_DS, desc_mn(s_bt, k, C::L * 128u), desc_mn(s_xw, k, 1024u),
+                     C::ID_DS, k > 0);
+        mma_commit(&bar[DS_FULL]);
+        // Y_inter = C~ g  (M = L, N = P, K = NST)
+        if (!mbar_wait(&bar[G_FULL], ph, ab)) return;
+        if (!mbar_wait(&bar[Y_EMPTY], ph ^ 1, ab)) return;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < NST / 16; ++k)
+            mma_bf16(tmem + C::TM_YI, desc_k(s_ct, k, C::L), desc_mn(s_g, k, 1024u), C::ID_Y,
+                     k > 0);
+        mma_commit(&bar[G_EMPTY]);
+        mma_commit(&bar[OPS_EMPTY]);
+        // Y_intra = (S o L) X  (M = L, N = P, K = L)
+        if (!mbar_wait(&bar[SL_FULL], ph, ab)) return;
+        if (!mbar_wait(&bar[X_FULL0 + st], (c >> 1) & 1, ab)) return;
+        tc_fence_after();
+        const uint32_t s_x = smem_u32(sm + C::OFF_X + st * C::X_BYTES);
+#pragma unroll
+        for (int k = 0; k < C::L / 16; ++k)
+            mma_bf16(tmem + C::TM_YA, desc_k(s_sl, k, C::L), desc_mn(s_x, k, 1024u), C::ID_Y,
+                     k > 0);
+        mma_commit(&bar[Y_FULL]);
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Rotation warpgroup: coefficients, rotated B~ / C~ and the w-scaled X operand.
+template <int NST, int Q, int R>
+__device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
+    using C = Cfg<NST, Q, R>;
+    const ScanArgs& a = p.a;
+    const int tid = threadIdx.x - 192;          // 0..127
+    const int rw = tid >> 5, lane = tid & 31;
+    const int pb = rw % C::PBLK, ts = rw / C::PBLK;
+    const int pair = pb * 32 + lane;             // this thread's state pair
+    const int hq = (blockIdx.x % a.H) & 3;       // column of this head in the 4-head dt tile
+    const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
+    uint8_t* ct = sm + C::OFF_CT;
+    uint8_t* bt = sm + C::OFF_BT;
+    const int atom = (2 * pair) >> 6, col = (2 * pair) & 63;
+    int raw_it = 0;
+    for (int c = 0; c < p.nchunks; ++c) {
+        const int st = c & 1;
+        const uint32_t ph2 = (c >> 1) & 1;
+        if (!warp_wait(&bar[DT_FULL0 + st], ph2, ab)) return;
+        const float* dtt = reinterpret_cast<const float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
+        const float* At = dtt + C::DT_BYTES / 4;
+        const float* lt = dtt + 2 * C::DT_BYTES / 4;
+        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + st * C::COEF_FLOATS};
+
+        // ---- per-token coefficients (rotation warp 0): log2-decay prefix sum, gamma, w
+        if (rw == 0) {
+            if (!warp_wait(&bar[COEF_EMPTY0 + st], ph2 ^ 1, ab)) return;
+            float carry = 0.f;
+            for (int t0 = 0; t0 < Q; t0 += 32) {
+                const int t = t0 + lane;
+                float l2 = 0.f, gm = 0.f, wv = 0.f;
+                if (t < Q) {
+                    const float d = dtt[t * 4 + hq], lm = lt[t * 4 + hq];
+                    l2 = d * At[t * 4 + hq] * kLog2e;
+                    gm = lm * d;
+                    const float dn = dtt[(t + 1) * 4 + hq], ln = lt[(t + 1) * 4 + hq];
+                    wv = gm + (1.f - ln) * dn;
+                }
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, l2, o);
+                    if (lane >= o) l2 += v;
+                }
+                l2 += carry;
+                if (t < Q) {
+                    cf.cum2()[t] = l2;
+                    cf.gam()[t] = gm;
+                    cf.w()[t] = wv;
+                }
+                carry = __shfl_sync(0xffffffffu, l2, 31);
+            }
+            if (lane == 0) *cf.cum2_end() = carry;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[CUM_READY0 + st]);
+        }
+
+        // ---- rotated operands: wait until the MMAs of the previous chunk released them
+        if (!warp_wait(&bar[OPS_EMPTY], (c & 1) ^ 1, ab)) return;
+        float psi_acc = 0.f;
+        for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
+            const int rs = raw_it & 1;
+            if (!warp_wait(&bar[RAW_FULL0 + rs], (raw_it >> 1) & 1, ab)) return;
+            const uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
+            const uint32_t* braw = reinterpret_cast<const uint32_t*>(raw);
+            const uint32_t* craw = reinterpret_cast<const uint32_t*>(raw + C::BRAW_BYTES);
+            const float* th = reinterpret_cast<const float*>(raw + 2 * C::BRAW_BYTES);
+            const int tb = s * C::RT;           // first token of the sub-chunk (chunk-relative)
+            const int j0 = ts * C::TPT, j1 = j0 + C::TPT;
+            float psi = psi_acc;
+            for (int j = 0; j < j0; ++j)
+                psi += angle ? th[j * C::PAIRS + pair] : dtt[(tb + j) * 4 + hq] * th[j * C::PAIRS + pair];
+            for (int j = j0; j < j1; ++j) {
+                const float d = dtt[(tb + j) * 4 + hq];
+                psi += angle ? th[j * C::PAIRS + pair] : d * th[j * C::PAIRS + pair];
+                const float pr = psi - 6.283185307179586f * rintf(psi * 0.15915494309189535f);
+                float sn, cn;
+                __sincosf(pr, &sn, &cn);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int rowr = j * R + r;
+                    const uint32_t bv = braw[(rowr * NST) / 2 + pair];
+                    const uint32_t cv = craw[(rowr * NST) / 2 + pair];
+                    const float b0 = bf16lo(bv), b1 = bf16hi(bv);
+                    const float c0 = bf16lo(cv), c1 = bf16hi(cv);
+                    // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1]
+                    const uint32_t bo = pack_bf16x2(fmaf(cn, b0, sn * b1), fmaf(cn, b1, -sn * b0));
+                    const uint32_t co = pack_bf16x2(fmaf(cn, c0, sn * c1), fmaf(cn, c1, -sn * c0));
+                    const int row = (tb + j) * R + r;
+                    const uint32_t off = (uint32_t)atom * C::L * 128u + sw128_off(row, col);
+                    *reinterpret_cast<uint32_t*>(bt + off) = bo;
+                    *reinterpret_cast<uint32_t*>(ct + off) = co;
+                }
+            }
+            for (int j = j1; j < C::RT; ++j)
+                psi += angle ? th[j * C::PAIRS + pair] : dtt[(tb + j) * 4 + hq] * th[j * C::PAIRS + pair];
+            psi_acc = psi;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[RAW_EMPTY0 + rs]);
+        }
+        if (ts == 0) cf.psi_end()[pair] = psi_acc;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[COEF_FULL0 + st]);
+        // the per-token coefficients of rotation warp 0 are needed below
+        if (!warp_wait(&bar[CUM_READY0 + st], ph2, ab)) return;
+
+        // ---- w-scaled X:  Xw[u, r] = e^{cum_end - cum_u} w_u x[u, r]
+        if (!warp_wait(&bar[X_FULL0 + st], ph2, ab)) return;
+        const uint8_t* xt = sm + C::OFF_X + st * C::X_BYTES;
+        uint8_t* xw = sm + C::OFF_XW;
+        const float cend = *cf.cum2_end();
+        for (int idx = tid; idx < C::L * 8; idx += 128) {
+            const int row = idx >> 3, ch = idx & 7;
+            const int u = row / R;
+            const float sc = exp2f(cend - cf.cum2()[u]) * cf.w()[u];
+            const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((ch ^ row) & 7) << 4);
+            uint4 v = *reinterpret_cast<const uint4*>(xt + off);
+            uint4 o;
+            o.x = pack_bf16x2(bf16lo(v.x) * sc, bf16hi(v.x) * sc);
+            o.y = pack_bf16x2(bf16lo(v.y) * sc, bf16hi(v.y) * sc);
+            o.z = pack_bf16x2(bf16lo(v.z) * sc, bf16hi(v.z) * sc);
+            o.w = pack_bf16x2(bf16lo(v.w) * sc, bf16hi(v.w) * sc);
+            *reinterpret_cast<uint4*>(xw + off) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&bar[OPS_FULL]);
+            mbar_arrive(&bar[DT_EMPTY0 + st]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Epilogue warpgroup: masks S, keeps the fp32 state, writes y.
+template <int NST, int Q, int R>
+__device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
+                         const Abort& ab) {
+    using C = Cfg<NST, Q, R>;
+    const ScanArgs& a = p.a;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = w & 3;                                   // TMEM lane quadrant of this warp
+    const int etid = threadIdx.x - 64;                     // 0..127
+    const int b = blockIdx.x / a.H, h = blockIdx.x % a.H, g = h / (a.H / a.G);
+    const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+    const float Dh = a.D ? a.D[h] : 0.f;
+    const long long T = a.T;
+    const size_t bh = (size_t)b * a.H + h;
+
+    // Rows owned in the L-row accumulators (S, Y): L == 128 -> row 32q + lane, all
+    // columns; L == 64 -> row 16q + lane%16, column half lane/16 (M = 64 layout).
+    constexpr bool kHalfL = (C::L == 64);
+    const int lrow = kHalfL ? 16 * q + (lane & 15) : 32 * q + lane;
+    const int lcol0 = kHalfL ? 32 * (lane >> 4) : 0;
+    constexpr int kLCols = kHalfL ? 32 : C::L;
+    constexpr int kYCols = kHalfL ? 32 : kP;
+    // Rows owned in the NST-row state accumulator, same rule.
+    constexpr bool kHalfN = (NST == 64);
+    const int nrow = kHalfN ? 16 * q + (lane & 15) : 32 * q + lane;
+    const int ncol0 = kHalfN ? 32 * (lane >> 4) : 0;
+    constexpr int kNCols = kHalfN ? 32 : kP;
+
+    float gv[kNCols];                                       // fp32 state, row nrow
+    uint8_t* gs = sm + C::OFF_G;
+    uint8_t* sl = sm + C::OFF_SL;
+
+    // g (bf16, MN-major [n][p]) for the Y_inter MMA
+    auto publish_g = [&]() {
+#pragma unroll
+        for (int j = 0; j < kNCols; j += 8) {
+            uint4 o;
+            o.x = pack_bf16x2(gv[j], gv[j + 1]);
+            o.y = pack_bf16x2(gv[j + 2], gv[j + 3]);
+            o.z = pack_bf16x2(gv[j + 4], gv[j + 5]);
+            o.w = pack_bf16x2(gv[j + 6], gv[j + 7]);
+            *reinterpret_cast<uint4*>(gs + sw128_off(nrow, ncol0 + j)) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[G_FULL]);
+    };
+
+    // ---- g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T
+    {
+        const float* h0 = a.h + (bh * NST + nrow) * kP + ncol0;
+        const float d0 = a.dt[(size_t)b * T * a.H + h], l0 = a.lam[(size_t)b * T * a.H + h];
+        const float beta0 = (1.f - l0) * d0;
+        const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(a.x_prev) + bh * R * kP;
+        const __nv_bfloat16* bp =
+            static_cast<const __nv_bfloat16*>(a.B_prev) + ((size_t)b * a.G + g) * R * NST;
+#pragma unroll
+        for (int j = 0; j < kNCols; j += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(h0 + j);
+            gv[j] = v.x; gv[j + 1] = v.y; gv[j + 2] = v.z; gv[j + 3] = v.w;
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const float bb = beta0 * __bfloat162float(bp[r * NST + nrow]);
+#pragma unroll
+            for (int j = 0; j < kNCols; ++j)
+                gv[j] = fmaf(bb, __bfloat162float(xp[r * kP + ncol0 + j]), gv[j]);
+        }
+    }
+    publish_g();
+
+    bool ok = true;
+    for (int c = 0; c < p.nchunks && ok; ++c) {
+        const uint32_t ph = c & 1, ph2 = (c >> 1) & 1;
+        const int st = c & 1;
+        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + st * C::COEF_FLOATS};
+        if (!(ok = warp_wait(&bar[COEF_FULL0 + st], ph2, ab))) break;
+        const float* cum2 = cf.cum2();
+
+        // ---- S o L  ->  bf16, K-major [row][col] with L[t,u] = e^{cum_t-cum_u} (u<t ? w_u : gamma_u)
+        if (!(ok = warp_wait(&bar[S_FULL], ph, ab))) break;
+        tc_fence_after();
+        {
+            const int t = lrow / R;
+            const float ct = cum2[t];
+#pragma unroll 1
+            for (int cb = 0; cb < kLCols; cb += 32) {
+                float s[32];
+                if (kHalfL)
+                    tmem_ld_16x32bx2_x32<32>(tq + C::TM_S, s);
+                else
+                    tmem_ld_32x32b_x32(tq + C::TM_S + cb, s);
+                tmem_wait_ld();
+                const int colb = lcol0 + cb;
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    float m[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int u = (colb + j + e) / R;
+                        const float cu = (u < t) ? cf.w()[u] : cf.gam()[u];
+                        m[e] = (u <= t) ? s[j + e] * exp2f(ct - cum2[u]) * cu : 0.f;
+                    }
+                    uint4 o;
+                    o.x = pack_bf16x2(m[0], m[1]);
+                    o.y = pack_bf16x2(m[2], m[3]);
+                    o.z = pack_bf16x2(m[4], m[5]);
+                    o.w = pack_bf16x2(m[6], m[7]);
+                    const int col = colb + j;
+                    *reinterpret_cast<uint4*>(sl + (col >> 6) * C::L * 128 +
+                                              sw128_off(lrow, col & 63)) = o;
+                }
+            }
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&bar[S_EMPTY]);
+            mbar_arrive(&bar[SL_FULL]);
+        }
+
+        // ---- state: g <- R(psi_end) (e^{cum_end} g + dS), then publish it for the next chunk
+        if (!(ok = warp_wait(&bar[DS_FULL], ph, ab))) break;
+        tc_fence_after();
+        {
+            const float dec = exp2f(*cf.cum2_end());
+#pragma unroll
+            for (int cb = 0; cb < kNCols; cb += 32) {
+                float d[32];
+                if (kHalfN)
+                    tmem_ld_16x32bx2_x32<32>(tq + C::TM_DS, d);
+                else
+                    tmem_ld_32x32b_x32(tq + C::TM_DS + cb, d);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) gv[cb + j] = fmaf(dec, gv[cb + j], d[j]);
+            }
+            float sn, cn;
+            sincosf(cf.psi_end()[nrow >> 1], &sn, &cn);
+            const bool odd = nrow & 1;
+#pragma unroll
+            for (int j = 0; j < kNCols; ++j) {
+                const float o = __shfl_xor_sync(0xffffffffu, gv[j], 1);
+                gv[j] = odd ? fmaf(sn, o, cn * gv[j]) : fmaf(cn, gv[j], -sn * o);
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[DS_EMPTY]);
+        if (c + 1 < p.nchunks) {
+            // the Y_inter MMA of this chunk must be done reading g_c
+            if (!(ok = warp_wait(&bar[G_EMPTY], ph, ab))) break;
+            publish_g();
+        }
+
+        // ---- y = Y_intra + e^{cum_t} Y_inter + D x   (written over the x tile, then TMA store)
+        if (!(ok = warp_wait(&bar[Y_FULL], ph, ab))) break;
+        if (!(ok = warp_wait(&bar[X_FULL0 + st], ph2, ab))) break;
+        tc_fence_after();
+        uint8_t* xt = sm + C::OFF_X + st * C::X_BYTES;
+        {
+            const float sc = exp2f(cum2[lrow / R]);
+#pragma unroll 1
+            for (int cb = 0; cb < kYCols; cb += 32) {
+                float ya[32], yi[32];
+                if (kHalfL) {
+                    tmem_ld_16x32bx2_x32<32>(tq + C::TM_YA, ya);
+                    tmem_ld_16x32bx2_x32<32>(tq + C::TM_YI, yi);
+                } else {
+                    tmem_ld_32x32b_x32(tq + C::TM_YA + cb, ya);
+                    tmem_ld_32x32b_x32(tq + C::TM_YI + cb, yi);
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    const uint32_t off = sw128_off(lrow, lcol0 + cb + j);
+                    const uint4 xv = *reinterpret_cast<const uint4*>(xt + off);
+                    const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float y0 = fmaf(sc, yi[j + 2 * e], ya[j + 2 * e]) + Dh * bf16lo(xs[e]);
+                        const float y1 =
+                            fmaf(sc, yi[j + 2 * e + 1], ya[j + 2 * e + 1]) + Dh * bf16hi(xs[e]);
+                        o[e] = pack_bf16x2(y0, y1);
+                    }
+                    *reinterpret_cast<uint4*>(xt + off) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&bar[Y_EMPTY]);
+            mbar_arrive(&bar[Y_STAGED]);
+        }
+        if (etid == 0) {
+            // all four warps have written their rows of y (and are done with this chunk's
+            // coefficients): store the tile, then hand the x stage back to the producer
+            ok = mbar_wait(&bar[Y_STAGED], ph, ab);
+            if (ok) {
+                mbar_arrive(&bar[COEF_EMPTY0 + st]);
+                tma_store_5d(&p.tm_y, xt, 0, 0, h, c * Q, b);
+                bulk_commit();
+                bulk_wait_read<0>();
+                mbar_arrive(&bar[X_EMPTY0 + st]);
+            }
+        }
+        if (w == 2) ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+
+    if (ok) {
+        // final state h_T (original frame) and the carried previous x
+        float* hT = a.h + (bh * NST + nrow) * kP + ncol0;
+#pragma unroll
+        for (int j = 0; j < kNCols; j += 4)
+            *reinterpret_cast<float4*>(hT + j) = make_float4(gv[j], gv[j + 1], gv[j + 2], gv[j + 3]);
+        if (etid == 0) {
+            // every epilogue warp passed chunk 0 (it read x_prev there) before the last
+            // Y_STAGED completed, so x_prev can be overwritten now
+            const uint4* xl = reinterpret_cast<const uint4*>(
+                static_cast<const __nv_bfloat16*>(a.x) + (((size_t)b * T + (T - 1)) * a.H + h) * R * kP);
+            uint4* xpo = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.x_prev) + bh * R * kP);
+            for (int e = 0; e < R * kP / 8; ++e) xpo[e] = xl[e];
+        }
+    }
+    if (etid == 0) bulk_wait<0>();
+}
+
+// Wait for a barrier phase with a fixed time limit, regardless of the abort flag
+// (used on the way out, to let in-flight copies and MMAs land before exiting).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t ns) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < ns) {
+    }
+}
+
+template <int NST, int Q, int R>
+__device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
+    using C = Cfg<NST, Q, R>;
+    const ScanArgs& a = p.a;
+    const int b = blockIdx.x / a.H, h = blockIdx.x % a.H, g = h / (a.H / a.G);
+    // loads issued per ring stage, so that an aborted CTA can wait for them to land
+    int n_dt[2] = {0, 0}, n_raw[2] = {0, 0}, n_x[2] = {0, 0};
+    int raw_it = 0;
+    bool ok = true;
+    for (int c = 0; c < p.nchunks && ok; ++c) {
+        const int t0 = c * Q, st = c & 1;
+        const uint32_t ph = ((c >> 1) & 1) ^ 1;
+        // per-chunk dt / A / lam (Q+1 tokens: the next chunk's first token is the lookahead)
+        if (!(ok = mbar_wait(&bar[DT_EMPTY0 + st], ph, ab))) break;
+        mbar_arrive_expect_tx(&bar[DT_FULL0 + st], 3 * C::DT_BOX);
+        float* dtt = reinterpret_cast<float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
+        tma_load_3d(dtt, &p.tm_dt, &bar[DT_FULL0 + st], h & ~3, t0, b);
+        tma_load_3d(dtt + C::DT_BYTES / 4, &p.tm_A, &bar[DT_FULL0 + st], h & ~3, t0, b);
+        tma_load_3d(dtt + 2 * C::DT_BYTES / 4, &p.tm_lam, &bar[DT_FULL0 + st], h & ~3, t0, b);
+        ++n_dt[st];
+        // raw B, C, theta in sub-chunks of RT tokens; the x tile after the first one
+        for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
+            const int rs = raw_it & 1;
+            if (!(ok = mbar_wait(&bar[RAW_EMPTY0 + rs], ((raw_it >> 1) & 1) ^ 1, ab))) break;
+            mbar_arrive_expect_tx(&bar[RAW_FULL0 + rs], C::RAW_BYTES);
+            uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
+            const int tr = t0 + s * C::RT;
+            tma_load_5d(raw, &p.tm_B, &bar[RAW_FULL0 + rs], 0, 0, g, tr, b);
+            tma_load_5d(raw + C::BRAW_BYTES, &p.tm_C, &bar[RAW_FULL0 + rs], 0, 0, g, tr, b);
+            tma_load_4d(raw + 2 * C::BRAW_BYTES, &p.tm_th, &bar[RAW_FULL0 + rs], 0, g, tr, b);
+            ++n_raw[rs];
+            if (s == 0) {
+                if (!(ok = mbar_wait(&bar[X_EMPTY0 + st], ph, ab))) break;
+                mbar_arrive_expect_tx(&bar[X_FULL0 + st], C::X_BYTES);
+                tma_load_5d(sm + C::OFF_X + st * C::X_BYTES, &p.tm_x, &bar[X_FULL0 + st], 0, 0, h,
+                            t0, b);
+                ++n_x[st];
+            }
+        }
+    }
+    if (!ok) {
+        // aborted: let every load already issued land before the CTA exits
+        for (int s = 0; s < 2; ++s) {
+            if (n_dt[s]) drain_wait(&bar[DT_FULL0 + s], (n_dt[s] - 1) & 1, 10000000ull);
+            if (n_raw[s]) drain_wait(&bar[RAW_FULL0 + s], (n_raw[s] - 1) & 1, 10000000ull);
+            if (n_x[s]) drain_wait(&bar[X_FULL0 + s], (n_x[s] - 1) & 1, 10000000ull);
+        }
+    }
+}
+
+template <int NST, int Q, int R>
+__global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_constant__ TcParams p) {
+    using C = Cfg<NST, Q, R>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+    const int w = threadIdx.x >> 5;
+
+    if (threadIdx.x == 0) {
+        const uint32_t counts[NUM_BARS] = {
+            1, 1, 4, 4,          // raw full / empty
+            1, 1, 4, 4,          // dt full / empty
+            1, 1, 1, 1,          // x full / empty
+            4, 4, 1, 1, 1, 1,    // coef full / empty, cumulative-decay ready
+            4, 1, 1, 4, 4, 1, 4, // ops full/empty, S full/empty, SL full, dS full/empty
+            4, 1, 1, 4, 4, 1     // g full/empty, y full/empty, y staged, drain
+        };
+        for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], counts[i]);
+        misc[1] = 0u;  // abort flag
+        fence_mbar_init();
+        tma_prefetch_desc(&p.tm_x);
+        tma_prefetch_desc(&p.tm_B);
+        tma_prefetch_desc(&p.tm_C);
+        tma_prefetch_desc(&p.tm_th);
+        tma_prefetch_desc(&p.tm_dt);
+    }
+    if (w == 0) {
+        tmem_alloc(&misc[0], kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.a.status, p.limit_ns};
+
+    if (w == 0) {
+        if ((threadIdx.x & 31) == 0) producer<NST, Q, R>(p, sm, bar, ab);
+    } else if (w == 1) {
+        if ((threadIdx.x & 31) == 0) {
+            mma_issuer<NST, Q, R>(p, sm, bar, tmem, ab);
+            // no MMA may still be writing TMEM when it is released
+            mma_commit(&bar[DRAIN]);
+            drain_wait(&bar[DRAIN], 0, 100000000ull);
+        }
+    } else if (w < 6) {
+        epilogue<NST, Q, R>(p, sm, bar, tmem, ab);
+    } else {
+        rotation<NST, Q, R>(p, sm, bar, ab);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// host side: tensor maps and launch
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no -lcuda)
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ptr,
+              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+              CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, dt, rank, const_cast<void*>(ptr), reinterpret_cast<const cuuint64_t*>(dims),
+                    reinterpret_cast<const cuuint64_t*>(strides_bytes),
+                    reinterpret_cast<const cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int NST, int Q, int R>
+cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
+    using C = Cfg<NST, Q, R>;
+    TcParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.a = a;
+    p.nchunks = (int)((a.T + Q - 1) / Q);
+    p.limit_ns = 2000000000ull;
+    const uint64_t T = a.T, Bn = a.batch, H = a.H, G = a.G;
+    bool ok = true;
+    {   // x, y: (P, R, H, T, b), box (64, R, 1, Q, 1), 128B swizzle
+        const uint64_t d[5] = {kP, R, H, T, Bn};
+        const uint64_t st[4] = {kP * 2, (uint64_t)R * kP * 2, H * R * kP * 2, T * H * R * kP * 2};
+        const uint32_t box[5] = {kP, R, 1, Q, 1};
+        ok &= make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.x, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+        ok &= make_map(&p.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.y, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    {   // B, C: (N, R, G, T, b), box (N, R, 1, RT, 1)
+        const uint64_t d[5] = {NST, R, G, T, Bn};
+        const uint64_t st[4] = {NST * 2, (uint64_t)R * NST * 2, G * R * NST * 2,
+                                T * G * R * NST * 2};
+        const uint32_t box[5] = {NST, R, 1, C::RT, 1};
+        ok &= make_map(&p.tm_B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.B, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+        ok &= make_map(&p.tm_C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.C, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    {   // theta: (N/2, G, T, b), box (N/2, 1, RT, 1)
+        const uint64_t d[4] = {NST / 2, G, T, Bn};
+        const uint64_t st[3] = {NST / 2 * 4, G * NST / 2 * 4, T * G * NST / 2 * 4};
+        const uint32_t box[4] = {NST / 2, 1, C::RT, 1};
+        ok &= make_map(&p.tm_th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.theta, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    {   // dt, A, lam: (H, T, b), box (4, Q+1, 1)
+        const uint64_t d[3] = {H, T, Bn};
+        const uint64_t st[2] = {H * 4, T * H * 4};
+        const uint32_t box[3] = {4, Q + 1, 1};
+        ok &= make_map(&p.tm_dt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.dt, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+        ok &= make_map(&p.tm_A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.A, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+        ok &= make_map(&p.tm_lam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.lam, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    scan_tc_kernel<NST, Q, R><<<(unsigned)(a.batch * a.H), kThreads, C::SMEM, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool scan_tc_supported(int N, int P, int R, int chunk, int H) {
+    if (P != kP || H % 4 != 0) return false;
+    if (N != 64 && N != 128) return false;
+    if (R == 1) return chunk == 64 || chunk == 128;
+    if (R == 2) return N == 64 && (chunk == 32 || chunk == 64);
+    if (R == 4) return N == 64 && (chunk == 16 || chunk == 32);
+    return false;
+}
+
 size_t scan_tc_workspace_bytes(int, int, int, int, int, long long, int) { return 0; }
-cudaError_t launch_scan_tc(const ScanArgs&, int, cudaStream_t) { return cudaErrorNotSupported; }
+
+cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s) {
+    const int N = a.N, Q = a.chunk;
+    if (R == 1) {
+        if (N == 128 && Q == 64) return launch_t<128, 64, 1>(a, s);
+        if (N == 128 && Q == 128) return launch_t<128, 128, 1>(a, s);
+        if (N == 64 && Q == 64) return launch_t<64, 64, 1>(a, s);
+        if (N == 64 && Q == 128) return launch_t<64, 128, 1>(a, s);
+    } else if (R == 2 && N == 64) {
+        if (Q == 32) return launch_t<64, 32, 2>(a, s);
+        if (Q == 64) return launch_t<64, 64, 2>(a, s);
+    } else if (R == 4 && N == 64) {
+        if (Q == 16) return launch_t<64, 16, 4>(a, s);
+        if (Q == 32) return launch_t<64, 32, 4>(a, s);
+    }
+    return cudaErrorNotSupported;
+}
 
 }  // namespace m3
