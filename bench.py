@@ -1,0 +1,438 @@
+"""Benchmark of the Mamba-3 mixer hot path on B200.
+
+One step = one m3_scan_fwd call over the SISO 1.5B-scale prefill workload
+(batch 8, 64 heads, T 4096, P 64, N 128, chunk 64, bf16 x/B/C, fp32 dt/A/lam/theta/state),
+i.e. every prefill step of the method.  Alongside, the batch-256 decode workloads
+(SISO N 128 and MIMO R 4 N 64; 1000 sequential tokens) are timed as a sub-metric.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs one independent replica per GPU (the path has no cross-GPU exchange:
+every (batch, head) recurrence is independent), launched with torch.distributed.run;
+times are CUDA-event device times, max over ranks.  Rank 0 prints one JSON line.
+
+`--impl reference` times the CPU oracle (plain fp64 C, OpenMP) on host cores on a
+bounded sample of the same workload and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from state_space_model_06_b200 import inputs, m3  # noqa: E402
+
+METRIC = ("prefill tokens/s/layer (% tensor peak); decode tok/s at batch 256 (% HBM BW)")
+WORKLOAD = "siso_prefill_1p5b"
+DECODES = ("decode_siso_b256", "decode_mimo_b256")
+DECODE_TOKENS = 1000
+DECODE_POOL = 32            # distinct pre-generated tokens, cycled over the 1000 steps
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def scan_algorithmic(w):
+    """Algorithmic bytes and FLOPs of one prefill call (each tensor read or written once;
+    FLOPs of the four chunk contractions, causal half of the intra-chunk products)."""
+    b, T, H, G, P, N, R, Q = w.batch, w.seqlen, w.nheads, w.ngroups, w.headdim, w.dstate, \
+        w.rank, w.chunk
+    e = 2
+    per_head_tok = 2 * P * R * e + 3 * 4                  # x in, y out, dt/A/lam
+    per_group_tok = 2 * N * R * e + (N // 2) * 4          # B, C, theta
+    state = b * H * N * P * 4 * 2 + b * H * R * P * e * 2 + b * G * R * N * e * 2
+    byts = b * T * (H * per_head_tok + G * per_group_tok) + state
+    nchunk = math.ceil(T / Q)
+    tri = Q * (Q + 1) // 2
+    flops_chunk = tri * R * R * 2 * N + tri * R * R * 2 * P + 2 * N * P * Q * R + 2 * Q * R * N * P
+    flops = b * H * nchunk * flops_chunk
+    return byts, flops
+
+
+def decode_algorithmic(w):
+    b, H, G, P, N, R = w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank
+    e = 2
+    byts = (2 * b * H * N * P * 4            # state read + write
+            + 4 * b * H * R * P * e          # x, x_prev in, x_prev out, y
+            + 4 * b * G * R * N * e          # B, C, B_prev in, B_prev out
+            + 3 * b * H * 4 + b * G * (N // 2) * 4 + H * 4)
+    return byts
+
+
+def source_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(kernel_src, workload):
+    """DRAM traffic per launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(workload)
+    if not ent or ent.get("source_sha256_16") != source_hash(kernel_src):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running (read only)."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index, period=0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop, self._t = period, threading.Event(), None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: clocks reported as unknown
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                fn = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = fn(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(self.reasons - {"gpu_idle"})}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- our arm
+def prefill_setup(w, dev, seed):
+    inp = inputs.make_scan_inputs(w.batch, w.seqlen, w.nheads, w.ngroups, w.headdim, w.dstate,
+                                  w.rank, io_dtype=w.io_dtype, theta_max=w.theta_max, seed=seed)
+    d = m3.Dims(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
+                m3.io_dtype_of(w.io_dtype))
+    g = {k: v.to(dev) for k, v in inp.items()}
+    st = m3.State(d, dev)
+    y = torch.empty_like(g["x"])
+    ws = m3.alloc_workspace(d, w.seqlen, w.chunk, dev)
+    return inp, d, g, st, y, ws
+
+
+def run_scan(w, d, g, st, y, ws, stream):
+    m3.m3_scan_fwd(d, w.seqlen, w.chunk, g["x"], g["B"], g["C"], g["dt"], g["A"], g["lam"],
+                   g["theta"], g["D"], st, y, ws, stream=stream)
+
+
+def time_prefill(w, d, g, st, y, ws, steps, warmup, stream, ws_world):
+    for _ in range(warmup):
+        m3.m3_state_init(d, st, stream=stream)
+        run_scan(w, d, g, st, y, ws, stream)
+    torch.cuda.synchronize()
+    barrier(ws_world)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        m3.m3_state_init(d, st, stream=stream)         # fresh sequence each step (memsets)
+        ev[i][0].record(stream)
+        run_scan(w, d, g, st, y, ws, stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws_world)
+    torch.cuda.synchronize()
+    status = m3.m3_query_status(ws, stream)
+    per = [a.elapsed_time(b) for a, b in ev]
+    return sum(per) / steps, status
+
+
+def time_prefill_e2e(w, d, inp, st, ws, steps, stream, dev):
+    """Same call through host buffers: pinned H2D of the step's inputs, the call, D2H of y."""
+    keys = ("x", "B", "C", "dt", "A", "lam", "theta", "D")
+    host = {k: inp[k].pin_memory() for k in keys}
+    devb = {k: torch.empty_like(inp[k], device=dev) for k in keys}
+    y = torch.empty_like(devb["x"])
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y.numel() * y.element_size()
+
+    def step():
+        with torch.cuda.stream(stream):
+            for k in keys:
+                devb[k].copy_(host[k], non_blocking=True)
+            m3.m3_state_init(d, st, stream=stream)
+            run_scan(w, d, devb, st, y, ws, stream)
+            y_host.copy_(y, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def time_decode(name, dev, stream, seed):
+    w = inputs.WORKLOADS[name]
+    inp = inputs.make_decode_inputs(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
+                                    tokens=DECODE_POOL, io_dtype=w.io_dtype,
+                                    theta_max=w.theta_max, seed=seed)
+    d = m3.Dims(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
+                m3.io_dtype_of(w.io_dtype))
+    g = {k: v.to(dev) for k, v in inp.items()}
+    st = m3.State(d, dev)
+    y = torch.empty_like(g["x"][0])
+    keys = ("x", "B", "C", "dt", "A", "lam", "theta")
+    tok = [[g[k][i] for k in keys] for i in range(DECODE_POOL)]
+
+    def reset():
+        st.h.copy_(g["h0"])
+        st.x_prev.copy_(g["x_prev"])
+        st.B_prev.copy_(g["B_prev"])
+
+    reset()
+    for t in range(10):
+        m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=stream)
+    reset()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(DECODE_TOKENS):
+        m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / DECODE_TOKENS
+    finite = bool(torch.isfinite(st.h).all().item())
+    byts = decode_algorithmic(w)
+    return {"tokens_per_s": w.batch / (ms / 1e3), "us_per_step": ms * 1e3,
+            "achieved_gbs": byts / (ms / 1e3) / 1e9, "alg_bytes_per_step": byts,
+            "state_finite": finite,
+            "config": {"batch": w.batch, "heads": w.nheads, "headdim": w.headdim,
+                       "dstate": w.dstate, "rank": w.rank, "tokens": DECODE_TOKENS,
+                       "distinct_tokens": DECODE_POOL}}
+
+
+def oracle_sample(w, seqlen, seed=0):
+    """Time the CPU oracle on batch row 0, all heads, the first `seqlen` tokens."""
+    import oracle
+    inp = inputs.make_scan_inputs(1, seqlen, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
+                                  io_dtype=w.io_dtype, theta_max=w.theta_max, seed=seed)
+    arr = {k: inp[k].double().numpy() for k in ("x", "B", "C", "dt", "A", "lam", "theta", "D")}
+    threads = min(oracle.max_threads(), w.nheads)
+    t0 = time.perf_counter()
+    oracle.scan(arr["x"], arr["B"], arr["C"], arr["dt"], arr["A"], arr["lam"], arr["theta"],
+                D=arr["D"], nthreads=threads)
+    dt = time.perf_counter() - t0
+    return seqlen / dt, threads, dt
+
+
+def ours(args):
+    ws_world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    w = inputs.WORKLOADS[WORKLOAD]
+    if args.batch:
+        # smaller batch of the same workload: only for short profiler captures
+        import dataclasses
+        w = dataclasses.replace(w, batch=args.batch)
+    pk, pk_kind = peaks()
+
+    inp, d, g, st, y, ws = prefill_setup(w, dev, seed=rank)
+    with ClockSampler(local) as clk:
+        ms, status = time_prefill(w, d, g, st, y, ws, args.steps, args.warmup, stream, ws_world)
+    if status != m3.M3_OK:
+        raise RuntimeError(f"device status {m3.m3_status_string(status)}")
+    ms_max = max_over_ranks(ms, ws_world)
+    tokens = w.batch * w.seqlen
+    value = ws_world * tokens / (ms_max / 1e3)
+    byts, flops = scan_algorithmic(w)
+    achieved = byts / (ms / 1e3) / 1e9
+    tflops = flops / (ms / 1e3) / 1e12
+    kernel_src = os.path.join(ROOT, "state_space_model_06_b200", "csrc", "scan_tc.cu")
+    traffic = committed_traffic(kernel_src, WORKLOAD)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; shapes and distributions of a 1.5B-scale Mamba-3 layer)",
+        "config": {"workload": WORKLOAD, "batch": w.batch, "heads": w.nheads,
+                   "groups": w.ngroups, "seqlen": w.seqlen, "headdim": w.headdim,
+                   "dstate": w.dstate, "rank": w.rank, "chunk": w.chunk,
+                   "io": "bf16 x/B/C/y, fp32 dt/A/lam/theta/state",
+                   "l2": f"inputs larger than L2 ({byts / 1e6:.0f} MB touched per step)",
+                   "parallelism": f"replicas x{ws_world} (independent (batch, head) work)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "peak_source": pk_kind, "kernel": "scan_tc_kernel<128,64,1>",
+                     "alg_bytes_per_launch": byts,
+                     "tensor": {"achieved_tflops": tflops, "peak_tflops": pk["bf16_tflops"],
+                                "frac": tflops / pk["bf16_tflops"],
+                                "alg_flops_per_launch": flops}},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    if args.prefill_only:
+        args.no_decode = args.no_e2e = args.no_cpu = True
+    if not args.no_decode:
+        line["decode"] = {}
+        for name in DECODES:
+            r = time_decode(name, dev, stream, seed=100 + rank)
+            r["hbm_frac"] = r["achieved_gbs"] / pk["hbm_gbs"]
+            r["tokens_per_s"] = max_over_ranks(1.0 / r["tokens_per_s"], ws_world)
+            r["tokens_per_s"] = ws_world / r["tokens_per_s"]
+            line["decode"][name] = r
+
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_prefill_e2e(w, d, inp, st, ws, min(args.steps, 5), stream, dev)
+        e2e_ms = max_over_ranks(e2e_ms, ws_world)
+        line["e2e"] = {"value": ws_world * tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                       "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h}
+
+    if rank == 0 and ws_world == 1 and not args.no_cpu:
+        tps, cores, secs = oracle_sample(w, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"batch row 0, all {w.nheads} heads, first "
+                                          f"{args.cpu_tokens} tokens ({secs:.1f} s of fp64 CPU work)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+def reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    ws_world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = inputs.WORKLOADS[WORKLOAD]
+    for _ in range(args.warmup):
+        oracle_sample(w, args.ref_tokens, seed=1)
+    times = []
+    cores = 0
+    for _ in range(args.steps):
+        _, cores, secs = oracle_sample(w, args.ref_tokens, seed=1)
+        times.append(secs)
+    sec = sum(times) / len(times)
+    value = args.ref_tokens / sec
+    sample = (f"each step: batch row 0, all {w.nheads} heads, first {args.ref_tokens} of "
+              f"{w.seqlen} tokens of the workload")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": ws_world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "batch": w.batch, "heads": w.nheads,
+                       "groups": w.ngroups, "seqlen": w.seqlen, "headdim": w.headdim,
+                       "dstate": w.dstate, "rank": w.rank, "chunk": w.chunk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling only)")
+    ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and CPU legs")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

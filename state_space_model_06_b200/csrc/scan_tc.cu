@@ -40,10 +40,26 @@ namespace m3 {
 
 using namespace sm100;
 
+// Optional timeline instrumentation: with -DM3_TRACE the kernel records clock64() at
+// each pipeline hand-off of one CTA into a device array (read by m3_trace_copy).
+#ifdef M3_TRACE
+#define M3_TRACE_CHUNKS 64
+#define M3_TRACE_EVENTS 32
+__device__ unsigned long long g_m3_trace[M3_TRACE_CHUNKS][M3_TRACE_EVENTS];
+__device__ int g_m3_trace_cta = 0;
+#define M3_TRACE_EV(c, e)                                                           \
+    do {                                                                            \
+        if ((int)blockIdx.x == g_m3_trace_cta && (c) < M3_TRACE_CHUNKS)             \
+            g_m3_trace[(c)][(e)] = clock64();                                       \
+    } while (0)
+#else
+#define M3_TRACE_EV(c, e) do { } while (0)
+#endif
+
 namespace {
 
 constexpr int kP = 64;               // head dimension handled by this kernel
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;       // 11 warps: TMA, MMA, 4 epilogue, 4 rotation, coefficients
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -51,68 +67,101 @@ enum Bar {
     RAW_FULL0, RAW_FULL1, RAW_EMPTY0, RAW_EMPTY1,
     DT_FULL0, DT_FULL1, DT_EMPTY0, DT_EMPTY1,
     X_FULL0, X_FULL1, X_EMPTY0, X_EMPTY1,
-    COEF_FULL0, COEF_FULL1, COEF_EMPTY0, COEF_EMPTY1, CUM_READY0, CUM_READY1,
-    OPS_FULL, OPS_EMPTY, S_FULL, S_EMPTY, SL_FULL, DS_FULL, DS_EMPTY,
-    G_FULL, G_EMPTY, Y_FULL, Y_EMPTY, Y_STAGED, DRAIN, NUM_BARS
+    COEF_FULL0, COEF_FULL1, COEF_EMPTY0, COEF_EMPTY1, RS0, RS1,
+    OPS_FULL0, OPS_FULL1, OPS_EMPTY0, OPS_EMPTY1, S_FULL, S_EMPTY, SL_FULL, DS_FULL, DS_EMPTY,
+    G_FULL, G_EMPTY, Y_FULL0, Y_FULL1, Y_EMPTY0, Y_EMPTY1, Y_STAGED, DRAIN, NUM_BARS
 };
+
+// arrival count of each barrier: 1 for TMA expect_tx / tcgen05.commit / single-thread
+// arrivals, 4 for one elected lane per warp of a four-warp group, 5 where the
+// coefficient warp joins the four rotation warps
+__device__ __forceinline__ uint32_t bar_count(int i) {
+    switch (i) {
+        case DT_EMPTY0: case DT_EMPTY1: case COEF_FULL0: case COEF_FULL1:
+        case OPS_FULL0: case OPS_FULL1:
+            return 5;
+        case RAW_EMPTY0: case RAW_EMPTY1: case RS0: case RS1:
+        case S_EMPTY: case SL_FULL: case DS_EMPTY: case G_FULL:
+        case Y_EMPTY0: case Y_EMPTY1: case Y_STAGED:
+            return 4;
+        default:
+            return 1;
+    }
+}
 
 template <int NST, int Q, int R>
 struct Cfg {
     static constexpr int L = Q * R;                 // rows of the intra-chunk tiles
     static constexpr int PAIRS = NST / 2;
-    static constexpr int PBLK = PAIRS / 32;         // rotation warps along the pairs
-    static constexpr int TSPLIT = 4 / PBLK;         // rotation warps along the tokens
+    static constexpr int PPT = PAIRS / 32;          // state pairs per rotation thread (1 or 2)
+    static constexpr int TSPLIT = 4;                // rotation warps along the tokens
     static_assert(L == 64 || L == 128, "rows per chunk must be 64 or 128");
     static_assert(NST == 64 || NST == 128, "dstate must be 64 or 128");
 
-    // bytes of the fixed (non-raw) buffers
+    // bytes of the buffers
     static constexpr int X_BYTES = L * 128;
     static constexpr int DT_BOX = (Q + 1) * 16;                 // 4 heads x (Q+1) tokens, fp32
     static constexpr int DT_BYTES = (DT_BOX + 127) / 128 * 128;  // 128-byte aligned tiles
     static constexpr int CT_BYTES = (NST / 64) * L * 128;
     static constexpr int XW_BYTES = L * 128;
+    static constexpr int SLOT_BYTES = 2 * CT_BYTES + XW_BYTES;  // C~, B~, Xw of one chunk
     static constexpr int SL_BYTES = (L / 64) * L * 128;
     static constexpr int G_BYTES = NST * 128;
-    static constexpr int COEF_FLOATS = 3 * Q + PAIRS + 4;
-    static constexpr int fixed_bytes() {
-        return 2 * X_BYTES + 2 * CT_BYTES + XW_BYTES + SL_BYTES + G_BYTES + 2 * 3 * DT_BYTES +
-               2 * COEF_FLOATS * 4 + NUM_BARS * 8 + 64;
+    static constexpr int COEF_FLOATS = 4 * Q + PAIRS + 4;
+    static constexpr int base_bytes() {
+        return 2 * X_BYTES + SL_BYTES + G_BYTES + 2 * 3 * DT_BYTES + 2 * COEF_FLOATS * 4 +
+               2 * 4 * PAIRS * 4 + NUM_BARS * 8 + 64;
     }
     static constexpr int raw_bytes(int rt) { return rt * R * NST * 2 * 2 + rt * PAIRS * 4; }
     static constexpr int kSmemLimit = 232448 - 1024;            // minus base alignment slack
-    static constexpr int pick_rt() {
-        return (fixed_bytes() + 2 * raw_bytes(Q < 32 ? Q : 32) <= kSmemLimit) ? (Q < 32 ? Q : 32)
-               : (fixed_bytes() + 2 * raw_bytes(16) <= kSmemLimit) ? 16 : 8;
+    // (operand slots, raw sub-chunk tokens): prefer two slots, then the largest sub-chunk
+    static constexpr int pick() {
+        for (int ops = 2; ops >= 1; --ops)
+            for (int rt = (Q < 32 ? Q : 32); rt >= TSPLIT; rt /= 2)
+                if (Q % rt == 0 && rt % TSPLIT == 0 &&
+                    base_bytes() + ops * SLOT_BYTES + 2 * raw_bytes(rt) <= kSmemLimit)
+                    return ops * 1000 + rt;
+        return 0;
     }
-    static constexpr int RT = pick_rt();                        // tokens per raw sub-chunk
+    static_assert(pick() != 0, "shared memory budget exceeded");
+    static constexpr int OPS = pick() / 1000;                   // operand slots
+    static constexpr int RT = pick() % 1000;                    // tokens per raw sub-chunk
     static constexpr int NSUB = Q / RT;
     static constexpr int TPT = RT / TSPLIT;                     // tokens per rotation thread
-    static_assert(RT % TSPLIT == 0 && Q % RT == 0, "bad raw sub-chunk");
     static constexpr int BRAW_BYTES = RT * R * NST * 2;
     static constexpr int TH_BYTES = RT * PAIRS * 4;
     static constexpr int RAW_BYTES = 2 * BRAW_BYTES + TH_BYTES;
 
     // shared memory offsets (SW128 tiles first, 1024-byte aligned)
     static constexpr int OFF_X = 0;                                   // [2] x / y staging
-    static constexpr int OFF_CT = OFF_X + 2 * X_BYTES;                // C~
-    static constexpr int OFF_BT = OFF_CT + CT_BYTES;                  // B~
-    static constexpr int OFF_XW = OFF_BT + CT_BYTES;                  // scaled X
-    static constexpr int OFF_SL = OFF_XW + XW_BYTES;                  // S o L
+    static constexpr int OFF_OPS = OFF_X + 2 * X_BYTES;               // [OPS] C~, B~, Xw
+    static constexpr int OFF_SL = OFF_OPS + OPS * SLOT_BYTES;         // S o L
     static constexpr int OFF_G = OFF_SL + SL_BYTES;                   // g (bf16)
     static constexpr int OFF_RAW = OFF_G + G_BYTES;                   // [2] B, C, theta
     static constexpr int OFF_DT = OFF_RAW + 2 * RAW_BYTES;            // [2] dt, A, lam
     static constexpr int OFF_COEF = OFF_DT + 2 * 3 * DT_BYTES;        // [2] coefficients
-    static constexpr int OFF_BAR = (OFF_COEF + 2 * COEF_FLOATS * 4 + 7) / 8 * 8;
+    static constexpr int OFF_RSUM = OFF_COEF + 2 * COEF_FLOATS * 4;   // [2][4][PAIRS] angle sums
+    static constexpr int OFF_BAR = (OFF_RSUM + 2 * 4 * PAIRS * 4 + 7) / 8 * 8;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;           // tmem base, abort flag
     // + alignment slack; at least 120 KB so that only one CTA fits on an SM (each CTA
     // allocates all 512 TMEM columns)
     static constexpr int SMEM_USED = OFF_MISC + 16 + 1024;
     static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
     static_assert(SMEM <= 232448, "shared memory budget exceeded");
-    static_assert(OFF_RAW % 16 == 0 && OFF_DT % 16 == 0, "TMA destinations must be 16B aligned");
+    static_assert(OFF_RAW % 128 == 0 && OFF_DT % 128 == 0, "TMA destinations must be aligned");
+    __device__ static uint8_t* ct(uint8_t* sm, int slot) { return sm + OFF_OPS + slot * SLOT_BYTES; }
+    __device__ static uint8_t* bt(uint8_t* sm, int slot) {
+        return sm + OFF_OPS + slot * SLOT_BYTES + CT_BYTES;
+    }
+    __device__ static uint8_t* xw(uint8_t* sm, int slot) {
+        return sm + OFF_OPS + slot * SLOT_BYTES + 2 * CT_BYTES;
+    }
 
     // TMEM columns
-    static constexpr uint32_t TM_S = 0, TM_DS = 128, TM_YA = 192, TM_YI = 256;
+    // TMEM columns: S, dS, and two buffers of (Y_intra, Y_inter)
+    static constexpr uint32_t TM_S = 0, TM_DS = 128, TM_G = 448;   // G: the fp32 carried state
+    __device__ static uint32_t tm_ya(int yb) { return 192u + 128u * yb; }
+    __device__ static uint32_t tm_yi(int yb) { return 256u + 128u * yb; }
 
     // instruction descriptors
     static constexpr uint32_t ID_S = idesc_bf16(L, L, false, false);
@@ -127,16 +176,25 @@ struct TcParams {
     unsigned long long limit_ns;
 };
 
-// coefficient slot layout (floats): cum2[Q] | gam[Q] | w[Q] | psi_end[N/2] | cum2_end
+// coefficient slot layout (floats): cum2[Q] | gam[Q] | w[Q] | ew[Q] | psi_end[N/2] | cum2_end
+//   cum2: chunk-relative log2-decay prefix; ew_u = log2(w_u) - cum2_u (mask exponent offset);
+//   psi_end: call-relative angle of each pair at the chunk end (reduced mod 2 pi)
 template <int NST, int Q, int R>
 struct Coef {
     float* base;
     __device__ float* cum2() const { return base; }
     __device__ float* gam() const { return base + Q; }
     __device__ float* w() const { return base + 2 * Q; }
-    __device__ float* psi_end() const { return base + 3 * Q; }
-    __device__ float* cum2_end() const { return base + 3 * Q + NST / 2; }
+    __device__ float* ew() const { return base + 3 * Q; }
+    __device__ float* psi_end() const { return base + 4 * Q; }
+    __device__ float* cum2_end() const { return base + 4 * Q + NST / 2; }
 };
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // A wait taken by all 32 lanes of a warp together: the outcome is made warp-uniform so
 // that no lane reaches a .sync.aligned tcgen05 instruction without the others.
@@ -165,13 +223,15 @@ template <int NST, int Q, int R>
 __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
                            const Abort& ab) {
     using C = Cfg<NST, Q, R>;
-    const uint32_t s_ct = smem_u32(sm + C::OFF_CT), s_bt = smem_u32(sm + C::OFF_BT);
-    const uint32_t s_xw = smem_u32(sm + C::OFF_XW), s_sl = smem_u32(sm + C::OFF_SL);
-    const uint32_t s_g = smem_u32(sm + C::OFF_G);
+    const uint32_t s_sl = smem_u32(sm + C::OFF_SL), s_g = smem_u32(sm + C::OFF_G);
     for (int c = 0; c < p.nchunks; ++c) {
         const uint32_t ph = c & 1;
-        const int st = c & 1;
-        if (!mbar_wait(&bar[OPS_FULL], ph, ab)) return;
+        const int st = c & 1, yb = c & 1;
+        const int slot = c % C::OPS;
+        const uint32_t s_ct = smem_u32(C::ct(sm, slot)), s_bt = smem_u32(C::bt(sm, slot));
+        const uint32_t s_xw = smem_u32(C::xw(sm, slot));
+        if (!mbar_wait(&bar[OPS_FULL0 + slot], (c / C::OPS) & 1, ab)) return;
+        M3_TRACE_EV(c, 6);
         tc_fence_after();
         // S = C~ B~^T   (M = L tokens*ranks, N = L, K = NST)
         if (!mbar_wait(&bar[S_EMPTY], ph ^ 1, ab)) return;
@@ -180,6 +240,7 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
         for (int k = 0; k < NST / 16; ++k)
             mma_bf16(tmem + C::TM_S, desc_k(s_ct, k, C::L), desc_k(s_bt, k, C::L), C::ID_S, k > 0);
         mma_commit(&bar[S_FULL]);
+        M3_TRACE_EV(c, 7);
         // dS = B~^T Xw  (M = NST, N = P, K = L)
         if (!mbar_wait(&bar[DS_EMPTY], ph ^ 1, ab)) return;
         tc_fence_after();
@@ -188,144 +249,243 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
             mma_bf16(tmem + C::TM_DS, desc_mn(s_bt, k, C::L * 128u), desc_mn(s_xw, k, 1024u),
                      C::ID_DS, k > 0);
         mma_commit(&bar[DS_FULL]);
+        M3_TRACE_EV(c, 8);
         // Y_inter = C~ g  (M = L, N = P, K = NST)
         if (!mbar_wait(&bar[G_FULL], ph, ab)) return;
-        if (!mbar_wait(&bar[Y_EMPTY], ph ^ 1, ab)) return;
+        M3_TRACE_EV(c, 9);
+        if (!mbar_wait(&bar[Y_EMPTY0 + yb], ((c >> 1) & 1) ^ 1, ab)) return;
+        M3_TRACE_EV(c, 10);
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < NST / 16; ++k)
-            mma_bf16(tmem + C::TM_YI, desc_k(s_ct, k, C::L), desc_mn(s_g, k, 1024u), C::ID_Y,
+            mma_bf16(tmem + C::tm_yi(yb), desc_k(s_ct, k, C::L), desc_mn(s_g, k, 1024u), C::ID_Y,
                      k > 0);
         mma_commit(&bar[G_EMPTY]);
-        mma_commit(&bar[OPS_EMPTY]);
+        mma_commit(&bar[OPS_EMPTY0 + slot]);
+        M3_TRACE_EV(c, 11);
         // Y_intra = (S o L) X  (M = L, N = P, K = L)
         if (!mbar_wait(&bar[SL_FULL], ph, ab)) return;
+        M3_TRACE_EV(c, 12);
         if (!mbar_wait(&bar[X_FULL0 + st], (c >> 1) & 1, ab)) return;
         tc_fence_after();
         const uint32_t s_x = smem_u32(sm + C::OFF_X + st * C::X_BYTES);
 #pragma unroll
         for (int k = 0; k < C::L / 16; ++k)
-            mma_bf16(tmem + C::TM_YA, desc_k(s_sl, k, C::L), desc_mn(s_x, k, 1024u), C::ID_Y,
+            mma_bf16(tmem + C::tm_ya(yb), desc_k(s_sl, k, C::L), desc_mn(s_x, k, 1024u), C::ID_Y,
                      k > 0);
-        mma_commit(&bar[Y_FULL]);
+        mma_commit(&bar[Y_FULL0 + yb]);
+        M3_TRACE_EV(c, 13);
     }
 }
 
 // ---------------------------------------------------------------------------------
-// Rotation warpgroup: coefficients, rotated B~ / C~ and the w-scaled X operand.
+// Rotation warpgroup: B~ and C~ operands.  Warp ts handles tokens [ts*TPT, (ts+1)*TPT)
+// of every raw sub-chunk; lane l handles state pairs PPT*l .. PPT*l+PPT-1 (all pairs of a
+// token across the warp).  The chunk-start angle of a thread's token range is the
+// running angle plus the angle sums of the earlier ranges, exchanged through shared
+// memory once per sub-chunk.
 template <int NST, int Q, int R>
 __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
     using C = Cfg<NST, Q, R>;
+    constexpr int PPT = C::PPT, TPT = C::TPT, PAIRS = C::PAIRS;
     const ScanArgs& a = p.a;
     const int tid = threadIdx.x - 192;          // 0..127
-    const int rw = tid >> 5, lane = tid & 31;
-    const int pb = rw % C::PBLK, ts = rw / C::PBLK;
-    const int pair = pb * 32 + lane;             // this thread's state pair
+    const int ts = tid >> 5, lane = tid & 31;
+    const int pair0 = lane * PPT;                // first state pair of this thread
     const int hq = (blockIdx.x % a.H) & 3;       // column of this head in the 4-head dt tile
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
-    uint8_t* ct = sm + C::OFF_CT;
-    uint8_t* bt = sm + C::OFF_BT;
-    const int atom = (2 * pair) >> 6, col = (2 * pair) & 63;
+    const int atom = (2 * pair0) >> 6, col = (2 * pair0) & 63;
+    float* rsum = reinterpret_cast<float*>(sm + C::OFF_RSUM);
     int raw_it = 0;
+    // call-relative angles of this thread's pairs (the RoPE frame of Proposition 4 starts
+    // at the first token of the call), reduced mod 2 pi at chunk boundaries
+    float psi_acc[PPT];
+#pragma unroll
+    for (int k = 0; k < PPT; ++k) psi_acc[k] = 0.f;
     for (int c = 0; c < p.nchunks; ++c) {
-        const int st = c & 1;
+        const int st = c & 1, slot = c % C::OPS;
+        const uint32_t ph2 = (c >> 1) & 1;
+        if (!warp_wait(&bar[DT_FULL0 + st], ph2, ab)) return;
+        if (tid == 0) M3_TRACE_EV(c, 0);
+        const float* dtt = reinterpret_cast<const float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
+        uint8_t* ct = C::ct(sm, slot);
+        uint8_t* bt = C::bt(sm, slot);
+        if (!warp_wait(&bar[OPS_EMPTY0 + slot], ((c / C::OPS) & 1) ^ 1, ab)) return;
+        if (tid == 0) M3_TRACE_EV(c, 1);
+        for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
+            const int rs = raw_it & 1;
+            if (!warp_wait(&bar[RAW_FULL0 + rs], (raw_it >> 1) & 1, ab)) return;
+            if (tid == 0 && s == 0) M3_TRACE_EV(c, 2);
+            const uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
+            const uint32_t* braw = reinterpret_cast<const uint32_t*>(raw);
+            const uint32_t* craw = reinterpret_cast<const uint32_t*>(raw + C::BRAW_BYTES);
+            const float* th = reinterpret_cast<const float*>(raw + 2 * C::BRAW_BYTES);
+            const int tb = s * C::RT;           // first token of the sub-chunk (chunk-relative)
+            const int j0 = ts * TPT;
+            // angle increments of the own tokens and their sum per pair
+            float ph[TPT][PPT], own[PPT];
+#pragma unroll
+            for (int k = 0; k < PPT; ++k) own[k] = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < TPT; ++jj) {
+                const int j = j0 + jj;
+                const float d = angle ? 1.f : dtt[(tb + j) * 4 + hq];
+                if constexpr (PPT == 2) {
+                    const float2 tv = *reinterpret_cast<const float2*>(th + j * PAIRS + pair0);
+                    ph[jj][0] = d * tv.x;
+                    ph[jj][1] = d * tv.y;
+                } else {
+                    ph[jj][0] = d * th[j * PAIRS + pair0];
+                }
+#pragma unroll
+                for (int k = 0; k < PPT; ++k) own[k] += ph[jj][k];
+            }
+            // exchange the range sums of the four token ranges
+            float* rb = rsum + (rs * 4) * PAIRS;
+#pragma unroll
+            for (int k = 0; k < PPT; ++k) rb[ts * PAIRS + pair0 + k] = own[k];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[RS0 + rs]);
+            // raw B, C of the own tokens (independent of the exchange)
+            uint32_t bv[TPT][R][PPT], cv[TPT][R][PPT];
+#pragma unroll
+            for (int jj = 0; jj < TPT; ++jj)
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int e = (((j0 + jj) * R + r) * NST) / 2 + pair0;
+                    if constexpr (PPT == 2) {
+                        const uint2 b2 = *reinterpret_cast<const uint2*>(braw + e);
+                        const uint2 c2 = *reinterpret_cast<const uint2*>(craw + e);
+                        bv[jj][r][0] = b2.x; bv[jj][r][1] = b2.y;
+                        cv[jj][r][0] = c2.x; cv[jj][r][1] = c2.y;
+                    } else {
+                        bv[jj][r][0] = braw[e];
+                        cv[jj][r][0] = craw[e];
+                    }
+                }
+            if (!warp_wait(&bar[RS0 + rs], (raw_it >> 1) & 1, ab)) return;
+            float psi[PPT], tot[PPT];
+#pragma unroll
+            for (int k = 0; k < PPT; ++k) {
+                float pre = 0.f, all = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float v = rb[q * PAIRS + pair0 + k];
+                    all += v;
+                    pre += (q < ts) ? v : 0.f;
+                }
+                psi[k] = psi_acc[k] + pre;
+                tot[k] = all;
+            }
+#pragma unroll
+            for (int jj = 0; jj < TPT; ++jj) {
+                float sn[PPT], cn[PPT];
+#pragma unroll
+                for (int k = 0; k < PPT; ++k) {
+                    psi[k] += ph[jj][k];
+                    __sincosf(psi[k], &sn[k], &cn[k]);   // |psi| < pi + one chunk of increments
+                }
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    uint32_t bo[PPT], co[PPT];
+#pragma unroll
+                    for (int k = 0; k < PPT; ++k) {
+                        const float b0 = bf16lo(bv[jj][r][k]), b1 = bf16hi(bv[jj][r][k]);
+                        const float c0 = bf16lo(cv[jj][r][k]), c1 = bf16hi(cv[jj][r][k]);
+                        // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1]
+                        bo[k] = pack_bf16x2(fmaf(cn[k], b0, sn[k] * b1), fmaf(cn[k], b1, -sn[k] * b0));
+                        co[k] = pack_bf16x2(fmaf(cn[k], c0, sn[k] * c1), fmaf(cn[k], c1, -sn[k] * c0));
+                    }
+                    const int row = (tb + j0 + jj) * R + r;
+                    const uint32_t off = (uint32_t)atom * C::L * 128u + sw128_off(row, col);
+                    if constexpr (PPT == 2) {
+                        *reinterpret_cast<uint2*>(bt + off) = make_uint2(bo[0], bo[1]);
+                        *reinterpret_cast<uint2*>(ct + off) = make_uint2(co[0], co[1]);
+                    } else {
+                        *reinterpret_cast<uint32_t*>(bt + off) = bo[0];
+                        *reinterpret_cast<uint32_t*>(ct + off) = co[0];
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < PPT; ++k) psi_acc[k] += tot[k];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[RAW_EMPTY0 + rs]);
+        }
+        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + st * C::COEF_FLOATS};
+#pragma unroll
+        for (int k = 0; k < PPT; ++k) {
+            psi_acc[k] -= 6.283185307179586f * rintf(psi_acc[k] * 0.15915494309189535f);
+            if (ts == 0) cf.psi_end()[pair0 + k] = psi_acc[k];
+        }
+        if (tid == 0) M3_TRACE_EV(c, 3);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&bar[COEF_FULL0 + st]);
+            mbar_arrive(&bar[OPS_FULL0 + slot]);
+            mbar_arrive(&bar[DT_EMPTY0 + st]);
+        }
+        if (tid == 0) M3_TRACE_EV(c, 5);
+    }
+}
+
+// Coefficient warp: per-token log2-decay prefix sum (warp scan), gamma, w and the mask
+// exponent offsets of each chunk, and the w-scaled X operand
+//   Xw[u, r] = 2^(cum2_end - cum2_u) w_u x[u, r].
+template <int NST, int Q, int R>
+__device__ void coefficients(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
+    using C = Cfg<NST, Q, R>;
+    const ScanArgs& a = p.a;
+    const int lane = threadIdx.x & 31;
+    const int hq = (blockIdx.x % a.H) & 3;
+    for (int c = 0; c < p.nchunks; ++c) {
+        const int st = c & 1, slot = c % C::OPS;
         const uint32_t ph2 = (c >> 1) & 1;
         if (!warp_wait(&bar[DT_FULL0 + st], ph2, ab)) return;
         const float* dtt = reinterpret_cast<const float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
         const float* At = dtt + C::DT_BYTES / 4;
         const float* lt = dtt + 2 * C::DT_BYTES / 4;
         Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + st * C::COEF_FLOATS};
-
-        // ---- per-token coefficients (rotation warp 0): log2-decay prefix sum, gamma, w
-        if (rw == 0) {
-            if (!warp_wait(&bar[COEF_EMPTY0 + st], ph2 ^ 1, ab)) return;
-            float carry = 0.f;
-            for (int t0 = 0; t0 < Q; t0 += 32) {
-                const int t = t0 + lane;
-                float l2 = 0.f, gm = 0.f, wv = 0.f;
-                if (t < Q) {
-                    const float d = dtt[t * 4 + hq], lm = lt[t * 4 + hq];
-                    l2 = d * At[t * 4 + hq] * kLog2e;
-                    gm = lm * d;
-                    const float dn = dtt[(t + 1) * 4 + hq], ln = lt[(t + 1) * 4 + hq];
-                    wv = gm + (1.f - ln) * dn;
-                }
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, l2, o);
-                    if (lane >= o) l2 += v;
-                }
-                l2 += carry;
-                if (t < Q) {
-                    cf.cum2()[t] = l2;
-                    cf.gam()[t] = gm;
-                    cf.w()[t] = wv;
-                }
-                carry = __shfl_sync(0xffffffffu, l2, 31);
+        if (!warp_wait(&bar[COEF_EMPTY0 + st], ph2 ^ 1, ab)) return;
+        float carry = 0.f;
+        for (int t0 = 0; t0 < Q; t0 += 32) {
+            const int t = t0 + lane;
+            float l2 = 0.f, gm = 0.f, wv = 0.f;
+            if (t < Q) {
+                const float d = dtt[t * 4 + hq], lm = lt[t * 4 + hq];
+                l2 = d * At[t * 4 + hq] * kLog2e;
+                gm = lm * d;
+                const float dn = dtt[(t + 1) * 4 + hq], ln = lt[(t + 1) * 4 + hq];
+                wv = gm + (1.f - ln) * dn;
             }
-            if (lane == 0) *cf.cum2_end() = carry;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[CUM_READY0 + st]);
-        }
-
-        // ---- rotated operands: wait until the MMAs of the previous chunk released them
-        if (!warp_wait(&bar[OPS_EMPTY], (c & 1) ^ 1, ab)) return;
-        float psi_acc = 0.f;
-        for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
-            const int rs = raw_it & 1;
-            if (!warp_wait(&bar[RAW_FULL0 + rs], (raw_it >> 1) & 1, ab)) return;
-            const uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
-            const uint32_t* braw = reinterpret_cast<const uint32_t*>(raw);
-            const uint32_t* craw = reinterpret_cast<const uint32_t*>(raw + C::BRAW_BYTES);
-            const float* th = reinterpret_cast<const float*>(raw + 2 * C::BRAW_BYTES);
-            const int tb = s * C::RT;           // first token of the sub-chunk (chunk-relative)
-            const int j0 = ts * C::TPT, j1 = j0 + C::TPT;
-            float psi = psi_acc;
-            for (int j = 0; j < j0; ++j)
-                psi += angle ? th[j * C::PAIRS + pair] : dtt[(tb + j) * 4 + hq] * th[j * C::PAIRS + pair];
-            for (int j = j0; j < j1; ++j) {
-                const float d = dtt[(tb + j) * 4 + hq];
-                psi += angle ? th[j * C::PAIRS + pair] : d * th[j * C::PAIRS + pair];
-                const float pr = psi - 6.283185307179586f * rintf(psi * 0.15915494309189535f);
-                float sn, cn;
-                __sincosf(pr, &sn, &cn);
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int rowr = j * R + r;
-                    const uint32_t bv = braw[(rowr * NST) / 2 + pair];
-                    const uint32_t cv = craw[(rowr * NST) / 2 + pair];
-                    const float b0 = bf16lo(bv), b1 = bf16hi(bv);
-                    const float c0 = bf16lo(cv), c1 = bf16hi(cv);
-                    // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1]
-                    const uint32_t bo = pack_bf16x2(fmaf(cn, b0, sn * b1), fmaf(cn, b1, -sn * b0));
-                    const uint32_t co = pack_bf16x2(fmaf(cn, c0, sn * c1), fmaf(cn, c1, -sn * c0));
-                    const int row = (tb + j) * R + r;
-                    const uint32_t off = (uint32_t)atom * C::L * 128u + sw128_off(row, col);
-                    *reinterpret_cast<uint32_t*>(bt + off) = bo;
-                    *reinterpret_cast<uint32_t*>(ct + off) = co;
-                }
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, l2, o);
+                if (lane >= o) l2 += v;
             }
-            for (int j = j1; j < C::RT; ++j)
-                psi += angle ? th[j * C::PAIRS + pair] : dtt[(tb + j) * 4 + hq] * th[j * C::PAIRS + pair];
-            psi_acc = psi;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[RAW_EMPTY0 + rs]);
+            l2 += carry;
+            if (t < Q) {
+                cf.cum2()[t] = l2;
+                cf.gam()[t] = gm;
+                cf.w()[t] = wv;
+                cf.ew()[t] = __log2f(wv) - l2;   // -inf when w = 0: the mask entry is 0
+            }
+            carry = __shfl_sync(0xffffffffu, l2, 31);
         }
-        if (ts == 0) cf.psi_end()[pair] = psi_acc;
+        if (lane == 0) *cf.cum2_end() = carry;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[COEF_FULL0 + st]);
-        // the per-token coefficients of rotation warp 0 are needed below
-        if (!warp_wait(&bar[CUM_READY0 + st], ph2, ab)) return;
 
-        // ---- w-scaled X:  Xw[u, r] = e^{cum_end - cum_u} w_u x[u, r]
         if (!warp_wait(&bar[X_FULL0 + st], ph2, ab)) return;
+        if (!warp_wait(&bar[OPS_EMPTY0 + slot], ((c / C::OPS) & 1) ^ 1, ab)) return;
+        if (lane == 0) M3_TRACE_EV(c, 4);
         const uint8_t* xt = sm + C::OFF_X + st * C::X_BYTES;
-        uint8_t* xw = sm + C::OFF_XW;
-        const float cend = *cf.cum2_end();
-        for (int idx = tid; idx < C::L * 8; idx += 128) {
+        uint8_t* xw = C::xw(sm, slot);
+#pragma unroll 4
+        for (int idx = lane; idx < C::L * 8; idx += 32) {
             const int row = idx >> 3, ch = idx & 7;
             const int u = row / R;
-            const float sc = exp2f(cend - cf.cum2()[u]) * cf.w()[u];
+            const float sc = ex2_approx(carry - cf.cum2()[u]) * cf.w()[u];
             const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((ch ^ row) & 7) << 4);
             uint4 v = *reinterpret_cast<const uint4*>(xt + off);
             uint4 o;
@@ -338,7 +498,8 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            mbar_arrive(&bar[OPS_FULL]);
+            mbar_arrive(&bar[COEF_FULL0 + st]);
+            mbar_arrive(&bar[OPS_FULL0 + slot]);
             mbar_arrive(&bar[DT_EMPTY0 + st]);
         }
     }
@@ -373,24 +534,34 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
     const int ncol0 = kHalfN ? 32 * (lane >> 4) : 0;
     constexpr int kNCols = kHalfN ? 32 : kP;
 
-    float gv[kNCols];                                       // fp32 state, row nrow
     uint8_t* gs = sm + C::OFF_G;
     uint8_t* sl = sm + C::OFF_SL;
 
-    // g (bf16, MN-major [n][p]) for the Y_inter MMA
-    auto publish_g = [&]() {
+    // The fp32 carried state g lives in TMEM columns TM_G.. with the lane layout of the
+    // dS accumulator (this thread: row nrow, columns ncol0..); 32 columns at a time.
+    auto tm_ld = [&](uint32_t col, int cb, uint32_t (&v)[32]) {
+        if (kHalfN)
+            tmem_ld_16x32bx2_x32<32>(tq + col, v);
+        else
+            tmem_ld_32x32b_x32(tq + col + cb, v);
+    };
+    auto tm_st = [&](uint32_t col, int cb, const uint32_t (&v)[32]) {
+        if (kHalfN)
+            tmem_st_16x32bx2_x32<32>(tq + col, v);
+        else
+            tmem_st_32x32b_x32(tq + col + cb, v);
+    };
+    // bf16 copy of 32 state columns for the Y_inter MMA operand (MN-major [n][p])
+    auto publish_block = [&](int cb, const uint32_t (&v)[32]) {
 #pragma unroll
-        for (int j = 0; j < kNCols; j += 8) {
+        for (int j = 0; j < 32; j += 8) {
             uint4 o;
-            o.x = pack_bf16x2(gv[j], gv[j + 1]);
-            o.y = pack_bf16x2(gv[j + 2], gv[j + 3]);
-            o.z = pack_bf16x2(gv[j + 4], gv[j + 5]);
-            o.w = pack_bf16x2(gv[j + 6], gv[j + 7]);
-            *reinterpret_cast<uint4*>(gs + sw128_off(nrow, ncol0 + j)) = o;
+            o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+            o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+            o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+            o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+            *reinterpret_cast<uint4*>(gs + sw128_off(nrow, ncol0 + cb + j)) = o;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[G_FULL]);
     };
 
     // ---- g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T
@@ -401,20 +572,32 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
         const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(a.x_prev) + bh * R * kP;
         const __nv_bfloat16* bp =
             static_cast<const __nv_bfloat16*>(a.B_prev) + ((size_t)b * a.G + g) * R * NST;
+#pragma unroll 1
+        for (int cb = 0; cb < kNCols; cb += 32) {
+            float gv[32];
 #pragma unroll
-        for (int j = 0; j < kNCols; j += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(h0 + j);
-            gv[j] = v.x; gv[j + 1] = v.y; gv[j + 2] = v.z; gv[j + 3] = v.w;
+            for (int j = 0; j < 32; j += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(h0 + cb + j);
+                gv[j] = v.x; gv[j + 1] = v.y; gv[j + 2] = v.z; gv[j + 3] = v.w;
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float bb = beta0 * __bfloat162float(bp[r * NST + nrow]);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    gv[j] = fmaf(bb, __bfloat162float(xp[r * kP + ncol0 + cb + j]), gv[j]);
+            }
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(gv[j]);
+            tm_st(C::TM_G, cb, v);
+            publish_block(cb, v);
         }
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const float bb = beta0 * __bfloat162float(bp[r * NST + nrow]);
-#pragma unroll
-            for (int j = 0; j < kNCols; ++j)
-                gv[j] = fmaf(bb, __bfloat162float(xp[r * kP + ncol0 + j]), gv[j]);
-        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[G_FULL]);
     }
-    publish_g();
 
     bool ok = true;
     for (int c = 0; c < p.nchunks && ok; ++c) {
@@ -422,17 +605,23 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
         const int st = c & 1;
         Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + st * C::COEF_FLOATS};
         if (!(ok = warp_wait(&bar[COEF_FULL0 + st], ph2, ab))) break;
+        if (etid == 0) M3_TRACE_EV(c, 14);
         const float* cum2 = cf.cum2();
 
         // ---- S o L  ->  bf16, K-major [row][col] with L[t,u] = e^{cum_t-cum_u} (u<t ? w_u : gamma_u)
         if (!(ok = warp_wait(&bar[S_FULL], ph, ab))) break;
+        if (etid == 0) M3_TRACE_EV(c, 15);
         tc_fence_after();
         {
+            // L[t,u] = 2^(cum2_t - cum2_u) w_u = 2^(cum2_t + ew_u) for u < t, gamma_t on the
+            // diagonal token; the skip D x is folded in as D on the (row == col) diagonal.
             const int t = lrow / R;
             const float ct = cum2[t];
+            const float gt = cf.gam()[t];
+            const float* ew = cf.ew();
 #pragma unroll 1
             for (int cb = 0; cb < kLCols; cb += 32) {
-                float s[32];
+                uint32_t s[32];
                 if (kHalfL)
                     tmem_ld_16x32bx2_x32<32>(tq + C::TM_S, s);
                 else
@@ -444,9 +633,12 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
                     float m[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int u = (colb + j + e) / R;
-                        const float cu = (u < t) ? cf.w()[u] : cf.gam()[u];
-                        m[e] = (u <= t) ? s[j + e] * exp2f(ct - cum2[u]) * cu : 0.f;
+                        const int col = colb + j + e;
+                        const int u = col / R;
+                        const float sv = __uint_as_float(s[j + e]);
+                        const float v = sv * ex2_approx(ct + ew[u]);
+                        m[e] = (u < t) ? v : 0.f;
+                        if (u == t) m[e] = sv * gt + (col == lrow ? Dh : 0.f);
                     }
                     uint4 o;
                     o.x = pack_bf16x2(m[0], m[1]);
@@ -466,72 +658,73 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
             mbar_arrive(&bar[S_EMPTY]);
             mbar_arrive(&bar[SL_FULL]);
         }
+        if (etid == 0) M3_TRACE_EV(c, 16);
 
-        // ---- state: g <- R(psi_end) (e^{cum_end} g + dS), then publish it for the next chunk
+        // ---- state (RoPE frame of the call): g <- e^{cum_end} g + dS, published for the next chunk
         if (!(ok = warp_wait(&bar[DS_FULL], ph, ab))) break;
+        if (etid == 0) M3_TRACE_EV(c, 17);
+        const bool more = c + 1 < p.nchunks;
+        // the Y_inter MMA of this chunk must be done reading g_c before g_{c+1} replaces it
+        if (more && !(ok = warp_wait(&bar[G_EMPTY], ph, ab))) break;
+        if (etid == 0) M3_TRACE_EV(c, 19);
         tc_fence_after();
         {
             const float dec = exp2f(*cf.cum2_end());
-#pragma unroll
+#pragma unroll 1
             for (int cb = 0; cb < kNCols; cb += 32) {
-                float d[32];
-                if (kHalfN)
-                    tmem_ld_16x32bx2_x32<32>(tq + C::TM_DS, d);
-                else
-                    tmem_ld_32x32b_x32(tq + C::TM_DS + cb, d);
+                uint32_t d[32], gq[32];
+                tm_ld(C::TM_DS, cb, d);
+                tm_ld(C::TM_G, cb, gq);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) gv[cb + j] = fmaf(dec, gv[cb + j], d[j]);
+                for (int j = 0; j < 32; ++j)
+                    gq[j] = __float_as_uint(fmaf(dec, __uint_as_float(gq[j]), __uint_as_float(d[j])));
+                tm_st(C::TM_G, cb, gq);
+                if (more) publish_block(cb, gq);
             }
-            float sn, cn;
-            sincosf(cf.psi_end()[nrow >> 1], &sn, &cn);
-            const bool odd = nrow & 1;
-#pragma unroll
-            for (int j = 0; j < kNCols; ++j) {
-                const float o = __shfl_xor_sync(0xffffffffu, gv[j], 1);
-                gv[j] = odd ? fmaf(sn, o, cn * gv[j]) : fmaf(cn, gv[j], -sn * o);
-            }
+            tmem_wait_st();
         }
         tc_fence_before();
+        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[DS_EMPTY]);
-        if (c + 1 < p.nchunks) {
-            // the Y_inter MMA of this chunk must be done reading g_c
-            if (!(ok = warp_wait(&bar[G_EMPTY], ph, ab))) break;
-            publish_g();
+        if (lane == 0) {
+            mbar_arrive(&bar[DS_EMPTY]);
+            if (more) mbar_arrive(&bar[G_FULL]);
         }
+        if (etid == 0) M3_TRACE_EV(c, 18);
 
-        // ---- y = Y_intra + e^{cum_t} Y_inter + D x   (written over the x tile, then TMA store)
-        if (!(ok = warp_wait(&bar[Y_FULL], ph, ab))) break;
+        // ---- y = Y_intra + e^{cum_t} Y_inter   (D x is in Y_intra; y is written over the
+        //      x tile, then stored with TMA)
+        const int yb = c & 1;
+        if (!(ok = warp_wait(&bar[Y_FULL0 + yb], ph2, ab))) break;
+        if (etid == 0) M3_TRACE_EV(c, 20);
         if (!(ok = warp_wait(&bar[X_FULL0 + st], ph2, ab))) break;
         tc_fence_after();
+        if (etid == 0) M3_TRACE_EV(c, 21);
         uint8_t* xt = sm + C::OFF_X + st * C::X_BYTES;
         {
             const float sc = exp2f(cum2[lrow / R]);
 #pragma unroll 1
             for (int cb = 0; cb < kYCols; cb += 32) {
-                float ya[32], yi[32];
+                uint32_t ya[32], yi[32];
                 if (kHalfL) {
-                    tmem_ld_16x32bx2_x32<32>(tq + C::TM_YA, ya);
-                    tmem_ld_16x32bx2_x32<32>(tq + C::TM_YI, yi);
+                    tmem_ld_16x32bx2_x32<32>(tq + C::tm_ya(yb), ya);
+                    tmem_ld_16x32bx2_x32<32>(tq + C::tm_yi(yb), yi);
                 } else {
-                    tmem_ld_32x32b_x32(tq + C::TM_YA + cb, ya);
-                    tmem_ld_32x32b_x32(tq + C::TM_YI + cb, yi);
+                    tmem_ld_32x32b_x32(tq + C::tm_ya(yb) + cb, ya);
+                    tmem_ld_32x32b_x32(tq + C::tm_yi(yb) + cb, yi);
                 }
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; j += 8) {
                     const uint32_t off = sw128_off(lrow, lcol0 + cb + j);
-                    const uint4 xv = *reinterpret_cast<const uint4*>(xt + off);
-                    const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
                     uint32_t o[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float y0 = fmaf(sc, yi[j + 2 * e], ya[j + 2 * e]) + Dh * bf16lo(xs[e]);
-                        const float y1 =
-                            fmaf(sc, yi[j + 2 * e + 1], ya[j + 2 * e + 1]) + Dh * bf16hi(xs[e]);
-                        o[e] = pack_bf16x2(y0, y1);
-                    }
+                    for (int e = 0; e < 4; ++e)
+                        o[e] = pack_bf16x2(
+                            fmaf(sc, __uint_as_float(yi[j + 2 * e]), __uint_as_float(ya[j + 2 * e])),
+                            fmaf(sc, __uint_as_float(yi[j + 2 * e + 1]),
+                                 __uint_as_float(ya[j + 2 * e + 1])));
                     *reinterpret_cast<uint4*>(xt + off) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
@@ -540,9 +733,10 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            mbar_arrive(&bar[Y_EMPTY]);
+            mbar_arrive(&bar[Y_EMPTY0 + yb]);
             mbar_arrive(&bar[Y_STAGED]);
         }
+        if (etid == 0) M3_TRACE_EV(c, 22);
         if (etid == 0) {
             // all four warps have written their rows of y (and are done with this chunk's
             // coefficients): store the tile, then hand the x stage back to the producer
@@ -552,6 +746,7 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
                 tma_store_5d(&p.tm_y, xt, 0, 0, h, c * Q, b);
                 bulk_commit();
                 bulk_wait_read<0>();
+                M3_TRACE_EV(c, 23);
                 mbar_arrive(&bar[X_EMPTY0 + st]);
             }
         }
@@ -559,11 +754,31 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
     }
 
     if (ok) {
-        // final state h_T (original frame) and the carried previous x
+        // final state: back from the RoPE frame of the call, h_T = R(psi_T) g
+        const float* pe = reinterpret_cast<const float*>(sm + C::OFF_COEF) +
+                          ((p.nchunks - 1) & 1) * C::COEF_FLOATS + 4 * Q;
+        float sn, cn;
+        sincosf(pe[nrow >> 1], &sn, &cn);
+        const bool odd = nrow & 1;
         float* hT = a.h + (bh * NST + nrow) * kP + ncol0;
+        tc_fence_after();
+#pragma unroll 1
+        for (int cb = 0; cb < kNCols; cb += 32) {
+            uint32_t gq[32];
+            tm_ld(C::TM_G, cb, gq);
+            tmem_wait_ld();
+            float gv[32];
 #pragma unroll
-        for (int j = 0; j < kNCols; j += 4)
-            *reinterpret_cast<float4*>(hT + j) = make_float4(gv[j], gv[j + 1], gv[j + 2], gv[j + 3]);
+            for (int j = 0; j < 32; ++j) {
+                const float gj = __uint_as_float(gq[j]);
+                const float o = __shfl_xor_sync(0xffffffffu, gj, 1);
+                gv[j] = odd ? fmaf(sn, o, cn * gj) : fmaf(cn, gj, -sn * o);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(hT + cb + j) =
+                    make_float4(gv[j], gv[j + 1], gv[j + 2], gv[j + 3]);
+        }
         if (etid == 0) {
             // every epilogue warp passed chunk 0 (it read x_prev there) before the last
             // Y_STAGED completed, so x_prev can be overwritten now
@@ -598,6 +813,7 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         const uint32_t ph = ((c >> 1) & 1) ^ 1;
         // per-chunk dt / A / lam (Q+1 tokens: the next chunk's first token is the lookahead)
         if (!(ok = mbar_wait(&bar[DT_EMPTY0 + st], ph, ab))) break;
+        M3_TRACE_EV(c, 24);
         mbar_arrive_expect_tx(&bar[DT_FULL0 + st], 3 * C::DT_BOX);
         float* dtt = reinterpret_cast<float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
         tma_load_3d(dtt, &p.tm_dt, &bar[DT_FULL0 + st], h & ~3, t0, b);
@@ -608,6 +824,7 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
             const int rs = raw_it & 1;
             if (!(ok = mbar_wait(&bar[RAW_EMPTY0 + rs], ((raw_it >> 1) & 1) ^ 1, ab))) break;
+            if (s == 0) M3_TRACE_EV(c, 25);
             mbar_arrive_expect_tx(&bar[RAW_FULL0 + rs], C::RAW_BYTES);
             uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
             const int tr = t0 + s * C::RT;
@@ -617,6 +834,7 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
             ++n_raw[rs];
             if (s == 0) {
                 if (!(ok = mbar_wait(&bar[X_EMPTY0 + st], ph, ab))) break;
+                M3_TRACE_EV(c, 26);
                 mbar_arrive_expect_tx(&bar[X_FULL0 + st], C::X_BYTES);
                 tma_load_5d(sm + C::OFF_X + st * C::X_BYTES, &p.tm_x, &bar[X_FULL0 + st], 0, 0, h,
                             t0, b);
@@ -645,15 +863,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     const int w = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
-        const uint32_t counts[NUM_BARS] = {
-            1, 1, 4, 4,          // raw full / empty
-            1, 1, 4, 4,          // dt full / empty
-            1, 1, 1, 1,          // x full / empty
-            4, 4, 1, 1, 1, 1,    // coef full / empty, cumulative-decay ready
-            4, 1, 1, 4, 4, 1, 4, // ops full/empty, S full/empty, SL full, dS full/empty
-            4, 1, 1, 4, 4, 1     // g full/empty, y full/empty, y staged, drain
-        };
-        for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], counts[i]);
+        for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], bar_count(i));
         misc[1] = 0u;  // abort flag
         fence_mbar_init();
         tma_prefetch_desc(&p.tm_x);
@@ -683,8 +893,10 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         }
     } else if (w < 6) {
         epilogue<NST, Q, R>(p, sm, bar, tmem, ab);
-    } else {
+    } else if (w < 10) {
         rotation<NST, Q, R>(p, sm, bar, ab);
+    } else {
+        coefficients<NST, Q, R>(p, sm, bar, ab);
     }
     tc_fence_before();
     __syncthreads();
@@ -786,6 +998,14 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+#ifdef M3_TRACE
+extern "C" int m3_trace_copy(void* dst, size_t bytes, int cta) {
+    if (cudaMemcpyToSymbol(g_m3_trace_cta, &cta, sizeof(int)) != cudaSuccess) return 1;
+    if (!dst) return 0;
+    return cudaMemcpyFromSymbol(dst, g_m3_trace, bytes) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 bool scan_tc_supported(int N, int P, int R, int chunk, int H) {
     if (P != kP || H % 4 != 0) return false;
