@@ -127,6 +127,33 @@ m3_status m3_scan_fwd(const m3_dims* dims, int32_t seqlen, int32_t chunk, const 
                       void* stream);
 
 /*
+ * Prefill without a workspace argument, for callers that cannot allocate device
+ * memory (for example a plugin inside a host framework whose caching allocator owns
+ * all of the device memory, or a serving loop that must not call cudaMalloc because
+ * it can synchronise the device).  The pages describe no such entry point; this is a
+ * deployment convenience of this library.
+ *
+ * Same arguments, layouts, results and errors as m3_scan_fwd, minus the workspace.
+ * The workspace is lent from one fixed scratch array compiled into the library
+ * (64 KiB, 256-byte aligned, held on every GPU that loads the library until the
+ * process exits); shapes whose m3_scan_workspace_bytes exceeds 64 KiB are rejected
+ * with M3_ERR_WORKSPACE.  Nothing is allocated: no cudaMalloc / cudaFree and no
+ * allocating library routine.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array, and each call clears the part that must
+ *     start at zero.  Calls that can overlap on the GPU (different streams without
+ *     ordering) race on it: order them.
+ *   - The device-side status word lives in the shared array and is not reported;
+ *     callers that need m3_query_status use m3_scan_fwd with their own workspace.
+ */
+m3_status m3_scan_fwd_noalloc(const m3_dims* dims, int32_t seqlen, int32_t chunk, const void* x,
+                              const void* B, const void* C, const float* dt, const float* A,
+                              const float* lam, const float* theta, const float* D,
+                              m3_state* state, void* y, uint32_t flags, void* stream);
+
+/*
  * Decode: one token of the recurrence for every (batch, head), fused in one
  * pass over the fp32 state ("Multi-Input, Multi-Output Formulation", SISO/MIMO
  * decode step, with the trapezoid and rotation of Propositions 1 and 4).

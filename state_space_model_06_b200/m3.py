@@ -24,7 +24,7 @@ M3_FLAG_THETA_IS_ANGLE = 1
 M3_FLAG_FORCE_SIMT = 2
 
 EXPORTED = ("m3_state_bytes", "m3_state_init", "m3_scan_workspace_bytes", "m3_scan_fwd",
-            "m3_decode_step", "m3_query_status", "m3_status_string")
+            "m3_decode_step", "m3_query_status", "m3_scan_fwd_noalloc", "m3_status_string")
 
 
 class M3Error(RuntimeError):
@@ -64,6 +64,8 @@ def load_library(path: str = LIB_PATH):
         lib.m3_scan_fwd.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp, vp, sz,
                                     u32, vp]
         lib.m3_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp, u32, vp]
+        lib.m3_scan_fwd_noalloc.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp,
+                                            u32, vp]
         lib.m3_query_status.argtypes = [vp, vp]
         lib.m3_status_string.argtypes = [ctypes.c_int]
         lib.m3_status_string.restype = ctypes.c_char_p
@@ -166,6 +168,17 @@ def m3_scan_fwd(dims: Dims, seqlen: int, chunk: int, x, B, C, dt, A, lam, theta,
         ctypes.byref(dims.c()), int(seqlen), int(chunk), _ptr(x), _ptr(B), _ptr(C), _ptr(dt),
         _ptr(A), _ptr(lam), _ptr(theta), _ptr(D), ctypes.byref(st), _ptr(y), _ptr(workspace),
         ws_bytes, int(flags), _stream(stream)), "m3_scan_fwd")
+
+
+def m3_scan_fwd_noalloc(dims: Dims, seqlen: int, chunk: int, x, B, C, dt, A, lam, theta, D,
+                        state: State, y, flags: int = 0, stream=None):
+    """Prefill for callers that cannot allocate device memory: no workspace argument;
+    the library lends its own fixed scratch (see include/m3.h)."""
+    st = state.c()
+    _check(load_library().m3_scan_fwd_noalloc(
+        ctypes.byref(dims.c()), int(seqlen), int(chunk), _ptr(x), _ptr(B), _ptr(C), _ptr(dt),
+        _ptr(A), _ptr(lam), _ptr(theta), _ptr(D), ctypes.byref(st), _ptr(y), int(flags),
+        _stream(stream)), "m3_scan_fwd_noalloc")
 
 
 def m3_decode_step(dims: Dims, x, B, C, dt, A, lam, theta, D, state: State, y, flags: int = 0,
