@@ -85,6 +85,11 @@ typedef struct {
 /* Flags (bitwise OR). */
 #define M3_FLAG_THETA_IS_ANGLE 1u  /* theta already holds the per-step angle: the dt multiply is skipped */
 #define M3_FLAG_FORCE_SIMT 2u      /* m3_scan_fwd: run the sequential fp32 CUDA-core kernel */
+/* Test hook for the failure path: the tensor-core prefill's MMA warp waits on a barrier
+ * that nothing completes, with a 50 ms limit instead of 2 s.  The bounded wait gives
+ * up, the kernel aborts cleanly (outputs are invalid), and m3_query_status reports
+ * M3_ERR_TIMEOUT; the CUDA context stays usable. */
+#define M3_FLAG_TEST_STALL 4u
 
 /* Bytes of each state buffer for `dims`.  Any out-pointer may be NULL. */
 m3_status m3_state_bytes(const m3_dims* dims, size_t* h_bytes, size_t* x_prev_bytes,

@@ -69,7 +69,7 @@ enum Bar {
     X_FULL0, X_FULL1, X_EMPTY0, X_EMPTY1,
     COEF_FULL0, COEF_FULL1, COEF_EMPTY0, COEF_EMPTY1, RS0, RS1,
     OPS_FULL0, OPS_FULL1, OPS_EMPTY0, OPS_EMPTY1, S_FULL, S_EMPTY, SL_FULL, DS_FULL, DS_EMPTY,
-    G_FULL, G_EMPTY, Y_FULL0, Y_FULL1, Y_EMPTY0, Y_EMPTY1, Y_STAGED, DRAIN, NUM_BARS
+    G_FULL, G_EMPTY, Y_FULL0, Y_FULL1, Y_EMPTY0, Y_EMPTY1, Y_STAGED, DRAIN, NEVER, NUM_BARS
 };
 
 // arrival count of each barrier: 1 for TMA expect_tx / tcgen05.commit / single-thread
@@ -224,6 +224,8 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
                            const Abort& ab) {
     using C = Cfg<NST, Q, R>;
     const uint32_t s_sl = smem_u32(sm + C::OFF_SL), s_g = smem_u32(sm + C::OFF_G);
+    // failure-path test hook: wait on a barrier nothing completes (bounded, then abort)
+    if ((p.a.flags & M3_FLAG_TEST_STALL) && !mbar_wait(&bar[NEVER], 0, ab)) return;
     for (int c = 0; c < p.nchunks; ++c) {
         const uint32_t ph = c & 1;
         const int st = c & 1, yb = c & 1;
@@ -949,7 +951,7 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
     std::memset(&p, 0, sizeof(p));
     p.a = a;
     p.nchunks = (int)((a.T + Q - 1) / Q);
-    p.limit_ns = 2000000000ull;
+    p.limit_ns = (a.flags & M3_FLAG_TEST_STALL) ? 50000000ull : 2000000000ull;
     const uint64_t T = a.T, Bn = a.batch, H = a.H, G = a.G;
     bool ok = true;
     {   // x, y: (P, R, H, T, b), box (64, R, 1, Q, 1), 128B swizzle

@@ -22,6 +22,7 @@ M3_OK, M3_ERR_NULL, M3_ERR_SHAPE, M3_ERR_DTYPE, M3_ERR_ALIGN, M3_ERR_UNSUPPORTED
 M3_F32, M3_BF16 = 0, 1
 M3_FLAG_THETA_IS_ANGLE = 1
 M3_FLAG_FORCE_SIMT = 2
+M3_FLAG_TEST_STALL = 4
 
 EXPORTED = ("m3_state_bytes", "m3_state_init", "m3_scan_workspace_bytes", "m3_scan_fwd",
             "m3_decode_step", "m3_query_status", "m3_scan_fwd_noalloc", "m3_status_string")
