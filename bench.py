@@ -165,12 +165,20 @@ def dist_setup():
 
 
 def max_over_ranks(x, ws):
+    """Maximum of a per-rank float over all ranks (device times are reported as the max)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, ms_per_rank, ws):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    ms = max_over_ranks(ms_per_rank, ws)
+    return ws * units_per_rank / (ms / 1e3), ms
 
 
 def barrier(ws):
@@ -288,6 +296,10 @@ def time_decode(name, dev, stream, seed):
                        "distinct_tokens": DECODE_POOL}}
 
 
+def w_dec_batch(name):
+    return inputs.WORKLOADS[name].batch
+
+
 def oracle_sample(w, seqlen, seed=0):
     """Time the CPU oracle on batch row 0, all heads, the first `seqlen` tokens."""
     import oracle
@@ -319,9 +331,8 @@ def ours(args):
         ms, status = time_prefill(w, d, g, st, y, ws, args.steps, args.warmup, stream, ws_world)
     if status != m3.M3_OK:
         raise RuntimeError(f"device status {m3.m3_status_string(status)}")
-    ms_max = max_over_ranks(ms, ws_world)
     tokens = w.batch * w.seqlen
-    value = ws_world * tokens / (ms_max / 1e3)
+    value, ms_max = job_throughput(tokens, ms, ws_world)
     byts, flops = scan_algorithmic(w)
     achieved = byts / (ms / 1e3) / 1e9
     tflops = flops / (ms / 1e3) / 1e12
@@ -357,14 +368,14 @@ def ours(args):
         for name in DECODES:
             r = time_decode(name, dev, stream, seed=100 + rank)
             r["hbm_frac"] = r["achieved_gbs"] / pk["hbm_gbs"]
-            r["tokens_per_s"] = max_over_ranks(1.0 / r["tokens_per_s"], ws_world)
-            r["tokens_per_s"] = ws_world / r["tokens_per_s"]
+            r["tokens_per_s"], _ = job_throughput(w_dec_batch(name), r["us_per_step"] / 1e3,
+                                                  ws_world)
             line["decode"][name] = r
 
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_prefill_e2e(w, d, inp, st, ws, min(args.steps, 5), stream, dev)
-        e2e_ms = max_over_ranks(e2e_ms, ws_world)
-        line["e2e"] = {"value": ws_world * tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e_value, e2e_ms = job_throughput(tokens, e2e_ms, ws_world)
+        line["e2e"] = {"value": e2e_value, "unit": "tokens/s",
                        "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h}
 

@@ -59,28 +59,35 @@ __device__ int g_m3_trace_cta = 0;
 namespace {
 
 constexpr int kP = 64;               // head dimension handled by this kernel
-constexpr int kThreads = 352;       // 11 warps: TMA, MMA, 4 epilogue, 4 rotation, coefficients
+constexpr int kThreads = 640;       // 20 warps: TMA, MMA, 4 epilogue, 8 rotation, coefficients,
+                                     // TMA x / y, 4 state
+constexpr int kRotWarps = 8;
+constexpr int kCoefSlots = 4;       // ring of per-chunk coefficient slots
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum Bar {
     RAW_FULL0, RAW_FULL1, RAW_EMPTY0, RAW_EMPTY1,
     DT_FULL0, DT_FULL1, DT_EMPTY0, DT_EMPTY1,
-    X_FULL0, X_FULL1, X_EMPTY0, X_EMPTY1,
-    COEF_FULL0, COEF_FULL1, COEF_EMPTY0, COEF_EMPTY1, RS0, RS1,
+    X_FULL0, X_FULL1, X_FULL2,
+    COEF_FULL0, COEF_FULL1, COEF_FULL2, COEF_FULL3, COEF_EMPTY0, COEF_EMPTY1, COEF_EMPTY2,
+    COEF_EMPTY3, CUM_READY0, CUM_READY1, CUM_READY2, CUM_READY3, PSI_READY0, PSI_READY1,
     OPS_FULL0, OPS_FULL1, OPS_EMPTY0, OPS_EMPTY1, S_FULL, S_EMPTY, SL_FULL, DS_FULL, DS_EMPTY,
     G_FULL, G_EMPTY, Y_FULL0, Y_FULL1, Y_EMPTY0, Y_EMPTY1, Y_STAGED, DRAIN, NEVER, NUM_BARS
 };
 
-// arrival count of each barrier: 1 for TMA expect_tx / tcgen05.commit / single-thread
-// arrivals, 4 for one elected lane per warp of a four-warp group, 5 where the
-// coefficient warp joins the four rotation warps
+// arrival count of each barrier: 1 for TMA expect_tx / tcgen05.commit / single-thread or
+// single-warp arrivals, 2 for the coefficient slots (x warp + state warpgroup), 4 for one
+// elected lane per warp of a four-warp group, 8 for the rotation warps, 9 where the
+// coefficient warp joins them
 __device__ __forceinline__ uint32_t bar_count(int i) {
     switch (i) {
-        case DT_EMPTY0: case DT_EMPTY1: case COEF_FULL0: case COEF_FULL1:
+        case DT_EMPTY0: case DT_EMPTY1: case RAW_EMPTY0: case RAW_EMPTY1:
+            return kRotWarps + 1;
         case OPS_FULL0: case OPS_FULL1:
-            return 5;
-        case RAW_EMPTY0: case RAW_EMPTY1: case RS0: case RS1:
+            return kRotWarps;
+        case COEF_EMPTY0: case COEF_EMPTY1: case COEF_EMPTY2: case COEF_EMPTY3:
+            return 2;
         case S_EMPTY: case SL_FULL: case DS_EMPTY: case G_FULL:
         case Y_EMPTY0: case Y_EMPTY1: case Y_STAGED:
             return 4;
@@ -93,8 +100,8 @@ template <int NST, int Q, int R>
 struct Cfg {
     static constexpr int L = Q * R;                 // rows of the intra-chunk tiles
     static constexpr int PAIRS = NST / 2;
-    static constexpr int PPT = PAIRS / 32;          // state pairs per rotation thread (1 or 2)
-    static constexpr int TSPLIT = 4;                // rotation warps along the tokens
+    static constexpr int PB = PAIRS / 32;           // rotation warps along the pairs (1 or 2)
+    static constexpr int TSPLIT = kRotWarps / PB;   // rotation warps along the tokens (8 or 4)
     static_assert(L == 64 || L == 128, "rows per chunk must be 64 or 128");
     static_assert(NST == 64 || NST == 128, "dstate must be 64 or 128");
 
@@ -109,22 +116,26 @@ struct Cfg {
     static constexpr int G_BYTES = NST * 128;
     static constexpr int COEF_FLOATS = 4 * Q + PAIRS + 4;
     static constexpr int base_bytes() {
-        return 2 * X_BYTES + SL_BYTES + G_BYTES + 2 * 3 * DT_BYTES + 2 * COEF_FLOATS * 4 +
-               2 * 4 * PAIRS * 4 + NUM_BARS * 8 + 64;
+        return SL_BYTES + G_BYTES + 2 * 3 * DT_BYTES + kCoefSlots * COEF_FLOATS * 4 +
+               2 * TSPLIT * PAIRS * 4 + NUM_BARS * 8 + 64;
     }
     static constexpr int raw_bytes(int rt) { return rt * R * NST * 2 * 2 + rt * PAIRS * 4; }
     static constexpr int kSmemLimit = 232448 - 1024;            // minus base alignment slack
-    // (operand slots, raw sub-chunk tokens): prefer two slots, then the largest sub-chunk
+    // (operand slots, x stages, raw sub-chunk tokens): prefer two operand slots, then three
+    // x stages, then the largest raw sub-chunk that fits
     static constexpr int pick() {
         for (int ops = 2; ops >= 1; --ops)
-            for (int rt = (Q < 32 ? Q : 32); rt >= TSPLIT; rt /= 2)
-                if (Q % rt == 0 && rt % TSPLIT == 0 &&
-                    base_bytes() + ops * SLOT_BYTES + 2 * raw_bytes(rt) <= kSmemLimit)
-                    return ops * 1000 + rt;
+            for (int xst = 3; xst >= 2; --xst)
+                for (int rt = (Q < 32 ? Q : 32); rt >= TSPLIT; rt /= 2)
+                    if (Q % rt == 0 && rt % TSPLIT == 0 &&
+                        base_bytes() + ops * SLOT_BYTES + xst * X_BYTES + 2 * raw_bytes(rt) <=
+                            kSmemLimit)
+                        return ops * 10000 + xst * 1000 + rt;
         return 0;
     }
     static_assert(pick() != 0, "shared memory budget exceeded");
-    static constexpr int OPS = pick() / 1000;                   // operand slots
+    static constexpr int OPS = pick() / 10000;                  // operand slots
+    static constexpr int XST = (pick() / 1000) % 10;            // x / y staging stages
     static constexpr int RT = pick() % 1000;                    // tokens per raw sub-chunk
     static constexpr int NSUB = Q / RT;
     static constexpr int TPT = RT / TSPLIT;                     // tokens per rotation thread
@@ -133,15 +144,16 @@ struct Cfg {
     static constexpr int RAW_BYTES = 2 * BRAW_BYTES + TH_BYTES;
 
     // shared memory offsets (SW128 tiles first, 1024-byte aligned)
-    static constexpr int OFF_X = 0;                                   // [2] x / y staging
-    static constexpr int OFF_OPS = OFF_X + 2 * X_BYTES;               // [OPS] C~, B~, Xw
+    static constexpr int OFF_X = 0;                                   // [XST] x / y staging
+    static constexpr int OFF_OPS = OFF_X + XST * X_BYTES;             // [OPS] C~, B~, Xw
     static constexpr int OFF_SL = OFF_OPS + OPS * SLOT_BYTES;         // S o L
     static constexpr int OFF_G = OFF_SL + SL_BYTES;                   // g (bf16)
     static constexpr int OFF_RAW = OFF_G + G_BYTES;                   // [2] B, C, theta
     static constexpr int OFF_DT = OFF_RAW + 2 * RAW_BYTES;            // [2] dt, A, lam
-    static constexpr int OFF_COEF = OFF_DT + 2 * 3 * DT_BYTES;        // [2] coefficients
-    static constexpr int OFF_RSUM = OFF_COEF + 2 * COEF_FLOATS * 4;   // [2][4][PAIRS] angle sums
-    static constexpr int OFF_BAR = (OFF_RSUM + 2 * 4 * PAIRS * 4 + 7) / 8 * 8;
+    static constexpr int OFF_COEF = OFF_DT + 2 * 3 * DT_BYTES;        // [kCoefSlots] coefficients
+    static constexpr int OFF_RSUM = OFF_COEF + kCoefSlots * COEF_FLOATS * 4;  // [2][TSPLIT][PAIRS]
+                                                                      // range start angles
+    static constexpr int OFF_BAR = (OFF_RSUM + 2 * TSPLIT * PAIRS * 4 + 7) / 8 * 8;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;           // tmem base, abort flag
     // + alignment slack; at least 120 KB so that only one CTA fits on an SM (each CTA
     // allocates all 512 TMEM columns)
@@ -228,7 +240,7 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
     if ((p.a.flags & M3_FLAG_TEST_STALL) && !mbar_wait(&bar[NEVER], 0, ab)) return;
     for (int c = 0; c < p.nchunks; ++c) {
         const uint32_t ph = c & 1;
-        const int st = c & 1, yb = c & 1;
+        const int yb = c & 1;
         const int slot = c % C::OPS;
         const uint32_t s_ct = smem_u32(C::ct(sm, slot)), s_bt = smem_u32(C::bt(sm, slot));
         const uint32_t s_xw = smem_u32(C::xw(sm, slot));
@@ -268,9 +280,10 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
         // Y_intra = (S o L) X  (M = L, N = P, K = L)
         if (!mbar_wait(&bar[SL_FULL], ph, ab)) return;
         M3_TRACE_EV(c, 12);
-        if (!mbar_wait(&bar[X_FULL0 + st], (c >> 1) & 1, ab)) return;
+        const int xs = c % C::XST;
+        if (!mbar_wait(&bar[X_FULL0 + xs], (c / C::XST) & 1, ab)) return;
         tc_fence_after();
-        const uint32_t s_x = smem_u32(sm + C::OFF_X + st * C::X_BYTES);
+        const uint32_t s_x = smem_u32(sm + C::OFF_X + xs * C::X_BYTES);
 #pragma unroll
         for (int k = 0; k < C::L / 16; ++k)
             mma_bf16(tmem + C::tm_ya(yb), desc_k(s_sl, k, C::L), desc_mn(s_x, k, 1024u), C::ID_Y,
@@ -281,29 +294,24 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
 }
 
 // ---------------------------------------------------------------------------------
-// Rotation warpgroup: B~ and C~ operands.  Warp ts handles tokens [ts*TPT, (ts+1)*TPT)
-// of every raw sub-chunk; lane l handles state pairs PPT*l .. PPT*l+PPT-1 (all pairs of a
-// token across the warp).  The chunk-start angle of a thread's token range is the
-// running angle plus the angle sums of the earlier ranges, exchanged through shared
-// memory once per sub-chunk.
+// Rotation warps: B~ and C~ operands.  Rotation warp rw handles state pairs
+// 32*(rw % PB) + lane and tokens [ts*TPT, (ts+1)*TPT) of every raw sub-chunk, with
+// ts = rw / PB.  The call-relative angle at the start of its token range comes from the
+// coefficient warp (per raw stage), so the rotation warps never wait on each other.
 template <int NST, int Q, int R>
 __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
     using C = Cfg<NST, Q, R>;
-    constexpr int PPT = C::PPT, TPT = C::TPT, PAIRS = C::PAIRS;
+    constexpr int TPT = C::TPT, PAIRS = C::PAIRS, TSPLIT = C::TSPLIT;
     const ScanArgs& a = p.a;
-    const int tid = threadIdx.x - 192;          // 0..127
-    const int ts = tid >> 5, lane = tid & 31;
-    const int pair0 = lane * PPT;                // first state pair of this thread
+    const int tid = threadIdx.x - 192;          // 0..255
+    const int rw = tid >> 5, lane = tid & 31;
+    const int ts = rw / C::PB;
+    const int pair = (rw % C::PB) * 32 + lane;   // this thread's state pair
     const int hq = (blockIdx.x % a.H) & 3;       // column of this head in the 4-head dt tile
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
-    const int atom = (2 * pair0) >> 6, col = (2 * pair0) & 63;
-    float* rsum = reinterpret_cast<float*>(sm + C::OFF_RSUM);
+    const int atom = (2 * pair) >> 6, col = (2 * pair) & 63;
+    const float* psib = reinterpret_cast<const float*>(sm + C::OFF_RSUM);
     int raw_it = 0;
-    // call-relative angles of this thread's pairs (the RoPE frame of Proposition 4 starts
-    // at the first token of the call), reduced mod 2 pi at chunk boundaries
-    float psi_acc[PPT];
-#pragma unroll
-    for (int k = 0; k < PPT; ++k) psi_acc[k] = 0.f;
     for (int c = 0; c < p.nchunks; ++c) {
         const int st = c & 1, slot = c % C::OPS;
         const uint32_t ph2 = (c >> 1) & 1;
@@ -324,107 +332,77 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
             const float* th = reinterpret_cast<const float*>(raw + 2 * C::BRAW_BYTES);
             const int tb = s * C::RT;           // first token of the sub-chunk (chunk-relative)
             const int j0 = ts * TPT;
-            // angle increments of the own tokens and their sum per pair
-            float ph[TPT][PPT], own[PPT];
-#pragma unroll
-            for (int k = 0; k < PPT; ++k) own[k] = 0.f;
+            float ph[TPT];
+            uint32_t bv[TPT][R], cv[TPT][R];
 #pragma unroll
             for (int jj = 0; jj < TPT; ++jj) {
                 const int j = j0 + jj;
                 const float d = angle ? 1.f : dtt[(tb + j) * 4 + hq];
-                if constexpr (PPT == 2) {
-                    const float2 tv = *reinterpret_cast<const float2*>(th + j * PAIRS + pair0);
-                    ph[jj][0] = d * tv.x;
-                    ph[jj][1] = d * tv.y;
-                } else {
-                    ph[jj][0] = d * th[j * PAIRS + pair0];
-                }
-#pragma unroll
-                for (int k = 0; k < PPT; ++k) own[k] += ph[jj][k];
-            }
-            // exchange the range sums of the four token ranges
-            float* rb = rsum + (rs * 4) * PAIRS;
-#pragma unroll
-            for (int k = 0; k < PPT; ++k) rb[ts * PAIRS + pair0 + k] = own[k];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[RS0 + rs]);
-            // raw B, C of the own tokens (independent of the exchange)
-            uint32_t bv[TPT][R][PPT], cv[TPT][R][PPT];
-#pragma unroll
-            for (int jj = 0; jj < TPT; ++jj)
+                ph[jj] = d * th[j * PAIRS + pair];
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const int e = (((j0 + jj) * R + r) * NST) / 2 + pair0;
-                    if constexpr (PPT == 2) {
-                        const uint2 b2 = *reinterpret_cast<const uint2*>(braw + e);
-                        const uint2 c2 = *reinterpret_cast<const uint2*>(craw + e);
-                        bv[jj][r][0] = b2.x; bv[jj][r][1] = b2.y;
-                        cv[jj][r][0] = c2.x; cv[jj][r][1] = c2.y;
-                    } else {
-                        bv[jj][r][0] = braw[e];
-                        cv[jj][r][0] = craw[e];
-                    }
+                    const int e = ((j * R + r) * NST) / 2 + pair;
+                    bv[jj][r] = braw[e];
+                    cv[jj][r] = craw[e];
                 }
-            if (!warp_wait(&bar[RS0 + rs], (raw_it >> 1) & 1, ab)) return;
-            float psi[PPT], tot[PPT];
-#pragma unroll
-            for (int k = 0; k < PPT; ++k) {
-                float pre = 0.f, all = 0.f;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float v = rb[q * PAIRS + pair0 + k];
-                    all += v;
-                    pre += (q < ts) ? v : 0.f;
-                }
-                psi[k] = psi_acc[k] + pre;
-                tot[k] = all;
             }
+            if (!warp_wait(&bar[PSI_READY0 + rs], (raw_it >> 1) & 1, ab)) return;
+            if (tid == 0) M3_TRACE_EV(c, s == 0 ? 28 : 31);
+            float psi = psib[(rs * TSPLIT + ts) * PAIRS + pair];
 #pragma unroll
             for (int jj = 0; jj < TPT; ++jj) {
-                float sn[PPT], cn[PPT];
-#pragma unroll
-                for (int k = 0; k < PPT; ++k) {
-                    psi[k] += ph[jj][k];
-                    __sincosf(psi[k], &sn[k], &cn[k]);   // |psi| < pi + one chunk of increments
-                }
+                psi += ph[jj];
+                float sn, cn;
+                __sincosf(psi, &sn, &cn);   // |psi| < pi + one chunk of angle increments
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    uint32_t bo[PPT], co[PPT];
-#pragma unroll
-                    for (int k = 0; k < PPT; ++k) {
-                        const float b0 = bf16lo(bv[jj][r][k]), b1 = bf16hi(bv[jj][r][k]);
-                        const float c0 = bf16lo(cv[jj][r][k]), c1 = bf16hi(cv[jj][r][k]);
-                        // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1]
-                        bo[k] = pack_bf16x2(fmaf(cn[k], b0, sn[k] * b1), fmaf(cn[k], b1, -sn[k] * b0));
-                        co[k] = pack_bf16x2(fmaf(cn[k], c0, sn[k] * c1), fmaf(cn[k], c1, -sn[k] * c0));
-                    }
+                    const float b0 = bf16lo(bv[jj][r]), b1 = bf16hi(bv[jj][r]);
+                    const float c0 = bf16lo(cv[jj][r]), c1 = bf16hi(cv[jj][r]);
+                    // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1]
+                    const uint32_t bo = pack_bf16x2(fmaf(cn, b0, sn * b1), fmaf(cn, b1, -sn * b0));
+                    const uint32_t co = pack_bf16x2(fmaf(cn, c0, sn * c1), fmaf(cn, c1, -sn * c0));
                     const int row = (tb + j0 + jj) * R + r;
                     const uint32_t off = (uint32_t)atom * C::L * 128u + sw128_off(row, col);
-                    if constexpr (PPT == 2) {
-                        *reinterpret_cast<uint2*>(bt + off) = make_uint2(bo[0], bo[1]);
-                        *reinterpret_cast<uint2*>(ct + off) = make_uint2(co[0], co[1]);
-                    } else {
-                        *reinterpret_cast<uint32_t*>(bt + off) = bo[0];
-                        *reinterpret_cast<uint32_t*>(ct + off) = co[0];
-                    }
+                    *reinterpret_cast<uint32_t*>(bt + off) = bo;
+                    *reinterpret_cast<uint32_t*>(ct + off) = co;
                 }
             }
-#pragma unroll
-            for (int k = 0; k < PPT; ++k) psi_acc[k] += tot[k];
+            if (tid == 0 && s == 0) M3_TRACE_EV(c, 29);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[RAW_EMPTY0 + rs]);
         }
-        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + st * C::COEF_FLOATS};
-#pragma unroll
-        for (int k = 0; k < PPT; ++k) {
-            psi_acc[k] -= 6.283185307179586f * rintf(psi_acc[k] * 0.15915494309189535f);
-            if (ts == 0) cf.psi_end()[pair0 + k] = psi_acc[k];
-        }
+        const int cs = c % kCoefSlots;
+        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
         if (tid == 0) M3_TRACE_EV(c, 3);
+
+        // ---- w-scaled X:  Xw[u, r] = 2^(cum2_end - cum2_u) w_u x[u, r]  (needs the
+        //      coefficient warp's decay prefix sums of this chunk)
+        if (!warp_wait(&bar[CUM_READY0 + cs], (c / kCoefSlots) & 1, ab)) return;
+        const int xs = c % C::XST;
+        if (!warp_wait(&bar[X_FULL0 + xs], (c / C::XST) & 1, ab)) return;
+        if (tid == 0) M3_TRACE_EV(c, 4);
+        {
+            const uint8_t* xt = sm + C::OFF_X + xs * C::X_BYTES;
+            uint8_t* xw = C::xw(sm, slot);
+            const float cend = *cf.cum2_end();
+#pragma unroll 2
+            for (int idx = tid; idx < C::L * 8; idx += 32 * kRotWarps) {
+                const int row = idx >> 3, ch = idx & 7;
+                const int u = row / R;
+                const float sc = ex2_approx(cend - cf.cum2()[u]) * cf.w()[u];
+                const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((ch ^ row) & 7) << 4);
+                uint4 v = *reinterpret_cast<const uint4*>(xt + off);
+                uint4 o;
+                o.x = pack_bf16x2(bf16lo(v.x) * sc, bf16hi(v.x) * sc);
+                o.y = pack_bf16x2(bf16lo(v.y) * sc, bf16hi(v.y) * sc);
+                o.z = pack_bf16x2(bf16lo(v.z) * sc, bf16hi(v.z) * sc);
+                o.w = pack_bf16x2(bf16lo(v.w) * sc, bf16hi(v.w) * sc);
+                *reinterpret_cast<uint4*>(xw + off) = o;
+            }
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            mbar_arrive(&bar[COEF_FULL0 + st]);
             mbar_arrive(&bar[OPS_FULL0 + slot]);
             mbar_arrive(&bar[DT_EMPTY0 + st]);
         }
@@ -432,24 +410,32 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
     }
 }
 
-// Coefficient warp: per-token log2-decay prefix sum (warp scan), gamma, w and the mask
-// exponent offsets of each chunk, and the w-scaled X operand
-//   Xw[u, r] = 2^(cum2_end - cum2_u) w_u x[u, r].
+// Coefficient warp: per chunk, the log2-decay prefix sum (warp scan), gamma, w and the
+// mask exponent offsets ew_u = log2(w_u) - cum2_u into a ring of slots; per raw sub-chunk,
+// the call-relative angle of every state pair at the start of each rotation warp's
+// token range (a running sum over the tokens, the RoPE frame of Proposition 4), and the
+// angle at the chunk end (reduced mod 2 pi).
 template <int NST, int Q, int R>
 __device__ void coefficients(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
     using C = Cfg<NST, Q, R>;
+    constexpr int PAIRS = C::PAIRS, PPL = PAIRS / 32, TSPLIT = C::TSPLIT, TPT = C::TPT;
     const ScanArgs& a = p.a;
     const int lane = threadIdx.x & 31;
     const int hq = (blockIdx.x % a.H) & 3;
+    const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
+    float* psib = reinterpret_cast<float*>(sm + C::OFF_RSUM);
+    float psi[PPL];                              // pairs PPL*lane .. PPL*lane + PPL - 1
+#pragma unroll
+    for (int k = 0; k < PPL; ++k) psi[k] = 0.f;
+    int raw_it = 0;
     for (int c = 0; c < p.nchunks; ++c) {
-        const int st = c & 1, slot = c % C::OPS;
-        const uint32_t ph2 = (c >> 1) & 1;
-        if (!warp_wait(&bar[DT_FULL0 + st], ph2, ab)) return;
+        const int st = c & 1, cs = c % kCoefSlots;
+        if (!warp_wait(&bar[DT_FULL0 + st], (c >> 1) & 1, ab)) return;
         const float* dtt = reinterpret_cast<const float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
         const float* At = dtt + C::DT_BYTES / 4;
         const float* lt = dtt + 2 * C::DT_BYTES / 4;
-        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + st * C::COEF_FLOATS};
-        if (!warp_wait(&bar[COEF_EMPTY0 + st], ph2 ^ 1, ab)) return;
+        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
+        if (!warp_wait(&bar[COEF_EMPTY0 + cs], ((c / kCoefSlots) & 1) ^ 1, ab)) return;
         float carry = 0.f;
         for (int t0 = 0; t0 < Q; t0 += 32) {
             const int t = t0 + lane;
@@ -477,170 +463,134 @@ __device__ void coefficients(const TcParams& p, uint8_t* sm, uint64_t* bar, cons
         }
         if (lane == 0) *cf.cum2_end() = carry;
         __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[CUM_READY0 + cs]);
 
-        if (!warp_wait(&bar[X_FULL0 + st], ph2, ab)) return;
-        if (!warp_wait(&bar[OPS_EMPTY0 + slot], ((c / C::OPS) & 1) ^ 1, ab)) return;
-        if (lane == 0) M3_TRACE_EV(c, 4);
-        const uint8_t* xt = sm + C::OFF_X + st * C::X_BYTES;
-        uint8_t* xw = C::xw(sm, slot);
-#pragma unroll 4
-        for (int idx = lane; idx < C::L * 8; idx += 32) {
-            const int row = idx >> 3, ch = idx & 7;
-            const int u = row / R;
-            const float sc = ex2_approx(carry - cf.cum2()[u]) * cf.w()[u];
-            const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((ch ^ row) & 7) << 4);
-            uint4 v = *reinterpret_cast<const uint4*>(xt + off);
-            uint4 o;
-            o.x = pack_bf16x2(bf16lo(v.x) * sc, bf16hi(v.x) * sc);
-            o.y = pack_bf16x2(bf16lo(v.y) * sc, bf16hi(v.y) * sc);
-            o.z = pack_bf16x2(bf16lo(v.z) * sc, bf16hi(v.z) * sc);
-            o.w = pack_bf16x2(bf16lo(v.w) * sc, bf16hi(v.w) * sc);
-            *reinterpret_cast<uint4*>(xw + off) = o;
+        // ---- range start angles of every raw sub-chunk of this chunk
+        for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
+            const int rs = raw_it & 1;
+            if (!warp_wait(&bar[RAW_FULL0 + rs], (raw_it >> 1) & 1, ab)) return;
+            const float* th = reinterpret_cast<const float*>(sm + C::OFF_RAW + rs * C::RAW_BYTES +
+                                                             2 * C::BRAW_BYTES);
+            float* pb = psib + rs * TSPLIT * PAIRS;
+            const int tb = s * C::RT;
+#pragma unroll
+            for (int q = 0; q < TSPLIT; ++q) {
+#pragma unroll
+                for (int k = 0; k < PPL; ++k) pb[q * PAIRS + PPL * lane + k] = psi[k];
+#pragma unroll
+                for (int jj = 0; jj < TPT; ++jj) {
+                    const int j = q * TPT + jj;
+                    const float d = angle ? 1.f : dtt[(tb + j) * 4 + hq];
+                    if constexpr (PPL == 2) {
+                        const float2 tv = *reinterpret_cast<const float2*>(th + j * PAIRS + 2 * lane);
+                        psi[0] = fmaf(d, tv.x, psi[0]);
+                        psi[1] = fmaf(d, tv.y, psi[1]);
+                    } else {
+                        psi[0] = fmaf(d, th[j * PAIRS + lane], psi[0]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bar[PSI_READY0 + rs]);
+                mbar_arrive(&bar[RAW_EMPTY0 + rs]);
+            }
         }
-        fence_proxy_async_smem();
+#pragma unroll
+        for (int k = 0; k < PPL; ++k) {
+            psi[k] -= 6.283185307179586f * rintf(psi[k] * 0.15915494309189535f);
+            cf.psi_end()[PPL * lane + k] = psi[k];
+        }
         __syncwarp();
         if (lane == 0) {
-            mbar_arrive(&bar[COEF_FULL0 + st]);
-            mbar_arrive(&bar[OPS_FULL0 + slot]);
+            mbar_arrive(&bar[COEF_FULL0 + cs]);
             mbar_arrive(&bar[DT_EMPTY0 + st]);
         }
     }
 }
 
 // ---------------------------------------------------------------------------------
-// Epilogue warpgroup: masks S, keeps the fp32 state, writes y.
+// TMEM lane layouts of the epilogue and state warpgroups (warp w reaches lane quadrant
+// w % 4).  Rows of an M = 128 accumulator: row 32q + lane, all columns.  Rows of an
+// M = 64 accumulator: row 16q + lane % 16, column half lane / 16.  TMEM is read and
+// written 16 of a thread's columns at a time.
+template <int NST, int Q, int R>
+struct Lanes {
+    uint32_t tq;    // TMEM address of this warp's lane quadrant
+    int lane, q;
+    __device__ Lanes(uint32_t tmem) {
+        lane = threadIdx.x & 31;
+        q = (threadIdx.x >> 5) & 3;
+        tq = tmem + ((uint32_t)(32 * q) << 16);
+    }
+    __device__ int row(bool half) const { return half ? 16 * q + (lane & 15) : 32 * q + lane; }
+    __device__ int col0(bool half) const { return half ? 32 * (lane >> 4) : 0; }
+    __device__ void ld16(bool half, uint32_t col, int cb, uint32_t (&v)[16]) const {
+        if (half)
+            tmem_ld_16x32bx2_x16<32>(tq + col + cb, v);
+        else
+            tmem_ld_32x32b_x16(tq + col + cb, v);
+    }
+    __device__ void st16(bool half, uint32_t col, int cb, const uint32_t (&v)[16]) const {
+        if (half)
+            tmem_st_16x32bx2_x16<32>(tq + col + cb, v);
+        else
+            tmem_st_32x32b_x16(tq + col + cb, v);
+    }
+};
+
+// Epilogue warpgroup (warps 2-5): masks S into the bf16 operand S o L and writes y.
 template <int NST, int Q, int R>
 __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
                          const Abort& ab) {
     using C = Cfg<NST, Q, R>;
     const ScanArgs& a = p.a;
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = w & 3;                                   // TMEM lane quadrant of this warp
+    const Lanes<NST, Q, R> ln(tmem);
+    const int lane = ln.lane;
     const int etid = threadIdx.x - 64;                     // 0..127
-    const int b = blockIdx.x / a.H, h = blockIdx.x % a.H, g = h / (a.H / a.G);
-    const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-    const float Dh = a.D ? a.D[h] : 0.f;
-    const long long T = a.T;
-    const size_t bh = (size_t)b * a.H + h;
-
-    // Rows owned in the L-row accumulators (S, Y): L == 128 -> row 32q + lane, all
-    // columns; L == 64 -> row 16q + lane%16, column half lane/16 (M = 64 layout).
+    const float Dh = a.D ? a.D[blockIdx.x % a.H] : 0.f;
     constexpr bool kHalfL = (C::L == 64);
-    const int lrow = kHalfL ? 16 * q + (lane & 15) : 32 * q + lane;
-    const int lcol0 = kHalfL ? 32 * (lane >> 4) : 0;
+    const int lrow = ln.row(kHalfL), lcol0 = ln.col0(kHalfL);
     constexpr int kLCols = kHalfL ? 32 : C::L;
     constexpr int kYCols = kHalfL ? 32 : kP;
-    // Rows owned in the NST-row state accumulator, same rule.
-    constexpr bool kHalfN = (NST == 64);
-    const int nrow = kHalfN ? 16 * q + (lane & 15) : 32 * q + lane;
-    const int ncol0 = kHalfN ? 32 * (lane >> 4) : 0;
-    constexpr int kNCols = kHalfN ? 32 : kP;
-
-    uint8_t* gs = sm + C::OFF_G;
     uint8_t* sl = sm + C::OFF_SL;
 
-    // The fp32 carried state g lives in TMEM columns TM_G.. with the lane layout of the
-    // dS accumulator (this thread: row nrow, columns ncol0..); 32 columns at a time.
-    auto tm_ld = [&](uint32_t col, int cb, uint32_t (&v)[32]) {
-        if (kHalfN)
-            tmem_ld_16x32bx2_x32<32>(tq + col, v);
-        else
-            tmem_ld_32x32b_x32(tq + col + cb, v);
-    };
-    auto tm_st = [&](uint32_t col, int cb, const uint32_t (&v)[32]) {
-        if (kHalfN)
-            tmem_st_16x32bx2_x32<32>(tq + col, v);
-        else
-            tmem_st_32x32b_x32(tq + col + cb, v);
-    };
-    // bf16 copy of 32 state columns for the Y_inter MMA operand (MN-major [n][p])
-    auto publish_block = [&](int cb, const uint32_t (&v)[32]) {
-#pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-            o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-            o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
-            o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
-            *reinterpret_cast<uint4*>(gs + sw128_off(nrow, ncol0 + cb + j)) = o;
-        }
-    };
-
-    // ---- g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T
-    {
-        const float* h0 = a.h + (bh * NST + nrow) * kP + ncol0;
-        const float d0 = a.dt[(size_t)b * T * a.H + h], l0 = a.lam[(size_t)b * T * a.H + h];
-        const float beta0 = (1.f - l0) * d0;
-        const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(a.x_prev) + bh * R * kP;
-        const __nv_bfloat16* bp =
-            static_cast<const __nv_bfloat16*>(a.B_prev) + ((size_t)b * a.G + g) * R * NST;
-#pragma unroll 1
-        for (int cb = 0; cb < kNCols; cb += 32) {
-            float gv[32];
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(h0 + cb + j);
-                gv[j] = v.x; gv[j + 1] = v.y; gv[j + 2] = v.z; gv[j + 3] = v.w;
-            }
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const float bb = beta0 * __bfloat162float(bp[r * NST + nrow]);
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    gv[j] = fmaf(bb, __bfloat162float(xp[r * kP + ncol0 + cb + j]), gv[j]);
-            }
-            uint32_t v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(gv[j]);
-            tm_st(C::TM_G, cb, v);
-            publish_block(cb, v);
-        }
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[G_FULL]);
-    }
-
-    bool ok = true;
-    for (int c = 0; c < p.nchunks && ok; ++c) {
+    for (int c = 0; c < p.nchunks; ++c) {
         const uint32_t ph = c & 1, ph2 = (c >> 1) & 1;
-        const int st = c & 1;
-        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + st * C::COEF_FLOATS};
-        if (!(ok = warp_wait(&bar[COEF_FULL0 + st], ph2, ab))) break;
+        const int cs = c % kCoefSlots;
+        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
+        if (!warp_wait(&bar[COEF_FULL0 + cs], (c / kCoefSlots) & 1, ab)) return;
         if (etid == 0) M3_TRACE_EV(c, 14);
         const float* cum2 = cf.cum2();
 
-        // ---- S o L  ->  bf16, K-major [row][col] with L[t,u] = e^{cum_t-cum_u} (u<t ? w_u : gamma_u)
-        if (!(ok = warp_wait(&bar[S_FULL], ph, ab))) break;
+        // ---- S o L -> bf16, K-major [row][col].  L[t,u] = 2^(cum2_t + ew_u) for u < t
+        //      (ew_u = log2 w_u - cum2_u), gamma_t on the diagonal token; the skip D x is
+        //      folded in as D on the (row == col) diagonal.
+        if (!warp_wait(&bar[S_FULL], ph, ab)) return;
         if (etid == 0) M3_TRACE_EV(c, 15);
         tc_fence_after();
         {
-            // L[t,u] = 2^(cum2_t - cum2_u) w_u = 2^(cum2_t + ew_u) for u < t, gamma_t on the
-            // diagonal token; the skip D x is folded in as D on the (row == col) diagonal.
             const int t = lrow / R;
             const float ct = cum2[t];
             const float gt = cf.gam()[t];
             const float* ew = cf.ew();
 #pragma unroll 1
-            for (int cb = 0; cb < kLCols; cb += 32) {
-                uint32_t s[32];
-                if (kHalfL)
-                    tmem_ld_16x32bx2_x32<32>(tq + C::TM_S, s);
-                else
-                    tmem_ld_32x32b_x32(tq + C::TM_S + cb, s);
+            for (int cb = 0; cb < kLCols; cb += 16) {
+                uint32_t sv[16];
+                ln.ld16(kHalfL, C::TM_S, cb, sv);
                 tmem_wait_ld();
                 const int colb = lcol0 + cb;
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
+                for (int j = 0; j < 16; j += 8) {
                     float m[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int col = colb + j + e;
                         const int u = col / R;
-                        const float sv = __uint_as_float(s[j + e]);
-                        const float v = sv * ex2_approx(ct + ew[u]);
+                        const float sv_f = __uint_as_float(sv[j + e]);
+                        const float v = sv_f * ex2_approx(ct + ew[u]);
                         m[e] = (u < t) ? v : 0.f;
-                        if (u == t) m[e] = sv * gt + (col == lrow ? Dh : 0.f);
+                        if (u == t) m[e] = sv_f * gt + (col == lrow ? Dh : 0.f);
                     }
                     uint4 o;
                     o.x = pack_bf16x2(m[0], m[1]);
@@ -662,63 +612,25 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
         }
         if (etid == 0) M3_TRACE_EV(c, 16);
 
-        // ---- state (RoPE frame of the call): g <- e^{cum_end} g + dS, published for the next chunk
-        if (!(ok = warp_wait(&bar[DS_FULL], ph, ab))) break;
-        if (etid == 0) M3_TRACE_EV(c, 17);
-        const bool more = c + 1 < p.nchunks;
-        // the Y_inter MMA of this chunk must be done reading g_c before g_{c+1} replaces it
-        if (more && !(ok = warp_wait(&bar[G_EMPTY], ph, ab))) break;
-        if (etid == 0) M3_TRACE_EV(c, 19);
-        tc_fence_after();
-        {
-            const float dec = exp2f(*cf.cum2_end());
-#pragma unroll 1
-            for (int cb = 0; cb < kNCols; cb += 32) {
-                uint32_t d[32], gq[32];
-                tm_ld(C::TM_DS, cb, d);
-                tm_ld(C::TM_G, cb, gq);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    gq[j] = __float_as_uint(fmaf(dec, __uint_as_float(gq[j]), __uint_as_float(d[j])));
-                tm_st(C::TM_G, cb, gq);
-                if (more) publish_block(cb, gq);
-            }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&bar[DS_EMPTY]);
-            if (more) mbar_arrive(&bar[G_FULL]);
-        }
-        if (etid == 0) M3_TRACE_EV(c, 18);
-
         // ---- y = Y_intra + e^{cum_t} Y_inter   (D x is in Y_intra; y is written over the
-        //      x tile, then stored with TMA)
+        //      x tile, which the x warp then stores with TMA)
         const int yb = c & 1;
-        if (!(ok = warp_wait(&bar[Y_FULL0 + yb], ph2, ab))) break;
+        if (!warp_wait(&bar[Y_FULL0 + yb], ph2, ab)) return;
         if (etid == 0) M3_TRACE_EV(c, 20);
-        if (!(ok = warp_wait(&bar[X_FULL0 + st], ph2, ab))) break;
+        const int xs = c % C::XST;
+        if (!warp_wait(&bar[X_FULL0 + xs], (c / C::XST) & 1, ab)) return;
         tc_fence_after();
-        if (etid == 0) M3_TRACE_EV(c, 21);
-        uint8_t* xt = sm + C::OFF_X + st * C::X_BYTES;
+        uint8_t* xt = sm + C::OFF_X + xs * C::X_BYTES;
         {
             const float sc = exp2f(cum2[lrow / R]);
 #pragma unroll 1
-            for (int cb = 0; cb < kYCols; cb += 32) {
-                uint32_t ya[32], yi[32];
-                if (kHalfL) {
-                    tmem_ld_16x32bx2_x32<32>(tq + C::tm_ya(yb), ya);
-                    tmem_ld_16x32bx2_x32<32>(tq + C::tm_yi(yb), yi);
-                } else {
-                    tmem_ld_32x32b_x32(tq + C::tm_ya(yb) + cb, ya);
-                    tmem_ld_32x32b_x32(tq + C::tm_yi(yb) + cb, yi);
-                }
+            for (int cb = 0; cb < kYCols; cb += 16) {
+                uint32_t ya[16], yi[16];
+                ln.ld16(kHalfL, C::tm_ya(yb), cb, ya);
+                ln.ld16(kHalfL, C::tm_yi(yb), cb, yi);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
+                for (int j = 0; j < 16; j += 8) {
                     const uint32_t off = sw128_off(lrow, lcol0 + cb + j);
                     uint32_t o[4];
 #pragma unroll
@@ -739,58 +651,147 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
             mbar_arrive(&bar[Y_STAGED]);
         }
         if (etid == 0) M3_TRACE_EV(c, 22);
-        if (etid == 0) {
-            // all four warps have written their rows of y (and are done with this chunk's
-            // coefficients): store the tile, then hand the x stage back to the producer
-            ok = mbar_wait(&bar[Y_STAGED], ph, ab);
-            if (ok) {
-                mbar_arrive(&bar[COEF_EMPTY0 + st]);
-                tma_store_5d(&p.tm_y, xt, 0, 0, h, c * Q, b);
-                bulk_commit();
-                bulk_wait_read<0>();
-                M3_TRACE_EV(c, 23);
-                mbar_arrive(&bar[X_EMPTY0 + st]);
-            }
+    }
+}
+
+// State warpgroup (warps 16-19): the fp32 carried state g in TMEM columns TM_G..,
+// g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T, per chunk g <- e^{cum_end} g + dS and its
+// bf16 copy for the Y_inter MMA; at the end h_T = R(psi_T) g and the carried x.
+template <int NST, int Q, int R>
+__device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
+                      const Abort& ab) {
+    using C = Cfg<NST, Q, R>;
+    const ScanArgs& a = p.a;
+    const Lanes<NST, Q, R> ln(tmem);
+    const int lane = ln.lane;
+    const int stid = threadIdx.x - 512;                    // 0..127
+    const int b = blockIdx.x / a.H, h = blockIdx.x % a.H, g = h / (a.H / a.G);
+    const long long T = a.T;
+    const size_t bh = (size_t)b * a.H + h;
+    constexpr bool kHalfN = (NST == 64);
+    const int nrow = ln.row(kHalfN), ncol0 = ln.col0(kHalfN);
+    constexpr int kNCols = kHalfN ? 32 : kP;
+    uint8_t* gs = sm + C::OFF_G;
+
+    auto publish16 = [&](int cb, const uint32_t (&v)[16]) {
+#pragma unroll
+        for (int j = 0; j < 16; j += 8) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+            o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+            o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+            o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+            *reinterpret_cast<uint4*>(gs + sw128_off(nrow, ncol0 + cb + j)) = o;
         }
-        if (w == 2) ok = __shfl_sync(0xffffffffu, ok, 0);
+    };
+
+    // ---- g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T
+    {
+        const float* h0 = a.h + (bh * NST + nrow) * kP + ncol0;
+        const float d0 = a.dt[(size_t)b * T * a.H + h], l0 = a.lam[(size_t)b * T * a.H + h];
+        const float beta0 = (1.f - l0) * d0;
+        const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(a.x_prev) + bh * R * kP;
+        const __nv_bfloat16* bp =
+            static_cast<const __nv_bfloat16*>(a.B_prev) + ((size_t)b * a.G + g) * R * NST;
+#pragma unroll 1
+        for (int cb = 0; cb < kNCols; cb += 16) {
+            float gv[16];
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(h0 + cb + j);
+                gv[j] = v.x; gv[j + 1] = v.y; gv[j + 2] = v.z; gv[j + 3] = v.w;
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float bb = beta0 * __bfloat162float(bp[r * NST + nrow]);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    gv[j] = fmaf(bb, __bfloat162float(xp[r * kP + ncol0 + cb + j]), gv[j]);
+            }
+            uint32_t v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(gv[j]);
+            ln.st16(kHalfN, C::TM_G, cb, v);
+            publish16(cb, v);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[G_FULL]);
     }
 
-    if (ok) {
-        // final state: back from the RoPE frame of the call, h_T = R(psi_T) g
-        const float* pe = reinterpret_cast<const float*>(sm + C::OFF_COEF) +
-                          ((p.nchunks - 1) & 1) * C::COEF_FLOATS + 4 * Q;
-        float sn, cn;
-        sincosf(pe[nrow >> 1], &sn, &cn);
-        const bool odd = nrow & 1;
-        float* hT = a.h + (bh * NST + nrow) * kP + ncol0;
+    for (int c = 0; c < p.nchunks; ++c) {
+        const uint32_t ph = c & 1;
+        const int cs = c % kCoefSlots;
+        Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
+        if (!warp_wait(&bar[COEF_FULL0 + cs], (c / kCoefSlots) & 1, ab)) return;
+        if (!warp_wait(&bar[DS_FULL], ph, ab)) return;
+        if (stid == 0) M3_TRACE_EV(c, 17);
+        const bool more = c + 1 < p.nchunks;
+        // the Y_inter MMA of this chunk must be done reading g_c before g_{c+1} replaces it
+        if (more && !warp_wait(&bar[G_EMPTY], ph, ab)) return;
+        if (stid == 0) M3_TRACE_EV(c, 19);
         tc_fence_after();
+        const float dec = exp2f(*cf.cum2_end());
+        if (c + 1 == p.nchunks) {
+            // last chunk: the call's final state goes back to the original frame,
+            // h_T = R(psi_T) (e^{cum_end} g + dS)
+            float sn, cn;
+            sincosf(cf.psi_end()[nrow >> 1], &sn, &cn);
+            const bool odd = nrow & 1;
+            float* hT = a.h + (bh * NST + nrow) * kP + ncol0;
 #pragma unroll 1
-        for (int cb = 0; cb < kNCols; cb += 32) {
-            uint32_t gq[32];
-            tm_ld(C::TM_G, cb, gq);
-            tmem_wait_ld();
-            float gv[32];
+            for (int cb = 0; cb < kNCols; cb += 16) {
+                uint32_t d[16], gq[16];
+                ln.ld16(kHalfN, C::TM_DS, cb, d);
+                ln.ld16(kHalfN, C::TM_G, cb, gq);
+                tmem_wait_ld();
+                float gv[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float gj = __uint_as_float(gq[j]);
-                const float o = __shfl_xor_sync(0xffffffffu, gj, 1);
-                gv[j] = odd ? fmaf(sn, o, cn * gj) : fmaf(cn, gj, -sn * o);
+                for (int j = 0; j < 16; ++j) {
+                    const float gj = fmaf(dec, __uint_as_float(gq[j]), __uint_as_float(d[j]));
+                    const float o = __shfl_xor_sync(0xffffffffu, gj, 1);
+                    gv[j] = odd ? fmaf(sn, o, cn * gj) : fmaf(cn, gj, -sn * o);
+                }
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4*>(hT + cb + j) =
+                        make_float4(gv[j], gv[j + 1], gv[j + 2], gv[j + 3]);
             }
+        } else {
+#pragma unroll 1
+            for (int cb = 0; cb < kNCols; cb += 16) {
+                uint32_t d[16], gq[16];
+                ln.ld16(kHalfN, C::TM_DS, cb, d);
+                ln.ld16(kHalfN, C::TM_G, cb, gq);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(hT + cb + j) =
-                    make_float4(gv[j], gv[j + 1], gv[j + 2], gv[j + 3]);
+                for (int j = 0; j < 16; ++j)
+                    gq[j] = __float_as_uint(fmaf(dec, __uint_as_float(gq[j]), __uint_as_float(d[j])));
+                ln.st16(kHalfN, C::TM_G, cb, gq);
+                publish16(cb, gq);
+            }
+            tmem_wait_st();
         }
-        if (etid == 0) {
-            // every epilogue warp passed chunk 0 (it read x_prev there) before the last
-            // Y_STAGED completed, so x_prev can be overwritten now
-            const uint4* xl = reinterpret_cast<const uint4*>(
-                static_cast<const __nv_bfloat16*>(a.x) + (((size_t)b * T + (T - 1)) * a.H + h) * R * kP);
-            uint4* xpo = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.x_prev) + bh * R * kP);
-            for (int e = 0; e < R * kP / 8; ++e) xpo[e] = xl[e];
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&bar[DS_EMPTY]);
+            if (more) mbar_arrive(&bar[G_FULL]);
+        }
+        if (stid == 0) {
+            M3_TRACE_EV(c, 18);
+            mbar_arrive(&bar[COEF_EMPTY0 + cs]);
         }
     }
-    if (etid == 0) bulk_wait<0>();
+    if (stid == 0) {
+        // only this warpgroup read x_prev (for g_0), so the carried x can be replaced now
+        const uint4* xl = reinterpret_cast<const uint4*>(
+            static_cast<const __nv_bfloat16*>(a.x) + (((size_t)b * T + (T - 1)) * a.H + h) * R * kP);
+        uint4* xpo = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.x_prev) + bh * R * kP);
+        for (int e = 0; e < R * kP / 8; ++e) xpo[e] = xl[e];
+    }
 }
 
 // Wait for a barrier phase with a fixed time limit, regardless of the abort flag
@@ -807,7 +808,7 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
     const ScanArgs& a = p.a;
     const int b = blockIdx.x / a.H, h = blockIdx.x % a.H, g = h / (a.H / a.G);
     // loads issued per ring stage, so that an aborted CTA can wait for them to land
-    int n_dt[2] = {0, 0}, n_raw[2] = {0, 0}, n_x[2] = {0, 0};
+    int n_dt[2] = {0, 0}, n_raw[2] = {0, 0};
     int raw_it = 0;
     bool ok = true;
     for (int c = 0; c < p.nchunks && ok; ++c) {
@@ -834,14 +835,6 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
             tma_load_5d(raw + C::BRAW_BYTES, &p.tm_C, &bar[RAW_FULL0 + rs], 0, 0, g, tr, b);
             tma_load_4d(raw + 2 * C::BRAW_BYTES, &p.tm_th, &bar[RAW_FULL0 + rs], 0, g, tr, b);
             ++n_raw[rs];
-            if (s == 0) {
-                if (!(ok = mbar_wait(&bar[X_EMPTY0 + st], ph, ab))) break;
-                M3_TRACE_EV(c, 26);
-                mbar_arrive_expect_tx(&bar[X_FULL0 + st], C::X_BYTES);
-                tma_load_5d(sm + C::OFF_X + st * C::X_BYTES, &p.tm_x, &bar[X_FULL0 + st], 0, 0, h,
-                            t0, b);
-                ++n_x[st];
-            }
         }
     }
     if (!ok) {
@@ -849,9 +842,43 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         for (int s = 0; s < 2; ++s) {
             if (n_dt[s]) drain_wait(&bar[DT_FULL0 + s], (n_dt[s] - 1) & 1, 10000000ull);
             if (n_raw[s]) drain_wait(&bar[RAW_FULL0 + s], (n_raw[s] - 1) & 1, 10000000ull);
-            if (n_x[s]) drain_wait(&bar[X_FULL0 + s], (n_x[s] - 1) & 1, 10000000ull);
         }
     }
+}
+
+// x tiles and y stores, on their own warp so that neither a stage waiting for its y
+// store nor the store itself holds up the B / C / theta loads.  x(c) is loaded into
+// stage c % XST; once the epilogue has written y(c) over it (Y_STAGED), the tile is
+// stored, and when the store has read it the stage takes x(c + XST).
+template <int NST, int Q, int R>
+__device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
+    using C = Cfg<NST, Q, R>;
+    const ScanArgs& a = p.a;
+    const int b = blockIdx.x / a.H, h = blockIdx.x % a.H;
+    int n_x[C::XST] = {};
+    auto load = [&](int c) {
+        const int xs = c % C::XST;
+        mbar_arrive_expect_tx(&bar[X_FULL0 + xs], C::X_BYTES);
+        tma_load_5d(sm + C::OFF_X + xs * C::X_BYTES, &p.tm_x, &bar[X_FULL0 + xs], 0, 0, h, c * Q,
+                    b);
+        ++n_x[xs];
+    };
+    for (int c = 0; c < C::XST && c < p.nchunks; ++c) load(c);
+    bool ok = true;
+    for (int c = 0; c < p.nchunks; ++c) {
+        if (!(ok = mbar_wait(&bar[Y_STAGED], c & 1, ab))) break;
+        const int xs = c % C::XST;
+        tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, c * Q, b);
+        bulk_commit();
+        mbar_arrive(&bar[COEF_EMPTY0 + c % kCoefSlots]);
+        bulk_wait_read<0>();
+        M3_TRACE_EV(c, 23);
+        if (c + C::XST < p.nchunks) load(c + C::XST);
+    }
+    if (!ok)
+        for (int s = 0; s < C::XST; ++s)
+            if (n_x[s]) drain_wait(&bar[X_FULL0 + s], (n_x[s] - 1) & 1, 10000000ull);
+    bulk_wait<0>();
 }
 
 template <int NST, int Q, int R>
@@ -895,10 +922,14 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         }
     } else if (w < 6) {
         epilogue<NST, Q, R>(p, sm, bar, tmem, ab);
-    } else if (w < 10) {
+    } else if (w >= 16) {
+        state<NST, Q, R>(p, sm, bar, tmem, ab);
+    } else if (w < 6 + kRotWarps) {
         rotation<NST, Q, R>(p, sm, bar, ab);
-    } else {
+    } else if (w == 6 + kRotWarps) {
         coefficients<NST, Q, R>(p, sm, bar, ab);
+    } else if ((threadIdx.x & 31) == 0) {
+        x_producer<NST, Q, R>(p, sm, bar, ab);
     }
     tc_fence_before();
     __syncthreads();
