@@ -71,7 +71,7 @@ enum Bar {
     DT_FULL0, DT_FULL1, DT_EMPTY0, DT_EMPTY1,
     X_FULL0, X_FULL1, X_FULL2,
     COEF_FULL0, COEF_FULL1, COEF_FULL2, COEF_FULL3, COEF_EMPTY0, COEF_EMPTY1, COEF_EMPTY2,
-    COEF_EMPTY3, CUM_READY0, CUM_READY1, CUM_READY2, CUM_READY3, PSI_READY0, PSI_READY1,
+    COEF_EMPTY3, CUM_READY0, CUM_READY1, CUM_READY2, CUM_READY3, RS0, RS1,
     OPS_FULL0, OPS_FULL1, OPS_EMPTY0, OPS_EMPTY1, S_FULL, S_EMPTY, SL_FULL, DS_FULL, DS_EMPTY,
     G_FULL, G_EMPTY, Y_FULL0, Y_FULL1, Y_EMPTY0, Y_EMPTY1, Y_STAGED, DRAIN, NEVER, NUM_BARS
 };
@@ -82,9 +82,10 @@ enum Bar {
 // coefficient warp joins them
 __device__ __forceinline__ uint32_t bar_count(int i) {
     switch (i) {
-        case DT_EMPTY0: case DT_EMPTY1: case RAW_EMPTY0: case RAW_EMPTY1:
+        case DT_EMPTY0: case DT_EMPTY1: case COEF_FULL0: case COEF_FULL1: case COEF_FULL2:
+        case COEF_FULL3:
             return kRotWarps + 1;
-        case OPS_FULL0: case OPS_FULL1:
+        case RAW_EMPTY0: case RAW_EMPTY1: case RS0: case RS1: case OPS_FULL0: case OPS_FULL1:
             return kRotWarps;
         case COEF_EMPTY0: case COEF_EMPTY1: case COEF_EMPTY2: case COEF_EMPTY3:
             return 2;
@@ -152,7 +153,7 @@ struct Cfg {
     static constexpr int OFF_DT = OFF_RAW + 2 * RAW_BYTES;            // [2] dt, A, lam
     static constexpr int OFF_COEF = OFF_DT + 2 * 3 * DT_BYTES;        // [kCoefSlots] coefficients
     static constexpr int OFF_RSUM = OFF_COEF + kCoefSlots * COEF_FLOATS * 4;  // [2][TSPLIT][PAIRS]
-                                                                      // range start angles
+                                                                      // range angle sums
     static constexpr int OFF_BAR = (OFF_RSUM + 2 * TSPLIT * PAIRS * 4 + 7) / 8 * 8;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;           // tmem base, abort flag
     // + alignment slack; at least 120 KB so that only one CTA fits on an SM (each CTA
@@ -294,10 +295,11 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
 }
 
 // ---------------------------------------------------------------------------------
-// Rotation warps: B~ and C~ operands.  Rotation warp rw handles state pairs
+// Rotation warps: B~ and C~ operands.  Rotation warp rw handles state pair
 // 32*(rw % PB) + lane and tokens [ts*TPT, (ts+1)*TPT) of every raw sub-chunk, with
-// ts = rw / PB.  The call-relative angle at the start of its token range comes from the
-// coefficient warp (per raw stage), so the rotation warps never wait on each other.
+// ts = rw / PB.  The starting angle of a thread's token range is the running angle plus
+// the angle sums of the earlier ranges, exchanged through shared memory once per
+// sub-chunk (bounded mbarrier hand-off).
 template <int NST, int Q, int R>
 __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
     using C = Cfg<NST, Q, R>;
@@ -310,8 +312,11 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
     const int hq = (blockIdx.x % a.H) & 3;       // column of this head in the 4-head dt tile
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     const int atom = (2 * pair) >> 6, col = (2 * pair) & 63;
-    const float* psib = reinterpret_cast<const float*>(sm + C::OFF_RSUM);
+    float* rsum = reinterpret_cast<float*>(sm + C::OFF_RSUM);
     int raw_it = 0;
+    // call-relative angle of this thread's pair (the RoPE frame of Proposition 4 starts at
+    // the first token of the call), reduced mod 2 pi at chunk boundaries
+    float psi_acc = 0.f;
     for (int c = 0; c < p.nchunks; ++c) {
         const int st = c & 1, slot = c % C::OPS;
         const uint32_t ph2 = (c >> 1) & 1;
@@ -332,23 +337,40 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
             const float* th = reinterpret_cast<const float*>(raw + 2 * C::BRAW_BYTES);
             const int tb = s * C::RT;           // first token of the sub-chunk (chunk-relative)
             const int j0 = ts * TPT;
-            float ph[TPT];
-            uint32_t bv[TPT][R], cv[TPT][R];
+            // angle increments of the own tokens and their sum
+            float ph[TPT], own = 0.f;
 #pragma unroll
             for (int jj = 0; jj < TPT; ++jj) {
                 const int j = j0 + jj;
                 const float d = angle ? 1.f : dtt[(tb + j) * 4 + hq];
                 ph[jj] = d * th[j * PAIRS + pair];
+                own += ph[jj];
+            }
+            // publish the range sum; load the own tokens' raw B, C meanwhile
+            float* rb = rsum + (rs * TSPLIT) * PAIRS;
+            rb[ts * PAIRS + pair] = own;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[RS0 + rs]);
+            if (tid == 0) M3_TRACE_EV(c, s == 0 ? 27 : 30);
+            uint32_t bv[TPT][R], cv[TPT][R];
+#pragma unroll
+            for (int jj = 0; jj < TPT; ++jj)
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const int e = ((j * R + r) * NST) / 2 + pair;
+                    const int e = (((j0 + jj) * R + r) * NST) / 2 + pair;
                     bv[jj][r] = braw[e];
                     cv[jj][r] = craw[e];
                 }
-            }
-            if (!warp_wait(&bar[PSI_READY0 + rs], (raw_it >> 1) & 1, ab)) return;
+            if (!warp_wait(&bar[RS0 + rs], (raw_it >> 1) & 1, ab)) return;
             if (tid == 0) M3_TRACE_EV(c, s == 0 ? 28 : 31);
-            float psi = psib[(rs * TSPLIT + ts) * PAIRS + pair];
+            float pre = 0.f, tot = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < TSPLIT; ++qq) {
+                const float v = rb[qq * PAIRS + pair];
+                tot += v;
+                pre += (qq < ts) ? v : 0.f;
+            }
+            float psi = psi_acc + pre;
 #pragma unroll
             for (int jj = 0; jj < TPT; ++jj) {
                 psi += ph[jj];
@@ -367,12 +389,15 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                     *reinterpret_cast<uint32_t*>(ct + off) = co;
                 }
             }
+            psi_acc += tot;
             if (tid == 0 && s == 0) M3_TRACE_EV(c, 29);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[RAW_EMPTY0 + rs]);
         }
         const int cs = c % kCoefSlots;
         Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
+        psi_acc -= 6.283185307179586f * rintf(psi_acc * 0.15915494309189535f);
+        if (ts == 0) cf.psi_end()[pair] = psi_acc;
         if (tid == 0) M3_TRACE_EV(c, 3);
 
         // ---- w-scaled X:  Xw[u, r] = 2^(cum2_end - cum2_u) w_u x[u, r]  (needs the
@@ -403,6 +428,7 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
+            mbar_arrive(&bar[COEF_FULL0 + cs]);
             mbar_arrive(&bar[OPS_FULL0 + slot]);
             mbar_arrive(&bar[DT_EMPTY0 + st]);
         }
@@ -410,24 +436,14 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
     }
 }
 
-// Coefficient warp: per chunk, the log2-decay prefix sum (warp scan), gamma, w and the
-// mask exponent offsets ew_u = log2(w_u) - cum2_u into a ring of slots; per raw sub-chunk,
-// the call-relative angle of every state pair at the start of each rotation warp's
-// token range (a running sum over the tokens, the RoPE frame of Proposition 4), and the
-// angle at the chunk end (reduced mod 2 pi).
+// Coefficient warp: per-token log2-decay prefix sum (warp scan), gamma, w and the mask
+// exponent offsets ew_u = log2(w_u) - cum2_u of each chunk, into a ring of slots.
 template <int NST, int Q, int R>
 __device__ void coefficients(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
     using C = Cfg<NST, Q, R>;
-    constexpr int PAIRS = C::PAIRS, PPL = PAIRS / 32, TSPLIT = C::TSPLIT, TPT = C::TPT;
     const ScanArgs& a = p.a;
     const int lane = threadIdx.x & 31;
     const int hq = (blockIdx.x % a.H) & 3;
-    const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
-    float* psib = reinterpret_cast<float*>(sm + C::OFF_RSUM);
-    float psi[PPL];                              // pairs PPL*lane .. PPL*lane + PPL - 1
-#pragma unroll
-    for (int k = 0; k < PPL; ++k) psi[k] = 0.f;
-    int raw_it = 0;
     for (int c = 0; c < p.nchunks; ++c) {
         const int st = c & 1, cs = c % kCoefSlots;
         if (!warp_wait(&bar[DT_FULL0 + st], (c >> 1) & 1, ab)) return;
@@ -463,46 +479,8 @@ __device__ void coefficients(const TcParams& p, uint8_t* sm, uint64_t* bar, cons
         }
         if (lane == 0) *cf.cum2_end() = carry;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[CUM_READY0 + cs]);
-
-        // ---- range start angles of every raw sub-chunk of this chunk
-        for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
-            const int rs = raw_it & 1;
-            if (!warp_wait(&bar[RAW_FULL0 + rs], (raw_it >> 1) & 1, ab)) return;
-            const float* th = reinterpret_cast<const float*>(sm + C::OFF_RAW + rs * C::RAW_BYTES +
-                                                             2 * C::BRAW_BYTES);
-            float* pb = psib + rs * TSPLIT * PAIRS;
-            const int tb = s * C::RT;
-#pragma unroll
-            for (int q = 0; q < TSPLIT; ++q) {
-#pragma unroll
-                for (int k = 0; k < PPL; ++k) pb[q * PAIRS + PPL * lane + k] = psi[k];
-#pragma unroll
-                for (int jj = 0; jj < TPT; ++jj) {
-                    const int j = q * TPT + jj;
-                    const float d = angle ? 1.f : dtt[(tb + j) * 4 + hq];
-                    if constexpr (PPL == 2) {
-                        const float2 tv = *reinterpret_cast<const float2*>(th + j * PAIRS + 2 * lane);
-                        psi[0] = fmaf(d, tv.x, psi[0]);
-                        psi[1] = fmaf(d, tv.y, psi[1]);
-                    } else {
-                        psi[0] = fmaf(d, th[j * PAIRS + lane], psi[0]);
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bar[PSI_READY0 + rs]);
-                mbar_arrive(&bar[RAW_EMPTY0 + rs]);
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < PPL; ++k) {
-            psi[k] -= 6.283185307179586f * rintf(psi[k] * 0.15915494309189535f);
-            cf.psi_end()[PPL * lane + k] = psi[k];
-        }
-        __syncwarp();
         if (lane == 0) {
+            mbar_arrive(&bar[CUM_READY0 + cs]);
             mbar_arrive(&bar[COEF_FULL0 + cs]);
             mbar_arrive(&bar[DT_EMPTY0 + st]);
         }
