@@ -122,8 +122,13 @@ m3_status m3_scan_workspace_bytes(const m3_dims* dims, int32_t seqlen, int32_t c
  * aligned; float arrays 4-byte aligned.  seqlen == 0 is a no-op returning M3_OK
  * (only dims, chunk and the state are validated; no other pointer is examined).
  * bf16 io runs on the tcgen05 tensor-core kernel where the shape is supported
- * (SISO N in {64,128}, P = 64; MIMO Q*R <= 256); other shapes and fp32 io run
- * the sequential fp32 CUDA-core kernel.
+ * (P = 64, nheads % 4 == 0, and N in {64, 128} for R = 1, N = 64 for R in {2, 4});
+ * other shapes and fp32 io run the sequential fp32 CUDA-core kernel.  The
+ * tensor-core kernel tiles chunk * R (token, rank) rows per chunk, 64 or 128 of
+ * them: a chunk whose chunk * R falls outside [64, 128] runs as the nearest tile
+ * (e.g. R = 4 with chunk 64 as 32-token tiles; "Multi-Input, Multi-Output
+ * Formulation" likewise shrinks the MIMO chunk by R to hold the intra-chunk
+ * FLOPs), which again changes rounding only.
  */
 m3_status m3_scan_fwd(const m3_dims* dims, int32_t seqlen, int32_t chunk, const void* x,
                       const void* B, const void* C, const float* dt, const float* A,

@@ -128,9 +128,10 @@ m3_status m3_scan_workspace_bytes(const m3_dims* d, int32_t seqlen, int32_t chun
     if (seqlen < 0) return M3_ERR_SHAPE;
     if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return M3_ERR_SHAPE;
     size_t extra = 0;
-    if (d->io_dtype == M3_BF16 && scan_tc_supported(d->dstate, d->headdim, d->rank, chunk, d->nheads))
+    const int qt = scan_tc_chunk(d->dstate, d->headdim, d->rank, chunk, d->nheads);
+    if (d->io_dtype == M3_BF16 && qt)
         extra = scan_tc_workspace_bytes(d->batch, d->nheads, d->dstate, d->headdim, d->rank,
-                                        seqlen, chunk);
+                                        seqlen, qt);
     *bytes = kStatusBytes + ((extra + 255) / 256) * 256;
     return M3_OK;
 }
@@ -157,9 +158,10 @@ m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const voi
 
     const int N = d->dstate, P = d->headdim, R = d->rank;
     // the tensor-core kernel reads dt / A / lam / theta with TMA (16-byte aligned rows)
-    const bool use_tc = !(flags & M3_FLAG_FORCE_SIMT) && d->io_dtype == M3_BF16 &&
-                        scan_tc_supported(N, P, R, chunk, d->nheads) && aligned(dt, 16) &&
-                        aligned(A, 16) && aligned(lam, 16) && aligned(theta, 16);
+    const int qt = scan_tc_chunk(N, P, R, chunk, d->nheads);
+    const bool use_tc = !(flags & M3_FLAG_FORCE_SIMT) && d->io_dtype == M3_BF16 && qt &&
+                        aligned(dt, 16) && aligned(A, 16) && aligned(lam, 16) &&
+                        aligned(theta, 16);
     int ppt = 0, ns = 0;
     if (!use_tc && (!rank_has_kernel(R) || !simt_shape(N, P, &ppt, &ns)))
         return M3_ERR_UNSUPPORTED;
@@ -172,7 +174,7 @@ m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const voi
     a.status = static_cast<uint32_t*>(workspace);
     a.ws = static_cast<char*>(workspace) + kStatusBytes;
     a.T = seqlen; a.batch = d->batch; a.H = d->nheads; a.G = d->ngroups; a.P = P; a.N = N;
-    a.chunk = chunk; a.ppt = ppt; a.ns = ns; a.flags = flags;
+    a.chunk = use_tc ? qt : chunk; a.ppt = ppt; a.ns = ns; a.flags = flags;
 
     if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return M3_ERR_CUDA;
     cudaError_t e = use_tc ? launch_scan_tc(a, R, s) : launch_scan_simt(a, R, d->io_dtype, s);
@@ -202,8 +204,8 @@ m3_status m3_decode_step(const m3_dims* d, const void* x, const void* B, const v
     std::memset(&a, 0, sizeof(a));
     a.x = x; a.B = B; a.C = C; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D;
     a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y;
-    a.H = d->nheads; a.G = d->ngroups; a.P = d->headdim; a.N = d->dstate; a.ppt = ppt;
-    a.flags = flags;
+    a.H = d->nheads; a.G = d->ngroups; a.P = d->headdim; a.N = d->dstate;
+    a.ppt = ppt; a.flags = flags;
     cudaError_t e = launch_decode(a, d->batch, d->rank, d->io_dtype, s);
     if (e != cudaSuccess) return launch_status(e);
     const size_t row = io_bytes(d->io_dtype) * (size_t)d->ngroups * d->rank * d->dstate;

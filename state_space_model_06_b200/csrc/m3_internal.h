@@ -16,7 +16,7 @@ cudaError_t launch_scan_simt(const ScanArgs& a, int R, int io_dtype, cudaStream_
 // tcgen05 chunked prefill (bf16 io).  Returns cudaErrorNotSupported for shapes
 // the kernel does not cover (the caller then reports M3_ERR_UNSUPPORTED or
 // falls back to the SIMT kernel).
-bool scan_tc_supported(int N, int P, int R, int chunk, int H);
+int scan_tc_chunk(int N, int P, int R, int chunk, int H);   // tile chunk, 0 = none
 size_t scan_tc_workspace_bytes(int batch, int H, int N, int P, int R, long long T, int chunk);
 cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s);
 

@@ -1018,19 +1018,23 @@ extern "C" int m3_trace_copy(void* dst, size_t bytes, int cta) {
 }
 #endif
 
-bool scan_tc_supported(int N, int P, int R, int chunk, int H) {
-    if (P != kP || H % 4 != 0) return false;
-    if (N != 64 && N != 128) return false;
-    if (R == 1) return chunk == 64 || chunk == 128;
-    if (R == 2) return N == 64 && (chunk == 32 || chunk == 64);
-    if (R == 4) return N == 64 && (chunk == 16 || chunk == 32);
-    return false;
+// The tile holds L = chunk * R (token, rank) rows with L in {64, 128}: the M = 64 / 128
+// MMA shapes, and the S and Y accumulators that fit TMEM.  A requested chunk whose L
+// falls outside is run with the nearest tile (L clamped into [64, 128]): the chunked form
+// is exact for any blocking, so only rounding changes.  Returns 0 where no tile applies.
+int scan_tc_chunk(int N, int P, int R, int chunk, int H) {
+    if (P != kP || H % 4 != 0) return 0;
+    if (R != 1 && R != 2 && R != 4) return 0;
+    if (N != 64 && (N != 128 || R != 1)) return 0;
+    int L = chunk * R;
+    L = L < 64 ? 64 : (L > 128 ? 128 : L);
+    return L / R;
 }
 
 size_t scan_tc_workspace_bytes(int, int, int, int, int, long long, int) { return 0; }
 
 cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s) {
-    const int N = a.N, Q = a.chunk;
+    const int N = a.N, Q = a.chunk;   // the tile chunk chosen by scan_tc_chunk
     if (R == 1) {
         if (N == 128 && Q == 64) return launch_t<128, 64, 1>(a, s);
         if (N == 128 && Q == 128) return launch_t<128, 128, 1>(a, s);

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 TOL = 2e-2
 
 
-def run_workload(w, chunk=None, calls=1, seed=0):
+def run_workload(w, chunk=None, calls=1, seed=0, flags=0):
     Q = chunk or w.chunk
     inp = inputs.make_scan_inputs(w.batch, w.seqlen, w.nheads, w.ngroups, w.headdim, w.dstate,
                                   w.rank, io_dtype=w.io_dtype, theta_max=w.theta_max, seed=seed)
@@ -34,7 +34,7 @@ def run_workload(w, chunk=None, calls=1, seed=0):
         sl = {k: inp[k][:, c * Tc:(c + 1) * Tc].contiguous().cuda() for k in KEYS}
         y = torch.empty_like(sl["x"])
         m3.m3_scan_fwd(d, Tc, Q, sl["x"], sl["B"], sl["C"], sl["dt"], sl["A"], sl["lam"],
-                       sl["theta"], D, st, y, ws)
+                       sl["theta"], D, st, y, ws, flags=flags)
         assert m3.m3_query_status(ws) == m3.M3_OK
         ys.append(y.cpu())
         del sl
@@ -68,12 +68,13 @@ def test_siso_prefill_1p5b_full():
     check(inp, yg, hg, [0, 7], [0, 37, 63])
 
 
-@pytest.mark.parametrize("chunk", [64, 32])
-def test_mimo_prefill_r4_full(chunk):
-    """chunk 64 with R = 4 runs the sequential kernel; chunk 32 the tensor-core kernel
-    (the pages' MIMO chunk rule C_MIMO = C_SISO / R)."""
+@pytest.mark.parametrize("chunk,flags", [(64, 0), (32, 0), (64, m3.M3_FLAG_FORCE_SIMT)],
+                         ids=["chunk64", "chunk32", "chunk64_sequential"])
+def test_mimo_prefill_r4_full(chunk, flags):
+    """R = 4 on the tensor-core kernel (chunk 64 runs as 32-token tiles, chunk * R = 128
+    rows) and on the sequential fp32 kernel."""
     w = inputs.WORKLOADS["mimo_prefill_r4"]
-    inp, yg, hg = run_workload(w, chunk=chunk, seed=1)
+    inp, yg, hg = run_workload(w, chunk=chunk, seed=1, flags=flags)
     check(inp, yg, hg, [3], [5, 60])
 
 

@@ -31,6 +31,9 @@ CASES = [
     (1, 4, 1, 64, 64, 2, 33, 32, math.pi / 8),       # MIMO R = 2, Q*R = 64
     (1, 4, 1, 64, 128, 1, 1, 64, math.pi / 8),       # T = 1
     (1, 4, 1, 64, 128, 1, 64, 64, math.pi / 8),      # exactly one chunk
+    (1, 4, 1, 64, 128, 1, 100, 32, math.pi / 8),     # chunk 32 runs as 64-token tiles
+    (1, 4, 1, 64, 64, 4, 150, 64, math.pi / 8),      # R = 4, chunk 64 runs as 32-token tiles
+    (1, 4, 1, 64, 64, 2, 90, 16, math.pi / 8),       # R = 2, chunk 16 runs as 32-token tiles
 ]
 
 
