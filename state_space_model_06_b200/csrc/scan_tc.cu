@@ -47,13 +47,16 @@ using namespace sm100;
 #define M3_TRACE_EVENTS 32
 __device__ unsigned long long g_m3_trace[M3_TRACE_CHUNKS][M3_TRACE_EVENTS];
 __device__ int g_m3_trace_cta = 0;
+__shared__ int s_m3_trace_on;   // copied from g_m3_trace_cta once per CTA
 #define M3_TRACE_EV(c, e)                                                           \
     do {                                                                            \
-        if ((int)blockIdx.x == g_m3_trace_cta && (c) < M3_TRACE_CHUNKS)             \
-            g_m3_trace[(c)][(e)] = clock64();                                       \
+        if (s_m3_trace_on && (c) < M3_TRACE_CHUNKS) g_m3_trace[(c)][(e)] = clock64(); \
     } while (0)
+#define M3_TRACE_INIT() \
+    do { if (threadIdx.x == 0) s_m3_trace_on = ((int)blockIdx.x == g_m3_trace_cta); } while (0)
 #else
 #define M3_TRACE_EV(c, e) do { } while (0)
+#define M3_TRACE_INIT() do { } while (0)
 #endif
 
 namespace {
@@ -862,13 +865,15 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
 template <int NST, int Q, int R>
 __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_constant__ TcParams p) {
     using C = Cfg<NST, Q, R>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base for the SW128 tiles, as an offset from smem_raw so that the
+    // compiler keeps every access in the shared address space
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     const int w = threadIdx.x >> 5;
 
+    M3_TRACE_INIT();
     if (threadIdx.x == 0) {
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], bar_count(i));
         misc[1] = 0u;  // abort flag

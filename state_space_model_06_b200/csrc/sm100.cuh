@@ -69,13 +69,20 @@ struct Abort {
     uint64_t limit_ns;
 };
 
+// The poll itself may suspend the thread (hint 20 us); the abort flag and the clock are
+// looked at only every 64 polls, so that waiting warps spend few issue slots.  The wait
+// stays bounded: at most 64 suspended polls pass between two looks at the clock.
 __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const Abort& ab) {
     const uint64_t t0 = globaltimer();
+    const uint64_t limit = ab.limit_ns;
+    volatile uint32_t* flag = ab.flag;
     while (true) {
-        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
-        if (*ab.flag) return false;
-        if (globaltimer() - t0 > ab.limit_ns) {
-            *ab.flag = 1u;
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+        if (*flag) return false;
+        if (globaltimer() - t0 > limit) {
+            *flag = 1u;
             if (ab.status) atomicOr(ab.status, (uint32_t)M3_ERR_TIMEOUT);
             return false;
         }
