@@ -374,22 +374,58 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                 pre += (qq < ts) ? v : 0.f;
             }
             float psi = psi_acc + pre;
+            float cn[TPT], sn[TPT];
 #pragma unroll
             for (int jj = 0; jj < TPT; ++jj) {
                 psi += ph[jj];
-                float sn, cn;
-                __sincosf(psi, &sn, &cn);   // |psi| < pi + one chunk of angle increments
+                __sincosf(psi, &sn[jj], &cn[jj]);   // |psi| < pi + one chunk of angle increments
+            }
+            // operand rows (tb + j0 + jj) * R + r; when the first of them is a multiple of 8
+            // the SW128 chunk of every row is a compile-time xor of this thread's chunk
+            const int row0 = (tb + j0) * R;
+            uint8_t* const cbase = ct + (uint32_t)atom * C::L * 128u + (uint32_t)(col & 7) * 2u;
+            const uint32_t cx = (uint32_t)((col >> 3) & 7);
+            auto store = [&](int jj, int r, uint32_t bo, uint32_t co) {
+                const int k = jj * R + r;
+                uint32_t off;
+                if constexpr ((TPT * R) % 8 == 0 && (C::RT * R) % 8 == 0)
+                    off = (uint32_t)(row0 + k) * 128u + ((cx ^ (uint32_t)(k & 7)) << 4);
+                else
+                    off = (uint32_t)(row0 + k) * 128u + ((cx ^ (uint32_t)((row0 + k) & 7)) << 4);
+                *reinterpret_cast<uint32_t*>(cbase + C::CT_BYTES + off) = bo;
+                *reinterpret_cast<uint32_t*>(cbase + off) = co;
+            };
+            // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1], two tokens per packed
+            // fp32x2 operation (their cos and sin form the packed operands)
+#pragma unroll
+            for (int jj = 0; jj + 1 < TPT; jj += 2) {
+                const float2 c2 = make_float2(cn[jj], cn[jj + 1]);
+                const float2 s2 = make_float2(sn[jj], sn[jj + 1]);
+                const float2 m2 = make_float2(-sn[jj], -sn[jj + 1]);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const uint32_t ba = bv[jj][r], bb = bv[jj + 1][r];
+                    const uint32_t ca = cv[jj][r], cb = cv[jj + 1][r];
+                    const float2 b0 = make_float2(bf16lo(ba), bf16lo(bb));
+                    const float2 b1 = make_float2(bf16hi(ba), bf16hi(bb));
+                    const float2 c0 = make_float2(bf16lo(ca), bf16lo(cb));
+                    const float2 c1 = make_float2(bf16hi(ca), bf16hi(cb));
+                    const float2 nb0 = __ffma2_rn(c2, b0, __fmul2_rn(s2, b1));
+                    const float2 nb1 = __ffma2_rn(c2, b1, __fmul2_rn(m2, b0));
+                    const float2 nc0 = __ffma2_rn(c2, c0, __fmul2_rn(s2, c1));
+                    const float2 nc1 = __ffma2_rn(c2, c1, __fmul2_rn(m2, c0));
+                    store(jj, r, pack_bf16x2(nb0.x, nb1.x), pack_bf16x2(nc0.x, nc1.x));
+                    store(jj + 1, r, pack_bf16x2(nb0.y, nb1.y), pack_bf16x2(nc0.y, nc1.y));
+                }
+            }
+            if constexpr (TPT % 2 == 1) {
+                const int jj = TPT - 1;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     const float b0 = bf16lo(bv[jj][r]), b1 = bf16hi(bv[jj][r]);
                     const float c0 = bf16lo(cv[jj][r]), c1 = bf16hi(cv[jj][r]);
-                    // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1]
-                    const uint32_t bo = pack_bf16x2(fmaf(cn, b0, sn * b1), fmaf(cn, b1, -sn * b0));
-                    const uint32_t co = pack_bf16x2(fmaf(cn, c0, sn * c1), fmaf(cn, c1, -sn * c0));
-                    const int row = (tb + j0 + jj) * R + r;
-                    const uint32_t off = (uint32_t)atom * C::L * 128u + sw128_off(row, col);
-                    *reinterpret_cast<uint32_t*>(bt + off) = bo;
-                    *reinterpret_cast<uint32_t*>(ct + off) = co;
+                    store(jj, r, pack_bf16x2(fmaf(cn[jj], b0, sn[jj] * b1), fmaf(cn[jj], b1, -sn[jj] * b0)),
+                          pack_bf16x2(fmaf(cn[jj], c0, sn[jj] * c1), fmaf(cn[jj], c1, -sn[jj] * c0)));
                 }
             }
             psi_acc += tot;
@@ -555,6 +591,7 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
             const float ct = cum2[t];
             const float gt = cf.gam()[t];
             const float* ew = cf.ew();
+            const int tR = t * R;                  // first column of the row's own token
 #pragma unroll 1
             for (int cb = 0; cb < kLCols; cb += 16) {
                 uint32_t sv[16];
@@ -567,11 +604,12 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int col = colb + j + e;
-                        const int u = col / R;
                         const float sv_f = __uint_as_float(sv[j + e]);
-                        const float v = sv_f * ex2_approx(ct + ew[u]);
-                        m[e] = (u < t) ? v : 0.f;
-                        if (u == t) m[e] = sv_f * gt + (col == lrow ? Dh : 0.f);
+                        // earlier tokens: decay times the trapezoid weight; the own token's
+                        // R columns: gamma (plus D on the diagonal); later tokens: 0
+                        const float v = sv_f * ex2_approx(ct + ew[col / R]);
+                        const float d = fmaf(sv_f, gt, col == lrow ? Dh : 0.f);
+                        m[e] = col < tR ? v : (col < tR + R ? d : 0.f);
                     }
                     uint4 o;
                     o.x = pack_bf16x2(m[0], m[1]);
