@@ -300,6 +300,23 @@ def w_dec_batch(name):
     return inputs.WORKLOADS[name].batch
 
 
+def oracle_workload(w, inp, rows):
+    """Time the CPU oracle on the first `rows` batch rows of the workload's own inputs (all
+    heads, all tokens), one row per call so that host memory stays bounded."""
+    import oracle
+    threads = min(oracle.max_threads(), w.nheads)
+    secs = 0.0
+    for b in range(rows):
+        arr = {k: inp[k][b:b + 1].double().numpy() for k in ("x", "B", "C", "dt", "A", "lam",
+                                                              "theta")}
+        D = inp["D"].double().numpy()
+        t0 = time.perf_counter()
+        oracle.scan(arr["x"], arr["B"], arr["C"], arr["dt"], arr["A"], arr["lam"], arr["theta"],
+                    D=D, nthreads=threads)
+        secs += time.perf_counter() - t0
+    return rows * w.seqlen / secs, threads, secs
+
+
 def oracle_sample(w, seqlen, seed=0):
     """Time the CPU oracle on batch row 0, all heads, the first `seqlen` tokens."""
     import oracle
@@ -380,10 +397,12 @@ def ours(args):
                        "d2h_bytes_per_step": d2h}
 
     if rank == 0 and ws_world == 1 and not args.no_cpu:
-        tps, cores, secs = oracle_sample(w, args.cpu_tokens)
+        rows = max(1, min(args.cpu_rows, w.batch))
+        tps, cores, secs = oracle_workload(w, inp, rows)
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": f"batch row 0, all {w.nheads} heads, first "
-                                          f"{args.cpu_tokens} tokens ({secs:.1f} s of fp64 CPU work)"}
+                                "sample": f"the workload's own inputs, batch rows 0..{rows - 1} of "
+                                          f"{w.batch}, all {w.nheads} heads and {w.seqlen} tokens "
+                                          f"({secs:.1f} s of fp64 CPU work)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_world > 1:
@@ -432,7 +451,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--cpu-rows", type=int, default=8,
+                    help="batch rows of the workload timed on the CPU oracle (default: all)")
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling only)")
     ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and CPU legs")
