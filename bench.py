@@ -256,7 +256,7 @@ def time_prefill_e2e(w, d, inp, st, ws, steps, stream, dev):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
-def time_decode(name, dev, stream, seed):
+def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS):
     w = inputs.WORKLOADS[name]
     inp = inputs.make_decode_inputs(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
                                     tokens=DECODE_POOL, io_dtype=w.io_dtype,
@@ -281,18 +281,18 @@ def time_decode(name, dev, stream, seed):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for t in range(DECODE_TOKENS):
+    for t in range(tokens):
         m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / DECODE_TOKENS
+    ms = e0.elapsed_time(e1) / tokens
     finite = bool(torch.isfinite(st.h).all().item())
     byts = decode_algorithmic(w)
     return {"tokens_per_s": w.batch / (ms / 1e3), "us_per_step": ms * 1e3,
             "achieved_gbs": byts / (ms / 1e3) / 1e9, "alg_bytes_per_step": byts,
             "state_finite": finite,
             "config": {"batch": w.batch, "heads": w.nheads, "headdim": w.headdim,
-                       "dstate": w.dstate, "rank": w.rank, "tokens": DECODE_TOKENS,
+                       "dstate": w.dstate, "rank": w.rank, "tokens": tokens,
                        "distinct_tokens": DECODE_POOL}}
 
 
@@ -382,8 +382,8 @@ def ours(args):
         args.no_decode = args.no_e2e = args.no_cpu = True
     if not args.no_decode:
         line["decode"] = {}
-        for name in DECODES:
-            r = time_decode(name, dev, stream, seed=100 + rank)
+        for name in (args.decode or DECODES):
+            r = time_decode(name, dev, stream, seed=100 + rank, tokens=args.decode_tokens)
             r["hbm_frac"] = r["achieved_gbs"] / pk["hbm_gbs"]
             r["tokens_per_s"], _ = job_throughput(w_dec_batch(name), r["us_per_step"] / 1e3,
                                                   ws_world)
@@ -454,6 +454,10 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8,
                     help="batch rows of the workload timed on the CPU oracle (default: all)")
     ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--decode", action="append", choices=DECODES,
+                    help="time only these decode workloads (profiling)")
+    ap.add_argument("--decode-tokens", type=int, default=DECODE_TOKENS,
+                    help="sequential decode tokens timed per workload")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling only)")
     ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and CPU legs")
     args = ap.parse_args()

@@ -20,13 +20,16 @@
 //   MIMO: rows are (token, rank) pairs; L is shared by the R x R blocks.
 //
 // Kernel: one CTA per (batch, head), persistent over the chunks of the sequence.
-//   warp 0      TMA producer (x, B, C, theta, dt/A/lam tiles; zero fill past T)
-//   warp 1      tcgen05.mma issuer:  S = C~ B~^T,  dS = B~^T (w-scaled X),
-//               Y_inter = C~ g,  Y_intra = (S o L) X      (fp32 accumulators in TMEM)
-//   warps 2-5   epilogue: mask S -> bf16 (S o L); fp32 state update in registers;
-//               y = Y_intra + e^{cum} Y_inter + D x, TMA store
-//   warps 6-9   rotation: per-token coefficients (warp scan), cumulative angles,
-//               sincos, rotate B and C into swizzled bf16 MMA operands, scale X
+//   warp 0       TMA producer (dt/A/lam per chunk, raw B, C, theta sub-chunks; zero fill past T)
+//   warp 1       tcgen05.mma issuer:  S = C~ B~^T,  dS = B~^T (w-scaled X),
+//                Y_inter = C~ g,  Y_intra = (S o L) X      (fp32 accumulators in TMEM)
+//   warps 2-5    epilogue: mask S -> bf16 (S o L); y = Y_intra + e^{cum} Y_inter over the x tile
+//   warps 6-13   rotation: cumulative angles, sincos, rotate B and C into swizzled bf16 MMA
+//                operands, w-scaled X
+//   warp 14      coefficients: log2-decay prefix (warp scan), gamma, w, mask exponent offsets
+//   warp 15      x tiles in, y tiles out (TMA)
+//   warps 16-19  state: g in TMEM (fp32), g <- e^{cum_end} g + dS, bf16 copy for Y_inter,
+//                h_T rotated back to the original frame at the end of the call
 // Every wait is bounded; a timeout raises a CTA-wide abort and records
 // M3_ERR_TIMEOUT in the workspace status word.
 #include <cuda.h>
