@@ -11,13 +11,17 @@
 // One CTA per (batch, head).  Thread (j, rg) owns float4 column chunk j of the
 // state and `ppt` state pairs (rows 2i, 2i+1) with i = rg + k * RG, so every
 // rotation is thread-local; the readout's sum over N is finished in shared memory.
+// All of a thread's state loads are issued before anything else, so the pairs per thread
+// set the bytes in flight per register: 8 for SISO, 4 for MIMO (whose R-fold arithmetic
+// per element needs the registers and threads).
 #include "m3_internal.h"
 
 namespace m3 {
 
-constexpr int kDecodeMaxPPT = 4;
 
-template <typename IO, int R>
+// MAXP: the largest pairs-per-thread count this instantiation handles (a.ppt <= MAXP); it
+// sizes the per-thread state registers, so each shape only pays for the pairs it uses.
+template <typename IO, int R, int MAXP>
 __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     extern __shared__ float sm[];
     const int N = a.N, P = a.P, H = a.H, G = a.G;
@@ -39,9 +43,9 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
 
     // 1. issue the state loads first: they are the whole cost of the step
     float4* hrow = reinterpret_cast<float4*>(a.h + (size_t)bh * N * P);
-    float4 v0[kDecodeMaxPPT], v1[kDecodeMaxPPT];
+    float4 v0[MAXP], v1[MAXP];
 #pragma unroll
-    for (int k = 0; k < kDecodeMaxPPT; ++k) {
+    for (int k = 0; k < MAXP; ++k) {
         if (k < a.ppt) {
             const int i = rg + k * RG;
             v0[k] = __ldcs(hrow + (size_t)(2 * i) * CPR + j);
@@ -87,7 +91,7 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
         for (int q = 0; q < 4; ++q) yp[r][q] = 0.f;
 
 #pragma unroll
-    for (int k = 0; k < kDecodeMaxPPT; ++k) {
+    for (int k = 0; k < MAXP; ++k) {
         if (k < a.ppt) {
             const int i = rg + k * RG;
             const float c = cs[i], s = sn[i];
@@ -137,28 +141,30 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     }
 }
 
-template <typename IO, int R>
+template <typename IO, int R, int MAXP>
 static cudaError_t launch_decode_t(const DecodeArgs& a, int batch, cudaStream_t s) {
     const int RG = (a.N / 2) / a.ppt;
     const int threads = (a.P / 4) * RG;
     const size_t smem = sizeof(float) * (size_t)(2 * R * a.P + 3 * R * a.N + a.N + RG * R * a.P);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<IO, R>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<IO, R, MAXP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    decode_kernel<IO, R><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
+    decode_kernel<IO, R, MAXP><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
 template <typename IO>
 static cudaError_t launch_decode_io(const DecodeArgs& a, int batch, int R, cudaStream_t s) {
+    if (a.ppt > 8 || (a.ppt > 4 && R != 1)) return cudaErrorNotSupported;
     switch (R) {
-        case 1: return launch_decode_t<IO, 1>(a, batch, s);
-        case 2: return launch_decode_t<IO, 2>(a, batch, s);
-        case 3: return launch_decode_t<IO, 3>(a, batch, s);
-        case 4: return launch_decode_t<IO, 4>(a, batch, s);
-        case 8: return launch_decode_t<IO, 8>(a, batch, s);
+        case 1: return a.ppt > 4 ? launch_decode_t<IO, 1, 8>(a, batch, s)
+                                 : launch_decode_t<IO, 1, 4>(a, batch, s);
+        case 2: return launch_decode_t<IO, 2, 4>(a, batch, s);
+        case 3: return launch_decode_t<IO, 3, 4>(a, batch, s);
+        case 4: return launch_decode_t<IO, 4, 4>(a, batch, s);
+        case 8: return launch_decode_t<IO, 8, 4>(a, batch, s);
         default: return cudaErrorNotSupported;
     }
 }

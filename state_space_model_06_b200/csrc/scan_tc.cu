@@ -79,13 +79,16 @@ enum Bar {
     COEF_FULL0, COEF_FULL1, COEF_FULL2, COEF_FULL3, COEF_EMPTY0, COEF_EMPTY1, COEF_EMPTY2,
     COEF_EMPTY3, CUM_READY0, CUM_READY1, CUM_READY2, CUM_READY3, RS0, RS1,
     OPS_FULL0, OPS_FULL1, OPS_EMPTY0, OPS_EMPTY1, S_FULL, S_EMPTY, SL_FULL, DS_FULL, DS_EMPTY,
-    G_FULL, G_EMPTY, Y_FULL0, Y_FULL1, Y_EMPTY0, Y_EMPTY1, Y_STAGED, DRAIN, NEVER, NUM_BARS
+    G_FULL, G_EMPTY, Y_FULL0, Y_FULL1, Y_EMPTY0, Y_EMPTY1, Y_STAGED0, Y_STAGED1, Y_STAGED2, DRAIN,
+    NEVER, NUM_BARS
 };
 
 // arrival count of each barrier: 1 for TMA expect_tx / tcgen05.commit / single-thread or
-// single-warp arrivals, 2 for the coefficient slots (x warp + state warpgroup), 4 for one
-// elected lane per warp of a four-warp group, 8 for the rotation warps, 9 where the
-// coefficient warp joins them
+// single-warp arrivals, 4 for one elected lane per warp of a four-warp group, 5 for the
+// coefficient slots (x warp + the four state warps), 8 for the rotation warps, 9 where the
+// coefficient warp joins them.  Every barrier that a role waits on can complete its next
+// phase only after that role has passed the current one (each y stage has its own
+// Y_STAGED barrier for this reason), so no waiter can miss a phase.
 __device__ __forceinline__ uint32_t bar_count(int i) {
     switch (i) {
         case DT_EMPTY0: case DT_EMPTY1: case COEF_FULL0: case COEF_FULL1: case COEF_FULL2:
@@ -94,9 +97,9 @@ __device__ __forceinline__ uint32_t bar_count(int i) {
         case RAW_EMPTY0: case RAW_EMPTY1: case RS0: case RS1: case OPS_FULL0: case OPS_FULL1:
             return kRotWarps;
         case COEF_EMPTY0: case COEF_EMPTY1: case COEF_EMPTY2: case COEF_EMPTY3:
-            return 2;
+            return 5;
         case S_EMPTY: case SL_FULL: case DS_EMPTY: case G_FULL:
-        case Y_EMPTY0: case Y_EMPTY1: case Y_STAGED:
+        case Y_EMPTY0: case Y_EMPTY1: case Y_STAGED0: case Y_STAGED1: case Y_STAGED2:
             return 4;
         default:
             return 1;
@@ -143,6 +146,7 @@ struct Cfg {
     static_assert(pick() != 0, "shared memory budget exceeded");
     static constexpr int OPS = pick() / 10000;                  // operand slots
     static constexpr int XST = (pick() / 1000) % 10;            // x / y staging stages
+    static_assert(XST >= 2 && XST <= 3, "one Y_STAGED barrier per x / y stage");
     static constexpr int RT = pick() % 1000;                    // tokens per raw sub-chunk
     static constexpr int NSUB = Q / RT;
     static constexpr int TPT = RT / TSPLIT;                     // tokens per rotation thread
@@ -670,7 +674,7 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
         __syncwarp();
         if (lane == 0) {
             mbar_arrive(&bar[Y_EMPTY0 + yb]);
-            mbar_arrive(&bar[Y_STAGED]);
+            mbar_arrive(&bar[Y_STAGED0 + xs]);
         }
         if (etid == 0) M3_TRACE_EV(c, 22);
     }
@@ -801,11 +805,9 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
         if (lane == 0) {
             mbar_arrive(&bar[DS_EMPTY]);
             if (more) mbar_arrive(&bar[G_FULL]);
+            mbar_arrive(&bar[COEF_EMPTY0 + cs]);   // this warp has read the slot's cum2_end
         }
-        if (stid == 0) {
-            M3_TRACE_EV(c, 18);
-            mbar_arrive(&bar[COEF_EMPTY0 + cs]);
-        }
+        if (stid == 0) M3_TRACE_EV(c, 18);
     }
     if (stid == 0) {
         // only this warpgroup read x_prev (for g_0), so the carried x can be replaced now
@@ -888,7 +890,7 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
     for (int c = 0; c < C::XST && c < p.nchunks; ++c) load(c);
     bool ok = true;
     for (int c = 0; c < p.nchunks; ++c) {
-        if (!(ok = mbar_wait(&bar[Y_STAGED], c & 1, ab))) break;
+        if (!(ok = mbar_wait(&bar[Y_STAGED0 + c % C::XST], (c / C::XST) & 1, ab))) break;
         const int xs = c % C::XST;
         tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, c * Q, b);
         bulk_commit();
