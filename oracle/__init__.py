@@ -60,6 +60,8 @@ def _load(path=None):
             [dp] * 12 + [ctypes.c_int]
         lib.m3o_scan.restype = ctypes.c_int
         lib.m3o_max_threads.restype = ctypes.c_int
+        lib.m3o_gate.argtypes = [ctypes.c_int64, dp, dp]
+        lib.m3o_gate.restype = None
         _libs[path] = lib
     return _libs[path]
 
@@ -80,12 +82,14 @@ def _ptr(a):
 
 
 def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
-         theta_is_angle: bool = False, nthreads: int = 0, lib_path=None):
+         theta_is_angle: bool = False, nthreads: int = 0, lib_path=None, z=None):
     """Run the recurrence over T tokens.
 
     Shapes: x [b,T,H,R,P]; B, C [b,T,G,R,N]; dt, A, lam [b,T,H];
     theta [b,T,G,N/2]; D [H] or None; h0 [b,H,N,P] or None (zeros);
-    x_prev [b,H,R,P] / B_prev [b,G,R,N] or None (fresh sequence: zeros).
+    x_prev [b,H,R,P] / B_prev [b,G,R,N] or None (fresh sequence: zeros);
+    z [b,T,H,R,P] or None: output gate, y <- y * SiLU(z) after the skip
+    ("Technical Approach", output gating).
 
     Returns (y [b,T,H,R,P], h_T, x_prev_out, B_prev_out), all float64.
     """
@@ -110,16 +114,21 @@ def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
                           _ptr(D), _ptr(h), _ptr(xp), _ptr(bp), _ptr(y), int(nthreads))
     if rc != 0:
         raise ValueError(f"m3o_scan rejected its arguments (code {rc})")
+    if z is not None:
+        z = _f64(z, (b, T, H, R, P), "z")
+        _load(lib_path).m3o_gate(y.size, _ptr(z), _ptr(y))
     return y, h, xp, bp
 
 
 def decode_step(x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev,
-                theta_is_angle: bool = False, nthreads: int = 0):
-    """One decode token: x [b,H,R,P], B/C [b,G,R,N], dt/A/lam [b,H], theta [b,G,N/2].
+                theta_is_angle: bool = False, nthreads: int = 0, z=None):
+    """One decode token: x [b,H,R,P], B/C [b,G,R,N], dt/A/lam [b,H], theta [b,G,N/2];
+    z [b,H,R,P] or None (output gate).
 
     Identical to ``scan`` with T = 1; returns (y [b,H,R,P], h, x_prev, B_prev).
     """
     ins = [np.asarray(v)[:, None] for v in (x, B, C, dt, A, lam, theta)]
     y, h, xp, bp = scan(*ins, D=D, h0=h, x_prev=x_prev, B_prev=B_prev,
-                        theta_is_angle=theta_is_angle, nthreads=nthreads)
+                        theta_is_angle=theta_is_angle, nthreads=nthreads,
+                        z=None if z is None else np.asarray(z)[:, None])
     return y[:, 0], h, xp, bp

@@ -26,6 +26,9 @@
  *   the input term is the rank-R sum  sum_r B_t[:,r] x_t[:,r]^T.  The readout is
  *   Y_t = H_t^T C_t (P x R), plus the per-head skip D * x_t.
  *
+ *   Output gate ("Technical Approach", output gating): the readout, skip included,
+ *   is multiplied element-wise by SiLU(z) = z / (1 + exp(-z)); m3o_gate applies it.
+ *
  *   Sequence start ("Parallel representation under SSD"): the unrolling starts
  *   from h_0 = gamma_0 B_0 x_0, i.e. a fresh state has h = 0 and no previous
  *   token (x_{-1} = 0, B_{-1} = 0).  Across calls the previous token (x, B) is
@@ -168,6 +171,12 @@ int m3o_decode(const m3o_dims* d, uint32_t flags, const double* x, const double*
 {
     return m3o_scan(d, 1, flags, x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev, y,
                     nthreads);
+}
+
+/* y[i] <- y[i] * SiLU(z[i]) for n elements: the output gate on the readout (skip included). */
+void m3o_gate(int64_t n, const double* z, double* y)
+{
+    for (int64_t i = 0; i < n; ++i) y[i] *= z[i] / (1.0 + exp(-z[i]));
 }
 
 int m3o_max_threads(void)
