@@ -227,6 +227,30 @@ def time_prefill(w, d, g, st, y, ws, steps, warmup, stream, ws_world):
     return sum(per) / steps, status
 
 
+def time_prefill_gated(w, d, g, z, st, y, ws, steps, warmup, stream):
+    """The same prefill step through m3_scan_fwd_gated (fused output gate y * SiLU(z))."""
+    def run():
+        m3.m3_scan_fwd_gated(d, w.seqlen, w.chunk, g["x"], g["B"], g["C"], g["dt"], g["A"],
+                             g["lam"], g["theta"], g["D"], z, st, y, ws, stream=stream)
+    for _ in range(warmup):
+        m3.m3_state_init(d, st, stream=stream)
+        run()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(steps):
+        m3.m3_state_init(d, st, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        per.append((e0, e1))
+    torch.cuda.synchronize()
+    status = m3.m3_query_status(ws, stream)
+    if status != m3.M3_OK:
+        raise RuntimeError(f"device status {m3.m3_status_string(status)}")
+    return sum(a.elapsed_time(b) for a, b in per) / steps
+
+
 def time_prefill_e2e(w, d, inp, st, ws, steps, stream, dev):
     """Same call through host buffers: pinned H2D of the step's inputs, the call, D2H of y."""
     keys = ("x", "B", "C", "dt", "A", "lam", "theta", "D")
@@ -256,7 +280,7 @@ def time_prefill_e2e(w, d, inp, st, ws, steps, stream, dev):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
-def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS):
+def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False):
     w = inputs.WORKLOADS[name]
     inp = inputs.make_decode_inputs(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
                                     tokens=DECODE_POOL, io_dtype=w.io_dtype,
@@ -268,6 +292,14 @@ def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS):
     y = torch.empty_like(g["x"][0])
     keys = ("x", "B", "C", "dt", "A", "lam", "theta")
     tok = [[g[k][i] for k in keys] for i in range(DECODE_POOL)]
+    z = inputs.make_gate(g["x"].shape, io_dtype=w.io_dtype, seed=seed).to(dev) if gated else None
+
+    def step(t):
+        if gated:
+            m3.m3_decode_step_gated(d, *tok[t % DECODE_POOL], g["D"], z[t % DECODE_POOL], st, y,
+                                    stream=stream)
+        else:
+            m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=stream)
 
     def reset():
         st.h.copy_(g["h0"])
@@ -276,18 +308,18 @@ def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS):
 
     reset()
     for t in range(10):
-        m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=stream)
+        step(t)
     reset()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for t in range(tokens):
-        m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=stream)
+        step(t)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / tokens
     finite = bool(torch.isfinite(st.h).all().item())
-    byts = decode_algorithmic(w)
+    byts = decode_algorithmic(w) + (w.batch * w.nheads * w.rank * w.headdim * 2 if gated else 0)
     return {"tokens_per_s": w.batch / (ms / 1e3), "us_per_step": ms * 1e3,
             "achieved_gbs": byts / (ms / 1e3) / 1e9, "alg_bytes_per_step": byts,
             "state_finite": finite,
@@ -379,7 +411,7 @@ def ours(args):
     }
 
     if args.prefill_only:
-        args.no_decode = args.no_e2e = args.no_cpu = True
+        args.no_decode = args.no_e2e = args.no_cpu = args.no_gate = True
     if not args.no_decode:
         line["decode"] = {}
         for name in (args.decode or DECODES):
@@ -388,6 +420,26 @@ def ours(args):
             r["tokens_per_s"], _ = job_throughput(w_dec_batch(name), r["us_per_step"] / 1e3,
                                                   ws_world)
             line["decode"][name] = r
+
+    if not args.no_gate:
+        # the fused output gate (y * SiLU(z)): the same prefill step plus z read once
+        z = inputs.make_gate(g["x"].shape, io_dtype=w.io_dtype, seed=rank).to(dev)
+        gms = time_prefill_gated(w, d, g, z, st, y, ws, min(args.steps, 20), 3, stream)
+        gval, gms_max = job_throughput(tokens, gms, ws_world)
+        gbytes = byts + z.numel() * z.element_size()
+        line["gated"] = {"prefill": {"tokens_per_s": gval, "ms_per_step": gms_max,
+                                     "alg_bytes_per_step": gbytes,
+                                     "achieved_gbs": gbytes / (gms / 1e3) / 1e9,
+                                     "hbm_frac": gbytes / (gms / 1e3) / 1e9 / pk["hbm_gbs"]}}
+        del z
+        if not args.no_decode:
+            for name in (args.decode or DECODES):
+                r = time_decode(name, dev, stream, seed=100 + rank, tokens=args.decode_tokens,
+                                gated=True)
+                r["hbm_frac"] = r["achieved_gbs"] / pk["hbm_gbs"]
+                r["tokens_per_s"], _ = job_throughput(w_dec_batch(name), r["us_per_step"] / 1e3,
+                                                      ws_world)
+                line["gated"][name] = r
 
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_prefill_e2e(w, d, inp, st, ws, min(args.steps, 5), stream, dev)
@@ -451,6 +503,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-gate", action="store_true", help="skip the fused-output-gate legs")
     ap.add_argument("--cpu-rows", type=int, default=8,
                     help="batch rows of the workload timed on the CPU oracle (default: all)")
     ap.add_argument("--ref-tokens", type=int, default=256)

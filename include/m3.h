@@ -137,6 +137,22 @@ m3_status m3_scan_fwd(const m3_dims* dims, int32_t seqlen, int32_t chunk, const 
                       void* stream);
 
 /*
+ * Prefill with the fused output gate ("Technical Approach", output gating: the readout
+ * y_t, skip included, is multiplied element-wise by SiLU(z_t) = z_t / (1 + e^-z_t)).
+ *
+ *   z: [b][T][H][R][P] in the io dtype (the layout of y), device pointer, 16-byte
+ *      aligned, read only.  NULL returns M3_ERR_NULL (unless seqlen == 0).
+ *
+ * Everything else -- arguments, state update, kernel choice, errors -- is as for
+ * m3_scan_fwd; the gate changes y only, never the state.
+ */
+m3_status m3_scan_fwd_gated(const m3_dims* dims, int32_t seqlen, int32_t chunk, const void* x,
+                            const void* B, const void* C, const float* dt, const float* A,
+                            const float* lam, const float* theta, const float* D,
+                            const void* z, m3_state* state, void* y, void* workspace,
+                            size_t workspace_bytes, uint32_t flags, void* stream);
+
+/*
  * Prefill without a workspace argument, for callers that cannot allocate device
  * memory (for example a plugin inside a host framework whose caching allocator owns
  * all of the device memory, or a serving loop that must not call cudaMalloc because
@@ -179,6 +195,15 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x, const void* B, cons
                          const float* dt, const float* A, const float* lam,
                          const float* theta, const float* D, m3_state* state, void* y,
                          uint32_t flags, void* stream);
+
+/*
+ * Decode step with the fused output gate: y = (h^T C + D x) * SiLU(z), z [b][H][R][P] in
+ * the io dtype, 16-byte aligned, not NULL (M3_ERR_NULL).  Otherwise as m3_decode_step.
+ */
+m3_status m3_decode_step_gated(const m3_dims* dims, const void* x, const void* B, const void* C,
+                               const float* dt, const float* A, const float* lam,
+                               const float* theta, const float* D, const void* z,
+                               m3_state* state, void* y, uint32_t flags, void* stream);
 
 /* Synchronise `stream` and report the device-side status word in `workspace`
  * (M3_OK, or M3_ERR_TIMEOUT when a bounded wait gave up). */

@@ -136,7 +136,9 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     for (int e = tid; e < R * P; e += blockDim.x) {
         float acc = 0.f;
         for (int k = 0; k < RG; ++k) acc += ypart[(size_t)k * R * P + e];
-        y[e] = from_f<IO>(acc + Dh * xs[e]);
+        float v = acc + Dh * xs[e];
+        if (a.z) v = gate_silu(v, to_f(static_cast<const IO*>(a.z)[(size_t)bh * R * P + e]));
+        y[e] = from_f<IO>(v);
         xpo[e] = x[e];   // x_prev <- x (this head only; read above before the barrier)
     }
 }

@@ -140,11 +140,16 @@ m3_status m3_scan_workspace_bytes(const m3_dims* d, int32_t seqlen, int32_t chun
     return M3_OK;
 }
 
-m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
-                      const void* B, const void* C, const float* dt, const float* A,
-                      const float* lam, const float* theta, const float* D, m3_state* state,
-                      void* y, void* workspace, size_t workspace_bytes, uint32_t flags,
-                      void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Prefill with an optional output gate z (null: none); validation happens before any launch.
+m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
+                    const void* B, const void* C, const float* dt, const float* A,
+                    const float* lam, const float* theta, const float* D, const void* z,
+                    m3_state* state, void* y, void* workspace, size_t workspace_bytes,
+                    uint32_t flags, void* stream) {
     m3_status st = check_dims(d);
     if (st != M3_OK) return st;
     if (seqlen < 0) return M3_ERR_SHAPE;
@@ -154,7 +159,7 @@ m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const voi
     if (!x || !B || !C || !dt || !A || !lam || !theta || !y) return M3_ERR_NULL;
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
         !aligned(dt, 4) || !aligned(A, 4) || !aligned(lam, 4) || !aligned(theta, 4) ||
-        (D && !aligned(D, 4)))
+        (D && !aligned(D, 4)) || (z && !aligned(z, 16)))
         return M3_ERR_ALIGN;
     size_t need = 0;
     m3_scan_workspace_bytes(d, seqlen, chunk, &need);
@@ -174,7 +179,7 @@ m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const voi
     ScanArgs a;
     std::memset(&a, 0, sizeof(a));
     a.x = x; a.B = B; a.C = C; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D;
-    a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y;
+    a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y; a.z = z;
     a.status = static_cast<uint32_t*>(workspace);
     a.ws = static_cast<char*>(workspace) + kStatusBytes;
     a.T = seqlen; a.batch = d->batch; a.H = d->nheads; a.G = d->ngroups; a.P = P; a.N = N;
@@ -188,17 +193,18 @@ m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const voi
     return launch_status(e);
 }
 
-m3_status m3_decode_step(const m3_dims* d, const void* x, const void* B, const void* C,
-                         const float* dt, const float* A, const float* lam,
-                         const float* theta, const float* D, m3_state* state, void* y,
-                         uint32_t flags, void* stream) {
+// Decode step with an optional output gate z (null: none).
+m3_status decode_impl(const m3_dims* d, const void* x, const void* B, const void* C,
+                      const float* dt, const float* A, const float* lam, const float* theta,
+                      const float* D, const void* z, m3_state* state, void* y, uint32_t flags,
+                      void* stream) {
     m3_status st = check_dims(d);
     if (st != M3_OK) return st;
     if (!x || !B || !C || !dt || !A || !lam || !theta || !y) return M3_ERR_NULL;
     if ((st = check_state(state)) != M3_OK) return st;
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
         !aligned(dt, 4) || !aligned(A, 4) || !aligned(lam, 4) || !aligned(theta, 4) ||
-        (D && !aligned(D, 4)))
+        (D && !aligned(D, 4)) || (z && !aligned(z, 16)))
         return M3_ERR_ALIGN;
     int ppt = 0;
     if (!rank_has_kernel(d->rank) || !decode_shape(d->dstate, d->headdim, d->rank, &ppt))
@@ -207,7 +213,7 @@ m3_status m3_decode_step(const m3_dims* d, const void* x, const void* B, const v
     DecodeArgs a;
     std::memset(&a, 0, sizeof(a));
     a.x = x; a.B = B; a.C = C; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D;
-    a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y;
+    a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y; a.z = z;
     a.H = d->nheads; a.G = d->ngroups; a.P = d->headdim; a.N = d->dstate;
     a.ppt = ppt; a.flags = flags;
     cudaError_t e = launch_decode(a, d->batch, d->rank, d->io_dtype, s);
@@ -215,6 +221,44 @@ m3_status m3_decode_step(const m3_dims* d, const void* x, const void* B, const v
     const size_t row = io_bytes(d->io_dtype) * (size_t)d->ngroups * d->rank * d->dstate;
     e = launch_copy_prev(state->B_prev, B, 1, 0, d->batch, row, s);
     return launch_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
+                      const void* B, const void* C, const float* dt, const float* A,
+                      const float* lam, const float* theta, const float* D, m3_state* state,
+                      void* y, void* workspace, size_t workspace_bytes, uint32_t flags,
+                      void* stream) {
+    return scan_impl(d, seqlen, chunk, x, B, C, dt, A, lam, theta, D, nullptr, state, y,
+                     workspace, workspace_bytes, flags, stream);
+}
+
+m3_status m3_scan_fwd_gated(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
+                            const void* B, const void* C, const float* dt, const float* A,
+                            const float* lam, const float* theta, const float* D,
+                            const void* z, m3_state* state, void* y, void* workspace,
+                            size_t workspace_bytes, uint32_t flags, void* stream) {
+    if (!z && seqlen != 0) return M3_ERR_NULL;
+    return scan_impl(d, seqlen, chunk, x, B, C, dt, A, lam, theta, D, z, state, y, workspace,
+                     workspace_bytes, flags, stream);
+}
+
+m3_status m3_decode_step(const m3_dims* d, const void* x, const void* B, const void* C,
+                         const float* dt, const float* A, const float* lam,
+                         const float* theta, const float* D, m3_state* state, void* y,
+                         uint32_t flags, void* stream) {
+    return decode_impl(d, x, B, C, dt, A, lam, theta, D, nullptr, state, y, flags, stream);
+}
+
+m3_status m3_decode_step_gated(const m3_dims* d, const void* x, const void* B, const void* C,
+                               const float* dt, const float* A, const float* lam,
+                               const float* theta, const float* D, const void* z,
+                               m3_state* state, void* y, uint32_t flags, void* stream) {
+    if (!z) return M3_ERR_NULL;
+    return decode_impl(d, x, B, C, dt, A, lam, theta, D, z, state, y, flags, stream);
 }
 
 m3_status m3_query_status(const void* workspace, void* stream) {

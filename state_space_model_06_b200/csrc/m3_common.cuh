@@ -23,6 +23,10 @@ __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
 
+// Output gate ("Technical Approach", output gating): the readout v (skip included) times
+// SiLU(z) = z / (1 + e^-z).  A large negative z gives e^-z = inf and a gate of -0.
+__device__ __forceinline__ float gate_silu(float v, float z) { return v * (z / (1.f + expf(-z))); }
+
 // Argument block of one decode step (device pointers, validated on the host).
 struct DecodeArgs {
     const void* x;       // [b][H][R][P] io
@@ -37,6 +41,7 @@ struct DecodeArgs {
     void* x_prev;        // [b][H][R][P] io
     const void* B_prev;  // [b][G][R][N] io (read only here; updated by a follow-up copy)
     void* y;             // [b][H][R][P] io
+    const void* z;       // [b][H][R][P] io: output gate, or null for none
     int H, G, P, N;
     int ppt;             // state pairs per thread
     uint32_t flags;
@@ -56,6 +61,7 @@ struct ScanArgs {
     void* x_prev;        // [b][H][R][P]   in/out
     const void* B_prev;  // [b][G][R][N]   read only here; updated by a follow-up copy
     void* y;             // [b][T][H][R][P] io
+    const void* z;       // [b][T][H][R][P] io: output gate, or null for none
     uint32_t* status;    // workspace status word (may be null)
     void* ws;            // workspace (after the status block)
     long long T;

@@ -130,7 +130,12 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
         if (k == 0) {
             IO* yt = static_cast<IO*>(a.y) + (bt * H + h) * R * P;
 #pragma unroll
-            for (int r = 0; r < R; ++r) yt[r * P + p] = from_f<IO>(yp[r] + Dh * xc[r * P + p]);
+            for (int r = 0; r < R; ++r) {
+                float v = yp[r] + Dh * xc[r * P + p];
+                if (a.z)
+                    v = gate_silu(v, to_f(static_cast<const IO*>(a.z)[(bt * H + h) * R * P + r * P + p]));
+                yt[r * P + p] = from_f<IO>(v);
+            }
         }
     }
 

@@ -106,7 +106,7 @@ __device__ __forceinline__ uint32_t bar_count(int i) {
     }
 }
 
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 struct Cfg {
     static constexpr int L = Q * R;                 // rows of the intra-chunk tiles
     static constexpr int PAIRS = NST / 2;
@@ -131,6 +131,8 @@ struct Cfg {
     }
     static constexpr int raw_bytes(int rt) { return rt * R * NST * 2 * 2 + rt * PAIRS * 4; }
     static constexpr int kSmemLimit = 232448 - 1024;            // minus base alignment slack
+    // with the output gate, every x / y stage has a z tile beside it
+    static constexpr int XZ_BYTES = (GT ? 2 : 1) * X_BYTES;
     // (operand slots, x stages, raw sub-chunk tokens): prefer two operand slots, then three
     // x stages, then the largest raw sub-chunk that fits
     static constexpr int pick() {
@@ -138,7 +140,7 @@ struct Cfg {
             for (int xst = 3; xst >= 2; --xst)
                 for (int rt = (Q < 32 ? Q : 32); rt >= TSPLIT; rt /= 2)
                     if (Q % rt == 0 && rt % TSPLIT == 0 &&
-                        base_bytes() + ops * SLOT_BYTES + xst * X_BYTES + 2 * raw_bytes(rt) <=
+                        base_bytes() + ops * SLOT_BYTES + xst * XZ_BYTES + 2 * raw_bytes(rt) <=
                             kSmemLimit)
                         return ops * 10000 + xst * 1000 + rt;
         return 0;
@@ -156,7 +158,8 @@ struct Cfg {
 
     // shared memory offsets (SW128 tiles first, 1024-byte aligned)
     static constexpr int OFF_X = 0;                                   // [XST] x / y staging
-    static constexpr int OFF_OPS = OFF_X + XST * X_BYTES;             // [OPS] C~, B~, Xw
+    static constexpr int OFF_Z = OFF_X + XST * X_BYTES;               // [XST] z (gate only)
+    static constexpr int OFF_OPS = OFF_X + XST * XZ_BYTES;            // [OPS] C~, B~, Xw
     static constexpr int OFF_SL = OFF_OPS + OPS * SLOT_BYTES;         // S o L
     static constexpr int OFF_G = OFF_SL + SL_BYTES;                   // g (bf16)
     static constexpr int OFF_RAW = OFF_G + G_BYTES;                   // [2] B, C, theta
@@ -193,7 +196,7 @@ struct Cfg {
 };
 
 struct TcParams {
-    CUtensorMap tm_x, tm_y, tm_B, tm_C, tm_th, tm_dt, tm_A, tm_lam;
+    CUtensorMap tm_x, tm_y, tm_z, tm_B, tm_C, tm_th, tm_dt, tm_A, tm_lam;
     ScanArgs a;
     int nchunks;
     unsigned long long limit_ns;
@@ -219,6 +222,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// SiLU(z) = z / (1 + e^-z) for the output gate ("Technical Approach", output gating); the
+// exponent is capped at 2^126 so that the fast division stays in its exact range (the gate
+// is then ~z * 2^-126, i.e. 0 at bf16 precision, for z below about -87).
+__device__ __forceinline__ float silu_fast(float z) {
+    return __fdividef(z, 1.f + ex2_approx(fminf(-z * kLog2e, 126.f)));
+}
+
 // A wait taken by all 32 lanes of a warp together: the outcome is made warp-uniform so
 // that no lane reaches a .sync.aligned tcgen05 instruction without the others.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
@@ -237,15 +247,15 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int k, uint32_t lbo) 
 }
 
 // ---------------------------------------------------------------------------------
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab);
 
 // ---------------------------------------------------------------------------------
 // ---------------------------------------------------------------------------------
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
                            const Abort& ab) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     const uint32_t s_sl = smem_u32(sm + C::OFF_SL), s_g = smem_u32(sm + C::OFF_G);
     // failure-path test hook: wait on a barrier nothing completes (bounded, then abort)
     if ((p.a.flags & M3_FLAG_TEST_STALL) && !mbar_wait(&bar[NEVER], 0, ab)) return;
@@ -310,9 +320,9 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
 // ts = rw / PB.  The starting angle of a thread's token range is the running angle plus
 // the angle sums of the earlier ranges, exchanged through shared memory once per
 // sub-chunk (bounded mbarrier hand-off).
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     constexpr int TPT = C::TPT, PAIRS = C::PAIRS, TSPLIT = C::TSPLIT;
     const ScanArgs& a = p.a;
     const int tid = threadIdx.x - 192;          // 0..255
@@ -484,9 +494,9 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
 
 // Coefficient warp: per-token log2-decay prefix sum (warp scan), gamma, w and the mask
 // exponent offsets ew_u = log2(w_u) - cum2_u of each chunk, into a ring of slots.
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __device__ void coefficients(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
     const int lane = threadIdx.x & 31;
     const int hq = (blockIdx.x % a.H) & 3;
@@ -564,10 +574,10 @@ struct Lanes {
 };
 
 // Epilogue warpgroup (warps 2-5): masks S into the bf16 operand S o L and writes y.
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
                          const Abort& ab) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
     const Lanes<NST, Q, R> ln(tmem);
     const int lane = ln.lane;
@@ -647,6 +657,7 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
         if (!warp_wait(&bar[X_FULL0 + xs], (c / C::XST) & 1, ab)) return;
         tc_fence_after();
         uint8_t* xt = sm + C::OFF_X + xs * C::X_BYTES;
+        const uint8_t* zt = sm + C::OFF_Z + xs * C::X_BYTES;   // z tile (gate only)
         {
             const float sc = exp2f(cum2[lrow / R]);
 #pragma unroll 1
@@ -658,13 +669,23 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
 #pragma unroll
                 for (int j = 0; j < 16; j += 8) {
                     const uint32_t off = sw128_off(lrow, lcol0 + cb + j);
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        v[e] = fmaf(sc, __uint_as_float(yi[j + e]), __uint_as_float(ya[j + e]));
+                    if constexpr (GT) {
+                        // the z tile has the x tile's layout: same swizzled offset
+                        const uint4 zq = *reinterpret_cast<const uint4*>(zt + off);
+                        const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            v[2 * e] *= silu_fast(bf16lo(zw[e]));
+                            v[2 * e + 1] *= silu_fast(bf16hi(zw[e]));
+                        }
+                    }
                     uint32_t o[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        o[e] = pack_bf16x2(
-                            fmaf(sc, __uint_as_float(yi[j + 2 * e]), __uint_as_float(ya[j + 2 * e])),
-                            fmaf(sc, __uint_as_float(yi[j + 2 * e + 1]),
-                                 __uint_as_float(ya[j + 2 * e + 1])));
+                    for (int e = 0; e < 4; ++e) o[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
                     *reinterpret_cast<uint4*>(xt + off) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
@@ -683,10 +704,10 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
 // State warpgroup (warps 16-19): the fp32 carried state g in TMEM columns TM_G..,
 // g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T, per chunk g <- e^{cum_end} g + dS and its
 // bf16 copy for the Y_inter MMA; at the end h_T = R(psi_T) g and the carried x.
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
                       const Abort& ab) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
     const Lanes<NST, Q, R> ln(tmem);
     const int lane = ln.lane;
@@ -826,9 +847,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
     }
 }
 
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
     const int b = blockIdx.x / a.H, h = blockIdx.x % a.H, g = h / (a.H / a.G);
     // loads issued per ring stage, so that an aborted CTA can wait for them to land
@@ -874,17 +895,20 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
 // store nor the store itself holds up the B / C / theta loads.  x(c) is loaded into
 // stage c % XST; once the epilogue has written y(c) over it (Y_STAGED), the tile is
 // stored, and when the store has read it the stage takes x(c + XST).
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
     const int b = blockIdx.x / a.H, h = blockIdx.x % a.H;
     int n_x[C::XST] = {};
     auto load = [&](int c) {
         const int xs = c % C::XST;
-        mbar_arrive_expect_tx(&bar[X_FULL0 + xs], C::X_BYTES);
+        mbar_arrive_expect_tx(&bar[X_FULL0 + xs], C::XZ_BYTES);
         tma_load_5d(sm + C::OFF_X + xs * C::X_BYTES, &p.tm_x, &bar[X_FULL0 + xs], 0, 0, h, c * Q,
                     b);
+        if constexpr (GT)
+            tma_load_5d(sm + C::OFF_Z + xs * C::X_BYTES, &p.tm_z, &bar[X_FULL0 + xs], 0, 0, h,
+                        c * Q, b);
         ++n_x[xs];
     };
     for (int c = 0; c < C::XST && c < p.nchunks; ++c) load(c);
@@ -905,9 +929,9 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
     bulk_wait<0>();
 }
 
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_constant__ TcParams p) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base for the SW128 tiles, as an offset from smem_raw so that the
     // compiler keeps every access in the shared address space
@@ -922,6 +946,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         misc[1] = 0u;  // abort flag
         fence_mbar_init();
         tma_prefetch_desc(&p.tm_x);
+        if (GT) tma_prefetch_desc(&p.tm_z);
         tma_prefetch_desc(&p.tm_B);
         tma_prefetch_desc(&p.tm_C);
         tma_prefetch_desc(&p.tm_th);
@@ -938,24 +963,24 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.a.status, p.limit_ns};
 
     if (w == 0) {
-        if ((threadIdx.x & 31) == 0) producer<NST, Q, R>(p, sm, bar, ab);
+        if ((threadIdx.x & 31) == 0) producer<NST, Q, R, GT>(p, sm, bar, ab);
     } else if (w == 1) {
         if ((threadIdx.x & 31) == 0) {
-            mma_issuer<NST, Q, R>(p, sm, bar, tmem, ab);
+            mma_issuer<NST, Q, R, GT>(p, sm, bar, tmem, ab);
             // no MMA may still be writing TMEM when it is released
             mma_commit(&bar[DRAIN]);
             drain_wait(&bar[DRAIN], 0, 100000000ull);
         }
     } else if (w < 6) {
-        epilogue<NST, Q, R>(p, sm, bar, tmem, ab);
+        epilogue<NST, Q, R, GT>(p, sm, bar, tmem, ab);
     } else if (w >= 16) {
-        state<NST, Q, R>(p, sm, bar, tmem, ab);
+        state<NST, Q, R, GT>(p, sm, bar, tmem, ab);
     } else if (w < 6 + kRotWarps) {
-        rotation<NST, Q, R>(p, sm, bar, ab);
+        rotation<NST, Q, R, GT>(p, sm, bar, ab);
     } else if (w == 6 + kRotWarps) {
-        coefficients<NST, Q, R>(p, sm, bar, ab);
+        coefficients<NST, Q, R, GT>(p, sm, bar, ab);
     } else if ((threadIdx.x & 31) == 0) {
-        x_producer<NST, Q, R>(p, sm, bar, ab);
+        x_producer<NST, Q, R, GT>(p, sm, bar, ab);
     }
     tc_fence_before();
     __syncthreads();
@@ -1001,9 +1026,9 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ptr,
     return r == CUDA_SUCCESS;
 }
 
-template <int NST, int Q, int R>
+template <int NST, int Q, int R, bool GT>
 cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
-    using C = Cfg<NST, Q, R>;
+    using C = Cfg<NST, Q, R, GT>;
     TcParams p;
     std::memset(&p, 0, sizeof(p));
     p.a = a;
@@ -1019,6 +1044,9 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_128B);
         ok &= make_map(&p.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.y, d, st, box,
                        CU_TENSOR_MAP_SWIZZLE_128B);
+        if (GT)
+            ok &= make_map(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.z, d, st, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
     }
     {   // B, C: (N, R, G, T, b), box (N, R, 1, RT, 1)
         const uint64_t d[5] = {NST, R, G, T, Bn};
@@ -1049,10 +1077,10 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R>,
+    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R, GT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<NST, Q, R><<<(unsigned)(a.batch * a.H), kThreads, C::SMEM, s>>>(p);
+    scan_tc_kernel<NST, Q, R, GT><<<(unsigned)(a.batch * a.H), kThreads, C::SMEM, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -1081,21 +1109,27 @@ int scan_tc_chunk(int N, int P, int R, int chunk, int H) {
 
 size_t scan_tc_workspace_bytes(int, int, int, int, int, long long, int) { return 0; }
 
-cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s) {
+template <bool GT>
+cudaError_t launch_scan_tc_g(const ScanArgs& a, int R, cudaStream_t s) {
     const int N = a.N, Q = a.chunk;   // the tile chunk chosen by scan_tc_chunk
     if (R == 1) {
-        if (N == 128 && Q == 64) return launch_t<128, 64, 1>(a, s);
-        if (N == 128 && Q == 128) return launch_t<128, 128, 1>(a, s);
-        if (N == 64 && Q == 64) return launch_t<64, 64, 1>(a, s);
-        if (N == 64 && Q == 128) return launch_t<64, 128, 1>(a, s);
+        if (N == 128 && Q == 64) return launch_t<128, 64, 1, GT>(a, s);
+        if (N == 128 && Q == 128) return launch_t<128, 128, 1, GT>(a, s);
+        if (N == 64 && Q == 64) return launch_t<64, 64, 1, GT>(a, s);
+        if (N == 64 && Q == 128) return launch_t<64, 128, 1, GT>(a, s);
     } else if (R == 2 && N == 64) {
-        if (Q == 32) return launch_t<64, 32, 2>(a, s);
-        if (Q == 64) return launch_t<64, 64, 2>(a, s);
+        if (Q == 32) return launch_t<64, 32, 2, GT>(a, s);
+        if (Q == 64) return launch_t<64, 64, 2, GT>(a, s);
     } else if (R == 4 && N == 64) {
-        if (Q == 16) return launch_t<64, 16, 4>(a, s);
-        if (Q == 32) return launch_t<64, 32, 4>(a, s);
+        if (Q == 16) return launch_t<64, 16, 4, GT>(a, s);
+        if (Q == 32) return launch_t<64, 32, 4, GT>(a, s);
     }
     return cudaErrorNotSupported;
+}
+
+// a.z selects the instantiation with the fused output gate
+cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s) {
+    return a.z ? launch_scan_tc_g<true>(a, R, s) : launch_scan_tc_g<false>(a, R, s);
 }
 
 }  // namespace m3

@@ -106,6 +106,14 @@ def make_scan_inputs(batch, seqlen, nheads, ngroups, headdim, dstate, rank=1,
     return inp
 
 
+def make_gate(shape, io_dtype=torch.bfloat16, seed=0):
+    """Output-gate input z ~ N(0, 1) of the given shape (the layout of y), rounded to the io
+    dtype.  Drawn from its own generator (seed + 7919) so that adding a gate never changes
+    the other inputs of a seeded workload."""
+    g = torch.Generator("cpu").manual_seed(seed + 7919)
+    return _randn(g, tuple(shape), dtype=io_dtype)
+
+
 def make_decode_inputs(batch, nheads, ngroups, headdim, dstate, rank=1, tokens=1,
                        io_dtype=torch.bfloat16, theta_max=math.pi / 8, seed=0):
     """Per-token decode inputs stacked over ``tokens`` plus the starting state.

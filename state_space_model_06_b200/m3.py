@@ -25,7 +25,8 @@ M3_FLAG_FORCE_SIMT = 2
 M3_FLAG_TEST_STALL = 4
 
 EXPORTED = ("m3_state_bytes", "m3_state_init", "m3_scan_workspace_bytes", "m3_scan_fwd",
-            "m3_decode_step", "m3_query_status", "m3_scan_fwd_noalloc", "m3_status_string")
+            "m3_decode_step", "m3_query_status", "m3_scan_fwd_noalloc", "m3_scan_fwd_gated",
+            "m3_decode_step_gated", "m3_status_string")
 
 
 class M3Error(RuntimeError):
@@ -65,6 +66,10 @@ def load_library(path: str = LIB_PATH):
         lib.m3_scan_fwd.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp, vp, sz,
                                     u32, vp]
         lib.m3_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp, u32, vp]
+        lib.m3_scan_fwd_gated.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sp,
+                                          vp, vp, sz, u32, vp]
+        lib.m3_decode_step_gated.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp,
+                                             u32, vp]
         lib.m3_scan_fwd_noalloc.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp,
                                             u32, vp]
         lib.m3_query_status.argtypes = [vp, vp]
@@ -180,6 +185,27 @@ def m3_scan_fwd_noalloc(dims: Dims, seqlen: int, chunk: int, x, B, C, dt, A, lam
         ctypes.byref(dims.c()), int(seqlen), int(chunk), _ptr(x), _ptr(B), _ptr(C), _ptr(dt),
         _ptr(A), _ptr(lam), _ptr(theta), _ptr(D), ctypes.byref(st), _ptr(y), int(flags),
         _stream(stream)), "m3_scan_fwd_noalloc")
+
+
+def m3_scan_fwd_gated(dims: Dims, seqlen: int, chunk: int, x, B, C, dt, A, lam, theta, D, z,
+                      state: State, y, workspace, flags: int = 0, stream=None):
+    """Prefill with the fused output gate y * SiLU(z) (z in the layout and dtype of y)."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = state.c()
+    _check(load_library().m3_scan_fwd_gated(
+        ctypes.byref(dims.c()), int(seqlen), int(chunk), _ptr(x), _ptr(B), _ptr(C), _ptr(dt),
+        _ptr(A), _ptr(lam), _ptr(theta), _ptr(D), _ptr(z), ctypes.byref(st), _ptr(y),
+        _ptr(workspace), ws_bytes, int(flags), _stream(stream)), "m3_scan_fwd_gated")
+
+
+def m3_decode_step_gated(dims: Dims, x, B, C, dt, A, lam, theta, D, z, state: State, y,
+                         flags: int = 0, stream=None):
+    """Decode step with the fused output gate y * SiLU(z)."""
+    st = state.c()
+    _check(load_library().m3_decode_step_gated(
+        ctypes.byref(dims.c()), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam),
+        _ptr(theta), _ptr(D), _ptr(z), ctypes.byref(st), _ptr(y), int(flags), _stream(stream)),
+        "m3_decode_step_gated")
 
 
 def m3_decode_step(dims: Dims, x, B, C, dt, A, lam, theta, D, state: State, y, flags: int = 0,

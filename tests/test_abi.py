@@ -102,6 +102,28 @@ def test_decode_validation_before_launch(lib):
                               p, 0, None) == m3.M3_ERR_UNSUPPORTED
 
 
+def test_gated_validation_before_launch(lib):
+    """The gated entry points check z (present, 16-byte aligned) before anything else runs."""
+    d = m3.Dims(1, 2, 1, 16, 16, 1, m3.M3_BF16)
+    st = m3.m3_state(0x2000, 0x3000, 0x4000)
+    p, ws = 0x1000, 0x100000
+
+    def scan(z, T=16):
+        return lib.m3_scan_fwd_gated(ctypes.byref(d.c()), T, 64, p, p, p, p, p, p, p, None, z,
+                                     ctypes.byref(st), p, ws, 1 << 20, 0, None)
+
+    assert scan(None) == m3.M3_ERR_NULL
+    assert scan(p + 8) == m3.M3_ERR_ALIGN
+    assert scan(None, T=0) == m3.M3_OK        # seqlen 0: a validated no-op
+
+    def dec(z):
+        return lib.m3_decode_step_gated(ctypes.byref(d.c()), p, p, p, p, p, p, p, None, z,
+                                        ctypes.byref(st), p, 0, None)
+
+    assert dec(None) == m3.M3_ERR_NULL
+    assert dec(p + 4) == m3.M3_ERR_ALIGN
+
+
 def test_binding_refuses_missing_library(tmp_path):
     old = m3._lib
     m3._lib = None
