@@ -59,6 +59,9 @@ def _load(path=None):
         lib.m3o_scan.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int64, ctypes.c_uint32] + \
             [dp] * 12 + [ctypes.c_int]
         lib.m3o_scan.restype = ctypes.c_int
+        lib.m3o_scan_ex.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int64, ctypes.c_uint32] + \
+            [dp] * 10 + [ctypes.c_double] + [dp] * 4 + [ctypes.c_int]
+        lib.m3o_scan_ex.restype = ctypes.c_int
         lib.m3o_max_threads.restype = ctypes.c_int
         lib.m3o_gate.argtypes = [ctypes.c_int64, dp, dp]
         lib.m3o_gate.restype = None
@@ -82,7 +85,8 @@ def _ptr(a):
 
 
 def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
-         theta_is_angle: bool = False, nthreads: int = 0, lib_path=None, z=None):
+         theta_is_angle: bool = False, nthreads: int = 0, lib_path=None, z=None,
+         B_bias=None, C_bias=None, bc_eps: float = 0.0):
     """Run the recurrence over T tokens.
 
     Shapes: x [b,T,H,R,P]; B, C [b,T,G,R,N]; dt, A, lam [b,T,H];
@@ -90,6 +94,9 @@ def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
     x_prev [b,H,R,P] / B_prev [b,G,R,N] or None (fresh sequence: zeros);
     z [b,T,H,R,P] or None: output gate, y <- y * SiLU(z) after the skip
     ("Technical Approach", output gating).
+    B_bias, C_bias [H,N] or None and bc_eps > 0: BC biases and BC normalisation
+    ("Technical Approach", BCNorm and BC biases): per token, each rank column of B and
+    C is scaled to unit RMS over N (when bc_eps > 0), then the head's bias is added.
 
     Returns (y [b,T,H,R,P], h_T, x_prev_out, B_prev_out), all float64.
     """
@@ -109,9 +116,18 @@ def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
     bp = np.zeros((b, G, R, N)) if B_prev is None else _f64(B_prev, (b, G, R, N), "B_prev").copy()
     y = np.zeros((b, T, H, R, P))
     dims = _Dims(b, H, G, P, N, R)
-    rc = _load(lib_path).m3o_scan(ctypes.byref(dims), T, THETA_IS_ANGLE if theta_is_angle else 0,
-                          _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta),
-                          _ptr(D), _ptr(h), _ptr(xp), _ptr(bp), _ptr(y), int(nthreads))
+    fl = THETA_IS_ANGLE if theta_is_angle else 0
+    if B_bias is None and C_bias is None and bc_eps <= 0.0:
+        rc = _load(lib_path).m3o_scan(ctypes.byref(dims), T, fl, _ptr(x), _ptr(B), _ptr(C),
+                                      _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta), _ptr(D),
+                                      _ptr(h), _ptr(xp), _ptr(bp), _ptr(y), int(nthreads))
+    else:
+        bb = None if B_bias is None else _f64(B_bias, (H, N), "B_bias")
+        cb = None if C_bias is None else _f64(C_bias, (H, N), "C_bias")
+        rc = _load(lib_path).m3o_scan_ex(ctypes.byref(dims), T, fl, _ptr(x), _ptr(B), _ptr(C),
+                                         _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta), _ptr(D),
+                                         _ptr(bb), _ptr(cb), float(bc_eps), _ptr(h), _ptr(xp),
+                                         _ptr(bp), _ptr(y), int(nthreads))
     if rc != 0:
         raise ValueError(f"m3o_scan rejected its arguments (code {rc})")
     if z is not None:
@@ -121,7 +137,8 @@ def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
 
 
 def decode_step(x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev,
-                theta_is_angle: bool = False, nthreads: int = 0, z=None):
+                theta_is_angle: bool = False, nthreads: int = 0, z=None, B_bias=None,
+                C_bias=None, bc_eps: float = 0.0):
     """One decode token: x [b,H,R,P], B/C [b,G,R,N], dt/A/lam [b,H], theta [b,G,N/2];
     z [b,H,R,P] or None (output gate).
 
@@ -130,5 +147,6 @@ def decode_step(x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev,
     ins = [np.asarray(v)[:, None] for v in (x, B, C, dt, A, lam, theta)]
     y, h, xp, bp = scan(*ins, D=D, h0=h, x_prev=x_prev, B_prev=B_prev,
                         theta_is_angle=theta_is_angle, nthreads=nthreads,
-                        z=None if z is None else np.asarray(z)[:, None])
+                        z=None if z is None else np.asarray(z)[:, None], B_bias=B_bias,
+                        C_bias=C_bias, bc_eps=bc_eps)
     return y[:, 0], h, xp, bp

@@ -29,6 +29,12 @@
  *   Output gate ("Technical Approach", output gating): the readout, skip included,
  *   is multiplied element-wise by SiLU(z) = z / (1 + exp(-z)); m3o_gate applies it.
  *
+ *   BC normalisation and BC biases ("Technical Approach", BCNorm and BC biases), in
+ *   m3o_scan_ex: each token's B and C column (one per rank r, length N) is scaled to
+ *   unit RMS, B / sqrt(mean_n B^2 + eps), then the head's bias vector (one value per
+ *   state channel n, shared by the rank columns) is added.  The carried previous
+ *   token's B is kept raw in the state and goes through the same map when used.
+ *
  *   Sequence start ("Parallel representation under SSD"): the unrolling starts
  *   from h_0 = gamma_0 B_0 x_0, i.e. a fresh state has h = 0 and no previous
  *   token (x_{-1} = 0, B_{-1} = 0).  Across calls the previous token (x, B) is
@@ -109,6 +115,23 @@ static void m3o_step(int N, int P, int R, double dt, double a, double lam,
     memcpy(bp, Bt, sizeof(double) * (size_t)R * N);
 }
 
+/* Effective B or C column set of one head: out[r][n] = norm(in[r][:])[n] + bias[n], where
+ * norm scales the column to unit RMS (eps > 0) or leaves it (eps <= 0); bias may be NULL. */
+static void m3o_bc_map(int N, int R, const double* in, const double* bias, double eps,
+                       double* out)
+{
+    for (int r = 0; r < R; ++r) {
+        double scale = 1.0;
+        if (eps > 0.0) {
+            double ss = 0.0;
+            for (int n = 0; n < N; ++n) ss += in[r * N + n] * in[r * N + n];
+            scale = 1.0 / sqrt(ss / N + eps);
+        }
+        for (int n = 0; n < N; ++n)
+            out[r * N + n] = in[r * N + n] * scale + (bias ? bias[n] : 0.0);
+    }
+}
+
 static int m3o_check(const m3o_dims* d, int64_t T)
 {
     if (!d) return 1;
@@ -123,12 +146,14 @@ static int m3o_check(const m3o_dims* d, int64_t T)
 /*
  * Run T tokens of the recurrence for every (batch, head).  The state (h, x_prev,
  * B_prev) is updated in place.  Returns 0 on success, non-zero on bad arguments.
- * nthreads <= 0 uses the OpenMP default.
+ * nthreads <= 0 uses the OpenMP default.  B_bias / C_bias [H][N] may be NULL; bc_eps > 0
+ * turns on the BC normalisation (see the header).
  */
-int m3o_scan(const m3o_dims* d, int64_t T, uint32_t flags, const double* x,
-             const double* B, const double* C, const double* dt, const double* A,
-             const double* lam, const double* theta, const double* D, double* h,
-             double* x_prev, double* B_prev, double* y, int nthreads)
+int m3o_scan_ex(const m3o_dims* d, int64_t T, uint32_t flags, const double* x,
+                const double* B, const double* C, const double* dt, const double* A,
+                const double* lam, const double* theta, const double* D, const double* B_bias,
+                const double* C_bias, double bc_eps, double* h, double* x_prev,
+                double* B_prev, double* y, int nthreads)
 {
     int rc = m3o_check(d, T);
     if (rc) return rc;
@@ -142,25 +167,41 @@ int m3o_scan(const m3o_dims* d, int64_t T, uint32_t flags, const double* x,
 #endif
     for (int64_t bh = 0; bh < (int64_t)Bn * H; ++bh) {
         const int b = (int)(bh / H), hh = (int)(bh % H), g = hh / hpg;
+        const double* bb = B_bias ? B_bias + (size_t)hh * N : NULL;
+        const double* cb = C_bias ? C_bias + (size_t)hh * N : NULL;
         double* bp = (double*)malloc(sizeof(double) * (size_t)R * N);
-        memcpy(bp, B_prev + ((size_t)b * G + g) * R * N, sizeof(double) * (size_t)R * N);
+        double* Bh = (double*)malloc(sizeof(double) * (size_t)R * N);
+        double* Ch = (double*)malloc(sizeof(double) * (size_t)R * N);
+        m3o_bc_map(N, R, B_prev + ((size_t)b * G + g) * R * N, bb, bc_eps, bp);
         double* xp = x_prev + ((size_t)b * H + hh) * R * P;
         double* hs = h + ((size_t)b * H + hh) * N * P;
         const double Dh = D ? D[hh] : 0.0;
         for (int64_t t = 0; t < T; ++t) {
             const size_t bt = (size_t)b * T + t;
+            m3o_bc_map(N, R, B + (bt * G + g) * R * N, bb, bc_eps, Bh);
+            m3o_bc_map(N, R, C + (bt * G + g) * R * N, cb, bc_eps, Ch);
             m3o_step(N, P, R, dt[bt * H + hh], A[bt * H + hh], lam[bt * H + hh],
-                     theta + (bt * G + g) * (N / 2), x + (bt * H + hh) * R * P,
-                     B + (bt * G + g) * R * N, C + (bt * G + g) * R * N, Dh, hs, xp, bp,
-                     y + (bt * H + hh) * R * P, flags);
+                     theta + (bt * G + g) * (N / 2), x + (bt * H + hh) * R * P, Bh, Ch, Dh, hs,
+                     xp, bp, y + (bt * H + hh) * R * P, flags);
         }
         free(bp);
+        free(Bh);
+        free(Ch);
     }
     /* B_prev <- B_{T-1}, once per group (every head of the group read the old value) */
     for (int b = 0; b < Bn; ++b)
         memcpy(B_prev + (size_t)b * G * R * N, B + ((size_t)b * T + (T - 1)) * G * R * N,
                sizeof(double) * (size_t)G * R * N);
     return 0;
+}
+
+int m3o_scan(const m3o_dims* d, int64_t T, uint32_t flags, const double* x,
+             const double* B, const double* C, const double* dt, const double* A,
+             const double* lam, const double* theta, const double* D, double* h,
+             double* x_prev, double* B_prev, double* y, int nthreads)
+{
+    return m3o_scan_ex(d, T, flags, x, B, C, dt, A, lam, theta, D, NULL, NULL, 0.0, h, x_prev,
+                       B_prev, y, nthreads);
 }
 
 /* A single decode step is the same recurrence for one token (T = 1). */
