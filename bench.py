@@ -38,6 +38,7 @@ WORKLOAD = "siso_prefill_1p5b"
 DECODES = ("decode_siso_b256", "decode_mimo_b256")
 DECODE_TOKENS = 1000
 DECODE_POOL = 32            # distinct pre-generated tokens, cycled over the 1000 steps
+BC_EPS = 1e-6              # BCNorm epsilon of the BC legs
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -227,11 +228,11 @@ def time_prefill(w, d, g, st, y, ws, steps, warmup, stream, ws_world):
     return sum(per) / steps, status
 
 
-def time_prefill_gated(w, d, g, z, st, y, ws, steps, warmup, stream):
-    """The same prefill step through m3_scan_fwd_gated (fused output gate y * SiLU(z))."""
+def time_prefill_ex(w, d, g, ex, st, y, ws, steps, warmup, stream):
+    """The same prefill step through m3_scan_fwd_ex with the fused parts in ``ex``."""
     def run():
-        m3.m3_scan_fwd_gated(d, w.seqlen, w.chunk, g["x"], g["B"], g["C"], g["dt"], g["A"],
-                             g["lam"], g["theta"], g["D"], z, st, y, ws, stream=stream)
+        m3.m3_scan_fwd_ex(d, w.seqlen, w.chunk, g["x"], g["B"], g["C"], g["dt"], g["A"],
+                          g["lam"], g["theta"], g["D"], ex, st, y, ws, stream=stream)
     for _ in range(warmup):
         m3.m3_state_init(d, st, stream=stream)
         run()
@@ -280,7 +281,7 @@ def time_prefill_e2e(w, d, inp, st, ws, steps, stream, dev):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
-def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False):
+def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False, bc=False):
     w = inputs.WORKLOADS[name]
     inp = inputs.make_decode_inputs(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
                                     tokens=DECODE_POOL, io_dtype=w.io_dtype,
@@ -293,13 +294,18 @@ def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False):
     keys = ("x", "B", "C", "dt", "A", "lam", "theta")
     tok = [[g[k][i] for k in keys] for i in range(DECODE_POOL)]
     z = inputs.make_gate(g["x"].shape, io_dtype=w.io_dtype, seed=seed).to(dev) if gated else None
+    bias = [v.to(dev) for v in inputs.make_bc_bias(w.nheads, w.dstate, seed=seed)] if bc else None
 
-    def step(t):
-        if gated:
+    def step(t):   # on the current stream: the capture stream while the graph is recorded
+        if bc:
+            ex = m3.Extras(z=None if z is None else z[t % DECODE_POOL], B_bias=bias[0],
+                           C_bias=bias[1], bc_norm_eps=BC_EPS)
+            m3.m3_decode_step_ex(d, *tok[t % DECODE_POOL], g["D"], ex, st, y, stream=None)
+        elif gated:
             m3.m3_decode_step_gated(d, *tok[t % DECODE_POOL], g["D"], z[t % DECODE_POOL], st, y,
-                                    stream=stream)
+                                    stream=None)
         else:
-            m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=stream)
+            m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=None)
 
     def reset():
         st.h.copy_(g["h0"])
@@ -309,15 +315,32 @@ def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False):
     reset()
     for t in range(10):
         step(t)
+    torch.cuda.synchronize()
+    # The DECODE_POOL sequential steps are captured once as a CUDA graph and the graph is
+    # replayed: a step takes ~0.2 ms of device time, about what a host launch through
+    # ctypes takes, so launching steps one by one would time the host.  The state carries
+    # over from replay to replay exactly as in a plain loop over the cycled tokens.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for t in range(DECODE_POOL):
+            step(t)
+    reps = max(1, -(-tokens // DECODE_POOL))
+    reset()
+    graph.replay()                      # warm-up replay
     reset()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for t in range(tokens):
-        step(t)
-    e1.record(stream)
+    cur = torch.cuda.current_stream()
+    e0.record(cur)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(cur)
     torch.cuda.synchronize()
+    tokens = reps * DECODE_POOL
     ms = e0.elapsed_time(e1) / tokens
+    del graph
+    if torch.equal(st.h, g["h0"]):
+        raise RuntimeError("decode graph replays left the state unchanged")
     finite = bool(torch.isfinite(st.h).all().item())
     byts = decode_algorithmic(w) + (w.batch * w.nheads * w.rank * w.headdim * 2 if gated else 0)
     return {"tokens_per_s": w.batch / (ms / 1e3), "us_per_step": ms * 1e3,
@@ -424,7 +447,7 @@ def ours(args):
     if not args.no_gate:
         # the fused output gate (y * SiLU(z)): the same prefill step plus z read once
         z = inputs.make_gate(g["x"].shape, io_dtype=w.io_dtype, seed=rank).to(dev)
-        gms = time_prefill_gated(w, d, g, z, st, y, ws, min(args.steps, 20), 3, stream)
+        gms = time_prefill_ex(w, d, g, m3.Extras(z=z), st, y, ws, min(args.steps, 20), 3, stream)
         gval, gms_max = job_throughput(tokens, gms, ws_world)
         gbytes = byts + z.numel() * z.element_size()
         line["gated"] = {"prefill": {"tokens_per_s": gval, "ms_per_step": gms_max,
@@ -440,6 +463,29 @@ def ours(args):
                 r["tokens_per_s"], _ = job_throughput(w_dec_batch(name), r["us_per_step"] / 1e3,
                                                       ws_world)
                 line["gated"][name] = r
+
+    if not args.no_gate:
+        # BCNorm + BC biases (and everything fused at once: norm, biases and the gate)
+        bb, cb = (v.to(dev) for v in inputs.make_bc_bias(w.nheads, w.dstate, seed=rank))
+        line["bc"] = {}
+        zfull = inputs.make_gate(g["x"].shape, io_dtype=w.io_dtype, seed=rank).to(dev)
+        for key, ex in (("prefill", m3.Extras(B_bias=bb, C_bias=cb, bc_norm_eps=BC_EPS)),
+                        ("prefill_all", m3.Extras(z=zfull, B_bias=bb, C_bias=cb,
+                                                  bc_norm_eps=BC_EPS))):
+            wsx = m3.alloc_workspace_ex(d, w.seqlen, w.chunk, ex, dev)
+            bms = time_prefill_ex(w, d, g, ex, st, y, wsx, min(args.steps, 20), 3, stream)
+            bval, bms_max = job_throughput(tokens, bms, ws_world)
+            line["bc"][key] = {"tokens_per_s": bval, "ms_per_step": bms_max}
+            del wsx
+        del zfull
+        if not args.no_decode:
+            for name in (args.decode or DECODES):
+                r = time_decode(name, dev, stream, seed=100 + rank, tokens=args.decode_tokens,
+                                bc=True)
+                r["hbm_frac"] = r["achieved_gbs"] / pk["hbm_gbs"]
+                r["tokens_per_s"], _ = job_throughput(w_dec_batch(name), r["us_per_step"] / 1e3,
+                                                      ws_world)
+                line["bc"][name] = r
 
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_prefill_e2e(w, d, inp, st, ws, min(args.steps, 5), stream, dev)

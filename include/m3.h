@@ -101,11 +101,38 @@ m3_status m3_state_bytes(const m3_dims* dims, size_t* h_bytes, size_t* x_prev_by
  * under SSD").  h0, when given, is a device pointer in the state.h layout. */
 m3_status m3_state_init(const m3_dims* dims, m3_state* state, const float* h0, void* stream);
 
+/*
+ * Optional parts of the Mamba-3 block fused into the recurrence kernels; a NULL
+ * m3_extras* (or an all-zero one) means none of them.
+ *
+ *   z           output gate ("Technical Approach", output gating): y <- y * SiLU(z) after
+ *               the skip.  Layout and io dtype of y, 16-byte aligned; NULL: no gate.
+ *   B_bias,     BC biases ("Technical Approach", BC biases): head-specific, channel-wise,
+ *   C_bias      [H][N] fp32, added to every rank column of B (and of the carried B_prev)
+ *               and of C; NULL: no bias.
+ *   bc_norm_eps BCNorm ("Technical Approach", BC normalisation): > 0 scales each token's
+ *               B and C rank columns (and B_prev's) to unit RMS over N before the bias,
+ *               v / sqrt(mean_n v^2 + eps); 0: off; negative or NaN: M3_ERR_SHAPE.
+ *
+ * The state keeps the raw previous-token B; the map is applied wherever it is used.
+ */
+typedef struct {
+    const void* z;
+    const float* B_bias;
+    const float* C_bias;
+    float bc_norm_eps;
+} m3_extras;
+
 /* Workspace bytes m3_scan_fwd needs for (dims, seqlen, chunk); at least 256
  * (the status word).  The workspace is caller-owned device memory, 256-byte
  * aligned, and must not be shared by calls that can overlap on the GPU. */
 m3_status m3_scan_workspace_bytes(const m3_dims* dims, int32_t seqlen, int32_t chunk,
                                   size_t* bytes);
+
+/* Workspace bytes of m3_scan_fwd_ex with these extras: the above plus, when BCNorm is on,
+ * one float per B, C and B_prev rank column of the call (its scales). */
+m3_status m3_scan_workspace_bytes_ex(const m3_dims* dims, int32_t seqlen, int32_t chunk,
+                                     const m3_extras* extras, size_t* bytes);
 
 /*
  * Prefill: run `seqlen` tokens of the recurrence for every (batch, head),
@@ -135,6 +162,17 @@ m3_status m3_scan_fwd(const m3_dims* dims, int32_t seqlen, int32_t chunk, const 
                       const float* lam, const float* theta, const float* D, m3_state* state,
                       void* y, void* workspace, size_t workspace_bytes, uint32_t flags,
                       void* stream);
+
+/*
+ * Prefill with the optional fused parts of m3_extras (extras may be NULL).  With BCNorm
+ * the call first launches a small kernel for the column scales (workspace, see
+ * m3_scan_workspace_bytes_ex).  Everything else is as for m3_scan_fwd.
+ */
+m3_status m3_scan_fwd_ex(const m3_dims* dims, int32_t seqlen, int32_t chunk, const void* x,
+                         const void* B, const void* C, const float* dt, const float* A,
+                         const float* lam, const float* theta, const float* D,
+                         const m3_extras* extras, m3_state* state, void* y, void* workspace,
+                         size_t workspace_bytes, uint32_t flags, void* stream);
 
 /*
  * Prefill with the fused output gate ("Technical Approach", output gating: the readout
@@ -195,6 +233,13 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x, const void* B, cons
                          const float* dt, const float* A, const float* lam,
                          const float* theta, const float* D, m3_state* state, void* y,
                          uint32_t flags, void* stream);
+
+/* Decode step with the optional fused parts of m3_extras (z [b][H][R][P]); BCNorm scales
+ * are computed inside the kernel.  Otherwise as m3_decode_step. */
+m3_status m3_decode_step_ex(const m3_dims* dims, const void* x, const void* B, const void* C,
+                            const float* dt, const float* A, const float* lam,
+                            const float* theta, const float* D, const m3_extras* extras,
+                            m3_state* state, void* y, uint32_t flags, void* stream);
 
 /*
  * Decode step with the fused output gate: y = (h^T C + D x) * SiLU(z), z [b][H][R][P] in

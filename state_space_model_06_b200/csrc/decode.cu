@@ -21,7 +21,8 @@ namespace m3 {
 
 // MAXP: the largest pairs-per-thread count this instantiation handles (a.ppt <= MAXP); it
 // sizes the per-thread state registers, so each shape only pays for the pairs it uses.
-template <typename IO, int R, int MAXP>
+// BCM: the instantiation with the BC map (BCNorm and BC biases) of m3_decode_step_ex.
+template <typename IO, int R, int MAXP, bool BCM>
 __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     extern __shared__ float sm[];
     const int N = a.N, P = a.P, H = a.H, G = a.G;
@@ -40,6 +41,7 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     float* cs = Cs + R * N;          // [N/2]
     float* sn = cs + N / 2;          // [N/2]
     float* ypart = sn + N / 2;       // [RG][R][P]
+    float* bcs = ypart + RG * R * P; // [3][R] BCNorm scales of B, B_prev, C
 
     // 1. issue the state loads first: they are the whole cost of the step
     float4* hrow = reinterpret_cast<float4*>(a.h + (size_t)bh * N * P);
@@ -79,6 +81,32 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
         sn[i] = s;
     }
     __syncthreads();
+
+    // BC map ("Technical Approach", BCNorm and BC biases): each rank column of B, B_prev
+    // and C scaled to unit RMS over N (when bc_eps > 0), plus the head's channel bias
+    if constexpr (BCM) {
+        // one thread per column (3R <= 24 columns of N <= 256): a plain serial sum
+        for (int c = tid; c < 3 * R; c += blockDim.x) {      // column c: B r, B_prev r, C r
+            float sc = 1.f;
+            if (a.bc_eps > 0.f) {
+                const float* v = (c < R ? Bs : (c < 2 * R ? Bps : Cs)) + (c % R) * N;
+                float ss = 0.f;
+                for (int n = 0; n < N; ++n) ss = fmaf(v[n], v[n], ss);
+                sc = rsqrtf(ss / (float)N + a.bc_eps);
+            }
+            bcs[c] = sc;
+        }
+        __syncthreads();
+        const float* Bb = a.B_bias ? a.B_bias + (size_t)h * N : nullptr;
+        const float* Cb = a.C_bias ? a.C_bias + (size_t)h * N : nullptr;
+        for (int e = tid; e < R * N; e += blockDim.x) {
+            const int r = e / N, n = e - r * N;
+            Bs[e] = bc_apply(Bs[e], bcs[r], Bb, n);
+            Bps[e] = bc_apply(Bps[e], bcs[R + r], Bb, n);
+            Cs[e] = bc_apply(Cs[e], bcs[2 * R + r], Cb, n);
+        }
+        __syncthreads();
+    }
 
     const float alpha = expf(dt * Av);
     const float beta = (1.f - lam) * dt * alpha;
@@ -143,37 +171,42 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     }
 }
 
-template <typename IO, int R, int MAXP>
+template <typename IO, int R, int MAXP, bool BCM>
 static cudaError_t launch_decode_t(const DecodeArgs& a, int batch, cudaStream_t s) {
     const int RG = (a.N / 2) / a.ppt;
     const int threads = (a.P / 4) * RG;
-    const size_t smem = sizeof(float) * (size_t)(2 * R * a.P + 3 * R * a.N + a.N + RG * R * a.P);
+    const size_t smem =
+        sizeof(float) * (size_t)(2 * R * a.P + 3 * R * a.N + a.N + RG * R * a.P + 3 * R);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<IO, R, MAXP>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<IO, R, MAXP, BCM>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    decode_kernel<IO, R, MAXP><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
+    decode_kernel<IO, R, MAXP, BCM><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
-template <typename IO>
+template <typename IO, bool BCM>
 static cudaError_t launch_decode_io(const DecodeArgs& a, int batch, int R, cudaStream_t s) {
     if (a.ppt > 8 || (a.ppt > 4 && R != 1)) return cudaErrorNotSupported;
     switch (R) {
-        case 1: return a.ppt > 4 ? launch_decode_t<IO, 1, 8>(a, batch, s)
-                                 : launch_decode_t<IO, 1, 4>(a, batch, s);
-        case 2: return launch_decode_t<IO, 2, 4>(a, batch, s);
-        case 3: return launch_decode_t<IO, 3, 4>(a, batch, s);
-        case 4: return launch_decode_t<IO, 4, 4>(a, batch, s);
-        case 8: return launch_decode_t<IO, 8, 4>(a, batch, s);
+        case 1: return a.ppt > 4 ? launch_decode_t<IO, 1, 8, BCM>(a, batch, s)
+                                 : launch_decode_t<IO, 1, 4, BCM>(a, batch, s);
+        case 2: return launch_decode_t<IO, 2, 4, BCM>(a, batch, s);
+        case 3: return launch_decode_t<IO, 3, 4, BCM>(a, batch, s);
+        case 4: return launch_decode_t<IO, 4, 4, BCM>(a, batch, s);
+        case 8: return launch_decode_t<IO, 8, 4, BCM>(a, batch, s);
         default: return cudaErrorNotSupported;
     }
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int batch, int R, int io_dtype, cudaStream_t s) {
-    if (io_dtype == M3_BF16) return launch_decode_io<__nv_bfloat16>(a, batch, R, s);
-    return launch_decode_io<float>(a, batch, R, s);
+    const bool bc = a.B_bias || a.C_bias || a.bc_eps > 0.f;
+    if (io_dtype == M3_BF16)
+        return bc ? launch_decode_io<__nv_bfloat16, true>(a, batch, R, s)
+                  : launch_decode_io<__nv_bfloat16, false>(a, batch, R, s);
+    return bc ? launch_decode_io<float, true>(a, batch, R, s)
+              : launch_decode_io<float, false>(a, batch, R, s);
 }
 
 // ---------------------------------------------------------------------------------

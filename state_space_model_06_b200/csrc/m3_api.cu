@@ -125,6 +125,32 @@ m3_status m3_state_init(const m3_dims* d, m3_state* state, const float* h0, void
     return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+
+bool bc_norm_on(const m3_extras* ex) { return ex && ex->bc_norm_eps > 0.f; }
+bool bc_any(const m3_extras* ex) { return ex && (ex->B_bias || ex->C_bias || ex->bc_norm_eps > 0.f); }
+
+// Bytes of the BCNorm scale buffer after the tensor-core workspace (256-byte aligned).
+size_t bc_bytes(const m3_dims* d, int32_t seqlen, const m3_extras* ex) {
+    if (!bc_norm_on(ex)) return 0;
+    const size_t n = sizeof(float) * bc_scale_floats(d->batch, seqlen, d->ngroups, d->rank);
+    return (n + 255) / 256 * 256;
+}
+
+}  // namespace
+
+extern "C" {
+
+m3_status m3_scan_workspace_bytes_ex(const m3_dims* d, int32_t seqlen, int32_t chunk,
+                                     const m3_extras* ex, size_t* bytes) {
+    m3_status st = m3_scan_workspace_bytes(d, seqlen, chunk, bytes);
+    if (st != M3_OK) return st;
+    *bytes += bc_bytes(d, seqlen, ex);
+    return M3_OK;
+}
+
 m3_status m3_scan_workspace_bytes(const m3_dims* d, int32_t seqlen, int32_t chunk, size_t* bytes) {
     m3_status st = check_dims(d);
     if (st != M3_OK) return st;
@@ -147,9 +173,10 @@ namespace {
 // Prefill with an optional output gate z (null: none); validation happens before any launch.
 m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
                     const void* B, const void* C, const float* dt, const float* A,
-                    const float* lam, const float* theta, const float* D, const void* z,
+                    const float* lam, const float* theta, const float* D, const m3_extras* ex,
                     m3_state* state, void* y, void* workspace, size_t workspace_bytes,
                     uint32_t flags, void* stream) {
+    const void* z = ex ? ex->z : nullptr;
     m3_status st = check_dims(d);
     if (st != M3_OK) return st;
     if (seqlen < 0) return M3_ERR_SHAPE;
@@ -159,10 +186,13 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
     if (!x || !B || !C || !dt || !A || !lam || !theta || !y) return M3_ERR_NULL;
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
         !aligned(dt, 4) || !aligned(A, 4) || !aligned(lam, 4) || !aligned(theta, 4) ||
-        (D && !aligned(D, 4)) || (z && !aligned(z, 16)))
+        (D && !aligned(D, 4)) || (z && !aligned(z, 16)) ||
+        (ex && ex->B_bias && !aligned(ex->B_bias, 4)) || (ex && ex->C_bias && !aligned(ex->C_bias, 4)))
         return M3_ERR_ALIGN;
-    size_t need = 0;
-    m3_scan_workspace_bytes(d, seqlen, chunk, &need);
+    if (ex && !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;   // negative or NaN epsilon
+    size_t base = 0;
+    m3_scan_workspace_bytes(d, seqlen, chunk, &base);
+    const size_t need = base + bc_bytes(d, seqlen, ex);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return M3_ERR_WORKSPACE;
 
     const int N = d->dstate, P = d->headdim, R = d->rank;
@@ -180,13 +210,23 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
     std::memset(&a, 0, sizeof(a));
     a.x = x; a.B = B; a.C = C; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D;
     a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y; a.z = z;
+    a.B_bias = ex ? ex->B_bias : nullptr;
+    a.C_bias = ex ? ex->C_bias : nullptr;
+    a.bc = bc_any(ex);
+    a.bc_scale = bc_norm_on(ex) ? reinterpret_cast<const float*>(static_cast<char*>(workspace) + base)
+                                : nullptr;
     a.status = static_cast<uint32_t*>(workspace);
     a.ws = static_cast<char*>(workspace) + kStatusBytes;
     a.T = seqlen; a.batch = d->batch; a.H = d->nheads; a.G = d->ngroups; a.P = P; a.N = N;
     a.chunk = use_tc ? qt : chunk; a.ppt = ppt; a.ns = ns; a.flags = flags;
 
     if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return M3_ERR_CUDA;
-    cudaError_t e = use_tc ? launch_scan_tc(a, R, s) : launch_scan_simt(a, R, d->io_dtype, s);
+    cudaError_t e = cudaSuccess;
+    if (a.bc_scale)
+        e = launch_bc_scales(a, R, d->io_dtype, ex->bc_norm_eps,
+                             reinterpret_cast<float*>(static_cast<char*>(workspace) + base), s);
+    if (e != cudaSuccess) return launch_status(e);
+    e = use_tc ? launch_scan_tc(a, R, s) : launch_scan_simt(a, R, d->io_dtype, s);
     if (e != cudaSuccess) return launch_status(e);
     const size_t row = io_bytes(d->io_dtype) * (size_t)d->ngroups * R * N;
     e = launch_copy_prev(state->B_prev, B, seqlen, seqlen - 1, d->batch, row, s);
@@ -196,16 +236,19 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
 // Decode step with an optional output gate z (null: none).
 m3_status decode_impl(const m3_dims* d, const void* x, const void* B, const void* C,
                       const float* dt, const float* A, const float* lam, const float* theta,
-                      const float* D, const void* z, m3_state* state, void* y, uint32_t flags,
-                      void* stream) {
+                      const float* D, const m3_extras* ex, m3_state* state, void* y,
+                      uint32_t flags, void* stream) {
+    const void* z = ex ? ex->z : nullptr;
     m3_status st = check_dims(d);
     if (st != M3_OK) return st;
     if (!x || !B || !C || !dt || !A || !lam || !theta || !y) return M3_ERR_NULL;
     if ((st = check_state(state)) != M3_OK) return st;
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
         !aligned(dt, 4) || !aligned(A, 4) || !aligned(lam, 4) || !aligned(theta, 4) ||
-        (D && !aligned(D, 4)) || (z && !aligned(z, 16)))
+        (D && !aligned(D, 4)) || (z && !aligned(z, 16)) ||
+        (ex && ex->B_bias && !aligned(ex->B_bias, 4)) || (ex && ex->C_bias && !aligned(ex->C_bias, 4)))
         return M3_ERR_ALIGN;
+    if (ex && !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;
     int ppt = 0;
     if (!rank_has_kernel(d->rank) || !decode_shape(d->dstate, d->headdim, d->rank, &ppt))
         return M3_ERR_UNSUPPORTED;
@@ -214,6 +257,9 @@ m3_status decode_impl(const m3_dims* d, const void* x, const void* B, const void
     std::memset(&a, 0, sizeof(a));
     a.x = x; a.B = B; a.C = C; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D;
     a.h = state->h; a.x_prev = state->x_prev; a.B_prev = state->B_prev; a.y = y; a.z = z;
+    a.B_bias = ex ? ex->B_bias : nullptr;
+    a.C_bias = ex ? ex->C_bias : nullptr;
+    a.bc_eps = ex ? ex->bc_norm_eps : 0.f;
     a.H = d->nheads; a.G = d->ngroups; a.P = d->headdim; a.N = d->dstate;
     a.ppt = ppt; a.flags = flags;
     cudaError_t e = launch_decode(a, d->batch, d->rank, d->io_dtype, s);
@@ -236,13 +282,25 @@ m3_status m3_scan_fwd(const m3_dims* d, int32_t seqlen, int32_t chunk, const voi
                      workspace, workspace_bytes, flags, stream);
 }
 
+m3_status m3_scan_fwd_ex(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
+                         const void* B, const void* C, const float* dt, const float* A,
+                         const float* lam, const float* theta, const float* D,
+                         const m3_extras* ex, m3_state* state, void* y, void* workspace,
+                         size_t workspace_bytes, uint32_t flags, void* stream) {
+    return scan_impl(d, seqlen, chunk, x, B, C, dt, A, lam, theta, D, ex, state, y, workspace,
+                     workspace_bytes, flags, stream);
+}
+
 m3_status m3_scan_fwd_gated(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
                             const void* B, const void* C, const float* dt, const float* A,
                             const float* lam, const float* theta, const float* D,
                             const void* z, m3_state* state, void* y, void* workspace,
                             size_t workspace_bytes, uint32_t flags, void* stream) {
     if (!z && seqlen != 0) return M3_ERR_NULL;
-    return scan_impl(d, seqlen, chunk, x, B, C, dt, A, lam, theta, D, z, state, y, workspace,
+    m3_extras ex;
+    std::memset(&ex, 0, sizeof(ex));
+    ex.z = z;
+    return scan_impl(d, seqlen, chunk, x, B, C, dt, A, lam, theta, D, &ex, state, y, workspace,
                      workspace_bytes, flags, stream);
 }
 
@@ -253,12 +311,22 @@ m3_status m3_decode_step(const m3_dims* d, const void* x, const void* B, const v
     return decode_impl(d, x, B, C, dt, A, lam, theta, D, nullptr, state, y, flags, stream);
 }
 
+m3_status m3_decode_step_ex(const m3_dims* d, const void* x, const void* B, const void* C,
+                            const float* dt, const float* A, const float* lam,
+                            const float* theta, const float* D, const m3_extras* ex,
+                            m3_state* state, void* y, uint32_t flags, void* stream) {
+    return decode_impl(d, x, B, C, dt, A, lam, theta, D, ex, state, y, flags, stream);
+}
+
 m3_status m3_decode_step_gated(const m3_dims* d, const void* x, const void* B, const void* C,
                                const float* dt, const float* A, const float* lam,
                                const float* theta, const float* D, const void* z,
                                m3_state* state, void* y, uint32_t flags, void* stream) {
     if (!z) return M3_ERR_NULL;
-    return decode_impl(d, x, B, C, dt, A, lam, theta, D, z, state, y, flags, stream);
+    m3_extras ex;
+    std::memset(&ex, 0, sizeof(ex));
+    ex.z = z;
+    return decode_impl(d, x, B, C, dt, A, lam, theta, D, &ex, state, y, flags, stream);
 }
 
 m3_status m3_query_status(const void* workspace, void* stream) {

@@ -27,6 +27,12 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return
 // SiLU(z) = z / (1 + e^-z).  A large negative z gives e^-z = inf and a gate of -0.
 __device__ __forceinline__ float gate_silu(float v, float z) { return v * (z / (1.f + expf(-z))); }
 
+// One element of the BC map ("Technical Approach", BCNorm and BC biases): v * s + bias,
+// with s the column's BCNorm scale (1 when off) and bias the head's channel bias (0 when off).
+__device__ __forceinline__ float bc_apply(float v, float s, const float* bias, int n) {
+    return fmaf(v, s, bias ? bias[n] : 0.f);
+}
+
 // Argument block of one decode step (device pointers, validated on the host).
 struct DecodeArgs {
     const void* x;       // [b][H][R][P] io
@@ -42,6 +48,9 @@ struct DecodeArgs {
     const void* B_prev;  // [b][G][R][N] io (read only here; updated by a follow-up copy)
     void* y;             // [b][H][R][P] io
     const void* z;       // [b][H][R][P] io: output gate, or null for none
+    const float* B_bias; // [H][N]: BC bias of B, or null
+    const float* C_bias; // [H][N]: BC bias of C, or null
+    float bc_eps;        // > 0: RMS-normalise B, B_prev and C columns over N (BCNorm)
     int H, G, P, N;
     int ppt;             // state pairs per thread
     uint32_t flags;
@@ -62,6 +71,12 @@ struct ScanArgs {
     const void* B_prev;  // [b][G][R][N]   read only here; updated by a follow-up copy
     void* y;             // [b][T][H][R][P] io
     const void* z;       // [b][T][H][R][P] io: output gate, or null for none
+    const float* B_bias; // [H][N]: BC bias of B, or null
+    const float* C_bias; // [H][N]: BC bias of C, or null
+    // BCNorm scales 1 / sqrt(mean_n v^2 + eps) (workspace; null when off), one per column:
+    // B [b][T][G][R], then C [b][T][G][R], then B_prev [b][G][R]
+    const float* bc_scale;
+    bool bc;             // any BC map (bias or normalisation) is applied
     uint32_t* status;    // workspace status word (may be null)
     void* ws;            // workspace (after the status block)
     long long T;

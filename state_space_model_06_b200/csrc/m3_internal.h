@@ -20,6 +20,12 @@ int scan_tc_chunk(int N, int P, int R, int chunk, int H);   // tile chunk, 0 = n
 size_t scan_tc_workspace_bytes(int batch, int H, int N, int P, int R, long long T, int chunk);
 cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s);
 
+// BCNorm scales of every B, C and B_prev column of a prefill call into a.bc_scale
+// (floats: b*T*G*R for B, the same for C, then b*G*R for B_prev).
+size_t bc_scale_floats(int batch, long long T, int G, int R);
+cudaError_t launch_bc_scales(const ScanArgs& a, int R, int io_dtype, float eps, float* out,
+                             cudaStream_t s);
+
 // B_prev <- B[:, t] for every (batch, group): the previous-token input of the
 // next call, written after every head of the group has read the old value.
 cudaError_t launch_copy_prev(void* B_prev, const void* B, long long T, long long t, int batch,

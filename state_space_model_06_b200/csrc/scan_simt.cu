@@ -48,12 +48,25 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
         }
     }
 
+    // BC map (BCNorm scale per column, head bias per channel): the scales of this call's
+    // columns start at sB (B), sC (C) and sP (B_prev); null scales mean 1
+    const float* Bb = a.B_bias ? a.B_bias + (size_t)h * N : nullptr;
+    const float* Cb = a.C_bias ? a.C_bias + (size_t)h * N : nullptr;
+    const size_t ncol = (size_t)a.batch * T * G * R;
+    const float* sB = a.bc_scale;
+    const float* sC = a.bc_scale ? a.bc_scale + ncol : nullptr;
+    const float* sP = a.bc_scale ? a.bc_scale + 2 * ncol : nullptr;
+
     // previous token of the first step comes from the carried state (buffer 1)
     {
         const IO* xp = static_cast<const IO*>(a.x_prev) + (size_t)bh * R * P;
         const IO* bp = static_cast<const IO*>(a.B_prev) + ((size_t)b * G + g) * R * N;
         for (int e = tid; e < R * P; e += nthr) buf1[e] = to_f(xp[e]);
-        for (int e = tid; e < R * N; e += nthr) buf1[R * P + e] = to_f(bp[e]);
+        for (int e = tid; e < R * N; e += nthr) {
+            const int r = e / N;
+            const float sc = sP ? sP[((size_t)b * G + g) * R + r] : 1.f;
+            buf1[R * P + e] = a.bc ? bc_apply(to_f(bp[e]), sc, Bb, e - r * N) : to_f(bp[e]);
+        }
     }
 
     const float Dh = a.D ? a.D[h] : 0.f;
@@ -70,9 +83,18 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
         const IO* Ct = static_cast<const IO*>(a.C) + (bt * G + g) * R * N;
         const float dt = a.dt[bt * H + h];
         for (int e = tid; e < R * P; e += nthr) cur[e] = to_f(xt[e]);
-        for (int e = tid; e < R * N; e += nthr) {
-            cur[R * P + e] = to_f(Bt[e]);
-            cur[R * P + R * N + e] = to_f(Ct[e]);
+        if (a.bc) {
+            for (int e = tid; e < R * N; e += nthr) {
+                const int r = e / N, n = e - r * N;
+                const size_t col = (bt * G + g) * R + r;
+                cur[R * P + e] = bc_apply(to_f(Bt[e]), sB ? sB[col] : 1.f, Bb, n);
+                cur[R * P + R * N + e] = bc_apply(to_f(Ct[e]), sC ? sC[col] : 1.f, Cb, n);
+            }
+        } else {
+            for (int e = tid; e < R * N; e += nthr) {
+                cur[R * P + e] = to_f(Bt[e]);
+                cur[R * P + R * N + e] = to_f(Ct[e]);
+            }
         }
         const float* th = a.theta + (bt * G + g) * (N / 2);
         for (int i = tid; i < N / 2; i += nthr) {

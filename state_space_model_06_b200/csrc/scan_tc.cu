@@ -325,7 +325,7 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
 // ts = rw / PB.  The starting angle of a thread's token range is the running angle plus
 // the angle sums of the earlier ranges, exchanged through shared memory once per
 // sub-chunk (bounded mbarrier hand-off).
-template <int NST, int Q, int R, bool GT>
+template <int NST, int Q, int R, bool GT, bool BC>
 __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     constexpr int TPT = C::TPT, PAIRS = C::PAIRS, TSPLIT = C::TSPLIT;
@@ -339,6 +339,16 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
     const int atom = (2 * pair) >> 6, col = (2 * pair) & 63;
     float* rsum = reinterpret_cast<float*>(sm + C::OFF_RSUM);
     int raw_it = 0;
+    // BC map ("Technical Approach", BCNorm and BC biases): B and C of this thread's pair
+    // channels become v * s + bias, s the column's BCNorm scale (1 when off), bias the head's
+    constexpr bool bc = BC;
+    const int hh = blockIdx.x % a.H, bq = blockIdx.x / a.H, gq = hh / (a.H / a.G);
+    float bb0 = 0.f, bb1 = 0.f, cb0 = 0.f, cb1 = 0.f;
+    if (a.B_bias) { bb0 = a.B_bias[hh * NST + 2 * pair]; bb1 = a.B_bias[hh * NST + 2 * pair + 1]; }
+    if (a.C_bias) { cb0 = a.C_bias[hh * NST + 2 * pair]; cb1 = a.C_bias[hh * NST + 2 * pair + 1]; }
+    const size_t ncol = (size_t)a.batch * a.T * a.G * R;
+    const float* sBq = a.bc_scale ? a.bc_scale + ((size_t)bq * a.T * a.G + gq) * R : nullptr;
+    const size_t sstride = (size_t)a.G * R;          // between consecutive tokens
     // call-relative angle of this thread's pair (the RoPE frame of Proposition 4 starts at
     // the first token of the call), reduced mod 2 pi at chunk boundaries
     float psi_acc = 0.f;
@@ -386,6 +396,21 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                     bv[jj][r] = braw[e];
                     cv[jj][r] = craw[e];
                 }
+            // BCNorm scales of the own tokens (1 past the end of the call: those rows are
+            // zero-filled and masked out)
+            float sb[TPT][R], sc[TPT][R];
+            if constexpr (bc) {
+#pragma unroll
+                for (int jj = 0; jj < TPT; ++jj) {
+                    const long long t = (long long)c * Q + tb + j0 + jj;
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const bool in = sBq && t < a.T;
+                        sb[jj][r] = in ? sBq[(size_t)t * sstride + r] : 1.f;
+                        sc[jj][r] = in ? sBq[ncol + (size_t)t * sstride + r] : 1.f;
+                    }
+                }
+            }
             if (!warp_wait(&bar[RS0 + rs], (raw_it >> 1) & 1, ab)) return;
             if (tid == 0) M3_TRACE_EV(c, s == 0 ? 28 : 31);
             float pre = 0.f, tot = 0.f;
@@ -428,10 +453,18 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                 for (int r = 0; r < R; ++r) {
                     const uint32_t ba = bv[jj][r], bb = bv[jj + 1][r];
                     const uint32_t ca = cv[jj][r], cb = cv[jj + 1][r];
-                    const float2 b0 = make_float2(bf16lo(ba), bf16lo(bb));
-                    const float2 b1 = make_float2(bf16hi(ba), bf16hi(bb));
-                    const float2 c0 = make_float2(bf16lo(ca), bf16lo(cb));
-                    const float2 c1 = make_float2(bf16hi(ca), bf16hi(cb));
+                    float2 b0 = make_float2(bf16lo(ba), bf16lo(bb));
+                    float2 b1 = make_float2(bf16hi(ba), bf16hi(bb));
+                    float2 c0 = make_float2(bf16lo(ca), bf16lo(cb));
+                    float2 c1 = make_float2(bf16hi(ca), bf16hi(cb));
+                    if constexpr (bc) {
+                        const float2 sb2 = make_float2(sb[jj][r], sb[jj + 1][r]);
+                        const float2 sc2 = make_float2(sc[jj][r], sc[jj + 1][r]);
+                        b0 = __ffma2_rn(b0, sb2, make_float2(bb0, bb0));
+                        b1 = __ffma2_rn(b1, sb2, make_float2(bb1, bb1));
+                        c0 = __ffma2_rn(c0, sc2, make_float2(cb0, cb0));
+                        c1 = __ffma2_rn(c1, sc2, make_float2(cb1, cb1));
+                    }
                     const float2 nb0 = __ffma2_rn(c2, b0, __fmul2_rn(s2, b1));
                     const float2 nb1 = __ffma2_rn(c2, b1, __fmul2_rn(m2, b0));
                     const float2 nc0 = __ffma2_rn(c2, c0, __fmul2_rn(s2, c1));
@@ -444,8 +477,14 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                 const int jj = TPT - 1;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const float b0 = bf16lo(bv[jj][r]), b1 = bf16hi(bv[jj][r]);
-                    const float c0 = bf16lo(cv[jj][r]), c1 = bf16hi(cv[jj][r]);
+                    float b0 = bf16lo(bv[jj][r]), b1 = bf16hi(bv[jj][r]);
+                    float c0 = bf16lo(cv[jj][r]), c1 = bf16hi(cv[jj][r]);
+                    if constexpr (bc) {
+                        b0 = fmaf(b0, sb[jj][r], bb0);
+                        b1 = fmaf(b1, sb[jj][r], bb1);
+                        c0 = fmaf(c0, sc[jj][r], cb0);
+                        c1 = fmaf(c1, sc[jj][r], cb1);
+                    }
                     store(jj, r, pack_bf16x2(fmaf(cn[jj], b0, sn[jj] * b1), fmaf(cn[jj], b1, -sn[jj] * b0)),
                           pack_bf16x2(fmaf(cn[jj], c0, sn[jj] * c1), fmaf(cn[jj], c1, -sn[jj] * c0)));
                 }
@@ -709,7 +748,7 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
 // State warpgroup (warps 16-19): the fp32 carried state g in TMEM columns TM_G..,
 // g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T, per chunk g <- e^{cum_end} g + dS and its
 // bf16 copy for the Y_inter MMA; at the end h_T = R(psi_T) g and the carried x.
-template <int NST, int Q, int R, bool GT>
+template <int NST, int Q, int R, bool GT, bool BC>
 __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
                       const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
@@ -745,6 +784,11 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
         const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(a.x_prev) + bh * R * kP;
         const __nv_bfloat16* bp =
             static_cast<const __nv_bfloat16*>(a.B_prev) + ((size_t)b * a.G + g) * R * NST;
+        // the carried previous token's B goes through the BC map as well
+        const float* sP = a.bc_scale
+                              ? a.bc_scale + 2 * (size_t)a.batch * T * a.G * R + ((size_t)b * a.G + g) * R
+                              : nullptr;
+        const float* Bb = a.B_bias ? a.B_bias + (size_t)h * NST : nullptr;
 #pragma unroll 1
         for (int cb = 0; cb < kNCols; cb += 16) {
             float gv[16];
@@ -755,7 +799,8 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
             }
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float bb = beta0 * __bfloat162float(bp[r * NST + nrow]);
+                const float bv0 = __bfloat162float(bp[r * NST + nrow]);
+                const float bb = beta0 * (BC ? bc_apply(bv0, sP ? sP[r] : 1.f, Bb, nrow) : bv0);
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
                     gv[j] = fmaf(bb, __bfloat162float(xp[r * kP + ncol0 + cb + j]), gv[j]);
@@ -934,7 +979,7 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
     bulk_wait<0>();
 }
 
-template <int NST, int Q, int R, bool GT>
+template <int NST, int Q, int R, bool GT, bool BC>
 __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_constant__ TcParams p) {
     using C = Cfg<NST, Q, R, GT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -979,9 +1024,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     } else if (w < 6) {
         epilogue<NST, Q, R, GT>(p, sm, bar, tmem, ab);
     } else if (w >= 16) {
-        state<NST, Q, R, GT>(p, sm, bar, tmem, ab);
+        state<NST, Q, R, GT, BC>(p, sm, bar, tmem, ab);
     } else if (w < 6 + kRotWarps) {
-        rotation<NST, Q, R, GT>(p, sm, bar, ab);
+        rotation<NST, Q, R, GT, BC>(p, sm, bar, ab);
     } else if (w == 6 + kRotWarps) {
         coefficients<NST, Q, R, GT>(p, sm, bar, ab);
     } else if ((threadIdx.x & 31) == 0) {
@@ -1031,7 +1076,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ptr,
     return r == CUDA_SUCCESS;
 }
 
-template <int NST, int Q, int R, bool GT>
+template <int NST, int Q, int R, bool GT, bool BC>
 cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
     using C = Cfg<NST, Q, R, GT>;
     TcParams p;
@@ -1082,10 +1127,10 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R, GT>,
+    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R, GT, BC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<NST, Q, R, GT><<<(unsigned)(a.batch * a.H), kThreads, C::SMEM, s>>>(p);
+    scan_tc_kernel<NST, Q, R, GT, BC><<<(unsigned)(a.batch * a.H), kThreads, C::SMEM, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -1114,27 +1159,28 @@ int scan_tc_chunk(int N, int P, int R, int chunk, int H) {
 
 size_t scan_tc_workspace_bytes(int, int, int, int, int, long long, int) { return 0; }
 
-template <bool GT>
+template <bool GT, bool BC>
 cudaError_t launch_scan_tc_g(const ScanArgs& a, int R, cudaStream_t s) {
     const int N = a.N, Q = a.chunk;   // the tile chunk chosen by scan_tc_chunk
     if (R == 1) {
-        if (N == 128 && Q == 64) return launch_t<128, 64, 1, GT>(a, s);
-        if (N == 128 && Q == 128) return launch_t<128, 128, 1, GT>(a, s);
-        if (N == 64 && Q == 64) return launch_t<64, 64, 1, GT>(a, s);
-        if (N == 64 && Q == 128) return launch_t<64, 128, 1, GT>(a, s);
+        if (N == 128 && Q == 64) return launch_t<128, 64, 1, GT, BC>(a, s);
+        if (N == 128 && Q == 128) return launch_t<128, 128, 1, GT, BC>(a, s);
+        if (N == 64 && Q == 64) return launch_t<64, 64, 1, GT, BC>(a, s);
+        if (N == 64 && Q == 128) return launch_t<64, 128, 1, GT, BC>(a, s);
     } else if (R == 2 && N == 64) {
-        if (Q == 32) return launch_t<64, 32, 2, GT>(a, s);
-        if (Q == 64) return launch_t<64, 64, 2, GT>(a, s);
+        if (Q == 32) return launch_t<64, 32, 2, GT, BC>(a, s);
+        if (Q == 64) return launch_t<64, 64, 2, GT, BC>(a, s);
     } else if (R == 4 && N == 64) {
-        if (Q == 16) return launch_t<64, 16, 4, GT>(a, s);
-        if (Q == 32) return launch_t<64, 32, 4, GT>(a, s);
+        if (Q == 16) return launch_t<64, 16, 4, GT, BC>(a, s);
+        if (Q == 32) return launch_t<64, 32, 4, GT, BC>(a, s);
     }
     return cudaErrorNotSupported;
 }
 
-// a.z selects the instantiation with the fused output gate
+// a.z and a.bc select the instantiation with the fused output gate and BC map
 cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s) {
-    return a.z ? launch_scan_tc_g<true>(a, R, s) : launch_scan_tc_g<false>(a, R, s);
+    if (a.z) return a.bc ? launch_scan_tc_g<true, true>(a, R, s) : launch_scan_tc_g<true, false>(a, R, s);
+    return a.bc ? launch_scan_tc_g<false, true>(a, R, s) : launch_scan_tc_g<false, false>(a, R, s);
 }
 
 }  // namespace m3

@@ -114,6 +114,15 @@ def make_gate(shape, io_dtype=torch.bfloat16, seed=0):
     return _randn(g, tuple(shape), dtype=io_dtype)
 
 
+def make_bc_bias(nheads, dstate, seed=0):
+    """BC biases B_bias, C_bias [H][N] float32: the pages' all-ones initialisation plus a
+    per-channel N(0, 0.3^2) spread (a trained layer's biases are not all equal).  Own
+    generator (seed + 104729): adding biases never changes the other seeded inputs."""
+    g = torch.Generator("cpu").manual_seed(seed + 104729)
+    return (1.0 + 0.3 * torch.randn((nheads, dstate), generator=g),
+            1.0 + 0.3 * torch.randn((nheads, dstate), generator=g))
+
+
 def make_decode_inputs(batch, nheads, ngroups, headdim, dstate, rank=1, tokens=1,
                        io_dtype=torch.bfloat16, theta_max=math.pi / 8, seed=0):
     """Per-token decode inputs stacked over ``tokens`` plus the starting state.

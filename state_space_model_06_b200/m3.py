@@ -26,7 +26,8 @@ M3_FLAG_TEST_STALL = 4
 
 EXPORTED = ("m3_state_bytes", "m3_state_init", "m3_scan_workspace_bytes", "m3_scan_fwd",
             "m3_decode_step", "m3_query_status", "m3_scan_fwd_noalloc", "m3_scan_fwd_gated",
-            "m3_decode_step_gated", "m3_status_string")
+            "m3_decode_step_gated", "m3_scan_workspace_bytes_ex", "m3_scan_fwd_ex",
+            "m3_decode_step_ex", "m3_status_string")
 
 
 class M3Error(RuntimeError):
@@ -44,6 +45,11 @@ class m3_dims(ctypes.Structure):
 
 class m3_state(ctypes.Structure):
     _fields_ = [("h", ctypes.c_void_p), ("x_prev", ctypes.c_void_p), ("B_prev", ctypes.c_void_p)]
+
+
+class m3_extras(ctypes.Structure):
+    _fields_ = [("z", ctypes.c_void_p), ("B_bias", ctypes.c_void_p), ("C_bias", ctypes.c_void_p),
+                ("bc_norm_eps", ctypes.c_float)]
 
 
 _lib = None
@@ -70,6 +76,11 @@ def load_library(path: str = LIB_PATH):
                                           vp, vp, sz, u32, vp]
         lib.m3_decode_step_gated.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp,
                                              u32, vp]
+        ep = ctypes.POINTER(m3_extras)
+        lib.m3_scan_workspace_bytes_ex.argtypes = [dp, i32, i32, ep, szp]
+        lib.m3_scan_fwd_ex.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, ep, sp, vp,
+                                       vp, sz, u32, vp]
+        lib.m3_decode_step_ex.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, ep, sp, vp, u32, vp]
         lib.m3_scan_fwd_noalloc.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp,
                                             u32, vp]
         lib.m3_query_status.argtypes = [vp, vp]
@@ -196,6 +207,59 @@ def m3_scan_fwd_gated(dims: Dims, seqlen: int, chunk: int, x, B, C, dt, A, lam, 
         ctypes.byref(dims.c()), int(seqlen), int(chunk), _ptr(x), _ptr(B), _ptr(C), _ptr(dt),
         _ptr(A), _ptr(lam), _ptr(theta), _ptr(D), _ptr(z), ctypes.byref(st), _ptr(y),
         _ptr(workspace), ws_bytes, int(flags), _stream(stream)), "m3_scan_fwd_gated")
+
+
+@dataclass
+class Extras:
+    """Optional fused parts (see m3_extras in include/m3.h): output gate z, BC biases
+    B_bias / C_bias [H][N] fp32, BCNorm epsilon (0: off)."""
+    z: object = None
+    B_bias: object = None
+    C_bias: object = None
+    bc_norm_eps: float = 0.0
+
+    def c(self) -> m3_extras:
+        return m3_extras(_ptr(self.z), _ptr(self.B_bias), _ptr(self.C_bias),
+                         float(self.bc_norm_eps))
+
+
+def _ex_ref(ex):
+    return ctypes.byref(ex.c()) if ex is not None else None
+
+
+def m3_scan_workspace_bytes_ex(dims: Dims, seqlen: int, chunk: int, ex) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().m3_scan_workspace_bytes_ex(ctypes.byref(dims.c()), int(seqlen),
+                                                     int(chunk), _ex_ref(ex), ctypes.byref(n)),
+           "m3_scan_workspace_bytes_ex")
+    return n.value
+
+
+def m3_scan_fwd_ex(dims: Dims, seqlen: int, chunk: int, x, B, C, dt, A, lam, theta, D, ex,
+                   state: State, y, workspace, flags: int = 0, stream=None):
+    """Prefill with the optional fused parts in ``ex`` (an Extras, or None)."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = state.c()
+    _check(load_library().m3_scan_fwd_ex(
+        ctypes.byref(dims.c()), int(seqlen), int(chunk), _ptr(x), _ptr(B), _ptr(C), _ptr(dt),
+        _ptr(A), _ptr(lam), _ptr(theta), _ptr(D), _ex_ref(ex), ctypes.byref(st), _ptr(y),
+        _ptr(workspace), ws_bytes, int(flags), _stream(stream)), "m3_scan_fwd_ex")
+
+
+def m3_decode_step_ex(dims: Dims, x, B, C, dt, A, lam, theta, D, ex, state: State, y,
+                      flags: int = 0, stream=None):
+    """Decode step with the optional fused parts in ``ex`` (an Extras, or None)."""
+    st = state.c()
+    _check(load_library().m3_decode_step_ex(
+        ctypes.byref(dims.c()), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam),
+        _ptr(theta), _ptr(D), _ex_ref(ex), ctypes.byref(st), _ptr(y), int(flags),
+        _stream(stream)), "m3_decode_step_ex")
+
+
+def alloc_workspace_ex(dims: Dims, seqlen: int, chunk: int, ex, device="cuda") -> torch.Tensor:
+    """A workspace tensor of the size m3_scan_fwd_ex needs with these extras."""
+    n = m3_scan_workspace_bytes_ex(dims, seqlen, chunk, ex)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def m3_decode_step_gated(dims: Dims, x, B, C, dt, A, lam, theta, D, z, state: State, y,

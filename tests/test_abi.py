@@ -124,6 +124,38 @@ def test_gated_validation_before_launch(lib):
     assert dec(p + 4) == m3.M3_ERR_ALIGN
 
 
+def test_extras_validation_before_launch(lib):
+    """m3_scan_fwd_ex / m3_decode_step_ex check the extras before anything runs, and the
+    BCNorm scales are part of the workspace size."""
+    d = m3.Dims(1, 2, 1, 16, 16, 1, m3.M3_BF16)
+    st = m3.m3_state(0x2000, 0x3000, 0x4000)
+    p, ws = 0x1000, 0x100000
+    base = m3.m3_scan_workspace_bytes(d, 64, 64)
+    assert m3.m3_scan_workspace_bytes_ex(d, 64, 64, None) == base
+    assert m3.m3_scan_workspace_bytes_ex(d, 64, 64, m3.Extras(B_bias=p)) == base
+    with_norm = m3.m3_scan_workspace_bytes_ex(d, 64, 64, m3.Extras(bc_norm_eps=1e-6))
+    assert with_norm >= base + 4 * (2 * 64 + 1)
+
+    def scan(ex, ws_bytes=1 << 20):
+        e = ex.c()
+        return lib.m3_scan_fwd_ex(ctypes.byref(d.c()), 64, 64, p, p, p, p, p, p, p, None,
+                                  ctypes.byref(e), ctypes.byref(st), p, ws, ws_bytes, 0, None)
+
+    assert scan(m3.Extras(bc_norm_eps=-1.0)) == m3.M3_ERR_SHAPE
+    assert scan(m3.Extras(bc_norm_eps=float("nan"))) == m3.M3_ERR_SHAPE
+    assert scan(m3.Extras(B_bias=p + 2)) == m3.M3_ERR_ALIGN
+    assert scan(m3.Extras(z=p + 8)) == m3.M3_ERR_ALIGN
+    assert scan(m3.Extras(bc_norm_eps=1e-6), ws_bytes=base) == m3.M3_ERR_WORKSPACE
+
+    def dec(ex):
+        e = ex.c()
+        return lib.m3_decode_step_ex(ctypes.byref(d.c()), p, p, p, p, p, p, p, None,
+                                     ctypes.byref(e), ctypes.byref(st), p, 0, None)
+
+    assert dec(m3.Extras(bc_norm_eps=-1.0)) == m3.M3_ERR_SHAPE
+    assert dec(m3.Extras(C_bias=p + 1)) == m3.M3_ERR_ALIGN
+
+
 def test_binding_refuses_missing_library(tmp_path):
     old = m3._lib
     m3._lib = None
