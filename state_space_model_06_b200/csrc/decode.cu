@@ -186,9 +186,232 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, int batch, cudaStream_t 
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------------
+// MIMO decode with 8 state pairs per thread.  With R rank columns the per-element work is
+// R times SISO's, so the update is written as one rank-2R product on packed fp32 pairs:
+//   h' = R(phi)(alpha h) + [beta R(phi) Bp | gamma B] [xp | x]^T
+// (the rotation is linear and moves onto Bp).  The per-head factors -- U = [beta R Bp |
+// gamma B] and C stored duplicated per row, (u, u), so that they feed the FFMA2 operands
+// directly, and V = [xp | x] -- are built in shared memory while the state loads are in
+// flight.  Thread (j, rg) keeps 8 pairs x 4 columns of the state in registers: twice the
+// 16-byte loads in flight per thread of the 4-pair kernel, at about a quarter of its
+// instructions per element.
+
+__device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z, v.w); }
+
+// Row groups merged per warp by shuffles before the shared-memory reduction.
+__host__ __device__ inline int mimo_wr(int cpr, int threads) {
+    return (threads % 32 == 0 && 32 % cpr == 0) ? 32 / cpr : 1;
+}
+
+static size_t mimo_smem_floats(int N, int P, int R, int ppt, bool bcm) {
+    const int np2 = N / 2, cpr = P / 4, rg = np2 / ppt;
+    const int rgw = rg / mimo_wr(cpr, cpr * rg);
+    return (size_t)np2 * 2 * R * 4 + (size_t)np2 * R * 4 + (size_t)np2 * 8 + 2 * R * P +
+           (size_t)rgw * R * P + (bcm ? 3 * R * N + 3 * R : 0);
+}
+
+template <typename IO, int R, int MAXP, bool BCM>
+__global__ void __launch_bounds__(512) decode_mimo_kernel(DecodeArgs a) {
+    extern __shared__ __align__(16) float sm[];
+    constexpr int R2 = 2 * R;
+    const int N = a.N, P = a.P, H = a.H, G = a.G, NP2 = a.N / 2, CPR = a.P / 4;
+    const int RG = NP2 / a.ppt, nthr = blockDim.x;
+    const int bh = blockIdx.x, b = bh / H, h = bh - b * H, g = h / (H / G);
+    const int tid = threadIdx.x, j = tid % CPR, rg = tid / CPR;
+    const int WR = mimo_wr(CPR, nthr), RGW = RG / WR;
+
+    float4* U4 = reinterpret_cast<float4*>(sm);            // [N/2][2R] (u0, u0, u1, u1)
+    float4* C4 = U4 + NP2 * R2;                             // [N/2][R]  (c0, c0, c1, c1)
+    float4* rot4 = C4 + NP2 * R;                            // [N/2][2]  (ac, ac, as, as), (-as, -as, 0, 0)
+    float* V = reinterpret_cast<float*>(rot4 + NP2 * 2);    // [2R][P]   rows xp_r, then x_r
+    float* ypart = V + R2 * P;                              // [RG / WR][R][P]
+    float* raw = ypart + RGW * R * P;                       // BC map: [3][R][N] B, B_prev, C
+    float* bcs = raw + 3 * R * N;                           // BC map: [3R] column scales
+
+    // 1. the state loads first: they are the whole cost of the step
+    float4* hrow = reinterpret_cast<float4*>(a.h + (size_t)bh * N * P);
+    float4 v0[MAXP], v1[MAXP];
+#pragma unroll
+    for (int k = 0; k < MAXP; ++k) {
+        if (k < a.ppt) {
+            const int i = rg + k * RG;
+            v0[k] = __ldcs(hrow + (size_t)(2 * i) * CPR + j);
+            v1[k] = __ldcs(hrow + (size_t)(2 * i + 1) * CPR + j);
+        }
+    }
+
+    // 2. this token's factors, in shared memory
+    const float dt = a.dt[bh], Av = a.A[bh], lam = a.lam[bh];
+    const float alpha = expf(dt * Av);
+    const float beta = (1.f - lam) * dt * alpha;
+    const float gamma = lam * dt;
+    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * R * P;
+    const IO* xp = static_cast<const IO*>(a.x_prev) + (size_t)bh * R * P;
+    const size_t gofs = ((size_t)b * G + g) * R * N;
+    const IO* Bg = static_cast<const IO*>(a.B) + gofs;
+    const IO* Bpg = static_cast<const IO*>(a.B_prev) + gofs;
+    const IO* Cg = static_cast<const IO*>(a.C) + gofs;
+    const float* th = a.theta + ((size_t)b * G + g) * NP2;
+    if constexpr (BCM) {
+        // BC map ("Technical Approach", BCNorm and BC biases) on B, B_prev and C first
+        for (int e = tid; e < R * N; e += nthr) {
+            raw[e] = to_f(Bg[e]);
+            raw[R * N + e] = to_f(Bpg[e]);
+            raw[2 * R * N + e] = to_f(Cg[e]);
+        }
+        __syncthreads();
+        for (int c = tid; c < 3 * R; c += nthr) {          // one thread per column: serial sum
+            float sc = 1.f;
+            if (a.bc_eps > 0.f) {
+                const float* v = raw + (size_t)c * N;       // columns B r, then B_prev r, then C r
+                float ss = 0.f;
+                for (int n = 0; n < N; ++n) ss = fmaf(v[n], v[n], ss);
+                sc = rsqrtf(ss / (float)N + a.bc_eps);
+            }
+            bcs[c] = sc;
+        }
+        __syncthreads();
+        const float* Bb = a.B_bias ? a.B_bias + (size_t)h * N : nullptr;
+        const float* Cb = a.C_bias ? a.C_bias + (size_t)h * N : nullptr;
+        for (int e = tid; e < R * N; e += nthr) {
+            const int r = e / N, n = e - r * N;
+            raw[e] = bc_apply(raw[e], bcs[r], Bb, n);
+            raw[R * N + e] = bc_apply(raw[R * N + e], bcs[R + r], Bb, n);
+            raw[2 * R * N + e] = bc_apply(raw[2 * R * N + e], bcs[2 * R + r], Cb, n);
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < NP2 * R; e += nthr) {
+        const int i = e / R, r = e - i * R;
+        const float phi = (a.flags & M3_FLAG_THETA_IS_ANGLE) ? th[i] : dt * th[i];
+        float sn, cs;
+        sincosf(phi, &sn, &cs);
+        if (r == 0) {
+            const float ac = alpha * cs, as = alpha * sn;
+            rot4[2 * i] = make_float4(ac, ac, as, as);
+            rot4[2 * i + 1] = make_float4(-as, -as, 0.f, 0.f);
+        }
+        const int n0 = r * N + 2 * i;
+        float p0, p1, q0, q1, c0, c1;
+        if constexpr (BCM) {
+            q0 = raw[n0]; q1 = raw[n0 + 1];
+            p0 = raw[R * N + n0]; p1 = raw[R * N + n0 + 1];
+            c0 = raw[2 * R * N + n0]; c1 = raw[2 * R * N + n0 + 1];
+        } else {
+            q0 = to_f(Bg[n0]); q1 = to_f(Bg[n0 + 1]);
+            p0 = to_f(Bpg[n0]); p1 = to_f(Bpg[n0 + 1]);
+            c0 = to_f(Cg[n0]); c1 = to_f(Cg[n0 + 1]);
+        }
+        const float ub0 = beta * (cs * p0 - sn * p1), ub1 = beta * (sn * p0 + cs * p1);
+        const float ug0 = gamma * q0, ug1 = gamma * q1;
+        U4[i * R2 + r] = make_float4(ub0, ub0, ub1, ub1);
+        U4[i * R2 + R + r] = make_float4(ug0, ug0, ug1, ug1);
+        C4[i * R + r] = make_float4(c0, c0, c1, c1);
+    }
+    for (int e = tid; e < R * P; e += nthr) {
+        V[e] = to_f(xp[e]);
+        V[R * P + e] = to_f(x[e]);
+    }
+    __syncthreads();
+
+    // 3. rotate + decay, rank-2R update, readout partials -- two columns per instruction
+    const float4* V4 = reinterpret_cast<const float4*>(V);
+    float2 ya[R], yb[R];     // readout partials of columns 4j, 4j+1 and 4j+2, 4j+3
+#pragma unroll
+    for (int r = 0; r < R; ++r) ya[r] = yb[r] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < MAXP; ++k) {
+        if (k < a.ppt) {
+            const int i = rg + k * RG;
+            const float4 rc = rot4[2 * i], rn = rot4[2 * i + 1];
+            // row 2i: ac h0 - as h1;  row 2i+1: as h0 + ac h1
+            float2 n0a = __ffma2_rn(lo2(rc), lo2(v0[k]), __fmul2_rn(lo2(rn), lo2(v1[k])));
+            float2 n0b = __ffma2_rn(lo2(rc), hi2(v0[k]), __fmul2_rn(lo2(rn), hi2(v1[k])));
+            float2 n1a = __ffma2_rn(hi2(rc), lo2(v0[k]), __fmul2_rn(lo2(rc), lo2(v1[k])));
+            float2 n1b = __ffma2_rn(hi2(rc), hi2(v0[k]), __fmul2_rn(lo2(rc), hi2(v1[k])));
+#pragma unroll
+            for (int q = 0; q < R2; ++q) {
+                const float4 u = U4[i * R2 + q];
+                const float4 v = V4[q * CPR + j];
+                n0a = __ffma2_rn(lo2(u), lo2(v), n0a);
+                n0b = __ffma2_rn(lo2(u), hi2(v), n0b);
+                n1a = __ffma2_rn(hi2(u), lo2(v), n1a);
+                n1b = __ffma2_rn(hi2(u), hi2(v), n1b);
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float4 c = C4[i * R + r];
+                ya[r] = __ffma2_rn(n0a, lo2(c), __ffma2_rn(n1a, hi2(c), ya[r]));
+                yb[r] = __ffma2_rn(n0b, lo2(c), __ffma2_rn(n1b, hi2(c), yb[r]));
+            }
+            __stcs(hrow + (size_t)(2 * i) * CPR + j, make_float4(n0a.x, n0a.y, n0b.x, n0b.y));
+            __stcs(hrow + (size_t)(2 * i + 1) * CPR + j, make_float4(n1a.x, n1a.y, n1b.x, n1b.y));
+        }
+    }
+
+    // 4. the readout's sum over N: row groups sharing a warp by shuffles, the rest through
+    //    shared memory
+    if (WR > 1) {
+        for (int off = CPR; off < 32; off <<= 1)
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                ya[r].x += __shfl_xor_sync(0xffffffffu, ya[r].x, off);
+                ya[r].y += __shfl_xor_sync(0xffffffffu, ya[r].y, off);
+                yb[r].x += __shfl_xor_sync(0xffffffffu, yb[r].x, off);
+                yb[r].y += __shfl_xor_sync(0xffffffffu, yb[r].y, off);
+            }
+    }
+    if (rg % WR == 0) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            *reinterpret_cast<float4*>(ypart + ((size_t)(rg / WR) * R + r) * P + 4 * j) =
+                make_float4(ya[r].x, ya[r].y, yb[r].x, yb[r].y);
+    }
+    __syncthreads();
+    const float Dh = a.D ? a.D[h] : 0.f;
+    IO* y = static_cast<IO*>(a.y) + (size_t)bh * R * P;
+    IO* xpo = static_cast<IO*>(a.x_prev) + (size_t)bh * R * P;
+    for (int e = tid; e < R * P; e += nthr) {
+        float acc = 0.f;
+        for (int w = 0; w < RGW; ++w) acc += ypart[(size_t)w * R * P + e];
+        float v = acc + Dh * V[R * P + e];
+        if (a.z) v = gate_silu(v, to_f(static_cast<const IO*>(a.z)[(size_t)bh * R * P + e]));
+        y[e] = from_f<IO>(v);
+        xpo[e] = x[e];   // x_prev <- x (this head only; read above before the barrier)
+    }
+}
+
+template <typename IO, int R, bool BCM>
+static cudaError_t launch_decode_mimo(const DecodeArgs& a, int batch, cudaStream_t s) {
+    const int RG = (a.N / 2) / a.ppt;
+    const int threads = (a.P / 4) * RG;
+    const size_t smem = sizeof(float) * mimo_smem_floats(a.N, a.P, R, a.ppt, BCM);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(decode_mimo_kernel<IO, R, 8, BCM>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    decode_mimo_kernel<IO, R, 8, BCM><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+// SISO: the plain kernel with 8 (or 4) pairs per thread.  MIMO: the rank-2R packed kernel
+// when the shape takes 8 pairs per thread, else the plain kernel with 4.
 template <typename IO, bool BCM>
 static cudaError_t launch_decode_io(const DecodeArgs& a, int batch, int R, cudaStream_t s) {
-    if (a.ppt > 8 || (a.ppt > 4 && R != 1)) return cudaErrorNotSupported;
+    if (a.ppt > 8) return cudaErrorNotSupported;
+    if (R != 1 && a.ppt == 8) {
+        switch (R) {
+            case 2: return launch_decode_mimo<IO, 2, BCM>(a, batch, s);
+            case 3: return launch_decode_mimo<IO, 3, BCM>(a, batch, s);
+            case 4: return launch_decode_mimo<IO, 4, BCM>(a, batch, s);
+            case 8: return launch_decode_mimo<IO, 8, BCM>(a, batch, s);
+            default: return cudaErrorNotSupported;
+        }
+    }
+    if (a.ppt > 4 && R != 1) return cudaErrorNotSupported;
     switch (R) {
         case 1: return a.ppt > 4 ? launch_decode_t<IO, 1, 8, BCM>(a, batch, s)
                                  : launch_decode_t<IO, 1, 4, BCM>(a, batch, s);

@@ -63,6 +63,15 @@ bool simt_shape(int N, int P, int* ppt, int* ns) {
 bool decode_shape(int N, int P, int R, int* ppt) {
     if (P % 4 || P > 256 || N > 256) return false;
     const int pairs = N / 2, cpr = P / 4;
+    // MIMO: 8 pairs per thread in the rank-2R packed kernel, with whole warps of at least 64
+    // threads (batch 256, N 64, R 4: see the decode notes)
+    if (R != 1 && pairs % 8 == 0) {
+        const int threads = cpr * (pairs / 8);
+        if (threads >= 64 && threads <= 512 && threads % 32 == 0) {
+            *ppt = 8;
+            return true;
+        }
+    }
     for (int c : {8, 4, 2, 1}) {
         if (pairs % c || (c == 8 && R != 1)) continue;
         const int threads = cpr * (pairs / c);
