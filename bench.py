@@ -2,8 +2,11 @@
 
 One step = one m3_scan_fwd call over the SISO 1.5B-scale prefill workload
 (batch 8, 64 heads, T 4096, P 64, N 128, chunk 64, bf16 x/B/C, fp32 dt/A/lam/theta/state),
-i.e. every prefill step of the method.  Alongside, the batch-256 decode workloads
-(SISO N 128 and MIMO R 4 N 64; 1000 sequential tokens) are timed as a sub-metric.
+i.e. every prefill step of the method.  Alongside, as sub-metrics: the batch-256 decode
+workloads (SISO N 128 and MIMO R 4 N 64; 1024 sequential tokens, the 32-token pool captured
+once as a CUDA graph and replayed), the same prefill and decode with the fused output gate
+("gated") and with BCNorm + BC biases ("bc"), the end-to-end call through pinned host
+buffers ("e2e"), and the CPU oracle on the workload's inputs ("cpu_baseline").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 

@@ -15,6 +15,8 @@
  *   MIMO ("Multi-Input, Multi-Output Formulation"): B_t, C_t are N x R and x_t is
  *     P x R; the input term is a rank-R sum and the readout is P x R:
  *     Y_t = h_t^T C_t + D x_t   (D is a per-head scalar skip; SISO is R = 1)
+ *   Optional fused parts (m3_extras, the *_ex and *_gated entry points): the output
+ *     gate y * SiLU(z), and BCNorm with head-specific BC biases on B and C.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
