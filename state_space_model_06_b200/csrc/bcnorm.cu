@@ -7,6 +7,10 @@
 // warps.  This prologue computes every scale of the call once (one warp per column; B and
 // C are read once more, about 3 % of the call's bytes at the 1.5B-scale shapes) into the
 // workspace, where the kernels read them as one float per token and rank column.
+//
+// Layout (floats): B scales [b][G][R][Tp], then C scales [b][G][R][Tp], then B_prev scales
+// [b][G][R]; Tp = T rounded up to a multiple of 4, so that every row of tokens starts on
+// 16 bytes and the tensor-core kernel can fetch a sub-chunk's scales with one TMA copy.
 #include "m3_internal.h"
 
 namespace m3 {
@@ -18,6 +22,7 @@ __global__ void __launch_bounds__(256) bc_scale_kernel(const IO* __restrict__ B,
                                                        const IO* __restrict__ C,
                                                        const IO* __restrict__ B_prev,
                                                        long long cols, long long prev_cols, int N,
+                                                       long long T, long long Tp, int GR,
                                                        float eps, float* __restrict__ out) {
     const long long total = 2 * cols + prev_cols;
     const int lane = threadIdx.x & 31;
@@ -32,7 +37,18 @@ __global__ void __launch_bounds__(256) bc_scale_kernel(const IO* __restrict__ B,
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane == 0) out[col] = rsqrtf(ss / (float)N + eps);
+        if (lane == 0) {
+            long long o;
+            if (col < 2 * cols) {
+                // input column c = (b T + t) GR + gr  ->  output ((b GR + gr) Tp + t)
+                const long long c = col < cols ? col : col - cols;
+                const long long gr = c % GR, bt = c / GR, t = bt % T, b = bt / T;
+                o = (col < cols ? 0 : cols / T * Tp) + (b * GR + gr) * Tp + t;
+            } else {
+                o = 2 * (cols / T) * Tp + (col - 2 * cols);
+            }
+            out[o] = rsqrtf(ss / (float)N + eps);
+        }
     }
 }
 
@@ -45,14 +61,15 @@ cudaError_t launch_t(const ScanArgs& a, int R, float eps, float* out, cudaStream
     if (blocks > 148 * 16) blocks = 148 * 16;
     bc_scale_kernel<IO><<<(unsigned)blocks, 256, 0, s>>>(
         static_cast<const IO*>(a.B), static_cast<const IO*>(a.C),
-        static_cast<const IO*>(a.B_prev), cols, prev_cols, a.N, eps, out);
+        static_cast<const IO*>(a.B_prev), cols, prev_cols, a.N, (long long)a.T,
+        (long long)bc_tpad(a.T), a.G * R, eps, out);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t bc_scale_floats(int batch, long long T, int G, int R) {
-    return (size_t)(2 * (long long)batch * T * G * R + (long long)batch * G * R);
+    return (size_t)(2 * (long long)batch * G * R * bc_tpad(T) + (long long)batch * G * R);
 }
 
 cudaError_t launch_bc_scales(const ScanArgs& a, int R, int io_dtype, float eps, float* out,

@@ -74,7 +74,7 @@ struct ScanArgs {
     const float* B_bias; // [H][N]: BC bias of B, or null
     const float* C_bias; // [H][N]: BC bias of C, or null
     // BCNorm scales 1 / sqrt(mean_n v^2 + eps) (workspace; null when off), one per column:
-    // B [b][T][G][R], then C [b][T][G][R], then B_prev [b][G][R]
+    // B [b][G][R][Tp], then C [b][G][R][Tp], then B_prev [b][G][R] (Tp: T rounded up to 4)
     const float* bc_scale;
     bool bc;             // any BC map (bias or normalisation) is applied
     uint32_t* status;    // workspace status word (may be null)

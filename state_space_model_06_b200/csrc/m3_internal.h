@@ -21,7 +21,8 @@ size_t scan_tc_workspace_bytes(int batch, int H, int N, int P, int R, long long 
 cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s);
 
 // BCNorm scales of every B, C and B_prev column of a prefill call into a.bc_scale
-// (floats: b*T*G*R for B, the same for C, then b*G*R for B_prev).
+// (floats: B [b][G][R][Tp], C [b][G][R][Tp], then B_prev [b][G][R]; Tp = bc_tpad(T)).
+__host__ __device__ inline long long bc_tpad(long long T) { return (T + 3) / 4 * 4; }
 size_t bc_scale_floats(int batch, long long T, int G, int R);
 cudaError_t launch_bc_scales(const ScanArgs& a, int R, int io_dtype, float eps, float* out,
                              cudaStream_t s);

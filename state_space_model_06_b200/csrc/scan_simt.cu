@@ -52,10 +52,12 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
     // columns start at sB (B), sC (C) and sP (B_prev); null scales mean 1
     const float* Bb = a.B_bias ? a.B_bias + (size_t)h * N : nullptr;
     const float* Cb = a.C_bias ? a.C_bias + (size_t)h * N : nullptr;
-    const size_t ncol = (size_t)a.batch * T * G * R;
-    const float* sB = a.bc_scale;
-    const float* sC = a.bc_scale ? a.bc_scale + ncol : nullptr;
-    const float* sP = a.bc_scale ? a.bc_scale + 2 * ncol : nullptr;
+    const long long Tp = (T + 3) / 4 * 4;
+    const size_t ncol = (size_t)a.batch * G * R * Tp;
+    // this (batch, group)'s rows of scales: B [R][Tp], C [R][Tp]; B_prev [R]
+    const float* sB = a.bc_scale ? a.bc_scale + ((size_t)b * G + g) * R * Tp : nullptr;
+    const float* sC = a.bc_scale ? sB + ncol : nullptr;
+    const float* sP = a.bc_scale ? a.bc_scale + 2 * ncol + ((size_t)b * G + g) * R : nullptr;
 
     // previous token of the first step comes from the carried state (buffer 1)
     {
@@ -64,7 +66,7 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
         for (int e = tid; e < R * P; e += nthr) buf1[e] = to_f(xp[e]);
         for (int e = tid; e < R * N; e += nthr) {
             const int r = e / N;
-            const float sc = sP ? sP[((size_t)b * G + g) * R + r] : 1.f;
+            const float sc = sP ? sP[r] : 1.f;
             buf1[R * P + e] = a.bc ? bc_apply(to_f(bp[e]), sc, Bb, e - r * N) : to_f(bp[e]);
         }
     }
@@ -86,9 +88,9 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
         if (a.bc) {
             for (int e = tid; e < R * N; e += nthr) {
                 const int r = e / N, n = e - r * N;
-                const size_t col = (bt * G + g) * R + r;
-                cur[R * P + e] = bc_apply(to_f(Bt[e]), sB ? sB[col] : 1.f, Bb, n);
-                cur[R * P + R * N + e] = bc_apply(to_f(Ct[e]), sC ? sC[col] : 1.f, Cb, n);
+                const size_t si = (size_t)r * Tp + t;
+                cur[R * P + e] = bc_apply(to_f(Bt[e]), sB ? sB[si] : 1.f, Bb, n);
+                cur[R * P + R * N + e] = bc_apply(to_f(Ct[e]), sC ? sC[si] : 1.f, Cb, n);
             }
         } else {
             for (int e = tid; e < R * N; e += nthr) {

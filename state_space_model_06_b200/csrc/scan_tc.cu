@@ -129,7 +129,12 @@ struct Cfg {
         return SL_BYTES + G_BYTES + 2 * 3 * DT_BYTES + kCoefSlots * COEF_FLOATS * 4 +
                2 * TSPLIT * PAIRS * 4 + NUM_BARS * 8 + 64;
     }
-    static constexpr int raw_bytes(int rt) { return rt * R * NST * 2 * 2 + rt * PAIRS * 4; }
+    // a raw stage: B, C (bf16), theta (fp32) and the BCNorm scales of B and C (fp32, [2][R][rt],
+    // padded to 128 bytes; fetched only with BCNorm)
+    static constexpr int sc_bytes(int rt) { return (2 * R * rt * 4 + 127) / 128 * 128; }
+    static constexpr int raw_bytes(int rt) {
+        return rt * R * NST * 2 * 2 + rt * PAIRS * 4 + sc_bytes(rt);
+    }
     static constexpr int kSmemLimit = 232448 - 1024;            // minus base alignment slack
     // with the output gate, every x / y stage has a z tile beside it
     static constexpr int XZ_BYTES = (GT ? 2 : 1) * X_BYTES;
@@ -154,7 +159,10 @@ struct Cfg {
     static constexpr int TPT = RT / TSPLIT;                     // tokens per rotation thread
     static constexpr int BRAW_BYTES = RT * R * NST * 2;
     static constexpr int TH_BYTES = RT * PAIRS * 4;
-    static constexpr int RAW_BYTES = 2 * BRAW_BYTES + TH_BYTES;
+    static constexpr int SC_OFF = 2 * BRAW_BYTES + TH_BYTES;    // BCNorm scales in a raw stage
+    static constexpr int SC_BOX = 2 * R * RT * 4;               // bytes the scale copy delivers
+    static constexpr int RAW_BYTES = SC_OFF + sc_bytes(RT);
+    static_assert(SC_OFF % 128 == 0 && RAW_BYTES % 128 == 0, "TMA destinations must be aligned");
 
     // shared memory offsets (SW128 tiles first, 1024-byte aligned)
     static constexpr int OFF_X = 0;                                   // [XST] x / y staging
@@ -196,7 +204,7 @@ struct Cfg {
 };
 
 struct TcParams {
-    CUtensorMap tm_x, tm_y, tm_z, tm_B, tm_C, tm_th, tm_dt, tm_A, tm_lam;
+    CUtensorMap tm_x, tm_y, tm_z, tm_B, tm_C, tm_th, tm_dt, tm_A, tm_lam, tm_sc;
     ScanArgs a;
     int nchunks;
     unsigned long long limit_ns;
@@ -252,7 +260,7 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int k, uint32_t lbo) 
 }
 
 // ---------------------------------------------------------------------------------
-template <int NST, int Q, int R, bool GT>
+template <int NST, int Q, int R, bool GT, bool BC>
 __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab);
 
 // ---------------------------------------------------------------------------------
@@ -342,13 +350,11 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
     // BC map ("Technical Approach", BCNorm and BC biases): B and C of this thread's pair
     // channels become v * s + bias, s the column's BCNorm scale (1 when off), bias the head's
     constexpr bool bc = BC;
-    const int hh = blockIdx.x % a.H, bq = blockIdx.x / a.H, gq = hh / (a.H / a.G);
+    const int hh = blockIdx.x % a.H;
     float bb0 = 0.f, bb1 = 0.f, cb0 = 0.f, cb1 = 0.f;
     if (a.B_bias) { bb0 = a.B_bias[hh * NST + 2 * pair]; bb1 = a.B_bias[hh * NST + 2 * pair + 1]; }
     if (a.C_bias) { cb0 = a.C_bias[hh * NST + 2 * pair]; cb1 = a.C_bias[hh * NST + 2 * pair + 1]; }
-    const size_t ncol = (size_t)a.batch * a.T * a.G * R;
-    const float* sBq = a.bc_scale ? a.bc_scale + ((size_t)bq * a.T * a.G + gq) * R : nullptr;
-    const size_t sstride = (size_t)a.G * R;          // between consecutive tokens
+    const bool has_sc = a.bc_scale != nullptr;       // BCNorm scales come with the raw stage
     // call-relative angle of this thread's pair (the RoPE frame of Proposition 4 starts at
     // the first token of the call), reduced mod 2 pi at chunk boundaries
     float psi_acc = 0.f;
@@ -396,20 +402,18 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                     bv[jj][r] = braw[e];
                     cv[jj][r] = craw[e];
                 }
-            // BCNorm scales of the own tokens (1 past the end of the call: those rows are
-            // zero-filled and masked out)
+            // BCNorm scales of the own tokens, [2][R][RT] in the raw stage (0 past the end
+            // of the call, where B and C are zero-filled and the rows are masked out)
             float sb[TPT][R], sc[TPT][R];
             if constexpr (bc) {
+                const float* scs = reinterpret_cast<const float*>(raw + C::SC_OFF);
 #pragma unroll
-                for (int jj = 0; jj < TPT; ++jj) {
-                    const long long t = (long long)c * Q + tb + j0 + jj;
+                for (int jj = 0; jj < TPT; ++jj)
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
-                        const bool in = sBq && t < a.T;
-                        sb[jj][r] = in ? sBq[(size_t)t * sstride + r] : 1.f;
-                        sc[jj][r] = in ? sBq[ncol + (size_t)t * sstride + r] : 1.f;
+                        sb[jj][r] = has_sc ? scs[r * C::RT + j0 + jj] : 1.f;
+                        sc[jj][r] = has_sc ? scs[(R + r) * C::RT + j0 + jj] : 1.f;
                     }
-                }
             }
             if (!warp_wait(&bar[RS0 + rs], (raw_it >> 1) & 1, ab)) return;
             if (tid == 0) M3_TRACE_EV(c, s == 0 ? 28 : 31);
@@ -785,9 +789,9 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
         const __nv_bfloat16* bp =
             static_cast<const __nv_bfloat16*>(a.B_prev) + ((size_t)b * a.G + g) * R * NST;
         // the carried previous token's B goes through the BC map as well
-        const float* sP = a.bc_scale
-                              ? a.bc_scale + 2 * (size_t)a.batch * T * a.G * R + ((size_t)b * a.G + g) * R
-                              : nullptr;
+        const float* sP =
+            a.bc_scale ? a.bc_scale + 2 * (size_t)a.batch * a.G * R * bc_tpad(T) + ((size_t)b * a.G + g) * R
+                       : nullptr;
         const float* Bb = a.B_bias ? a.B_bias + (size_t)h * NST : nullptr;
 #pragma unroll 1
         for (int cb = 0; cb < kNCols; cb += 16) {
@@ -897,7 +901,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
     }
 }
 
-template <int NST, int Q, int R, bool GT>
+template <int NST, int Q, int R, bool GT, bool BC>
 __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
@@ -923,12 +927,15 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
             const int rs = raw_it & 1;
             if (!(ok = mbar_wait(&bar[RAW_EMPTY0 + rs], ((raw_it >> 1) & 1) ^ 1, ab))) break;
             if (s == 0) M3_TRACE_EV(c, 25);
-            mbar_arrive_expect_tx(&bar[RAW_FULL0 + rs], C::RAW_BYTES);
+            const bool sc = BC && a.bc_scale != nullptr;
+            mbar_arrive_expect_tx(&bar[RAW_FULL0 + rs], C::SC_OFF + (sc ? C::SC_BOX : 0));
             uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
             const int tr = t0 + s * C::RT;
             tma_load_5d(raw, &p.tm_B, &bar[RAW_FULL0 + rs], 0, 0, g, tr, b);
             tma_load_5d(raw + C::BRAW_BYTES, &p.tm_C, &bar[RAW_FULL0 + rs], 0, 0, g, tr, b);
             tma_load_4d(raw + 2 * C::BRAW_BYTES, &p.tm_th, &bar[RAW_FULL0 + rs], 0, g, tr, b);
+            if (sc)   // BCNorm scales of B and C for these tokens: x = token (RT-aligned)
+                tma_load_5d(raw + C::SC_OFF, &p.tm_sc, &bar[RAW_FULL0 + rs], tr, 0, g, b, 0);
             ++n_raw[rs];
         }
     }
@@ -1013,7 +1020,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.a.status, p.limit_ns};
 
     if (w == 0) {
-        if ((threadIdx.x & 31) == 0) producer<NST, Q, R, GT>(p, sm, bar, ab);
+        if ((threadIdx.x & 31) == 0) producer<NST, Q, R, GT, BC>(p, sm, bar, ab);
     } else if (w == 1) {
         if ((threadIdx.x & 31) == 0) {
             mma_issuer<NST, Q, R, GT>(p, sm, bar, tmem, ab);
@@ -1124,6 +1131,16 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
         ok &= make_map(&p.tm_A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.A, d, st, box,
                        CU_TENSOR_MAP_SWIZZLE_NONE);
         ok &= make_map(&p.tm_lam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.lam, d, st, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    if (BC && a.bc_scale) {
+        // BCNorm scales: (token, R, G, b, {B, C}) with rows of Tp tokens, box (RT, R, 1, 1, 2).
+        // The token extent is T: the copy zero-fills past the end of the call.
+        const uint64_t Tp = (uint64_t)bc_tpad(a.T);
+        const uint64_t d[5] = {T, (uint64_t)R, G, Bn, 2};
+        const uint64_t st[4] = {Tp * 4, (uint64_t)R * Tp * 4, G * R * Tp * 4, Bn * G * R * Tp * 4};
+        const uint32_t box[5] = {(uint32_t)C::RT, (uint32_t)R, 1, 1, 2};
+        ok &= make_map(&p.tm_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, a.bc_scale, d, st, box,
                        CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     if (!ok) return cudaErrorInvalidValue;
