@@ -5,7 +5,8 @@ One step = one m3_scan_fwd call over the SISO 1.5B-scale prefill workload
 i.e. every prefill step of the method.  Alongside, as sub-metrics: the batch-256 decode
 workloads (SISO N 128 and MIMO R 4 N 64; 1024 sequential tokens, the 32-token pool captured
 once as a CUDA graph and replayed), the same prefill and decode with the fused output gate
-("gated") and with BCNorm + BC biases ("bc"), the end-to-end call through pinned host
+("gated") and with BCNorm + BC biases ("bc"), the MIMO rank-4 prefill plain and with the
+lightweight expansion of x and z ("mimo"), the end-to-end call through pinned host
 buffers ("e2e"), and the CPU oracle on the workload's inputs ("cpu_baseline").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -354,6 +355,37 @@ def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False, bc=F
                        "distinct_tokens": DECODE_POOL}}
 
 
+def mimo_leg(args, dev, stream, rank, ws_world, pk):
+    """The MIMO prefill workload (rank 4, N 64, 32-token tiles): plain, with the
+    lightweight expansion of x (x read as [b][T][H][P]), and with the expansion of x and z
+    plus the fused gate.  Algorithmic bytes count each tensor as the call reads it."""
+    w = inputs.WORKLOADS["mimo_prefill_r4"]
+    inp, d, g, st, y, ws = prefill_setup(w, dev, seed=200 + rank)
+    del inp
+    byts, _ = scan_algorithmic(w)
+    b, T, H, R, P = w.batch, w.seqlen, w.nheads, w.rank, w.headdim
+    xio = b * T * H * P * 2                      # one bf16 value per head channel and token
+    x1 = g["x"][:, :, :, 0, :].contiguous()
+    wx, wz = (v.to(dev) for v in inputs.make_expand(H, R, P, seed=200 + rank))
+    z1 = inputs.make_gate((b, T, H, P), io_dtype=w.io_dtype, seed=200 + rank).to(dev)
+    legs = (("prefill", g["x"], None, byts),
+            ("prefill_expanded", x1, m3.Extras(x_expand=wx), byts - xio * (R - 1)),
+            ("prefill_expanded_gated", x1, m3.Extras(z=z1, x_expand=wx, z_expand=wz),
+             byts - xio * (R - 1) + xio))
+    out = {}
+    for key, x, ex, nbytes in legs:
+        gx = dict(g)
+        gx["x"] = x
+        ms = time_prefill_ex(w, d, gx, ex, st, y, ws, min(args.steps, 20), 3, stream)
+        val, ms_max = job_throughput(b * T, ms, ws_world)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[key] = {"tokens_per_s": val, "ms_per_step": ms_max, "alg_bytes_per_step": nbytes,
+                    "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"]}
+    out["config"] = {"workload": w.name, "batch": b, "heads": H, "seqlen": T, "headdim": P,
+                     "dstate": w.dstate, "rank": R, "chunk": w.chunk}
+    return out
+
+
 def w_dec_batch(name):
     return inputs.WORKLOADS[name].batch
 
@@ -437,7 +469,7 @@ def ours(args):
     }
 
     if args.prefill_only:
-        args.no_decode = args.no_e2e = args.no_cpu = args.no_gate = True
+        args.no_decode = args.no_e2e = args.no_cpu = args.no_gate = args.no_mimo = True
     if not args.no_decode:
         line["decode"] = {}
         for name in (args.decode or DECODES):
@@ -489,6 +521,9 @@ def ours(args):
                 r["tokens_per_s"], _ = job_throughput(w_dec_batch(name), r["us_per_step"] / 1e3,
                                                       ws_world)
                 line["bc"][name] = r
+
+    if not args.no_mimo:
+        line["mimo"] = mimo_leg(args, dev, stream, rank, ws_world, pk)
 
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_prefill_e2e(w, d, inp, st, ws, min(args.steps, 5), stream, dev)
@@ -553,6 +588,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-gate", action="store_true", help="skip the fused-output-gate legs")
+    ap.add_argument("--no-mimo", action="store_true", help="skip the MIMO prefill legs")
     ap.add_argument("--cpu-rows", type=int, default=8,
                     help="batch rows of the workload timed on the CPU oracle (default: all)")
     ap.add_argument("--ref-tokens", type=int, default=256)

@@ -16,7 +16,8 @@
  *     P x R; the input term is a rank-R sum and the readout is P x R:
  *     Y_t = h_t^T C_t + D x_t   (D is a per-head scalar skip; SISO is R = 1)
  *   Optional fused parts (m3_extras, the *_ex and *_gated entry points): the output
- *     gate y * SiLU(z), and BCNorm with head-specific BC biases on B and C.
+ *     gate y * SiLU(z), BCNorm with head-specific BC biases on B and C, and the MIMO
+ *     lightweight expansion of x and z from P to P x R values per head.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
@@ -115,14 +116,27 @@ m3_status m3_state_init(const m3_dims* dims, m3_state* state, const float* h0, v
  *   bc_norm_eps BCNorm ("Technical Approach", BC normalisation): > 0 scales each token's
  *               B and C rank columns (and B_prev's) to unit RMS over N before the bias,
  *               v / sqrt(mean_n v^2 + eps); 0: off; negative or NaN: M3_ERR_SHAPE.
+ *   x_expand    MIMO lightweight expansion of the input ("Multi-Input, Multi-Output (MIMO)
+ *               Formulation", MIMO Parameterization Choices): [H][R][P] fp32, 16-byte
+ *               aligned, a data-independent per-head vector.  When set, x holds one value
+ *               per head channel, [b][T][H][P] (decode [b][H][P]), and the recurrence uses
+ *               X[r][p] = x[p] * x_expand[h][r][p], rounded to the io dtype (the value an
+ *               expanded io-dtype x would hold).  NULL: x is [..][H][R][P] as stated above.
+ *   z_expand    the same for the gate: z is [b][T][H][P] (decode [b][H][P]) and the gate
+ *               uses Z[r][p] = z[p] * z_expand[h][r][p], rounded to the io dtype.  Needs z
+ *               (M3_ERR_NULL without it).  NULL: z has the layout of y.
  *
- * The state keeps the raw previous-token B; the map is applied wherever it is used.
+ * The state keeps the raw previous-token B; the map is applied wherever it is used.  With
+ * x_expand, state.x_prev holds the expanded previous token X [b][H][R][P], so a state
+ * moves unchanged between expanded and unexpanded calls.  y is always [..][H][R][P].
  */
 typedef struct {
     const void* z;
     const float* B_bias;
     const float* C_bias;
     float bc_norm_eps;
+    const float* x_expand;
+    const float* z_expand;
 } m3_extras;
 
 /* Workspace bytes m3_scan_fwd needs for (dims, seqlen, chunk); at least 256

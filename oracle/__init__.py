@@ -65,6 +65,9 @@ def _load(path=None):
         lib.m3o_max_threads.restype = ctypes.c_int
         lib.m3o_gate.argtypes = [ctypes.c_int64, dp, dp]
         lib.m3o_gate.restype = None
+        lib.m3o_expand.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   dp, dp, dp]
+        lib.m3o_expand.restype = None
         _libs[path] = lib
     return _libs[path]
 
@@ -84,9 +87,24 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double)) if a is not None else None
 
 
+def expand(v, w, lib_path=None):
+    """MIMO lightweight expansion: v [..., H, P] times w [H, R, P] gives [..., H, R, P]
+    with out[..., h, r, p] = v[..., h, p] * w[h, r, p] (float64)."""
+    w = np.asarray(w)
+    H, R, P = w.shape
+    v = np.asarray(v)
+    lead = v.shape[:-2]
+    v = _f64(v, tuple(lead) + (H, P), "expanded input")
+    w = _f64(w, (H, R, P), "expansion weights")
+    out = np.zeros(tuple(lead) + (H, R, P))
+    rows = int(np.prod(lead)) if lead else 1
+    _load(lib_path).m3o_expand(rows, H, R, P, _ptr(v), _ptr(w), _ptr(out))
+    return out
+
+
 def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
          theta_is_angle: bool = False, nthreads: int = 0, lib_path=None, z=None,
-         B_bias=None, C_bias=None, bc_eps: float = 0.0):
+         B_bias=None, C_bias=None, bc_eps: float = 0.0, x_expand=None, z_expand=None):
     """Run the recurrence over T tokens.
 
     Shapes: x [b,T,H,R,P]; B, C [b,T,G,R,N]; dt, A, lam [b,T,H];
@@ -97,9 +115,17 @@ def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
     B_bias, C_bias [H,N] or None and bc_eps > 0: BC biases and BC normalisation
     ("Technical Approach", BCNorm and BC biases): per token, each rank column of B and
     C is scaled to unit RMS over N (when bc_eps > 0), then the head's bias is added.
+    x_expand / z_expand [H,R,P] or None: MIMO lightweight expansion ("Multi-Input,
+    Multi-Output (MIMO) Formulation", MIMO Parameterization Choices); x (z) is then
+    [b,T,H,P] and the recurrence uses expand(x, x_expand) (the gate expand(z, z_expand)).
+    x_prev stays the expanded [b,H,R,P] previous input.
 
     Returns (y [b,T,H,R,P], h_T, x_prev_out, B_prev_out), all float64.
     """
+    if x_expand is not None:
+        x = expand(x, x_expand, lib_path)
+    if z is not None and z_expand is not None:
+        z = expand(z, z_expand, lib_path)
     x = np.asarray(x)
     b, T, H, R, P = x.shape
     G, N = np.asarray(B).shape[2], np.asarray(B).shape[4]
@@ -138,9 +164,9 @@ def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
 
 def decode_step(x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev,
                 theta_is_angle: bool = False, nthreads: int = 0, z=None, B_bias=None,
-                C_bias=None, bc_eps: float = 0.0):
-    """One decode token: x [b,H,R,P], B/C [b,G,R,N], dt/A/lam [b,H], theta [b,G,N/2];
-    z [b,H,R,P] or None (output gate).
+                C_bias=None, bc_eps: float = 0.0, x_expand=None, z_expand=None):
+    """One decode token: x [b,H,R,P] ([b,H,P] with x_expand), B/C [b,G,R,N], dt/A/lam
+    [b,H], theta [b,G,N/2]; z [b,H,R,P] ([b,H,P] with z_expand) or None (output gate).
 
     Identical to ``scan`` with T = 1; returns (y [b,H,R,P], h, x_prev, B_prev).
     """
@@ -148,5 +174,5 @@ def decode_step(x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev,
     y, h, xp, bp = scan(*ins, D=D, h0=h, x_prev=x_prev, B_prev=B_prev,
                         theta_is_angle=theta_is_angle, nthreads=nthreads,
                         z=None if z is None else np.asarray(z)[:, None], B_bias=B_bias,
-                        C_bias=C_bias, bc_eps=bc_eps)
+                        C_bias=C_bias, bc_eps=bc_eps, x_expand=x_expand, z_expand=z_expand)
     return y[:, 0], h, xp, bp

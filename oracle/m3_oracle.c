@@ -35,6 +35,12 @@
  *   state channel n, shared by the rank columns) is added.  The carried previous
  *   token's B is kept raw in the state and goes through the same map when used.
  *
+ *   MIMO lightweight expansion ("Multi-Input, Multi-Output (MIMO) Formulation", MIMO
+ *   Parameterization Choices), in m3o_expand: the per-head input x (and gate z) has P
+ *   values per token; a learned data-independent vector w [H][R][P] scales it element-wise
+ *   to the rank-R input, X[r][p] = x[p] * w[h][r][p], which then enters the recurrence
+ *   (and the skip) like any MIMO input.
+ *
  *   Sequence start ("Parallel representation under SSD"): the unrolling starts
  *   from h_0 = gamma_0 B_0 x_0, i.e. a fresh state has h = 0 and no previous
  *   token (x_{-1} = 0, B_{-1} = 0).  Across calls the previous token (x, B) is
@@ -212,6 +218,19 @@ int m3o_decode(const m3o_dims* d, uint32_t flags, const double* x, const double*
 {
     return m3o_scan(d, 1, flags, x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev, y,
                     nthreads);
+}
+
+/* out[row][h][r][p] = in[row][h][p] * w[h][r][p] for rows of H heads: the lightweight
+ * expansion of a per-head P-vector to the P x R MIMO input (or gate). */
+void m3o_expand(int64_t rows, int H, int R, int P, const double* in, const double* w,
+                double* out)
+{
+    for (int64_t i = 0; i < rows; ++i)
+        for (int h = 0; h < H; ++h)
+            for (int r = 0; r < R; ++r)
+                for (int p = 0; p < P; ++p)
+                    out[((i * H + h) * R + r) * P + p] =
+                        in[(i * H + h) * P + p] * w[((size_t)h * R + r) * P + p];
 }
 
 /* y[i] <- y[i] * SiLU(z[i]) for n elements: the output gate on the readout (skip included). */

@@ -18,6 +18,14 @@
 
 namespace m3 {
 
+// Gate input of output element e = r * P + p of head h (bh = batch * H + h): z [b][H][R][P],
+// or with the MIMO lightweight expansion z [b][H][P] times the head's weights z_expand[h][r][p].
+template <typename IO>
+__device__ __forceinline__ float gate_z(const DecodeArgs& a, size_t bh, int h, int R, int P, int e) {
+    const IO* z = static_cast<const IO*>(a.z);
+    if (a.z_expand) return expand_io<IO>(to_f(z[bh * P + e % P]), a.z_expand[(size_t)h * R * P + e]);
+    return to_f(z[bh * R * P + e]);
+}
 
 // MAXP: the largest pairs-per-thread count this instantiation handles (a.ppt <= MAXP); it
 // sizes the per-thread state registers, so each shape only pays for the pairs it uses.
@@ -56,14 +64,16 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     }
 
     // 2. stage this token's small inputs in shared memory
-    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * R * P;
+    // x: [R][P], or one value per channel expanded by the head's weights [R][P]
+    const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
+    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * (wx ? 1 : R) * P;
     const IO* xp = static_cast<const IO*>(a.x_prev) + (size_t)bh * R * P;
     const size_t gofs = ((size_t)b * G + g) * R * N;
     const IO* Bg = static_cast<const IO*>(a.B) + gofs;
     const IO* Bpg = static_cast<const IO*>(a.B_prev) + gofs;
     const IO* Cg = static_cast<const IO*>(a.C) + gofs;
     for (int e = tid; e < R * P; e += blockDim.x) {
-        xs[e] = to_f(x[e]);
+        xs[e] = wx ? expand_io<IO>(to_f(x[e % P]), wx[e]) : to_f(x[e]);
         xps[e] = to_f(xp[e]);
     }
     for (int e = tid; e < R * N; e += blockDim.x) {
@@ -165,9 +175,9 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
         float acc = 0.f;
         for (int k = 0; k < RG; ++k) acc += ypart[(size_t)k * R * P + e];
         float v = acc + Dh * xs[e];
-        if (a.z) v = gate_silu(v, to_f(static_cast<const IO*>(a.z)[(size_t)bh * R * P + e]));
+        if (a.z) v = gate_silu(v, gate_z<IO>(a, bh, h, R, P, e));
         y[e] = from_f<IO>(v);
-        xpo[e] = x[e];   // x_prev <- x (this head only; read above before the barrier)
+        xpo[e] = from_f<IO>(xs[e]);   // x_prev <- X (this head only; exact in the io dtype)
     }
 }
 
@@ -247,7 +257,8 @@ __global__ void __launch_bounds__(512) decode_mimo_kernel(DecodeArgs a) {
     const float alpha = expf(dt * Av);
     const float beta = (1.f - lam) * dt * alpha;
     const float gamma = lam * dt;
-    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * R * P;
+    const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
+    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * (wx ? 1 : R) * P;
     const IO* xp = static_cast<const IO*>(a.x_prev) + (size_t)bh * R * P;
     const size_t gofs = ((size_t)b * G + g) * R * N;
     const IO* Bg = static_cast<const IO*>(a.B) + gofs;
@@ -312,7 +323,7 @@ __global__ void __launch_bounds__(512) decode_mimo_kernel(DecodeArgs a) {
     }
     for (int e = tid; e < R * P; e += nthr) {
         V[e] = to_f(xp[e]);
-        V[R * P + e] = to_f(x[e]);
+        V[R * P + e] = wx ? expand_io<IO>(to_f(x[e % P]), wx[e]) : to_f(x[e]);
     }
     __syncthreads();
 
@@ -377,9 +388,9 @@ __global__ void __launch_bounds__(512) decode_mimo_kernel(DecodeArgs a) {
         float acc = 0.f;
         for (int w = 0; w < RGW; ++w) acc += ypart[(size_t)w * R * P + e];
         float v = acc + Dh * V[R * P + e];
-        if (a.z) v = gate_silu(v, to_f(static_cast<const IO*>(a.z)[(size_t)bh * R * P + e]));
+        if (a.z) v = gate_silu(v, gate_z<IO>(a, bh, h, R, P, e));
         y[e] = from_f<IO>(v);
-        xpo[e] = x[e];   // x_prev <- x (this head only; read above before the barrier)
+        xpo[e] = from_f<IO>(V[R * P + e]);   // x_prev <- X (this head only; exact)
     }
 }
 

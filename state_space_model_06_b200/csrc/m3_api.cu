@@ -196,9 +196,12 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
         !aligned(dt, 4) || !aligned(A, 4) || !aligned(lam, 4) || !aligned(theta, 4) ||
         (D && !aligned(D, 4)) || (z && !aligned(z, 16)) ||
-        (ex && ex->B_bias && !aligned(ex->B_bias, 4)) || (ex && ex->C_bias && !aligned(ex->C_bias, 4)))
+        (ex && ex->B_bias && !aligned(ex->B_bias, 4)) || (ex && ex->C_bias && !aligned(ex->C_bias, 4)) ||
+        (ex && ex->x_expand && !aligned(ex->x_expand, 16)) ||
+        (ex && ex->z_expand && !aligned(ex->z_expand, 16)))
         return M3_ERR_ALIGN;
     if (ex && !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;   // negative or NaN epsilon
+    if (ex && ex->z_expand && !z) return M3_ERR_NULL;           // an expanded gate needs z
     size_t base = 0;
     m3_scan_workspace_bytes(d, seqlen, chunk, &base);
     const size_t need = base + bc_bytes(d, seqlen, ex);
@@ -222,6 +225,8 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
     a.B_bias = ex ? ex->B_bias : nullptr;
     a.C_bias = ex ? ex->C_bias : nullptr;
     a.bc = bc_any(ex);
+    a.x_expand = ex ? ex->x_expand : nullptr;
+    a.z_expand = ex ? ex->z_expand : nullptr;
     a.bc_scale = bc_norm_on(ex) ? reinterpret_cast<const float*>(static_cast<char*>(workspace) + base)
                                 : nullptr;
     a.status = static_cast<uint32_t*>(workspace);
@@ -255,9 +260,12 @@ m3_status decode_impl(const m3_dims* d, const void* x, const void* B, const void
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
         !aligned(dt, 4) || !aligned(A, 4) || !aligned(lam, 4) || !aligned(theta, 4) ||
         (D && !aligned(D, 4)) || (z && !aligned(z, 16)) ||
-        (ex && ex->B_bias && !aligned(ex->B_bias, 4)) || (ex && ex->C_bias && !aligned(ex->C_bias, 4)))
+        (ex && ex->B_bias && !aligned(ex->B_bias, 4)) || (ex && ex->C_bias && !aligned(ex->C_bias, 4)) ||
+        (ex && ex->x_expand && !aligned(ex->x_expand, 16)) ||
+        (ex && ex->z_expand && !aligned(ex->z_expand, 16)))
         return M3_ERR_ALIGN;
     if (ex && !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;
+    if (ex && ex->z_expand && !z) return M3_ERR_NULL;
     int ppt = 0;
     if (!rank_has_kernel(d->rank) || !decode_shape(d->dstate, d->headdim, d->rank, &ppt))
         return M3_ERR_UNSUPPORTED;
@@ -269,6 +277,8 @@ m3_status decode_impl(const m3_dims* d, const void* x, const void* B, const void
     a.B_bias = ex ? ex->B_bias : nullptr;
     a.C_bias = ex ? ex->C_bias : nullptr;
     a.bc_eps = ex ? ex->bc_norm_eps : 0.f;
+    a.x_expand = ex ? ex->x_expand : nullptr;
+    a.z_expand = ex ? ex->z_expand : nullptr;
     a.H = d->nheads; a.G = d->ngroups; a.P = d->headdim; a.N = d->dstate;
     a.ppt = ppt; a.flags = flags;
     cudaError_t e = launch_decode(a, d->batch, d->rank, d->io_dtype, s);

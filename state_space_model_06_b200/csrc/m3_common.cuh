@@ -33,6 +33,12 @@ __device__ __forceinline__ float bc_apply(float v, float s, const float* bias, i
     return fmaf(v, s, bias ? bias[n] : 0.f);
 }
 
+// MIMO lightweight expansion ("Multi-Input, Multi-Output (MIMO) Formulation", MIMO
+// Parameterization Choices): one stored value v of a head channel p times the head's
+// data-independent weight w[r][p] gives rank column r's value, rounded to the io dtype.
+template <typename IO>
+__device__ __forceinline__ float expand_io(float v, float w) { return to_f(from_f<IO>(v * w)); }
+
 // Argument block of one decode step (device pointers, validated on the host).
 struct DecodeArgs {
     const void* x;       // [b][H][R][P] io
@@ -51,6 +57,8 @@ struct DecodeArgs {
     const float* B_bias; // [H][N]: BC bias of B, or null
     const float* C_bias; // [H][N]: BC bias of C, or null
     float bc_eps;        // > 0: RMS-normalise B, B_prev and C columns over N (BCNorm)
+    const float* x_expand;  // [H][R][P]: x is [b][H][P], X[r][p] = x[p] w[h][r][p]; or null
+    const float* z_expand;  // [H][R][P]: z is [b][H][P], likewise; or null
     int H, G, P, N;
     int ppt;             // state pairs per thread
     uint32_t flags;
@@ -77,6 +85,8 @@ struct ScanArgs {
     // B [b][G][R][Tp], then C [b][G][R][Tp], then B_prev [b][G][R] (Tp: T rounded up to 4)
     const float* bc_scale;
     bool bc;             // any BC map (bias or normalisation) is applied
+    const float* x_expand;  // [H][R][P]: x is [b][T][H][P], X[r][p] = x[p] w[h][r][p]; or null
+    const float* z_expand;  // [H][R][P]: z is [b][T][H][P], likewise; or null
     uint32_t* status;    // workspace status word (may be null)
     void* ws;            // workspace (after the status block)
     long long T;

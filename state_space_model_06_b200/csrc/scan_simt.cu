@@ -80,11 +80,17 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
         const float* prv = (t & 1) ? buf0 : buf1;
         __syncthreads();   // token t-1 is done with `cur` (it held token t-2) and cs/sn/scal
         const size_t bt = (size_t)b * T + t;
-        const IO* xt = static_cast<const IO*>(a.x) + (bt * H + h) * R * P;
+        // x of this token: [R][P], or one value per channel expanded by the head's weights
+        const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
+        const IO* xt = static_cast<const IO*>(a.x) + (bt * H + h) * (wx ? 1 : R) * P;
         const IO* Bt = static_cast<const IO*>(a.B) + (bt * G + g) * R * N;
         const IO* Ct = static_cast<const IO*>(a.C) + (bt * G + g) * R * N;
         const float dt = a.dt[bt * H + h];
-        for (int e = tid; e < R * P; e += nthr) cur[e] = to_f(xt[e]);
+        if (wx) {
+            for (int e = tid; e < R * P; e += nthr) cur[e] = expand_io<IO>(to_f(xt[e % P]), wx[e]);
+        } else {
+            for (int e = tid; e < R * P; e += nthr) cur[e] = to_f(xt[e]);
+        }
         if (a.bc) {
             for (int e = tid; e < R * N; e += nthr) {
                 const int r = e / N, n = e - r * N;
@@ -156,8 +162,13 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 float v = yp[r] + Dh * xc[r * P + p];
-                if (a.z)
-                    v = gate_silu(v, to_f(static_cast<const IO*>(a.z)[(bt * H + h) * R * P + r * P + p]));
+                if (a.z) {
+                    const IO* zt = static_cast<const IO*>(a.z);
+                    const float zv = a.z_expand
+                        ? expand_io<IO>(to_f(zt[(bt * H + h) * P + p]), a.z_expand[((size_t)h * R + r) * P + p])
+                        : to_f(zt[(bt * H + h) * R * P + r * P + p]);
+                    v = gate_silu(v, zv);
+                }
                 yt[r * P + p] = from_f<IO>(v);
             }
         }
@@ -172,10 +183,14 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
         }
     }
     if (k == 0 && T > 0) {
-        const IO* xl = static_cast<const IO*>(a.x) + (((size_t)b * T + (T - 1)) * H + h) * R * P;
+        // x_prev <- X_{T-1}: the expanded value when x comes with expansion weights
+        const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
+        const IO* xl =
+            static_cast<const IO*>(a.x) + (((size_t)b * T + (T - 1)) * H + h) * (wx ? 1 : R) * P;
         IO* xpo = static_cast<IO*>(a.x_prev) + (size_t)bh * R * P;
 #pragma unroll
-        for (int r = 0; r < R; ++r) xpo[r * P + p] = xl[r * P + p];
+        for (int r = 0; r < R; ++r)
+            xpo[r * P + p] = wx ? from_f<IO>(to_f(xl[p]) * wx[r * P + p]) : xl[r * P + p];
     }
 }
 

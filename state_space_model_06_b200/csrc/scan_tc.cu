@@ -80,7 +80,7 @@ enum Bar {
     COEF_EMPTY3, CUM_READY0, CUM_READY1, CUM_READY2, CUM_READY3, RS0, RS1,
     OPS_FULL0, OPS_FULL1, OPS_EMPTY0, OPS_EMPTY1, S_FULL, S_EMPTY, SL_FULL, DS_FULL, DS_EMPTY,
     G_FULL, G_EMPTY, Y_FULL0, Y_FULL1, Y_EMPTY0, Y_EMPTY1, Y_STAGED0, Y_STAGED1, Y_STAGED2, DRAIN,
-    NEVER, NUM_BARS
+    NEVER, XR_FULL, NUM_BARS
 };
 
 // arrival count of each barrier: 1 for TMA expect_tx / tcgen05.commit / single-thread or
@@ -205,6 +205,7 @@ struct Cfg {
 
 struct TcParams {
     CUtensorMap tm_x, tm_y, tm_z, tm_B, tm_C, tm_th, tm_dt, tm_A, tm_lam, tm_sc;
+    CUtensorMap tm_xr, tm_zr;   // one value per head channel (MIMO lightweight expansion)
     ScanArgs a;
     int nchunks;
     unsigned long long limit_ns;
@@ -752,7 +753,7 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
 // State warpgroup (warps 16-19): the fp32 carried state g in TMEM columns TM_G..,
 // g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T, per chunk g <- e^{cum_end} g + dS and its
 // bf16 copy for the Y_inter MMA; at the end h_T = R(psi_T) g and the carried x.
-template <int NST, int Q, int R, bool GT, bool BC>
+template <int NST, int Q, int R, bool GT, bool BC, bool XE>
 __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
                       const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
@@ -885,11 +886,21 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
         if (stid == 0) M3_TRACE_EV(c, 18);
     }
     if (stid == 0) {
-        // only this warpgroup read x_prev (for g_0), so the carried x can be replaced now
-        const uint4* xl = reinterpret_cast<const uint4*>(
-            static_cast<const __nv_bfloat16*>(a.x) + (((size_t)b * T + (T - 1)) * a.H + h) * R * kP);
-        uint4* xpo = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.x_prev) + bh * R * kP);
-        for (int e = 0; e < R * kP / 8; ++e) xpo[e] = xl[e];
+        // only this warpgroup read x_prev (for g_0), so the carried x can be replaced now;
+        // with the lightweight expansion it takes the expanded X_{T-1}, as the stage held it
+        const size_t row = ((size_t)b * T + (T - 1)) * a.H + h;
+        if (XE && a.x_expand) {
+            const __nv_bfloat16* xl = static_cast<const __nv_bfloat16*>(a.x) + row * kP;
+            const float* wx = a.x_expand + (size_t)h * R * kP;
+            __nv_bfloat16* xpo = static_cast<__nv_bfloat16*>(a.x_prev) + bh * R * kP;
+            for (int e = 0; e < R * kP; ++e)
+                xpo[e] = __float2bfloat16_rn(__bfloat162float(xl[e % kP]) * wx[e]);
+        } else {
+            const uint4* xl = reinterpret_cast<const uint4*>(
+                static_cast<const __nv_bfloat16*>(a.x) + row * R * kP);
+            uint4* xpo = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.x_prev) + bh * R * kP);
+            for (int e = 0; e < R * kP / 8; ++e) xpo[e] = xl[e];
+        }
     }
 }
 
@@ -952,41 +963,149 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
 // store nor the store itself holds up the B / C / theta loads.  x(c) is loaded into
 // stage c % XST; once the epilogue has written y(c) over it (Y_STAGED), the tile is
 // stored, and when the store has read it the stage takes x(c + XST).
-template <int NST, int Q, int R, bool GT>
+//
+// MIMO lightweight expansion ("Multi-Input, Multi-Output (MIMO) Formulation", MIMO
+// Parameterization Choices): x (and z) then hold one value per head channel, and the
+// stage's (token, rank) row is X[u, r][p] = x_u[p] w[r][p], rounded to bf16.  The chunk's
+// Q raw rows are copied, unswizzled, into the stage's last Q rows and expanded in place by
+// the whole warp, token batch after token batch: every lane reads its batch before any
+// lane writes it, and the rows a batch writes, [t0 R, (t0 + k) R), lie below the raw row
+// (R - 1) Q + t0 + k of the first later token because (t0 + k)(R - 1) <= Q (R - 1).  The
+// stage is published on X_FULL once expanded.
+template <int NST, int Q, int R, bool GT, bool XE>
 __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
+    const int lane = threadIdx.x & 31;
     const int b = blockIdx.x / a.H, h = blockIdx.x % a.H;
-    int n_x[C::XST] = {};
-    auto load = [&](int c) {
-        const int xs = c % C::XST;
-        mbar_arrive_expect_tx(&bar[X_FULL0 + xs], C::XZ_BYTES);
-        tma_load_5d(sm + C::OFF_X + xs * C::X_BYTES, &p.tm_x, &bar[X_FULL0 + xs], 0, 0, h, c * Q,
-                    b);
-        if constexpr (GT)
-            tma_load_5d(sm + C::OFF_Z + xs * C::X_BYTES, &p.tm_z, &bar[X_FULL0 + xs], 0, 0, h,
+    if constexpr (!XE) {   // lane 0 alone: every tile comes by TMA
+        if (lane != 0) return;
+        int n_x[C::XST] = {};
+        auto load = [&](int c) {
+            const int xs = c % C::XST;
+            mbar_arrive_expect_tx(&bar[X_FULL0 + xs], C::XZ_BYTES);
+            tma_load_5d(sm + C::OFF_X + xs * C::X_BYTES, &p.tm_x, &bar[X_FULL0 + xs], 0, 0, h,
                         c * Q, b);
-        ++n_x[xs];
-    };
-    for (int c = 0; c < C::XST && c < p.nchunks; ++c) load(c);
-    bool ok = true;
-    for (int c = 0; c < p.nchunks; ++c) {
-        if (!(ok = mbar_wait(&bar[Y_STAGED0 + c % C::XST], (c / C::XST) & 1, ab))) break;
-        const int xs = c % C::XST;
-        tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, c * Q, b);
-        bulk_commit();
-        mbar_arrive(&bar[COEF_EMPTY0 + c % kCoefSlots]);
-        bulk_wait_read<0>();
-        M3_TRACE_EV(c, 23);
-        if (c + C::XST < p.nchunks) load(c + C::XST);
+            if constexpr (GT)
+                tma_load_5d(sm + C::OFF_Z + xs * C::X_BYTES, &p.tm_z, &bar[X_FULL0 + xs], 0, 0, h,
+                            c * Q, b);
+            ++n_x[xs];
+        };
+        for (int c = 0; c < C::XST && c < p.nchunks; ++c) load(c);
+        bool ok = true;
+        for (int c = 0; c < p.nchunks; ++c) {
+            if (!(ok = mbar_wait(&bar[Y_STAGED0 + c % C::XST], (c / C::XST) & 1, ab))) break;
+            const int xs = c % C::XST;
+            tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, c * Q, b);
+            bulk_commit();
+            mbar_arrive(&bar[COEF_EMPTY0 + c % kCoefSlots]);
+            bulk_wait_read<0>();
+            M3_TRACE_EV(c, 23);
+            if (c + C::XST < p.nchunks) load(c + C::XST);
+        }
+        if (!ok)
+            for (int s = 0; s < C::XST; ++s)
+                if (n_x[s]) drain_wait(&bar[X_FULL0 + s], (n_x[s] - 1) & 1, 10000000ull);
+        bulk_wait<0>();
+        return;
+    } else {
+    const bool xe = a.x_expand != nullptr, ze = GT && a.z_expand != nullptr;
+    // expansion: lane = (rank r, 16-byte column chunk ch) for TPL tokens side by side
+    constexpr int CMB = 8 * R, TPL = 32 / CMB;
+    static_assert(32 % CMB == 0 && Q % (2 * TPL) == 0, "expansion lane layout");
+    const int r = (lane % CMB) >> 3, ch = lane & 7, toff = lane / CMB;
+    // this lane's 8 weights w[r][8 ch .. 8 ch + 7] as 4 pairs (packed fp32x2 products)
+    float2 wx[4], wz[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wx[j] = wz[j] = make_float2(0.f, 0.f);
+    if (xe) {
+        const float2* w2 = reinterpret_cast<const float2*>(a.x_expand + ((size_t)h * R + r) * kP + 8 * ch);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) wx[j] = w2[j];
     }
-    if (!ok)
-        for (int s = 0; s < C::XST; ++s)
-            if (n_x[s]) drain_wait(&bar[X_FULL0 + s], (n_x[s] - 1) & 1, 10000000ull);
-    bulk_wait<0>();
+    if (ze) {
+        const float2* w2 = reinterpret_cast<const float2*>(a.z_expand + ((size_t)h * R + r) * kP + 8 * ch);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) wz[j] = w2[j];
+    }
+    auto mul2 = [](uint32_t v, float2 w) {   // two bf16 values times two weights, rounded
+        const float2 p = __fmul2_rn(make_float2(bf16lo(v), bf16hi(v)), w);
+        return pack_bf16x2(p.x, p.y);
+    };
+    // the stage's last Q rows (raw, unswizzled) -> its rows (u, r) (128B-swizzled), in place
+    auto expand = [&](uint8_t* tile, const float2 (&w)[4]) {
+        const uint8_t* raw = tile + (R - 1) * Q * 128;
+#pragma unroll 1
+        for (int t0 = 0; t0 < Q; t0 += 2 * TPL) {
+            uint4 v[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                v[k] = *reinterpret_cast<const uint4*>(raw + (t0 + k * TPL + toff) * 128 + ch * 16);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int row = (t0 + k * TPL + toff) * R + r;
+                const uint4 o = make_uint4(mul2(v[k].x, w[0]), mul2(v[k].y, w[1]),
+                                           mul2(v[k].z, w[2]), mul2(v[k].w, w[3]));
+                *reinterpret_cast<uint4*>(tile + row * 128 + (((ch ^ row) & 7) << 4)) = o;
+            }
+            __syncwarp();
+        }
+    };
+    int n_xr = 0;           // copies issued on XR_FULL (each one phase)
+    bool pending = false;   // a copy on XR_FULL has not been waited for
+    // every copy of stage c lands on XR_FULL; the expanded stage is published on X_FULL
+    auto load = [&](int c) -> bool {
+        const int xs = c % C::XST;
+        uint8_t* xt = sm + C::OFF_X + xs * C::X_BYTES;
+        uint8_t* zt = sm + C::OFF_Z + xs * C::X_BYTES;
+        if (lane == 0) {
+            const int bytes = (xe ? Q * 128 : C::X_BYTES) + (GT ? (ze ? Q * 128 : C::X_BYTES) : 0);
+            mbar_arrive_expect_tx(&bar[XR_FULL], bytes);
+            if (xe)
+                tma_load_4d(xt + (R - 1) * Q * 128, &p.tm_xr, &bar[XR_FULL], 0, h, c * Q, b);
+            else
+                tma_load_5d(xt, &p.tm_x, &bar[XR_FULL], 0, 0, h, c * Q, b);
+            if constexpr (GT) {
+                if (ze)
+                    tma_load_4d(zt + (R - 1) * Q * 128, &p.tm_zr, &bar[XR_FULL], 0, h, c * Q, b);
+                else
+                    tma_load_5d(zt, &p.tm_z, &bar[XR_FULL], 0, 0, h, c * Q, b);
+            }
+        }
+        pending = true;
+        if (!warp_wait(&bar[XR_FULL], n_xr++ & 1, ab)) return false;
+        pending = false;
+        if (xe) expand(xt, wx);
+        if (ze) expand(zt, wz);
+        fence_proxy_async_smem();   // the expanded rows are read by the MMAs and the y store
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[X_FULL0 + xs]);
+        return true;
+    };
+    bool ok = true;
+    for (int c = 0; c < C::XST && c < p.nchunks && ok; ++c) ok = load(c);
+    for (int c = 0; c < p.nchunks && ok; ++c) {
+        if (!(ok = warp_wait(&bar[Y_STAGED0 + c % C::XST], (c / C::XST) & 1, ab))) break;
+        const int xs = c % C::XST;
+        if (lane == 0) {
+            tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, c * Q, b);
+            bulk_commit();
+            mbar_arrive(&bar[COEF_EMPTY0 + c % kCoefSlots]);
+            bulk_wait_read<0>();
+        }
+        __syncwarp();
+        if (lane == 0) M3_TRACE_EV(c, 23);
+        if (c + C::XST < p.nchunks) ok = load(c + C::XST);
+    }
+    if (lane == 0) {
+        if (pending) drain_wait(&bar[XR_FULL], (n_xr - 1) & 1, 10000000ull);
+        bulk_wait<0>();
+    }
+    }
 }
 
-template <int NST, int Q, int R, bool GT, bool BC>
+template <int NST, int Q, int R, bool GT, bool BC, bool XE>
 __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_constant__ TcParams p) {
     using C = Cfg<NST, Q, R, GT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1002,8 +1121,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], bar_count(i));
         misc[1] = 0u;  // abort flag
         fence_mbar_init();
-        tma_prefetch_desc(&p.tm_x);
-        if (GT) tma_prefetch_desc(&p.tm_z);
+        tma_prefetch_desc(XE && p.a.x_expand ? &p.tm_xr : &p.tm_x);
+        if (GT) tma_prefetch_desc(XE && p.a.z_expand ? &p.tm_zr : &p.tm_z);
         tma_prefetch_desc(&p.tm_B);
         tma_prefetch_desc(&p.tm_C);
         tma_prefetch_desc(&p.tm_th);
@@ -1031,13 +1150,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     } else if (w < 6) {
         epilogue<NST, Q, R, GT>(p, sm, bar, tmem, ab);
     } else if (w >= 16) {
-        state<NST, Q, R, GT, BC>(p, sm, bar, tmem, ab);
+        state<NST, Q, R, GT, BC, XE>(p, sm, bar, tmem, ab);
     } else if (w < 6 + kRotWarps) {
         rotation<NST, Q, R, GT, BC>(p, sm, bar, ab);
     } else if (w == 6 + kRotWarps) {
         coefficients<NST, Q, R, GT>(p, sm, bar, ab);
-    } else if ((threadIdx.x & 31) == 0) {
-        x_producer<NST, Q, R, GT>(p, sm, bar, ab);
+    } else if (XE || (threadIdx.x & 31) == 0) {
+        x_producer<NST, Q, R, GT, XE>(p, sm, bar, ab);
     }
     tc_fence_before();
     __syncthreads();
@@ -1083,7 +1202,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ptr,
     return r == CUDA_SUCCESS;
 }
 
-template <int NST, int Q, int R, bool GT, bool BC>
+template <int NST, int Q, int R, bool GT, bool BC, bool XE>
 cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
     using C = Cfg<NST, Q, R, GT>;
     TcParams p;
@@ -1097,13 +1216,26 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
         const uint64_t d[5] = {kP, R, H, T, Bn};
         const uint64_t st[4] = {kP * 2, (uint64_t)R * kP * 2, H * R * kP * 2, T * H * R * kP * 2};
         const uint32_t box[5] = {kP, R, 1, Q, 1};
-        ok &= make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.x, d, st, box,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+        if (!a.x_expand)
+            ok &= make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.x, d, st, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
         ok &= make_map(&p.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.y, d, st, box,
                        CU_TENSOR_MAP_SWIZZLE_128B);
-        if (GT)
+        if (GT && !a.z_expand)
             ok &= make_map(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.z, d, st, box,
                            CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (a.x_expand || (GT && a.z_expand)) {
+        // x, z of the lightweight expansion: (P, H, T, b), box (64, 1, Q, 1), unswizzled rows
+        const uint64_t d[4] = {kP, H, T, Bn};
+        const uint64_t st[3] = {kP * 2, H * kP * 2, T * H * kP * 2};
+        const uint32_t box[4] = {kP, 1, Q, 1};
+        if (a.x_expand)
+            ok &= make_map(&p.tm_xr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.x, d, st, box,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (GT && a.z_expand)
+            ok &= make_map(&p.tm_zr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.z, d, st, box,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     {   // B, C: (N, R, G, T, b), box (N, R, 1, RT, 1)
         const uint64_t d[5] = {NST, R, G, T, Bn};
@@ -1144,10 +1276,10 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R, GT, BC>,
+    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R, GT, BC, XE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<NST, Q, R, GT, BC><<<(unsigned)(a.batch * a.H), kThreads, C::SMEM, s>>>(p);
+    scan_tc_kernel<NST, Q, R, GT, BC, XE><<<(unsigned)(a.batch * a.H), kThreads, C::SMEM, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -1176,28 +1308,35 @@ int scan_tc_chunk(int N, int P, int R, int chunk, int H) {
 
 size_t scan_tc_workspace_bytes(int, int, int, int, int, long long, int) { return 0; }
 
-template <bool GT, bool BC>
+template <bool GT, bool BC, bool XE>
 cudaError_t launch_scan_tc_g(const ScanArgs& a, int R, cudaStream_t s) {
     const int N = a.N, Q = a.chunk;   // the tile chunk chosen by scan_tc_chunk
     if (R == 1) {
-        if (N == 128 && Q == 64) return launch_t<128, 64, 1, GT, BC>(a, s);
-        if (N == 128 && Q == 128) return launch_t<128, 128, 1, GT, BC>(a, s);
-        if (N == 64 && Q == 64) return launch_t<64, 64, 1, GT, BC>(a, s);
-        if (N == 64 && Q == 128) return launch_t<64, 128, 1, GT, BC>(a, s);
+        if (N == 128 && Q == 64) return launch_t<128, 64, 1, GT, BC, XE>(a, s);
+        if (N == 128 && Q == 128) return launch_t<128, 128, 1, GT, BC, XE>(a, s);
+        if (N == 64 && Q == 64) return launch_t<64, 64, 1, GT, BC, XE>(a, s);
+        if (N == 64 && Q == 128) return launch_t<64, 128, 1, GT, BC, XE>(a, s);
     } else if (R == 2 && N == 64) {
-        if (Q == 32) return launch_t<64, 32, 2, GT, BC>(a, s);
-        if (Q == 64) return launch_t<64, 64, 2, GT, BC>(a, s);
+        if (Q == 32) return launch_t<64, 32, 2, GT, BC, XE>(a, s);
+        if (Q == 64) return launch_t<64, 64, 2, GT, BC, XE>(a, s);
     } else if (R == 4 && N == 64) {
-        if (Q == 16) return launch_t<64, 16, 4, GT, BC>(a, s);
-        if (Q == 32) return launch_t<64, 32, 4, GT, BC>(a, s);
+        if (Q == 16) return launch_t<64, 16, 4, GT, BC, XE>(a, s);
+        if (Q == 32) return launch_t<64, 32, 4, GT, BC, XE>(a, s);
     }
     return cudaErrorNotSupported;
 }
 
-// a.z and a.bc select the instantiation with the fused output gate and BC map
+template <bool GT, bool BC>
+cudaError_t launch_scan_tc_x(const ScanArgs& a, int R, cudaStream_t s) {
+    const bool xe = a.x_expand || (GT && a.z_expand);
+    return xe ? launch_scan_tc_g<GT, BC, true>(a, R, s) : launch_scan_tc_g<GT, BC, false>(a, R, s);
+}
+
+// a.z, a.bc and the expansion weights select the instantiation with the fused output gate,
+// the BC map and the MIMO lightweight expansion
 cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s) {
-    if (a.z) return a.bc ? launch_scan_tc_g<true, true>(a, R, s) : launch_scan_tc_g<true, false>(a, R, s);
-    return a.bc ? launch_scan_tc_g<false, true>(a, R, s) : launch_scan_tc_g<false, false>(a, R, s);
+    if (a.z) return a.bc ? launch_scan_tc_x<true, true>(a, R, s) : launch_scan_tc_x<true, false>(a, R, s);
+    return a.bc ? launch_scan_tc_x<false, true>(a, R, s) : launch_scan_tc_x<false, false>(a, R, s);
 }
 
 }  // namespace m3

@@ -123,6 +123,16 @@ def make_bc_bias(nheads, dstate, seed=0):
             1.0 + 0.3 * torch.randn((nheads, dstate), generator=g))
 
 
+def make_expand(nheads, rank, headdim, seed=0):
+    """MIMO lightweight-expansion weights x_expand, z_expand [H][R][P] float32, N(0, 1) (the
+    pages fix no initialisation; unit scale keeps X = x * w at the scale of x).  Own
+    generator (seed + 15485863): adding them never changes the other seeded inputs.  The
+    per-channel input x [.., H, P] of an expanded workload is rank column 0 of the drawn x."""
+    g = torch.Generator("cpu").manual_seed(seed + 15485863)
+    return (torch.randn((nheads, rank, headdim), generator=g),
+            torch.randn((nheads, rank, headdim), generator=g))
+
+
 def make_decode_inputs(batch, nheads, ngroups, headdim, dstate, rank=1, tokens=1,
                        io_dtype=torch.bfloat16, theta_max=math.pi / 8, seed=0):
     """Per-token decode inputs stacked over ``tokens`` plus the starting state.

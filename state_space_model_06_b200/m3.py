@@ -49,7 +49,8 @@ class m3_state(ctypes.Structure):
 
 class m3_extras(ctypes.Structure):
     _fields_ = [("z", ctypes.c_void_p), ("B_bias", ctypes.c_void_p), ("C_bias", ctypes.c_void_p),
-                ("bc_norm_eps", ctypes.c_float)]
+                ("bc_norm_eps", ctypes.c_float), ("x_expand", ctypes.c_void_p),
+                ("z_expand", ctypes.c_void_p)]
 
 
 _lib = None
@@ -212,15 +213,18 @@ def m3_scan_fwd_gated(dims: Dims, seqlen: int, chunk: int, x, B, C, dt, A, lam, 
 @dataclass
 class Extras:
     """Optional fused parts (see m3_extras in include/m3.h): output gate z, BC biases
-    B_bias / C_bias [H][N] fp32, BCNorm epsilon (0: off)."""
+    B_bias / C_bias [H][N] fp32, BCNorm epsilon (0: off), MIMO lightweight expansion
+    weights x_expand / z_expand [H][R][P] fp32 (x, z then hold [..][H][P])."""
     z: object = None
     B_bias: object = None
     C_bias: object = None
     bc_norm_eps: float = 0.0
+    x_expand: object = None
+    z_expand: object = None
 
     def c(self) -> m3_extras:
         return m3_extras(_ptr(self.z), _ptr(self.B_bias), _ptr(self.C_bias),
-                         float(self.bc_norm_eps))
+                         float(self.bc_norm_eps), _ptr(self.x_expand), _ptr(self.z_expand))
 
 
 def _ex_ref(ex):

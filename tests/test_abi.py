@@ -155,6 +155,35 @@ def test_extras_validation_before_launch(lib):
     assert dec(m3.Extras(bc_norm_eps=-1.0)) == m3.M3_ERR_SHAPE
     assert dec(m3.Extras(C_bias=p + 1)) == m3.M3_ERR_ALIGN
 
+    # MIMO lightweight expansion: 16-byte aligned weights; an expanded gate needs z
+    for call in (scan, dec):
+        assert call(m3.Extras(x_expand=p + 4)) == m3.M3_ERR_ALIGN
+        assert call(m3.Extras(z_expand=p)) == m3.M3_ERR_NULL
+        assert call(m3.Extras(z=p, z_expand=p + 8)) == m3.M3_ERR_ALIGN
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The binding's ctypes structs have the C header's sizes and field offsets."""
+    import subprocess
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "m3.h"\n'
+        'int main(void) {\n'
+        '  printf("%zu %zu %zu\\n", sizeof(m3_dims), sizeof(m3_state), sizeof(m3_extras));\n'
+        '  printf("%zu %zu %zu %zu %zu %zu\\n", offsetof(m3_extras, z), offsetof(m3_extras, B_bias),'
+        ' offsetof(m3_extras, C_bias), offsetof(m3_extras, bc_norm_eps),'
+        ' offsetof(m3_extras, x_expand), offsetof(m3_extras, z_expand));\n'
+        '  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    out = subprocess.check_output([str(exe)]).decode().split()
+    sizes = [int(v) for v in out[:3]]
+    offs = [int(v) for v in out[3:]]
+    assert sizes == [ctypes.sizeof(m3.m3_dims), ctypes.sizeof(m3.m3_state),
+                     ctypes.sizeof(m3.m3_extras)]
+    assert offs == [getattr(m3.m3_extras, f).offset for f in
+                    ("z", "B_bias", "C_bias", "bc_norm_eps", "x_expand", "z_expand")]
+
 
 def test_binding_refuses_missing_library(tmp_path):
     old = m3._lib
