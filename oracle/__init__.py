@@ -68,6 +68,9 @@ def _load(path=None):
         lib.m3o_expand.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    dp, dp, dp]
         lib.m3o_expand.restype = None
+        lib.m3o_scan_bwd.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int64, ctypes.c_uint32] + \
+            [dp] * 24 + [ctypes.c_int]
+        lib.m3o_scan_bwd.restype = ctypes.c_int
         _libs[path] = lib
     return _libs[path]
 
@@ -160,6 +163,50 @@ def scan(x, B, C, dt, A, lam, theta, D=None, h0=None, x_prev=None, B_prev=None,
         z = _f64(z, (b, T, H, R, P), "z")
         _load(lib_path).m3o_gate(y.size, _ptr(z), _ptr(y))
     return y, h, xp, bp
+
+
+def scan_bwd(x, B, C, dt, A, lam, theta, dy, D=None, h0=None, x_prev=None, B_prev=None,
+             dhT=None, theta_is_angle: bool = False, nthreads: int = 0, lib_path=None):
+    """Reverse-mode gradients of ``scan`` (no fused extras) for a loss with dL/dy = dy
+    [b,T,H,R,P] and dL/dh_T = dhT [b,H,N,P] (None: zero).
+
+    Returns a dict of float64 arrays: dx [b,T,H,R,P]; dB, dC [b,T,G,R,N] and dtheta
+    [b,T,G,N/2] (summed over the heads of each group); ddt, dA, dlam [b,T,H]; dD [H] (summed
+    over batch and tokens; None without D); dh0 [b,H,N,P]; dx_prev [b,H,R,P]; dB_prev
+    [b,G,R,N].  The carried x_prev / B_prev outputs of the call get no gradient here.
+    """
+    x = np.asarray(x)
+    b, T, H, R, P = x.shape
+    G, N = np.asarray(B).shape[2], np.asarray(B).shape[4]
+    ins = dict(
+        x=_f64(x, (b, T, H, R, P), "x"), B=_f64(B, (b, T, G, R, N), "B"),
+        C=_f64(C, (b, T, G, R, N), "C"), dt=_f64(dt, (b, T, H), "dt"),
+        A=_f64(A, (b, T, H), "A"), lam=_f64(lam, (b, T, H), "lam"),
+        theta=_f64(theta, (b, T, G, N // 2), "theta"))
+    D = None if D is None else _f64(D, (H,), "D")
+    h0 = None if h0 is None else _f64(h0, (b, H, N, P), "h0")
+    xp = None if x_prev is None else _f64(x_prev, (b, H, R, P), "x_prev")
+    bp = None if B_prev is None else _f64(B_prev, (b, G, R, N), "B_prev")
+    dy = _f64(dy, (b, T, H, R, P), "dy")
+    dhT = None if dhT is None else _f64(dhT, (b, H, N, P), "dhT")
+    out = dict(dx=np.zeros((b, T, H, R, P)), dB=np.zeros((b, T, G, R, N)),
+               dC=np.zeros((b, T, G, R, N)), ddt=np.zeros((b, T, H)), dA=np.zeros((b, T, H)),
+               dlam=np.zeros((b, T, H)), dtheta=np.zeros((b, T, G, N // 2)),
+               dD=np.zeros(H), dh0=np.zeros((b, H, N, P)), dx_prev=np.zeros((b, H, R, P)),
+               dB_prev=np.zeros((b, G, R, N)))
+    dims = _Dims(b, H, G, P, N, R)
+    fl = THETA_IS_ANGLE if theta_is_angle else 0
+    rc = _load(lib_path).m3o_scan_bwd(
+        ctypes.byref(dims), T, fl, *(_ptr(ins[k]) for k in ("x", "B", "C", "dt", "A", "lam",
+                                                           "theta")),
+        _ptr(D), _ptr(h0), _ptr(xp), _ptr(bp), _ptr(dy), _ptr(dhT),
+        *(_ptr(out[k]) for k in ("dx", "dB", "dC", "ddt", "dA", "dlam", "dtheta", "dD", "dh0",
+                                 "dx_prev", "dB_prev")), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"m3o_scan_bwd rejected its arguments (code {rc})")
+    if D is None:
+        out["dD"] = None
+    return out
 
 
 def decode_step(x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev,

@@ -220,6 +220,211 @@ int m3o_decode(const m3o_dims* d, uint32_t flags, const double* x, const double*
                     nthreads);
 }
 
+/*
+ * Backward pass (reverse-mode derivative) of m3o_scan for a scalar loss L whose gradients
+ * with respect to the outputs are dy [b][T][H][R][P] (dL/dy) and dhT [b][H][N][P] (dL/dh_T,
+ * may be NULL: zero).  The derivative is taken through the recurrence exactly as m3o_step
+ * evaluates it (Proposition 1 with the rotation of Propositions 2 and 4), one token at a
+ * time in reverse, with the states h_t recomputed by m3o_step itself:
+ *
+ *   forward, per token:  M = alpha h_{t-1} + beta Bp Xp^T;  U = R(phi) M;
+ *                        h_t = U + gamma B_t X_t^T;  Y_t = h_t^T C_t + D X_t
+ *   reverse, per token (Lam = dL/dh_t, starting from dhT):
+ *     Lam += C_t dY_t^T;  dC_t = h_t dY_t^T;  dX_t += D dY_t;  dD += <dY_t, X_t>
+ *     dgamma = <Lam, B_t X_t^T>;  dB_t += gamma Lam X_t;  dX_t += gamma B_t^T Lam
+ *     dM = R(phi)^T Lam;  dphi_i = sum_p (Lam_{2i+1} U_{2i} - Lam_{2i} U_{2i+1})
+ *     dalpha = <dM, h_{t-1}>;  dbeta = <dM, Bp Xp^T>;  dBp += beta dM Xp;  dXp += beta Bp^T dM
+ *     Lam <- alpha dM
+ *   and through alpha = exp(dt A), beta = (1 - lam) dt alpha, gamma = lam dt, phi = dt theta:
+ *     ddt = dalpha alpha A + dbeta (1 - lam)(alpha + dt alpha A) + dgamma lam + sum_i dphi_i theta_i
+ *     dA = dalpha alpha dt + dbeta (1 - lam) dt alpha dt,  dlam = -dbeta dt alpha + dgamma dt
+ *     dtheta_i = dphi_i dt  (dphi_i with M3O_THETA_IS_ANGLE)
+ *   Bp, Xp of token t are B_{t-1}, X_{t-1} (B_prev, x_prev at t = 0), so dBp / dXp add to the
+ *   previous token's dB / dX, or form dB_prev / dx_prev; dh0 is the final Lam.
+ *
+ * B, C, theta and B_prev are shared by the heads of a group, so their gradients are sums over
+ * those heads; dD sums over batch and tokens.  The gradients of the carried x_prev / B_prev
+ * outputs (copies of the last token) are not inputs here: a caller chaining calls adds them
+ * to dx / dB of the last token.  Outputs are overwritten.  h0, x_prev, B_prev may be NULL
+ * (zeros); with D NULL there is no skip and dD is left untouched (may be NULL).
+ * Parallel over batch rows (the heads of a row share its group gradients).
+ */
+int m3o_scan_bwd(const m3o_dims* d, int64_t T, uint32_t flags, const double* x,
+                 const double* B, const double* C, const double* dt, const double* A,
+                 const double* lam, const double* theta, const double* D, const double* h0,
+                 const double* x_prev, const double* B_prev, const double* dy, const double* dhT,
+                 double* dx, double* dB, double* dC, double* ddt, double* dA, double* dlam,
+                 double* dtheta, double* dD, double* dh0, double* dx_prev, double* dB_prev,
+                 int nthreads)
+{
+    int rc = m3o_check(d, T);
+    if (rc) return rc;
+    const int Bn = d->batch, H = d->nheads, G = d->ngroups, P = d->headdim, N = d->dstate,
+              R = d->rank;
+    const int hpg = H / G;
+    memset(dx, 0, sizeof(double) * (size_t)Bn * T * H * R * P);
+    memset(dB, 0, sizeof(double) * (size_t)Bn * T * G * R * N);
+    memset(dC, 0, sizeof(double) * (size_t)Bn * T * G * R * N);
+    memset(ddt, 0, sizeof(double) * (size_t)Bn * T * H);
+    memset(dA, 0, sizeof(double) * (size_t)Bn * T * H);
+    memset(dlam, 0, sizeof(double) * (size_t)Bn * T * H);
+    memset(dtheta, 0, sizeof(double) * (size_t)Bn * T * G * (N / 2));
+    memset(dh0, 0, sizeof(double) * (size_t)Bn * H * N * P);
+    memset(dx_prev, 0, sizeof(double) * (size_t)Bn * H * R * P);
+    memset(dB_prev, 0, sizeof(double) * (size_t)Bn * G * R * N);
+    double* dDb = (double*)calloc((size_t)(Bn > 0 ? Bn : 1) * H, sizeof(double));
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (int b = 0; b < Bn; ++b) {
+        const size_t NP = (size_t)N * P;
+        double* hs = (double*)malloc(sizeof(double) * (size_t)(T + 1) * NP);  /* h_{t-1}, t=0..T */
+        double* xp = (double*)malloc(sizeof(double) * (size_t)R * P);
+        double* bp = (double*)malloc(sizeof(double) * (size_t)R * N);
+        double* Y = (double*)malloc(sizeof(double) * (size_t)R * P);
+        double* Lam = (double*)malloc(sizeof(double) * NP);
+        double* dM = (double*)malloc(sizeof(double) * NP);
+        for (int hh = 0; hh < H; ++hh) {
+            const int g = hh / hpg;
+            const double Dh = D ? D[hh] : 0.0;
+            /* forward, keeping every state: hs[t + 1] = h_t, hs[0] = h0 */
+            if (h0) memcpy(hs, h0 + ((size_t)b * H + hh) * NP, sizeof(double) * NP);
+            else memset(hs, 0, sizeof(double) * NP);
+            if (x_prev) memcpy(xp, x_prev + ((size_t)b * H + hh) * R * P, sizeof(double) * R * P);
+            else memset(xp, 0, sizeof(double) * R * P);
+            if (B_prev) memcpy(bp, B_prev + ((size_t)b * G + g) * R * N, sizeof(double) * R * N);
+            else memset(bp, 0, sizeof(double) * R * N);
+            for (int64_t t = 0; t < T; ++t) {
+                const size_t bt = (size_t)b * T + t;
+                memcpy(hs + (t + 1) * NP, hs + t * NP, sizeof(double) * NP);
+                m3o_step(N, P, R, dt[bt * H + hh], A[bt * H + hh], lam[bt * H + hh],
+                         theta + (bt * G + g) * (N / 2), x + (bt * H + hh) * R * P,
+                         B + (bt * G + g) * R * N, C + (bt * G + g) * R * N, Dh,
+                         hs + (t + 1) * NP, xp, bp, Y, flags);
+            }
+            /* reverse */
+            if (dhT) memcpy(Lam, dhT + ((size_t)b * H + hh) * NP, sizeof(double) * NP);
+            else memset(Lam, 0, sizeof(double) * NP);
+            for (int64_t t = T - 1; t >= 0; --t) {
+                const size_t bt = (size_t)b * T + t;
+                const double dtv = dt[bt * H + hh], av = A[bt * H + hh], lv = lam[bt * H + hh];
+                const double alpha = exp(dtv * av);
+                const double beta = (1.0 - lv) * dtv * alpha;
+                const double gamma = lv * dtv;
+                const double* X = x + (bt * H + hh) * R * P;
+                const double* Bt = B + (bt * G + g) * R * N;
+                const double* Ct = C + (bt * G + g) * R * N;
+                const double* th = theta + (bt * G + g) * (N / 2);
+                const double* dY = dy + (bt * H + hh) * R * P;
+                const double* ht = hs + (t + 1) * NP;
+                const double* hprev = hs + t * NP;
+                const double* Xp = t > 0 ? x + ((bt - 1) * H + hh) * R * P
+                                         : (x_prev ? x_prev + ((size_t)b * H + hh) * R * P : NULL);
+                const double* Bp = t > 0 ? B + ((bt - 1) * G + g) * R * N
+                                         : (B_prev ? B_prev + ((size_t)b * G + g) * R * N : NULL);
+                double* dXt = dx + (bt * H + hh) * R * P;
+                double* dBt = dB + (bt * G + g) * R * N;
+                double* dCt = dC + (bt * G + g) * R * N;
+                double* dBp = t > 0 ? dB + ((bt - 1) * G + g) * R * N : dB_prev + ((size_t)b * G + g) * R * N;
+                double* dXpo = t > 0 ? dx + ((bt - 1) * H + hh) * R * P : dx_prev + ((size_t)b * H + hh) * R * P;
+
+                /* readout Y = h^T C + D X */
+                for (int n = 0; n < N; ++n)
+                    for (int p = 0; p < P; ++p) {
+                        double v = 0.0;
+                        for (int r = 0; r < R; ++r) v += Ct[r * N + n] * dY[r * P + p];
+                        Lam[n * P + p] += v;
+                    }
+                for (int r = 0; r < R; ++r)
+                    for (int n = 0; n < N; ++n) {
+                        double v = 0.0;
+                        for (int p = 0; p < P; ++p) v += ht[n * P + p] * dY[r * P + p];
+                        dCt[r * N + n] += v;
+                    }
+                for (int e = 0; e < R * P; ++e) {
+                    dXt[e] += Dh * dY[e];
+                    if (D) dDb[(size_t)b * H + hh] += dY[e] * X[e];
+                }
+                /* h_t = U + gamma B X^T */
+                double dgamma = 0.0;
+                for (int r = 0; r < R; ++r)
+                    for (int n = 0; n < N; ++n) {
+                        double v = 0.0;
+                        for (int p = 0; p < P; ++p) v += Lam[n * P + p] * X[r * P + p];
+                        dgamma += Bt[r * N + n] * v;
+                        dBt[r * N + n] += gamma * v;
+                    }
+                for (int r = 0; r < R; ++r)
+                    for (int p = 0; p < P; ++p) {
+                        double v = 0.0;
+                        for (int n = 0; n < N; ++n) v += Bt[r * N + n] * Lam[n * P + p];
+                        dXt[r * P + p] += gamma * v;
+                    }
+                /* U = R(phi) M, U = h_t - gamma B X^T */
+                double dphi_theta = 0.0;
+                for (int i = 0; i < N / 2; ++i) {
+                    const double phi = (flags & M3O_THETA_IS_ANGLE) ? th[i] : dtv * th[i];
+                    const double c = cos(phi), s = sin(phi);
+                    double dphi = 0.0;
+                    for (int p = 0; p < P; ++p) {
+                        double bx0 = 0.0, bx1 = 0.0;
+                        for (int r = 0; r < R; ++r) {
+                            bx0 += Bt[r * N + 2 * i] * X[r * P + p];
+                            bx1 += Bt[r * N + 2 * i + 1] * X[r * P + p];
+                        }
+                        const double u0 = ht[(2 * i) * P + p] - gamma * bx0;
+                        const double u1 = ht[(2 * i + 1) * P + p] - gamma * bx1;
+                        const double l0 = Lam[(2 * i) * P + p], l1 = Lam[(2 * i + 1) * P + p];
+                        dphi += l1 * u0 - l0 * u1;
+                        dM[(2 * i) * P + p] = c * l0 + s * l1;
+                        dM[(2 * i + 1) * P + p] = -s * l0 + c * l1;
+                    }
+                    if (flags & M3O_THETA_IS_ANGLE) {
+                        dtheta[(bt * G + g) * (N / 2) + i] += dphi;
+                    } else {
+                        dtheta[(bt * G + g) * (N / 2) + i] += dphi * dtv;
+                        dphi_theta += dphi * th[i];
+                    }
+                }
+                /* M = alpha h_{t-1} + beta Bp Xp^T */
+                double dalpha = 0.0, dbeta = 0.0;
+                for (size_t e = 0; e < NP; ++e) dalpha += dM[e] * hprev[e];
+                for (int r = 0; r < R; ++r)
+                    for (int n = 0; n < N; ++n) {
+                        double v = 0.0;
+                        for (int p = 0; p < P; ++p) v += dM[n * P + p] * (Xp ? Xp[r * P + p] : 0.0);
+                        if (Bp) dbeta += Bp[r * N + n] * v;
+                        dBp[r * N + n] += beta * v;
+                    }
+                for (int r = 0; r < R; ++r)
+                    for (int p = 0; p < P; ++p) {
+                        double v = 0.0;
+                        for (int n = 0; n < N; ++n) v += (Bp ? Bp[r * N + n] : 0.0) * dM[n * P + p];
+                        dXpo[r * P + p] += beta * v;
+                    }
+                for (size_t e = 0; e < NP; ++e) Lam[e] = alpha * dM[e];
+                /* coefficients */
+                ddt[bt * H + hh] = dalpha * alpha * av + dbeta * (1.0 - lv) * (alpha + dtv * alpha * av) +
+                                   dgamma * lv + dphi_theta;
+                dA[bt * H + hh] = dalpha * alpha * dtv + dbeta * (1.0 - lv) * dtv * alpha * dtv;
+                dlam[bt * H + hh] = -dbeta * dtv * alpha + dgamma * dtv;
+            }
+            memcpy(dh0 + ((size_t)b * H + hh) * NP, Lam, sizeof(double) * NP);
+        }
+        free(hs); free(xp); free(bp); free(Y); free(Lam); free(dM);
+    }
+    if (D && dD) {
+        for (int hh = 0; hh < H; ++hh) {
+            double v = 0.0;
+            for (int b = 0; b < Bn; ++b) v += dDb[(size_t)b * H + hh];
+            dD[hh] = v;
+        }
+    }
+    free(dDb);
+    return 0;
+}
+
 /* out[row][h][r][p] = in[row][h][p] * w[h][r][p] for rows of H heads: the lightweight
  * expansion of a per-head P-vector to the P x R MIMO input (or gate). */
 void m3o_expand(int64_t rows, int H, int R, int P, const double* in, const double* w,
