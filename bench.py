@@ -6,7 +6,8 @@ i.e. every prefill step of the method.  Alongside, as sub-metrics: the batch-256
 workloads (SISO N 128 and MIMO R 4 N 64; 1024 sequential tokens, the 32-token pool captured
 once as a CUDA graph and replayed), the same prefill and decode with the fused output gate
 ("gated") and with BCNorm + BC biases ("bc"), the MIMO rank-4 prefill plain and with the
-lightweight expansion of x and z ("mimo"), the end-to-end call through pinned host
+lightweight expansion of x and z ("mimo"), the backward pass of the prefill workload
+("backward"), the end-to-end call through pinned host
 buffers ("e2e"), and the CPU oracle on the workload's inputs ("cpu_baseline").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -386,6 +387,46 @@ def mimo_leg(args, dev, stream, rank, ws_world, pk):
     return out
 
 
+def backward_leg(args, w, d, g, dev, stream, rank, ws_world, pk):
+    """The backward pass (m3_scan_bwd) of the prefill workload: gradients of every input and
+    of the starting state for a random dL/dy, inputs resident in HBM.  Algorithmic bytes: the
+    forward inputs and dy read once, the fp32 gradients and dh0 written once."""
+    T = w.seqlen
+    st = m3.State(d, dev)
+    m3.m3_state_init(d, st, stream=stream)
+    gen = torch.Generator().manual_seed(300 + rank)
+    dy = torch.randn(g["x"].shape, generator=gen).to(w.io_dtype).to(dev)
+    gr = m3.alloc_grads(d, T, dev)
+    ws = m3.alloc_bwd_workspace(d, T, dev)
+
+    def run():
+        m3.m3_scan_bwd(d, T, g["x"], g["B"], g["C"], g["dt"], g["A"], g["lam"], g["theta"],
+                       g["D"], st, dy, None, gr, ws, stream=stream)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 3))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if m3.m3_query_status(ws, stream) != m3.M3_OK:
+        raise RuntimeError("backward: device status not OK")
+    ms = e0.elapsed_time(e1) / steps
+    b, H, G, P, N, R = w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank
+    e = 2
+    reads = b * T * (2 * H * R * P * e + 12 * H + G * (2 * R * N * e + 2 * N)) + b * H * N * P * 4
+    writes = sum(v.numel() * 4 for v in gr.values())
+    val, ms_max = job_throughput(b * T, ms, ws_world)
+    gbs = (reads + writes) / (ms / 1e3) / 1e9
+    del ws, gr, dy
+    return {"tokens_per_s": val, "ms_per_step": ms_max, "alg_bytes_per_step": reads + writes,
+            "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"], "steps": steps,
+            "kernel": "scan_bwd_kernel (sequential fp32, checkpoints every 16 tokens)"}
+
+
 def w_dec_batch(name):
     return inputs.WORKLOADS[name].batch
 
@@ -470,6 +511,7 @@ def ours(args):
 
     if args.prefill_only:
         args.no_decode = args.no_e2e = args.no_cpu = args.no_gate = args.no_mimo = True
+        args.no_bwd = True
     if not args.no_decode:
         line["decode"] = {}
         for name in (args.decode or DECODES):
@@ -524,6 +566,9 @@ def ours(args):
 
     if not args.no_mimo:
         line["mimo"] = mimo_leg(args, dev, stream, rank, ws_world, pk)
+
+    if not args.no_bwd:
+        line["backward"] = backward_leg(args, w, d, g, dev, stream, rank, ws_world, pk)
 
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_prefill_e2e(w, d, inp, st, ws, min(args.steps, 5), stream, dev)
@@ -589,6 +634,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-gate", action="store_true", help="skip the fused-output-gate legs")
     ap.add_argument("--no-mimo", action="store_true", help="skip the MIMO prefill legs")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward-pass leg")
     ap.add_argument("--cpu-rows", type=int, default=8,
                     help="batch rows of the workload timed on the CPU oracle (default: all)")
     ap.add_argument("--ref-tokens", type=int, default=256)

@@ -266,6 +266,56 @@ m3_status m3_decode_step_gated(const m3_dims* dims, const void* x, const void* B
                                const float* theta, const float* D, const void* z,
                                m3_state* state, void* y, uint32_t flags, void* stream);
 
+/*
+ * Backward pass of m3_scan_fwd (without extras): the reverse-mode gradients of a scalar loss
+ * L given dL/dy and dL/dh_T.  The pages describe only the forward recurrence; this is its
+ * derivative, taken token by token in reverse through the same operations (Proposition 1
+ * with the rotation of Propositions 2 and 4; MIMO rank-R input and readout):
+ *   Lam = dL/dh_t:  Lam += C dy^T;  dC = h_t dy^T;  dx = D dy + gamma B^T Lam (+ beta B^T dM of
+ *   the next token);  dB = gamma Lam x^T (+ beta dM x^T of the next token);  dM = R(phi)^T Lam;
+ *   Lam <- alpha dM;  and through alpha = e^{dt A}, beta = (1 - lam) dt alpha, gamma = lam dt,
+ *   phi = dt theta to ddt, dA, dlam, dtheta.
+ *
+ *   in : the forward call's inputs x, B, C (io dtype), dt, A, lam, theta, D (may be NULL);
+ *        state0: the state that forward call STARTED from (h0, x_prev, B_prev; read only);
+ *        dy [b][T][H][R][P] io dtype; dhT [b][H][N][P] fp32 or NULL (zero).
+ *   out: grads (fp32, caller-owned, overwritten, not NULL except dD):
+ *        dx [b][T][H][R][P]; dB, dC [b][T][G][R][N] and dtheta [b][T][G][N/2], each summed
+ *        over the heads of its group; ddt, dA, dlam [b][T][H]; dD [H] summed over batch and
+ *        tokens (ignored when D is NULL; may be NULL); dh0 [b][H][N][P]; dx_prev [b][H][R][P];
+ *        dB_prev [b][G][R][N] (summed over the group's heads).
+ *   The carried x_prev / B_prev outputs of the forward call (copies of its last token) get no
+ *   gradient here: a caller chaining calls adds theirs to dx / dB of the last token.
+ *   The states are recomputed inside (checkpoints every 16 tokens in the workspace); the
+ *   call runs sequential fp32 kernels, one CTA per (batch, head).  Supported: N even, N <= 256,
+ *   P <= 64, R in {1, 2, 3, 4, 8} (else M3_ERR_UNSUPPORTED).  seqlen 0 does nothing.
+ *   Group sums use fp32 atomics, so dB, dC, dtheta, dB_prev and dD may differ in the last
+ *   bits from run to run.
+ */
+typedef struct {
+    float* dx;
+    float* dB;
+    float* dC;
+    float* ddt;
+    float* dA;
+    float* dlam;
+    float* dtheta;
+    float* dD;
+    float* dh0;
+    float* dx_prev;
+    float* dB_prev;
+} m3_grads;
+
+/* Workspace bytes of m3_scan_bwd for (dims, seqlen): the status block plus, per (batch,
+ * head), one N x P fp32 state per 16 tokens and one 16-token segment of states. */
+m3_status m3_scan_bwd_workspace_bytes(const m3_dims* dims, int32_t seqlen, size_t* bytes);
+
+m3_status m3_scan_bwd(const m3_dims* dims, int32_t seqlen, const void* x, const void* B,
+                      const void* C, const float* dt, const float* A, const float* lam,
+                      const float* theta, const float* D, const m3_state* state0,
+                      const void* dy, const float* dhT, const m3_grads* grads, void* workspace,
+                      size_t workspace_bytes, uint32_t flags, void* stream);
+
 /* Synchronise `stream` and report the device-side status word in `workspace`
  * (M3_OK, or M3_ERR_TIMEOUT when a bounded wait gave up). */
 m3_status m3_query_status(const void* workspace, void* stream);

@@ -348,6 +348,72 @@ m3_status m3_decode_step_gated(const m3_dims* d, const void* x, const void* B, c
     return decode_impl(d, x, B, C, dt, A, lam, theta, D, &ex, state, y, flags, stream);
 }
 
+m3_status m3_scan_bwd_workspace_bytes(const m3_dims* d, int32_t seqlen, size_t* bytes) {
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    if (!bytes) return M3_ERR_NULL;
+    if (seqlen < 0) return M3_ERR_SHAPE;
+    const size_t fl = scan_bwd_ws_floats(d->batch, d->nheads, d->dstate, d->headdim, seqlen);
+    *bytes = kStatusBytes + ((fl * sizeof(float) + 255) / 256) * 256;
+    return M3_OK;
+}
+
+m3_status m3_scan_bwd(const m3_dims* d, int32_t seqlen, const void* x, const void* B,
+                      const void* C, const float* dt, const float* A, const float* lam,
+                      const float* theta, const float* D, const m3_state* state0,
+                      const void* dy, const float* dhT, const m3_grads* gr, void* workspace,
+                      size_t workspace_bytes, uint32_t flags, void* stream) {
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    if (seqlen < 0) return M3_ERR_SHAPE;
+    if ((st = check_state(state0)) != M3_OK) return st;
+    if (!gr) return M3_ERR_NULL;
+    if (seqlen == 0) return M3_OK;
+    if (!x || !B || !C || !dt || !A || !lam || !theta || !dy) return M3_ERR_NULL;
+    if (!gr->dx || !gr->dB || !gr->dC || !gr->ddt || !gr->dA || !gr->dlam || !gr->dtheta ||
+        !gr->dh0 || !gr->dx_prev || !gr->dB_prev)
+        return M3_ERR_NULL;
+    const void* f4[] = {dt, A, lam, theta, D, dhT, gr->dx, gr->dB, gr->dC, gr->ddt, gr->dA,
+                        gr->dlam, gr->dtheta, gr->dD, gr->dh0, gr->dx_prev, gr->dB_prev};
+    for (const void* q : f4)
+        if (q && !aligned(q, 4)) return M3_ERR_ALIGN;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(dy, 16))
+        return M3_ERR_ALIGN;
+    const int N = d->dstate, P = d->headdim, R = d->rank;
+    if (!scan_bwd_shape_ok(N, P, R)) return M3_ERR_UNSUPPORTED;
+    size_t need = 0;
+    m3_scan_bwd_workspace_bytes(d, seqlen, &need);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return M3_ERR_WORKSPACE;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.x = x; a.B = B; a.C = C; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D;
+    a.h0 = state0->h; a.x_prev = state0->x_prev; a.B_prev = state0->B_prev;
+    a.dy = dy; a.dhT = dhT;
+    a.dx = gr->dx; a.dB = gr->dB; a.dC = gr->dC; a.ddt = gr->ddt; a.dA = gr->dA;
+    a.dlam = gr->dlam; a.dtheta = gr->dtheta; a.dD = D ? gr->dD : nullptr; a.dh0 = gr->dh0;
+    a.dx_prev = gr->dx_prev; a.dB_prev = gr->dB_prev;
+    a.nseg = scan_bwd_nseg(seqlen);
+    float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+    a.ckpt = ws;
+    a.segbuf = ws + (size_t)d->batch * d->nheads * (size_t)N * P * a.nseg;
+    a.T = seqlen; a.batch = d->batch; a.H = d->nheads; a.G = d->ngroups; a.P = P; a.N = N;
+    a.flags = flags;
+
+    // the group sums are accumulated: clear them first (stream-ordered)
+    const size_t bT = (size_t)d->batch * seqlen;
+    const size_t G = d->ngroups;
+    if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess ||
+        cudaMemsetAsync(gr->dB, 0, sizeof(float) * bT * G * R * N, s) != cudaSuccess ||
+        cudaMemsetAsync(gr->dC, 0, sizeof(float) * bT * G * R * N, s) != cudaSuccess ||
+        cudaMemsetAsync(gr->dtheta, 0, sizeof(float) * bT * G * (N / 2), s) != cudaSuccess ||
+        cudaMemsetAsync(gr->dB_prev, 0, sizeof(float) * d->batch * G * R * N, s) != cudaSuccess ||
+        (a.dD && cudaMemsetAsync(gr->dD, 0, sizeof(float) * d->nheads, s) != cudaSuccess))
+        return M3_ERR_CUDA;
+    return launch_status(launch_scan_bwd(a, R, d->io_dtype, s));
+}
+
 m3_status m3_query_status(const void* workspace, void* stream) {
     if (!workspace) return M3_ERR_NULL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

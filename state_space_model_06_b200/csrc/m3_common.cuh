@@ -96,4 +96,38 @@ struct ScanArgs {
     uint32_t flags;
 };
 
+// Argument block of one backward call (gradients of m3_scan_fwd without extras).
+struct BwdArgs {
+    const void* x;       // [b][T][H][R][P] io
+    const void* B;       // [b][T][G][R][N] io
+    const void* C;       // [b][T][G][R][N] io
+    const float* dt;     // [b][T][H]
+    const float* A;      // [b][T][H]
+    const float* lam;    // [b][T][H]
+    const float* theta;  // [b][T][G][N/2]
+    const float* D;      // [H] or null
+    const float* h0;     // [b][H][N][P]   state the forward call started from
+    const void* x_prev;  // [b][H][R][P] io
+    const void* B_prev;  // [b][G][R][N] io
+    const void* dy;      // [b][T][H][R][P] io: dL/dy
+    const float* dhT;    // [b][H][N][P]: dL/dh_T, or null
+    float* dx;           // [b][T][H][R][P]
+    float* dB;           // [b][T][G][R][N]  (summed over the group's heads; zeroed by the host)
+    float* dC;           // [b][T][G][R][N]  (likewise)
+    float* ddt;          // [b][T][H]
+    float* dA;           // [b][T][H]
+    float* dlam;         // [b][T][H]
+    float* dtheta;       // [b][T][G][N/2]   (likewise)
+    float* dD;           // [H] (summed over batch and tokens; zeroed by the host) or null
+    float* dh0;          // [b][H][N][P]
+    float* dx_prev;      // [b][H][R][P]
+    float* dB_prev;      // [b][G][R][N]     (likewise)
+    float* ckpt;         // workspace: [b][H][nseg][N][P] states before each segment
+    float* segbuf;       // workspace: [b][H][seg][N][P] recomputed states of one segment
+    int nseg;
+    long long T;
+    int batch, H, G, P, N;
+    uint32_t flags;
+};
+
 }  // namespace m3

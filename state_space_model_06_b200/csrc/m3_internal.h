@@ -27,6 +27,14 @@ size_t bc_scale_floats(int batch, long long T, int G, int R);
 cudaError_t launch_bc_scales(const ScanArgs& a, int R, int io_dtype, float eps, float* out,
                              cudaStream_t s);
 
+// backward pass (sequential fp32, one CTA per (batch, head)): shapes it covers, workspace
+// floats (checkpoints every scan_bwd_seg_tokens() tokens plus one segment of states per head)
+bool scan_bwd_shape_ok(int N, int P, int R);
+size_t scan_bwd_ws_floats(int batch, int H, int N, int P, long long T);
+int scan_bwd_nseg(long long T);
+int scan_bwd_seg_tokens();
+cudaError_t launch_scan_bwd(const BwdArgs& a, int R, int io_dtype, cudaStream_t s);
+
 // B_prev <- B[:, t] for every (batch, group): the previous-token input of the
 // next call, written after every head of the group has read the old value.
 cudaError_t launch_copy_prev(void* B_prev, const void* B, long long T, long long t, int batch,

@@ -27,7 +27,8 @@ M3_FLAG_TEST_STALL = 4
 EXPORTED = ("m3_state_bytes", "m3_state_init", "m3_scan_workspace_bytes", "m3_scan_fwd",
             "m3_decode_step", "m3_query_status", "m3_scan_fwd_noalloc", "m3_scan_fwd_gated",
             "m3_decode_step_gated", "m3_scan_workspace_bytes_ex", "m3_scan_fwd_ex",
-            "m3_decode_step_ex", "m3_status_string")
+            "m3_decode_step_ex", "m3_scan_bwd_workspace_bytes", "m3_scan_bwd",
+            "m3_status_string")
 
 
 class M3Error(RuntimeError):
@@ -45,6 +46,11 @@ class m3_dims(ctypes.Structure):
 
 class m3_state(ctypes.Structure):
     _fields_ = [("h", ctypes.c_void_p), ("x_prev", ctypes.c_void_p), ("B_prev", ctypes.c_void_p)]
+
+
+class m3_grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dx", "dB", "dC", "ddt", "dA", "dlam", "dtheta",
+                                               "dD", "dh0", "dx_prev", "dB_prev")]
 
 
 class m3_extras(ctypes.Structure):
@@ -84,6 +90,9 @@ def load_library(path: str = LIB_PATH):
         lib.m3_decode_step_ex.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, ep, sp, vp, u32, vp]
         lib.m3_scan_fwd_noalloc.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp,
                                             u32, vp]
+        lib.m3_scan_bwd_workspace_bytes.argtypes = [dp, i32, szp]
+        lib.m3_scan_bwd.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp, vp,
+                                    ctypes.POINTER(m3_grads), vp, sz, u32, vp]
         lib.m3_query_status.argtypes = [vp, vp]
         lib.m3_status_string.argtypes = [ctypes.c_int]
         lib.m3_status_string.restype = ctypes.c_char_p
@@ -294,3 +303,45 @@ def alloc_workspace(dims: Dims, seqlen: int, chunk: int, device="cuda") -> torch
     """A workspace tensor of the size m3_scan_fwd needs (256-byte aligned by torch)."""
     n = m3_scan_workspace_bytes(dims, seqlen, chunk)
     return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+GRAD_NAMES = ("dx", "dB", "dC", "ddt", "dA", "dlam", "dtheta", "dD", "dh0", "dx_prev", "dB_prev")
+
+
+def alloc_grads(dims: Dims, seqlen: int, device="cuda") -> dict:
+    """fp32 gradient tensors of m3_scan_bwd, in its layouts."""
+    b, H, G, P, N, R, T = (dims.batch, dims.nheads, dims.ngroups, dims.headdim, dims.dstate,
+                           dims.rank, seqlen)
+    f = dict(dtype=torch.float32, device=device)
+    return dict(dx=torch.empty(b, T, H, R, P, **f), dB=torch.empty(b, T, G, R, N, **f),
+                dC=torch.empty(b, T, G, R, N, **f), ddt=torch.empty(b, T, H, **f),
+                dA=torch.empty(b, T, H, **f), dlam=torch.empty(b, T, H, **f),
+                dtheta=torch.empty(b, T, G, N // 2, **f), dD=torch.empty(H, **f),
+                dh0=torch.empty(b, H, N, P, **f), dx_prev=torch.empty(b, H, R, P, **f),
+                dB_prev=torch.empty(b, G, R, N, **f))
+
+
+def m3_scan_bwd_workspace_bytes(dims: Dims, seqlen: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().m3_scan_bwd_workspace_bytes(ctypes.byref(dims.c()), int(seqlen),
+                                                      ctypes.byref(n)),
+           "m3_scan_bwd_workspace_bytes")
+    return n.value
+
+
+def alloc_bwd_workspace(dims: Dims, seqlen: int, device="cuda") -> torch.Tensor:
+    return torch.zeros(m3_scan_bwd_workspace_bytes(dims, seqlen), dtype=torch.uint8,
+                       device=device)
+
+
+def m3_scan_bwd(dims: Dims, seqlen: int, x, B, C, dt, A, lam, theta, D, state0: State, dy,
+                dhT, grads: dict, workspace, flags: int = 0, stream=None):
+    """Backward pass of m3_scan_fwd: gradients into ``grads`` (see alloc_grads); state0 is
+    the state the forward call started from (read only); dhT may be None."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = state0.c()
+    g = m3_grads(*(_ptr(grads.get(k)) for k in GRAD_NAMES))
+    _check(load_library().m3_scan_bwd(
+        ctypes.byref(dims.c()), int(seqlen), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A),
+        _ptr(lam), _ptr(theta), _ptr(D), ctypes.byref(st), _ptr(dy), _ptr(dhT), ctypes.byref(g),
+        _ptr(workspace), ws_bytes, int(flags), _stream(stream)), "m3_scan_bwd")
