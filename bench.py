@@ -424,7 +424,7 @@ def backward_leg(args, w, d, g, dev, stream, rank, ws_world, pk):
     del ws, gr, dy
     return {"tokens_per_s": val, "ms_per_step": ms_max, "alg_bytes_per_step": reads + writes,
             "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"], "steps": steps,
-            "kernel": "scan_bwd_kernel (sequential fp32, checkpoints every 16 tokens)"}
+            "kernel": "scan_bwd_kernel (sequential fp32, segment checkpoints) + group sums"}
 
 
 def w_dec_batch(name):

@@ -286,11 +286,11 @@ m3_status m3_decode_step_gated(const m3_dims* dims, const void* x, const void* B
  *        dB_prev [b][G][R][N] (summed over the group's heads).
  *   The carried x_prev / B_prev outputs of the forward call (copies of its last token) get no
  *   gradient here: a caller chaining calls adds theirs to dx / dB of the last token.
- *   The states are recomputed inside (checkpoints every 16 tokens in the workspace); the
- *   call runs sequential fp32 kernels, one CTA per (batch, head).  Supported: N even, N <= 256,
- *   P <= 64, R in {1, 2, 3, 4, 8} (else M3_ERR_UNSUPPORTED).  seqlen 0 does nothing.
- *   Group sums use fp32 atomics, so dB, dC, dtheta, dB_prev and dD may differ in the last
- *   bits from run to run.
+ *   The states are recomputed inside (checkpoints every segment of up to 16 tokens, in the
+ *   workspace); the call runs a sequential fp32 kernel, one CTA per (batch, head), then sums
+ *   the per-head shares of the group gradients (deterministic: no atomics).  Supported: N
+ *   even, N <= 256, P <= 64, R in {1, 2, 3, 4, 8} (else M3_ERR_UNSUPPORTED).  seqlen 0 does
+ *   nothing.
  */
 typedef struct {
     float* dx;
@@ -306,8 +306,9 @@ typedef struct {
     float* dB_prev;
 } m3_grads;
 
-/* Workspace bytes of m3_scan_bwd for (dims, seqlen): the status block plus, per (batch,
- * head), one N x P fp32 state per 16 tokens and one 16-token segment of states. */
+/* Workspace bytes of m3_scan_bwd for (dims, seqlen): the status block; per (batch, head)
+ * one N x P fp32 state per segment and one segment of states; and the per-head shares of
+ * the group gradients (2 R N + N/2 floats per token and head). */
 m3_status m3_scan_bwd_workspace_bytes(const m3_dims* dims, int32_t seqlen, size_t* bytes);
 
 m3_status m3_scan_bwd(const m3_dims* dims, int32_t seqlen, const void* x, const void* B,

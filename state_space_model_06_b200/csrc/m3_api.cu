@@ -353,7 +353,8 @@ m3_status m3_scan_bwd_workspace_bytes(const m3_dims* d, int32_t seqlen, size_t* 
     if (st != M3_OK) return st;
     if (!bytes) return M3_ERR_NULL;
     if (seqlen < 0) return M3_ERR_SHAPE;
-    const size_t fl = scan_bwd_ws_floats(d->batch, d->nheads, d->dstate, d->headdim, seqlen);
+    const size_t fl = scan_bwd_workspace(d->batch, d->nheads, d->dstate, d->headdim, d->rank,
+                                         seqlen).floats;
     *bytes = kStatusBytes + ((fl * sizeof(float) + 255) / 256) * 256;
     return M3_OK;
 }
@@ -394,23 +395,14 @@ m3_status m3_scan_bwd(const m3_dims* d, int32_t seqlen, const void* x, const voi
     a.dx = gr->dx; a.dB = gr->dB; a.dC = gr->dC; a.ddt = gr->ddt; a.dA = gr->dA;
     a.dlam = gr->dlam; a.dtheta = gr->dtheta; a.dD = D ? gr->dD : nullptr; a.dh0 = gr->dh0;
     a.dx_prev = gr->dx_prev; a.dB_prev = gr->dB_prev;
-    a.nseg = scan_bwd_nseg(seqlen);
+    const BwdWorkspace wp = scan_bwd_workspace(d->batch, d->nheads, N, P, R, seqlen);
     float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
-    a.ckpt = ws;
-    a.segbuf = ws + (size_t)d->batch * d->nheads * (size_t)N * P * a.nseg;
+    a.seg = wp.seg; a.nseg = wp.nseg;
+    a.ckpt = ws + wp.ckpt; a.segbuf = ws + wp.segbuf; a.pB = ws + wp.pB; a.pC = ws + wp.pC;
+    a.pth = ws + wp.pth; a.pBprev = ws + wp.pBprev; a.pD = ws + wp.pD;
     a.T = seqlen; a.batch = d->batch; a.H = d->nheads; a.G = d->ngroups; a.P = P; a.N = N;
     a.flags = flags;
-
-    // the group sums are accumulated: clear them first (stream-ordered)
-    const size_t bT = (size_t)d->batch * seqlen;
-    const size_t G = d->ngroups;
-    if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess ||
-        cudaMemsetAsync(gr->dB, 0, sizeof(float) * bT * G * R * N, s) != cudaSuccess ||
-        cudaMemsetAsync(gr->dC, 0, sizeof(float) * bT * G * R * N, s) != cudaSuccess ||
-        cudaMemsetAsync(gr->dtheta, 0, sizeof(float) * bT * G * (N / 2), s) != cudaSuccess ||
-        cudaMemsetAsync(gr->dB_prev, 0, sizeof(float) * d->batch * G * R * N, s) != cudaSuccess ||
-        (a.dD && cudaMemsetAsync(gr->dD, 0, sizeof(float) * d->nheads, s) != cudaSuccess))
-        return M3_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return M3_ERR_CUDA;
     return launch_status(launch_scan_bwd(a, R, d->io_dtype, s));
 }
 

@@ -112,19 +112,25 @@ struct BwdArgs {
     const void* dy;      // [b][T][H][R][P] io: dL/dy
     const float* dhT;    // [b][H][N][P]: dL/dh_T, or null
     float* dx;           // [b][T][H][R][P]
-    float* dB;           // [b][T][G][R][N]  (summed over the group's heads; zeroed by the host)
+    float* dB;           // [b][T][G][R][N]  (summed over the group's heads)
     float* dC;           // [b][T][G][R][N]  (likewise)
     float* ddt;          // [b][T][H]
     float* dA;           // [b][T][H]
     float* dlam;         // [b][T][H]
     float* dtheta;       // [b][T][G][N/2]   (likewise)
-    float* dD;           // [H] (summed over batch and tokens; zeroed by the host) or null
+    float* dD;           // [H] (summed over batch and tokens) or null
     float* dh0;          // [b][H][N][P]
     float* dx_prev;      // [b][H][R][P]
     float* dB_prev;      // [b][G][R][N]     (likewise)
-    float* ckpt;         // workspace: [b][H][nseg][N][P] states before each segment
-    float* segbuf;       // workspace: [b][H][seg][N][P] recomputed states of one segment
-    int nseg;
+    // workspace
+    float* ckpt;         // [b][H][nseg][N][P] states before each segment
+    float* segbuf;       // [b][H][seg][N][P] recomputed states of one segment
+    float* pB;           // [b][T][H][R][N] per-head shares of dB
+    float* pC;           // [b][T][H][R][N] per-head shares of dC
+    float* pth;          // [b][T][H][N/2]  per-head shares of dtheta
+    float* pBprev;       // [b][H][R][N]    per-head shares of dB_prev
+    float* pD;           // [b][H]          per-(row, head) shares of dD
+    int seg, nseg;       // tokens per segment, segments
     long long T;
     int batch, H, G, P, N;
     uint32_t flags;

@@ -27,12 +27,15 @@ size_t bc_scale_floats(int batch, long long T, int G, int R);
 cudaError_t launch_bc_scales(const ScanArgs& a, int R, int io_dtype, float eps, float* out,
                              cudaStream_t s);
 
-// backward pass (sequential fp32, one CTA per (batch, head)): shapes it covers, workspace
-// floats (checkpoints every scan_bwd_seg_tokens() tokens plus one segment of states per head)
+// backward pass (sequential fp32, one CTA per (batch, head)): the shapes it covers and its
+// workspace plan (float offsets of the checkpoints, the segment buffer and the per-head
+// partial sums), then the kernels (the pass itself and the group / batch sums)
+struct BwdWorkspace {
+    int seg, nseg;
+    size_t ckpt, segbuf, pB, pC, pth, pBprev, pD, floats;
+};
 bool scan_bwd_shape_ok(int N, int P, int R);
-size_t scan_bwd_ws_floats(int batch, int H, int N, int P, long long T);
-int scan_bwd_nseg(long long T);
-int scan_bwd_seg_tokens();
+BwdWorkspace scan_bwd_workspace(int batch, int H, int N, int P, int R, long long T);
 cudaError_t launch_scan_bwd(const BwdArgs& a, int R, int io_dtype, cudaStream_t s);
 
 // B_prev <- B[:, t] for every (batch, group): the previous-token input of the

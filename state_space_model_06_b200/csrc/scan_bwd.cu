@@ -13,49 +13,73 @@
 // and through alpha = e^{dt A}, beta = (1 - lam) dt alpha, gamma = lam dt, phi = dt theta.
 //
 // One CTA per (batch, head), sequential in time, fp32.  Thread (pair i, column block cb) holds
-// h_t and Lam for state rows 2i, 2i+1 and up to kCP columns in registers.  The states of the
-// forward are recomputed: a first pass stores h at every kSeg-th token (checkpoints); then, for
-// each segment from the last, its kSeg states are recomputed into a small buffer (kSeg N P
-// floats per head, L2-resident) and the segment is swept in reverse.  Sums over columns (dC,
-// dB, the angle and the scalar terms) are warp shuffles across the CB lanes of a pair; sums
-// over the state pairs (dX and the scalars of dt, A, lam) go through shared memory.  B, C,
-// theta and B_prev are shared by the heads of a group, so their gradients are accumulated
-// with fp32 atomics (order-dependent rounding only).
+// h_t and Lam for state rows 2i, 2i+1 and up to CPM columns in registers.  Tokens are taken in
+// segments of `seg` (<= 16, by the shared-memory budget): a segment's inputs are staged in
+// shared memory at once (X and B from the token before the segment, so the previous token's
+// X and B need no copy; the coefficients and the rotation's cos / sin precomputed), so that
+// forward steps need no barrier.  A first pass stores h before every segment (checkpoints);
+// then, from the last segment, its states are recomputed into a per-head buffer (seg N P
+// floats, L2-resident) and the segment is swept in reverse.  Sums over columns (dC, dB, the
+// angle and the scalar terms) are shuffles across a pair's CB lanes; sums over state pairs
+// (dX, and the scalars of dt, A, lam) go through shared memory, spread over all threads.
+// B, C, theta, B_prev and D are shared across heads or batch rows: each head writes its own
+// partial sums to the workspace and a second kernel adds them up (deterministic).
 #include "m3_internal.h"
 
 namespace m3 {
 
 namespace {
 
-constexpr int kCP = 16;    // most columns per thread
-constexpr int kSeg = 16;   // tokens per checkpoint segment
+// ranks of 3 and more keep R-fold partial sums per pair in registers: at most 512 threads
+__host__ __device__ constexpr int bwd_max_threads(int R) { return R >= 3 ? 512 : 1024; }
 
 struct BwdShape {
     int CB, CP, NT;        // column blocks, columns per block, threads
+    int KS;                // threads per dX element in the pair sums (power of two)
 };
 
-__host__ __device__ inline BwdShape bwd_shape(int N, int P) {
+// At most 8 columns per thread; down to 4 while the threads fit (more, lighter threads hide
+// the per-token latency chain better).
+__host__ __device__ inline BwdShape bwd_shape(int N, int P, int R) {
     BwdShape s;
-    s.CB = P <= 16 ? 1 : (P <= 32 ? 2 : 4);
+    s.CB = 1;
+    while ((P + s.CB - 1) / s.CB > 8) s.CB *= 2;
+    while (s.CB < 16 && (P + 2 * s.CB - 1) / (2 * s.CB) >= 4 &&
+           (N / 2) * 2 * s.CB <= bwd_max_threads(R))
+        s.CB *= 2;
     s.CP = (P + s.CB - 1) / s.CB;
     s.NT = (N / 2) * s.CB;
+    s.KS = 1;
+    while (s.KS < 32 && 2 * s.KS * R * P <= s.NT) s.KS *= 2;
     return s;
 }
 
-// shared memory floats: staging of one token (X, dY, Xp [R][P]; B, C, Bp [R][N]; cos, sin
-// [N/2]; 8 scalars), the carried dX of the previous token [R][P], the per-pair partials of the
-// pair sums ([N/2][R][P] twice) and of the scalars ([4][N/2])
-__host__ __device__ inline size_t bwd_smem_floats(int N, int P, int R) {
-    return (size_t)3 * R * P + 3 * R * N + N + 8 + R * P + 2 * (size_t)(N / 2) * R * P + 4 * (N / 2);
+// shared memory floats with segments of `seg` tokens: X, B of seg + 1 tokens; dY, C,
+// coefficients [8], cos, sin of seg tokens; the carried dX [R][P]; the pair partials
+// ([N/2][R][P] twice) and the scalar partials ([4][N/2])
+__host__ __device__ inline size_t bwd_smem_floats(int N, int P, int R, int seg) {
+    const size_t RP = (size_t)R * P, RN = (size_t)R * N;
+    return (seg + 1) * (RP + RN) + seg * (RP + RN + 8 + N) + RP + 2 * (size_t)(N / 2) * RP +
+           4 * (N / 2);
 }
 
-template <typename IO, int R>
-__global__ void __launch_bounds__(512) scan_bwd_kernel(BwdArgs a) {
+// longest segment (<= 16 tokens) whose staging keeps two CTAs on an SM, else one
+inline int bwd_seg(int N, int P, int R) {
+    for (int budget : {100 * 1024, 227 * 1024})
+        for (int seg = 16; seg >= 1; seg /= 2)
+            if (sizeof(float) * bwd_smem_floats(N, P, R, seg) <= (size_t)budget) return seg;
+    return 0;
+}
+
+// CPM: columns per thread the registers are sized for (4 or 8; the shape's CP <= CPM)
+template <typename IO, int R, int CPM>
+__global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a) {
     extern __shared__ float sm[];
-    const int N = a.N, P = a.P, H = a.H, G = a.G;
+    const int N = a.N, P = a.P, H = a.H, G = a.G, SEG = a.seg;
+    const int RP = R * P, RN = R * N, NH = N / 2;
     const long long T = a.T;
-    const BwdShape sh = bwd_shape(N, P);
-    const int CB = sh.CB, CP = sh.CP, NT = sh.NT;
+    const BwdShape sh = bwd_shape(N, P, R);
+    const int CB = sh.CB, CP = sh.CP, NT = sh.NT, KS = sh.KS;
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh - b * H, g = h / (H / G);
     const int tid = threadIdx.x;
@@ -66,81 +90,97 @@ __global__ void __launch_bounds__(512) scan_bwd_kernel(BwdArgs a) {
     const int wlanes = min(32, NT - (tid & ~31));
     const unsigned full = wlanes == 32 ? 0xffffffffu : ((1u << wlanes) - 1u);
 
-    float* sX = sm;                    // [R][P]
-    float* sG = sX + R * P;            // [R][P] dY
-    float* sXp = sG + R * P;           // [R][P] previous token's X
-    float* sB = sXp + R * P;           // [R][N]
-    float* sC = sB + R * N;            // [R][N]
-    float* sBp = sC + R * N;           // [R][N] previous token's B
-    float* scs = sBp + R * N;          // [N/2]
-    float* ssn = scs + N / 2;          // [N/2]
-    float* ssc = ssn + N / 2;          // alpha beta gamma dt A lam
-    float* cxp = ssc + 8;              // [R][P] dX of the previous token (beta part)
-    float* pu = cxp + R * P;           // [N/2][R][P] gamma B^T Lam partials
-    float* pp = pu + (size_t)(N / 2) * R * P;   // [N/2][R][P] beta Bp^T dM partials
-    float* red = pp + (size_t)(N / 2) * R * P;  // [4][N/2] dalpha dbeta dgamma sum dphi theta
+    float* sX = sm;                                  // [SEG+1][R][P] tokens t0-1 .. t1-1
+    float* sB = sX + (size_t)(SEG + 1) * RP;         // [SEG+1][R][N]
+    float* sG = sB + (size_t)(SEG + 1) * RN;         // [SEG][R][P] dY
+    float* sC = sG + (size_t)SEG * RP;               // [SEG][R][N]
+    float* sK = sC + (size_t)SEG * RN;               // [SEG][8] alpha beta gamma dt A lam
+    float* sCs = sK + (size_t)SEG * 8;               // [SEG][N/2] cos
+    float* sSn = sCs + (size_t)SEG * NH;             // [SEG][N/2] sin
+    float* cxp = sSn + (size_t)SEG * NH;             // [R][P] dX of the previous token
+    float* pu = cxp + RP;                            // [N/2][R][P] B^T Lam per pair
+    float* pp = pu + (size_t)NH * RP;                // [N/2][R][P] Bp^T dM per pair
+    float* red = pp + (size_t)NH * RP;               // [4][N/2] dalpha dbeta dgamma dphi.theta
 
     const size_t NP = (size_t)N * P;
     float* ck = a.ckpt + (size_t)bh * a.nseg * NP;       // checkpoints: h before each segment
-    float* sb = a.segbuf + (size_t)bh * kSeg * NP;       // recomputed states of one segment
+    float* sb = a.segbuf + (size_t)bh * SEG * NP;        // recomputed states of one segment
     const IO* xg = static_cast<const IO*>(a.x);
     const IO* Bg = static_cast<const IO*>(a.B);
     const IO* Cg = static_cast<const IO*>(a.C);
     const IO* dyg = static_cast<const IO*>(a.dy);
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
 
-    // stage token t (t >= 0): X, B, C (C and dY only when `rev`), the previous token's X, B
-    // (the carried state at t = 0), the rotation and the coefficients
-    auto stage = [&](long long t, bool rev) {
-        const size_t bt = (size_t)b * T + t;
-        for (int e = tid; e < R * P; e += NT) {
-            sX[e] = to_f(xg[(bt * H + h) * R * P + e]);
-            if (rev) sG[e] = to_f(dyg[(bt * H + h) * R * P + e]);
-            sXp[e] = t > 0 ? to_f(xg[((bt - 1) * H + h) * R * P + e])
-                           : to_f(static_cast<const IO*>(a.x_prev)[(size_t)bh * R * P + e]);
+    // stage tokens [t0, t1): X, B of t0-1 .. t1-1 (the carried state for t0 - 1 = -1);
+    // with `rev` also dY and C; the coefficients and the rotation of every token
+    auto stage = [&](long long t0, long long t1, bool rev) {
+        const int nt = (int)(t1 - t0);
+        for (int e = tid; e < (nt + 1) * RP; e += NT) {
+            const int u = e / RP, k = e - u * RP;
+            const long long t = t0 - 1 + u;
+            sX[e] = t >= 0 ? to_f(xg[(((size_t)b * T + t) * H + h) * RP + k])
+                           : to_f(static_cast<const IO*>(a.x_prev)[(size_t)bh * RP + k]);
         }
-        for (int e = tid; e < R * N; e += NT) {
-            sB[e] = to_f(Bg[(bt * G + g) * R * N + e]);
-            if (rev) sC[e] = to_f(Cg[(bt * G + g) * R * N + e]);
-            sBp[e] = t > 0 ? to_f(Bg[((bt - 1) * G + g) * R * N + e])
-                           : to_f(static_cast<const IO*>(a.B_prev)[((size_t)b * G + g) * R * N + e]);
+        for (int e = tid; e < (nt + 1) * RN; e += NT) {
+            const int u = e / RN, k = e - u * RN;
+            const long long t = t0 - 1 + u;
+            sB[e] = t >= 0 ? to_f(Bg[(((size_t)b * T + t) * G + g) * RN + k])
+                           : to_f(static_cast<const IO*>(a.B_prev)[((size_t)b * G + g) * RN + k]);
         }
-        const float dt = a.dt[bt * H + h];
-        for (int k = tid; k < N / 2; k += NT) {
-            const float th = a.theta[(bt * G + g) * (N / 2) + k];
-            float s, c;
-            sincosf(angle ? th : dt * th, &s, &c);
-            scs[k] = c;
-            ssn[k] = s;
+        if (rev) {
+            for (int e = tid; e < nt * RP; e += NT) {
+                const int u = e / RP, k = e - u * RP;
+                sG[e] = to_f(dyg[(((size_t)b * T + t0 + u) * H + h) * RP + k]);
+            }
+            for (int e = tid; e < nt * RN; e += NT) {
+                const int u = e / RN, k = e - u * RN;
+                sC[e] = to_f(Cg[(((size_t)b * T + t0 + u) * G + g) * RN + k]);
+            }
         }
-        if (tid == 0) {
-            const float Av = a.A[bt * H + h], lv = a.lam[bt * H + h];
+        for (int u = tid; u < nt; u += NT) {
+            const size_t bt = (size_t)b * T + t0 + u;
+            const float dt = a.dt[bt * H + h], Av = a.A[bt * H + h], lv = a.lam[bt * H + h];
             const float al = expf(dt * Av);
-            ssc[0] = al;
-            ssc[1] = (1.f - lv) * dt * al;
-            ssc[2] = lv * dt;
-            ssc[3] = dt;
-            ssc[4] = Av;
-            ssc[5] = lv;
+            float* k8 = sK + u * 8;
+            k8[0] = al;
+            k8[1] = (1.f - lv) * dt * al;
+            k8[2] = lv * dt;
+            k8[3] = dt;
+            k8[4] = Av;
+            k8[5] = lv;
+        }
+        for (int e = tid; e < nt * NH; e += NT) {
+            const int u = e / NH, k = e - u * NH;
+            const size_t bt = (size_t)b * T + t0 + u;
+            const float th = a.theta[(bt * G + g) * NH + k];
+            float s, c;
+            sincosf(angle ? th : a.dt[bt * H + h] * th, &s, &c);
+            sCs[e] = c;
+            sSn[e] = s;
         }
     };
 
-    // one forward step of this thread's state elements (staged token)
-    float hs[2][kCP];
-    auto fwd_step = [&]() {
-        const float al = ssc[0], be = ssc[1], ga = ssc[2];
-        const float c = scs[i], s = ssn[i];
+    float hs[2][CPM];
+    // one forward step of this thread's state elements for staged token u
+    auto fwd_step = [&](int u) {
+        const float* k8 = sK + u * 8;
+        const float al = k8[0], be = k8[1], ga = k8[2];
+        const float c = sCs[u * NH + i], s = sSn[u * NH + i];
+        const float* Xt = sX + (size_t)(u + 1) * RP;
+        const float* Xq = sX + (size_t)u * RP;
+        const float* Bt = sB + (size_t)(u + 1) * RN;
+        const float* Bq = sB + (size_t)u * RN;
 #pragma unroll
-        for (int q = 0; q < kCP; ++q) {
+        for (int q = 0; q < CPM; ++q) {
             const int p = c0 + q;
             if (q < CP && p < P) {
                 float ub0 = 0.f, ub1 = 0.f, ug0 = 0.f, ug1 = 0.f;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    ub0 = fmaf(sBp[r * N + n0], sXp[r * P + p], ub0);
-                    ub1 = fmaf(sBp[r * N + n1], sXp[r * P + p], ub1);
-                    ug0 = fmaf(sB[r * N + n0], sX[r * P + p], ug0);
-                    ug1 = fmaf(sB[r * N + n1], sX[r * P + p], ug1);
+                    ub0 = fmaf(Bq[r * N + n0], Xq[r * P + p], ub0);
+                    ub1 = fmaf(Bq[r * N + n1], Xq[r * P + p], ub1);
+                    ug0 = fmaf(Bt[r * N + n0], Xt[r * P + p], ug0);
+                    ug1 = fmaf(Bt[r * N + n1], Xt[r * P + p], ug1);
                 }
                 const float m0 = fmaf(al, hs[0][q], be * ub0), m1 = fmaf(al, hs[1][q], be * ub1);
                 hs[0][q] = fmaf(c, m0, fmaf(-s, m1, ga * ug0));
@@ -150,7 +190,7 @@ __global__ void __launch_bounds__(512) scan_bwd_kernel(BwdArgs a) {
     };
     auto load_state = [&](const float* src) {
 #pragma unroll
-        for (int q = 0; q < kCP; ++q) {
+        for (int q = 0; q < CPM; ++q) {
             const int p = c0 + q;
             if (q < CP && p < P) {
                 hs[0][q] = src[(size_t)n0 * P + p];
@@ -162,7 +202,7 @@ __global__ void __launch_bounds__(512) scan_bwd_kernel(BwdArgs a) {
     };
     auto store_state = [&](float* dst) {
 #pragma unroll
-        for (int q = 0; q < kCP; ++q) {
+        for (int q = 0; q < CPM; ++q) {
             const int p = c0 + q;
             if (q < CP && p < P) {
                 dst[(size_t)n0 * P + p] = hs[0][q];
@@ -173,89 +213,115 @@ __global__ void __launch_bounds__(512) scan_bwd_kernel(BwdArgs a) {
 
     // ---- pass 1: forward from h0, keeping h before every segment
     load_state(a.h0 + (size_t)bh * NP);
-    for (long long t = 0; t < T; ++t) {
-        if (t % kSeg == 0) store_state(ck + (size_t)(t / kSeg) * NP);
+    for (int seg = 0; seg < a.nseg; ++seg) {
+        const long long t0 = (long long)seg * SEG, t1 = t0 + SEG < T ? t0 + SEG : T;
+        store_state(ck + (size_t)seg * NP);
+        __syncthreads();            // the previous segment's steps are done with the staging
+        stage(t0, t1, false);
         __syncthreads();
-        stage(t, false);
-        __syncthreads();
-        fwd_step();
+        for (int u = 0; u < (int)(t1 - t0); ++u) fwd_step(u);
     }
 
     // ---- pass 2: segments in reverse; recompute their states, then sweep them backwards
-    float lam_[2][kCP];
+    float lam_[2][CPM];
     if (a.dhT) {
         load_state(a.dhT + (size_t)bh * NP);
 #pragma unroll
-        for (int q = 0; q < kCP; ++q) { lam_[0][q] = hs[0][q]; lam_[1][q] = hs[1][q]; }
+        for (int q = 0; q < CPM; ++q) { lam_[0][q] = hs[0][q]; lam_[1][q] = hs[1][q]; }
     } else {
 #pragma unroll
-        for (int q = 0; q < kCP; ++q) lam_[0][q] = lam_[1][q] = 0.f;
+        for (int q = 0; q < CPM; ++q) lam_[0][q] = lam_[1][q] = 0.f;
     }
-    for (int e = tid; e < R * P; e += NT) cxp[e] = 0.f;
+    for (int e = tid; e < RP; e += NT) cxp[e] = 0.f;
+    float carry[2][R];              // beta_{t+1} dM_{t+1} X_t^T of this pair: dB of token t
+#pragma unroll
+    for (int r = 0; r < R; ++r) carry[0][r] = carry[1][r] = 0.f;
     float dD_acc = 0.f;
     const float Dh = a.D ? a.D[h] : 0.f;
+    // pair sums: dX element e by KS adjacent lanes (ks = lane offset), or a strided loop
+    const bool ps_on = tid < KS * RP || KS == 1;
+    const unsigned ps_mask = __ballot_sync(full, tid < KS * RP);
     for (int seg = a.nseg - 1; seg >= 0; --seg) {
-        const long long t0 = (long long)seg * kSeg;
-        const long long t1 = t0 + kSeg < T ? t0 + kSeg : T;
+        const long long t0 = (long long)seg * SEG, t1 = t0 + SEG < T ? t0 + SEG : T;
+        const int nt = (int)(t1 - t0);
+        __syncthreads();
+        stage(t0, t1, true);
+        __syncthreads();
         load_state(ck + (size_t)seg * NP);
-        for (long long t = t0; t < t1; ++t) {
-            __syncthreads();
-            stage(t, false);
-            __syncthreads();
-            fwd_step();
-            store_state(sb + (size_t)(t - t0) * NP);
+        for (int u = 0; u < nt; ++u) {
+            fwd_step(u);
+            if (u + 1 < nt) store_state(sb + (size_t)u * NP);   // h_{t0+u}: h_{t-1} of the next
         }
-        for (long long t = t1 - 1; t >= t0; --t) {
-            // this thread's h_t (registers) and h_{t-1} (read per column below)
-            load_state(sb + (size_t)(t - t0) * NP);
-            const float* hprev = t > t0 ? sb + (size_t)(t - 1 - t0) * NP : ck + (size_t)seg * NP;
-            __syncthreads();   // the previous token's pair sums are done with the staging
-            stage(t, true);
-            __syncthreads();
-            const float al = ssc[0], be = ssc[1], ga = ssc[2];
-            const float c = scs[i], s = ssn[i];
+        // hs = h_{t1-1}
+        for (int u = nt - 1; u >= 0; --u) {
+            const long long t = t0 + u;
+            const size_t bt = (size_t)b * T + t;
+            const float* hprev = u > 0 ? sb + (size_t)(u - 1) * NP : ck + (size_t)seg * NP;
+            const float* k8 = sK + u * 8;
+            const float al = k8[0], be = k8[1], ga = k8[2];
+            const float c = sCs[u * NH + i], s = sSn[u * NH + i];
+            const float* Xt = sX + (size_t)(u + 1) * RP;
+            const float* Xq = sX + (size_t)u * RP;
+            const float* Bt = sB + (size_t)(u + 1) * RN;
+            const float* Bq = sB + (size_t)u * RN;
+            const float* Gt = sG + (size_t)u * RP;
+            const float* Ct = sC + (size_t)u * RN;
             float cn[2][R], tn[2][R], sn[2][R];
 #pragma unroll
             for (int r = 0; r < R; ++r) cn[0][r] = cn[1][r] = tn[0][r] = tn[1][r] = sn[0][r] = sn[1][r] = 0.f;
             float dphi = 0.f, dal = 0.f;
+            // h_{t-1} of this thread's elements, 4 columns at a time: each group's loads are
+            // issued before any of them is used
+            float hpv[2][4];
 #pragma unroll
-            for (int q = 0; q < kCP; ++q) {
+            for (int q = 0; q < CPM; ++q) {
                 const int p = c0 + q;
+                if (q % 4 == 0) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const bool in = q + j < CP && p + j < P;
+                        hpv[0][j] = in ? hprev[(size_t)n0 * P + p + j] : 0.f;
+                        hpv[1][j] = in ? hprev[(size_t)n1 * P + p + j] : 0.f;
+                    }
+                }
                 if (q < CP && p < P) {
+                    const float hp0 = hpv[0][q % 4], hp1 = hpv[1][q % 4];
                     float l0 = lam_[0][q], l1 = lam_[1][q];
                     float bx0 = 0.f, bx1 = 0.f;
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
-                        const float gv = sG[r * P + p], xv = sX[r * P + p];
-                        l0 = fmaf(sC[r * N + n0], gv, l0);
-                        l1 = fmaf(sC[r * N + n1], gv, l1);
+                        const float gv = Gt[r * P + p], xv = Xt[r * P + p];
+                        l0 = fmaf(Ct[r * N + n0], gv, l0);
+                        l1 = fmaf(Ct[r * N + n1], gv, l1);
                         cn[0][r] = fmaf(hs[0][q], gv, cn[0][r]);
                         cn[1][r] = fmaf(hs[1][q], gv, cn[1][r]);
-                        bx0 = fmaf(sB[r * N + n0], xv, bx0);
-                        bx1 = fmaf(sB[r * N + n1], xv, bx1);
+                        bx0 = fmaf(Bt[r * N + n0], xv, bx0);
+                        bx1 = fmaf(Bt[r * N + n1], xv, bx1);
                     }
-                    float* pur = pu + (size_t)i * R * P + p;
-                    float* ppr = pp + (size_t)i * R * P + p;
+                    float* pur = pu + (size_t)i * RP + p;
+                    float* ppr = pp + (size_t)i * RP + p;
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
-                        const float xv = sX[r * P + p];
+                        const float xv = Xt[r * P + p];
                         tn[0][r] = fmaf(l0, xv, tn[0][r]);
                         tn[1][r] = fmaf(l1, xv, tn[1][r]);
-                        pur[r * P] = fmaf(sB[r * N + n0], l0, sB[r * N + n1] * l1);
+                        pur[r * P] = fmaf(Bt[r * N + n0], l0, Bt[r * N + n1] * l1);
                     }
                     const float u0 = fmaf(-ga, bx0, hs[0][q]), u1 = fmaf(-ga, bx1, hs[1][q]);
                     dphi = fmaf(l1, u0, fmaf(-l0, u1, dphi));
                     const float dm0 = fmaf(c, l0, s * l1), dm1 = fmaf(-s, l0, c * l1);
-                    dal = fmaf(dm0, hprev[(size_t)n0 * P + p], fmaf(dm1, hprev[(size_t)n1 * P + p], dal));
+                    dal = fmaf(dm0, hp0, fmaf(dm1, hp1, dal));
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
-                        const float xpv = sXp[r * P + p];
+                        const float xpv = Xq[r * P + p];
                         sn[0][r] = fmaf(dm0, xpv, sn[0][r]);
                         sn[1][r] = fmaf(dm1, xpv, sn[1][r]);
-                        ppr[r * P] = fmaf(sBp[r * N + n0], dm0, sBp[r * N + n1] * dm1);
+                        ppr[r * P] = fmaf(Bq[r * N + n0], dm0, Bq[r * N + n1] * dm1);
                     }
                     lam_[0][q] = al * dm0;
                     lam_[1][q] = al * dm1;
+                    hs[0][q] = hp0;      // h_{t-1} is the next token's h_t
+                    hs[1][q] = hp1;
                 }
             }
             // sums over this pair's column blocks
@@ -272,83 +338,174 @@ __global__ void __launch_bounds__(512) scan_bwd_kernel(BwdArgs a) {
                 dphi += __shfl_xor_sync(full, dphi, off);
                 dal += __shfl_xor_sync(full, dal, off);
             }
-            const size_t bt = (size_t)b * T + t;
             if (cb == 0) {
+                // this head's share of the group gradients of token t (and of t - 1's B)
                 float dga = 0.f, dbe = 0.f;
-                float* dCt = a.dC + (bt * G + g) * R * N;
-                float* dBt = a.dB + (bt * G + g) * R * N;
-                float* dBp = t > 0 ? a.dB + ((bt - 1) * G + g) * R * N : a.dB_prev + ((size_t)b * G + g) * R * N;
+                float* pCt = a.pC + (bt * H + h) * RN;
+                float* pBt = a.pB + (bt * H + h) * RN;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    dga = fmaf(sB[r * N + n0], tn[0][r], fmaf(sB[r * N + n1], tn[1][r], dga));
-                    dbe = fmaf(sBp[r * N + n0], sn[0][r], fmaf(sBp[r * N + n1], sn[1][r], dbe));
-                    atomicAdd(dCt + r * N + n0, cn[0][r]);
-                    atomicAdd(dCt + r * N + n1, cn[1][r]);
-                    atomicAdd(dBt + r * N + n0, ga * tn[0][r]);
-                    atomicAdd(dBt + r * N + n1, ga * tn[1][r]);
-                    atomicAdd(dBp + r * N + n0, be * sn[0][r]);
-                    atomicAdd(dBp + r * N + n1, be * sn[1][r]);
+                    dga = fmaf(Bt[r * N + n0], tn[0][r], fmaf(Bt[r * N + n1], tn[1][r], dga));
+                    dbe = fmaf(Bq[r * N + n0], sn[0][r], fmaf(Bq[r * N + n1], sn[1][r], dbe));
+                    pCt[r * N + n0] = cn[0][r];
+                    pCt[r * N + n1] = cn[1][r];
+                    pBt[r * N + n0] = fmaf(ga, tn[0][r], carry[0][r]);
+                    pBt[r * N + n1] = fmaf(ga, tn[1][r], carry[1][r]);
+                    carry[0][r] = be * sn[0][r];
+                    carry[1][r] = be * sn[1][r];
                 }
-                const float th = a.theta[(bt * G + g) * (N / 2) + i];
-                atomicAdd(a.dtheta + (bt * G + g) * (N / 2) + i, angle ? dphi : dphi * ssc[3]);
+                const float th = a.theta[(bt * G + g) * NH + i];
+                a.pth[(bt * H + h) * NH + i] = angle ? dphi : dphi * k8[3];
                 red[i] = dal;
-                red[N / 2 + i] = dbe;
-                red[N + i] = dga;
-                red[3 * (N / 2) + i] = angle ? 0.f : dphi * th;
+                red[NH + i] = dbe;
+                red[2 * NH + i] = dga;
+                red[3 * NH + i] = angle ? 0.f : dphi * th;
             }
             __syncthreads();
-            // sums over the pairs: dX of this token and the carried dX of the previous one
-            float* dXt = a.dx + (bt * H + h) * R * P;
-            for (int e = tid; e < R * P; e += NT) {
+            // sums over the pairs: dX of this token, the carried dX of the previous one
+            float* dXt = a.dx + (bt * H + h) * RP;
+            if (KS > 1) {
+                const int e = tid / KS, ks = tid - e * KS;
                 float su = 0.f, spv = 0.f;
-                for (int k = 0; k < N / 2; ++k) {
-                    su += pu[(size_t)k * R * P + e];
-                    spv += pp[(size_t)k * R * P + e];
+                if (ps_on) {
+                    for (int k = ks; k < NH; k += KS) {
+                        su += pu[(size_t)k * RP + e];
+                        spv += pp[(size_t)k * RP + e];
+                    }
                 }
-                const float gv = sG[e];
-                dXt[e] = fmaf(Dh, gv, fmaf(ga, su, cxp[e]));
-                dD_acc = fmaf(gv, sX[e], dD_acc);
-                cxp[e] = be * spv;   // X_{t-1}'s share (read and written by this thread only)
+                if (tid < KS * RP) {
+                    for (int off = KS >> 1; off > 0; off >>= 1) {
+                        su += __shfl_xor_sync(ps_mask, su, off);
+                        spv += __shfl_xor_sync(ps_mask, spv, off);
+                    }
+                    if (ks == 0) {
+                        const float gv = Gt[e];
+                        dXt[e] = fmaf(Dh, gv, fmaf(ga, su, cxp[e]));
+                        dD_acc = fmaf(gv, Xt[e], dD_acc);
+                        cxp[e] = be * spv;
+                    }
+                }
+            } else {
+                for (int e = tid; e < RP; e += NT) {
+                    float su = 0.f, spv = 0.f;
+                    for (int k = 0; k < NH; ++k) {
+                        su += pu[(size_t)k * RP + e];
+                        spv += pp[(size_t)k * RP + e];
+                    }
+                    const float gv = Gt[e];
+                    dXt[e] = fmaf(Dh, gv, fmaf(ga, su, cxp[e]));
+                    dD_acc = fmaf(gv, Xt[e], dD_acc);
+                    cxp[e] = be * spv;
+                }
             }
-            if (tid == 0) {
+            // the scalars: dalpha, dbeta, dgamma and sum_i dphi_i theta_i over the pairs
+            if (tid < 32) {
                 float v[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int k = 0; k < N / 2; ++k)
+                if (NT >= 32) {
+                    for (int k = tid; k < NH; k += 32)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) v[j] += red[j * (N / 2) + k];
-                const float dt = ssc[3], Av = ssc[4], lv = ssc[5];
-                const float dalpha = v[0], dbeta = v[1], dgamma = v[2];
-                a.ddt[bt * H + h] = dalpha * al * Av + dbeta * (1.f - lv) * (al + dt * al * Av) +
-                                    dgamma * lv + v[3];
-                a.dA[bt * H + h] = dalpha * al * dt + dbeta * (1.f - lv) * dt * al * dt;
-                a.dlam[bt * H + h] = -dbeta * dt * al + dgamma * dt;
+                        for (int j = 0; j < 4; ++j) v[j] += red[j * NH + k];
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) v[j] += __shfl_xor_sync(0xffffffffu, v[j], off);
+                } else if (tid == 0) {
+                    for (int k = 0; k < NH; ++k)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) v[j] += red[j * NH + k];
+                }
+                if (tid == 0) {
+                    const float dt = k8[3], Av = k8[4], lv = k8[5];
+                    a.ddt[bt * H + h] = v[0] * al * Av + v[1] * (1.f - lv) * (al + dt * al * Av) +
+                                        v[2] * lv + v[3];
+                    a.dA[bt * H + h] = v[0] * al * dt + v[1] * (1.f - lv) * dt * al * dt;
+                    a.dlam[bt * H + h] = -v[1] * dt * al + v[2] * dt;
+                }
             }
+            __syncthreads();   // pu, pp, red and cxp are free for the next token
         }
     }
-    __syncthreads();
-    // initial state: dh0 = Lam, dx_prev = the carried dX of token 0, dD over this row's tokens
+    // starting state: dh0 = Lam, dx_prev = the carried dX of token 0, dB_prev = the carried
+    // dB; this head's share of dD
 #pragma unroll
-    for (int q = 0; q < kCP; ++q) {
+    for (int q = 0; q < CPM; ++q) {
         const int p = c0 + q;
         if (q < CP && p < P) {
             a.dh0[(size_t)bh * NP + (size_t)n0 * P + p] = lam_[0][q];
             a.dh0[(size_t)bh * NP + (size_t)n1 * P + p] = lam_[1][q];
         }
     }
-    for (int e = tid; e < R * P; e += NT) a.dx_prev[(size_t)bh * R * P + e] = cxp[e];
-    if (a.D && a.dD && tid < R * P) atomicAdd(a.dD + h, dD_acc);
+    for (int e = tid; e < RP; e += NT) a.dx_prev[(size_t)bh * RP + e] = cxp[e];
+    if (cb == 0) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            a.pBprev[(size_t)bh * RN + r * N + n0] = carry[0][r];
+            a.pBprev[(size_t)bh * RN + r * N + n1] = carry[1][r];
+        }
+    }
+    __syncthreads();
+    pu[tid] = dD_acc;                // NT <= (N/2) R P floats of pu
+    __syncthreads();
+    if (tid == 0) {
+        float v = 0.f;
+        for (int k = 0; k < NT; ++k) v += pu[k];
+        a.pD[bh] = v;
+    }
+}
+
+// out[(o G + g) inner + k] = sum over the group's heads j of in[(o H + g hpg + j) inner + k]
+__global__ void group_sum_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                 long long outer, int G, int hpg, int inner) {
+    const long long n = outer * G * inner;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long o = e / ((long long)G * inner);
+        const int rem = (int)(e - o * G * inner);
+        const int g = rem / inner, k = rem - g * inner;
+        const float* src = in + ((o * G + g) * (long long)hpg) * inner + k;
+        float v = 0.f;
+        for (int j = 0; j < hpg; ++j) v += src[(long long)j * inner];
+        out[e] = v;
+    }
+}
+
+// dD[h] = sum over batch rows of the per-(row, head) partials
+__global__ void batch_sum_kernel(const float* __restrict__ in, float* __restrict__ out, int batch,
+                                 int H) {
+    for (int hh = blockIdx.x * blockDim.x + threadIdx.x; hh < H; hh += gridDim.x * blockDim.x) {
+        float v = 0.f;
+        for (int bb = 0; bb < batch; ++bb) v += in[(size_t)bb * H + hh];
+        out[hh] = v;
+    }
+}
+
+cudaError_t launch_group_sum(const float* in, float* out, long long outer, int G, int hpg,
+                             int inner, cudaStream_t s) {
+    const long long n = outer * G * inner;
+    if (n == 0) return cudaSuccess;
+    const long long blocks = (n + 255) / 256;
+    group_sum_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, s>>>(
+        in, out, outer, G, hpg, inner);
+    return cudaGetLastError();
+}
+
+template <typename IO, int R, int CPM>
+cudaError_t launch_bwd_c(const BwdArgs& a, cudaStream_t s) {
+    const BwdShape sh = bwd_shape(a.N, a.P, R);
+    const size_t smem = sizeof(float) * bwd_smem_floats(a.N, a.P, R, a.seg);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<IO, R, CPM>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    scan_bwd_kernel<IO, R, CPM><<<(unsigned)(a.batch * a.H), sh.NT, smem, s>>>(a);
+    return cudaGetLastError();
 }
 
 template <typename IO, int R>
 cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t s) {
-    const BwdShape sh = bwd_shape(a.N, a.P);
-    const size_t smem = sizeof(float) * bwd_smem_floats(a.N, a.P, R);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<IO, R>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    scan_bwd_kernel<IO, R><<<(unsigned)(a.batch * a.H), sh.NT, smem, s>>>(a);
-    return cudaGetLastError();
+    return bwd_shape(a.N, a.P, R).CP <= 4 ? launch_bwd_c<IO, R, 4>(a, s)
+                                          : launch_bwd_c<IO, R, 8>(a, s);
 }
 
 template <typename IO>
@@ -368,23 +525,49 @@ cudaError_t launch_bwd_io(const BwdArgs& a, int R, cudaStream_t s) {
 bool scan_bwd_shape_ok(int N, int P, int R) {
     if (N < 2 || N > 256 || (N & 1) || P < 1 || P > 64) return false;
     if (R != 1 && R != 2 && R != 3 && R != 4 && R != 8) return false;
-    const BwdShape sh = bwd_shape(N, P);
-    if (sh.NT > 512) return false;
-    return sizeof(float) * bwd_smem_floats(N, P, R) <= 227 * 1024;
+    const BwdShape sh = bwd_shape(N, P, R);
+    // the pair partials buffer ([N/2][R][P]) also collects one float per thread at the end
+    return sh.CP <= 8 && sh.NT <= bwd_max_threads(R) && sh.NT <= (N / 2) * R * P &&
+           bwd_seg(N, P, R) > 0;
 }
 
-size_t scan_bwd_ws_floats(int batch, int H, int N, int P, long long T) {
-    const long long nseg = (T + kSeg - 1) / kSeg;
-    return (size_t)batch * H * (size_t)N * P * (size_t)(nseg + kSeg);
+int scan_bwd_seg(int N, int P, int R) { return bwd_seg(N, P, R); }
+
+BwdWorkspace scan_bwd_workspace(int batch, int H, int N, int P, int R, long long T) {
+    BwdWorkspace w;
+    const int seg = bwd_seg(N, P, R);
+    w.seg = seg > 0 ? seg : 1;
+    w.nseg = (int)((T + w.seg - 1) / w.seg);
+    const size_t bH = (size_t)batch * H, NP = (size_t)N * P;
+    size_t o = 0;
+    w.ckpt = o;   o += bH * w.nseg * NP;
+    w.segbuf = o; o += bH * w.seg * NP;
+    w.pB = o;     o += (size_t)batch * T * H * R * N;
+    w.pC = o;     o += (size_t)batch * T * H * R * N;
+    w.pth = o;    o += (size_t)batch * T * H * (N / 2);
+    w.pBprev = o; o += bH * R * N;
+    w.pD = o;     o += bH;
+    w.floats = o;
+    return w;
 }
-
-int scan_bwd_nseg(long long T) { return (int)((T + kSeg - 1) / kSeg); }
-
-int scan_bwd_seg_tokens() { return kSeg; }
 
 cudaError_t launch_scan_bwd(const BwdArgs& a, int R, int io_dtype, cudaStream_t s) {
-    if (io_dtype == M3_BF16) return launch_bwd_io<__nv_bfloat16>(a, R, s);
-    return launch_bwd_io<float>(a, R, s);
+    cudaError_t e = io_dtype == M3_BF16 ? launch_bwd_io<__nv_bfloat16>(a, R, s)
+                                        : launch_bwd_io<float>(a, R, s);
+    if (e != cudaSuccess) return e;
+    // group sums of the per-head partials (B, C, theta, B_prev) and the batch sum of D
+    const int hpg = a.H / a.G, RN = R * a.N;
+    const long long bT = (long long)a.batch * a.T;
+    if ((e = launch_group_sum(a.pB, a.dB, bT, a.G, hpg, RN, s)) != cudaSuccess) return e;
+    if ((e = launch_group_sum(a.pC, a.dC, bT, a.G, hpg, RN, s)) != cudaSuccess) return e;
+    if ((e = launch_group_sum(a.pth, a.dtheta, bT, a.G, hpg, a.N / 2, s)) != cudaSuccess) return e;
+    if ((e = launch_group_sum(a.pBprev, a.dB_prev, a.batch, a.G, hpg, RN, s)) != cudaSuccess)
+        return e;
+    if (a.dD) {
+        batch_sum_kernel<<<1, 256, 0, s>>>(a.pD, a.dD, a.batch, a.H);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace m3
