@@ -468,10 +468,10 @@ def ours(args):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     w = inputs.WORKLOADS[WORKLOAD]
-    if args.batch:
-        # smaller batch of the same workload: only for short profiler captures
+    if args.batch or args.seqlen:
+        # a smaller case of the same workload: only for short profiler captures
         import dataclasses
-        w = dataclasses.replace(w, batch=args.batch)
+        w = dataclasses.replace(w, batch=args.batch or w.batch, seqlen=args.seqlen or w.seqlen)
     pk, pk_kind = peaks()
 
     inp, d, g, st, y, ws = prefill_setup(w, dev, seed=rank)
@@ -485,7 +485,8 @@ def ours(args):
     achieved = byts / (ms / 1e3) / 1e9
     tflops = flops / (ms / 1e3) / 1e12
     kernel_src = os.path.join(ROOT, "state_space_model_06_b200", "csrc", "scan_tc.cu")
-    traffic = committed_traffic(kernel_src, WORKLOAD)
+    # the committed DRAM counters describe the full workload only
+    traffic = None if (args.batch or args.seqlen) else committed_traffic(kernel_src, WORKLOAD)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_world,
@@ -643,6 +644,8 @@ def main():
     ap.add_argument("--decode-tokens", type=int, default=DECODE_TOKENS,
                     help="sequential decode tokens timed per workload")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling only)")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the sequence length (profiling only)")
     ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and CPU legs")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

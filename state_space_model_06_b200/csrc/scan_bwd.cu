@@ -56,10 +56,10 @@ __host__ __device__ inline BwdShape bwd_shape(int N, int P, int R) {
 
 // shared memory floats with segments of `seg` tokens: X, B of seg + 1 tokens; dY, C,
 // coefficients [8], cos, sin of seg tokens; the carried dX [R][P]; the pair partials
-// ([N/2][R][P] twice) and the scalar partials ([4][N/2])
+// ([N/2] rows of R P + 16, twice) and the scalar partials ([4][N/2])
 __host__ __device__ inline size_t bwd_smem_floats(int N, int P, int R, int seg) {
     const size_t RP = (size_t)R * P, RN = (size_t)R * N;
-    return (seg + 1) * (RP + RN) + seg * (RP + RN + 8 + N) + RP + 2 * (size_t)(N / 2) * RP +
+    return (seg + 1) * (RP + RN) + seg * (RP + RN + 8 + N) + RP + 2 * (size_t)(N / 2) * (RP + 16) +
            4 * (N / 2);
 }
 
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     const int tid = threadIdx.x;
     const int i = tid / CB, cb = tid - i * CB;          // state pair, column block
     const int n0 = 2 * i, n1 = 2 * i + 1;
-    const int c0 = cb * CP;                              // first column of this thread
+    // this thread's columns: cb, cb + CB, cb + 2 CB, ... (adjacent lanes, adjacent columns)
     // lanes of this warp that exist (a pair's CB lanes never straddle a warp: CB divides 32)
     const int wlanes = min(32, NT - (tid & ~31));
     const unsigned full = wlanes == 32 ? 0xffffffffu : ((1u << wlanes) - 1u);
@@ -98,9 +98,11 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     float* sCs = sK + (size_t)SEG * 8;               // [SEG][N/2] cos
     float* sSn = sCs + (size_t)SEG * NH;             // [SEG][N/2] sin
     float* cxp = sSn + (size_t)SEG * NH;             // [R][P] dX of the previous token
-    float* pu = cxp + RP;                            // [N/2][R][P] B^T Lam per pair
-    float* pp = pu + (size_t)NH * RP;                // [N/2][R][P] Bp^T dM per pair
-    float* red = pp + (size_t)NH * RP;               // [4][N/2] dalpha dbeta dgamma dphi.theta
+    const int RPS = RP + 16;                         // padded row: two pairs of a warp in
+                                                     // different banks
+    float* pu = cxp + RP;                            // [N/2][RPS] B^T Lam per pair
+    float* pp = pu + (size_t)NH * RPS;               // [N/2][RPS] Bp^T dM per pair
+    float* red = pp + (size_t)NH * RPS;              // [4][N/2] dalpha dbeta dgamma dphi.theta
 
     const size_t NP = (size_t)N * P;
     float* ck = a.ckpt + (size_t)bh * a.nseg * NP;       // checkpoints: h before each segment
@@ -172,8 +174,8 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
         const float* Bq = sB + (size_t)u * RN;
 #pragma unroll
         for (int q = 0; q < CPM; ++q) {
-            const int p = c0 + q;
-            if (q < CP && p < P) {
+            const int p = cb + q * CB;
+            if (p < P) {
                 float ub0 = 0.f, ub1 = 0.f, ug0 = 0.f, ug1 = 0.f;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
@@ -191,8 +193,8 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     auto load_state = [&](const float* src) {
 #pragma unroll
         for (int q = 0; q < CPM; ++q) {
-            const int p = c0 + q;
-            if (q < CP && p < P) {
+            const int p = cb + q * CB;
+            if (p < P) {
                 hs[0][q] = src[(size_t)n0 * P + p];
                 hs[1][q] = src[(size_t)n1 * P + p];
             } else {
@@ -203,8 +205,8 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     auto store_state = [&](float* dst) {
 #pragma unroll
         for (int q = 0; q < CPM; ++q) {
-            const int p = c0 + q;
-            if (q < CP && p < P) {
+            const int p = cb + q * CB;
+            if (p < P) {
                 dst[(size_t)n0 * P + p] = hs[0][q];
                 dst[(size_t)n1 * P + p] = hs[1][q];
             }
@@ -275,16 +277,17 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
             float hpv[2][4];
 #pragma unroll
             for (int q = 0; q < CPM; ++q) {
-                const int p = c0 + q;
+                const int p = cb + q * CB;
                 if (q % 4 == 0) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const bool in = q + j < CP && p + j < P;
-                        hpv[0][j] = in ? hprev[(size_t)n0 * P + p + j] : 0.f;
-                        hpv[1][j] = in ? hprev[(size_t)n1 * P + p + j] : 0.f;
+                        const int pj = p + j * CB;
+                        const bool in = q + j < CPM && pj < P;
+                        hpv[0][j] = in ? hprev[(size_t)n0 * P + pj] : 0.f;
+                        hpv[1][j] = in ? hprev[(size_t)n1 * P + pj] : 0.f;
                     }
                 }
-                if (q < CP && p < P) {
+                if (p < P) {
                     const float hp0 = hpv[0][q % 4], hp1 = hpv[1][q % 4];
                     float l0 = lam_[0][q], l1 = lam_[1][q];
                     float bx0 = 0.f, bx1 = 0.f;
@@ -298,8 +301,8 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
                         bx0 = fmaf(Bt[r * N + n0], xv, bx0);
                         bx1 = fmaf(Bt[r * N + n1], xv, bx1);
                     }
-                    float* pur = pu + (size_t)i * RP + p;
-                    float* ppr = pp + (size_t)i * RP + p;
+                    float* pur = pu + (size_t)i * RPS + p;
+                    float* ppr = pp + (size_t)i * RPS + p;
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         const float xv = Xt[r * P + p];
@@ -369,8 +372,8 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
                 float su = 0.f, spv = 0.f;
                 if (ps_on) {
                     for (int k = ks; k < NH; k += KS) {
-                        su += pu[(size_t)k * RP + e];
-                        spv += pp[(size_t)k * RP + e];
+                        su += pu[(size_t)k * RPS + e];
+                        spv += pp[(size_t)k * RPS + e];
                     }
                 }
                 if (tid < KS * RP) {
@@ -389,8 +392,8 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
                 for (int e = tid; e < RP; e += NT) {
                     float su = 0.f, spv = 0.f;
                     for (int k = 0; k < NH; ++k) {
-                        su += pu[(size_t)k * RP + e];
-                        spv += pp[(size_t)k * RP + e];
+                        su += pu[(size_t)k * RPS + e];
+                        spv += pp[(size_t)k * RPS + e];
                     }
                     const float gv = Gt[e];
                     dXt[e] = fmaf(Dh, gv, fmaf(ga, su, cxp[e]));
@@ -429,8 +432,8 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     // dB; this head's share of dD
 #pragma unroll
     for (int q = 0; q < CPM; ++q) {
-        const int p = c0 + q;
-        if (q < CP && p < P) {
+        const int p = cb + q * CB;
+        if (p < P) {
             a.dh0[(size_t)bh * NP + (size_t)n0 * P + p] = lam_[0][q];
             a.dh0[(size_t)bh * NP + (size_t)n1 * P + p] = lam_[1][q];
         }
