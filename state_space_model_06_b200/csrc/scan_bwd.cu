@@ -35,7 +35,6 @@ __host__ __device__ constexpr int bwd_max_threads(int R) { return R >= 3 ? 512 :
 
 struct BwdShape {
     int CB, CP, NT;        // column blocks, columns per block, threads
-    int KS;                // threads per dX element in the pair sums (power of two)
 };
 
 // At most 8 columns per thread; down to 4 while the threads fit (more, lighter threads hide
@@ -49,18 +48,15 @@ __host__ __device__ inline BwdShape bwd_shape(int N, int P, int R) {
         s.CB *= 2;
     s.CP = (P + s.CB - 1) / s.CB;
     s.NT = (N / 2) * s.CB;
-    s.KS = 1;
-    while (s.KS < 32 && 2 * s.KS * R * P <= s.NT) s.KS *= 2;
     return s;
 }
 
 // shared memory floats with segments of `seg` tokens: X, B of seg + 1 tokens; dY, C,
-// coefficients [8], cos, sin of seg tokens; the carried dX [R][P]; the pair partials
-// ([N/2] rows of R P + 16, twice) and the scalar partials ([4][N/2])
+// coefficients [8], cos, sin of seg tokens; the carried dX [R][P]; the segment's sums over
+// the state pairs (B^T Lam and Bp^T dM [seg][R][P], the four scalars [seg][4]); one scratch
 __host__ __device__ inline size_t bwd_smem_floats(int N, int P, int R, int seg) {
     const size_t RP = (size_t)R * P, RN = (size_t)R * N;
-    return (seg + 1) * (RP + RN) + seg * (RP + RN + 8 + N) + RP + 2 * (size_t)(N / 2) * (RP + 16) +
-           4 * (N / 2);
+    return (seg + 1) * (RP + RN) + seg * (RP + RN + 8 + N) + RP + 2 * seg * RP + 4 * seg + 4;
 }
 
 // longest segment (<= 16 tokens) whose staging keeps two CTAs on an SM, else one
@@ -79,7 +75,7 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     const int RP = R * P, RN = R * N, NH = N / 2;
     const long long T = a.T;
     const BwdShape sh = bwd_shape(N, P, R);
-    const int CB = sh.CB, CP = sh.CP, NT = sh.NT, KS = sh.KS;
+    const int CB = sh.CB, NT = sh.NT;
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh - b * H, g = h / (H / G);
     const int tid = threadIdx.x;
@@ -89,6 +85,7 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     // lanes of this warp that exist (a pair's CB lanes never straddle a warp: CB divides 32)
     const int wlanes = min(32, NT - (tid & ~31));
     const unsigned full = wlanes == 32 ? 0xffffffffu : ((1u << wlanes) - 1u);
+    const int lane = tid & 31;
 
     float* sX = sm;                                  // [SEG+1][R][P] tokens t0-1 .. t1-1
     float* sB = sX + (size_t)(SEG + 1) * RP;         // [SEG+1][R][N]
@@ -98,11 +95,10 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     float* sCs = sK + (size_t)SEG * 8;               // [SEG][N/2] cos
     float* sSn = sCs + (size_t)SEG * NH;             // [SEG][N/2] sin
     float* cxp = sSn + (size_t)SEG * NH;             // [R][P] dX of the previous token
-    const int RPS = RP + 16;                         // padded row: two pairs of a warp in
-                                                     // different banks
-    float* pu = cxp + RP;                            // [N/2][RPS] B^T Lam per pair
-    float* pp = pu + (size_t)NH * RPS;               // [N/2][RPS] Bp^T dM per pair
-    float* red = pp + (size_t)NH * RPS;              // [4][N/2] dalpha dbeta dgamma dphi.theta
+    float* accU = cxp + RP;                          // [SEG][R][P] sum over pairs of B^T Lam
+    float* accP = accU + (size_t)SEG * RP;           // [SEG][R][P] sum over pairs of Bp^T dM
+    float* accK = accP + (size_t)SEG * RP;           // [SEG][4] dalpha dbeta dgamma dphi.theta
+    float* scratch = accK + (size_t)SEG * 4;
 
     const size_t NP = (size_t)N * P;
     float* ck = a.ckpt + (size_t)bh * a.nseg * NP;       // checkpoints: h before each segment
@@ -224,6 +220,17 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
         for (int u = 0; u < (int)(t1 - t0); ++u) fwd_step(u);
     }
 
+    // v summed over the state pairs this warp holds, added to *dst (shared) once per warp and
+    // column; the lanes of a partial warp add their own values
+    auto pair_add = [&](float* dst, float v, bool on) {
+        if (wlanes == 32) {
+            for (int off = CB; off < 32; off <<= 1) v += __shfl_xor_sync(full, v, off);
+            if (lane < CB && on) atomicAdd(dst, v);
+        } else if (on) {
+            atomicAdd(dst, v);
+        }
+    };
+
     // ---- pass 2: segments in reverse; recompute their states, then sweep them backwards
     float lam_[2][CPM];
     if (a.dhT) {
@@ -240,14 +247,13 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
     for (int r = 0; r < R; ++r) carry[0][r] = carry[1][r] = 0.f;
     float dD_acc = 0.f;
     const float Dh = a.D ? a.D[h] : 0.f;
-    // pair sums: dX element e by KS adjacent lanes (ks = lane offset), or a strided loop
-    const bool ps_on = tid < KS * RP || KS == 1;
-    const unsigned ps_mask = __ballot_sync(full, tid < KS * RP);
     for (int seg = a.nseg - 1; seg >= 0; --seg) {
         const long long t0 = (long long)seg * SEG, t1 = t0 + SEG < T ? t0 + SEG : T;
         const int nt = (int)(t1 - t0);
         __syncthreads();
         stage(t0, t1, true);
+        for (int e = tid; e < 2 * nt * RP; e += NT) accU[e < nt * RP ? e : SEG * RP + e - nt * RP] = 0.f;
+        for (int e = tid; e < 4 * nt; e += NT) accK[e] = 0.f;
         __syncthreads();
         load_state(ck + (size_t)seg * NP);
         for (int u = 0; u < nt; ++u) {
@@ -272,6 +278,7 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
 #pragma unroll
             for (int r = 0; r < R; ++r) cn[0][r] = cn[1][r] = tn[0][r] = tn[1][r] = sn[0][r] = sn[1][r] = 0.f;
             float dphi = 0.f, dal = 0.f;
+            float vu[R], vp[R];
             // h_{t-1} of this thread's elements, 4 columns at a time: each group's loads are
             // issued before any of them is used
             float hpv[2][4];
@@ -287,6 +294,8 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
                         hpv[1][j] = in ? hprev[(size_t)n1 * P + pj] : 0.f;
                     }
                 }
+#pragma unroll
+                for (int r = 0; r < R; ++r) vu[r] = vp[r] = 0.f;
                 if (p < P) {
                     const float hp0 = hpv[0][q % 4], hp1 = hpv[1][q % 4];
                     float l0 = lam_[0][q], l1 = lam_[1][q];
@@ -301,14 +310,12 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
                         bx0 = fmaf(Bt[r * N + n0], xv, bx0);
                         bx1 = fmaf(Bt[r * N + n1], xv, bx1);
                     }
-                    float* pur = pu + (size_t)i * RPS + p;
-                    float* ppr = pp + (size_t)i * RPS + p;
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         const float xv = Xt[r * P + p];
                         tn[0][r] = fmaf(l0, xv, tn[0][r]);
                         tn[1][r] = fmaf(l1, xv, tn[1][r]);
-                        pur[r * P] = fmaf(Bt[r * N + n0], l0, Bt[r * N + n1] * l1);
+                        vu[r] = fmaf(Bt[r * N + n0], l0, Bt[r * N + n1] * l1);
                     }
                     const float u0 = fmaf(-ga, bx0, hs[0][q]), u1 = fmaf(-ga, bx1, hs[1][q]);
                     dphi = fmaf(l1, u0, fmaf(-l0, u1, dphi));
@@ -319,12 +326,19 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
                         const float xpv = Xq[r * P + p];
                         sn[0][r] = fmaf(dm0, xpv, sn[0][r]);
                         sn[1][r] = fmaf(dm1, xpv, sn[1][r]);
-                        ppr[r * P] = fmaf(Bq[r * N + n0], dm0, Bq[r * N + n1] * dm1);
+                        vp[r] = fmaf(Bq[r * N + n0], dm0, Bq[r * N + n1] * dm1);
                     }
                     lam_[0][q] = al * dm0;
                     lam_[1][q] = al * dm1;
                     hs[0][q] = hp0;      // h_{t-1} is the next token's h_t
                     hs[1][q] = hp1;
+                }
+                // this column's sums over the pairs, for dX of t and of t - 1 (uniform code:
+                // every lane of the warp takes part)
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    pair_add(accU + (size_t)u * RP + r * P + p, vu[r], p < P);
+                    pair_add(accP + (size_t)u * RP + r * P + p, vp[r], p < P);
                 }
             }
             // sums over this pair's column blocks
@@ -341,15 +355,21 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
                 dphi += __shfl_xor_sync(full, dphi, off);
                 dal += __shfl_xor_sync(full, dal, off);
             }
+            // per pair (every lane of a pair holds the pair's sums): the scalar terms
+            float dga = 0.f, dbe = 0.f;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                dga = fmaf(Bt[r * N + n0], tn[0][r], fmaf(Bt[r * N + n1], tn[1][r], dga));
+                dbe = fmaf(Bq[r * N + n0], sn[0][r], fmaf(Bq[r * N + n1], sn[1][r], dbe));
+            }
+            const float th = a.theta[(bt * G + g) * NH + i];
+            const float dpt = angle ? 0.f : dphi * th;
             if (cb == 0) {
                 // this head's share of the group gradients of token t (and of t - 1's B)
-                float dga = 0.f, dbe = 0.f;
                 float* pCt = a.pC + (bt * H + h) * RN;
                 float* pBt = a.pB + (bt * H + h) * RN;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    dga = fmaf(Bt[r * N + n0], tn[0][r], fmaf(Bt[r * N + n1], tn[1][r], dga));
-                    dbe = fmaf(Bq[r * N + n0], sn[0][r], fmaf(Bq[r * N + n1], sn[1][r], dbe));
                     pCt[r * N + n0] = cn[0][r];
                     pCt[r * N + n1] = cn[1][r];
                     pBt[r * N + n0] = fmaf(ga, tn[0][r], carry[0][r]);
@@ -357,76 +377,51 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
                     carry[0][r] = be * sn[0][r];
                     carry[1][r] = be * sn[1][r];
                 }
-                const float th = a.theta[(bt * G + g) * NH + i];
                 a.pth[(bt * H + h) * NH + i] = angle ? dphi : dphi * k8[3];
-                red[i] = dal;
-                red[NH + i] = dbe;
-                red[2 * NH + i] = dga;
-                red[3 * NH + i] = angle ? 0.f : dphi * th;
             }
-            __syncthreads();
-            // sums over the pairs: dX of this token, the carried dX of the previous one
-            float* dXt = a.dx + (bt * H + h) * RP;
-            if (KS > 1) {
-                const int e = tid / KS, ks = tid - e * KS;
-                float su = 0.f, spv = 0.f;
-                if (ps_on) {
-                    for (int k = ks; k < NH; k += KS) {
-                        su += pu[(size_t)k * RPS + e];
-                        spv += pp[(size_t)k * RPS + e];
+            // the scalars summed over the pairs: a full warp folds its pairs, a partial warp's
+            // pairs add their own
+            {
+                float v0 = dal, v1 = dbe, v2 = dga, v3 = dpt;
+                if (wlanes == 32) {
+                    for (int off = CB; off < 32; off <<= 1) {
+                        v0 += __shfl_xor_sync(full, v0, off);
+                        v1 += __shfl_xor_sync(full, v1, off);
+                        v2 += __shfl_xor_sync(full, v2, off);
+                        v3 += __shfl_xor_sync(full, v3, off);
                     }
                 }
-                if (tid < KS * RP) {
-                    for (int off = KS >> 1; off > 0; off >>= 1) {
-                        su += __shfl_xor_sync(ps_mask, su, off);
-                        spv += __shfl_xor_sync(ps_mask, spv, off);
-                    }
-                    if (ks == 0) {
-                        const float gv = Gt[e];
-                        dXt[e] = fmaf(Dh, gv, fmaf(ga, su, cxp[e]));
-                        dD_acc = fmaf(gv, Xt[e], dD_acc);
-                        cxp[e] = be * spv;
-                    }
-                }
-            } else {
-                for (int e = tid; e < RP; e += NT) {
-                    float su = 0.f, spv = 0.f;
-                    for (int k = 0; k < NH; ++k) {
-                        su += pu[(size_t)k * RPS + e];
-                        spv += pp[(size_t)k * RPS + e];
-                    }
-                    const float gv = Gt[e];
-                    dXt[e] = fmaf(Dh, gv, fmaf(ga, su, cxp[e]));
-                    dD_acc = fmaf(gv, Xt[e], dD_acc);
-                    cxp[e] = be * spv;
+                if (wlanes == 32 ? lane == 0 : cb == 0) {
+                    atomicAdd(accK + u * 4 + 0, v0);
+                    atomicAdd(accK + u * 4 + 1, v1);
+                    atomicAdd(accK + u * 4 + 2, v2);
+                    atomicAdd(accK + u * 4 + 3, v3);
                 }
             }
-            // the scalars: dalpha, dbeta, dgamma and sum_i dphi_i theta_i over the pairs
-            if (tid < 32) {
-                float v[4] = {0.f, 0.f, 0.f, 0.f};
-                if (NT >= 32) {
-                    for (int k = tid; k < NH; k += 32)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) v[j] += red[j * NH + k];
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) v[j] += __shfl_xor_sync(0xffffffffu, v[j], off);
-                } else if (tid == 0) {
-                    for (int k = 0; k < NH; ++k)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) v[j] += red[j * NH + k];
-                }
-                if (tid == 0) {
-                    const float dt = k8[3], Av = k8[4], lv = k8[5];
-                    a.ddt[bt * H + h] = v[0] * al * Av + v[1] * (1.f - lv) * (al + dt * al * Av) +
-                                        v[2] * lv + v[3];
-                    a.dA[bt * H + h] = v[0] * al * dt + v[1] * (1.f - lv) * dt * al * dt;
-                    a.dlam[bt * H + h] = -v[1] * dt * al + v[2] * dt;
-                }
-            }
-            __syncthreads();   // pu, pp, red and cxp are free for the next token
         }
+        __syncthreads();
+        // the segment's dX: D dY + gamma_t (B^T Lam)_t + beta_{t+1} (Bp^T dM)_{t+1}, the last
+        // term from the next segment (cxp) for the segment's last token
+        for (int e = tid; e < nt * RP; e += NT) {
+            const int u = e / RP, k = e - u * RP;
+            const size_t bt = (size_t)b * T + t0 + u;
+            const float nxt = u + 1 < nt ? sK[(u + 1) * 8 + 1] * accP[(size_t)(u + 1) * RP + k] : cxp[k];
+            const float gv = sG[(size_t)u * RP + k];
+            a.dx[(bt * H + h) * RP + k] = fmaf(Dh, gv, fmaf(sK[u * 8 + 2], accU[(size_t)u * RP + k], nxt));
+            dD_acc = fmaf(gv, sX[(size_t)(u + 1) * RP + k], dD_acc);
+        }
+        // the coefficients' gradients of the segment's tokens
+        for (int u = tid; u < nt; u += NT) {
+            const size_t bt = (size_t)b * T + t0 + u;
+            const float* k8 = sK + u * 8;
+            const float al = k8[0], dt = k8[3], Av = k8[4], lv = k8[5];
+            const float v0 = accK[u * 4], v1 = accK[u * 4 + 1], v2 = accK[u * 4 + 2], v3 = accK[u * 4 + 3];
+            a.ddt[bt * H + h] = v0 * al * Av + v1 * (1.f - lv) * (al + dt * al * Av) + v2 * lv + v3;
+            a.dA[bt * H + h] = v0 * al * dt + v1 * (1.f - lv) * dt * al * dt;
+            a.dlam[bt * H + h] = -v1 * dt * al + v2 * dt;
+        }
+        __syncthreads();   // every read of cxp above is done
+        for (int k = tid; k < RP; k += NT) cxp[k] = sK[1] * accP[k];   // X_{t0-1}'s share
     }
     // starting state: dh0 = Lam, dx_prev = the carried dX of token 0, dB_prev = the carried
     // dB; this head's share of dD
@@ -446,14 +441,11 @@ __global__ void __launch_bounds__(bwd_max_threads(R)) scan_bwd_kernel(BwdArgs a)
             a.pBprev[(size_t)bh * RN + r * N + n1] = carry[1][r];
         }
     }
+    if (tid == 0) *scratch = 0.f;
     __syncthreads();
-    pu[tid] = dD_acc;                // NT <= (N/2) R P floats of pu
+    atomicAdd(scratch, dD_acc);
     __syncthreads();
-    if (tid == 0) {
-        float v = 0.f;
-        for (int k = 0; k < NT; ++k) v += pu[k];
-        a.pD[bh] = v;
-    }
+    if (tid == 0) a.pD[bh] = *scratch;
 }
 
 // out[(o G + g) inner + k] = sum over the group's heads j of in[(o H + g hpg + j) inner + k]
@@ -529,9 +521,7 @@ bool scan_bwd_shape_ok(int N, int P, int R) {
     if (N < 2 || N > 256 || (N & 1) || P < 1 || P > 64) return false;
     if (R != 1 && R != 2 && R != 3 && R != 4 && R != 8) return false;
     const BwdShape sh = bwd_shape(N, P, R);
-    // the pair partials buffer ([N/2][R][P]) also collects one float per thread at the end
-    return sh.CP <= 8 && sh.NT <= bwd_max_threads(R) && sh.NT <= (N / 2) * R * P &&
-           bwd_seg(N, P, R) > 0;
+    return sh.CP <= 8 && sh.NT <= bwd_max_threads(R) && bwd_seg(N, P, R) > 0;
 }
 
 int scan_bwd_seg(int N, int P, int R) { return bwd_seg(N, P, R); }
