@@ -193,3 +193,32 @@ def test_binding_refuses_missing_library(tmp_path):
             m3.load_library(str(tmp_path / "missing.so"))
     finally:
         m3._lib = old
+
+
+def test_backward_validation_before_launch(lib):
+    """m3_scan_bwd checks its arguments (nulls, alignment, supported shape, workspace size)
+    before anything is launched."""
+    d = m3.Dims(1, 2, 1, 16, 16, 1, m3.M3_F32)
+    st = m3.m3_state(0x2000, 0x3000, 0x4000)
+    p, ws = 0x1000, 0x100000
+    need = m3.m3_scan_bwd_workspace_bytes(d, 64)
+    assert need >= 256 + 4 * (2 * 16 * 16 * 4)          # status block + a few states
+    full = m3.m3_grads(*([p] * 11))
+
+    def bwd(dims=d, grads=full, dy=p, ws_bytes=need, T=64, state=st):
+        return lib.m3_scan_bwd(ctypes.byref(dims.c()), T, p, p, p, p, p, p, p, None,
+                               ctypes.byref(state), dy, None,
+                               ctypes.byref(grads) if grads is not None else None, ws, ws_bytes,
+                               0, None)
+
+    assert bwd(T=0) == m3.M3_OK                                   # nothing to do
+    assert bwd(T=-1) == m3.M3_ERR_SHAPE
+    assert bwd(grads=None) == m3.M3_ERR_NULL
+    assert bwd(dy=None) == m3.M3_ERR_NULL
+    assert bwd(grads=m3.m3_grads(*([p] * 10 + [None]))) == m3.M3_ERR_NULL   # dB_prev
+    assert bwd(grads=m3.m3_grads(*([p + 2] + [p] * 10))) == m3.M3_ERR_ALIGN
+    assert bwd(dy=p + 8) == m3.M3_ERR_ALIGN
+    assert bwd(state=m3.m3_state(0x2000, 0, 0x4000)) == m3.M3_ERR_NULL
+    assert bwd(ws_bytes=need - 256) == m3.M3_ERR_WORKSPACE
+    assert bwd(dims=m3.Dims(1, 2, 1, 128, 16, 1, m3.M3_F32),
+               ws_bytes=1 << 30) == m3.M3_ERR_UNSUPPORTED      # headdim 128: no kernel
