@@ -288,8 +288,10 @@ m3_status m3_decode_step_gated(const m3_dims* dims, const void* x, const void* B
  *   gradient here: a caller chaining calls adds theirs to dx / dB of the last token.
  *   The states are recomputed inside (checkpoints every segment of up to 16 tokens, in the
  *   workspace); the call runs a sequential fp32 kernel, one CTA per (batch, head), then sums
- *   the per-head shares of the group gradients (deterministic: no atomics).  Supported: N
- *   even, N <= 256, P <= 64, R in {1, 2, 3, 4, 8} (else M3_ERR_UNSUPPORTED).  seqlen 0 does
+ *   the per-head shares of the group gradients in a fixed order.  The sums over state pairs
+ *   inside a head use shared-memory atomics, so dx, ddt, dA and dlam may differ in the last
+ *   bits from run to run.  Supported: N even, N <= 256, P <= 64, R in {1, 2, 3, 4, 8}, within
+ *   the kernel's thread and shared-memory limits (else M3_ERR_UNSUPPORTED).  seqlen 0 does
  *   nothing.
  */
 typedef struct {

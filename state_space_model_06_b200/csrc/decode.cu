@@ -30,7 +30,9 @@ __device__ __forceinline__ float gate_z(const DecodeArgs& a, size_t bh, int h, i
 // MAXP: the largest pairs-per-thread count this instantiation handles (a.ppt <= MAXP); it
 // sizes the per-thread state registers, so each shape only pays for the pairs it uses.
 // BCM: the instantiation with the BC map (BCNorm and BC biases) of m3_decode_step_ex.
-template <typename IO, int R, int MAXP, bool BCM>
+// XE: the instantiation with the MIMO lightweight expansion of x or z (the plain ones hold
+// none of its code).
+template <typename IO, int R, int MAXP, bool BCM, bool XE>
 __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     extern __shared__ float sm[];
     const int N = a.N, P = a.P, H = a.H, G = a.G;
@@ -64,16 +66,19 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
     }
 
     // 2. stage this token's small inputs in shared memory
-    // x: [R][P], or one value per channel expanded by the head's weights [R][P]
-    const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
-    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * (wx ? 1 : R) * P;
+    // x: [R][P], or (XE) one value per channel expanded by the head's weights [R][P]
+    const float* wx = XE && a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
+    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * (XE && wx ? 1 : R) * P;
     const IO* xp = static_cast<const IO*>(a.x_prev) + (size_t)bh * R * P;
     const size_t gofs = ((size_t)b * G + g) * R * N;
     const IO* Bg = static_cast<const IO*>(a.B) + gofs;
     const IO* Bpg = static_cast<const IO*>(a.B_prev) + gofs;
     const IO* Cg = static_cast<const IO*>(a.C) + gofs;
     for (int e = tid; e < R * P; e += blockDim.x) {
-        xs[e] = wx ? expand_io<IO>(to_f(x[e % P]), wx[e]) : to_f(x[e]);
+        if constexpr (XE)
+            xs[e] = wx ? expand_io<IO>(to_f(x[e % P]), wx[e]) : to_f(x[e]);
+        else
+            xs[e] = to_f(x[e]);
         xps[e] = to_f(xp[e]);
     }
     for (int e = tid; e < R * N; e += blockDim.x) {
@@ -175,24 +180,30 @@ __global__ void __launch_bounds__(512) decode_kernel(DecodeArgs a) {
         float acc = 0.f;
         for (int k = 0; k < RG; ++k) acc += ypart[(size_t)k * R * P + e];
         float v = acc + Dh * xs[e];
-        if (a.z) v = gate_silu(v, gate_z<IO>(a, bh, h, R, P, e));
-        y[e] = from_f<IO>(v);
-        xpo[e] = from_f<IO>(xs[e]);   // x_prev <- X (this head only; exact in the io dtype)
+        if constexpr (XE) {
+            if (a.z) v = gate_silu(v, gate_z<IO>(a, bh, h, R, P, e));
+            y[e] = from_f<IO>(v);
+            xpo[e] = from_f<IO>(xs[e]);   // x_prev <- X (this head only; exact in the io dtype)
+        } else {
+            if (a.z) v = gate_silu(v, to_f(static_cast<const IO*>(a.z)[(size_t)bh * R * P + e]));
+            y[e] = from_f<IO>(v);
+            xpo[e] = x[e];   // x_prev <- x (this head only; read above before the barrier)
+        }
     }
 }
 
-template <typename IO, int R, int MAXP, bool BCM>
+template <typename IO, int R, int MAXP, bool BCM, bool XE>
 static cudaError_t launch_decode_t(const DecodeArgs& a, int batch, cudaStream_t s) {
     const int RG = (a.N / 2) / a.ppt;
     const int threads = (a.P / 4) * RG;
     const size_t smem =
         sizeof(float) * (size_t)(2 * R * a.P + 3 * R * a.N + a.N + RG * R * a.P + 3 * R);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<IO, R, MAXP, BCM>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<IO, R, MAXP, BCM, XE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    decode_kernel<IO, R, MAXP, BCM><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
+    decode_kernel<IO, R, MAXP, BCM, XE><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -222,7 +233,7 @@ static size_t mimo_smem_floats(int N, int P, int R, int ppt, bool bcm) {
            (size_t)rgw * R * P + (bcm ? 3 * R * N + 3 * R : 0);
 }
 
-template <typename IO, int R, int MAXP, bool BCM>
+template <typename IO, int R, int MAXP, bool BCM, bool XE>
 __global__ void __launch_bounds__(512) decode_mimo_kernel(DecodeArgs a) {
     extern __shared__ __align__(16) float sm[];
     constexpr int R2 = 2 * R;
@@ -257,8 +268,8 @@ __global__ void __launch_bounds__(512) decode_mimo_kernel(DecodeArgs a) {
     const float alpha = expf(dt * Av);
     const float beta = (1.f - lam) * dt * alpha;
     const float gamma = lam * dt;
-    const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
-    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * (wx ? 1 : R) * P;
+    const float* wx = XE && a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
+    const IO* x = static_cast<const IO*>(a.x) + (size_t)bh * (XE && wx ? 1 : R) * P;
     const IO* xp = static_cast<const IO*>(a.x_prev) + (size_t)bh * R * P;
     const size_t gofs = ((size_t)b * G + g) * R * N;
     const IO* Bg = static_cast<const IO*>(a.B) + gofs;
@@ -323,7 +334,10 @@ __global__ void __launch_bounds__(512) decode_mimo_kernel(DecodeArgs a) {
     }
     for (int e = tid; e < R * P; e += nthr) {
         V[e] = to_f(xp[e]);
-        V[R * P + e] = wx ? expand_io<IO>(to_f(x[e % P]), wx[e]) : to_f(x[e]);
+        if constexpr (XE)
+            V[R * P + e] = wx ? expand_io<IO>(to_f(x[e % P]), wx[e]) : to_f(x[e]);
+        else
+            V[R * P + e] = to_f(x[e]);
     }
     __syncthreads();
 
@@ -388,59 +402,71 @@ __global__ void __launch_bounds__(512) decode_mimo_kernel(DecodeArgs a) {
         float acc = 0.f;
         for (int w = 0; w < RGW; ++w) acc += ypart[(size_t)w * R * P + e];
         float v = acc + Dh * V[R * P + e];
-        if (a.z) v = gate_silu(v, gate_z<IO>(a, bh, h, R, P, e));
-        y[e] = from_f<IO>(v);
-        xpo[e] = from_f<IO>(V[R * P + e]);   // x_prev <- X (this head only; exact)
+        if constexpr (XE) {
+            if (a.z) v = gate_silu(v, gate_z<IO>(a, bh, h, R, P, e));
+            y[e] = from_f<IO>(v);
+            xpo[e] = from_f<IO>(V[R * P + e]);   // x_prev <- X (this head only; exact)
+        } else {
+            if (a.z) v = gate_silu(v, to_f(static_cast<const IO*>(a.z)[(size_t)bh * R * P + e]));
+            y[e] = from_f<IO>(v);
+            xpo[e] = x[e];   // x_prev <- x (this head only; read above before the barrier)
+        }
     }
 }
 
-template <typename IO, int R, bool BCM>
+template <typename IO, int R, bool BCM, bool XE>
 static cudaError_t launch_decode_mimo(const DecodeArgs& a, int batch, cudaStream_t s) {
     const int RG = (a.N / 2) / a.ppt;
     const int threads = (a.P / 4) * RG;
     const size_t smem = sizeof(float) * mimo_smem_floats(a.N, a.P, R, a.ppt, BCM);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_mimo_kernel<IO, R, 8, BCM>,
+        cudaError_t e = cudaFuncSetAttribute(decode_mimo_kernel<IO, R, 8, BCM, XE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    decode_mimo_kernel<IO, R, 8, BCM><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
+    decode_mimo_kernel<IO, R, 8, BCM, XE><<<(unsigned)(batch * a.H), threads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
 // SISO: the plain kernel with 8 (or 4) pairs per thread.  MIMO: the rank-2R packed kernel
 // when the shape takes 8 pairs per thread, else the plain kernel with 4.
-template <typename IO, bool BCM>
+template <typename IO, bool BCM, bool XE>
 static cudaError_t launch_decode_io(const DecodeArgs& a, int batch, int R, cudaStream_t s) {
     if (a.ppt > 8) return cudaErrorNotSupported;
     if (R != 1 && a.ppt == 8) {
         switch (R) {
-            case 2: return launch_decode_mimo<IO, 2, BCM>(a, batch, s);
-            case 3: return launch_decode_mimo<IO, 3, BCM>(a, batch, s);
-            case 4: return launch_decode_mimo<IO, 4, BCM>(a, batch, s);
-            case 8: return launch_decode_mimo<IO, 8, BCM>(a, batch, s);
+            case 2: return launch_decode_mimo<IO, 2, BCM, XE>(a, batch, s);
+            case 3: return launch_decode_mimo<IO, 3, BCM, XE>(a, batch, s);
+            case 4: return launch_decode_mimo<IO, 4, BCM, XE>(a, batch, s);
+            case 8: return launch_decode_mimo<IO, 8, BCM, XE>(a, batch, s);
             default: return cudaErrorNotSupported;
         }
     }
     if (a.ppt > 4 && R != 1) return cudaErrorNotSupported;
     switch (R) {
-        case 1: return a.ppt > 4 ? launch_decode_t<IO, 1, 8, BCM>(a, batch, s)
-                                 : launch_decode_t<IO, 1, 4, BCM>(a, batch, s);
-        case 2: return launch_decode_t<IO, 2, 4, BCM>(a, batch, s);
-        case 3: return launch_decode_t<IO, 3, 4, BCM>(a, batch, s);
-        case 4: return launch_decode_t<IO, 4, 4, BCM>(a, batch, s);
-        case 8: return launch_decode_t<IO, 8, 4, BCM>(a, batch, s);
+        case 1: return a.ppt > 4 ? launch_decode_t<IO, 1, 8, BCM, XE>(a, batch, s)
+                                 : launch_decode_t<IO, 1, 4, BCM, XE>(a, batch, s);
+        case 2: return launch_decode_t<IO, 2, 4, BCM, XE>(a, batch, s);
+        case 3: return launch_decode_t<IO, 3, 4, BCM, XE>(a, batch, s);
+        case 4: return launch_decode_t<IO, 4, 4, BCM, XE>(a, batch, s);
+        case 8: return launch_decode_t<IO, 8, 4, BCM, XE>(a, batch, s);
         default: return cudaErrorNotSupported;
     }
+}
+
+template <typename IO, bool BCM>
+static cudaError_t launch_decode_x(const DecodeArgs& a, int batch, int R, cudaStream_t s) {
+    return (a.x_expand || a.z_expand) ? launch_decode_io<IO, BCM, true>(a, batch, R, s)
+                                      : launch_decode_io<IO, BCM, false>(a, batch, R, s);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int batch, int R, int io_dtype, cudaStream_t s) {
     const bool bc = a.B_bias || a.C_bias || a.bc_eps > 0.f;
     if (io_dtype == M3_BF16)
-        return bc ? launch_decode_io<__nv_bfloat16, true>(a, batch, R, s)
-                  : launch_decode_io<__nv_bfloat16, false>(a, batch, R, s);
-    return bc ? launch_decode_io<float, true>(a, batch, R, s)
-              : launch_decode_io<float, false>(a, batch, R, s);
+        return bc ? launch_decode_x<__nv_bfloat16, true>(a, batch, R, s)
+                  : launch_decode_x<__nv_bfloat16, false>(a, batch, R, s);
+    return bc ? launch_decode_x<float, true>(a, batch, R, s)
+              : launch_decode_x<float, false>(a, batch, R, s);
 }
 
 // ---------------------------------------------------------------------------------

@@ -21,9 +21,11 @@
 // then, from the last segment, its states are recomputed into a per-head buffer (seg N P
 // floats, L2-resident) and the segment is swept in reverse.  Sums over columns (dC, dB, the
 // angle and the scalar terms) are shuffles across a pair's CB lanes; sums over state pairs
-// (dX, and the scalars of dt, A, lam) go through shared memory, spread over all threads.
-// B, C, theta, B_prev and D are shared across heads or batch rows: each head writes its own
-// partial sums to the workspace and a second kernel adds them up (deterministic).
+// (dX, and the scalars of dt, A, lam) are folded per warp and added into per-segment shared
+// accumulators (shared-memory atomics: the order of the adds, and so the last bits of dX,
+// ddt, dA and dlam, may vary from run to run).  B, C, theta, B_prev and D are shared across
+// heads or batch rows: each head writes its own partial sums to the workspace and a second
+// kernel adds them up in a fixed order.
 #include "m3_internal.h"
 
 namespace m3 {
