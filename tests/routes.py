@@ -172,6 +172,81 @@ def bruteforce_txt(x, B, C, dt, A, lam, theta, D=None, theta_is_angle=False):
     return y
 
 
+def bruteforce_bwd(x, B, C, dt, A, lam, theta, dy, D=None, theta_is_angle=False):
+    """Reverse-mode gradients of the materialised parallel form (fresh sequence), derived by
+    hand through its own quantities rather than through the recurrence:
+
+        Y_t = sum_{s<=t} L[t,s] (C~_t . B~_s) X_s + D X_t,   C~ = R(-psi) C, B~ = R(-psi) B,
+        L[t,s] = exp(cum_t - cum_s) w[t,s],  w[t,s] = gamma_s + [s < t] (1 - lam_{s+1}) dt_{s+1},
+        cum_t = sum_{k<=t} dt_k A_k,  psi_t = sum_{k<=t} dt_k theta_k  ("Parallel representation
+        under SSD"; Proposition 4 for the rotation).
+
+    With G = dL/dY and S the (token, rank) score matrix: dX = (L o S)^T G + D G;
+    dS = L o (G X^T); dL = <S, G X^T> per (t, s); dC~ = dS B~, dB~ = dS^T C~, rotated back by
+    R(psi); dpsi_t = sum over ranks of dC~_0 C~_1 - dC~_1 C~_0 (and the same for B~), summed
+    backwards over tokens into the per-step angles; dL splits into dcum (through the
+    exponential) and dw (gamma_s and the next token's (1 - lam) dt), which reach dt, A and lam.
+    Returns the gradients of the inputs (no starting state) as float64 arrays; B, C, theta
+    gradients are summed over the heads of each group.
+    """
+    b, T, H, R, P, G, N, hpg = _heads(x, B)
+    out = dict(dx=np.zeros(x.shape), dB=np.zeros(B.shape), dC=np.zeros(C.shape),
+               ddt=np.zeros(dt.shape), dA=np.zeros(A.shape), dlam=np.zeros(lam.shape),
+               dtheta=np.zeros(theta.shape), dD=None if D is None else np.zeros(D.shape))
+    tri = np.tril(np.ones((T, T)))
+    strict = np.tril(np.ones((T, T)), -1)
+    for bi in range(b):
+        for h in range(H):
+            g = h // hpg
+            d, a, l = dt[bi, :, h], A[bi, :, h], lam[bi, :, h]
+            cum = np.cumsum(d * a)
+            E = np.exp(np.where(tri > 0, cum[:, None] - cum[None, :], 0.0)) * tri
+            nxt = np.zeros(T)
+            nxt[:-1] = (1.0 - l[1:]) * d[1:]
+            w = (l * d)[None, :] * tri + nxt[None, :] * strict
+            L = E * w
+            th = theta[bi, :, g]
+            ang = th if theta_is_angle else d[:, None] * th
+            psi = np.cumsum(ang, axis=0)
+            bt = np.stack([_rot_pairs(B[bi, t, g], -psi[t]) for t in range(T)])   # [T,R,N]
+            ct = np.stack([_rot_pairs(C[bi, t, g], -psi[t]) for t in range(T)])
+            S = np.einsum("trn,usn->trus", ct, bt)
+            X, Gy = x[bi, :, h], dy[bi, :, h]
+            Dh = 0.0 if D is None else D[h]
+            M = S * L[:, None, :, None]
+            out["dx"][bi, :, h] = np.einsum("trus,trp->usp", M, Gy) + Dh * Gy
+            GX = np.einsum("trp,usp->trus", Gy, X)
+            dS = GX * L[:, None, :, None]
+            dL = np.einsum("trus,trus->tu", S, GX)
+            dct = np.einsum("trus,usn->trn", dS, bt)
+            dbt = np.einsum("trus,trn->usn", dS, ct)
+            out["dC"][bi, :, g] += np.stack([_rot_pairs(dct[t], psi[t]) for t in range(T)])
+            out["dB"][bi, :, g] += np.stack([_rot_pairs(dbt[t], psi[t]) for t in range(T)])
+            dpsi = ((dct[..., 0::2] * ct[..., 1::2] - dct[..., 1::2] * ct[..., 0::2]).sum(axis=1) +
+                    (dbt[..., 0::2] * bt[..., 1::2] - dbt[..., 1::2] * bt[..., 0::2]).sum(axis=1))
+            dang = np.cumsum(dpsi[::-1], axis=0)[::-1]
+            dE, dw = dL * w, dL * E
+            dcum = (dE * E).sum(axis=1) - (dE * E).sum(axis=0)
+            dga = (dw * tri).sum(axis=0)
+            dnx = (dw * strict).sum(axis=0)
+            ddt_, dlam_ = dga * l, dga * d
+            ddt_[1:] += dnx[:-1] * (1.0 - l[1:])
+            dlam_[1:] -= dnx[:-1] * d[1:]
+            dda = np.cumsum(dcum[::-1])[::-1]
+            ddt_ += dda * a
+            if theta_is_angle:
+                out["dtheta"][bi, :, g] += dang
+            else:
+                out["dtheta"][bi, :, g] += dang * d[:, None]
+                ddt_ += (dang * th).sum(axis=1)
+            out["ddt"][bi, :, h] = ddt_
+            out["dA"][bi, :, h] = dda * d
+            out["dlam"][bi, :, h] = dlam_
+            if D is not None:
+                out["dD"][h] += float((Gy * X).sum())
+    return out
+
+
 def implicit_conv_route(x, B, C, dt, A, lam, D=None, h0=None, x_prev=None, B_prev=None):
     """Remark 4 (theta = 0): width-2 data-dependent convolution on v_t = B_t x_t^T,
 

@@ -7,8 +7,10 @@ weights, dL/dv for every element v of every input (x, B, C, dt, A, lam, theta, D
 initial state h0, x_prev, B_prev) must match (L(v + e) - L(v - e)) / 2e to the central
 difference's error (O(e^2) truncation plus rounding), at shapes where each finite difference
 is cheap.  Groups shared by two heads (G = 1, H = 2) check the head sums of the B, C and theta
-gradients; the pre-scaled angle flag checks the theta path without dt.  Planted mistakes in a
-copy of the backward's C source are caught.
+gradients; the pre-scaled angle flag checks the theta path without dt.  A second, independent
+derivation (the hand-derived gradients of the materialised T x T form, tests/routes.py) must
+agree with the oracle's reverse pass through the recurrence for a fresh sequence.  Planted
+mistakes in a copy of the backward's C source are caught.
 """
 import math
 import os
@@ -18,6 +20,7 @@ import numpy as np
 import pytest
 
 import oracle
+import routes
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "m3_oracle.c")
 KEYS = ("x", "B", "C", "dt", "A", "lam", "theta", "D", "h0", "x_prev", "B_prev")
@@ -84,6 +87,19 @@ def test_gradients_match_finite_differences(angle):
 def test_gradients_match_finite_differences_siso_groups():
     """R = 1, two groups of two heads, odd headdim."""
     assert _max_fd_error(9, False, b=1, T=6, H=4, G=2, P=5, N=6, R=1) < 1e-7
+
+
+@pytest.mark.parametrize("angle,R,G", [(False, 2, 1), (True, 1, 2), (False, 3, 2)])
+def test_gradients_match_materialised_form_derivative(angle, R, G):
+    """An independent derivation: the hand-derived gradients of the materialised T x T form
+    (L o C~B~^T) X (tests/routes.py) equal the oracle's reverse pass through the recurrence,
+    for a fresh sequence."""
+    v, Wy, _ = _problem(21 + R, b=2, T=12, H=4, G=G, P=3, N=6, R=R)
+    args = [v[k] for k in ("x", "B", "C", "dt", "A", "lam", "theta")]
+    g = oracle.scan_bwd(*args, Wy, D=v["D"], theta_is_angle=angle)
+    r = routes.bruteforce_bwd(*args, Wy, D=v["D"], theta_is_angle=angle)
+    for k in ("dx", "dB", "dC", "ddt", "dA", "dlam", "dtheta", "dD"):
+        assert np.max(np.abs(g[k] - r[k])) <= 1e-11 * max(1.0, np.max(np.abs(r[k]))), k
 
 
 def test_zero_loss_weights_give_zero_gradients():
