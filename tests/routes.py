@@ -247,6 +247,156 @@ def bruteforce_bwd(x, B, C, dt, A, lam, theta, dy, D=None, theta_is_angle=False)
     return out
 
 
+def chunked_bwd(x, B, C, dt, A, lam, theta, dy, chunk, D=None, h0=None, x_prev=None,
+                B_prev=None, dhT=None, theta_is_angle=False):
+    """Reverse-mode gradients of the chunked form, in the call's rotated frame (the algorithm
+    a chunked backward runs; "Parallel representation under SSD" with Proposition 4).
+
+    Forward, per chunk [t0, t1) with m = cum_{t0-1} (0 before the call):
+        Y_t = e^{cum_t - m} C~_t^T g + sum_{s in chunk, s<=t} L[t,s] (C~_t . B~_s) X_s + D X_t
+        g  <- e^{cum_{t1-1} - m} g + sum_{s in chunk} e^{cum_{t1-1} - cum_s} w_s B~_s X_s^T
+    where w_s = gamma_s + (1 - lam_{s+1}) dt_{s+1} carries the next token's trapezoid share
+    (w_{T-1} = gamma_{T-1}), the starting g = h0 + (1 - lam_0) dt_0 B_prev x_prev^T, and
+    h_T = R(psi_{T-1}) g.  The backward keeps the adjoint of g between chunks (in reverse),
+    takes the intra-chunk terms as in bruteforce_bwd, and routes every exponential, weight and
+    angle to dt, A, lam and theta.  Returns all gradients, the starting state's included.
+    """
+    b, T, H, R, P, G, N, hpg = _heads(x, B)
+    NH = N // 2
+    out = dict(dx=np.zeros(x.shape), dB=np.zeros(B.shape), dC=np.zeros(C.shape),
+               ddt=np.zeros(dt.shape), dA=np.zeros(A.shape), dlam=np.zeros(lam.shape),
+               dtheta=np.zeros(theta.shape), dD=None if D is None else np.zeros(D.shape),
+               dh0=np.zeros((b, H, N, P)), dx_prev=np.zeros((b, H, R, P)),
+               dB_prev=np.zeros((b, G, R, N)))
+    for bi in range(b):
+        for h in range(H):
+            g = h // hpg
+            d, a, l = dt[bi, :, h], A[bi, :, h], lam[bi, :, h]
+            th = theta[bi, :, g]
+            X, Gy = x[bi, :, h], dy[bi, :, h]
+            Dh = 0.0 if D is None else D[h]
+            cum = np.cumsum(d * a)
+            ang = th if theta_is_angle else d[:, None] * th
+            psi = np.cumsum(ang, axis=0)
+            bt = np.stack([_rot_pairs(B[bi, t, g], -psi[t]) for t in range(T)])   # [T,R,N]
+            ct = np.stack([_rot_pairs(C[bi, t, g], -psi[t]) for t in range(T)])
+            w = l * d
+            w[:-1] = w[:-1] + (1.0 - l[1:]) * d[1:]
+            xp0 = np.zeros((R, P)) if x_prev is None else x_prev[bi, h]
+            bp0 = np.zeros((R, N)) if B_prev is None else B_prev[bi, g]
+            g0 = (np.zeros((N, P)) if h0 is None else h0[bi, h].copy())
+            g0 = g0 + (1.0 - l[0]) * d[0] * np.einsum("rn,rp->np", bp0, xp0)
+            bounds = list(range(0, T, chunk)) + [T]
+            chunks = list(zip(bounds[:-1], bounds[1:]))
+            # forward: the state entering every chunk
+            gin, gs = [], g0
+            for t0, t1 in chunks:
+                gin.append(gs)
+                m = cum[t0 - 1] if t0 > 0 else 0.0
+                V = np.einsum("s,srn,srp->np", np.exp(cum[t1 - 1] - cum[t0:t1]) * w[t0:t1],
+                              bt[t0:t1], X[t0:t1])
+                gs = np.exp(cum[t1 - 1] - m) * gs + V
+            gT = gs
+            hT = _rot_pairs(gT.T, psi[T - 1]).T                              # [N,P]
+            # reverse
+            dX, dbt, dct = Dh * Gy, np.zeros(bt.shape), np.zeros(ct.shape)
+            dcum, dw, dpsi = np.zeros(T), np.zeros(T), np.zeros((T, NH))
+            dga_i, dnx_i = np.zeros(T), np.zeros(T)        # intra-chunk band weights
+            if dhT is not None:
+                dH = dhT[bi, h]
+                dg = _rot_pairs(dH.T, -psi[T - 1]).T
+                dpsi[T - 1] += (dH[1::2] * hT[0::2] - dH[0::2] * hT[1::2]).sum(axis=1)
+            else:
+                dg = np.zeros((N, P))
+            for (t0, t1), gi in zip(chunks[::-1], gin[::-1]):
+                m = cum[t0 - 1] if t0 > 0 else 0.0
+                # state update
+                Eend = np.exp(cum[t1 - 1] - m)
+                dgin = Eend * dg
+                q = Eend * float((dg * gi).sum())
+                dcum[t1 - 1] += q
+                if t0 > 0:
+                    dcum[t0 - 1] -= q
+                for s in range(t0, t1):
+                    es = np.exp(cum[t1 - 1] - cum[s])
+                    Vs = np.einsum("rn,rp->np", bt[s], X[s])
+                    dv = float((dg * Vs).sum())
+                    dw[s] += es * dv
+                    dcum[t1 - 1] += es * w[s] * dv
+                    dcum[s] -= es * w[s] * dv
+                    dbt[s] += es * w[s] * np.einsum("np,rp->rn", dg, X[s])
+                    dX[s] += es * w[s] * np.einsum("rn,np->rp", bt[s], dg)
+                # inter-chunk output: e^{cum_t - m} C~_t^T g_in
+                for t in range(t0, t1):
+                    f = np.exp(cum[t] - m)
+                    Z = np.einsum("rn,np->rp", ct[t], gi)
+                    dct[t] += f * np.einsum("np,rp->rn", gi, Gy[t])
+                    dgin += f * np.einsum("rn,rp->np", ct[t], Gy[t])
+                    q = f * float((Gy[t] * Z).sum())
+                    dcum[t] += q
+                    if t0 > 0:
+                        dcum[t0 - 1] -= q
+                # intra-chunk: L[t,s] = e^{cum_t - cum_s}(gamma_s + [s<t](1 - lam_{s+1}) dt_{s+1})
+                n = t1 - t0
+                tri = np.tril(np.ones((n, n)))
+                strict = np.tril(np.ones((n, n)), -1)
+                cc = cum[t0:t1]
+                E = np.exp(np.where(tri > 0, cc[:, None] - cc[None, :], 0.0)) * tri
+                nx = np.zeros(n)
+                nx[:-1] = (1.0 - l[t0 + 1:t1]) * d[t0 + 1:t1]
+                om = (l[t0:t1] * d[t0:t1])[None, :] * tri + nx[None, :] * strict
+                L = E * om
+                S = np.einsum("trn,usn->trus", ct[t0:t1], bt[t0:t1])
+                GX = np.einsum("trp,usp->trus", Gy[t0:t1], X[t0:t1])
+                dX[t0:t1] += np.einsum("trus,trp->usp", S * L[:, None, :, None], Gy[t0:t1])
+                dS = GX * L[:, None, :, None]
+                dL = np.einsum("trus,trus->tu", S, GX)
+                dct[t0:t1] += np.einsum("trus,usn->trn", dS, bt[t0:t1])
+                dbt[t0:t1] += np.einsum("trus,trn->usn", dS, ct[t0:t1])
+                dE, dom = dL * om, dL * E
+                dcum[t0:t1] += (dE * E).sum(axis=1) - (dE * E).sum(axis=0)
+                dga_i[t0:t1] += (dom * tri).sum(axis=0)
+                dnx_i[t0:t1] += (dom * strict).sum(axis=0)
+                dg = dgin
+            # the starting state g0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T
+            out["dh0"][bi, h] = dg
+            k0 = (1.0 - l[0]) * d[0]
+            v0 = float((dg * np.einsum("rn,rp->np", bp0, xp0)).sum())
+            out["dx_prev"][bi, h] = k0 * np.einsum("rn,np->rp", bp0, dg)
+            out["dB_prev"][bi, g] += k0 * np.einsum("np,rp->rn", dg, xp0)
+            # rotation back, angles
+            out["dC"][bi, :, g] += np.stack([_rot_pairs(dct[t], psi[t]) for t in range(T)])
+            out["dB"][bi, :, g] += np.stack([_rot_pairs(dbt[t], psi[t]) for t in range(T)])
+            dpsi += ((dct[..., 0::2] * ct[..., 1::2] - dct[..., 1::2] * ct[..., 0::2]).sum(axis=1) +
+                     (dbt[..., 0::2] * bt[..., 1::2] - dbt[..., 1::2] * bt[..., 0::2]).sum(axis=1))
+            dang = np.cumsum(dpsi[::-1], axis=0)[::-1]
+            # coefficients: w (state), the intra band weights, gamma, cum
+            ddt_, dlam_ = np.zeros(T), np.zeros(T)
+            dga = dw + dga_i
+            dnx = dnx_i.copy()
+            dnx[:-1] += dw[:-1]
+            ddt_ += dga * l
+            dlam_ += dga * d
+            ddt_[1:] += dnx[:-1] * (1.0 - l[1:])
+            dlam_[1:] -= dnx[:-1] * d[1:]
+            ddt_[0] += (1.0 - l[0]) * v0
+            dlam_[0] -= d[0] * v0
+            dda = np.cumsum(dcum[::-1])[::-1]
+            ddt_ += dda * a
+            if theta_is_angle:
+                out["dtheta"][bi, :, g] += dang
+            else:
+                out["dtheta"][bi, :, g] += dang * d[:, None]
+                ddt_ += (dang * th).sum(axis=1)
+            out["dx"][bi, :, h] = dX
+            out["ddt"][bi, :, h] = ddt_
+            out["dA"][bi, :, h] = dda * d
+            out["dlam"][bi, :, h] = dlam_
+            if D is not None:
+                out["dD"][h] += float((Gy * X).sum())
+    return out
+
+
 def implicit_conv_route(x, B, C, dt, A, lam, D=None, h0=None, x_prev=None, B_prev=None):
     """Remark 4 (theta = 0): width-2 data-dependent convolution on v_t = B_t x_t^T,
 

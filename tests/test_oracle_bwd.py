@@ -7,9 +7,10 @@ weights, dL/dv for every element v of every input (x, B, C, dt, A, lam, theta, D
 initial state h0, x_prev, B_prev) must match (L(v + e) - L(v - e)) / 2e to the central
 difference's error (O(e^2) truncation plus rounding), at shapes where each finite difference
 is cheap.  Groups shared by two heads (G = 1, H = 2) check the head sums of the B, C and theta
-gradients; the pre-scaled angle flag checks the theta path without dt.  A second, independent
-derivation (the hand-derived gradients of the materialised T x T form, tests/routes.py) must
-agree with the oracle's reverse pass through the recurrence for a fresh sequence.  Planted
+gradients; the pre-scaled angle flag checks the theta path without dt.  Two more, independent
+derivations (tests/routes.py) must agree with the oracle's reverse pass through the
+recurrence: the hand-derived gradients of the materialised T x T form (fresh sequence), and
+the chunked backward with an adjoint state between chunks (any starting state).  Planted
 mistakes in a copy of the backward's C source are caught.
 """
 import math
@@ -100,6 +101,22 @@ def test_gradients_match_materialised_form_derivative(angle, R, G):
     r = routes.bruteforce_bwd(*args, Wy, D=v["D"], theta_is_angle=angle)
     for k in ("dx", "dB", "dC", "ddt", "dA", "dlam", "dtheta", "dD"):
         assert np.max(np.abs(g[k] - r[k])) <= 1e-11 * max(1.0, np.max(np.abs(r[k]))), k
+
+
+@pytest.mark.parametrize("angle,R,G,chunk,T", [(False, 2, 1, 4, 13), (True, 1, 2, 5, 12),
+                                                (False, 3, 2, 3, 10), (False, 1, 1, 16, 9)])
+def test_gradients_match_chunked_form_derivative(angle, R, G, chunk, T):
+    """The chunked backward (adjoint state between chunks in the call's rotated frame,
+    materialised-form derivative inside each chunk; tests/routes.py) equals the oracle's
+    reverse pass with a starting state, dL/dh_T and ragged chunks."""
+    v, Wy, Wh = _problem(31 + R, b=2, T=T, H=4, G=G, P=3, N=6, R=R)
+    args = [v[k] for k in ("x", "B", "C", "dt", "A", "lam", "theta")]
+    st = dict(D=v["D"], h0=v["h0"], x_prev=v["x_prev"], B_prev=v["B_prev"], dhT=Wh,
+              theta_is_angle=angle)
+    g = oracle.scan_bwd(*args, Wy, **st)
+    r = routes.chunked_bwd(*args, Wy, chunk, **st)
+    for k in GRAD.values():
+        assert np.max(np.abs(g[k] - r[k])) <= 1e-12 * max(1.0, np.max(np.abs(r[k]))), k
 
 
 def test_zero_loss_weights_give_zero_gradients():
