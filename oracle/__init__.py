@@ -209,6 +209,101 @@ def scan_bwd(x, B, C, dt, A, lam, theta, dy, D=None, h0=None, x_prev=None, B_pre
     return out
 
 
+def _bc_map(v, bias, eps):
+    """BC map of the columns v [..., N] (the same map m3o_bc_map applies): scale to unit RMS
+    when eps > 0, then add the bias (None: 0).  Returns (map(v), scale [..., 1])."""
+    if eps > 0.0:
+        s = 1.0 / np.sqrt((v * v).mean(axis=-1, keepdims=True) + eps)
+    else:
+        s = np.ones(v.shape[:-1] + (1,))
+    return v * s + (0.0 if bias is None else bias), s
+
+
+def _bc_map_bwd(v, s, du, eps):
+    """dL/dv of u = v s(v) + bias given du: s du - (s^3 / N) v <du, v> (RMS scale), or du."""
+    if eps <= 0.0:
+        return du
+    return s * du - (s ** 3 / v.shape[-1]) * v * (du * v).sum(axis=-1, keepdims=True)
+
+
+def scan_bwd_ex(x, B, C, dt, A, lam, theta, dy, D=None, h0=None, x_prev=None, B_prev=None,
+                dhT=None, theta_is_angle=False, z=None, B_bias=None, C_bias=None,
+                bc_eps: float = 0.0, x_expand=None, z_expand=None, nthreads: int = 0):
+    """Reverse-mode gradients of ``scan`` with the fused extras (output gate, BC map, MIMO
+    lightweight expansion), for dL/dy = dy [b,T,H,R,P] and dL/dh_T = dhT.
+
+    Built on ``scan_bwd``: the extras' effective inputs are formed per head (X = x * x_expand,
+    Z = z * z_expand; B, C, B_prev through the BC map with the head's bias; theta per head),
+    the recurrence's backward runs with one group per head, and the chain goes back through
+    the gate (SiLU'(Z) = sig(Z) (1 + Z (1 - sig(Z)))), the RMS scale's Jacobian and the
+    expansion weights, summing over the heads of each group.  Layouts as in ``scan``.
+    Returns the dict of ``scan_bwd`` plus dz, dB_bias, dC_bias, dx_expand, dz_expand (None
+    where the part is off).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    X = expand(x, x_expand) if x_expand is not None else x
+    b, T, H, R, P = X.shape
+    B = np.asarray(B, dtype=np.float64)
+    C = np.asarray(C, dtype=np.float64)
+    G, N = B.shape[2], B.shape[4]
+    gidx = np.arange(H) // (H // G)
+    Bh, Ch = B[:, :, gidx], C[:, :, gidx]                       # [b,T,H,R,N]
+    Bp = np.zeros((b, G, R, N)) if B_prev is None else np.asarray(B_prev, dtype=np.float64)
+    Bph = Bp[:, gidx]                                           # [b,H,R,N]
+    bb = None if B_bias is None else np.asarray(B_bias, dtype=np.float64)
+    cb = None if C_bias is None else np.asarray(C_bias, dtype=np.float64)
+    Be, sB = _bc_map(Bh, None if bb is None else bb[None, None, :, None, :], bc_eps)
+    Ce, sC = _bc_map(Ch, None if cb is None else cb[None, None, :, None, :], bc_eps)
+    Bpe, sP = _bc_map(Bph, None if bb is None else bb[None, :, None, :], bc_eps)
+    th = np.asarray(theta, dtype=np.float64)[:, :, gidx]
+    Z = None
+    dy = np.asarray(dy, dtype=np.float64)
+    dy_pre, dZ = dy, None
+    if z is not None:
+        z = np.asarray(z, dtype=np.float64)
+        Z = expand(z, z_expand) if z_expand is not None else z
+        y_pre = scan(X, Be, Ce, dt, A, lam, th, D=D, h0=h0, x_prev=x_prev, B_prev=Bpe,
+                     theta_is_angle=theta_is_angle, nthreads=nthreads)[0]
+        sig = 1.0 / (1.0 + np.exp(-Z))
+        dy_pre = dy * Z * sig
+        dZ = dy * y_pre * sig * (1.0 + Z * (1.0 - sig))
+    g = scan_bwd(X, Be, Ce, dt, A, lam, th, dy_pre, D=D, h0=h0, x_prev=x_prev, B_prev=Bpe,
+                 dhT=dhT, theta_is_angle=theta_is_angle, nthreads=nthreads)
+    out = dict(g)
+
+    def to_groups(v, axis):
+        acc = np.zeros(v.shape[:axis] + (G,) + v.shape[axis + 1:])
+        for hh in range(H):
+            idx = [slice(None)] * v.ndim
+            idx[axis] = hh
+            oidx = list(idx)
+            oidx[axis] = gidx[hh]
+            acc[tuple(oidx)] += v[tuple(idx)]
+        return acc
+
+    out["dB"] = to_groups(_bc_map_bwd(Bh, sB, g["dB"], bc_eps), 2)
+    out["dC"] = to_groups(_bc_map_bwd(Ch, sC, g["dC"], bc_eps), 2)
+    out["dB_prev"] = to_groups(_bc_map_bwd(Bph, sP, g["dB_prev"], bc_eps), 1)
+    out["dtheta"] = to_groups(g["dtheta"], 2)
+    out["dB_bias"] = None if bb is None else g["dB"].sum(axis=(0, 1, 3)) + g["dB_prev"].sum(axis=(0, 2))
+    out["dC_bias"] = None if cb is None else g["dC"].sum(axis=(0, 1, 3))
+    if x_expand is not None:
+        w = np.asarray(x_expand, dtype=np.float64)
+        out["dx"] = (g["dx"] * w).sum(axis=-2)
+        out["dx_expand"] = (g["dx"] * x[..., None, :]).sum(axis=(0, 1))
+    else:
+        out["dx_expand"] = None
+    out["dz"], out["dz_expand"] = None, None
+    if z is not None:
+        if z_expand is not None:
+            wz = np.asarray(z_expand, dtype=np.float64)
+            out["dz"] = (dZ * wz).sum(axis=-2)
+            out["dz_expand"] = (dZ * z[..., None, :]).sum(axis=(0, 1))
+        else:
+            out["dz"] = dZ
+    return out
+
+
 def decode_step(x, B, C, dt, A, lam, theta, D, h, x_prev, B_prev,
                 theta_is_angle: bool = False, nthreads: int = 0, z=None, B_bias=None,
                 C_bias=None, bc_eps: float = 0.0, x_expand=None, z_expand=None):
