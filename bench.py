@@ -3,7 +3,7 @@
 One step = one m3_scan_fwd call over the SISO 1.5B-scale prefill workload
 (batch 8, 64 heads, T 4096, P 64, N 128, chunk 64, bf16 x/B/C, fp32 dt/A/lam/theta/state),
 i.e. every prefill step of the method.  Alongside, as sub-metrics: the batch-256 decode
-workloads (SISO N 128 and MIMO R 4 N 64; 1024 sequential tokens, the 32-token pool captured
+workloads (SISO N 128 and MIMO R 4 N 64; 1000 sequential steps with fresh tokens, captured
 once as a CUDA graph and replayed), the same prefill and decode with the fused output gate
 ("gated") and with BCNorm + BC biases ("bc"), the MIMO rank-4 prefill plain and with the
 lightweight expansion of x and z ("mimo"), the backward pass of the prefill workload
@@ -41,8 +41,7 @@ from state_space_model_06_b200 import inputs, m3  # noqa: E402
 METRIC = ("prefill tokens/s/layer (% tensor peak); decode tok/s at batch 256 (% HBM BW)")
 WORKLOAD = "siso_prefill_1p5b"
 DECODES = ("decode_siso_b256", "decode_mimo_b256")
-DECODE_TOKENS = 1000
-DECODE_POOL = 32            # distinct pre-generated tokens, cycled over the 1000 steps
+DECODE_TOKENS = 1000        # sequential decode steps, each with a fresh pre-generated token
 BC_EPS = 1e-6              # BCNorm epsilon of the BC legs
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -287,30 +286,35 @@ def time_prefill_e2e(w, d, inp, st, ws, steps, stream, dev):
 
 
 def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False, bc=False):
+    """`tokens` sequential decode steps of the workload, each with its own fresh token
+    (drawn up front on the device by the seeded generator of ``inputs``).  The whole
+    sequence is captured once as one CUDA graph and replayed: a step is ~0.2 ms of device
+    time, about what a host launch through ctypes costs, so steps launched one by one would
+    time the host.  The state is reset to the drawn starting state before each replay."""
     w = inputs.WORKLOADS[name]
-    inp = inputs.make_decode_inputs(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
-                                    tokens=DECODE_POOL, io_dtype=w.io_dtype,
-                                    theta_max=w.theta_max, seed=seed)
+    g = inputs.make_decode_inputs(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
+                                  tokens=tokens, io_dtype=w.io_dtype, theta_max=w.theta_max,
+                                  seed=seed, device=dev)
     d = m3.Dims(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
                 m3.io_dtype_of(w.io_dtype))
-    g = {k: v.to(dev) for k, v in inp.items()}
     st = m3.State(d, dev)
     y = torch.empty_like(g["x"][0])
     keys = ("x", "B", "C", "dt", "A", "lam", "theta")
-    tok = [[g[k][i] for k in keys] for i in range(DECODE_POOL)]
-    z = inputs.make_gate(g["x"].shape, io_dtype=w.io_dtype, seed=seed).to(dev) if gated else None
+    z = None
+    if gated:
+        z = inputs.make_gate(g["x"].shape, io_dtype=w.io_dtype, seed=seed, device=dev)
     bias = [v.to(dev) for v in inputs.make_bc_bias(w.nheads, w.dstate, seed=seed)] if bc else None
 
     def step(t):   # on the current stream: the capture stream while the graph is recorded
+        tok = [g[k][t] for k in keys]
         if bc:
-            ex = m3.Extras(z=None if z is None else z[t % DECODE_POOL], B_bias=bias[0],
-                           C_bias=bias[1], bc_norm_eps=BC_EPS)
-            m3.m3_decode_step_ex(d, *tok[t % DECODE_POOL], g["D"], ex, st, y, stream=None)
+            ex = m3.Extras(z=None if z is None else z[t], B_bias=bias[0], C_bias=bias[1],
+                           bc_norm_eps=BC_EPS)
+            m3.m3_decode_step_ex(d, *tok, g["D"], ex, st, y, stream=None)
         elif gated:
-            m3.m3_decode_step_gated(d, *tok[t % DECODE_POOL], g["D"], z[t % DECODE_POOL], st, y,
-                                    stream=None)
+            m3.m3_decode_step_gated(d, *tok, g["D"], z[t], st, y, stream=None)
         else:
-            m3.m3_decode_step(d, *tok[t % DECODE_POOL], g["D"], st, y, stream=None)
+            m3.m3_decode_step(d, *tok, g["D"], st, y, stream=None)
 
     def reset():
         st.h.copy_(g["h0"])
@@ -321,15 +325,10 @@ def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False, bc=F
     for t in range(10):
         step(t)
     torch.cuda.synchronize()
-    # The DECODE_POOL sequential steps are captured once as a CUDA graph and the graph is
-    # replayed: a step takes ~0.2 ms of device time, about what a host launch through
-    # ctypes takes, so launching steps one by one would time the host.  The state carries
-    # over from replay to replay exactly as in a plain loop over the cycled tokens.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        for t in range(DECODE_POOL):
+        for t in range(tokens):
             step(t)
-    reps = max(1, -(-tokens // DECODE_POOL))
     reset()
     graph.replay()                      # warm-up replay
     reset()
@@ -337,23 +336,22 @@ def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False, bc=F
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     cur = torch.cuda.current_stream()
     e0.record(cur)
-    for _ in range(reps):
-        graph.replay()
+    graph.replay()
     e1.record(cur)
     torch.cuda.synchronize()
-    tokens = reps * DECODE_POOL
     ms = e0.elapsed_time(e1) / tokens
     del graph
     if torch.equal(st.h, g["h0"]):
-        raise RuntimeError("decode graph replays left the state unchanged")
+        raise RuntimeError("decode graph replay left the state unchanged")
     finite = bool(torch.isfinite(st.h).all().item())
     byts = decode_algorithmic(w) + (w.batch * w.nheads * w.rank * w.headdim * 2 if gated else 0)
+    del g, z
     return {"tokens_per_s": w.batch / (ms / 1e3), "us_per_step": ms * 1e3,
             "achieved_gbs": byts / (ms / 1e3) / 1e9, "alg_bytes_per_step": byts,
             "state_finite": finite,
             "config": {"batch": w.batch, "heads": w.nheads, "headdim": w.headdim,
                        "dstate": w.dstate, "rank": w.rank, "tokens": tokens,
-                       "distinct_tokens": DECODE_POOL}}
+                       "distinct_tokens": tokens}}
 
 
 def mimo_leg(args, dev, stream, rank, ws_world, pk):

@@ -40,6 +40,7 @@
  *     never traps; a bounded device-side wait that gives up writes
  *     M3_ERR_TIMEOUT into the workspace status word (see m3_query_status).
  *   - Value ranges are the caller's contract: dt > 0, A <= 0, lam in [0, 1].
+ *     M3_FLAG_DEBUG_CHECKS adds a non-trapping device scan of them.
  */
 #ifndef M3_H
 #define M3_H
@@ -61,7 +62,9 @@ typedef enum {
     M3_ERR_WORKSPACE = 6,   /* workspace missing or smaller than m3_scan_workspace_bytes */
     M3_ERR_LAUNCH = 7,      /* a kernel launch failed (cudaGetLastError) */
     M3_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up (reported by m3_query_status) */
-    M3_ERR_CUDA = 9         /* another CUDA runtime call failed */
+    M3_ERR_CUDA = 9,        /* another CUDA runtime call failed */
+    M3_ERR_RANGE = 10       /* M3_FLAG_DEBUG_CHECKS found an input outside its range
+                               (reported by m3_query_status) */
 } m3_status;
 
 typedef enum { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
@@ -93,6 +96,15 @@ typedef struct {
  * up, the kernel aborts cleanly (outputs are invalid), and m3_query_status reports
  * M3_ERR_TIMEOUT; the CUDA context stays usable. */
 #define M3_FLAG_TEST_STALL 4u
+/* Debug scan of the caller's value ranges (m3_scan_fwd and its variants, m3_scan_bwd): one
+ * extra kernel reads every input of the call once before the call runs and checks
+ * dt > 0, A <= 0, lam in [0, 1] ("Technical Approach", Proposition 1: dt after softplus,
+ * alpha = exp(dt A) <= 1, lam after sigmoid) and that every other value (x, B, C, theta,
+ * D, z, the state) is finite.  It never traps and changes nothing: a violation sets a bit
+ * in the workspace status word, which m3_query_status reports as M3_ERR_RANGE (a timeout
+ * takes precedence).  The call itself still runs, on whatever it was given.  The decode
+ * step has no workspace to report into: it rejects this flag with M3_ERR_UNSUPPORTED. */
+#define M3_FLAG_DEBUG_CHECKS 8u
 
 /* Bytes of each state buffer for `dims`.  Any out-pointer may be NULL. */
 m3_status m3_state_bytes(const m3_dims* dims, size_t* h_bytes, size_t* x_prev_bytes,
@@ -214,19 +226,24 @@ m3_status m3_scan_fwd_gated(const m3_dims* dims, int32_t seqlen, int32_t chunk, 
  * deployment convenience of this library.
  *
  * Same arguments, layouts, results and errors as m3_scan_fwd, minus the workspace.
- * The workspace is lent from one fixed scratch array compiled into the library
- * (64 KiB, 256-byte aligned, held on every GPU that loads the library until the
- * process exits); shapes whose m3_scan_workspace_bytes exceeds 64 KiB are rejected
- * with M3_ERR_WORKSPACE.  Nothing is allocated: no cudaMalloc / cudaFree and no
- * allocating library routine.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any stream
- *     capture.
- *   - Every call shares the one array, and each call clears the part that must
- *     start at zero.  Calls that can overlap on the GPU (different streams without
- *     ordering) race on it: order them.
- *   - The device-side status word lives in the shared array and is not reported;
- *     callers that need m3_query_status use m3_scan_fwd with their own workspace.
+ * Every host-side check of m3_scan_fwd runs first, before any CUDA call.  The workspace
+ * is lent from one fixed scratch array compiled into the library (64 KiB, 256-byte
+ * aligned, held on every GPU that loads the library until the process exits); shapes
+ * whose m3_scan_workspace_bytes exceeds 64 KiB are rejected with M3_ERR_WORKSPACE.
+ * Nothing is allocated: no cudaMalloc / cudaFree and no allocating library routine.
+ *   - `stream` must belong to the current device (the array's address is per device);
+ *     a stream of another device is rejected with M3_ERR_UNSUPPORTED.
+ *   - Each call looks up the array's device address on the current device.  The first
+ *     call on a device loads it there: make that first call before any stream capture.
+ *     The lookup is not cached, so a device reset between calls does no harm.
+ *   - Every call shares the one array, and each call clears the part that must start at
+ *     zero.  Calls that can overlap on the GPU (different streams without ordering) race
+ *     on it: order them.
+ *   - The device-side status word lives in the shared array and is not reported.  A call
+ *     whose bounded device-side wait gave up (see m3_query_status) leaves y and the state
+ *     undefined without saying so; callers that need to know use m3_scan_fwd with their
+ *     own workspace and m3_query_status.  For the same reason M3_FLAG_DEBUG_CHECKS is
+ *     rejected here with M3_ERR_UNSUPPORTED.
  */
 m3_status m3_scan_fwd_noalloc(const m3_dims* dims, int32_t seqlen, int32_t chunk, const void* x,
                               const void* B, const void* C, const float* dt, const float* A,
@@ -319,8 +336,9 @@ m3_status m3_scan_bwd(const m3_dims* dims, int32_t seqlen, const void* x, const 
                       const void* dy, const float* dhT, const m3_grads* grads, void* workspace,
                       size_t workspace_bytes, uint32_t flags, void* stream);
 
-/* Synchronise `stream` and report the device-side status word in `workspace`
- * (M3_OK, or M3_ERR_TIMEOUT when a bounded wait gave up). */
+/* Synchronise `stream` and report the device-side status word in `workspace`:
+ * M3_OK, M3_ERR_TIMEOUT when a bounded wait gave up, or M3_ERR_RANGE when the debug
+ * scan of M3_FLAG_DEBUG_CHECKS found an input outside its range. */
 m3_status m3_query_status(const void* workspace, void* stream);
 
 /* Static English text for a status code. */

@@ -105,6 +105,7 @@ const char* m3_status_string(m3_status s) {
         case M3_ERR_LAUNCH: return "kernel launch failed";
         case M3_ERR_TIMEOUT: return "a bounded device-side wait timed out";
         case M3_ERR_CUDA: return "CUDA runtime call failed";
+        case M3_ERR_RANGE: return "an input value is outside its documented range (debug checks)";
     }
     return "unknown status";
 }
@@ -177,20 +178,22 @@ m3_status m3_scan_workspace_bytes(const m3_dims* d, int32_t seqlen, int32_t chun
 
 }  // extern "C"
 
-namespace {
+namespace m3 {
 
-// Prefill with an optional output gate z (null: none); validation happens before any launch.
-m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
-                    const void* B, const void* C, const float* dt, const float* A,
-                    const float* lam, const float* theta, const float* D, const m3_extras* ex,
-                    m3_state* state, void* y, void* workspace, size_t workspace_bytes,
-                    uint32_t flags, void* stream) {
+m3_status scan_validate(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
+                        const void* B, const void* C, const float* dt, const float* A,
+                        const float* lam, const float* theta, const float* D,
+                        const m3_extras* ex, const m3_state* state, const void* y,
+                        uint32_t flags, size_t* need) {
     const void* z = ex ? ex->z : nullptr;
     m3_status st = check_dims(d);
     if (st != M3_OK) return st;
     if (seqlen < 0) return M3_ERR_SHAPE;
     if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return M3_ERR_SHAPE;
     if ((st = check_state(state)) != M3_OK) return st;
+    size_t base = 0;
+    m3_scan_workspace_bytes(d, seqlen, chunk, &base);
+    *need = base + bc_bytes(d, seqlen, ex);
     if (seqlen == 0) return M3_OK;   // no tokens: nothing is read, written or launched
     if (!x || !B || !C || !dt || !A || !lam || !theta || !y) return M3_ERR_NULL;
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
@@ -202,10 +205,36 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
         return M3_ERR_ALIGN;
     if (ex && !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;   // negative or NaN epsilon
     if (ex && ex->z_expand && !z) return M3_ERR_NULL;           // an expanded gate needs z
+    const int N = d->dstate, P = d->headdim, R = d->rank;
+    const int qt = scan_tc_chunk(N, P, R, chunk, d->nheads);
+    const bool use_tc = !(flags & M3_FLAG_FORCE_SIMT) && d->io_dtype == M3_BF16 && qt &&
+                        aligned(dt, 16) && aligned(A, 16) && aligned(lam, 16) &&
+                        aligned(theta, 16);
+    int ppt = 0, ns = 0;
+    if (!use_tc && (!rank_has_kernel(R) || !simt_shape(N, P, &ppt, &ns)))
+        return M3_ERR_UNSUPPORTED;
+    return M3_OK;
+}
+
+}  // namespace m3
+
+namespace {
+
+// Prefill with the optional fused parts of `ex` (null: none); every check happens before
+// any launch.
+m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
+                    const void* B, const void* C, const float* dt, const float* A,
+                    const float* lam, const float* theta, const float* D, const m3_extras* ex,
+                    m3_state* state, void* y, void* workspace, size_t workspace_bytes,
+                    uint32_t flags, void* stream) {
+    const void* z = ex ? ex->z : nullptr;
+    size_t need = 0;
+    m3_status st = scan_validate(d, seqlen, chunk, x, B, C, dt, A, lam, theta, D, ex, state, y,
+                                 flags, &need);
+    if (st != M3_OK || seqlen == 0) return st;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return M3_ERR_WORKSPACE;
     size_t base = 0;
     m3_scan_workspace_bytes(d, seqlen, chunk, &base);
-    const size_t need = base + bc_bytes(d, seqlen, ex);
-    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return M3_ERR_WORKSPACE;
 
     const int N = d->dstate, P = d->headdim, R = d->rank;
     // the tensor-core kernel reads dt / A / lam / theta with TMA (16-byte aligned rows)
@@ -214,8 +243,7 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
                         aligned(dt, 16) && aligned(A, 16) && aligned(lam, 16) &&
                         aligned(theta, 16);
     int ppt = 0, ns = 0;
-    if (!use_tc && (!rank_has_kernel(R) || !simt_shape(N, P, &ppt, &ns)))
-        return M3_ERR_UNSUPPORTED;
+    if (!use_tc) simt_shape(N, P, &ppt, &ns);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     ScanArgs a;
@@ -236,6 +264,24 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
 
     if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return M3_ERR_CUDA;
     cudaError_t e = cudaSuccess;
+    if (flags & M3_FLAG_DEBUG_CHECKS) {
+        const size_t b = d->batch, T = seqlen, H = d->nheads, G = d->ngroups;
+        const size_t xw = (ex && ex->x_expand) ? 1 : R, zw = (ex && ex->z_expand) ? 1 : R;
+        RangeCheckArgs rc;
+        std::memset(&rc, 0, sizeof(rc));
+        rc.x = x; rc.n_x = b * T * H * xw * P;
+        rc.B = B; rc.C = C; rc.n_BC = b * T * G * R * N;
+        rc.z = z; rc.n_z = z ? b * T * H * zw * P : 0;
+        rc.x_prev = state->x_prev; rc.n_xp = b * H * R * P;
+        rc.B_prev = state->B_prev; rc.n_bp = b * G * R * N;
+        rc.dt = dt; rc.A = A; rc.lam = lam; rc.n_coef = b * T * H;
+        rc.theta = theta; rc.n_theta = b * T * G * (N / 2);
+        rc.D = D; rc.n_D = D ? H : 0;
+        rc.h = state->h; rc.n_h = b * H * N * P;
+        rc.status = a.status;
+        e = launch_range_checks(rc, d->io_dtype, s);
+        if (e != cudaSuccess) return launch_status(e);
+    }
     if (a.bc_scale)
         e = launch_bc_scales(a, R, d->io_dtype, ex->bc_norm_eps,
                              reinterpret_cast<float*>(static_cast<char*>(workspace) + base), s);
@@ -266,6 +312,7 @@ m3_status decode_impl(const m3_dims* d, const void* x, const void* B, const void
         return M3_ERR_ALIGN;
     if (ex && !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;
     if (ex && ex->z_expand && !z) return M3_ERR_NULL;
+    if (flags & M3_FLAG_DEBUG_CHECKS) return M3_ERR_UNSUPPORTED;   // no status word to report into
     int ppt = 0;
     if (!rank_has_kernel(d->rank) || !decode_shape(d->dstate, d->headdim, d->rank, &ppt))
         return M3_ERR_UNSUPPORTED;
@@ -403,6 +450,23 @@ m3_status m3_scan_bwd(const m3_dims* d, int32_t seqlen, const void* x, const voi
     a.T = seqlen; a.batch = d->batch; a.H = d->nheads; a.G = d->ngroups; a.P = P; a.N = N;
     a.flags = flags;
     if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return M3_ERR_CUDA;
+    if (flags & M3_FLAG_DEBUG_CHECKS) {
+        const size_t b = d->batch, T = seqlen, H = d->nheads, G = d->ngroups;
+        RangeCheckArgs rc;
+        std::memset(&rc, 0, sizeof(rc));
+        rc.x = x; rc.n_x = b * T * H * R * P;
+        rc.B = B; rc.C = C; rc.n_BC = b * T * G * R * N;
+        rc.z = dy; rc.n_z = b * T * H * R * P;   // dL/dy: finite
+        rc.x_prev = state0->x_prev; rc.n_xp = b * H * R * P;
+        rc.B_prev = state0->B_prev; rc.n_bp = b * G * R * N;
+        rc.dt = dt; rc.A = A; rc.lam = lam; rc.n_coef = b * T * H;
+        rc.theta = theta; rc.n_theta = b * T * G * (N / 2);
+        rc.D = D; rc.n_D = D ? H : 0;
+        rc.h = state0->h; rc.n_h = b * H * N * P;
+        rc.status = static_cast<uint32_t*>(workspace);
+        cudaError_t e = launch_range_checks(rc, d->io_dtype, s);
+        if (e != cudaSuccess) return launch_status(e);
+    }
     return launch_status(launch_scan_bwd(a, R, d->io_dtype, s));
 }
 
@@ -413,7 +477,10 @@ m3_status m3_query_status(const void* workspace, void* stream) {
     uint32_t word = 0;
     if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
         return M3_ERR_CUDA;
-    return word == 0 ? M3_OK : M3_ERR_TIMEOUT;
+    if (word == 0) return M3_OK;
+    if (word & M3_STATUS_TIMEOUT_BIT) return M3_ERR_TIMEOUT;
+    if (word & M3_STATUS_RANGE_BIT) return M3_ERR_RANGE;
+    return M3_ERR_TIMEOUT;
 }
 
 }  // extern "C"

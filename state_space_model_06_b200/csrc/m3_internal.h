@@ -7,6 +7,30 @@
 
 namespace m3 {
 
+// Bits of the workspace status word: a bounded device-side wait that gave up ORs in the
+// timeout code; the debug range scan ORs in the range bit.
+constexpr uint32_t M3_STATUS_TIMEOUT_BIT = (uint32_t)M3_ERR_TIMEOUT;
+constexpr uint32_t M3_STATUS_RANGE_BIT = 1u << 8;
+
+// The inputs the debug range scan of M3_FLAG_DEBUG_CHECKS reads (null: not checked) and
+// their element counts.
+struct RangeCheckArgs {
+    const void *x, *B, *C, *z, *x_prev, *B_prev;   // io dtype: finite
+    const float *dt, *A, *lam;                     // dt > 0, A <= 0, lam in [0, 1]
+    const float *theta, *D, *h;                    // finite
+    size_t n_x, n_BC, n_z, n_xp, n_bp, n_coef, n_theta, n_D, n_h;
+    uint32_t* status;
+};
+cudaError_t launch_range_checks(const RangeCheckArgs& a, int io_dtype, cudaStream_t s);
+
+// Every host-side check m3_scan_fwd_ex makes before it launches anything, except the
+// workspace checks; sets *need to the workspace bytes the call needs.
+m3_status scan_validate(const m3_dims* d, int32_t seqlen, int32_t chunk, const void* x,
+                        const void* B, const void* C, const float* dt, const float* A,
+                        const float* lam, const float* theta, const float* D,
+                        const m3_extras* ex, const m3_state* state, const void* y,
+                        uint32_t flags, size_t* need);
+
 // decode step: one CTA per (batch, head); template on io type and rank
 cudaError_t launch_decode(const DecodeArgs& a, int batch, int R, int io_dtype, cudaStream_t s);
 

@@ -43,25 +43,6 @@ namespace m3 {
 
 using namespace sm100;
 
-// Optional timeline instrumentation: with -DM3_TRACE the kernel records clock64() at
-// each pipeline hand-off of one CTA into a device array (read by m3_trace_copy).
-#ifdef M3_TRACE
-#define M3_TRACE_CHUNKS 64
-#define M3_TRACE_EVENTS 32
-__device__ unsigned long long g_m3_trace[M3_TRACE_CHUNKS][M3_TRACE_EVENTS];
-__device__ int g_m3_trace_cta = 0;
-__shared__ int s_m3_trace_on;   // copied from g_m3_trace_cta once per CTA
-#define M3_TRACE_EV(c, e)                                                           \
-    do {                                                                            \
-        if (s_m3_trace_on && (c) < M3_TRACE_CHUNKS) g_m3_trace[(c)][(e)] = clock64(); \
-    } while (0)
-#define M3_TRACE_INIT() \
-    do { if (threadIdx.x == 0) s_m3_trace_on = ((int)blockIdx.x == g_m3_trace_cta); } while (0)
-#else
-#define M3_TRACE_EV(c, e) do { } while (0)
-#define M3_TRACE_INIT() do { } while (0)
-#endif
-
 namespace {
 
 constexpr int kP = 64;               // head dimension handled by this kernel
@@ -280,7 +261,6 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
         const uint32_t s_ct = smem_u32(C::ct(sm, slot)), s_bt = smem_u32(C::bt(sm, slot));
         const uint32_t s_xw = smem_u32(C::xw(sm, slot));
         if (!mbar_wait(&bar[OPS_FULL0 + slot], (c / C::OPS) & 1, ab)) return;
-        M3_TRACE_EV(c, 6);
         tc_fence_after();
         // S = C~ B~^T   (M = L tokens*ranks, N = L, K = NST)
         if (!mbar_wait(&bar[S_EMPTY], ph ^ 1, ab)) return;
@@ -289,7 +269,6 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
         for (int k = 0; k < NST / 16; ++k)
             mma_bf16(tmem + C::TM_S, desc_k(s_ct, k, C::L), desc_k(s_bt, k, C::L), C::ID_S, k > 0);
         mma_commit(&bar[S_FULL]);
-        M3_TRACE_EV(c, 7);
         // dS = B~^T Xw  (M = NST, N = P, K = L)
         if (!mbar_wait(&bar[DS_EMPTY], ph ^ 1, ab)) return;
         tc_fence_after();
@@ -298,12 +277,9 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
             mma_bf16(tmem + C::TM_DS, desc_mn(s_bt, k, C::L * 128u), desc_mn(s_xw, k, 1024u),
                      C::ID_DS, k > 0);
         mma_commit(&bar[DS_FULL]);
-        M3_TRACE_EV(c, 8);
         // Y_inter = C~ g  (M = L, N = P, K = NST)
         if (!mbar_wait(&bar[G_FULL], ph, ab)) return;
-        M3_TRACE_EV(c, 9);
         if (!mbar_wait(&bar[Y_EMPTY0 + yb], ((c >> 1) & 1) ^ 1, ab)) return;
-        M3_TRACE_EV(c, 10);
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < NST / 16; ++k)
@@ -311,10 +287,8 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
                      k > 0);
         mma_commit(&bar[G_EMPTY]);
         mma_commit(&bar[OPS_EMPTY0 + slot]);
-        M3_TRACE_EV(c, 11);
         // Y_intra = (S o L) X  (M = L, N = P, K = L)
         if (!mbar_wait(&bar[SL_FULL], ph, ab)) return;
-        M3_TRACE_EV(c, 12);
         const int xs = c % C::XST;
         if (!mbar_wait(&bar[X_FULL0 + xs], (c / C::XST) & 1, ab)) return;
         tc_fence_after();
@@ -324,7 +298,6 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
             mma_bf16(tmem + C::tm_ya(yb), desc_k(s_sl, k, C::L), desc_mn(s_x, k, 1024u), C::ID_Y,
                      k > 0);
         mma_commit(&bar[Y_FULL0 + yb]);
-        M3_TRACE_EV(c, 13);
     }
 }
 
@@ -363,16 +336,13 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         const int st = c & 1, slot = c % C::OPS;
         const uint32_t ph2 = (c >> 1) & 1;
         if (!warp_wait(&bar[DT_FULL0 + st], ph2, ab)) return;
-        if (tid == 0) M3_TRACE_EV(c, 0);
         const float* dtt = reinterpret_cast<const float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
         uint8_t* ct = C::ct(sm, slot);
         uint8_t* bt = C::bt(sm, slot);
         if (!warp_wait(&bar[OPS_EMPTY0 + slot], ((c / C::OPS) & 1) ^ 1, ab)) return;
-        if (tid == 0) M3_TRACE_EV(c, 1);
         for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
             const int rs = raw_it & 1;
             if (!warp_wait(&bar[RAW_FULL0 + rs], (raw_it >> 1) & 1, ab)) return;
-            if (tid == 0 && s == 0) M3_TRACE_EV(c, 2);
             const uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
             const uint32_t* braw = reinterpret_cast<const uint32_t*>(raw);
             const uint32_t* craw = reinterpret_cast<const uint32_t*>(raw + C::BRAW_BYTES);
@@ -393,7 +363,6 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
             rb[ts * PAIRS + pair] = own;
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[RS0 + rs]);
-            if (tid == 0) M3_TRACE_EV(c, s == 0 ? 27 : 30);
             uint32_t bv[TPT][R], cv[TPT][R];
 #pragma unroll
             for (int jj = 0; jj < TPT; ++jj)
@@ -417,7 +386,6 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                     }
             }
             if (!warp_wait(&bar[RS0 + rs], (raw_it >> 1) & 1, ab)) return;
-            if (tid == 0) M3_TRACE_EV(c, s == 0 ? 28 : 31);
             float pre = 0.f, tot = 0.f;
 #pragma unroll
             for (int qq = 0; qq < TSPLIT; ++qq) {
@@ -495,7 +463,6 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                 }
             }
             psi_acc += tot;
-            if (tid == 0 && s == 0) M3_TRACE_EV(c, 29);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[RAW_EMPTY0 + rs]);
         }
@@ -503,14 +470,12 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
         psi_acc -= 6.283185307179586f * rintf(psi_acc * 0.15915494309189535f);
         if (ts == 0) cf.psi_end()[pair] = psi_acc;
-        if (tid == 0) M3_TRACE_EV(c, 3);
 
         // ---- w-scaled X:  Xw[u, r] = 2^(cum2_end - cum2_u) w_u x[u, r]  (needs the
         //      coefficient warp's decay prefix sums of this chunk)
         if (!warp_wait(&bar[CUM_READY0 + cs], (c / kCoefSlots) & 1, ab)) return;
         const int xs = c % C::XST;
         if (!warp_wait(&bar[X_FULL0 + xs], (c / C::XST) & 1, ab)) return;
-        if (tid == 0) M3_TRACE_EV(c, 4);
         {
             const uint8_t* xt = sm + C::OFF_X + xs * C::X_BYTES;
             uint8_t* xw = C::xw(sm, slot);
@@ -537,7 +502,6 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
             mbar_arrive(&bar[OPS_FULL0 + slot]);
             mbar_arrive(&bar[DT_EMPTY0 + st]);
         }
-        if (tid == 0) M3_TRACE_EV(c, 5);
     }
 }
 
@@ -643,14 +607,12 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
         const int cs = c % kCoefSlots;
         Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
         if (!warp_wait(&bar[COEF_FULL0 + cs], (c / kCoefSlots) & 1, ab)) return;
-        if (etid == 0) M3_TRACE_EV(c, 14);
         const float* cum2 = cf.cum2();
 
         // ---- S o L -> bf16, K-major [row][col].  L[t,u] = 2^(cum2_t + ew_u) for u < t
         //      (ew_u = log2 w_u - cum2_u), gamma_t on the diagonal token; the skip D x is
         //      folded in as D on the (row == col) diagonal.
         if (!warp_wait(&bar[S_FULL], ph, ab)) return;
-        if (etid == 0) M3_TRACE_EV(c, 15);
         tc_fence_after();
         {
             const int t = lrow / R;
@@ -695,13 +657,11 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
             mbar_arrive(&bar[S_EMPTY]);
             mbar_arrive(&bar[SL_FULL]);
         }
-        if (etid == 0) M3_TRACE_EV(c, 16);
 
         // ---- y = Y_intra + e^{cum_t} Y_inter   (D x is in Y_intra; y is written over the
         //      x tile, which the x warp then stores with TMA)
         const int yb = c & 1;
         if (!warp_wait(&bar[Y_FULL0 + yb], ph2, ab)) return;
-        if (etid == 0) M3_TRACE_EV(c, 20);
         const int xs = c % C::XST;
         if (!warp_wait(&bar[X_FULL0 + xs], (c / C::XST) & 1, ab)) return;
         tc_fence_after();
@@ -746,7 +706,6 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
             mbar_arrive(&bar[Y_EMPTY0 + yb]);
             mbar_arrive(&bar[Y_STAGED0 + xs]);
         }
-        if (etid == 0) M3_TRACE_EV(c, 22);
     }
 }
 
@@ -828,11 +787,9 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
         Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
         if (!warp_wait(&bar[COEF_FULL0 + cs], (c / kCoefSlots) & 1, ab)) return;
         if (!warp_wait(&bar[DS_FULL], ph, ab)) return;
-        if (stid == 0) M3_TRACE_EV(c, 17);
         const bool more = c + 1 < p.nchunks;
         // the Y_inter MMA of this chunk must be done reading g_c before g_{c+1} replaces it
         if (more && !warp_wait(&bar[G_EMPTY], ph, ab)) return;
-        if (stid == 0) M3_TRACE_EV(c, 19);
         tc_fence_after();
         const float dec = exp2f(*cf.cum2_end());
         if (c + 1 == p.nchunks) {
@@ -883,7 +840,6 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
             if (more) mbar_arrive(&bar[G_FULL]);
             mbar_arrive(&bar[COEF_EMPTY0 + cs]);   // this warp has read the slot's cum2_end
         }
-        if (stid == 0) M3_TRACE_EV(c, 18);
     }
     if (stid == 0) {
         // only this warpgroup read x_prev (for g_0), so the carried x can be replaced now;
@@ -926,7 +882,6 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         const uint32_t ph = ((c >> 1) & 1) ^ 1;
         // per-chunk dt / A / lam (Q+1 tokens: the next chunk's first token is the lookahead)
         if (!(ok = mbar_wait(&bar[DT_EMPTY0 + st], ph, ab))) break;
-        M3_TRACE_EV(c, 24);
         mbar_arrive_expect_tx(&bar[DT_FULL0 + st], 3 * C::DT_BOX);
         float* dtt = reinterpret_cast<float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
         tma_load_3d(dtt, &p.tm_dt, &bar[DT_FULL0 + st], h & ~3, t0, b);
@@ -937,7 +892,6 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
         for (int s = 0; s < C::NSUB; ++s, ++raw_it) {
             const int rs = raw_it & 1;
             if (!(ok = mbar_wait(&bar[RAW_EMPTY0 + rs], ((raw_it >> 1) & 1) ^ 1, ab))) break;
-            if (s == 0) M3_TRACE_EV(c, 25);
             const bool sc = BC && a.bc_scale != nullptr;
             mbar_arrive_expect_tx(&bar[RAW_FULL0 + rs], C::SC_OFF + (sc ? C::SC_BOX : 0));
             uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
@@ -1000,7 +954,6 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
             bulk_commit();
             mbar_arrive(&bar[COEF_EMPTY0 + c % kCoefSlots]);
             bulk_wait_read<0>();
-            M3_TRACE_EV(c, 23);
             if (c + C::XST < p.nchunks) load(c + C::XST);
         }
         if (!ok)
@@ -1095,7 +1048,6 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
             bulk_wait_read<0>();
         }
         __syncwarp();
-        if (lane == 0) M3_TRACE_EV(c, 23);
         if (c + C::XST < p.nchunks) ok = load(c + C::XST);
     }
     if (lane == 0) {
@@ -1116,7 +1068,6 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     const int w = threadIdx.x >> 5;
 
-    M3_TRACE_INIT();
     if (threadIdx.x == 0) {
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], bar_count(i));
         misc[1] = 0u;  // abort flag
@@ -1285,13 +1236,6 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-#ifdef M3_TRACE
-extern "C" int m3_trace_copy(void* dst, size_t bytes, int cta) {
-    if (cudaMemcpyToSymbol(g_m3_trace_cta, &cta, sizeof(int)) != cudaSuccess) return 1;
-    if (!dst) return 0;
-    return cudaMemcpyFromSymbol(dst, g_m3_trace, bytes) == cudaSuccess ? 0 : 1;
-}
-#endif
 
 // The tile holds L = chunk * R (token, rank) rows with L in {64, 128}: the M = 64 / 128
 // MMA shapes, and the S and Y accumulators that fit TMEM.  A requested chunk whose L

@@ -61,10 +61,11 @@ WORKLOADS = {
 
 
 def _randn(g, shape, std=1.0, mean=0.0, dtype=torch.float32):
-    """Draw N(mean, std^2) one leading row at a time, rounded to ``dtype``."""
-    out = torch.empty(shape, dtype=dtype)
+    """Draw N(mean, std^2) one leading row at a time, rounded to ``dtype`` (on the
+    generator's device)."""
+    out = torch.empty(shape, dtype=dtype, device=g.device)
     for i in range(shape[0]):
-        r = torch.randn(shape[1:], generator=g)
+        r = torch.randn(shape[1:], generator=g, device=g.device)
         if std != 1.0:
             r.mul_(std)
         if mean != 0.0:
@@ -106,11 +107,11 @@ def make_scan_inputs(batch, seqlen, nheads, ngroups, headdim, dstate, rank=1,
     return inp
 
 
-def make_gate(shape, io_dtype=torch.bfloat16, seed=0):
+def make_gate(shape, io_dtype=torch.bfloat16, seed=0, device="cpu"):
     """Output-gate input z ~ N(0, 1) of the given shape (the layout of y), rounded to the io
     dtype.  Drawn from its own generator (seed + 7919) so that adding a gate never changes
-    the other inputs of a seeded workload."""
-    g = torch.Generator("cpu").manual_seed(seed + 7919)
+    the other inputs of a seeded workload; ``device`` as for ``make_decode_inputs``."""
+    g = torch.Generator(device).manual_seed(seed + 7919)
     return _randn(g, tuple(shape), dtype=io_dtype)
 
 
@@ -134,25 +135,37 @@ def make_expand(nheads, rank, headdim, seed=0):
 
 
 def make_decode_inputs(batch, nheads, ngroups, headdim, dstate, rank=1, tokens=1,
-                       io_dtype=torch.bfloat16, theta_max=math.pi / 8, seed=0):
+                       io_dtype=torch.bfloat16, theta_max=math.pi / 8, seed=0, device="cpu"):
     """Per-token decode inputs stacked over ``tokens`` plus the starting state.
 
     x [tok,b,H,R,P], B, C [tok,b,G,R,N] (io dtype); dt, A, lam [tok,b,H];
     theta [tok,b,G,N/2]; D [H]; h0 [b,H,N,P] ~ N(0,1) float32;
     x_prev [b,H,R,P], B_prev [b,G,R,N] drawn like x and B (io dtype).
+
+    ``device`` selects the generator: "cpu" (the default; a CPU ``torch.Generator``) or a
+    CUDA device, where torch's seeded device generator draws the same distributions in the
+    same order straight into device memory.  The two give different values for one seed.
+    Long full-size decode horizons (1000 fresh tokens of batch 256 are gigabytes) are drawn
+    on the device; a test that checks them against the oracle copies the slices it checks
+    back to the host.
     """
     b, H, G, P, N, R, K = batch, nheads, ngroups, headdim, dstate, rank, tokens
-    g = torch.Generator("cpu").manual_seed(seed)
+    g = torch.Generator(device).manual_seed(seed)
+    dev = g.device
+
+    def rn(shape):
+        return torch.randn(shape, generator=g, device=dev)
+
     inp = {}
     inp["x"] = _randn(g, (K, b, H, R, P), dtype=io_dtype)
     inp["B"] = _randn(g, (K, b, G, R, N), std=1.0 / math.sqrt(N), dtype=io_dtype)
     inp["C"] = _randn(g, (K, b, G, R, N), std=1.0 / math.sqrt(N), dtype=io_dtype)
-    inp["dt"] = torch.nn.functional.softplus(torch.randn((K, b, H), generator=g) - 2.0)
-    inp["A"] = -torch.exp(torch.randn((K, b, H), generator=g) * math.sqrt(0.5))
-    inp["lam"] = torch.sigmoid(torch.randn((K, b, H), generator=g))
-    inp["theta"] = (torch.rand((K, b, G, N // 2), generator=g) * 2.0 - 1.0) * theta_max
-    inp["D"] = torch.randn((H,), generator=g)
+    inp["dt"] = torch.nn.functional.softplus(rn((K, b, H)) - 2.0)
+    inp["A"] = -torch.exp(rn((K, b, H)) * math.sqrt(0.5))
+    inp["lam"] = torch.sigmoid(rn((K, b, H)))
+    inp["theta"] = (torch.rand((K, b, G, N // 2), generator=g, device=dev) * 2.0 - 1.0) * theta_max
+    inp["D"] = rn((H,))
     inp["h0"] = _randn(g, (b, H, N, P))
-    inp["x_prev"] = torch.randn((b, H, R, P), generator=g).to(io_dtype)
-    inp["B_prev"] = (torch.randn((b, G, R, N), generator=g) / math.sqrt(N)).to(io_dtype)
+    inp["x_prev"] = rn((b, H, R, P)).to(io_dtype)
+    inp["B_prev"] = (rn((b, G, R, N)) / math.sqrt(N)).to(io_dtype)
     return inp

@@ -18,11 +18,12 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libm3.so")
 
 M3_OK, M3_ERR_NULL, M3_ERR_SHAPE, M3_ERR_DTYPE, M3_ERR_ALIGN, M3_ERR_UNSUPPORTED, \
-    M3_ERR_WORKSPACE, M3_ERR_LAUNCH, M3_ERR_TIMEOUT, M3_ERR_CUDA = range(10)
+    M3_ERR_WORKSPACE, M3_ERR_LAUNCH, M3_ERR_TIMEOUT, M3_ERR_CUDA, M3_ERR_RANGE = range(11)
 M3_F32, M3_BF16 = 0, 1
 M3_FLAG_THETA_IS_ANGLE = 1
 M3_FLAG_FORCE_SIMT = 2
 M3_FLAG_TEST_STALL = 4
+M3_FLAG_DEBUG_CHECKS = 8
 
 EXPORTED = ("m3_state_bytes", "m3_state_init", "m3_scan_workspace_bytes", "m3_scan_fwd",
             "m3_decode_step", "m3_query_status", "m3_scan_fwd_noalloc", "m3_scan_fwd_gated",
@@ -295,7 +296,8 @@ def m3_decode_step(dims: Dims, x, B, C, dt, A, lam, theta, D, state: State, y, f
 
 
 def m3_query_status(workspace, stream=None) -> int:
-    """Synchronise the stream and return the device-side status word (M3_OK or M3_ERR_TIMEOUT)."""
+    """Synchronise the stream and return the device-side status word (M3_OK, M3_ERR_TIMEOUT or
+    M3_ERR_RANGE)."""
     return int(load_library().m3_query_status(_ptr(workspace), _stream(stream)))
 
 

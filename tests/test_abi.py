@@ -222,3 +222,43 @@ def test_backward_validation_before_launch(lib):
     assert bwd(ws_bytes=need - 256) == m3.M3_ERR_WORKSPACE
     assert bwd(dims=m3.Dims(1, 2, 1, 128, 16, 1, m3.M3_F32),
                ws_bytes=1 << 30) == m3.M3_ERR_UNSUPPORTED      # headdim 128: no kernel
+
+
+def test_status_strings_cover_range_code(lib):
+    assert "range" in m3.m3_status_string(m3.M3_ERR_RANGE)
+
+
+def test_noalloc_validation_before_any_cuda_call(lib):
+    """m3_scan_fwd_noalloc makes every host-side check of m3_scan_fwd before it asks the CUDA
+    runtime for anything: bad arguments come back as the same status codes, here on a
+    machine without a GPU."""
+    d = m3.Dims(1, 2, 1, 16, 16, 1, m3.M3_BF16)
+    p = 0x1000
+
+    def call(T=16, chunk=64, x=p, y=p, state=None, flags=0, dims=d):
+        st = state if state is not None else m3.m3_state(0x2000, 0x3000, 0x4000)
+        return lib.m3_scan_fwd_noalloc(ctypes.byref(dims.c()), T, chunk, x, p, p, p, p, p, p,
+                                       None, ctypes.byref(st), y, flags, None)
+
+    assert call(x=0) == m3.M3_ERR_NULL
+    assert call(state=m3.m3_state(0x2000, 0, 0x4000)) == m3.M3_ERR_NULL
+    assert call(y=p + 8) == m3.M3_ERR_ALIGN
+    assert call(chunk=48) == m3.M3_ERR_SHAPE
+    assert call(T=-1) == m3.M3_ERR_SHAPE
+    assert call(dims=m3.Dims(1, 3, 2, 16, 16, 1, m3.M3_BF16)) == m3.M3_ERR_SHAPE
+    assert call(T=0) == m3.M3_OK                        # validated no-op
+    # the debug scan reports into a status word this entry point never reads back
+    assert call(flags=m3.M3_FLAG_DEBUG_CHECKS) == m3.M3_ERR_UNSUPPORTED
+    import torch
+    if not torch.cuda.is_available():
+        # valid arguments reach the device lookup, which fails cleanly without a GPU
+        assert call() == m3.M3_ERR_CUDA
+
+
+def test_decode_rejects_debug_checks(lib):
+    """The decode step has no workspace status word for the debug scan to report into."""
+    d = m3.Dims(1, 2, 1, 16, 16, 1, m3.M3_BF16)
+    st = m3.m3_state(0x2000, 0x3000, 0x4000)
+    p = 0x1000
+    assert lib.m3_decode_step(ctypes.byref(d.c()), p, p, p, p, p, p, p, None, ctypes.byref(st),
+                              p, m3.M3_FLAG_DEBUG_CHECKS, None) == m3.M3_ERR_UNSUPPORTED

@@ -81,3 +81,51 @@ def test_decode_full_size_sampled(name):
     assert rel_slices(hg[bsel][:, hsel], ho, (2, 3)) <= 2e-2
     assert np.all(np.isfinite(yg)) and np.all(np.isfinite(hg))
     assert np.array_equal(bpg, f64(inp["B"][steps - 1]))
+
+
+@pytest.mark.parametrize("name", ["decode_siso_b256", "decode_mimo_b256"])
+def test_decode_full_size_1000_tokens(name):
+    """The batch-256 decode configurations over their stated horizon: 1000 sequential steps,
+    each with a fresh token, at full size in the launch configuration the bench times.  The
+    oracle recomputes sampled (batch, head) slices over all 1000 steps (every y and the final
+    state); every output of every step is checked to be finite.  The fp32 state must stay
+    within the bf16 bar after 1000 updates, not only after a few."""
+    w = inputs.WORKLOADS[name]
+    steps = w.extra["tokens"]
+    inp = inputs.make_decode_inputs(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
+                                    tokens=steps, io_dtype=w.io_dtype, theta_max=w.theta_max,
+                                    seed=9, device="cuda")
+    d = m3.Dims(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank, m3.M3_BF16)
+    bsel = torch.tensor([0, 5, 128, 201, 255])
+    hsel = torch.tensor([0, 21, 63])
+    st = m3.State(d)
+    st.h.copy_(inp["h0"])
+    st.x_prev.copy_(inp["x_prev"])
+    st.B_prev.copy_(inp["B_prev"])
+    y = torch.empty_like(inp["x"][0])
+    ysel = torch.empty((steps, len(bsel), len(hsel), w.rank, w.headdim), dtype=y.dtype,
+                       device="cuda")
+    finite = torch.ones((), dtype=torch.bool, device="cuda")
+    bs, hs = bsel.cuda(), hsel.cuda()
+    for t in range(steps):
+        m3.m3_decode_step(d, *(inp[k][t] for k in KEYS), inp["D"], st, y)
+        ysel[t] = y[bs][:, hs]
+        finite &= torch.isfinite(y).all()
+    torch.cuda.synchronize()
+    assert bool(finite) and bool(torch.isfinite(st.h).all())
+    # the oracle on the sampled slices, fed the same (already rounded) inputs
+    # (only the sampled slices come back to the host: the full inputs are gigabytes)
+    sub = {k: f64(inp[k][:, bs]) for k in ("B", "C", "theta")}
+    sub.update({k: f64(inp[k][:, bs][:, :, hs]) for k in ("x", "dt", "A", "lam")})
+    h = f64(inp["h0"][bs][:, hs])
+    xp = f64(inp["x_prev"][bs][:, hs])
+    bp = f64(inp["B_prev"][bs])
+    Dh = f64(inp["D"][hs])
+    yo = []
+    for t in range(steps):
+        yt, h, xp, bp = oracle.decode_step(*(sub[k][t] for k in KEYS), Dh, h, xp, bp)
+        yo.append(yt)
+    yo = np.stack(yo)
+    assert rel_slices(f64(ysel), yo, (0, 3, 4)) <= 2e-2
+    assert rel_slices(f64(st.h[bs][:, hs]), h, (2, 3)) <= 2e-2
+    assert torch.equal(st.B_prev, inp["B"][steps - 1])

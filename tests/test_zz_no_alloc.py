@@ -12,11 +12,10 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import f64, rel_slices
+from gpu_helpers import f64
 from state_space_model_06_b200 import inputs, m3
 
 pytestmark = pytest.mark.gpu
-TOL = 2e-2
 
 
 def _run(fn, inp, d, T, Q, **kw):
@@ -45,7 +44,22 @@ def test_noalloc_matches_workspace_entry_point(shape):
         ws = m3.alloc_workspace(d, T, Q)
         ref = _run(lambda *a: m3.m3_scan_fwd(*a[:-1], a[-1], ws), inp, d, T, Q)
         got = _run(m3.m3_scan_fwd_noalloc, inp, d, T, Q)
-        assert rel_slices(got[0], ref[0], (1, 3, 4)) <= TOL, call
-        assert rel_slices(got[1], ref[1], (2, 3)) <= TOL, call
-        assert np.array_equal(got[2], ref[2]) and np.array_equal(got[3], ref[3])
+        # the same deterministic kernel on the same inputs: bit-identical results, so that
+        # nothing left in the shared scratch by the previous call can hide
+        for k in range(4):
+            assert np.array_equal(got[k], ref[k]), (call, k)
         assert np.all(np.isfinite(got[0]))
+
+
+def test_noalloc_on_a_side_stream():
+    """A stream of the current device other than the default one works the same way."""
+    b, H, G, P, N, R, T, Q = 1, 4, 1, 64, 128, 1, 130, 64
+    d = m3.Dims(b, H, G, P, N, R, m3.M3_BF16)
+    inp = inputs.make_scan_inputs(b, T, H, G, P, N, R, io_dtype=torch.bfloat16, seed=23)
+    ws = m3.alloc_workspace(d, T, Q)
+    ref = _run(lambda *a: m3.m3_scan_fwd(*a[:-1], a[-1], ws), inp, d, T, Q)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        got = _run(lambda *a: m3.m3_scan_fwd_noalloc(*a, stream=side), inp, d, T, Q)
+    for k in range(4):
+        assert np.array_equal(got[k], ref[k]), k
