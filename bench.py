@@ -6,8 +6,9 @@ i.e. every prefill step of the method.  Alongside, as sub-metrics: the batch-256
 workloads (SISO N 128 and MIMO R 4 N 64; 1000 sequential steps with fresh tokens, captured
 once as a CUDA graph and replayed), the same prefill and decode with the fused output gate
 ("gated") and with BCNorm + BC biases ("bc"), the MIMO rank-4 prefill plain and with the
-lightweight expansion of x and z ("mimo"), the backward pass of the prefill workload
-("backward"), the end-to-end call through pinned host
+lightweight expansion of x and z ("mimo"), the long-context workload of 16 chained calls
+("longctx") and the fp32 parity workload ("small_f32"), the backward pass of the prefill
+workload ("backward"), the end-to-end call through pinned host
 buffers ("e2e"), and the CPU oracle on the workload's inputs ("cpu_baseline").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -22,6 +23,7 @@ bounded sample of the same workload and prints the same line with "impl": "refer
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -425,6 +427,90 @@ def backward_leg(args, w, d, g, dev, stream, rank, ws_world, pk):
             "kernel": "scan_bwd_kernel (sequential fp32, segment checkpoints) + group sums"}
 
 
+def longctx_leg(args, dev, stream, rank, ws_world, pk):
+    """The long-context workload: batch 1, 64 heads, 65536 tokens as 16 chained calls of 4096
+    (state and previous token carried from call to call), chunk 128, fast rotation.  One step
+    is the 16 calls; the state is reset outside the timed interval."""
+    w = inputs.WORKLOADS["siso_longctx_carry"]
+    Tc = w.seqlen // w.calls
+    inp = inputs.make_scan_inputs(w.batch, w.seqlen, w.nheads, w.ngroups, w.headdim, w.dstate,
+                                  w.rank, io_dtype=w.io_dtype, theta_max=w.theta_max,
+                                  seed=400 + rank)
+    d = m3.Dims(w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank,
+                m3.io_dtype_of(w.io_dtype))
+    keys = ("x", "B", "C", "dt", "A", "lam", "theta")
+    calls = [{k: inp[k][:, c * Tc:(c + 1) * Tc].contiguous().to(dev) for k in keys}
+             for c in range(w.calls)]
+    D = inp["D"].to(dev)
+    del inp
+    st = m3.State(d, dev)
+    ys = [torch.empty_like(c["x"]) for c in calls]
+    ws = m3.alloc_workspace(d, Tc, w.chunk, dev)
+
+    def run():
+        for c, y in zip(calls, ys):
+            m3.m3_scan_fwd(d, Tc, w.chunk, c["x"], c["B"], c["C"], c["dt"], c["A"], c["lam"],
+                           c["theta"], D, st, y, ws, stream=stream)
+    for _ in range(3):
+        m3.m3_state_init(d, st, stream=stream)
+        run()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 10))
+    per = []
+    for _ in range(steps):
+        m3.m3_state_init(d, st, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        per.append((e0, e1))
+    torch.cuda.synchronize()
+    if m3.m3_query_status(ws, stream) != m3.M3_OK:
+        raise RuntimeError("longctx: device status not OK")
+    ms = sum(a.elapsed_time(b) for a, b in per) / steps
+    # bytes and flops per call; flops of the contractions as run: with N = 128 the kernel
+    # runs chunk 128 as 64-token tiles
+    wc = dataclasses.replace(w, seqlen=Tc, chunk=64 if w.dstate == 128 else w.chunk)
+    byts, flops = scan_algorithmic(wc)
+    byts, flops = byts * w.calls, flops * w.calls
+    val, ms_max = job_throughput(w.batch * w.seqlen, ms, ws_world)
+    gbs = byts / (ms / 1e3) / 1e9
+    return {"tokens_per_s": val, "ms_per_step": ms_max, "calls_per_step": w.calls,
+            "alg_bytes_per_step": byts, "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"],
+            "tensor_frac": flops / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
+            "config": {"workload": w.name, "batch": w.batch, "heads": w.nheads,
+                       "seqlen": w.seqlen, "calls": w.calls, "headdim": w.headdim,
+                       "dstate": w.dstate, "chunk": w.chunk, "theta_max": w.theta_max}}
+
+
+def small_f32_leg(args, dev, stream, rank, ws_world):
+    """The fp32 parity workload (batch 1, 2 heads, T 256, P 16, N 16): the sequential fp32
+    CUDA-core kernel; latency-bound by design (one call is a few microseconds of work)."""
+    w = inputs.WORKLOADS["siso_f32_small"]
+    inp, d, g, st, y, ws = prefill_setup(w, dev, seed=500 + rank)
+    del inp
+    for _ in range(5):
+        m3.m3_state_init(d, st, stream=stream)
+        run_scan(w, d, g, st, y, ws, stream)
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 50))
+    per = []
+    for _ in range(steps):
+        m3.m3_state_init(d, st, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run_scan(w, d, g, st, y, ws, stream)
+        e1.record(stream)
+        per.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in per) / steps
+    val, ms_max = job_throughput(w.batch * w.seqlen, ms, ws_world)
+    return {"tokens_per_s": val, "us_per_call": ms_max * 1e3, "kernel": "scan_simt_kernel (fp32)",
+            "config": {"workload": w.name, "batch": w.batch, "heads": w.nheads,
+                       "seqlen": w.seqlen, "headdim": w.headdim, "dstate": w.dstate,
+                       "chunk": w.chunk, "io": "fp32"}}
+
+
 def w_dec_batch(name):
     return inputs.WORKLOADS[name].batch
 
@@ -468,7 +554,6 @@ def ours(args):
     w = inputs.WORKLOADS[WORKLOAD]
     if args.batch or args.seqlen:
         # a smaller case of the same workload: only for short profiler captures
-        import dataclasses
         w = dataclasses.replace(w, batch=args.batch or w.batch, seqlen=args.seqlen or w.seqlen)
     pk, pk_kind = peaks()
 
@@ -510,7 +595,7 @@ def ours(args):
 
     if args.prefill_only:
         args.no_decode = args.no_e2e = args.no_cpu = args.no_gate = args.no_mimo = True
-        args.no_bwd = True
+        args.no_bwd = args.no_longctx = True
     if not args.no_decode:
         line["decode"] = {}
         for name in (args.decode or DECODES):
@@ -565,6 +650,10 @@ def ours(args):
 
     if not args.no_mimo:
         line["mimo"] = mimo_leg(args, dev, stream, rank, ws_world, pk)
+
+    if not args.no_longctx:
+        line["longctx"] = longctx_leg(args, dev, stream, rank, ws_world, pk)
+        line["small_f32"] = small_f32_leg(args, dev, stream, rank, ws_world)
 
     if not args.no_bwd:
         line["backward"] = backward_leg(args, w, d, g, dev, stream, rank, ws_world, pk)
@@ -634,6 +723,8 @@ def main():
     ap.add_argument("--no-gate", action="store_true", help="skip the fused-output-gate legs")
     ap.add_argument("--no-mimo", action="store_true", help="skip the MIMO prefill legs")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward-pass leg")
+    ap.add_argument("--no-longctx", action="store_true",
+                    help="skip the long-context and fp32 small-workload legs")
     ap.add_argument("--cpu-rows", type=int, default=8,
                     help="batch rows of the workload timed on the CPU oracle (default: all)")
     ap.add_argument("--ref-tokens", type=int, default=256)

@@ -59,7 +59,7 @@ typedef enum {
     M3_ERR_DTYPE = 3,       /* unknown io dtype */
     M3_ERR_ALIGN = 4,       /* a pointer is not aligned as documented */
     M3_ERR_UNSUPPORTED = 5, /* valid arguments that no kernel of this build handles */
-    M3_ERR_WORKSPACE = 6,   /* workspace missing or smaller than m3_scan_workspace_bytes */
+    M3_ERR_WORKSPACE = 6,   /* workspace missing, misaligned or below its minimum size */
     M3_ERR_LAUNCH = 7,      /* a kernel launch failed (cudaGetLastError) */
     M3_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up (reported by m3_query_status) */
     M3_ERR_CUDA = 9,        /* another CUDA runtime call failed */
@@ -151,14 +151,23 @@ typedef struct {
     const float* z_expand;
 } m3_extras;
 
-/* Workspace bytes m3_scan_fwd needs for (dims, seqlen, chunk); at least 256
+/* Workspace bytes m3_scan_fwd uses for (dims, seqlen, chunk); at least 256
  * (the status word).  The workspace is caller-owned device memory, 256-byte
- * aligned, and must not be shared by calls that can overlap on the GPU. */
+ * aligned, and must not be shared by calls that can overlap on the GPU.
+ * Where batch * nheads is at most a third of the SMs of the current device (long
+ * sequences with few streams, such as batch 1 x 32 heads), the bf16 tensor-core path
+ * splits each sequence into segments run side by side ("Parallel representation under SSD": the carried
+ * state is affine in the state entering a segment, so segments compose), and the size
+ * includes their records: per (batch, head, segment) two N x P fp32 states, the
+ * segment's decay and N/2 angles.  A workspace of at least the minimum (256 bytes, plus
+ * the BCNorm scales of m3_scan_workspace_bytes_ex) but without room for the records is
+ * accepted: the call then runs unsegmented, with the same results up to rounding.
+ * Layout: [status 256][BCNorm scales][segment records]. */
 m3_status m3_scan_workspace_bytes(const m3_dims* dims, int32_t seqlen, int32_t chunk,
                                   size_t* bytes);
 
 /* Workspace bytes of m3_scan_fwd_ex with these extras: the above plus, when BCNorm is on,
- * one float per B, C and B_prev rank column of the call (its scales). */
+ * one float per B, C and B_prev rank column of the call (its scales; 256-byte rounded). */
 m3_status m3_scan_workspace_bytes_ex(const m3_dims* dims, int32_t seqlen, int32_t chunk,
                                      const m3_extras* extras, size_t* bytes);
 
@@ -228,8 +237,10 @@ m3_status m3_scan_fwd_gated(const m3_dims* dims, int32_t seqlen, int32_t chunk, 
  * Same arguments, layouts, results and errors as m3_scan_fwd, minus the workspace.
  * Every host-side check of m3_scan_fwd runs first, before any CUDA call.  The workspace
  * is lent from one fixed scratch array compiled into the library (64 KiB, 256-byte
- * aligned, held on every GPU that loads the library until the process exits); shapes
- * whose m3_scan_workspace_bytes exceeds 64 KiB are rejected with M3_ERR_WORKSPACE.
+ * aligned, held on every GPU that loads the library until the process exits), which
+ * holds the status word: the call runs without sequence segments, as m3_scan_fwd does
+ * with a workspace of that size.  Shapes whose minimum workspace exceeded 64 KiB would
+ * be rejected with M3_ERR_WORKSPACE (none does: without extras the minimum is 256 B).
  * Nothing is allocated: no cudaMalloc / cudaFree and no allocating library routine.
  *   - `stream` must belong to the current device (the array's address is per device);
  *     a stream of another device is rejected with M3_ERR_UNSUPPORTED.

@@ -142,7 +142,8 @@ namespace {
 bool bc_norm_on(const m3_extras* ex) { return ex && ex->bc_norm_eps > 0.f; }
 bool bc_any(const m3_extras* ex) { return ex && (ex->B_bias || ex->C_bias || ex->bc_norm_eps > 0.f); }
 
-// Bytes of the BCNorm scale buffer after the tensor-core workspace (256-byte aligned).
+// Bytes of the BCNorm scale buffer after the status block (256-byte aligned).  The
+// workspace is laid out as [status block][BCNorm scales][tensor-core segment records].
 size_t bc_bytes(const m3_dims* d, int32_t seqlen, const m3_extras* ex) {
     if (!bc_norm_on(ex)) return 0;
     const size_t n = sizeof(float) * bc_scale_floats(d->batch, seqlen, d->ngroups, d->rank);
@@ -191,9 +192,9 @@ m3_status scan_validate(const m3_dims* d, int32_t seqlen, int32_t chunk, const v
     if (seqlen < 0) return M3_ERR_SHAPE;
     if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return M3_ERR_SHAPE;
     if ((st = check_state(state)) != M3_OK) return st;
-    size_t base = 0;
-    m3_scan_workspace_bytes(d, seqlen, chunk, &base);
-    *need = base + bc_bytes(d, seqlen, ex);
+    // the minimum: the status block and the BCNorm scales; the segment records that
+    // m3_scan_workspace_bytes adds are optional (without them the call runs unsegmented)
+    *need = kStatusBytes + bc_bytes(d, seqlen, ex);
     if (seqlen == 0) return M3_OK;   // no tokens: nothing is read, written or launched
     if (!x || !B || !C || !dt || !A || !lam || !theta || !y) return M3_ERR_NULL;
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
@@ -233,8 +234,7 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
                                  flags, &need);
     if (st != M3_OK || seqlen == 0) return st;
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return M3_ERR_WORKSPACE;
-    size_t base = 0;
-    m3_scan_workspace_bytes(d, seqlen, chunk, &base);
+    const size_t base = kStatusBytes;   // the BCNorm scales follow the status block
 
     const int N = d->dstate, P = d->headdim, R = d->rank;
     // the tensor-core kernel reads dt / A / lam / theta with TMA (16-byte aligned rows)
@@ -258,7 +258,8 @@ m3_status scan_impl(const m3_dims* d, int32_t seqlen, int32_t chunk, const void*
     a.bc_scale = bc_norm_on(ex) ? reinterpret_cast<const float*>(static_cast<char*>(workspace) + base)
                                 : nullptr;
     a.status = static_cast<uint32_t*>(workspace);
-    a.ws = static_cast<char*>(workspace) + kStatusBytes;
+    a.ws = static_cast<char*>(workspace) + need;
+    a.ws_bytes = workspace_bytes - need;
     a.T = seqlen; a.batch = d->batch; a.H = d->nheads; a.G = d->ngroups; a.P = P; a.N = N;
     a.chunk = use_tc ? qt : chunk; a.ppt = ppt; a.ns = ns; a.flags = flags;
 

@@ -88,7 +88,8 @@ struct ScanArgs {
     const float* x_expand;  // [H][R][P]: x is [b][T][H][P], X[r][p] = x[p] w[h][r][p]; or null
     const float* z_expand;  // [H][R][P]: z is [b][T][H][P], likewise; or null
     uint32_t* status;    // workspace status word (may be null)
-    void* ws;            // workspace (after the status block)
+    void* ws;            // workspace after the status block and the BCNorm scales
+    size_t ws_bytes;     // bytes at ws (the tensor-core kernel's segment records)
     long long T;
     int batch, H, G, P, N;
     int chunk;

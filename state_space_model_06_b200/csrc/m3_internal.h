@@ -42,6 +42,9 @@ cudaError_t launch_scan_simt(const ScanArgs& a, int R, int io_dtype, cudaStream_
 // falls back to the SIMT kernel).
 int scan_tc_chunk(int N, int P, int R, int chunk, int H);   // tile chunk, 0 = none
 size_t scan_tc_workspace_bytes(int batch, int H, int N, int P, int R, long long T, int chunk);
+// sequence segments per (batch, head) the tensor-core prefill uses for nch chunks over BH
+// (batch * head) streams, given the workspace for their records
+int scan_tc_segments(int BH, long long nch);
 cudaError_t launch_scan_tc(const ScanArgs& a, int R, cudaStream_t s);
 
 // BCNorm scales of every B, C and B_prev column of a prefill call into a.bc_scale

@@ -188,9 +188,56 @@ struct TcParams {
     CUtensorMap tm_x, tm_y, tm_z, tm_B, tm_C, tm_th, tm_dt, tm_A, tm_lam, tm_sc;
     CUtensorMap tm_xr, tm_zr;   // one value per head channel (MIMO lightweight expansion)
     ScanArgs a;
-    int nchunks;
+    int nch_total;      // chunks of the call
+    int S;              // segments per (batch, head); 1: the call is one segment
+    float* seg;         // segment records (S > 1), see seg_rec_floats
     unsigned long long limit_ns;
 };
+
+// Segment records, fp32, one per (segment s, batch * head bh) at index s * batch * H + bh:
+//   M    [N][P]  the segment's final state when it starts from no state (segment pass)
+//   G0   [N][P]  the segment's initial state g_0: h0 plus the first token's beta term for
+//                segment 0; the beta term alone from the segment pass and the entry state
+//                added by the chain step for the others
+//   dec          the segment's total decay, e^{sum of its log-decays}
+//   psi  [N/2]   the angles of the segment's final frame (segment-relative)
+__host__ __device__ constexpr size_t seg_rec_floats(int N, int P) {
+    return 2 * (size_t)N * P + 4 + N / 2;
+}
+__host__ __device__ constexpr size_t seg_off_g0(int N, int P) { return (size_t)N * P; }
+__host__ __device__ constexpr size_t seg_off_dec(int N, int P) { return 2 * (size_t)N * P; }
+__host__ __device__ constexpr size_t seg_off_psi(int N, int P) { return 2 * (size_t)N * P + 4; }
+
+// One CTA's share of the call: (batch b, head h, segment s).  The call's chunks are split
+// into S contiguous runs ("Parallel representation under SSD": the carried state is an
+// affine function of the state entering the run, so runs compose).  The segment pass
+// (MAP) runs segments 0 .. S-2 from no entry state (segment S-1 only prepares its g_0);
+// the output pass runs every segment from its prepared g_0.
+struct Unit {
+    int b, h, g, s;
+    size_t bh;
+    int nch;              // chunks this launch runs for the unit
+    long long t0, tend;   // the segment's first token and its end (exclusive)
+    bool last;            // the segment holds the call's last token
+};
+template <int Q, bool MAP>
+__device__ __forceinline__ Unit unit_of(const TcParams& p) {
+    const ScanArgs& a = p.a;
+    const int BH = a.batch * a.H;
+    Unit u;
+    u.s = (int)(blockIdx.x / BH);
+    u.bh = blockIdx.x % BH;
+    u.b = (int)(u.bh / a.H);
+    u.h = (int)(u.bh % a.H);
+    u.g = u.h / (a.H / a.G);
+    const int c0 = (int)((long long)u.s * p.nch_total / p.S);
+    const int c1 = (int)((long long)(u.s + 1) * p.nch_total / p.S);
+    u.last = u.s == p.S - 1;
+    u.nch = (MAP && u.last) ? 0 : c1 - c0;
+    u.t0 = (long long)c0 * Q;
+    u.tend = u.last ? a.T : (long long)c1 * Q;
+    return u;
+}
 
 // coefficient slot layout (floats): cum2[Q] | gam[Q] | w[Q] | ew[Q] | psi_end[N/2] | cum2_end
 //   cum2: chunk-relative log2-decay prefix; ew_u = log2(w_u) - cum2_u (mask exponent offset);
@@ -242,25 +289,43 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int k, uint32_t lbo) 
 }
 
 // ---------------------------------------------------------------------------------
-template <int NST, int Q, int R, bool GT, bool BC>
-__device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab);
+template <int NST, int Q, int R, bool GT, bool BC, bool MAP>
+__device__ void producer(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* bar,
+                         const Abort& ab);
 
 // ---------------------------------------------------------------------------------
 // ---------------------------------------------------------------------------------
-template <int NST, int Q, int R, bool GT>
-__device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
-                           const Abort& ab) {
+template <int NST, int Q, int R, bool GT, bool MAP>
+__device__ void mma_issuer(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* bar,
+                           uint32_t tmem, const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     const uint32_t s_sl = smem_u32(sm + C::OFF_SL), s_g = smem_u32(sm + C::OFF_G);
     // failure-path test hook: wait on a barrier nothing completes (bounded, then abort)
     if ((p.a.flags & M3_FLAG_TEST_STALL) && !mbar_wait(&bar[NEVER], 0, ab)) return;
-    for (int c = 0; c < p.nchunks; ++c) {
+    for (int c = 0; c < u.nch; ++c) {
         const uint32_t ph = c & 1;
         const int yb = c & 1;
         const int slot = c % C::OPS;
         const uint32_t s_ct = smem_u32(C::ct(sm, slot)), s_bt = smem_u32(C::bt(sm, slot));
         const uint32_t s_xw = smem_u32(C::xw(sm, slot));
         if (!mbar_wait(&bar[OPS_FULL0 + slot], (c / C::OPS) & 1, ab)) return;
+        if constexpr (MAP) {
+            // segment pass: dS only.  Once the operands are published the rotation warps
+            // no longer read x(c) or the chunk's coefficients: release the stage for the x
+            // warp (in place of the four epilogue warps of the output pass).
+            const int xs = c % C::XST;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mbar_arrive(&bar[Y_STAGED0 + xs]);
+            if (!mbar_wait(&bar[DS_EMPTY], ph ^ 1, ab)) return;
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < C::L / 16; ++k)
+                mma_bf16(tmem + C::TM_DS, desc_mn(s_bt, k, C::L * 128u), desc_mn(s_xw, k, 1024u),
+                         C::ID_DS, k > 0);
+            mma_commit(&bar[DS_FULL]);
+            mma_commit(&bar[OPS_EMPTY0 + slot]);
+            continue;
+        }
         tc_fence_after();
         // S = C~ B~^T   (M = L tokens*ranks, N = L, K = NST)
         if (!mbar_wait(&bar[S_EMPTY], ph ^ 1, ab)) return;
@@ -307,8 +372,9 @@ __device__ void mma_issuer(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32
 // ts = rw / PB.  The starting angle of a thread's token range is the running angle plus
 // the angle sums of the earlier ranges, exchanged through shared memory once per
 // sub-chunk (bounded mbarrier hand-off).
-template <int NST, int Q, int R, bool GT, bool BC>
-__device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
+template <int NST, int Q, int R, bool GT, bool BC, bool MAP>
+__device__ void rotation(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* bar,
+                         const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     constexpr int TPT = C::TPT, PAIRS = C::PAIRS, TSPLIT = C::TSPLIT;
     const ScanArgs& a = p.a;
@@ -316,7 +382,7 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
     const int rw = tid >> 5, lane = tid & 31;
     const int ts = rw / C::PB;
     const int pair = (rw % C::PB) * 32 + lane;   // this thread's state pair
-    const int hq = (blockIdx.x % a.H) & 3;       // column of this head in the 4-head dt tile
+    const int hq = u.h & 3;                      // column of this head in the 4-head dt tile
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     const int atom = (2 * pair) >> 6, col = (2 * pair) & 63;
     float* rsum = reinterpret_cast<float*>(sm + C::OFF_RSUM);
@@ -324,15 +390,15 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
     // BC map ("Technical Approach", BCNorm and BC biases): B and C of this thread's pair
     // channels become v * s + bias, s the column's BCNorm scale (1 when off), bias the head's
     constexpr bool bc = BC;
-    const int hh = blockIdx.x % a.H;
+    const int hh = u.h;
     float bb0 = 0.f, bb1 = 0.f, cb0 = 0.f, cb1 = 0.f;
     if (a.B_bias) { bb0 = a.B_bias[hh * NST + 2 * pair]; bb1 = a.B_bias[hh * NST + 2 * pair + 1]; }
     if (a.C_bias) { cb0 = a.C_bias[hh * NST + 2 * pair]; cb1 = a.C_bias[hh * NST + 2 * pair + 1]; }
     const bool has_sc = a.bc_scale != nullptr;       // BCNorm scales come with the raw stage
-    // call-relative angle of this thread's pair (the RoPE frame of Proposition 4 starts at
-    // the first token of the call), reduced mod 2 pi at chunk boundaries
+    // segment-relative angle of this thread's pair (the RoPE frame of Proposition 4 starts at
+    // the first token of the segment), reduced mod 2 pi at chunk boundaries
     float psi_acc = 0.f;
-    for (int c = 0; c < p.nchunks; ++c) {
+    for (int c = 0; c < u.nch; ++c) {
         const int st = c & 1, slot = c % C::OPS;
         const uint32_t ph2 = (c >> 1) & 1;
         if (!warp_wait(&bar[DT_FULL0 + st], ph2, ab)) return;
@@ -370,7 +436,7 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                 for (int r = 0; r < R; ++r) {
                     const int e = (((j0 + jj) * R + r) * NST) / 2 + pair;
                     bv[jj][r] = braw[e];
-                    cv[jj][r] = craw[e];
+                    cv[jj][r] = MAP ? 0u : craw[e];   // the segment pass needs no C~
                 }
             // BCNorm scales of the own tokens, [2][R][RT] in the raw stage (0 past the end
             // of the call, where B and C are zero-filled and the rows are masked out)
@@ -413,7 +479,7 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
                 else
                     off = (uint32_t)(row0 + k) * 128u + ((cx ^ (uint32_t)((row0 + k) & 7)) << 4);
                 *reinterpret_cast<uint32_t*>(cbase + C::CT_BYTES + off) = bo;
-                *reinterpret_cast<uint32_t*>(cbase + off) = co;
+                if constexpr (!MAP) *reinterpret_cast<uint32_t*>(cbase + off) = co;
             };
             // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1], two tokens per packed
             // fp32x2 operation (their cos and sin form the packed operands)
@@ -508,12 +574,15 @@ __device__ void rotation(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
 // Coefficient warp: per-token log2-decay prefix sum (warp scan), gamma, w and the mask
 // exponent offsets ew_u = log2(w_u) - cum2_u of each chunk, into a ring of slots.
 template <int NST, int Q, int R, bool GT>
-__device__ void coefficients(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
+__device__ void coefficients(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* bar,
+                             const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
-    const ScanArgs& a = p.a;
     const int lane = threadIdx.x & 31;
-    const int hq = (blockIdx.x % a.H) & 3;
-    for (int c = 0; c < p.nchunks; ++c) {
+    const int hq = u.h & 3;
+    for (int c = 0; c < u.nch; ++c) {
+        // tokens at or past the segment end lend no beta term to the last token: its
+        // w is gamma alone, as at the end of the call
+        const long long tnext = u.t0 + (long long)c * Q + 1;
         const int st = c & 1, cs = c % kCoefSlots;
         if (!warp_wait(&bar[DT_FULL0 + st], (c >> 1) & 1, ab)) return;
         const float* dtt = reinterpret_cast<const float*>(sm + C::OFF_DT + st * 3 * C::DT_BYTES);
@@ -529,7 +598,8 @@ __device__ void coefficients(const TcParams& p, uint8_t* sm, uint64_t* bar, cons
                 const float d = dtt[t * 4 + hq], lm = lt[t * 4 + hq];
                 l2 = d * At[t * 4 + hq] * kLog2e;
                 gm = lm * d;
-                const float dn = dtt[(t + 1) * 4 + hq], ln = lt[(t + 1) * 4 + hq];
+                const float dn = tnext + t < u.tend ? dtt[(t + 1) * 4 + hq] : 0.f;
+                const float ln = lt[(t + 1) * 4 + hq];
                 wv = gm + (1.f - ln) * dn;
             }
 #pragma unroll
@@ -588,21 +658,21 @@ struct Lanes {
 
 // Epilogue warpgroup (warps 2-5): masks S into the bf16 operand S o L and writes y.
 template <int NST, int Q, int R, bool GT>
-__device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
-                         const Abort& ab) {
+__device__ void epilogue(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* bar,
+                         uint32_t tmem, const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
     const Lanes<NST, Q, R> ln(tmem);
     const int lane = ln.lane;
     const int etid = threadIdx.x - 64;                     // 0..127
-    const float Dh = a.D ? a.D[blockIdx.x % a.H] : 0.f;
+    const float Dh = a.D ? a.D[u.h] : 0.f;
     constexpr bool kHalfL = (C::L == 64);
     const int lrow = ln.row(kHalfL), lcol0 = ln.col0(kHalfL);
     constexpr int kLCols = kHalfL ? 32 : C::L;
     constexpr int kYCols = kHalfL ? 32 : kP;
     uint8_t* sl = sm + C::OFF_SL;
 
-    for (int c = 0; c < p.nchunks; ++c) {
+    for (int c = 0; c < u.nch; ++c) {
         const uint32_t ph = c & 1, ph2 = (c >> 1) & 1;
         const int cs = c % kCoefSlots;
         Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
@@ -712,21 +782,28 @@ __device__ void epilogue(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t
 // State warpgroup (warps 16-19): the fp32 carried state g in TMEM columns TM_G..,
 // g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T, per chunk g <- e^{cum_end} g + dS and its
 // bf16 copy for the Y_inter MMA; at the end h_T = R(psi_T) g and the carried x.
-template <int NST, int Q, int R, bool GT, bool BC, bool XE>
-__device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tmem,
-                      const Abort& ab) {
+// Segmented calls: the segment pass (MAP) starts segment s from h0 (s = 0) or from no
+// state (s > 0) plus the beta term of its first token, whose previous token is then the
+// call's token t0 - 1; it records that g_0 and, instead of h_T, the segment's final
+// state, total decay and final angles.  The output pass starts from the recorded g_0
+// (completed by the chain step), and only the last segment writes h_T and the carried x.
+template <int NST, int Q, int R, bool GT, bool BC, bool XE, bool MAP>
+__device__ void state(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* bar,
+                      uint32_t tmem, const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
     const Lanes<NST, Q, R> ln(tmem);
     const int lane = ln.lane;
     const int stid = threadIdx.x - 512;                    // 0..127
-    const int b = blockIdx.x / a.H, h = blockIdx.x % a.H, g = h / (a.H / a.G);
+    const int b = u.b, h = u.h, g = u.g;
     const long long T = a.T;
-    const size_t bh = (size_t)b * a.H + h;
+    const size_t bh = u.bh;
     constexpr bool kHalfN = (NST == 64);
     const int nrow = ln.row(kHalfN), ncol0 = ln.col0(kHalfN);
     constexpr int kNCols = kHalfN ? 32 : kP;
     uint8_t* gs = sm + C::OFF_G;
+    float* rec = p.S > 1 ? p.seg + ((size_t)u.s * a.batch * a.H + bh) * seg_rec_floats(NST, kP)
+                         : nullptr;
 
     auto publish16 = [&](int cb, const uint32_t (&v)[16]) {
 #pragma unroll
@@ -740,82 +817,131 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
         }
     };
 
-    // ---- g_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T
+    // ---- g_0 = h0 + (1 - lam_t0) dt_t0 B_prev x_prev^T
     {
-        const float* h0 = a.h + (bh * NST + nrow) * kP + ncol0;
-        const float d0 = a.dt[(size_t)b * T * a.H + h], l0 = a.lam[(size_t)b * T * a.H + h];
+        const bool prepared = !MAP && p.S > 1;   // recorded by the segment pass and the chain
+        const bool carried = u.s == 0;           // the previous token is the carried one
+        const size_t tok0 = (size_t)b * T + u.t0;  // the segment's first token
+        const float d0 = a.dt[tok0 * a.H + h], l0 = a.lam[tok0 * a.H + h];
         const float beta0 = (1.f - l0) * d0;
-        const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(a.x_prev) + bh * R * kP;
         const __nv_bfloat16* bp =
-            static_cast<const __nv_bfloat16*>(a.B_prev) + ((size_t)b * a.G + g) * R * NST;
-        // the carried previous token's B goes through the BC map as well
-        const float* sP =
-            a.bc_scale ? a.bc_scale + 2 * (size_t)a.batch * a.G * R * bc_tpad(T) + ((size_t)b * a.G + g) * R
-                       : nullptr;
+            carried ? static_cast<const __nv_bfloat16*>(a.B_prev) + ((size_t)b * a.G + g) * R * NST
+                    : static_cast<const __nv_bfloat16*>(a.B) + ((tok0 - 1) * a.G + g) * R * NST;
+        // BCNorm scale of the previous token's B (rank r): the carried token's, or the
+        // call's token t0 - 1
+        const size_t Tp = (size_t)bc_tpad(T);
+        auto bscale = [&](int r) -> float {
+            if (!a.bc_scale) return 1.f;
+            return carried ? a.bc_scale[2 * (size_t)a.batch * a.G * R * Tp +
+                                        ((size_t)b * a.G + g) * R + r]
+                           : a.bc_scale[(((size_t)b * a.G + g) * R + r) * Tp + (u.t0 - 1)];
+        };
+        // the previous token's X: the carried (already expanded) x, or the call's x at
+        // t0 - 1, expanded and rounded as the x stages hold it
+        const float* wx = (!carried && XE && a.x_expand) ? a.x_expand + (size_t)h * R * kP : nullptr;
+        const __nv_bfloat16* xp =
+            carried ? static_cast<const __nv_bfloat16*>(a.x_prev) + bh * R * kP
+                    : static_cast<const __nv_bfloat16*>(a.x) + ((tok0 - 1) * a.H + h) * (wx ? 1 : R) * kP;
+        auto xval = [&](int r, int col) -> float {
+            if (wx)
+                return __bfloat162float(
+                    __float2bfloat16_rn(__bfloat162float(xp[col]) * wx[r * kP + col]));
+            return __bfloat162float(xp[r * kP + col]);
+        };
         const float* Bb = a.B_bias ? a.B_bias + (size_t)h * NST : nullptr;
+        const float* h0 = a.h + (bh * NST + nrow) * kP + ncol0;
+        float* g0r = rec ? rec + seg_off_g0(NST, kP) + (size_t)nrow * kP + ncol0 : nullptr;
 #pragma unroll 1
         for (int cb = 0; cb < kNCols; cb += 16) {
             float gv[16];
+            if (prepared) {
 #pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(h0 + cb + j);
-                gv[j] = v.x; gv[j + 1] = v.y; gv[j + 2] = v.z; gv[j + 3] = v.w;
-            }
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(g0r + cb + j);
+                    gv[j] = v.x; gv[j + 1] = v.y; gv[j + 2] = v.z; gv[j + 3] = v.w;
+                }
+            } else {
+                // the segment pass starts a later segment from no state
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const float bv0 = __bfloat162float(bp[r * NST + nrow]);
-                const float bb = beta0 * (BC ? bc_apply(bv0, sP ? sP[r] : 1.f, Bb, nrow) : bv0);
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 v = carried ? *reinterpret_cast<const float4*>(h0 + cb + j)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+                    gv[j] = v.x; gv[j + 1] = v.y; gv[j + 2] = v.z; gv[j + 3] = v.w;
+                }
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    gv[j] = fmaf(bb, __bfloat162float(xp[r * kP + ncol0 + cb + j]), gv[j]);
+                for (int r = 0; r < R; ++r) {
+                    const float bv0 = __bfloat162float(bp[r * NST + nrow]);
+                    const float bb = beta0 * (BC ? bc_apply(bv0, bscale(r), Bb, nrow) : bv0);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) gv[j] = fmaf(bb, xval(r, ncol0 + cb + j), gv[j]);
+                }
+                if (MAP) {
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4)
+                        *reinterpret_cast<float4*>(g0r + cb + j) =
+                            make_float4(gv[j], gv[j + 1], gv[j + 2], gv[j + 3]);
+                }
             }
             uint32_t v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(gv[j]);
             ln.st16(kHalfN, C::TM_G, cb, v);
-            publish16(cb, v);
+            if constexpr (!MAP) publish16(cb, v);
         }
         tmem_wait_st();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[G_FULL]);
+        if constexpr (!MAP) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[G_FULL]);
+        }
     }
 
-    for (int c = 0; c < p.nchunks; ++c) {
+    float cum_seg = 0.f;   // the segment's summed log2-decay (segment pass)
+    for (int c = 0; c < u.nch; ++c) {
         const uint32_t ph = c & 1;
         const int cs = c % kCoefSlots;
         Coef<NST, Q, R> cf{reinterpret_cast<float*>(sm + C::OFF_COEF) + cs * C::COEF_FLOATS};
         if (!warp_wait(&bar[COEF_FULL0 + cs], (c / kCoefSlots) & 1, ab)) return;
         if (!warp_wait(&bar[DS_FULL], ph, ab)) return;
-        const bool more = c + 1 < p.nchunks;
+        const bool more = c + 1 < u.nch;
         // the Y_inter MMA of this chunk must be done reading g_c before g_{c+1} replaces it
-        if (more && !warp_wait(&bar[G_EMPTY], ph, ab)) return;
+        if (!MAP && more && !warp_wait(&bar[G_EMPTY], ph, ab)) return;
         tc_fence_after();
-        const float dec = exp2f(*cf.cum2_end());
-        if (c + 1 == p.nchunks) {
-            // last chunk: the call's final state goes back to the original frame,
-            // h_T = R(psi_T) (e^{cum_end} g + dS)
+        const float c2e = *cf.cum2_end();
+        const float dec = exp2f(c2e);
+        cum_seg += c2e;
+        if (c + 1 == u.nch) {
+            // last chunk: the final state goes back to the original frame,
+            // h_T = R(psi_T) (e^{cum_end} g + dS): the call's h_T (its last segment), or the
+            // segment's final state of the segment pass
+            float* out = MAP ? rec + (size_t)nrow * kP + ncol0
+                             : (u.last ? a.h + (bh * NST + nrow) * kP + ncol0 : nullptr);
             float sn, cn;
             sincosf(cf.psi_end()[nrow >> 1], &sn, &cn);
             const bool odd = nrow & 1;
-            float* hT = a.h + (bh * NST + nrow) * kP + ncol0;
+            if (out) {
 #pragma unroll 1
-            for (int cb = 0; cb < kNCols; cb += 16) {
-                uint32_t d[16], gq[16];
-                ln.ld16(kHalfN, C::TM_DS, cb, d);
-                ln.ld16(kHalfN, C::TM_G, cb, gq);
-                tmem_wait_ld();
-                float gv[16];
+                for (int cb = 0; cb < kNCols; cb += 16) {
+                    uint32_t d[16], gq[16];
+                    ln.ld16(kHalfN, C::TM_DS, cb, d);
+                    ln.ld16(kHalfN, C::TM_G, cb, gq);
+                    tmem_wait_ld();
+                    float gv[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float gj = fmaf(dec, __uint_as_float(gq[j]), __uint_as_float(d[j]));
-                    const float o = __shfl_xor_sync(0xffffffffu, gj, 1);
-                    gv[j] = odd ? fmaf(sn, o, cn * gj) : fmaf(cn, gj, -sn * o);
+                    for (int j = 0; j < 16; ++j) {
+                        const float gj = fmaf(dec, __uint_as_float(gq[j]), __uint_as_float(d[j]));
+                        const float o = __shfl_xor_sync(0xffffffffu, gj, 1);
+                        gv[j] = odd ? fmaf(sn, o, cn * gj) : fmaf(cn, gj, -sn * o);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4)
+                        *reinterpret_cast<float4*>(out + cb + j) =
+                            make_float4(gv[j], gv[j + 1], gv[j + 2], gv[j + 3]);
                 }
-#pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                    *reinterpret_cast<float4*>(hT + cb + j) =
-                        make_float4(gv[j], gv[j + 1], gv[j + 2], gv[j + 3]);
+            }
+            if (MAP) {
+                if (!odd && ncol0 == 0) rec[seg_off_psi(NST, kP) + (nrow >> 1)] = cf.psi_end()[nrow >> 1];
+                if (stid == 0) rec[seg_off_dec(NST, kP)] = exp2f(cum_seg);
             }
         } else {
 #pragma unroll 1
@@ -828,29 +954,30 @@ __device__ void state(const TcParams& p, uint8_t* sm, uint64_t* bar, uint32_t tm
                 for (int j = 0; j < 16; ++j)
                     gq[j] = __float_as_uint(fmaf(dec, __uint_as_float(gq[j]), __uint_as_float(d[j])));
                 ln.st16(kHalfN, C::TM_G, cb, gq);
-                publish16(cb, gq);
+                if constexpr (!MAP) publish16(cb, gq);
             }
             tmem_wait_st();
         }
         tc_fence_before();
-        fence_proxy_async_smem();
+        if constexpr (!MAP) fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
             mbar_arrive(&bar[DS_EMPTY]);
-            if (more) mbar_arrive(&bar[G_FULL]);
+            if (!MAP && more) mbar_arrive(&bar[G_FULL]);
             mbar_arrive(&bar[COEF_EMPTY0 + cs]);   // this warp has read the slot's cum2_end
         }
     }
-    if (stid == 0) {
-        // only this warpgroup read x_prev (for g_0), so the carried x can be replaced now;
-        // with the lightweight expansion it takes the expanded X_{T-1}, as the stage held it
+    if (!MAP && u.last && stid == 0) {
+        // only this warpgroup read x_prev (for g_0, and in a segmented call the segment
+        // pass read it before this launch), so the carried x can be replaced now; with the
+        // lightweight expansion it takes the expanded X_{T-1}, as the stage held it
         const size_t row = ((size_t)b * T + (T - 1)) * a.H + h;
         if (XE && a.x_expand) {
             const __nv_bfloat16* xl = static_cast<const __nv_bfloat16*>(a.x) + row * kP;
-            const float* wx = a.x_expand + (size_t)h * R * kP;
+            const float* wxl = a.x_expand + (size_t)h * R * kP;
             __nv_bfloat16* xpo = static_cast<__nv_bfloat16*>(a.x_prev) + bh * R * kP;
             for (int e = 0; e < R * kP; ++e)
-                xpo[e] = __float2bfloat16_rn(__bfloat162float(xl[e % kP]) * wx[e]);
+                xpo[e] = __float2bfloat16_rn(__bfloat162float(xl[e % kP]) * wxl[e]);
         } else {
             const uint4* xl = reinterpret_cast<const uint4*>(
                 static_cast<const __nv_bfloat16*>(a.x) + row * R * kP);
@@ -868,17 +995,18 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
     }
 }
 
-template <int NST, int Q, int R, bool GT, bool BC>
-__device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
+template <int NST, int Q, int R, bool GT, bool BC, bool MAP>
+__device__ void producer(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* bar,
+                         const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
-    const int b = blockIdx.x / a.H, h = blockIdx.x % a.H, g = h / (a.H / a.G);
+    const int b = u.b, h = u.h, g = u.g;
     // loads issued per ring stage, so that an aborted CTA can wait for them to land
     int n_dt[2] = {0, 0}, n_raw[2] = {0, 0};
     int raw_it = 0;
     bool ok = true;
-    for (int c = 0; c < p.nchunks && ok; ++c) {
-        const int t0 = c * Q, st = c & 1;
+    for (int c = 0; c < u.nch && ok; ++c) {
+        const int t0 = (int)(u.t0 + (long long)c * Q), st = c & 1;
         const uint32_t ph = ((c >> 1) & 1) ^ 1;
         // per-chunk dt / A / lam (Q+1 tokens: the next chunk's first token is the lookahead)
         if (!(ok = mbar_wait(&bar[DT_EMPTY0 + st], ph, ab))) break;
@@ -893,11 +1021,14 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
             const int rs = raw_it & 1;
             if (!(ok = mbar_wait(&bar[RAW_EMPTY0 + rs], ((raw_it >> 1) & 1) ^ 1, ab))) break;
             const bool sc = BC && a.bc_scale != nullptr;
-            mbar_arrive_expect_tx(&bar[RAW_FULL0 + rs], C::SC_OFF + (sc ? C::SC_BOX : 0));
+            // the segment pass reads no C
+            mbar_arrive_expect_tx(&bar[RAW_FULL0 + rs],
+                                  C::SC_OFF - (MAP ? C::BRAW_BYTES : 0) + (sc ? C::SC_BOX : 0));
             uint8_t* raw = sm + C::OFF_RAW + rs * C::RAW_BYTES;
             const int tr = t0 + s * C::RT;
             tma_load_5d(raw, &p.tm_B, &bar[RAW_FULL0 + rs], 0, 0, g, tr, b);
-            tma_load_5d(raw + C::BRAW_BYTES, &p.tm_C, &bar[RAW_FULL0 + rs], 0, 0, g, tr, b);
+            if (!MAP)
+                tma_load_5d(raw + C::BRAW_BYTES, &p.tm_C, &bar[RAW_FULL0 + rs], 0, 0, g, tr, b);
             tma_load_4d(raw + 2 * C::BRAW_BYTES, &p.tm_th, &bar[RAW_FULL0 + rs], 0, g, tr, b);
             if (sc)   // BCNorm scales of B and C for these tokens: x = token (RT-aligned)
                 tma_load_5d(raw + C::SC_OFF, &p.tm_sc, &bar[RAW_FULL0 + rs], tr, 0, g, b, 0);
@@ -916,7 +1047,8 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
 // x tiles and y stores, on their own warp so that neither a stage waiting for its y
 // store nor the store itself holds up the B / C / theta loads.  x(c) is loaded into
 // stage c % XST; once the epilogue has written y(c) over it (Y_STAGED), the tile is
-// stored, and when the store has read it the stage takes x(c + XST).
+// stored, and when the store has read it the stage takes x(c + XST).  In the segment pass
+// nothing is stored: Y_STAGED then says the rotation warps are done with x(c).
 //
 // MIMO lightweight expansion ("Multi-Input, Multi-Output (MIMO) Formulation", MIMO
 // Parameterization Choices): x (and z) then hold one value per head channel, and the
@@ -926,12 +1058,15 @@ __device__ void producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Ab
 // lane writes it, and the rows a batch writes, [t0 R, (t0 + k) R), lie below the raw row
 // (R - 1) Q + t0 + k of the first later token because (t0 + k)(R - 1) <= Q (R - 1).  The
 // stage is published on X_FULL once expanded.
-template <int NST, int Q, int R, bool GT, bool XE>
-__device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const Abort& ab) {
+template <int NST, int Q, int R, bool GT, bool XE, bool MAP>
+__device__ void x_producer(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* bar,
+                           const Abort& ab) {
     using C = Cfg<NST, Q, R, GT>;
     const ScanArgs& a = p.a;
     const int lane = threadIdx.x & 31;
-    const int b = blockIdx.x / a.H, h = blockIdx.x % a.H;
+    const int b = u.b, h = u.h;
+    // token coordinate of chunk c of the segment
+    auto tok = [&](int c) { return (int)(u.t0 + (long long)c * Q); };
     if constexpr (!XE) {   // lane 0 alone: every tile comes by TMA
         if (lane != 0) return;
         int n_x[C::XST] = {};
@@ -939,22 +1074,24 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
             const int xs = c % C::XST;
             mbar_arrive_expect_tx(&bar[X_FULL0 + xs], C::XZ_BYTES);
             tma_load_5d(sm + C::OFF_X + xs * C::X_BYTES, &p.tm_x, &bar[X_FULL0 + xs], 0, 0, h,
-                        c * Q, b);
+                        tok(c), b);
             if constexpr (GT)
                 tma_load_5d(sm + C::OFF_Z + xs * C::X_BYTES, &p.tm_z, &bar[X_FULL0 + xs], 0, 0, h,
-                            c * Q, b);
+                            tok(c), b);
             ++n_x[xs];
         };
-        for (int c = 0; c < C::XST && c < p.nchunks; ++c) load(c);
+        for (int c = 0; c < C::XST && c < u.nch; ++c) load(c);
         bool ok = true;
-        for (int c = 0; c < p.nchunks; ++c) {
+        for (int c = 0; c < u.nch; ++c) {
             if (!(ok = mbar_wait(&bar[Y_STAGED0 + c % C::XST], (c / C::XST) & 1, ab))) break;
             const int xs = c % C::XST;
-            tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, c * Q, b);
-            bulk_commit();
+            if constexpr (!MAP) {
+                tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, tok(c), b);
+                bulk_commit();
+            }
             mbar_arrive(&bar[COEF_EMPTY0 + c % kCoefSlots]);
-            bulk_wait_read<0>();
-            if (c + C::XST < p.nchunks) load(c + C::XST);
+            if constexpr (!MAP) bulk_wait_read<0>();
+            if (c + C::XST < u.nch) load(c + C::XST);
         }
         if (!ok)
             for (int s = 0; s < C::XST; ++s)
@@ -1016,14 +1153,14 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
             const int bytes = (xe ? Q * 128 : C::X_BYTES) + (GT ? (ze ? Q * 128 : C::X_BYTES) : 0);
             mbar_arrive_expect_tx(&bar[XR_FULL], bytes);
             if (xe)
-                tma_load_4d(xt + (R - 1) * Q * 128, &p.tm_xr, &bar[XR_FULL], 0, h, c * Q, b);
+                tma_load_4d(xt + (R - 1) * Q * 128, &p.tm_xr, &bar[XR_FULL], 0, h, tok(c), b);
             else
-                tma_load_5d(xt, &p.tm_x, &bar[XR_FULL], 0, 0, h, c * Q, b);
+                tma_load_5d(xt, &p.tm_x, &bar[XR_FULL], 0, 0, h, tok(c), b);
             if constexpr (GT) {
                 if (ze)
-                    tma_load_4d(zt + (R - 1) * Q * 128, &p.tm_zr, &bar[XR_FULL], 0, h, c * Q, b);
+                    tma_load_4d(zt + (R - 1) * Q * 128, &p.tm_zr, &bar[XR_FULL], 0, h, tok(c), b);
                 else
-                    tma_load_5d(zt, &p.tm_z, &bar[XR_FULL], 0, 0, h, c * Q, b);
+                    tma_load_5d(zt, &p.tm_z, &bar[XR_FULL], 0, 0, h, tok(c), b);
             }
         }
         pending = true;
@@ -1037,18 +1174,20 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
         return true;
     };
     bool ok = true;
-    for (int c = 0; c < C::XST && c < p.nchunks && ok; ++c) ok = load(c);
-    for (int c = 0; c < p.nchunks && ok; ++c) {
+    for (int c = 0; c < C::XST && c < u.nch && ok; ++c) ok = load(c);
+    for (int c = 0; c < u.nch && ok; ++c) {
         if (!(ok = warp_wait(&bar[Y_STAGED0 + c % C::XST], (c / C::XST) & 1, ab))) break;
         const int xs = c % C::XST;
         if (lane == 0) {
-            tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, c * Q, b);
-            bulk_commit();
+            if constexpr (!MAP) {
+                tma_store_5d(&p.tm_y, sm + C::OFF_X + xs * C::X_BYTES, 0, 0, h, tok(c), b);
+                bulk_commit();
+            }
             mbar_arrive(&bar[COEF_EMPTY0 + c % kCoefSlots]);
-            bulk_wait_read<0>();
+            if constexpr (!MAP) bulk_wait_read<0>();
         }
         __syncwarp();
-        if (c + C::XST < p.nchunks) ok = load(c + C::XST);
+        if (c + C::XST < u.nch) ok = load(c + C::XST);
     }
     if (lane == 0) {
         if (pending) drain_wait(&bar[XR_FULL], (n_xr - 1) & 1, 10000000ull);
@@ -1057,9 +1196,11 @@ __device__ void x_producer(const TcParams& p, uint8_t* sm, uint64_t* bar, const 
     }
 }
 
-template <int NST, int Q, int R, bool GT, bool BC, bool XE>
+// MAP: the segment pass of a segmented call (no C~, S, Y or y; see Unit and state).
+template <int NST, int Q, int R, bool GT, bool BC, bool XE, bool MAP>
 __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_constant__ TcParams p) {
     using C = Cfg<NST, Q, R, GT>;
+    const Unit u = unit_of<Q, MAP>(p);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base for the SW128 tiles, as an offset from smem_raw so that the
     // compiler keeps every access in the shared address space
@@ -1075,7 +1216,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         tma_prefetch_desc(XE && p.a.x_expand ? &p.tm_xr : &p.tm_x);
         if (GT) tma_prefetch_desc(XE && p.a.z_expand ? &p.tm_zr : &p.tm_z);
         tma_prefetch_desc(&p.tm_B);
-        tma_prefetch_desc(&p.tm_C);
+        if (!MAP) tma_prefetch_desc(&p.tm_C);
         tma_prefetch_desc(&p.tm_th);
         tma_prefetch_desc(&p.tm_dt);
     }
@@ -1090,24 +1231,24 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.a.status, p.limit_ns};
 
     if (w == 0) {
-        if ((threadIdx.x & 31) == 0) producer<NST, Q, R, GT, BC>(p, sm, bar, ab);
+        if ((threadIdx.x & 31) == 0) producer<NST, Q, R, GT, BC, MAP>(p, u, sm, bar, ab);
     } else if (w == 1) {
         if ((threadIdx.x & 31) == 0) {
-            mma_issuer<NST, Q, R, GT>(p, sm, bar, tmem, ab);
+            mma_issuer<NST, Q, R, GT, MAP>(p, u, sm, bar, tmem, ab);
             // no MMA may still be writing TMEM when it is released
             mma_commit(&bar[DRAIN]);
             drain_wait(&bar[DRAIN], 0, 100000000ull);
         }
     } else if (w < 6) {
-        epilogue<NST, Q, R, GT>(p, sm, bar, tmem, ab);
+        if constexpr (!MAP) epilogue<NST, Q, R, GT>(p, u, sm, bar, tmem, ab);
     } else if (w >= 16) {
-        state<NST, Q, R, GT, BC, XE>(p, sm, bar, tmem, ab);
+        state<NST, Q, R, GT, BC, XE, MAP>(p, u, sm, bar, tmem, ab);
     } else if (w < 6 + kRotWarps) {
-        rotation<NST, Q, R, GT, BC>(p, sm, bar, ab);
+        rotation<NST, Q, R, GT, BC, MAP>(p, u, sm, bar, ab);
     } else if (w == 6 + kRotWarps) {
-        coefficients<NST, Q, R, GT>(p, sm, bar, ab);
+        coefficients<NST, Q, R, GT>(p, u, sm, bar, ab);
     } else if (XE || (threadIdx.x & 31) == 0) {
-        x_producer<NST, Q, R, GT, XE>(p, sm, bar, ab);
+        x_producer<NST, Q, R, GT, XE, MAP>(p, u, sm, bar, ab);
     }
     tc_fence_before();
     __syncthreads();
@@ -1115,6 +1256,36 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Chain step between the segment pass and the output pass of a segmented call: the state
+// entering segment s + 1 is dec_s R(psi_s) h_in(s) + M_s (M_0 already holds h0), and the
+// output pass starts segment s from G0_s + h_in(s).  One thread per (batch * head, state
+// pair, column), sequential over the segments.
+__global__ void seg_chain_kernel(float* seg, int BH, int S, int N, int P) {
+    const size_t rec = seg_rec_floats(N, P);
+    const int per = (N / 2) * P;
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long long)BH * per) return;
+    const int bh = (int)(idx / per), rem = (int)(idx % per), i = rem / P, col = rem % P;
+    const size_t e0 = (size_t)(2 * i) * P + col, e1 = e0 + P;
+    const float* r0 = seg + (size_t)bh * rec;
+    float he = r0[e0], ho = r0[e1];   // the state entering segment 1
+    for (int s = 1; s < S; ++s) {
+        float* r = seg + ((size_t)s * BH + bh) * rec;
+        float* g0 = r + seg_off_g0(N, P);
+        g0[e0] += he;
+        g0[e1] += ho;
+        if (s + 1 < S) {
+            const float dec = r[seg_off_dec(N, P)];
+            float sn, cn;
+            sincosf(r[seg_off_psi(N, P) + i], &sn, &cn);
+            const float ne = fmaf(dec, fmaf(cn, he, -sn * ho), r[e0]);
+            const float no = fmaf(dec, fmaf(sn, he, cn * ho), r[e1]);
+            he = ne;
+            ho = no;
+        }
     }
 }
 
@@ -1153,13 +1324,23 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ptr,
     return r == CUDA_SUCCESS;
 }
 
+template <int NST, int Q, int R, bool GT, bool BC, bool XE, bool MAP>
+cudaError_t launch_k(const TcParams& p, unsigned grid, cudaStream_t s) {
+    using C = Cfg<NST, Q, R, GT>;
+    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R, GT, BC, XE, MAP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    scan_tc_kernel<NST, Q, R, GT, BC, XE, MAP><<<grid, kThreads, C::SMEM, s>>>(p);
+    return cudaGetLastError();
+}
+
 template <int NST, int Q, int R, bool GT, bool BC, bool XE>
 cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
     using C = Cfg<NST, Q, R, GT>;
     TcParams p;
     std::memset(&p, 0, sizeof(p));
     p.a = a;
-    p.nchunks = (int)((a.T + Q - 1) / Q);
+    p.nch_total = (int)((a.T + Q - 1) / Q);
     p.limit_ns = (a.flags & M3_FLAG_TEST_STALL) ? 50000000ull : 2000000000ull;
     const uint64_t T = a.T, Bn = a.batch, H = a.H, G = a.G;
     bool ok = true;
@@ -1227,11 +1408,22 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<NST, Q, R, GT, BC, XE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    scan_tc_kernel<NST, Q, R, GT, BC, XE><<<(unsigned)(a.batch * a.H), kThreads, C::SMEM, s>>>(p);
-    return cudaGetLastError();
+    // Sequence segments: when the workspace holds their records, the call runs as the
+    // segment pass, the chain step and the output pass.
+    const int BH = a.batch * a.H;
+    int S = scan_tc_segments(BH, p.nch_total);
+    const size_t seg_bytes = (size_t)BH * S * seg_rec_floats(NST, kP) * sizeof(float);
+    if (S > 1 && (!a.ws || a.ws_bytes < seg_bytes)) S = 1;
+    p.S = S;
+    p.seg = S > 1 ? static_cast<float*>(a.ws) : nullptr;
+    if (S > 1) {
+        cudaError_t e = launch_k<NST, Q, R, false, BC, XE, true>(p, (unsigned)(BH * S), s);
+        if (e != cudaSuccess) return e;
+        const long long n = (long long)BH * (NST / 2) * kP;
+        seg_chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p.seg, BH, S, NST, kP);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return launch_k<NST, Q, R, GT, BC, XE, false>(p, (unsigned)(BH * S), s);
 }
 
 }  // namespace
@@ -1240,24 +1432,55 @@ cudaError_t launch_t(const ScanArgs& a, cudaStream_t s) {
 // The tile holds L = chunk * R (token, rank) rows with L in {64, 128}: the M = 64 / 128
 // MMA shapes, and the S and Y accumulators that fit TMEM.  A requested chunk whose L
 // falls outside is run with the nearest tile (L clamped into [64, 128]): the chunked form
-// is exact for any blocking, so only rounding changes.  Returns 0 where no tile applies.
+// is exact for any blocking, so only rounding changes.  With N = 128 a 128-row tile
+// leaves shared memory for a single operand slot, which serialises the rotation warps
+// and the MMAs; chunk 128 then runs as 64-token tiles.  Returns 0 where no tile applies.
 int scan_tc_chunk(int N, int P, int R, int chunk, int H) {
     if (P != kP || H % 4 != 0) return 0;
     if (R != 1 && R != 2 && R != 4) return 0;
     if (N != 64 && (N != 128 || R != 1)) return 0;
     int L = chunk * R;
     L = L < 64 ? 64 : (L > 128 ? 128 : L);
+    if (N == 128) L = 64;
     return L / R;
 }
 
-size_t scan_tc_workspace_bytes(int, int, int, int, int, long long, int) { return 0; }
+// Segments per (batch, head) for a call of nch chunks over BH (batch * head) streams: one
+// stream per SM of the current device, at least two chunks per segment, at most 16
+// segments.  A segment pass chunk costs about 0.8 of an output pass chunk (measured on
+// B200: 63 us for 32 chunks against 77 us), so two segments (1.8 / 2 of the time, before
+// the chain step and the extra launches) do not pay: fewer than three means 1 (none).
+int scan_tc_segments(int BH, long long nch) {
+    // SM count per device, looked up once (the launch path calls this for every call)
+    static int sms_of[64] = {};
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+        if (!sms_of[dev]) {
+            int n = 0;
+            if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+                n > 0)
+                sms_of[dev] = n;
+        }
+        if (sms_of[dev]) sms = sms_of[dev];
+    }
+    long long S = BH > 0 ? sms / BH : 1;
+    if (S > nch / 2) S = nch / 2;
+    if (S > 16) S = 16;
+    return S < 3 ? 1 : (int)S;
+}
+
+// The segment records of a call that would be segmented (see scan_tc_segments); 0 otherwise.
+size_t scan_tc_workspace_bytes(int batch, int H, int N, int P, int, long long T, int chunk) {
+    const long long nch = (T + chunk - 1) / chunk;
+    const int S = scan_tc_segments(batch * H, nch);
+    return S > 1 ? (size_t)batch * H * S * seg_rec_floats(N, P) * sizeof(float) : 0;
+}
 
 template <bool GT, bool BC, bool XE>
 cudaError_t launch_scan_tc_g(const ScanArgs& a, int R, cudaStream_t s) {
     const int N = a.N, Q = a.chunk;   // the tile chunk chosen by scan_tc_chunk
     if (R == 1) {
         if (N == 128 && Q == 64) return launch_t<128, 64, 1, GT, BC, XE>(a, s);
-        if (N == 128 && Q == 128) return launch_t<128, 128, 1, GT, BC, XE>(a, s);
         if (N == 64 && Q == 64) return launch_t<64, 64, 1, GT, BC, XE>(a, s);
         if (N == 64 && Q == 128) return launch_t<64, 128, 1, GT, BC, XE>(a, s);
     } else if (R == 2 && N == 64) {

@@ -72,7 +72,7 @@ struct Abort {
 // The poll itself may suspend the thread (hint 20 us); the abort flag and the clock are
 // looked at only every 64 polls, so that waiting warps spend few issue slots.  The wait
 // stays bounded: at most 64 suspended polls pass between two looks at the clock.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const Abort& ab) {
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const Abort& ab) {
     const uint64_t t0 = globaltimer();
     const uint64_t limit = ab.limit_ns;
     volatile uint32_t* flag = ab.flag;

@@ -119,6 +119,7 @@ def test_bc_call_split(chunk):
     ((4, 8, 2, 64, 64, 4), torch.bfloat16, 2e-2, "norm+bias+gate"),
     ((2, 6, 3, 8, 6, 3), torch.float32, 1e-5, "norm+bias+gate"),
     ((2, 4, 1, 16, 16, 2), torch.float32, 1e-5, "bias"),
+    ((2, 4, 2, 64, 64, 2), torch.float32, 1e-5, "norm+bias+gate"),
 ])
 def test_bc_decode_matches_oracle(shape, io, tol, parts):
     b, H, G, P, N, R = shape

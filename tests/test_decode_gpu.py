@@ -50,6 +50,11 @@ def oracle_decode(inp, steps, bsel=slice(None), hsel=slice(None)):
     ((3, 4, 4, 16, 16, 2), torch.float32, 1e-5),
     ((2, 4, 1, 32, 256, 1), torch.float32, 1e-5),
     ((2, 6, 3, 8, 6, 3), torch.float32, 1e-5),
+    # P = 64 at several batch / group / rank mixes, fp32 and bf16 io
+    ((40, 8, 8, 64, 64, 2), torch.bfloat16, 2e-2),
+    ((3, 4, 2, 64, 128, 1), torch.float32, 1e-5),
+    ((2, 4, 1, 64, 128, 2), torch.bfloat16, 2e-2),
+    ((5, 6, 3, 64, 64, 4), torch.float32, 1e-5),
 ])
 def test_decode_steps(shape, io, tol):
     b, H, G, P, N, R = shape

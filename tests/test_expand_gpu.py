@@ -130,6 +130,7 @@ def test_expanded_scan_chained_calls():
     ((4, 8, 1, 64, 128, 1), torch.bfloat16, 2e-2),
     ((4, 8, 2, 64, 64, 4), torch.bfloat16, 2e-2),
     ((2, 6, 3, 8, 6, 3), torch.float32, 1e-5),
+    ((3, 4, 2, 64, 64, 2), torch.float32, 1e-5),
 ])
 def test_expanded_decode_matches_oracle(shape, io, tol):
     b, H, G, P, N, R = shape
