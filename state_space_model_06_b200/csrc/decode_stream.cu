@@ -1,0 +1,303 @@
+// decode_stream.cu -- MIMO decode step (N = 64, P = 64, rank 2 or 4) as a persistent
+// streaming kernel.
+//
+// Mamba-3 paper summary, "Multi-Input, Multi-Output Formulation": at decode time each
+// head's N x P fp32 state is read and written once per token, so the step is bound by
+// HBM.  With one CTA per head, each CTA's 16 KB state is loaded into registers, updated
+// and stored, and an SM only has the loads of its resident CTAs in flight while they
+// compute: a copy-only version of that shape stops at about two thirds of HBM.
+//
+// Here each warp owns a stream of heads (bh = global warp, + number of warps, ...): the
+// 16 KB state arrives in shared memory by one bulk copy into the warp's slot, the per-head
+// factors are built by the warp itself (one lane per state pair) while the copy flies,
+// and the warp needs no CTA-wide barrier.  Eight warps per SM, two on each sub-partition:
+// while one waits for its copy the other updates its head.  (Measured on B200 for the
+// batch-256 rank-4 step: 8 warps x 1 slot 102.6 us, 6 x 1 117, 4 x 2 127, 4 x 3 131, 5 x 2
+// 133: the heads are dealt to the warps statically, so every sub-partition must carry the
+// same number of warps.)  The update is the one of the per-head kernels:
+//   h' = R(phi)(alpha h) + [beta R(phi) Bp | gamma B] [xp | x]^T,
+//   Y  = h'^T C + D x  (times SiLU(z) with the output gate),
+// on packed fp32 pairs, with the new state written from registers straight to HBM.
+// Lane (j, half) holds column chunk j (4 columns) and the state pairs half*16 .. +15.
+#include "m3_internal.h"
+#include "sm100.cuh"
+
+namespace m3 {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kSW = 8;                           // warps per CTA (one CTA per SM)
+constexpr int kSlots = 1;                        // state slots per warp (heads in flight)
+constexpr int kNP = 32;                          // state pairs (N = 64)
+constexpr int kPc = 64;                          // columns (P = 64)
+constexpr int kStateBytes = 2 * kNP * kPc * 4;   // 16 KB per head
+
+template <int R>
+struct SCfg {
+    static constexpr int FAC_F4 = kNP * (2 + 3 * R);   // rot [2], U [2R], C [R] per pair
+    static constexpr int WARP_BYTES = kSlots * kStateBytes + FAC_F4 * 16;
+    static constexpr int SMEM = kSW * WARP_BYTES + kSW * kSlots * 8 + 128;   // + barriers, align
+    static_assert(SMEM <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z, v.w); }
+
+// four consecutive io values as floats
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    return make_float4(bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y));
+}
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+}
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+// the two values of a state pair (rows 2i, 2i+1) of one rank column
+__device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    return make_float2(bf16lo(u), bf16hi(u));
+}
+__device__ __forceinline__ float2 load2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+
+// The small per-head inputs, fetched one head ahead into registers.
+template <typename IO, int R>
+struct Small {
+    float dt, A, lam, th, D;
+    float2 bq[R], bp[R], cc[R];   // this lane's pair (rows 2 lane, 2 lane + 1) of B, B_prev, C
+    float4 x[R], xp[R], z[R];     // this lane's column chunk of x, x_prev, z
+    __device__ void load(const DecodeArgs& a, int bh, int lane) {
+        const int H = a.H, G = a.G, N = a.N, P = a.P;
+        const int b = bh / H, h = bh - b * H, g = h / (H / G);
+        const int j = lane & 15;
+        dt = a.dt[bh];
+        A = a.A[bh];
+        lam = a.lam[bh];
+        D = a.D ? a.D[h] : 0.f;
+        th = a.theta[((size_t)b * G + g) * (N / 2) + lane];
+        const size_t gofs = ((size_t)b * G + g) * R * N + 2 * lane;
+        const IO* Bg = static_cast<const IO*>(a.B) + gofs;
+        const IO* Bpg = static_cast<const IO*>(a.B_prev) + gofs;
+        const IO* Cg = static_cast<const IO*>(a.C) + gofs;
+        const size_t xofs = (size_t)bh * R * P + 4 * j;
+        const IO* x0 = static_cast<const IO*>(a.x) + xofs;
+        const IO* xp0 = static_cast<const IO*>(a.x_prev) + xofs;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            bq[r] = load2(Bg + r * N);
+            bp[r] = load2(Bpg + r * N);
+            cc[r] = load2(Cg + r * N);
+            x[r] = load4(x0 + r * P);
+            xp[r] = load4(xp0 + r * P);
+            z[r] = a.z ? load4(static_cast<const IO*>(a.z) + xofs + r * P)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+};
+
+template <typename IO, int R>
+__global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeArgs a, int nbh) {
+    using C = SCfg<R>;
+    constexpr int R2 = 2 * R;
+    extern __shared__ __align__(128) uint8_t sm_raw[];
+    uint8_t* smb = sm_raw + ((128u - (smem_u32(sm_raw) & 127u)) & 127u);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = lane & 15, half = lane >> 4;
+    uint8_t* wb = smb + w * C::WARP_BYTES;
+    const float* slot0 = reinterpret_cast<const float*>(wb);
+    float4* rot4 = reinterpret_cast<float4*>(wb + kSlots * kStateBytes);   // [32][2]
+    float4* U4 = rot4 + kNP * 2;                                       // [32][2R]
+    float4* C4 = U4 + kNP * R2;                                        // [32][R]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smb + kSW * C::WARP_BYTES) + kSlots * w;
+    if (lane == 0) {
+        for (int s = 0; s < kSlots; ++s) mbar_init(&bar[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    const int gw = blockIdx.x * kSW + w, NW = gridDim.x * kSW;
+    const int nmine = gw < nbh ? (nbh - gw + NW - 1) / NW : 0;
+    auto issue = [&](int i) {   // lane 0: the state of this warp's i-th head into its slot
+        const int s = i % kSlots;
+        mbar_arrive_expect_tx(&bar[s], kStateBytes);
+        bulk_load(wb + s * kStateBytes, a.h + (size_t)(gw + i * NW) * 2 * kNP * kPc, kStateBytes,
+                  &bar[s]);
+    };
+    if (lane == 0)
+        for (int i = 0; i < kSlots && i < nmine; ++i) issue(i);
+    Small<IO, R> nx;
+    if (nmine > 0) nx.load(a, gw, lane);
+    const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
+    int issued = nmine < kSlots ? nmine : kSlots;   // copies issued
+    bool ok = true;
+
+    for (int i = 0; i < nmine && ok; ++i) {
+        const int bh = gw + i * NW;
+        const Small<IO, R> cur = nx;
+        // ---- this head's factors: lane = state pair
+        {
+            const float alpha = expf(cur.dt * cur.A);
+            const float beta = (1.f - cur.lam) * cur.dt * alpha;
+            const float gamma = cur.lam * cur.dt;
+            float sn, cs;
+            sincosf(angle ? cur.th : cur.dt * cur.th, &sn, &cs);
+            const float ac = alpha * cs, as = alpha * sn;
+            rot4[2 * lane] = make_float4(ac, ac, as, as);
+            rot4[2 * lane + 1] = make_float4(-as, -as, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float p0 = cur.bp[r].x, p1 = cur.bp[r].y;
+                const float ub0 = beta * (cs * p0 - sn * p1), ub1 = beta * (sn * p0 + cs * p1);
+                const float ug0 = gamma * cur.bq[r].x, ug1 = gamma * cur.bq[r].y;
+                U4[lane * R2 + r] = make_float4(ub0, ub0, ub1, ub1);
+                U4[lane * R2 + R + r] = make_float4(ug0, ug0, ug1, ug1);
+                C4[lane * R + r] = make_float4(cur.cc[r].x, cur.cc[r].x, cur.cc[r].y, cur.cc[r].y);
+            }
+        }
+        __syncwarp();
+        // the next head's small inputs fly while this one is updated
+        if (i + 1 < nmine) nx.load(a, bh + NW, lane);
+
+        // ---- wait for this head's state (bounded)
+        const int s = i % kSlots;
+        const uint32_t par = (i / kSlots) & 1;
+        {
+            const uint64_t t0 = globaltimer();
+            bool got = mbar_try_wait(&bar[s], par);
+            while (!got && globaltimer() - t0 < 2000000000ull)
+                got = mbar_try_wait_hint(&bar[s], par, 20000u);
+            ok = __all_sync(0xffffffffu, got);
+        }
+        float2 ya[R], yb[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) ya[r] = yb[r] = make_float2(0.f, 0.f);
+        if (ok) {
+            const float* st = slot0 + s * (kStateBytes / 4);
+            float4* hrow = reinterpret_cast<float4*>(a.h + (size_t)bh * 2 * kNP * kPc);
+#pragma unroll 2
+            for (int kk = 0; kk < kNP / 2; ++kk) {
+                const int ip = half * (kNP / 2) + kk;
+                const float4 h0 = *reinterpret_cast<const float4*>(st + (2 * ip) * kPc + 4 * j);
+                const float4 h1 = *reinterpret_cast<const float4*>(st + (2 * ip + 1) * kPc + 4 * j);
+                const float4 rc = rot4[2 * ip], rn = rot4[2 * ip + 1];
+                // row 2i: ac h0 - as h1;  row 2i+1: as h0 + ac h1
+                float2 n0a = __ffma2_rn(lo2(rc), lo2(h0), __fmul2_rn(lo2(rn), lo2(h1)));
+                float2 n0b = __ffma2_rn(lo2(rc), hi2(h0), __fmul2_rn(lo2(rn), hi2(h1)));
+                float2 n1a = __ffma2_rn(hi2(rc), lo2(h0), __fmul2_rn(lo2(rc), lo2(h1)));
+                float2 n1b = __ffma2_rn(hi2(rc), hi2(h0), __fmul2_rn(lo2(rc), hi2(h1)));
+#pragma unroll
+                for (int q = 0; q < R2; ++q) {
+                    const float4 u = U4[ip * R2 + q];
+                    const float4 v = q < R ? cur.xp[q] : cur.x[q - R];
+                    n0a = __ffma2_rn(lo2(u), lo2(v), n0a);
+                    n0b = __ffma2_rn(lo2(u), hi2(v), n0b);
+                    n1a = __ffma2_rn(hi2(u), lo2(v), n1a);
+                    n1b = __ffma2_rn(hi2(u), hi2(v), n1b);
+                }
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float4 c = C4[ip * R + r];
+                    ya[r] = __ffma2_rn(n0a, lo2(c), __ffma2_rn(n1a, hi2(c), ya[r]));
+                    yb[r] = __ffma2_rn(n0b, lo2(c), __ffma2_rn(n1b, hi2(c), yb[r]));
+                }
+                __stcs(hrow + (size_t)(2 * ip) * (kPc / 4) + j, make_float4(n0a.x, n0a.y, n0b.x, n0b.y));
+                __stcs(hrow + (size_t)(2 * ip + 1) * (kPc / 4) + j,
+                       make_float4(n1a.x, n1a.y, n1b.x, n1b.y));
+            }
+        }
+        // ---- readout: the two halves' partial sums over the state rows
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            ya[r].x += __shfl_xor_sync(0xffffffffu, ya[r].x, 16);
+            ya[r].y += __shfl_xor_sync(0xffffffffu, ya[r].y, 16);
+            yb[r].x += __shfl_xor_sync(0xffffffffu, yb[r].x, 16);
+            yb[r].y += __shfl_xor_sync(0xffffffffu, yb[r].y, 16);
+        }
+        if (half == 0) {
+            IO* y = static_cast<IO*>(a.y) + (size_t)bh * R * kPc + 4 * j;
+            IO* xpo = static_cast<IO*>(a.x_prev) + (size_t)bh * R * kPc + 4 * j;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float4 v = make_float4(ya[r].x, ya[r].y, yb[r].x, yb[r].y);
+                if (!ok) v = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                         __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+                v.x = fmaf(cur.D, cur.x[r].x, v.x);
+                v.y = fmaf(cur.D, cur.x[r].y, v.y);
+                v.z = fmaf(cur.D, cur.x[r].z, v.z);
+                v.w = fmaf(cur.D, cur.x[r].w, v.w);
+                if (a.z) {
+                    v.x = gate_silu(v.x, cur.z[r].x);
+                    v.y = gate_silu(v.y, cur.z[r].y);
+                    v.z = gate_silu(v.z, cur.z[r].z);
+                    v.w = gate_silu(v.w, cur.z[r].w);
+                }
+                store4(y + r * kPc, v);
+                store4(xpo + r * kPc, cur.x[r]);   // x_prev <- x (exact in the io dtype)
+            }
+        }
+        // the slot is free once every lane has read it: the copy of head i + kSlots goes there
+        __syncwarp();
+        fence_proxy_async_smem();
+        if (ok && lane == 0 && i + kSlots < nmine) {
+            issue(i + kSlots);
+            ++issued;
+        }
+    }
+    if (!ok && lane == 0) {
+        // a copy did not land in time (this head's y is NaN): let the copies issued into
+        // each slot land (bounded) before the CTA's shared memory is released
+        for (int s = 0; s < kSlots; ++s) {
+            const int n = (issued - s + kSlots - 1) / kSlots;   // copies issued into slot s
+            if (n == 0) continue;
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&bar[s], (n - 1) & 1) && globaltimer() - t0 < 10000000ull) {
+            }
+        }
+    }
+}
+
+int num_sms() {
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!sms[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+            sms[dev] = n;
+    }
+    return sms[dev] ? sms[dev] : 148;
+}
+
+template <typename IO, int R>
+cudaError_t launch_stream_t(const DecodeArgs& a, int batch, cudaStream_t s) {
+    using C = SCfg<R>;
+    cudaError_t e = cudaFuncSetAttribute(decode_mimo_stream_kernel<IO, R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    const int nbh = batch * a.H;
+    int grid = num_sms();
+    const int need = (nbh + kSW - 1) / kSW;
+    if (grid > need) grid = need;
+    decode_mimo_stream_kernel<IO, R><<<grid, kSW * 32, C::SMEM, s>>>(a, nbh);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_stream_ok(const DecodeArgs& a, int R) {
+    const bool bcm = a.B_bias || a.C_bias || a.bc_eps > 0.f;
+    return a.N == 2 * kNP && a.P == kPc && (R == 2 || R == 4) && !bcm && !a.x_expand &&
+           !a.z_expand;
+}
+
+cudaError_t launch_decode_stream(const DecodeArgs& a, int batch, int R, int io_dtype,
+                                 cudaStream_t s) {
+    if (io_dtype == M3_BF16)
+        return R == 2 ? launch_stream_t<__nv_bfloat16, 2>(a, batch, s)
+                      : launch_stream_t<__nv_bfloat16, 4>(a, batch, s);
+    return R == 2 ? launch_stream_t<float, 2>(a, batch, s) : launch_stream_t<float, 4>(a, batch, s);
+}
+
+}  // namespace m3

@@ -329,7 +329,9 @@ m3_status decode_impl(const m3_dims* d, const void* x, const void* B, const void
     a.z_expand = ex ? ex->z_expand : nullptr;
     a.H = d->nheads; a.G = d->ngroups; a.P = d->headdim; a.N = d->dstate;
     a.ppt = ppt; a.flags = flags;
-    cudaError_t e = launch_decode(a, d->batch, d->rank, d->io_dtype, s);
+    cudaError_t e = decode_stream_ok(a, d->rank)
+                        ? launch_decode_stream(a, d->batch, d->rank, d->io_dtype, s)
+                        : launch_decode(a, d->batch, d->rank, d->io_dtype, s);
     if (e != cudaSuccess) return launch_status(e);
     const size_t row = io_bytes(d->io_dtype) * (size_t)d->ngroups * d->rank * d->dstate;
     e = launch_copy_prev(state->B_prev, B, 1, 0, d->batch, row, s);
