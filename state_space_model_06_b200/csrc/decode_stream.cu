@@ -1,5 +1,5 @@
-// decode_stream.cu -- MIMO decode step (N = 64, P = 64, rank 2 or 4) as a persistent
-// streaming kernel.
+// decode_stream.cu -- MIMO decode step (N = 64, P = 64, rank 2 or 4; the output gate, the
+// BC map and the lightweight expansion fused) as a persistent streaming kernel.
 //
 // Mamba-3 paper summary, "Multi-Input, Multi-Output Formulation": at decode time each
 // head's N x P fp32 state is read and written once per token, so the step is bound by
@@ -62,12 +62,23 @@ __device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
 }
 __device__ __forceinline__ float2 load2(const float* p) { return *reinterpret_cast<const float2*>(p); }
 
+// v * w rounded to the io dtype, four channels (the MIMO lightweight expansion)
+template <typename IO>
+__device__ __forceinline__ float4 expand4(float4 v, float4 w) {
+    return make_float4(expand_io<IO>(v.x, w.x), expand_io<IO>(v.y, w.y), expand_io<IO>(v.z, w.z),
+                       expand_io<IO>(v.w, w.w));
+}
+
 // The small per-head inputs, fetched one head ahead into registers.
-template <typename IO, int R>
+// XE: x (and z with z_expand) hold one value per head channel, [b][H][P], and rank column r
+// is that value times the head's weight w[r][p], rounded to the io dtype ("Multi-Input,
+// Multi-Output (MIMO) Formulation", MIMO Parameterization Choices).
+template <typename IO, int R, bool BCM, bool XE>
 struct Small {
     float dt, A, lam, th, D;
     float2 bq[R], bp[R], cc[R];   // this lane's pair (rows 2 lane, 2 lane + 1) of B, B_prev, C
-    float4 x[R], xp[R], z[R];     // this lane's column chunk of x, x_prev, z
+    float2 biasB, biasC;          // the head's BC biases of this lane's pair (BC map)
+    float4 x[R], xp[R], z[R];     // this lane's column chunk of x, x_prev, z (rank columns)
     __device__ void load(const DecodeArgs& a, int bh, int lane) {
         const int H = a.H, G = a.G, N = a.N, P = a.P;
         const int b = bh / H, h = bh - b * H, g = h / (H / G);
@@ -81,23 +92,42 @@ struct Small {
         const IO* Bg = static_cast<const IO*>(a.B) + gofs;
         const IO* Bpg = static_cast<const IO*>(a.B_prev) + gofs;
         const IO* Cg = static_cast<const IO*>(a.C) + gofs;
+        if constexpr (BCM) {
+            biasB = a.B_bias ? load2(a.B_bias + (size_t)h * N + 2 * lane) : make_float2(0.f, 0.f);
+            biasC = a.C_bias ? load2(a.C_bias + (size_t)h * N + 2 * lane) : make_float2(0.f, 0.f);
+        }
         const size_t xofs = (size_t)bh * R * P + 4 * j;
-        const IO* x0 = static_cast<const IO*>(a.x) + xofs;
         const IO* xp0 = static_cast<const IO*>(a.x_prev) + xofs;
+        const bool xe = XE && a.x_expand, ze = XE && a.z_expand;
+        float4 x1 = make_float4(0.f, 0.f, 0.f, 0.f), z1 = x1;
+        if (xe) x1 = load4(static_cast<const IO*>(a.x) + (size_t)bh * P + 4 * j);
+        if (ze) z1 = load4(static_cast<const IO*>(a.z) + (size_t)bh * P + 4 * j);
+        const float* wx = xe ? a.x_expand + ((size_t)h * R) * P + 4 * j : nullptr;
+        const float* wz = ze ? a.z_expand + ((size_t)h * R) * P + 4 * j : nullptr;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             bq[r] = load2(Bg + r * N);
             bp[r] = load2(Bpg + r * N);
             cc[r] = load2(Cg + r * N);
-            x[r] = load4(x0 + r * P);
+            x[r] = xe ? expand4<IO>(x1, load4(wx + r * P))
+                      : load4(static_cast<const IO*>(a.x) + xofs + r * P);
             xp[r] = load4(xp0 + r * P);
-            z[r] = a.z ? load4(static_cast<const IO*>(a.z) + xofs + r * P)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (ze)
+                z[r] = expand4<IO>(z1, load4(wz + r * P));
+            else
+                z[r] = a.z ? load4(static_cast<const IO*>(a.z) + xofs + r * P)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
 };
 
-template <typename IO, int R>
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <typename IO, int R, bool BCM, bool XE>
 __global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeArgs a, int nbh) {
     using C = SCfg<R>;
     constexpr int R2 = 2 * R;
@@ -127,7 +157,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeA
     };
     if (lane == 0)
         for (int i = 0; i < kSlots && i < nmine; ++i) issue(i);
-    Small<IO, R> nx;
+    Small<IO, R, BCM, XE> nx;
     if (nmine > 0) nx.load(a, gw, lane);
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     int issued = nmine < kSlots ? nmine : kSlots;   // copies issued
@@ -135,7 +165,25 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeA
 
     for (int i = 0; i < nmine && ok; ++i) {
         const int bh = gw + i * NW;
-        const Small<IO, R> cur = nx;
+        Small<IO, R, BCM, XE> cur = nx;
+        if constexpr (BCM) {
+            // BC map ("Technical Approach", BCNorm and BC biases): each rank column of B,
+            // B_prev and C scaled to unit RMS over N (when bc_eps > 0; the lanes hold the
+            // column's N values as pairs), plus the head's channel bias
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float sq = 1.f, sp = 1.f, sc = 1.f;
+                if (a.bc_eps > 0.f) {
+                    const float invn = 1.f / (float)a.N;
+                    sq = rsqrtf(warp_sum(cur.bq[r].x * cur.bq[r].x + cur.bq[r].y * cur.bq[r].y) * invn + a.bc_eps);
+                    sp = rsqrtf(warp_sum(cur.bp[r].x * cur.bp[r].x + cur.bp[r].y * cur.bp[r].y) * invn + a.bc_eps);
+                    sc = rsqrtf(warp_sum(cur.cc[r].x * cur.cc[r].x + cur.cc[r].y * cur.cc[r].y) * invn + a.bc_eps);
+                }
+                cur.bq[r] = make_float2(fmaf(cur.bq[r].x, sq, cur.biasB.x), fmaf(cur.bq[r].y, sq, cur.biasB.y));
+                cur.bp[r] = make_float2(fmaf(cur.bp[r].x, sp, cur.biasB.x), fmaf(cur.bp[r].y, sp, cur.biasB.y));
+                cur.cc[r] = make_float2(fmaf(cur.cc[r].x, sc, cur.biasC.x), fmaf(cur.cc[r].y, sc, cur.biasC.y));
+            }
+        }
         // ---- this head's factors: lane = state pair
         {
             const float alpha = expf(cur.dt * cur.A);
@@ -270,34 +318,48 @@ int num_sms() {
     return sms[dev] ? sms[dev] : 148;
 }
 
-template <typename IO, int R>
+template <typename IO, int R, bool BCM, bool XE>
 cudaError_t launch_stream_t(const DecodeArgs& a, int batch, cudaStream_t s) {
     using C = SCfg<R>;
-    cudaError_t e = cudaFuncSetAttribute(decode_mimo_stream_kernel<IO, R>,
+    cudaError_t e = cudaFuncSetAttribute(decode_mimo_stream_kernel<IO, R, BCM, XE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const int nbh = batch * a.H;
     int grid = num_sms();
     const int need = (nbh + kSW - 1) / kSW;
     if (grid > need) grid = need;
-    decode_mimo_stream_kernel<IO, R><<<grid, kSW * 32, C::SMEM, s>>>(a, nbh);
+    decode_mimo_stream_kernel<IO, R, BCM, XE><<<grid, kSW * 32, C::SMEM, s>>>(a, nbh);
     return cudaGetLastError();
+}
+
+template <typename IO, bool BCM, bool XE>
+cudaError_t launch_stream_r(const DecodeArgs& a, int batch, int R, cudaStream_t s) {
+    return R == 2 ? launch_stream_t<IO, 2, BCM, XE>(a, batch, s)
+                  : launch_stream_t<IO, 4, BCM, XE>(a, batch, s);
+}
+
+template <typename IO>
+cudaError_t launch_stream_io(const DecodeArgs& a, int batch, int R, cudaStream_t s) {
+    const bool bcm = a.B_bias || a.C_bias || a.bc_eps > 0.f;
+    const bool xe = a.x_expand || a.z_expand;
+    if (bcm) return xe ? launch_stream_r<IO, true, true>(a, batch, R, s)
+                       : launch_stream_r<IO, true, false>(a, batch, R, s);
+    return xe ? launch_stream_r<IO, false, true>(a, batch, R, s)
+              : launch_stream_r<IO, false, false>(a, batch, R, s);
 }
 
 }  // namespace
 
 bool decode_stream_ok(const DecodeArgs& a, int R) {
-    const bool bcm = a.B_bias || a.C_bias || a.bc_eps > 0.f;
-    return a.N == 2 * kNP && a.P == kPc && (R == 2 || R == 4) && !bcm && !a.x_expand &&
-           !a.z_expand;
+    return a.N == 2 * kNP && a.P == kPc && (R == 2 || R == 4);
 }
 
+// The BC map and the lightweight expansion are compile-time variants, so the plain
+// instantiations hold none of their code.
 cudaError_t launch_decode_stream(const DecodeArgs& a, int batch, int R, int io_dtype,
                                  cudaStream_t s) {
-    if (io_dtype == M3_BF16)
-        return R == 2 ? launch_stream_t<__nv_bfloat16, 2>(a, batch, s)
-                      : launch_stream_t<__nv_bfloat16, 4>(a, batch, s);
-    return R == 2 ? launch_stream_t<float, 2>(a, batch, s) : launch_stream_t<float, 4>(a, batch, s);
+    return io_dtype == M3_BF16 ? launch_stream_io<__nv_bfloat16>(a, batch, R, s)
+                               : launch_stream_io<float>(a, batch, R, s);
 }
 
 }  // namespace m3
