@@ -10,11 +10,12 @@
 // Here each warp owns a stream of heads (bh = global warp, + number of warps, ...): the
 // 16 KB state arrives in shared memory by one bulk copy into the warp's slot, the per-head
 // factors are built by the warp itself (one lane per state pair) while the copy flies,
-// and the warp needs no CTA-wide barrier.  Eight warps per SM, two on each sub-partition:
-// while one waits for its copy the other updates its head.  (Measured on B200 for the
-// batch-256 rank-4 step: 8 warps x 1 slot 102.6 us, 6 x 1 117, 4 x 2 127, 4 x 3 131, 5 x 2
-// 133: the heads are dealt to the warps statically, so every sub-partition must carry the
-// same number of warps.)  The update is the one of the per-head kernels:
+// and the warp needs no CTA-wide barrier.  For N = 64 eight warps per SM, two on each
+// sub-partition: while one waits for its copy the other updates its head.  For N = 128
+// (SISO) a head's 32 KB state is split into two 16 KB halves of its rows, each updated by
+// one warp of a stream (four warps per SM, two slots each); the readout's sum over N then
+// meets in shared memory (see the exchange below).  The update is the one of the per-head
+// kernels:
 //   h' = R(phi)(alpha h) + [beta R(phi) Bp | gamma B] [xp | x]^T,
 //   Y  = h'^T C + D x  (times SiLU(z) with the output gate),
 // on packed fp32 pairs, with the new state written from registers straight to HBM.
@@ -28,18 +29,35 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kSW = 8;                           // warps per CTA (one CTA per SM)
-constexpr int kSlots = 1;                        // state slots per warp (heads in flight)
+// warps per CTA (one CTA per SM) and state slots per warp (heads in flight), whole heads
+// (HV = 1) and half-heads (HV = 2).  Measured per batch-256 step on B200: whole rank-4 heads
+// 8 x 1 102.6 us (6 x 1 117, 4 x 2 127, 5 x 2 133); SISO half-heads 4 x 2 172.9 us (8 x 1
+// 189.3, 6 x 2 188.6, 4 x 3 182.0).  The heads are dealt to the warps statically, so the four
+// SM sub-partitions must carry equal numbers of warps.
+constexpr int kSW1 = 8, kSlots1 = 1;
+constexpr int kSW2 = 4, kSlots2 = 2;
 constexpr int kNP = 32;                          // state pairs (N = 64)
 constexpr int kPc = 64;                          // columns (P = 64)
 constexpr int kStateBytes = 2 * kNP * kPc * 4;   // 16 KB per head
 
-template <int R>
+constexpr int kEx = 4;                           // readout exchange slots per stream (HV = 2)
+
+// HV: warps per head.  1: a warp updates a whole head (N = 64).  2 (N = 128): the two
+// warps of a stream update one half of the head's state rows each, and the second to
+// finish adds the other's readout partial.
+template <int R, int HV>
 struct SCfg {
+    static constexpr int SW = HV == 1 ? kSW1 : kSW2;
+    static constexpr int SLOTS = HV == 1 ? kSlots1 : kSlots2;
     static constexpr int FAC_F4 = kNP * (2 + 3 * R);   // rot [2], U [2R], C [R] per pair
-    static constexpr int WARP_BYTES = kSlots * kStateBytes + FAC_F4 * 16;
-    static constexpr int SMEM = kSW * WARP_BYTES + kSW * kSlots * 8 + 128;   // + barriers, align
+    static constexpr int WARP_BYTES = SLOTS * kStateBytes + FAC_F4 * 16;
+    static constexpr int STREAMS = SW / HV;            // head streams per CTA
+    static constexpr int OFF_EX = SW * WARP_BYTES + SW * SLOTS * 8;   // exchange area
+    static constexpr int EX_FLOATS = HV == 2 ? STREAMS * kEx * 2 * R * kPc : 0;
+    static constexpr int EX_BYTES = HV == 2 ? EX_FLOATS * 4 + STREAMS * kEx * 4 : 0;
+    static constexpr int SMEM = OFF_EX + EX_BYTES + 128;   // + alignment
     static_assert(SMEM <= 232448, "shared memory");
+    static_assert(OFF_EX % 16 == 0, "exchange alignment");
 };
 
 __device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
@@ -79,22 +97,23 @@ struct Small {
     float2 bq[R], bp[R], cc[R];   // this lane's pair (rows 2 lane, 2 lane + 1) of B, B_prev, C
     float2 biasB, biasC;          // the head's BC biases of this lane's pair (BC map)
     float4 x[R], xp[R], z[R];     // this lane's column chunk of x, x_prev, z (rank columns)
-    __device__ void load(const DecodeArgs& a, int bh, int lane) {
+    // pb: the first state pair of this warp's rows
+    __device__ void load(const DecodeArgs& a, int bh, int lane, int pb) {
         const int H = a.H, G = a.G, N = a.N, P = a.P;
         const int b = bh / H, h = bh - b * H, g = h / (H / G);
-        const int j = lane & 15;
+        const int j = lane & 15, pr = pb + lane;
         dt = a.dt[bh];
         A = a.A[bh];
         lam = a.lam[bh];
         D = a.D ? a.D[h] : 0.f;
-        th = a.theta[((size_t)b * G + g) * (N / 2) + lane];
-        const size_t gofs = ((size_t)b * G + g) * R * N + 2 * lane;
+        th = a.theta[((size_t)b * G + g) * (N / 2) + pr];
+        const size_t gofs = ((size_t)b * G + g) * R * N + 2 * pr;
         const IO* Bg = static_cast<const IO*>(a.B) + gofs;
         const IO* Bpg = static_cast<const IO*>(a.B_prev) + gofs;
         const IO* Cg = static_cast<const IO*>(a.C) + gofs;
         if constexpr (BCM) {
-            biasB = a.B_bias ? load2(a.B_bias + (size_t)h * N + 2 * lane) : make_float2(0.f, 0.f);
-            biasC = a.C_bias ? load2(a.C_bias + (size_t)h * N + 2 * lane) : make_float2(0.f, 0.f);
+            biasB = a.B_bias ? load2(a.B_bias + (size_t)h * N + 2 * pr) : make_float2(0.f, 0.f);
+            biasC = a.C_bias ? load2(a.C_bias + (size_t)h * N + 2 * pr) : make_float2(0.f, 0.f);
         }
         const size_t xofs = (size_t)bh * R * P + 4 * j;
         const IO* xp0 = static_cast<const IO*>(a.x_prev) + xofs;
@@ -127,9 +146,11 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-template <typename IO, int R, bool BCM, bool XE>
-__global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeArgs a, int nbh) {
-    using C = SCfg<R>;
+template <typename IO, int R, bool BCM, bool XE, int HV>
+__global__ void __launch_bounds__((HV == 1 ? kSW1 : kSW2) * 32, 1)
+    decode_mimo_stream_kernel(DecodeArgs a, int nbh) {
+    using C = SCfg<R, HV>;
+    static_assert(HV == 1 || (HV == 2 && !BCM), "the BC map's column sums need the whole head");
     constexpr int R2 = 2 * R;
     extern __shared__ __align__(128) uint8_t sm_raw[];
     uint8_t* smb = sm_raw + ((128u - (smem_u32(sm_raw) & 127u)) & 127u);
@@ -137,28 +158,39 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeA
     const int j = lane & 15, half = lane >> 4;
     uint8_t* wb = smb + w * C::WARP_BYTES;
     const float* slot0 = reinterpret_cast<const float*>(wb);
+    constexpr int kSlots = C::SLOTS;
     float4* rot4 = reinterpret_cast<float4*>(wb + kSlots * kStateBytes);   // [32][2]
     float4* U4 = rot4 + kNP * 2;                                       // [32][2R]
     float4* C4 = U4 + kNP * R2;                                        // [32][R]
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smb + kSW * C::WARP_BYTES) + kSlots * w;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smb + C::SW * C::WARP_BYTES) + kSlots * w;
     if (lane == 0) {
         for (int s = 0; s < kSlots; ++s) mbar_init(&bar[s], 1);
         fence_mbar_init();
     }
     __syncwarp();
+    if constexpr (HV == 2) {   // the exchange counters start at 0 before any warp uses them
+        unsigned* c0 = reinterpret_cast<unsigned*>(reinterpret_cast<float*>(smb + C::OFF_EX) +
+                                                   C::EX_FLOATS);
+        for (int k = threadIdx.x; k < C::STREAMS * kEx; k += blockDim.x) c0[k] = 0u;
+        __syncthreads();
+    }
 
-    const int gw = blockIdx.x * kSW + w, NW = gridDim.x * kSW;
+    // head stream sw of the CTA; with HV = 2 warp w updates the state rows of half hf
+    const int sw = w % C::STREAMS, hf = w / C::STREAMS;
+    const int gw = blockIdx.x * C::STREAMS + sw, NW = gridDim.x * C::STREAMS;
     const int nmine = gw < nbh ? (nbh - gw + NW - 1) / NW : 0;
+    constexpr size_t kHeadFloats = (size_t)HV * 2 * kNP * kPc;
+    const size_t hoff = (size_t)hf * 2 * kNP * kPc;   // this warp's rows within the head
     auto issue = [&](int i) {   // lane 0: the state of this warp's i-th head into its slot
         const int s = i % kSlots;
         mbar_arrive_expect_tx(&bar[s], kStateBytes);
-        bulk_load(wb + s * kStateBytes, a.h + (size_t)(gw + i * NW) * 2 * kNP * kPc, kStateBytes,
-                  &bar[s]);
+        bulk_load(wb + s * kStateBytes, a.h + (size_t)(gw + i * NW) * kHeadFloats + hoff,
+                  kStateBytes, &bar[s]);
     };
     if (lane == 0)
         for (int i = 0; i < kSlots && i < nmine; ++i) issue(i);
     Small<IO, R, BCM, XE> nx;
-    if (nmine > 0) nx.load(a, gw, lane);
+    if (nmine > 0) nx.load(a, gw, lane, hf * kNP);
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     int issued = nmine < kSlots ? nmine : kSlots;   // copies issued
     bool ok = true;
@@ -206,7 +238,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeA
         }
         __syncwarp();
         // the next head's small inputs fly while this one is updated
-        if (i + 1 < nmine) nx.load(a, bh + NW, lane);
+        if (i + 1 < nmine) nx.load(a, bh + NW, lane, hf * kNP);
 
         // ---- wait for this head's state (bounded)
         const int s = i % kSlots;
@@ -223,7 +255,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeA
         for (int r = 0; r < R; ++r) ya[r] = yb[r] = make_float2(0.f, 0.f);
         if (ok) {
             const float* st = slot0 + s * (kStateBytes / 4);
-            float4* hrow = reinterpret_cast<float4*>(a.h + (size_t)bh * 2 * kNP * kPc);
+            float4* hrow = reinterpret_cast<float4*>(a.h + (size_t)bh * kHeadFloats + hoff);
 #pragma unroll 2
             for (int kk = 0; kk < kNP / 2; ++kk) {
                 const int ip = half * (kNP / 2) + kk;
@@ -263,7 +295,54 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeA
             yb[r].x += __shfl_xor_sync(0xffffffffu, yb[r].x, 16);
             yb[r].y += __shfl_xor_sync(0xffffffffu, yb[r].y, 16);
         }
-        if (half == 0) {
+        bool writer = true;   // this warp writes y and x_prev
+        if constexpr (HV == 2) {
+            // The two warps of the stream meet through exchange slot i % kEx: each writes
+            // its partial readout there and arrives on the slot's counter; the second to
+            // arrive adds the other's partial and writes the head's outputs, then arrives
+            // once more to free the slot.  Use u = i / kEx of a slot spans counter values
+            // 3u .. 3u + 3; a warp more than kEx heads ahead of its partner waits (bounded)
+            // until the slot's previous use is over.
+            float* exb = reinterpret_cast<float*>(smb + C::OFF_EX);
+            unsigned* cnt = reinterpret_cast<unsigned*>(exb + C::EX_FLOATS) + sw * kEx;
+            const int es = i % kEx;
+            const unsigned base = 3u * (unsigned)(i / kEx);
+            bool fr = true;
+            if (lane == 0) {
+                const uint64_t t0 = globaltimer();
+                while (*reinterpret_cast<volatile unsigned*>(&cnt[es]) < base &&
+                       globaltimer() - t0 < 2000000000ull) {
+                }
+                fr = *reinterpret_cast<volatile unsigned*>(&cnt[es]) >= base;
+            }
+            fr = __shfl_sync(0xffffffffu, fr ? 1 : 0, 0) != 0;
+            if (!fr) ok = false;
+            float* mine = exb + ((size_t)(sw * kEx + es) * 2 + hf) * R * kPc;
+            const float* other = exb + ((size_t)(sw * kEx + es) * 2 + (hf ^ 1)) * R * kPc;
+            if (half == 0) {
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    *reinterpret_cast<float4*>(mine + r * kPc + 4 * j) =
+                        make_float4(ya[r].x, ya[r].y, yb[r].x, yb[r].y);
+            }
+            __syncwarp();
+            unsigned old = 0;
+            if (lane == 0) {
+                __threadfence_block();
+                old = atomicAdd(&cnt[es], 1u);
+                __threadfence_block();
+            }
+            old = __shfl_sync(0xffffffffu, old, 0);
+            writer = old == base + 1;
+            if (writer && half == 0) {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float4 o = *reinterpret_cast<const float4*>(other + r * kPc + 4 * j);
+                    ya[r].x += o.x; ya[r].y += o.y; yb[r].x += o.z; yb[r].y += o.w;
+                }
+            }
+        }
+        if (writer && half == 0) {
             IO* y = static_cast<IO*>(a.y) + (size_t)bh * R * kPc + 4 * j;
             IO* xpo = static_cast<IO*>(a.x_prev) + (size_t)bh * R * kPc + 4 * j;
 #pragma unroll
@@ -283,6 +362,17 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_mimo_stream_kernel(DecodeA
                 }
                 store4(y + r * kPc, v);
                 store4(xpo + r * kPc, cur.x[r]);   // x_prev <- x (exact in the io dtype)
+            }
+        }
+        if constexpr (HV == 2) {
+            if (writer) {   // the other warp's partial is read: free the exchange slot
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence_block();
+                    atomicAdd(reinterpret_cast<unsigned*>(reinterpret_cast<float*>(smb + C::OFF_EX) +
+                                                          C::EX_FLOATS) + sw * kEx + i % kEx,
+                              1u);
+                }
             }
         }
         // the slot is free once every lane has read it: the copy of head i + kSlots goes there
@@ -318,17 +408,17 @@ int num_sms() {
     return sms[dev] ? sms[dev] : 148;
 }
 
-template <typename IO, int R, bool BCM, bool XE>
+template <typename IO, int R, bool BCM, bool XE, int HV = 1>
 cudaError_t launch_stream_t(const DecodeArgs& a, int batch, cudaStream_t s) {
-    using C = SCfg<R>;
-    cudaError_t e = cudaFuncSetAttribute(decode_mimo_stream_kernel<IO, R, BCM, XE>,
+    using C = SCfg<R, HV>;
+    cudaError_t e = cudaFuncSetAttribute(decode_mimo_stream_kernel<IO, R, BCM, XE, HV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const int nbh = batch * a.H;
     int grid = num_sms();
-    const int need = (nbh + kSW - 1) / kSW;
+    const int need = (nbh + C::STREAMS - 1) / C::STREAMS;
     if (grid > need) grid = need;
-    decode_mimo_stream_kernel<IO, R, BCM, XE><<<grid, kSW * 32, C::SMEM, s>>>(a, nbh);
+    decode_mimo_stream_kernel<IO, R, BCM, XE, HV><<<grid, C::SW * 32, C::SMEM, s>>>(a, nbh);
     return cudaGetLastError();
 }
 
@@ -350,14 +440,22 @@ cudaError_t launch_stream_io(const DecodeArgs& a, int batch, int R, cudaStream_t
 
 }  // namespace
 
+// MIMO N = 64 (rank 2, 4; every fused part), and SISO N = 128 as half-heads (plain or
+// with the output gate: the BC map's column sums would need the whole head)
 bool decode_stream_ok(const DecodeArgs& a, int R) {
-    return a.N == 2 * kNP && a.P == kPc && (R == 2 || R == 4);
+    if (a.P != kPc) return false;
+    if (a.N == 2 * kNP) return R == 2 || R == 4;
+    const bool bcm = a.B_bias || a.C_bias || a.bc_eps > 0.f;
+    return a.N == 4 * kNP && R == 1 && !bcm && !a.x_expand && !a.z_expand;
 }
 
 // The BC map and the lightweight expansion are compile-time variants, so the plain
 // instantiations hold none of their code.
 cudaError_t launch_decode_stream(const DecodeArgs& a, int batch, int R, int io_dtype,
                                  cudaStream_t s) {
+    if (a.N == 4 * kNP)
+        return io_dtype == M3_BF16 ? launch_stream_t<__nv_bfloat16, 1, false, false, 2>(a, batch, s)
+                                   : launch_stream_t<float, 1, false, false, 2>(a, batch, s);
     return io_dtype == M3_BF16 ? launch_stream_io<__nv_bfloat16>(a, batch, R, s)
                                : launch_stream_io<float>(a, batch, R, s);
 }
