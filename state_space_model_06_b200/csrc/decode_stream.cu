@@ -148,7 +148,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 template <typename IO, int R, bool BCM, bool XE, int HV>
 __global__ void __launch_bounds__((HV == 1 ? kSW1 : kSW2) * 32, 1)
-    decode_mimo_stream_kernel(DecodeArgs a, int nbh) {
+    decode_stream_kernel(DecodeArgs a, int nbh) {
     using C = SCfg<R, HV>;
     static_assert(HV == 1 || (HV == 2 && !BCM), "the BC map's column sums need the whole head");
     constexpr int R2 = 2 * R;
@@ -411,14 +411,14 @@ int num_sms() {
 template <typename IO, int R, bool BCM, bool XE, int HV = 1>
 cudaError_t launch_stream_t(const DecodeArgs& a, int batch, cudaStream_t s) {
     using C = SCfg<R, HV>;
-    cudaError_t e = cudaFuncSetAttribute(decode_mimo_stream_kernel<IO, R, BCM, XE, HV>,
+    cudaError_t e = cudaFuncSetAttribute(decode_stream_kernel<IO, R, BCM, XE, HV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const int nbh = batch * a.H;
     int grid = num_sms();
     const int need = (nbh + C::STREAMS - 1) / C::STREAMS;
     if (grid > need) grid = need;
-    decode_mimo_stream_kernel<IO, R, BCM, XE, HV><<<grid, C::SW * 32, C::SMEM, s>>>(a, nbh);
+    decode_stream_kernel<IO, R, BCM, XE, HV><<<grid, C::SW * 32, C::SMEM, s>>>(a, nbh);
     return cudaGetLastError();
 }
 

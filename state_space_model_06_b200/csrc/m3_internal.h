@@ -34,9 +34,9 @@ m3_status scan_validate(const m3_dims* d, int32_t seqlen, int32_t chunk, const v
 // decode step: one CTA per (batch, head); template on io type and rank
 cudaError_t launch_decode(const DecodeArgs& a, int batch, int R, int io_dtype, cudaStream_t s);
 
-// MIMO decode step (N = P = 64, rank 2 or 4; gate, BC map and expansion fused) as a persistent
-// kernel: each warp streams its heads, the next head's state in flight while it updates
-// the current one
+// Decode step as a persistent streaming kernel (MIMO N = P = 64, rank 2 or 4, every fused
+// part; SISO N = 128, P = 64 as half-heads, plain or gated): each warp streams heads or
+// half-heads through a bulk-copied shared-memory slot
 bool decode_stream_ok(const DecodeArgs& a, int R);
 cudaError_t launch_decode_stream(const DecodeArgs& a, int batch, int R, int io_dtype,
                                  cudaStream_t s);
