@@ -39,11 +39,15 @@ m3_status check_state(const m3_state* st) {
 bool rank_has_kernel(int R) { return R == 1 || R == 2 || R == 3 || R == 4 || R == 8; }
 
 // SIMT prefill thread shape: ns lanes per state column (a power of two <= 32),
-// ppt pairs per lane; P * ns threads.
+// ppt pairs per lane; P * ns threads.  At most 8 pairs per lane, and more lanes (down to
+// one pair each) while the CTA has fewer than 256 threads: one CTA per (batch, head) runs
+// its tokens one after the other, so a small CTA would leave the token chain to a few
+// threads (measured on B200 for b1 H2 P16 N16 T256: 16 threads, 460 us per call).
 bool simt_shape(int N, int P, int* ppt, int* ns) {
     const int pairs = N / 2;
     int n = 1;
     while ((pairs + n - 1) / n > 8 && n < 32) n *= 2;
+    while (P * n < 256 && 2 * n <= pairs && n < 32) n *= 2;
     int p = (pairs + n - 1) / n;
     while (P * n > 1024 && n > 1) {
         n /= 2;

@@ -9,15 +9,24 @@
 // One CTA per (batch, head).  Column p of the N x P state is independent of the
 // other columns (x_t[p] only enters column p), so thread (p, k) owns column p and
 // a contiguous block of `ppt` state pairs; the `ns` lanes of one column are
-// adjacent, so the readout's sum over N is a warp-shuffle reduction.  Each token's
-// small inputs are staged in shared memory; the previous token's stay in the other
-// half of a ping-pong buffer for the trapezoid's beta term.
+// adjacent, so the readout's sum over N is a warp-shuffle reduction.  Tokens go in
+// blocks of up to TB: the whole CTA stages a block's inputs in shared memory at once
+// (x, B, C after the BC map, z, the rotation's cos / sin and alpha, beta, gamma per
+// token), so the token loop itself reads no global memory and needs no barrier.  Slot 0
+// of the block holds the previous token (the carried one, then the last of the block
+// before) for the trapezoid's beta term.
 #include "m3_internal.h"
 
 namespace m3 {
 
+// Floats of one staged token: x [R][P], B [R][N], C [R][N], z [R][P] (gate only),
+// cos / sin [N/2] each, alpha / beta / gamma.
+__host__ __device__ inline int simt_token_floats(int N, int P, int R, bool gate) {
+    return R * P + 2 * R * N + (gate ? R * P : 0) + N + 4;
+}
+
 template <typename IO, int R, int PPTMAX>
-__global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
+__global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a, int TB) {
     extern __shared__ float sm[];
     const int N = a.N, P = a.P, H = a.H, G = a.G;
     const long long T = a.T;
@@ -26,13 +35,12 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
     const int b = bh / H, h = bh - b * H, g = h / (H / G);
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int p = tid / ns, k = tid - p * ns;
-
-    const int buf_floats = R * P + 2 * R * N;
-    float* buf0 = sm;                      // token t even: x[R][P], B[R][N], C[R][N]
-    float* buf1 = sm + buf_floats;         // token t odd
-    float* cs = sm + 2 * buf_floats;       // [N/2]
-    float* sn = cs + N / 2;                // [N/2]
-    float* scal = sn + N / 2;              // alpha, beta, gamma
+    const bool gate = a.z != nullptr;
+    const int TF = simt_token_floats(N, P, R, gate);
+    // token slot layout (slot 0: the previous token; slots 1..TB: the block)
+    const int oX = 0, oB = R * P, oC = oB + R * N, oZ = oC + R * N;
+    const int oCS = oZ + (gate ? R * P : 0), oSN = oCS + N / 2, oSC = oSN + N / 2;
+    auto slot = [&](int s) { return sm + (size_t)s * TF; };
 
     // state column p, pairs i = k*ppt + j
     float hs[2 * PPTMAX];
@@ -59,118 +67,140 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
     const float* sC = a.bc_scale ? sB + ncol : nullptr;
     const float* sP = a.bc_scale ? a.bc_scale + 2 * ncol + ((size_t)b * G + g) * R : nullptr;
 
-    // previous token of the first step comes from the carried state (buffer 1)
+    // slot 0 of the first block: the carried previous token
     {
+        float* s0 = slot(0);
         const IO* xp = static_cast<const IO*>(a.x_prev) + (size_t)bh * R * P;
         const IO* bp = static_cast<const IO*>(a.B_prev) + ((size_t)b * G + g) * R * N;
-        for (int e = tid; e < R * P; e += nthr) buf1[e] = to_f(xp[e]);
+        for (int e = tid; e < R * P; e += nthr) s0[oX + e] = to_f(xp[e]);
         for (int e = tid; e < R * N; e += nthr) {
             const int r = e / N;
             const float sc = sP ? sP[r] : 1.f;
-            buf1[R * P + e] = a.bc ? bc_apply(to_f(bp[e]), sc, Bb, e - r * N) : to_f(bp[e]);
+            s0[oB + e] = a.bc ? bc_apply(to_f(bp[e]), sc, Bb, e - r * N) : to_f(bp[e]);
         }
     }
 
     const float Dh = a.D ? a.D[h] : 0.f;
     const int warp_lanes = min(32, nthr - (tid & ~31));
     const unsigned lane_mask = warp_lanes == 32 ? 0xffffffffu : ((1u << warp_lanes) - 1u);
+    const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
+    const float* wz = a.z_expand ? a.z_expand + (size_t)h * R * P : nullptr;
 
-    for (long long t = 0; t < T; ++t) {
-        float* cur = (t & 1) ? buf1 : buf0;
-        const float* prv = (t & 1) ? buf0 : buf1;
-        __syncthreads();   // token t-1 is done with `cur` (it held token t-2) and cs/sn/scal
-        const size_t bt = (size_t)b * T + t;
-        // x of this token: [R][P], or one value per channel expanded by the head's weights
-        const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
-        const IO* xt = static_cast<const IO*>(a.x) + (bt * H + h) * (wx ? 1 : R) * P;
-        const IO* Bt = static_cast<const IO*>(a.B) + (bt * G + g) * R * N;
-        const IO* Ct = static_cast<const IO*>(a.C) + (bt * G + g) * R * N;
-        const float dt = a.dt[bt * H + h];
-        if (wx) {
-            for (int e = tid; e < R * P; e += nthr) cur[e] = expand_io<IO>(to_f(xt[e % P]), wx[e]);
-        } else {
-            for (int e = tid; e < R * P; e += nthr) cur[e] = to_f(xt[e]);
+    for (long long t0 = 0; t0 < T; t0 += TB) {
+        const int nt = (int)(T - t0 < TB ? T - t0 : TB);
+        __syncthreads();   // the previous block's tokens are done
+        // ---- stage tokens t0 .. t0 + nt - 1 into slots 1 .. nt
+        for (int e = tid; e < nt * R * P; e += nthr) {
+            const int tt = e / (R * P), q = e - tt * (R * P);
+            const size_t bt = (size_t)b * T + t0 + tt;
+            float* d = slot(1 + tt);
+            const IO* xt = static_cast<const IO*>(a.x) + (bt * H + h) * (wx ? 1 : R) * P;
+            d[oX + q] = wx ? expand_io<IO>(to_f(xt[q % P]), wx[q]) : to_f(xt[q]);
+            if (gate) {
+                const IO* zt = static_cast<const IO*>(a.z);
+                d[oZ + q] = wz ? expand_io<IO>(to_f(zt[(bt * H + h) * P + q % P]), wz[q])
+                               : to_f(zt[(bt * H + h) * R * P + q]);
+            }
         }
-        if (a.bc) {
-            for (int e = tid; e < R * N; e += nthr) {
-                const int r = e / N, n = e - r * N;
+        for (int e = tid; e < nt * R * N; e += nthr) {
+            const int tt = e / (R * N), q = e - tt * (R * N);
+            const int r = q / N, n = q - r * N;
+            const long long t = t0 + tt;
+            const size_t bt = (size_t)b * T + t;
+            float* d = slot(1 + tt);
+            const float bv = to_f(static_cast<const IO*>(a.B)[(bt * G + g) * R * N + q]);
+            const float cv = to_f(static_cast<const IO*>(a.C)[(bt * G + g) * R * N + q]);
+            if (a.bc) {
                 const size_t si = (size_t)r * Tp + t;
-                cur[R * P + e] = bc_apply(to_f(Bt[e]), sB ? sB[si] : 1.f, Bb, n);
-                cur[R * P + R * N + e] = bc_apply(to_f(Ct[e]), sC ? sC[si] : 1.f, Cb, n);
-            }
-        } else {
-            for (int e = tid; e < R * N; e += nthr) {
-                cur[R * P + e] = to_f(Bt[e]);
-                cur[R * P + R * N + e] = to_f(Ct[e]);
+                d[oB + q] = bc_apply(bv, sB ? sB[si] : 1.f, Bb, n);
+                d[oC + q] = bc_apply(cv, sC ? sC[si] : 1.f, Cb, n);
+            } else {
+                d[oB + q] = bv;
+                d[oC + q] = cv;
             }
         }
-        const float* th = a.theta + (bt * G + g) * (N / 2);
-        for (int i = tid; i < N / 2; i += nthr) {
-            const float phi = (a.flags & M3_FLAG_THETA_IS_ANGLE) ? th[i] : dt * th[i];
-            float s, c;
-            sincosf(phi, &s, &c);
-            cs[i] = c;
-            sn[i] = s;
+        for (int e = tid; e < nt * (N / 2); e += nthr) {
+            const int tt = e / (N / 2), i = e - tt * (N / 2);
+            const size_t bt = (size_t)b * T + t0 + tt;
+            const float dt = a.dt[bt * H + h];
+            const float th = a.theta[(bt * G + g) * (N / 2) + i];
+            const float phi = (a.flags & M3_FLAG_THETA_IS_ANGLE) ? th : dt * th;
+            float sv, cv;
+            sincosf(phi, &sv, &cv);
+            float* d = slot(1 + tt);
+            d[oCS + i] = cv;
+            d[oSN + i] = sv;
         }
-        if (tid == 0) {
+        for (int tt = tid; tt < nt; tt += nthr) {
+            const size_t bt = (size_t)b * T + t0 + tt;
+            const float dt = a.dt[bt * H + h];
             const float Av = a.A[bt * H + h], lam = a.lam[bt * H + h];
             const float alpha = expf(dt * Av);
-            scal[0] = alpha;
-            scal[1] = (1.f - lam) * dt * alpha;
-            scal[2] = lam * dt;
+            float* d = slot(1 + tt);
+            d[oSC + 0] = alpha;
+            d[oSC + 1] = (1.f - lam) * dt * alpha;
+            d[oSC + 2] = lam * dt;
         }
         __syncthreads();
 
-        const float alpha = scal[0], beta = scal[1], gamma = scal[2];
-        const float* xc = cur;
-        const float* Bc = cur + R * P;
-        const float* Cc = cur + R * P + R * N;
-        const float* xq = prv;
-        const float* Bq = prv + R * P;
-        float yp[R];
+        // ---- the block's tokens: no global reads, no barrier
+        for (int tt = 0; tt < nt; ++tt) {
+            const float* cur = slot(1 + tt);
+            const float* prv = slot(tt);
+            const size_t bt = (size_t)b * T + t0 + tt;
+            const float alpha = cur[oSC], beta = cur[oSC + 1], gamma = cur[oSC + 2];
+            const float* xc = cur + oX;
+            const float* Bc = cur + oB;
+            const float* Cc = cur + oC;
+            const float* xq = prv + oX;
+            const float* Bq = prv + oB;
+            float yp[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) yp[r] = 0.f;
+            for (int r = 0; r < R; ++r) yp[r] = 0.f;
 #pragma unroll
-        for (int j = 0; j < PPTMAX; ++j) {
-            const int i = k * ppt + j;
-            if (j < ppt && i < N / 2) {
-                float ub0 = 0.f, ub1 = 0.f, ug0 = 0.f, ug1 = 0.f;
+            for (int j = 0; j < PPTMAX; ++j) {
+                const int i = k * ppt + j;
+                if (j < ppt && i < N / 2) {
+                    float ub0 = 0.f, ub1 = 0.f, ug0 = 0.f, ug1 = 0.f;
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        ub0 = fmaf(Bq[r * N + 2 * i], xq[r * P + p], ub0);
+                        ub1 = fmaf(Bq[r * N + 2 * i + 1], xq[r * P + p], ub1);
+                        ug0 = fmaf(Bc[r * N + 2 * i], xc[r * P + p], ug0);
+                        ug1 = fmaf(Bc[r * N + 2 * i + 1], xc[r * P + p], ug1);
+                    }
+                    const float m0 = fmaf(alpha, hs[2 * j], beta * ub0);
+                    const float m1 = fmaf(alpha, hs[2 * j + 1], beta * ub1);
+                    const float c = cur[oCS + i], s = cur[oSN + i];
+                    const float n0 = fmaf(c, m0, fmaf(-s, m1, gamma * ug0));
+                    const float n1 = fmaf(s, m0, fmaf(c, m1, gamma * ug1));
+                    hs[2 * j] = n0;
+                    hs[2 * j + 1] = n1;
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+                        yp[r] = fmaf(n0, Cc[r * N + 2 * i], fmaf(n1, Cc[r * N + 2 * i + 1], yp[r]));
+                }
+            }
+            for (int off = ns >> 1; off > 0; off >>= 1)
+#pragma unroll
+                for (int r = 0; r < R; ++r) yp[r] += __shfl_xor_sync(lane_mask, yp[r], off);
+            if (k == 0) {
+                IO* yt = static_cast<IO*>(a.y) + (bt * H + h) * R * P;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    ub0 = fmaf(Bq[r * N + 2 * i], xq[r * P + p], ub0);
-                    ub1 = fmaf(Bq[r * N + 2 * i + 1], xq[r * P + p], ub1);
-                    ug0 = fmaf(Bc[r * N + 2 * i], xc[r * P + p], ug0);
-                    ug1 = fmaf(Bc[r * N + 2 * i + 1], xc[r * P + p], ug1);
+                    float v = yp[r] + Dh * xc[r * P + p];
+                    if (gate) v = gate_silu(v, cur[oZ + r * P + p]);
+                    yt[r * P + p] = from_f<IO>(v);
                 }
-                const float m0 = fmaf(alpha, hs[2 * j], beta * ub0);
-                const float m1 = fmaf(alpha, hs[2 * j + 1], beta * ub1);
-                const float c = cs[i], s = sn[i];
-                const float n0 = fmaf(c, m0, fmaf(-s, m1, gamma * ug0));
-                const float n1 = fmaf(s, m0, fmaf(c, m1, gamma * ug1));
-                hs[2 * j] = n0;
-                hs[2 * j + 1] = n1;
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-                    yp[r] = fmaf(n0, Cc[r * N + 2 * i], fmaf(n1, Cc[r * N + 2 * i + 1], yp[r]));
             }
         }
-        for (int off = ns >> 1; off > 0; off >>= 1)
-#pragma unroll
-            for (int r = 0; r < R; ++r) yp[r] += __shfl_xor_sync(lane_mask, yp[r], off);
-        if (k == 0) {
-            IO* yt = static_cast<IO*>(a.y) + (bt * H + h) * R * P;
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                float v = yp[r] + Dh * xc[r * P + p];
-                if (a.z) {
-                    const IO* zt = static_cast<const IO*>(a.z);
-                    const float zv = a.z_expand
-                        ? expand_io<IO>(to_f(zt[(bt * H + h) * P + p]), a.z_expand[((size_t)h * R + r) * P + p])
-                        : to_f(zt[(bt * H + h) * R * P + r * P + p]);
-                    v = gate_silu(v, zv);
-                }
-                yt[r * P + p] = from_f<IO>(v);
-            }
+        // ---- the block's last token becomes slot 0 of the next block
+        __syncthreads();
+        if (t0 + nt < T) {
+            const float* last = slot(nt);
+            float* s0 = slot(0);
+            for (int e = tid; e < R * P; e += nthr) s0[oX + e] = last[oX + e];
+            for (int e = tid; e < R * N; e += nthr) s0[oB + e] = last[oB + e];
         }
     }
 
@@ -184,7 +214,6 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
     }
     if (k == 0 && T > 0) {
         // x_prev <- X_{T-1}: the expanded value when x comes with expansion weights
-        const float* wx = a.x_expand ? a.x_expand + (size_t)h * R * P : nullptr;
         const IO* xl =
             static_cast<const IO*>(a.x) + (((size_t)b * T + (T - 1)) * H + h) * (wx ? 1 : R) * P;
         IO* xpo = static_cast<IO*>(a.x_prev) + (size_t)bh * R * P;
@@ -194,16 +223,21 @@ __global__ void __launch_bounds__(1024) scan_simt_kernel(ScanArgs a) {
     }
 }
 
+// Tokens per staged block: up to 64, within 96 KB of shared memory (TB + 1 token slots).
 template <typename IO, int R, int PPTMAX>
 static cudaError_t launch_simt_t(const ScanArgs& a, cudaStream_t s) {
     const int threads = a.P * a.ns;
-    const size_t smem = sizeof(float) * (size_t)(2 * (R * a.P + 2 * R * a.N) + a.N + 4);
+    const int tf = simt_token_floats(a.N, a.P, R, a.z != nullptr);
+    int TB = (int)((96 * 1024) / (sizeof(float) * (size_t)tf)) - 1;
+    if (TB > 64) TB = 64;
+    if (TB < 1) TB = 1;
+    const size_t smem = sizeof(float) * (size_t)tf * (TB + 1);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(scan_simt_kernel<IO, R, PPTMAX>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    scan_simt_kernel<IO, R, PPTMAX><<<(unsigned)(a.batch * a.H), threads, smem, s>>>(a);
+    scan_simt_kernel<IO, R, PPTMAX><<<(unsigned)(a.batch * a.H), threads, smem, s>>>(a, TB);
     return cudaGetLastError();
 }
 
