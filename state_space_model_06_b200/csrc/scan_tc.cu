@@ -481,8 +481,26 @@ __device__ void rotation(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t
                 *reinterpret_cast<uint32_t*>(cbase + C::CT_BYTES + off) = bo;
                 if constexpr (!MAP) *reinterpret_cast<uint32_t*>(cbase + off) = co;
             };
-            // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1], two tokens per packed
-            // fp32x2 operation (their cos and sin form the packed operands)
+            // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1]
+            if constexpr (!bc) {
+                // on the packed bf16 pair itself: (cos, cos) (v0, v1) + (sin, -sin) (v1, v0)
+#pragma unroll
+                for (int jj = 0; jj < TPT; ++jj) {
+                    const __nv_bfloat162 cc = __floats2bfloat162_rn(cn[jj], cn[jj]);
+                    const __nv_bfloat162 ss = __floats2bfloat162_rn(sn[jj], -sn[jj]);
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const uint32_t ub = bv[jj][r], uc = cv[jj][r];
+                        const __nv_bfloat162 vb = *reinterpret_cast<const __nv_bfloat162*>(&ub);
+                        const __nv_bfloat162 vc = *reinterpret_cast<const __nv_bfloat162*>(&uc);
+                        const __nv_bfloat162 nb = __hfma2(cc, vb, __hmul2(ss, __lowhigh2highlow(vb)));
+                        const __nv_bfloat162 nc = __hfma2(cc, vc, __hmul2(ss, __lowhigh2highlow(vc)));
+                        store(jj, r, *reinterpret_cast<const uint32_t*>(&nb),
+                              *reinterpret_cast<const uint32_t*>(&nc));
+                    }
+                }
+            } else {
+            // two tokens per packed fp32x2 operation (their cos and sin form the packed operands)
 #pragma unroll
             for (int jj = 0; jj + 1 < TPT; jj += 2) {
                 const float2 c2 = make_float2(cn[jj], cn[jj + 1]);
@@ -527,6 +545,7 @@ __device__ void rotation(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t
                     store(jj, r, pack_bf16x2(fmaf(cn[jj], b0, sn[jj] * b1), fmaf(cn[jj], b1, -sn[jj] * b0)),
                           pack_bf16x2(fmaf(cn[jj], c0, sn[jj] * c1), fmaf(cn[jj], c1, -sn[jj] * c0)));
                 }
+            }
             }
             psi_acc += tot;
             __syncwarp();
