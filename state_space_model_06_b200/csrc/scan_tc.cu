@@ -572,12 +572,13 @@ __device__ void rotation(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t
                 const float sc = ex2_approx(cend - cf.cum2()[u]) * cf.w()[u];
                 const uint32_t off = (uint32_t)row * 128u + ((uint32_t)((ch ^ row) & 7) << 4);
                 uint4 v = *reinterpret_cast<const uint4*>(xt + off);
-                uint4 o;
-                o.x = pack_bf16x2(bf16lo(v.x) * sc, bf16hi(v.x) * sc);
-                o.y = pack_bf16x2(bf16lo(v.y) * sc, bf16hi(v.y) * sc);
-                o.z = pack_bf16x2(bf16lo(v.z) * sc, bf16hi(v.z) * sc);
-                o.w = pack_bf16x2(bf16lo(v.w) * sc, bf16hi(v.w) * sc);
-                *reinterpret_cast<uint4*>(xw + off) = o;
+                // on the packed bf16 pairs: the weight is rounded to bf16 once
+                const __nv_bfloat162 s2 = __float2bfloat162_rn(sc);
+                auto mul = [&](uint32_t u) {
+                    const __nv_bfloat162 t = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&u), s2);
+                    return *reinterpret_cast<const uint32_t*>(&t);
+                };
+                *reinterpret_cast<uint4*>(xw + off) = make_uint4(mul(v.x), mul(v.y), mul(v.z), mul(v.w));
             }
         }
         fence_proxy_async_smem();
