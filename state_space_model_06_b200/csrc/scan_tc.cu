@@ -416,13 +416,14 @@ __device__ void rotation(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t
             const int tb = s * C::RT;           // first token of the sub-chunk (chunk-relative)
             const int j0 = ts * TPT;
             // angle increments of the own tokens and their sum
+            // (running sums over the own tokens, one FMA each)
             float ph[TPT], own = 0.f;
 #pragma unroll
             for (int jj = 0; jj < TPT; ++jj) {
                 const int j = j0 + jj;
                 const float d = angle ? 1.f : dtt[(tb + j) * 4 + hq];
-                ph[jj] = d * th[j * PAIRS + pair];
-                own += ph[jj];
+                own = fmaf(d, th[j * PAIRS + pair], own);
+                ph[jj] = own;
             }
             // publish the range sum; load the own tokens' raw B, C meanwhile
             float* rb = rsum + (rs * TSPLIT) * PAIRS;
@@ -459,13 +460,11 @@ __device__ void rotation(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t
                 tot += v;
                 pre += (qq < ts) ? v : 0.f;
             }
-            float psi = psi_acc + pre;
+            const float psi0 = psi_acc + pre;
             float cn[TPT], sn[TPT];
 #pragma unroll
-            for (int jj = 0; jj < TPT; ++jj) {
-                psi += ph[jj];
-                __sincosf(psi, &sn[jj], &cn[jj]);   // |psi| < pi + one chunk of angle increments
-            }
+            for (int jj = 0; jj < TPT; ++jj)   // |psi| < pi + one chunk of angle increments
+                __sincosf(psi0 + ph[jj], &sn[jj], &cn[jj]);
             // operand rows (tb + j0 + jj) * R + r; when the first of them is a multiple of 8
             // the SW128 chunk of every row is a compile-time xor of this thread's chunk
             const int row0 = (tb + j0) * R;
@@ -483,18 +482,20 @@ __device__ void rotation(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t
             };
             // R(-psi) [v0; v1] = [cos v0 + sin v1; -sin v0 + cos v1]
             if constexpr (!bc) {
-                // on the packed bf16 pair itself: (cos, cos) (v0, v1) + (sin, -sin) (v1, v0)
+                // on the packed bf16 pair itself: (v0, v0) (cos, -sin) + (v1, v1) (sin, cos)
 #pragma unroll
                 for (int jj = 0; jj < TPT; ++jj) {
-                    const __nv_bfloat162 cc = __floats2bfloat162_rn(cn[jj], cn[jj]);
-                    const __nv_bfloat162 ss = __floats2bfloat162_rn(sn[jj], -sn[jj]);
+                    const __nv_bfloat162 k0 = __floats2bfloat162_rn(cn[jj], -sn[jj]);
+                    const __nv_bfloat162 k1 = __floats2bfloat162_rn(sn[jj], cn[jj]);
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         const uint32_t ub = bv[jj][r], uc = cv[jj][r];
                         const __nv_bfloat162 vb = *reinterpret_cast<const __nv_bfloat162*>(&ub);
                         const __nv_bfloat162 vc = *reinterpret_cast<const __nv_bfloat162*>(&uc);
-                        const __nv_bfloat162 nb = __hfma2(cc, vb, __hmul2(ss, __lowhigh2highlow(vb)));
-                        const __nv_bfloat162 nc = __hfma2(cc, vc, __hmul2(ss, __lowhigh2highlow(vc)));
+                        const __nv_bfloat162 nb =
+                            __hfma2(__high2bfloat162(vb), k1, __hmul2(__low2bfloat162(vb), k0));
+                        const __nv_bfloat162 nc =
+                            __hfma2(__high2bfloat162(vc), k1, __hmul2(__low2bfloat162(vc), k0));
                         store(jj, r, *reinterpret_cast<const uint32_t*>(&nb),
                               *reinterpret_cast<const uint32_t*>(&nc));
                     }
@@ -770,8 +771,14 @@ __device__ void epilogue(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t
                     const uint32_t off = sw128_off(lrow, lcol0 + cb + j);
                     float v[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        v[e] = fmaf(sc, __uint_as_float(yi[j + e]), __uint_as_float(ya[j + e]));
+                    for (int e = 0; e < 8; e += 2) {   // packed fp32x2: two columns per FMA
+                        const float2 r2 = __ffma2_rn(
+                            make_float2(sc, sc),
+                            make_float2(__uint_as_float(yi[j + e]), __uint_as_float(yi[j + e + 1])),
+                            make_float2(__uint_as_float(ya[j + e]), __uint_as_float(ya[j + e + 1])));
+                        v[e] = r2.x;
+                        v[e + 1] = r2.y;
+                    }
                     if constexpr (GT) {
                         // the z tile has the x tile's layout: same swizzled offset
                         const uint4 zq = *reinterpret_cast<const uint4*>(zt + off);
@@ -971,8 +978,14 @@ __device__ void state(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t* b
                 ln.ld16(kHalfN, C::TM_G, cb, gq);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    gq[j] = __float_as_uint(fmaf(dec, __uint_as_float(gq[j]), __uint_as_float(d[j])));
+                for (int j = 0; j < 16; j += 2) {   // packed fp32x2: two columns per FMA
+                    const float2 r2 = __ffma2_rn(
+                        make_float2(dec, dec),
+                        make_float2(__uint_as_float(gq[j]), __uint_as_float(gq[j + 1])),
+                        make_float2(__uint_as_float(d[j]), __uint_as_float(d[j + 1])));
+                    gq[j] = __float_as_uint(r2.x);
+                    gq[j + 1] = __float_as_uint(r2.y);
+                }
                 ln.st16(kHalfN, C::TM_G, cb, gq);
                 if constexpr (!MAP) publish16(cb, gq);
             }
