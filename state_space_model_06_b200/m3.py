@@ -10,7 +10,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from dataclasses import dataclass
+from dataclasses import dataclass, replace
 
 import torch
 
@@ -166,6 +166,14 @@ class State:
 
     def c(self) -> m3_state:
         return m3_state(self.h.data_ptr(), self.x_prev.data_ptr(), self.B_prev.data_ptr())
+
+    def rows(self, lo: int, hi: int) -> "State":
+        """Batch rows [lo, hi) of this state (the same memory), for a call on a slice of
+        the batch: every tensor of the state leads with the batch axis."""
+        v = State.__new__(State)
+        v.dims = replace(self.dims, batch=hi - lo)
+        v.h, v.x_prev, v.B_prev = self.h[lo:hi], self.x_prev[lo:hi], self.B_prev[lo:hi]
+        return v
 
 
 def m3_state_bytes(dims: Dims):

@@ -73,3 +73,35 @@ def test_tc_agrees_with_sequential_kernel(Q):
     yt, ht, _, _ = gpu_scan(inp, d, T, Q)
     ys, hs, _, _ = gpu_scan(inp, d, T, Q, flags=m3.M3_FLAG_FORCE_SIMT)
     assert rel_slices(yt, ys, (1, 3, 4)) <= TOL and rel_slices(ht, hs, (2, 3)) <= TOL
+
+
+def test_tc_batch_row_slices_equal_one_call():
+    """Calls on slices of the batch rows (State.rows views of one state) give exactly the
+    results of one call over the whole batch: the rows are independent.  (The pipelined
+    end-to-end bench leg runs the batch this way.)"""
+    b, H, G, P, N, R, T, Q = 4, 4, 1, 64, 128, 1, 200, 64
+    inp = inputs.make_scan_inputs(b, T, H, G, P, N, R, io_dtype=torch.bfloat16, seed=14,
+                                  h0_random=True, carry_prev=True)
+    d = dims_of(b, H, G, P, N, R)
+    g = {k: v.cuda() for k, v in inp.items()}
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")   # unsegmented either way
+
+    def fresh():
+        st = m3.State(d)
+        st.h.copy_(g["h0"])
+        st.x_prev.copy_(g["x_prev"])
+        st.B_prev.copy_(g["B_prev"])
+        return st
+
+    st1, y1 = fresh(), torch.empty_like(g["x"])
+    m3.m3_scan_fwd(d, T, Q, g["x"], g["B"], g["C"], g["dt"], g["A"], g["lam"], g["theta"],
+                   g["D"], st1, y1, ws)
+    st2, y2 = fresh(), torch.empty_like(g["x"])
+    for lo, hi in ((0, 1), (1, 3), (3, 4)):
+        sv = st2.rows(lo, hi)
+        m3.m3_scan_fwd(sv.dims, T, Q, *(g[k][lo:hi] for k in ("x", "B", "C", "dt", "A", "lam", "theta")),
+                       g["D"], sv, y2[lo:hi], ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert torch.equal(st1.h, st2.h) and torch.equal(st1.x_prev, st2.x_prev)
+    assert torch.equal(st1.B_prev, st2.B_prev)
