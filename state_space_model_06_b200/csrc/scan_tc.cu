@@ -720,15 +720,21 @@ __device__ void epilogue(const TcParams& p, const Unit& u, uint8_t* sm, uint64_t
 #pragma unroll
                 for (int j = 0; j < 16; j += 8) {
                     float m[8];
+                    // the R columns of one token share their mask value (colb + j is a
+                    // multiple of 8, so of R): one exp2 per token, not per column
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int col = colb + j + e;
-                        const float sv_f = __uint_as_float(sv[j + e]);
-                        // earlier tokens: decay times the trapezoid weight; the own token's
-                        // R columns: gamma (plus D on the diagonal); later tokens: 0
-                        const float v = sv_f * ex2_approx(ct + ew[col / R]);
-                        const float d = fmaf(sv_f, gt, col == lrow ? Dh : 0.f);
-                        m[e] = col < tR ? v : (col < tR + R ? d : 0.f);
+                    for (int e0 = 0; e0 < 8; e0 += R) {
+                        const int u = (colb + j + e0) / R;
+                        const float lv = ex2_approx(ct + ew[u]);
+#pragma unroll
+                        for (int rr = 0; rr < R; ++rr) {
+                            const int e = e0 + rr, col = colb + j + e;
+                            const float sv_f = __uint_as_float(sv[j + e]);
+                            // earlier tokens: decay times the trapezoid weight; the own
+                            // token's R columns: gamma (plus D on the diagonal); later: 0
+                            const float d = fmaf(sv_f, gt, col == lrow ? Dh : 0.f);
+                            m[e] = col < tR ? sv_f * lv : (col < tR + R ? d : 0.f);
+                        }
                     }
                     uint4 o;
                     o.x = pack_bf16x2(m[0], m[1]);
