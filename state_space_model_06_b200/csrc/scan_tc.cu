@@ -119,12 +119,15 @@ struct Cfg {
     static constexpr int kSmemLimit = 232448 - 1024;            // minus base alignment slack
     // with the output gate, every x / y stage has a z tile beside it
     static constexpr int XZ_BYTES = (GT ? 2 : 1) * X_BYTES;
-    // (operand slots, x stages, raw sub-chunk tokens): prefer two operand slots, then three
-    // x stages, then the largest raw sub-chunk that fits
+    // (operand slots, x stages, raw sub-chunk tokens): prefer two operand slots, then the
+    // largest raw sub-chunk, then three x stages.  Every raw sub-chunk costs the rotation warps
+    // an angle-sum exchange and a hand-off, so the sub-chunk size comes before the x stages:
+    // the rank-4 MIMO tile (N 64, 32 tokens) went from 8-token sub-chunks with 3 x stages to
+    // 16-token sub-chunks with 2, 1.84 -> 1.64 ms per 1.5B-scale MIMO call on B200.
     static constexpr int pick() {
         for (int ops = 2; ops >= 1; --ops)
-            for (int xst = 3; xst >= 2; --xst)
-                for (int rt = (Q < 32 ? Q : 32); rt >= TSPLIT; rt /= 2)
+            for (int rt = (Q < 32 ? Q : 32); rt >= TSPLIT; rt /= 2)
+                for (int xst = 3; xst >= 2; --xst)
                     if (Q % rt == 0 && rt % TSPLIT == 0 &&
                         base_bytes() + ops * SLOT_BYTES + xst * XZ_BYTES + 2 * raw_bytes(rt) <=
                             kSmemLimit)
