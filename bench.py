@@ -460,7 +460,9 @@ def backward_leg(args, w, d, g, dev, stream, rank, ws_world, pk):
     del ws, gr, dy
     return {"tokens_per_s": val, "ms_per_step": ms_max, "alg_bytes_per_step": reads + writes,
             "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"], "steps": steps,
-            "kernel": "scan_bwd_kernel (sequential fp32, segment checkpoints) + group sums"}
+            "kernel": "chunked tensor-core backward: bwd_vu_kernel (chunk products), "
+                      "bwd_scan_kernel (chunk states and adjoints), bwd_grads_kernel "
+                      "(chunk gradients), bwd_finish_kernel (angle carries)"}
 
 
 def longctx_leg(args, dev, stream, rank, ws_world, pk):

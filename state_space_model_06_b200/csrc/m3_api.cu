@@ -409,7 +409,12 @@ m3_status m3_scan_bwd_workspace_bytes(const m3_dims* d, int32_t seqlen, size_t* 
     if (seqlen < 0) return M3_ERR_SHAPE;
     const size_t fl = scan_bwd_workspace(d->batch, d->nheads, d->dstate, d->headdim, d->rank,
                                          seqlen).floats;
-    *bytes = kStatusBytes + ((fl * sizeof(float) + 255) / 256) * 256;
+    size_t need = ((fl * sizeof(float) + 255) / 256) * 256;
+    if (scan_bwd_tc_ok(d->io_dtype, d->dstate, d->headdim, d->rank)) {
+        const size_t tc = scan_bwd_tc_workspace_bytes(d->batch, d->nheads, d->dstate, seqlen);
+        if (tc > need) need = tc;
+    }
+    *bytes = kStatusBytes + need;
     return M3_OK;
 }
 
@@ -473,6 +478,23 @@ m3_status m3_scan_bwd(const m3_dims* d, int32_t seqlen, const void* x, const voi
         rc.status = static_cast<uint32_t*>(workspace);
         cudaError_t e = launch_range_checks(rc, d->io_dtype, s);
         if (e != cudaSuccess) return launch_status(e);
+    }
+    const bool tc = !(flags & M3_FLAG_FORCE_SIMT) && scan_bwd_tc_ok(d->io_dtype, N, P, R) &&
+                    aligned(gr->dx, 16) && aligned(gr->dB, 16) && aligned(gr->dC, 16);
+    if (tc) {
+        // the group-shared gradients and dD are accumulated with atomics
+        const size_t b = d->batch, T = seqlen, G = d->ngroups;
+        if (cudaMemsetAsync(gr->dB, 0, b * T * G * N * sizeof(float), s) != cudaSuccess ||
+            cudaMemsetAsync(gr->dC, 0, b * T * G * N * sizeof(float), s) != cudaSuccess ||
+            cudaMemsetAsync(gr->dtheta, 0, b * T * G * (N / 2) * sizeof(float), s) != cudaSuccess ||
+            cudaMemsetAsync(gr->dB_prev, 0, b * G * N * sizeof(float), s) != cudaSuccess ||
+            (D && gr->dD && cudaMemsetAsync(gr->dD, 0, d->nheads * sizeof(float), s) != cudaSuccess))
+            return M3_ERR_CUDA;
+        return launch_status(launch_scan_bwd_tc(a, static_cast<char*>(workspace) + kStatusBytes,
+                                                static_cast<uint32_t*>(workspace),
+                                                (flags & M3_FLAG_TEST_STALL) ? 50000000ull
+                                                                             : 2000000000ull,
+                                                s));
     }
     return launch_status(launch_scan_bwd(a, R, d->io_dtype, s));
 }

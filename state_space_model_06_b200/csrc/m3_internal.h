@@ -72,6 +72,14 @@ bool scan_bwd_shape_ok(int N, int P, int R);
 BwdWorkspace scan_bwd_workspace(int batch, int H, int N, int P, int R, long long T);
 cudaError_t launch_scan_bwd(const BwdArgs& a, int R, int io_dtype, cudaStream_t s);
 
+// chunked backward on the tensor cores (SISO, bf16 io, P 64, N 64 / 128): the shapes it
+// covers, its workspace bytes (after the status block) and the launch (four kernels; dB, dC,
+// dtheta, dB_prev and dD are accumulated with atomics and must be zero on entry)
+bool scan_bwd_tc_ok(int io_dtype, int N, int P, int R);
+size_t scan_bwd_tc_workspace_bytes(int batch, int H, int N, long long T);
+cudaError_t launch_scan_bwd_tc(const BwdArgs& a, void* ws, uint32_t* status,
+                               unsigned long long limit_ns, cudaStream_t s);
+
 // B_prev <- B[:, t] for every (batch, group): the previous-token input of the
 // next call, written after every head of the group has read the old value.
 cudaError_t launch_copy_prev(void* B_prev, const void* B, long long T, long long t, int batch,

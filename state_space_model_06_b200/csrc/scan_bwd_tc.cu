@@ -1,0 +1,1132 @@
+// scan_bwd_tc.cu -- chunked backward pass of the Mamba-3 recurrence on the tensor cores
+// (SISO, bf16 x / B / C / dy, P = 64, N in {64, 128}).
+//
+// Reverse-mode gradients of the chunked form ("Parallel representation under SSD", with the
+// rotation of Propositions 3 and 4).  Per chunk [t0, t1) of Q = 64 tokens, with cum the prefix
+// of the log-decays dt A, psi the prefix of the angles, B~ = R(-psi) B, C~ = R(-psi) C,
+//     gamma_s = lam_s dt_s,   w_s = gamma_s + (1 - lam_{s+1}) dt_{s+1},
+//     L[t, s] = e^{cum_t - cum_s} (gamma_s + [s < t] (1 - lam_{s+1}) dt_{s+1})    (s <= t),
+// and g the state entering the chunk (in the rotated frame), the forward is
+//     Y_t = e^{cum_t - m} C~_t g + sum_s L[t, s] (C~_t . B~_s) X_s + D X_t
+//     g  <- e^{cum_end - m} g + sum_s e^{cum_end - cum_s} w_s B~_s X_s^T.
+// The backward keeps the adjoint dg of g between chunks.  Four launches:
+//   1. chunk products, per (batch, head, chunk): V = B~^T diag(e w) X and U = C~^T diag(f) dY
+//      on the tensor cores (e_s = e^{cum_end - cum_s}, f_t = e^{cum_t - m}), in the chunk's own
+//      frame (angles counted from the chunk start), with the chunk's total log-decay and angles;
+//   2. chunk scan, per (batch, head): the state entering every chunk (forward) and the adjoint
+//      of the state leaving it (reverse), turned into the call's frame and stored as bf16
+//      operand tiles; the starting state's gradients and the dL/dh_T terms;
+//   3. chunk gradients, per (batch, head, chunk), on the tensor cores: S = C~ B~^T and
+//      dY X^T; the masked tiles L o S and dS = L o (dY X^T); then
+//          dX  = (L o S)^T dY + diag(e w) B~ dg + D dY,
+//          dC~ = dS B~ + diag(f) dY g^T,      dB~ = dS^T C~ + diag(e w) X dg^T,
+//      rotated back by R(psi); the log-decay, band-weight and angle chains from row and
+//      column sums of the same tiles;
+//   4. finish, per (batch, head, chunk): the angle gradient carried from later chunks and the
+//      next token's share of the trapezoid weight w of the chunk's last token.
+// Every reverse-mode term is the one the oracle's chunked route takes; the group-shared
+// gradients (B, C, theta, B_prev) and dD are added with atomics, so their last bits may vary
+// from run to run.  Every wait is bounded; a timeout writes M3_ERR_TIMEOUT to the status word.
+#include <cuda_bf16.h>
+
+#include "m3_internal.h"
+#include "sm100.cuh"
+
+namespace m3 {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kQ = 64;     // chunk tokens
+constexpr int kPc = 64;    // head channels
+constexpr float kTwoPi = 6.28318530717958647692f;
+constexpr float kInvTwoPi = 0.15915494309189533577f;
+constexpr float kLog2e = 1.44269504088896340736f;
+
+struct TcBwd {
+    BwdArgs a;
+    int nch;                  // chunks of the call
+    float* V;                 // [BH][nch][N][P] chunk-frame state products
+    float* U;                 // [BH][nch][N][P] chunk-frame adjoint products
+    uint16_t* gin;            // [BH][nch] bf16 tile images [N][P] of the entering state
+    uint16_t* dgo;            // [BH][nch] bf16 tile images [N][P] of the leaving adjoint
+    float* ctot;              // [BH][nch] total log-decay of the chunk
+    float* atot;              // [BH][nch][N/2] total angle of the chunk
+    float* P0;                // [BH][nch + 1][N/2] angle before the chunk (mod 2 pi)
+    float* q;                 // [BH][nch] e^{ctot} <dg_out, g_in>
+    float* dtot;              // [BH][nch][N/2] sum of the chunk's angle gradients
+    float* spill;             // [BH][nch] band-weight gradient owed to the next token
+    float* extra;             // [BH][N/2] angle gradient of the last token from dL/dh_T
+    float* v0;                // [BH] <dg_0, B_prev x_prev^T>
+    uint32_t* status;
+    unsigned long long limit_ns;
+};
+
+__device__ __forceinline__ float wrap_angle(float x) {
+    return fmaf(-kTwoPi, rintf(x * kInvTwoPi), x);
+}
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float bf_at(const void* base, size_t i) {
+    return __uint_as_float((uint32_t)(static_cast<const uint16_t*>(base)[i]) << 16);
+}
+__device__ __forceinline__ uint16_t to_bf(float v) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+__device__ __forceinline__ uint32_t scale2(uint32_t v, float s) {
+    return pack_bf16x2(bf16lo(v) * s, bf16hi(v) * s);
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ bool warp_wait_b(uint64_t* bar, uint32_t parity, const Abort& ab) {
+    const bool r = mbar_wait(bar, parity, ab);
+    return __all_sync(0xffffffffu, r);
+}
+__device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity, uint64_t ns) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < ns) {
+    }
+}
+
+// K-major SW128 operand (rows of 64 elements, 128 B), K step kk of 16 elements; 64-element
+// K atoms are rows * 128 B apart.
+__device__ __forceinline__ uint64_t bdesc_k(uint32_t base, int kk, int rows) {
+    return sdesc_sw128(base + (uint32_t)(kk >> 2) * rows * 128u + (uint32_t)(kk & 3) * 32u, 16u,
+                       1024u);
+}
+// MN-major SW128 operand (each 128 B row holds 64 MN elements of one K index), K step kk of
+// 16 rows; 64-element MN atoms are `lbo` bytes apart.
+__device__ __forceinline__ uint64_t bdesc_mn(uint32_t base, int kk, uint32_t lbo) {
+    return sdesc_sw128(base + (uint32_t)kk * 2048u, lbo, 1024u);
+}
+// byte offset of element (row, col) in a tile of `rows` rows whose columns come in 64-wide
+// SW128 atoms placed rows * 128 B apart
+__device__ __forceinline__ uint32_t tile_off(int row, int col, int rows) {
+    return (uint32_t)(col >> 6) * rows * 128u + sw128_off(row, col & 63);
+}
+
+// Per-token coefficients of tokens [t0, t0 + Q) of (b, h), by one warp, into shared arrays.
+// Tokens past T have dt = A = lam = 0 (no decay, no input).  u = Q is the next chunk's first
+// token (its dt and lam give the last token's trapezoid share).
+struct Coefs {
+    float* dd;    // dt          [Q + 1]
+    float* ll;    // lam         [Q + 1]
+    float* aa;    // A           [Q]
+    float* cr;    // chunk-relative inclusive prefix of dt A   [Q]
+    float* gam;   // lam dt      [Q]
+    float* nx;    // (1 - lam_{u+1}) dt_{u+1}   [Q]
+    float* ew;    // e_u w_u     [Q]
+    float* ee;    // e_u = e^{cr_{Q-1} - cr_u}  [Q]
+    float* ff;    // f_u = e^{cr_u}             [Q]
+    __device__ explicit Coefs(float* base) {
+        dd = base;
+        ll = dd + kQ + 1;
+        aa = ll + kQ + 1;
+        cr = aa + kQ;
+        gam = cr + kQ;
+        nx = gam + kQ;
+        ew = nx + kQ;
+        ee = ew + kQ;
+        ff = ee + kQ;
+    }
+    static constexpr int kFloats = 2 * (kQ + 1) + 7 * kQ;
+};
+
+__device__ void chunk_coefs(const BwdArgs& a, int b, int h, long long t0, const Coefs& k) {
+    const int lane = threadIdx.x & 31;
+    const long long T = a.T;
+    float d2[2], l2[2], a2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const long long t = t0 + 2 * lane + i;
+        const bool ok = t < T;
+        const size_t o = ((size_t)b * T + (ok ? t : 0)) * a.H + h;
+        d2[i] = ok ? a.dt[o] : 0.f;
+        l2[i] = ok ? a.lam[o] : 0.f;
+        a2[i] = ok ? a.A[o] : 0.f;
+    }
+    const float e0 = d2[0] * a2[0], e1 = d2[1] * a2[1];
+    float s = e0 + e1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += v;
+    }
+    const float cend = __shfl_sync(0xffffffffu, s, 31);
+    const float c0 = (s - (e0 + e1)) + e0, c1 = c0 + e1;
+    const float cc[2] = {c0, c1};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int u = 2 * lane + i;
+        k.dd[u] = d2[i];
+        k.ll[u] = l2[i];
+        k.aa[u] = a2[i];
+        k.cr[u] = cc[i];
+        k.gam[u] = l2[i] * d2[i];
+        k.ee[u] = ex2f((cend - cc[i]) * kLog2e);
+        k.ff[u] = ex2f(cc[i] * kLog2e);
+    }
+    if (lane == 0) {
+        const long long t = t0 + kQ;
+        const bool ok = t < T;
+        const size_t o = ((size_t)b * T + (ok ? t : 0)) * a.H + h;
+        k.dd[kQ] = ok ? a.dt[o] : 0.f;
+        k.ll[kQ] = ok ? a.lam[o] : 0.f;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int u = 2 * lane + i;
+        const float nx = (1.f - k.ll[u + 1]) * k.dd[u + 1];
+        k.nx[u] = nx;
+        k.ew[u] = k.ee[u] * (k.gam[u] + nx);
+    }
+    __syncwarp();
+}
+
+// ------------------------------------------------------------------------------------
+// 1. chunk products
+template <int NST>
+struct VuCfg {
+    static constexpr int NH = NST / 2;
+    static constexpr int OFF_B = 0;                          // B~ [NST/64][Q][64] bf16
+    static constexpr int OFF_C = kQ * NST * 2;               // C~
+    static constexpr int OFF_XW = 2 * kQ * NST * 2;          // diag(e w) X [Q][64]
+    static constexpr int OFF_DYF = OFF_XW + kQ * kPc * 2;    // diag(f) dY [Q][64]
+    static constexpr int OFF_COEF = OFF_DYF + kQ * kPc * 2;
+    static constexpr int OFF_BAR = (OFF_COEF + Coefs::kFloats * 4 + 7) / 8 * 8;
+    static constexpr int OFF_MISC = OFF_BAR + 8;
+    static constexpr int USED = OFF_MISC + 16 + 1024;
+    // at least 50 KB, so that at most four CTAs (4 x 128 TMEM columns) share an SM
+    static constexpr int SMEM = USED > 51200 ? USED : 51200;
+    static constexpr uint32_t ID = idesc_bf16(NST, kPc, true, true);
+    static_assert(SMEM * 5 > 233472 && SMEM * 4 <= 233472 - 4096, "four CTAs per SM");
+};
+
+template <int NST>
+__global__ void __launch_bounds__(128) bwd_vu_kernel(const __grid_constant__ TcBwd p) {
+    using C = VuCfg<NST>;
+    constexpr int NH = C::NH;
+    const BwdArgs& a = p.a;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+    const Coefs k(reinterpret_cast<float*>(sm + C::OFF_COEF));
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int c = (int)(blockIdx.x % p.nch);
+    const size_t bh = blockIdx.x / p.nch;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H), g = h / (a.H / a.G);
+    const long long t0 = (long long)c * kQ;
+    const size_t cc = bh * p.nch + c;
+
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        misc[1] = 0u;
+        fence_mbar_init();
+    }
+    if (w == 1) {
+        tmem_alloc(&misc[0], 128);
+        tmem_relinquish();
+    }
+    if (w == 0) chunk_coefs(a, b, h, t0, k);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    const Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.status, p.limit_ns};
+    if (tid == 0) p.ctot[cc] = k.cr[kQ - 1];
+
+    // B~, C~ in the chunk's frame: thread j (B) and NH + j (C) walk the chunk's tokens
+    if (tid < 2 * NH) {
+        const bool isC = tid >= NH;
+        const int j = isC ? tid - NH : tid;
+        const uint16_t* src = static_cast<const uint16_t*>(isC ? a.C : a.B);
+        uint8_t* tile = sm + (isC ? C::OFF_C : C::OFF_B);
+        const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
+        float rho = 0.f;
+#pragma unroll 4
+        for (int u = 0; u < kQ; ++u) {
+            const long long t = t0 + u;
+            float v0 = 0.f, v1 = 0.f, th = 0.f;
+            if (t < a.T) {
+                const size_t row = ((size_t)b * a.T + t) * a.G + g;
+                const uint32_t pr = *reinterpret_cast<const uint32_t*>(src + row * NST + 2 * j);
+                v0 = bf16lo(pr);
+                v1 = bf16hi(pr);
+                th = a.theta[row * NH + j];
+            }
+            rho += angle ? th : k.dd[u] * th;
+            float sn, cs;
+            __sincosf(wrap_angle(rho), &sn, &cs);
+            *reinterpret_cast<uint32_t*>(tile + tile_off(u, 2 * j, kQ)) =
+                pack_bf16x2(fmaf(cs, v0, sn * v1), fmaf(cs, v1, -sn * v0));
+        }
+        if (!isC) p.atot[cc * NH + j] = rho;
+    }
+    // diag(e w) X and diag(f) dY
+    {
+        const uint16_t* xg = static_cast<const uint16_t*>(a.x);
+        const uint16_t* yg = static_cast<const uint16_t*>(a.dy);
+        for (int i = tid; i < 2 * kQ * 8; i += 128) {
+            const bool isY = i >= kQ * 8;
+            const int e = isY ? i - kQ * 8 : i;
+            const int u = e >> 3, ch = e & 7;
+            const long long t = t0 + u;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (t < a.T)
+                v = *reinterpret_cast<const uint4*>((isY ? yg : xg) +
+                                                    (((size_t)b * a.T + t) * a.H + h) * kPc + ch * 8);
+            const float s = isY ? k.ff[u] : k.ew[u];
+            const uint4 o = make_uint4(scale2(v.x, s), scale2(v.y, s), scale2(v.z, s), scale2(v.w, s));
+            *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DYF : C::OFF_XW) + sw128_off(u, ch * 8)) = o;
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t sb = smem_u32(sm);
+#pragma unroll
+        for (int kk = 0; kk < kQ / 16; ++kk)
+            mma_bf16(tmem, bdesc_mn(sb + C::OFF_B, kk, kQ * 128), bdesc_mn(sb + C::OFF_XW, kk, kQ * 128),
+                     C::ID, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < kQ / 16; ++kk)
+            mma_bf16(tmem + 64, bdesc_mn(sb + C::OFF_C, kk, kQ * 128),
+                     bdesc_mn(sb + C::OFF_DYF, kk, kQ * 128), C::ID, kk > 0);
+        mma_commit(&bar[0]);
+    }
+    const bool ok = warp_wait_b(&bar[0], 0, ab);
+    tc_fence_after();
+    if (ok) {
+        const int q = w & 3;
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+        float* Vo = p.V + cc * (size_t)NST * kPc;
+        float* Uo = p.U + cc * (size_t)NST * kPc;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            float* dst0 = m ? Uo : Vo;
+#pragma unroll
+            for (int cb = 0; cb < 32; cb += 16) {
+                uint32_t r[16], r2[16];
+                int n, col, col2;
+                if constexpr (NST == 128) {   // M = 128: row = lane of the quadrant
+                    tmem_ld_32x32b_x16(tq + 64 * m + 2 * cb, r);
+                    tmem_ld_32x32b_x16(tq + 64 * m + 2 * cb + 16, r2);
+                    n = 32 * q + lane;
+                    col = 2 * cb;
+                    col2 = 2 * cb + 16;
+                } else {                      // M = 64: 16 rows per quadrant, column halves
+                    tmem_ld_16x32bx2_x16<32>(tq + 64 * m + cb, r);
+                    n = 16 * q + (lane & 15);
+                    col = cb + 32 * (lane >> 4);
+                    col2 = -1;
+                }
+                tmem_wait_ld();
+                float4* d = reinterpret_cast<float4*>(dst0 + (size_t)n * kPc + col);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    d[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                       __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                if (col2 >= 0) {
+                    float4* d2 = reinterpret_cast<float4*>(dst0 + (size_t)n * kPc + col2);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        d2[i] = make_float4(__uint_as_float(r2[4 * i]), __uint_as_float(r2[4 * i + 1]),
+                                            __uint_as_float(r2[4 * i + 2]), __uint_as_float(r2[4 * i + 3]));
+                }
+            }
+        }
+    }
+    if (tid == 0 && !ok) drain(&bar[0], 0, 100000000ull);
+    tc_fence_before();
+    __syncthreads();
+    if (w == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// 2. chunk scan: thread (channel p, pair group pg) holds state rows 2j, 2j+1 of column p for
+// the pairs j = pg + NPG k, k < 8.
+template <int NST>
+__global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant__ TcBwd p) {
+    constexpr int NH = NST / 2, NPG = NST / 16, NT = 4 * NST, NW = NT / 32;
+    const BwdArgs& a = p.a;
+    __shared__ float red[2][NW];
+    __shared__ float part[NPG][kPc];
+    __shared__ float exs[NH];
+    const int tid = threadIdx.x, pc = tid & 63, pg = tid >> 6, lane = tid & 31, w = tid >> 5;
+    const size_t bh = blockIdx.x;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H), g = h / (a.H / a.G);
+    const int nch = p.nch;
+    const size_t NP = (size_t)NST * kPc;
+    if (tid < NH) exs[tid] = 0.f;
+    __syncthreads();
+
+    // starting state g0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T
+    const size_t o0 = (size_t)b * a.T * a.H + h;
+    const float k0 = (1.f - a.lam[o0]) * a.dt[o0];
+    const float xp = bf_at(a.x_prev, bh * kPc + pc);
+    float ge[8], go[8], bpe[8], bpo[8], P[8];
+#pragma unroll
+    for (int kx = 0; kx < 8; ++kx) {
+        const int j = pg + NPG * kx;
+        const size_t bp = ((size_t)b * a.G + g) * NST + 2 * j;
+        bpe[kx] = bf_at(a.B_prev, bp);
+        bpo[kx] = bf_at(a.B_prev, bp + 1);
+        ge[kx] = fmaf(k0 * bpe[kx], xp, a.h0[bh * NP + (size_t)(2 * j) * kPc + pc]);
+        go[kx] = fmaf(k0 * bpo[kx], xp, a.h0[bh * NP + (size_t)(2 * j + 1) * kPc + pc]);
+        P[kx] = 0.f;
+    }
+    // forward: the state entering every chunk, then the chunk's contribution in the call frame
+    for (int c = 0; c < nch; ++c) {
+        const size_t cc = bh * nch + c;
+        uint8_t* gt = reinterpret_cast<uint8_t*>(p.gin) + cc * NP * 2;
+        const float* V = p.V + cc * NP;
+        const float dec = ex2f(p.ctot[cc] * kLog2e);
+#pragma unroll
+        for (int kx = 0; kx < 8; ++kx) {
+            const int j = pg + NPG * kx;
+            if (pc == 0) p.P0[(bh * (nch + 1) + c) * NH + j] = P[kx];
+            *reinterpret_cast<uint16_t*>(gt + sw128_off(2 * j, pc)) = to_bf(ge[kx]);
+            *reinterpret_cast<uint16_t*>(gt + sw128_off(2 * j + 1, pc)) = to_bf(go[kx]);
+            const float v0 = V[(size_t)(2 * j) * kPc + pc], v1 = V[(size_t)(2 * j + 1) * kPc + pc];
+            float sn, cs;
+            __sincosf(P[kx], &sn, &cs);
+            ge[kx] = fmaf(dec, ge[kx], fmaf(cs, v0, sn * v1));
+            go[kx] = fmaf(dec, go[kx], fmaf(cs, v1, -sn * v0));
+            P[kx] = wrap_angle(P[kx] + p.atot[cc * NH + j]);
+        }
+    }
+    // the final state and dL/dh_T: dg = R(-psi_T) dH; the last token's angle gradient
+    // sum_p dH_odd (R(psi_T) g)_even - dH_even (R(psi_T) g)_odd
+    float de[8], dq[8];
+#pragma unroll
+    for (int kx = 0; kx < 8; ++kx) {
+        const int j = pg + NPG * kx;
+        if (pc == 0) p.P0[(bh * (nch + 1) + nch) * NH + j] = P[kx];
+        de[kx] = 0.f;
+        dq[kx] = 0.f;
+        if (a.dhT) {
+            float sn, cs;
+            __sincosf(P[kx], &sn, &cs);
+            const float d0 = a.dhT[bh * NP + (size_t)(2 * j) * kPc + pc];
+            const float d1 = a.dhT[bh * NP + (size_t)(2 * j + 1) * kPc + pc];
+            de[kx] = fmaf(cs, d0, sn * d1);
+            dq[kx] = fmaf(cs, d1, -sn * d0);
+            const float h0 = fmaf(cs, ge[kx], -sn * go[kx]), h1 = fmaf(sn, ge[kx], cs * go[kx]);
+            const float ex = warp_sum(fmaf(d1, h0, -d0 * h1));
+            if (lane == 0) atomicAdd(&exs[j], ex);
+        }
+    }
+    __syncthreads();   // the chunk-start angles (global) and exs are complete
+    if (tid < NH) p.extra[bh * NH + tid] = exs[tid];
+    // reverse: the adjoint of the state leaving every chunk
+    for (int c = nch - 1; c >= 0; --c) {
+        const size_t cc = bh * nch + c;
+        uint8_t* dt_ = reinterpret_cast<uint8_t*>(p.dgo) + cc * NP * 2;
+        const uint8_t* gt = reinterpret_cast<const uint8_t*>(p.gin) + cc * NP * 2;
+        const float* Uc = p.U + cc * NP;
+        const float dec = ex2f(p.ctot[cc] * kLog2e);
+        float s = 0.f;
+#pragma unroll
+        for (int kx = 0; kx < 8; ++kx) {
+            const int j = pg + NPG * kx;
+            *reinterpret_cast<uint16_t*>(dt_ + sw128_off(2 * j, pc)) = to_bf(de[kx]);
+            *reinterpret_cast<uint16_t*>(dt_ + sw128_off(2 * j + 1, pc)) = to_bf(dq[kx]);
+            const float g0 = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j, pc)) << 16);
+            const float g1 = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j + 1, pc)) << 16);
+            s = fmaf(de[kx], g0, fmaf(dq[kx], g1, s));
+            const float u0 = Uc[(size_t)(2 * j) * kPc + pc], u1 = Uc[(size_t)(2 * j + 1) * kPc + pc];
+            float sn, cs;
+            __sincosf(p.P0[(bh * (nch + 1) + c) * NH + j], &sn, &cs);
+            de[kx] = fmaf(dec, de[kx], fmaf(cs, u0, sn * u1));
+            dq[kx] = fmaf(dec, dq[kx], fmaf(cs, u1, -sn * u0));
+        }
+        s = warp_sum(s);
+        if (lane == 0) red[c & 1][w] = s;
+        __syncthreads();
+        if (tid == 0) {
+            float t = 0.f;
+            for (int i = 0; i < NW; ++i) t += red[c & 1][i];
+            p.q[cc] = dec * t;
+        }
+    }
+    // the starting state: dh0 = dg; dx_prev = k0 B_prev^T dg; dB_prev += k0 dg x_prev;
+    // v0 = <dg, B_prev x_prev^T> (for dt_0 and lam_0)
+    float pp = 0.f;
+#pragma unroll
+    for (int kx = 0; kx < 8; ++kx) {
+        const int j = pg + NPG * kx;
+        a.dh0[bh * NP + (size_t)(2 * j) * kPc + pc] = de[kx];
+        a.dh0[bh * NP + (size_t)(2 * j + 1) * kPc + pc] = dq[kx];
+        pp = fmaf(de[kx], bpe[kx], fmaf(dq[kx], bpo[kx], pp));
+        const float se = warp_sum(de[kx] * xp), so = warp_sum(dq[kx] * xp);
+        if (lane == 0) {
+            float* db = a.dB_prev + ((size_t)b * a.G + g) * NST + 2 * j;
+            atomicAdd(db, k0 * se);
+            atomicAdd(db + 1, k0 * so);
+        }
+    }
+    part[pg][pc] = pp;
+    const float sv = warp_sum(pp * xp);
+    __syncthreads();
+    if (lane == 0) red[0][w] = sv;
+    if (tid < kPc) {
+        float t = 0.f;
+        for (int i = 0; i < NPG; ++i) t += part[i][tid];
+        a.dx_prev[bh * kPc + tid] = k0 * t;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float t = 0.f;
+        for (int i = 0; i < NW; ++i) t += red[0][i];
+        p.v0[bh] = t;
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// 3. chunk gradients
+template <int NST>
+struct GrCfg {
+    static constexpr int NH = NST / 2;
+    static constexpr int T64 = kQ * 128;                      // one [Q][64] bf16 tile
+    static constexpr int OFF_X = 0, OFF_DY = T64, OFF_MS = 2 * T64, OFF_DS = 3 * T64;
+    static constexpr int OFF_C = 4 * T64;                     // C~ [NST/64][Q][64]
+    static constexpr int OFF_B = OFF_C + kQ * NST * 2;        // B~
+    static constexpr int OFF_GIN = OFF_B + kQ * NST * 2;      // g_in [NST][64]
+    static constexpr int OFF_DG = OFF_GIN + NST * kPc * 2;    // dg_out [NST][64]
+    static constexpr int PSI_LD = NH + 1;
+    static constexpr int OFF_PSI = OFF_DG + NST * kPc * 2;    // fp32 [Q][NH + 1]
+    static constexpr int OFF_SEG = OFF_PSI + kQ * PSI_LD * 4; // fp32 [256 / NH][NH]
+    static constexpr int OFF_COEF = OFF_SEG + 256 * 4;
+    static constexpr int NACC = 9;
+    static constexpr int OFF_ACC = OFF_COEF + Coefs::kFloats * 4;
+    static constexpr int OFF_BAR = (OFF_ACC + (NACC * kQ + 4) * 4 + 7) / 8 * 8;
+    static constexpr int OFF_MISC = OFF_BAR + 3 * 8;
+    static constexpr int USED = OFF_MISC + 16 + 1024;
+    // at least 120 KB: one CTA per SM (each allocates all 512 TMEM columns)
+    static constexpr int SMEM = USED > 122880 ? USED : 122880;
+    static_assert(SMEM <= 232448, "shared memory budget exceeded");
+    static constexpr uint32_t TM_S = 0, TM_GX = 64, TM_DX = 128, TM_DC = 192, TM_DB = 192 + NST;
+    static constexpr uint32_t ID_QQ = idesc_bf16(kQ, kQ, false, false);    // S, dY X^T
+    static constexpr uint32_t ID_BDG = idesc_bf16(kQ, kPc, false, true);   // B~ dg
+    static constexpr uint32_t ID_KN = idesc_bf16(kQ, NST, false, false);   // dY g^T, X dg^T
+    static constexpr uint32_t ID_MSDY = idesc_bf16(kQ, kPc, true, true);   // (L o S)^T dY
+    static constexpr uint32_t ID_DSB = idesc_bf16(kQ, NST, false, true);   // dS B~
+    static constexpr uint32_t ID_DSC = idesc_bf16(kQ, NST, true, true);    // dS^T C~
+};
+
+// TMEM access of an M = 64 accumulator by 8 warps: warp w reaches lane quadrant w % 4 (rows
+// 16 q .. 16 q + 15 at lanes 32 q .. 32 q + 15); 16-column blocks cb of the first half go to
+// warp group w / 4 in turn; a thread's lane half (lane / 16) takes block cb + NC / 2.
+template <int NC>
+__device__ __forceinline__ void ld_blk(uint32_t tq, uint32_t col, int cb, uint32_t (&r)[16]) {
+    tmem_ld_16x32bx2_x16<NC / 2>(tq + col + cb, r);
+}
+template <int NC>
+__device__ __forceinline__ void st_blk(uint32_t tq, uint32_t col, int cb, const uint32_t (&r)[16]) {
+    tmem_st_16x32bx2_x16<NC / 2>(tq + col + cb, r);
+}
+
+// sum over the 16 lanes of a half warp of 16 per-lane column values: lane l ends with the
+// sum of column l % 16 (recursive halving: 15 shuffles)
+__device__ __forceinline__ float colsum16(float (&v)[16], int lane) {
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+            const float send = up ? v[i] : v[i + o];
+            const float keep = up ? v[i + o] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
+template <int NST>
+__global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant__ TcBwd p) {
+    using C = GrCfg<NST>;
+    constexpr int NH = C::NH, PSI_LD = C::PSI_LD;
+    const BwdArgs& a = p.a;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+    const Coefs k(reinterpret_cast<float*>(sm + C::OFF_COEF));
+    float* acc = reinterpret_cast<float*>(sm + C::OFF_ACC);
+    float* rs = acc;              // row sums of dL om E
+    float* cs = acc + kQ;         // column sums of dL om E
+    float* ga = acc + 2 * kQ;     // column sums of dL E over t >= s
+    float* dgd = acc + 3 * kQ;    // diagonal dL E
+    float* dv = acc + 4 * kQ;     // <X_s, (B~ dg)_s>
+    float* qz = acc + 5 * kQ;     // <C~_t, (dY g^T)_t>
+    float* dcm = acc + 6 * kQ;    // log-decay gradient, then its suffix sums
+    float* dnx = acc + 7 * kQ;    // band-weight gradient owed to the next token
+    float* misc2 = acc + 8 * kQ;  // [0] dD partial, [1..2] warp sums
+    float* psi = reinterpret_cast<float*>(sm + C::OFF_PSI);
+    float* segt = reinterpret_cast<float*>(sm + C::OFF_SEG);
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int c = (int)(blockIdx.x % p.nch);
+    const size_t bh = blockIdx.x / p.nch;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H), g = h / (a.H / a.G);
+    const long long t0 = (long long)c * kQ;
+    const int nv = (int)(a.T - t0 < kQ ? a.T - t0 : kQ);
+    const size_t cc = bh * p.nch + c;
+    const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
+    const uint32_t tile_bytes = NST * kPc * 2;
+
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+        misc[1] = 0u;
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar[0], 2 * tile_bytes);
+        bulk_load(sm + C::OFF_GIN, reinterpret_cast<const uint8_t*>(p.gin) + cc * tile_bytes,
+                  tile_bytes, &bar[0]);
+        bulk_load(sm + C::OFF_DG, reinterpret_cast<const uint8_t*>(p.dgo) + cc * tile_bytes,
+                  tile_bytes, &bar[0]);
+    }
+    if (w == 0) {
+        __syncwarp();
+        tmem_alloc(&misc[0], 512);
+        tmem_relinquish();
+    }
+    if (w == 1) chunk_coefs(a, b, h, t0, k);
+    for (int i = tid; i < C::NACC * kQ + 4; i += 256) acc[i] = 0.f;
+    // angles: thread (pair j, token segment sg) sums its segment's angles
+    constexpr int SEGS = 256 / NH, TPS = kQ / SEGS;
+    const int jj = tid % NH, sg = tid / NH;
+    float rho[TPS];
+    {
+        float r = 0.f;
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) {
+            const long long t = t0 + sg * TPS + i;
+            float th = 0.f, d = 0.f;
+            if (t < a.T) {
+                th = a.theta[(((size_t)b * a.T + t) * a.G + g) * NH + jj];
+                d = a.dt[((size_t)b * a.T + t) * a.H + h];
+            }
+            r += angle ? th : d * th;
+            rho[i] = r;
+        }
+        segt[sg * NH + jj] = r;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    const Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.status, p.limit_ns};
+    {
+        float off = p.P0[(bh * (p.nch + 1) + c) * NH + jj];
+        for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + jj];
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) psi[(sg * TPS + i) * PSI_LD + jj] = wrap_angle(off + rho[i]);
+    }
+    // X and dY tiles
+    {
+        const uint16_t* xg = static_cast<const uint16_t*>(a.x);
+        const uint16_t* yg = static_cast<const uint16_t*>(a.dy);
+        for (int i = tid; i < 2 * kQ * 8; i += 256) {
+            const bool isY = i >= kQ * 8;
+            const int e = isY ? i - kQ * 8 : i;
+            const int u = e >> 3, ch = e & 7;
+            const long long t = t0 + u;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (t < a.T)
+                v = *reinterpret_cast<const uint4*>((isY ? yg : xg) +
+                                                    (((size_t)b * a.T + t) * a.H + h) * kPc + ch * 8);
+            *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DY : C::OFF_X) + sw128_off(u, ch * 8)) = v;
+        }
+    }
+    __syncthreads();   // psi complete
+    // B~, C~ in the call frame: thread (pair j, token u) for tasks i = tid + 256 m
+    {
+        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
+        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
+        for (int i = tid; i < kQ * NH; i += 256) {
+            const int j = i % NH, u = i / NH;
+            const long long t = t0 + u;
+            uint32_t pb = 0u, pcv = 0u;
+            if (t < a.T) {
+                const size_t row = (((size_t)b * a.T + t) * a.G + g) * NST + 2 * j;
+                pb = *reinterpret_cast<const uint32_t*>(Bg + row);
+                pcv = *reinterpret_cast<const uint32_t*>(Cg + row);
+            }
+            float sn, cs2;
+            __sincosf(psi[u * PSI_LD + j], &sn, &cs2);
+            const float b0 = bf16lo(pb), b1 = bf16hi(pb), c0 = bf16lo(pcv), c1 = bf16hi(pcv);
+            const uint32_t off = tile_off(u, 2 * j, kQ);
+            *reinterpret_cast<uint32_t*>(sm + C::OFF_B + off) =
+                pack_bf16x2(fmaf(cs2, b0, sn * b1), fmaf(cs2, b1, -sn * b0));
+            *reinterpret_cast<uint32_t*>(sm + C::OFF_C + off) =
+                pack_bf16x2(fmaf(cs2, c0, sn * c1), fmaf(cs2, c1, -sn * c0));
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    const uint32_t sb = smem_u32(sm);
+    int issued = 0;   // thread 0: MMA batches issued
+    if (tid == 0) {
+        if (mbar_wait(&bar[0], 0, ab)) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < NST / 16; ++kk)
+                mma_bf16(tmem + C::TM_S, bdesc_k(sb + C::OFF_C, kk, kQ), bdesc_k(sb + C::OFF_B, kk, kQ),
+                         C::ID_QQ, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < kPc / 16; ++kk)
+                mma_bf16(tmem + C::TM_GX, bdesc_k(sb + C::OFF_DY, kk, kQ), bdesc_k(sb + C::OFF_X, kk, kQ),
+                         C::ID_QQ, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < NST / 16; ++kk)
+                mma_bf16(tmem + C::TM_DX, bdesc_k(sb + C::OFF_B, kk, kQ),
+                         bdesc_mn(sb + C::OFF_DG, kk, tile_bytes), C::ID_BDG, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < kPc / 16; ++kk)
+                mma_bf16(tmem + C::TM_DC, bdesc_k(sb + C::OFF_DY, kk, kQ),
+                         bdesc_k(sb + C::OFF_GIN, kk, NST), C::ID_KN, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < kPc / 16; ++kk)
+                mma_bf16(tmem + C::TM_DB, bdesc_k(sb + C::OFF_X, kk, kQ),
+                         bdesc_k(sb + C::OFF_DG, kk, NST), C::ID_KN, kk > 0);
+            mma_commit(&bar[1]);
+            issued = 1;
+        } else {
+            // nothing issued: let the copies land before the CTA exits
+            drain(&bar[0], 0, 100000000ull);
+        }
+    }
+
+    // ---- first epilogue: masks, band and decay sums, state-term dot products, row scales
+    const int q4 = w & 3, wg = w >> 2, hf = lane >> 4;
+    const int t = 16 * q4 + (lane & 15);          // this thread's accumulator row
+    const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
+    bool ok = warp_wait_b(&bar[1], 0, ab);
+    tc_fence_after();
+    if (ok) {
+        const float crt = k.cr[t];
+        // S and dY X^T: columns cb + 32 hf + i
+        {
+            const int cb = 16 * wg, col0 = cb + 32 * hf;
+            uint32_t sv[16], gv[16];
+            ld_blk<64>(tq, C::TM_S, cb, sv);
+            ld_blk<64>(tq, C::TM_GX, cb, gv);
+            tmem_wait_ld();
+            float ca[16], cbv[16], rsum = 0.f, ddiag = 0.f;
+            uint32_t ms[8], ds[8];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                float mv[2], dvv[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int s = col0 + i + e;
+                    const bool in = s <= t;
+                    const float E = in ? ex2f((crt - k.cr[s]) * kLog2e) : 0.f;
+                    const float om = in ? k.gam[s] + (s < t ? k.nx[s] : 0.f) : 0.f;
+                    const float L = E * om;
+                    const float S = __uint_as_float(sv[i + e]), G = __uint_as_float(gv[i + e]);
+                    mv[e] = S * L;
+                    dvv[e] = G * L;
+                    const float dL = S * G;
+                    const float dom = dL * E;
+                    ca[i + e] = dom * om;
+                    cbv[i + e] = dom;
+                    rsum += dom * om;
+                    if (s == t) {
+                        dgd[t] = dom;
+                        ddiag = G;
+                    }
+                }
+                ms[i / 2] = pack_bf16x2(mv[0], mv[1]);
+                ds[i / 2] = pack_bf16x2(dvv[0], dvv[1]);
+            }
+            *reinterpret_cast<uint4*>(sm + C::OFF_MS + sw128_off(t, col0)) = make_uint4(ms[0], ms[1], ms[2], ms[3]);
+            *reinterpret_cast<uint4*>(sm + C::OFF_MS + sw128_off(t, col0 + 8)) = make_uint4(ms[4], ms[5], ms[6], ms[7]);
+            *reinterpret_cast<uint4*>(sm + C::OFF_DS + sw128_off(t, col0)) = make_uint4(ds[0], ds[1], ds[2], ds[3]);
+            *reinterpret_cast<uint4*>(sm + C::OFF_DS + sw128_off(t, col0 + 8)) = make_uint4(ds[4], ds[5], ds[6], ds[7]);
+            if (ddiag != 0.f) atomicAdd(&misc2[0], ddiag);
+            const float csum = colsum16(ca, lane), gsum = colsum16(cbv, lane);
+            atomicAdd(&cs[col0 + (lane & 15)], csum);
+            atomicAdd(&ga[col0 + (lane & 15)], gsum);
+            rsum += __shfl_xor_sync(0xffffffffu, rsum, 16);
+            if (hf == 0) atomicAdd(&rs[t], rsum);
+        }
+        // B~ dg: <X_s, .> for the state-update weight, then the row scale e_s w_s
+        {
+            const int cb = 16 * wg, col0 = cb + 32 * hf;
+            uint32_t v[16];
+            ld_blk<64>(tq, C::TM_DX, cb, v);
+            tmem_wait_ld();
+            const uint4 x0 = *reinterpret_cast<const uint4*>(sm + C::OFF_X + sw128_off(t, col0));
+            const uint4 x1 = *reinterpret_cast<const uint4*>(sm + C::OFF_X + sw128_off(t, col0 + 8));
+            const uint32_t xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            float d = 0.f;
+            const float sc = k.ew[t];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
+                d = fmaf(bf16lo(xs[i]), a0, fmaf(bf16hi(xs[i]), a1, d));
+                v[2 * i] = __float_as_uint(a0 * sc);
+                v[2 * i + 1] = __float_as_uint(a1 * sc);
+            }
+            st_blk<64>(tq, C::TM_DX, cb, v);
+            d += __shfl_xor_sync(0xffffffffu, d, 16);
+            if (hf == 0) atomicAdd(&dv[t], d);
+        }
+        // dY g^T: <C~_t, .> for the output term, then the row scale f_t; X dg^T: row scale e w
+        {
+            float d = 0.f;
+            const float sf = k.ff[t], se = k.ew[t];
+#pragma unroll
+            for (int m = 0; m < NST / 64; ++m) {
+                const int cb = 16 * (wg + 2 * m), col0 = cb + (NST / 2) * hf;
+                uint32_t v[16], u2[16];
+                ld_blk<NST>(tq, C::TM_DC, cb, v);
+                ld_blk<NST>(tq, C::TM_DB, cb, u2);
+                tmem_wait_ld();
+                const uint4 c0 = *reinterpret_cast<const uint4*>(sm + C::OFF_C + tile_off(t, col0, kQ));
+                const uint4 c1 = *reinterpret_cast<const uint4*>(sm + C::OFF_C + tile_off(t, col0 + 8, kQ));
+                const uint32_t ct[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
+                    d = fmaf(bf16lo(ct[i]), a0, fmaf(bf16hi(ct[i]), a1, d));
+                    v[2 * i] = __float_as_uint(a0 * sf);
+                    v[2 * i + 1] = __float_as_uint(a1 * sf);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) u2[i] = __float_as_uint(__uint_as_float(u2[i]) * se);
+                st_blk<NST>(tq, C::TM_DC, cb, v);
+                st_blk<NST>(tq, C::TM_DB, cb, u2);
+            }
+            d += __shfl_xor_sync(0xffffffffu, d, 16);
+            if (hf == 0) atomicAdd(&qz[t], d);
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    ok = ok && *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u;
+    if (tid == 0 && issued == 1) {
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kQ / 16; ++kk)
+                mma_bf16(tmem + C::TM_DX, bdesc_mn(sb + C::OFF_MS, kk, kQ * 128),
+                         bdesc_mn(sb + C::OFF_DY, kk, kQ * 128), C::ID_MSDY, 1);
+#pragma unroll
+            for (int kk = 0; kk < kQ / 16; ++kk)
+                mma_bf16(tmem + C::TM_DC, bdesc_k(sb + C::OFF_DS, kk, kQ),
+                         bdesc_mn(sb + C::OFF_B, kk, kQ * 128), C::ID_DSB, 1);
+#pragma unroll
+            for (int kk = 0; kk < kQ / 16; ++kk)
+                mma_bf16(tmem + C::TM_DB, bdesc_mn(sb + C::OFF_DS, kk, kQ * 128),
+                         bdesc_mn(sb + C::OFF_C, kk, kQ * 128), C::ID_DSC, 1);
+            mma_commit(&bar[2]);
+            issued = 2;
+        } else {
+            drain(&bar[1], 0, 100000000ull);
+        }
+    }
+
+    // ---- second epilogue: dX; dC~, dB~ rotated back, angle gradients per (token, pair)
+    ok = ok && warp_wait_b(&bar[2], 0, ab);
+    tc_fence_after();
+    if (ok) {
+        const long long tg = t0 + t;
+        const bool live = t < nv;
+        {
+            const int cb = 16 * wg, col0 = cb + 32 * hf;
+            uint32_t v[16];
+            ld_blk<64>(tq, C::TM_DX, cb, v);
+            tmem_wait_ld();
+            const float Dh = a.D ? a.D[h] : 0.f;
+            const uint4 y0 = *reinterpret_cast<const uint4*>(sm + C::OFF_DY + sw128_off(t, col0));
+            const uint4 y1 = *reinterpret_cast<const uint4*>(sm + C::OFF_DY + sw128_off(t, col0 + 8));
+            const uint32_t ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+            if (live) {
+                float4* dst = reinterpret_cast<float4*>(a.dx + (((size_t)b * a.T + tg) * a.H + h) * kPc + col0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_float4(fmaf(Dh, bf16lo(ys[2 * i]), __uint_as_float(v[4 * i])),
+                                         fmaf(Dh, bf16hi(ys[2 * i]), __uint_as_float(v[4 * i + 1])),
+                                         fmaf(Dh, bf16lo(ys[2 * i + 1]), __uint_as_float(v[4 * i + 2])),
+                                         fmaf(Dh, bf16hi(ys[2 * i + 1]), __uint_as_float(v[4 * i + 3])));
+            }
+        }
+        const size_t grow = (((size_t)b * a.T + (live ? tg : 0)) * a.G + g) * NST;
+        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
+        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
+#pragma unroll
+        for (int m = 0; m < NST / 64; ++m) {
+            const int cb = 16 * (wg + 2 * m), col0 = cb + (NST / 2) * hf;
+            uint32_t vc[16], vb[16];
+            ld_blk<NST>(tq, C::TM_DC, cb, vc);
+            ld_blk<NST>(tq, C::TM_DB, cb, vb);
+            tmem_wait_ld();
+            uint4 rb[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+            uint4 rc[2] = {rb[0], rb[1]};
+            if (live) {
+                rb[0] = *reinterpret_cast<const uint4*>(Bg + grow + col0);
+                rb[1] = *reinterpret_cast<const uint4*>(Bg + grow + col0 + 8);
+                rc[0] = *reinterpret_cast<const uint4*>(Cg + grow + col0);
+                rc[1] = *reinterpret_cast<const uint4*>(Cg + grow + col0 + 8);
+            }
+            const uint32_t bw[8] = {rb[0].x, rb[0].y, rb[0].z, rb[0].w, rb[1].x, rb[1].y, rb[1].z, rb[1].w};
+            const uint32_t cw[8] = {rc[0].x, rc[0].y, rc[0].z, rc[0].w, rc[1].x, rc[1].y, rc[1].z, rc[1].w};
+            float oc[16], ob[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int j = col0 / 2 + i;
+                float sn, cs2;
+                __sincosf(psi[t * PSI_LD + j], &sn, &cs2);
+                const float c0 = bf16lo(cw[i]), c1 = bf16hi(cw[i]);
+                const float b0 = bf16lo(bw[i]), b1 = bf16hi(bw[i]);
+                const float ct0 = fmaf(cs2, c0, sn * c1), ct1 = fmaf(cs2, c1, -sn * c0);
+                const float bt0 = fmaf(cs2, b0, sn * b1), bt1 = fmaf(cs2, b1, -sn * b0);
+                const float dc0 = __uint_as_float(vc[2 * i]), dc1 = __uint_as_float(vc[2 * i + 1]);
+                const float db0 = __uint_as_float(vb[2 * i]), db1 = __uint_as_float(vb[2 * i + 1]);
+                psi[t * PSI_LD + j] = fmaf(dc0, ct1, -dc1 * ct0) + fmaf(db0, bt1, -db1 * bt0);
+                oc[2 * i] = fmaf(cs2, dc0, -sn * dc1);
+                oc[2 * i + 1] = fmaf(sn, dc0, cs2 * dc1);
+                ob[2 * i] = fmaf(cs2, db0, -sn * db1);
+                ob[2 * i + 1] = fmaf(sn, db0, cs2 * db1);
+            }
+            if (live) {
+                float4* dC = reinterpret_cast<float4*>(a.dC + grow + col0);
+                float4* dB = reinterpret_cast<float4*>(a.dB + grow + col0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    atomicAdd(dC + i, make_float4(oc[4 * i], oc[4 * i + 1], oc[4 * i + 2], oc[4 * i + 3]));
+                    atomicAdd(dB + i, make_float4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]));
+                }
+            }
+        }
+    }
+    __syncthreads();
+    ok = ok && *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u;
+    if (ok) {
+        // angles: suffix sums over the chunk's tokens per pair; dtheta gets dang (x dt), the
+        // dt gradient dang . theta (summed over pairs below)
+        if (tid < NH) {
+            const int j = tid;
+            float sacc = 0.f;
+            for (int u = kQ - 1; u >= 0; --u) {
+                sacc += psi[u * PSI_LD + j];
+                float contrib = 0.f;
+                if (u < nv) {
+                    const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
+                    const float th = a.theta[row * NH + j];
+                    atomicAdd(&a.dtheta[row * NH + j], angle ? sacc : sacc * k.dd[u]);
+                    contrib = angle ? 0.f : sacc * th;
+                }
+                psi[u * PSI_LD + j] = contrib;
+            }
+            p.dtot[cc * NH + j] = sacc;
+        }
+        // the log-decay gradient of every token (chunk-local: its terms sum to zero over the
+        // chunk, so the suffix sums that reach dA and dt stay inside the chunk)
+        if (tid < kQ) {
+            const int u = tid;
+            const float ewdv = k.ew[u] * dv[u];
+            dcm[u] = rs[u] - cs[u] + k.ff[u] * qz[u] - ewdv;
+            const float sw = warp_sum(ewdv);
+            if (lane == 0) misc2[1 + w] = sw;
+            const float dw = k.ee[u] * dv[u];
+            dnx[u] = ga[u] - dgd[u] + dw;
+        }
+    }
+    __syncthreads();
+    if (ok && tid < kQ) {
+        const int u = tid;
+        float v = dcm[u];
+        if (u == nv - 1) v += misc2[1] + misc2[2] + p.q[cc];
+        // suffix sum over u within the warp, then warp 0 adds warp 1's total
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float x = __shfl_down_sync(0xffffffffu, v, o);
+            if (lane + o < 32) v += x;
+        }
+        const float w1 = __shfl_sync(0xffffffffu, v, 0);
+        if (w == 1 && lane == 0) misc2[3] = w1;
+        __syncwarp();
+        dcm[u] = v;
+    }
+    __syncthreads();
+    if (ok && tid < kQ) {
+        const int u = tid;
+        const float dda = dcm[u] + (w == 0 ? misc2[3] : 0.f);
+        float dpt = 0.f;
+        for (int j = 0; j < NH; ++j) dpt += psi[u * PSI_LD + j];
+        const float dga = k.ee[u] * dv[u] + ga[u];
+        float ddt = fmaf(dda, k.aa[u], fmaf(dga, k.ll[u], dpt));
+        float dlam = dga * k.dd[u];
+        if (u > 0) {
+            ddt = fmaf(dnx[u - 1], 1.f - k.ll[u], ddt);
+            dlam = fmaf(-dnx[u - 1], k.dd[u], dlam);
+        }
+        if (c == 0 && u == 0) {
+            const float v0 = p.v0[bh];
+            ddt = fmaf(1.f - k.ll[0], v0, ddt);
+            dlam = fmaf(-k.dd[0], v0, dlam);
+        }
+        if (u < nv) {
+            const size_t o = ((size_t)b * a.T + t0 + u) * a.H + h;
+            a.ddt[o] = ddt;
+            a.dA[o] = dda * k.dd[u];
+            a.dlam[o] = dlam;
+        }
+        if (u == kQ - 1) p.spill[cc] = dnx[u];
+        if (u == 0 && a.D && a.dD) atomicAdd(&a.dD[h], misc2[0]);
+    }
+    if (tid == 0) {
+        if (issued == 2) drain(&bar[2], 0, 100000000ull);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// 4. finish: the angle gradient carried in from later chunks (and from dL/dh_T) and the
+// next-token share of the previous chunk's last trapezoid weight
+__global__ void __launch_bounds__(64) bwd_finish_kernel(const __grid_constant__ TcBwd p) {
+    const BwdArgs& a = p.a;
+    const int NH = a.N / 2;
+    __shared__ float car[64];
+    const int tid = threadIdx.x;
+    const int c = (int)(blockIdx.x % p.nch);
+    const size_t bh = blockIdx.x / p.nch;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H), g = h / (a.H / a.G);
+    const long long t0 = (long long)c * kQ;
+    const int nv = (int)(a.T - t0 < kQ ? a.T - t0 : kQ);
+    const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
+    if (tid < NH) {
+        float s = p.extra[bh * NH + tid];
+        for (int c2 = c + 1; c2 < p.nch; ++c2) s += p.dtot[(bh * p.nch + c2) * NH + tid];
+        car[tid] = s;
+        for (int u = 0; u < nv; ++u) {
+            const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
+            const float d = a.dt[((size_t)b * a.T + t0 + u) * a.H + h];
+            atomicAdd(&a.dtheta[row * NH + tid], angle ? s : s * d);
+        }
+    }
+    __syncthreads();
+    if (tid < nv) {
+        const size_t o = ((size_t)b * a.T + t0 + tid) * a.H + h;
+        float add = 0.f;
+        if (!angle) {
+            const float* th = a.theta + (((size_t)b * a.T + t0 + tid) * a.G + g) * NH;
+            for (int j = 0; j < NH; ++j) add = fmaf(car[j], th[j], add);
+        }
+        float dl = 0.f;
+        if (tid == 0 && c > 0) {
+            const float s = p.spill[bh * p.nch + c - 1];
+            add = fmaf(s, 1.f - a.lam[o], add);
+            dl = -s * a.dt[o];
+        }
+        a.ddt[o] += add;
+        if (dl != 0.f) a.dlam[o] += dl;
+    }
+}
+
+struct Layout {
+    size_t V, U, gin, dgo, ctot, atot, P0, q, dtot, spill, extra, v0, bytes;
+};
+
+Layout layout(int batch, int H, int N, long long T) {
+    const size_t BH = (size_t)batch * H, nch = (size_t)((T + kQ - 1) / kQ), NP = (size_t)N * kPc;
+    const size_t NH = N / 2;
+    Layout L;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    L.V = take(BH * nch * NP * 4);
+    L.U = take(BH * nch * NP * 4);
+    L.gin = take(BH * nch * NP * 2);
+    L.dgo = take(BH * nch * NP * 2);
+    L.ctot = take(BH * nch * 4);
+    L.atot = take(BH * nch * NH * 4);
+    L.P0 = take(BH * (nch + 1) * NH * 4);
+    L.q = take(BH * nch * 4);
+    L.dtot = take(BH * nch * NH * 4);
+    L.spill = take(BH * nch * 4);
+    L.extra = take(BH * NH * 4);
+    L.v0 = take(BH * 4);
+    L.bytes = o;
+    return L;
+}
+
+template <int NST>
+cudaError_t launch_n(const TcBwd& p, long long units, cudaStream_t s) {
+    const int smv = VuCfg<NST>::SMEM, smg = GrCfg<NST>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(bwd_vu_kernel<NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smv);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_grads_kernel<NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smg);
+    if (e != cudaSuccess) return e;
+    bwd_vu_kernel<NST><<<(unsigned)units, 128, smv, s>>>(p);
+    bwd_scan_kernel<NST><<<(unsigned)((size_t)p.a.batch * p.a.H), 4 * NST, 0, s>>>(p);
+    bwd_grads_kernel<NST><<<(unsigned)units, 256, smg, s>>>(p);
+    bwd_finish_kernel<<<(unsigned)units, 64, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool scan_bwd_tc_ok(int io_dtype, int N, int P, int R) {
+    return io_dtype == M3_BF16 && R == 1 && P == kPc && (N == 64 || N == 128);
+}
+
+size_t scan_bwd_tc_workspace_bytes(int batch, int H, int N, long long T) {
+    return layout(batch, H, N, T).bytes;
+}
+
+cudaError_t launch_scan_bwd_tc(const BwdArgs& a, void* ws, uint32_t* status, unsigned long long limit_ns,
+                               cudaStream_t s) {
+    const Layout L = layout(a.batch, a.H, a.N, a.T);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    TcBwd p;
+    p.a = a;
+    p.nch = (int)((a.T + kQ - 1) / kQ);
+    p.V = reinterpret_cast<float*>(base + L.V);
+    p.U = reinterpret_cast<float*>(base + L.U);
+    p.gin = reinterpret_cast<uint16_t*>(base + L.gin);
+    p.dgo = reinterpret_cast<uint16_t*>(base + L.dgo);
+    p.ctot = reinterpret_cast<float*>(base + L.ctot);
+    p.atot = reinterpret_cast<float*>(base + L.atot);
+    p.P0 = reinterpret_cast<float*>(base + L.P0);
+    p.q = reinterpret_cast<float*>(base + L.q);
+    p.dtot = reinterpret_cast<float*>(base + L.dtot);
+    p.spill = reinterpret_cast<float*>(base + L.spill);
+    p.extra = reinterpret_cast<float*>(base + L.extra);
+    p.v0 = reinterpret_cast<float*>(base + L.v0);
+    p.status = status;
+    p.limit_ns = limit_ns;
+    const long long units = (long long)a.batch * a.H * p.nch;
+    return a.N == 128 ? launch_n<128>(p, units, s) : launch_n<64>(p, units, s);
+}
+
+}  // namespace m3

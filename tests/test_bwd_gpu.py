@@ -1,5 +1,7 @@
 """Parity of the backward pass (m3_scan_bwd, reverse-mode gradients of the recurrence) with
-the fp64 oracle's backward, through the C ABI, on the same rounded inputs.
+the fp64 oracle's backward, through the C ABI, on the same rounded inputs: the sequential fp32
+kernel (every shape it covers; SISO bf16 P 64 shapes through M3_FLAG_FORCE_SIMT, which would
+otherwise take the chunked tensor-core path checked in test_bwd_tc_gpu.py).
 
 The kernel computes in fp32 (checkpoints every 16 tokens, recomputed segments), so the
 bar is fp32 accumulation error: max |gpu - ref| / max |ref| per gradient tensor.  The full
@@ -65,7 +67,8 @@ CASES = [
     (1, 3, 3, 8, 6, 3, 40, torch.float32, 0, False),       # G = H, no dL/dh_T
     (1, 2, 1, 16, 16, 1, 256, torch.float32, 0, True),     # the small fp32 SISO workload
     (1, 2, 1, 16, 16, 1, 50, torch.float32, m3.M3_FLAG_THETA_IS_ANGLE, True),
-    (1, 4, 1, 64, 128, 1, 100, torch.bfloat16, 0, True),   # 1.5B-scale SISO head shape
+    (1, 4, 1, 64, 128, 1, 100, torch.bfloat16, m3.M3_FLAG_FORCE_SIMT, True),   # 1.5B-scale
+    #                                   SISO head shape, on the sequential kernel
     (1, 4, 2, 64, 64, 4, 70, torch.bfloat16, 0, True),     # MIMO R = 4
     (2, 2, 1, 40, 10, 2, 33, torch.float32, 0, True),      # two column blocks, partial warp
 ]
@@ -110,7 +113,7 @@ def test_backward_fullsize_sampled_heads():
     gen = torch.Generator().manual_seed(12)
     dy = torch.randn((b, T, H, R, P), generator=gen).to(w.io_dtype)
     d = m3.Dims(b, H, G, P, N, R, m3.M3_BF16)
-    got = _gpu_bwd(inp, dy, None, d, T)
+    got = _gpu_bwd(inp, dy, None, d, T, m3.M3_FLAG_FORCE_SIMT)
     heads = [0, 37]
     sub = {k: inp[k][:1] for k in KEYS}
     for k in ("x", "dt", "A", "lam"):

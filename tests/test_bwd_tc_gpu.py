@@ -1,0 +1,150 @@
+"""Parity of the chunked tensor-core backward (m3_scan_bwd for SISO bf16, P 64, N 64 / 128)
+with the fp64 oracle's backward, through the C ABI.
+
+The chunked backward multiplies bf16 operands on the tensor cores (the rotated B and C, the
+masked score tiles, the chunk states and their adjoints), so the bar is the bf16 one of the
+forward kernel: max |gpu - ref| / max |ref| per gradient tensor <= 2e-2.  The sequential fp32
+kernel (M3_FLAG_FORCE_SIMT) stays the 2e-4 reference for the same shapes.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import KEYS, f64
+from state_space_model_06_b200 import inputs, m3
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+def _rel(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-30))
+
+
+def _problem(b, H, G, N, T, seed, dhT=True, theta_max=1.0):
+    inp = inputs.make_scan_inputs(b, T, H, G, 64, N, 1, io_dtype=torch.bfloat16,
+                                  theta_max=theta_max, seed=seed, h0_random=True, carry_prev=True)
+    gen = torch.Generator().manual_seed(seed + 5)
+    dy = torch.randn((b, T, H, 1, 64), generator=gen).to(torch.bfloat16)
+    dh = torch.randn((b, H, N, 64), generator=gen) if dhT else None
+    return inp, dy, dh
+
+
+def _gpu_bwd(inp, dy, dh, d, T, flags=0, with_D=True):
+    g = {k: v.cuda() for k, v in inp.items()}
+    st = m3.State(d)
+    st.h.copy_(g["h0"])
+    st.x_prev.copy_(g["x_prev"])
+    st.B_prev.copy_(g["B_prev"])
+    gr = m3.alloc_grads(d, T)
+    for v in gr.values():
+        v.fill_(float("nan"))
+    ws = m3.alloc_bwd_workspace(d, T)
+    m3.m3_scan_bwd(d, T, *(g[k] for k in KEYS), g["D"] if with_D else None, st, dy.cuda(),
+                   None if dh is None else dh.cuda(), gr, ws, flags)
+    assert m3.m3_query_status(ws) == m3.M3_OK
+    torch.cuda.synchronize()
+    assert torch.equal(st.h.cpu(), inp["h0"]) and torch.equal(st.x_prev.cpu(), inp["x_prev"])
+    return {k: f64(v) for k, v in gr.items()}
+
+
+def _oracle_bwd(inp, dy, dh, angle=False, with_D=True):
+    return oracle.scan_bwd(*(f64(inp[k]) for k in KEYS), f64(dy),
+                           D=f64(inp["D"]) if with_D else None, h0=f64(inp["h0"]),
+                           x_prev=f64(inp["x_prev"]), B_prev=f64(inp["B_prev"]),
+                           dhT=None if dh is None else f64(dh), theta_is_angle=angle)
+
+
+CASES = [
+    # (b, H, G, N, T, flags, dhT, theta_max)
+    (1, 2, 1, 128, 100, 0, True, 1.0),          # two chunks, ragged tail, shared group
+    (1, 4, 1, 128, 64, 0, True, 1.0),           # exactly one chunk
+    (2, 4, 2, 64, 200, 0, True, 1.0),           # N 64, two groups, four chunks
+    (1, 2, 2, 128, 300, 0, False, math.pi),     # G = H, no dL/dh_T, fast rotation
+    (1, 2, 1, 128, 130, m3.M3_FLAG_THETA_IS_ANGLE, True, 0.1),
+    (1, 3, 1, 128, 1, 0, True, 1.0),            # one token
+    (1, 2, 1, 64, 65, 0, True, 1.0),            # one token past a chunk
+]
+
+
+def _id(c):
+    return (f"b{c[0]}H{c[1]}G{c[2]}N{c[3]}T{c[4]}{'A' if c[5] else ''}"
+            f"{'' if c[6] else 'nodh'}")
+
+
+@pytest.mark.parametrize("case", CASES, ids=[_id(c) for c in CASES])
+def test_tc_backward_matches_oracle(case):
+    b, H, G, N, T, flags, with_dh, tmax = case
+    inp, dy, dh = _problem(b, H, G, N, T, seed=61, dhT=with_dh, theta_max=tmax)
+    d = m3.Dims(b, H, G, 64, N, 1, m3.M3_BF16)
+    got = _gpu_bwd(inp, dy, dh, d, T, flags)
+    ref = _oracle_bwd(inp, dy, dh, angle=bool(flags & m3.M3_FLAG_THETA_IS_ANGLE))
+    errs = {k: _rel(got[k], ref[k]) for k in m3.GRAD_NAMES}
+    for k in m3.GRAD_NAMES:
+        assert np.all(np.isfinite(got[k])), k
+    assert all(e <= TOL for e in errs.values()), errs
+
+
+def test_tc_backward_without_D():
+    inp, dy, dh = _problem(1, 2, 1, 128, 150, seed=62)
+    d = m3.Dims(1, 2, 1, 64, 128, 1, m3.M3_BF16)
+    got = _gpu_bwd(inp, dy, dh, d, 150, with_D=False)
+    ref = _oracle_bwd(inp, dy, dh, with_D=False)
+    for k in m3.GRAD_NAMES:
+        if k == "dD":
+            continue
+        assert _rel(got[k], ref[k]) <= TOL, (k, _rel(got[k], ref[k]))
+
+
+def test_tc_backward_against_sequential_kernel():
+    """The chunked tensor-core path and the sequential fp32 kernel (M3_FLAG_FORCE_SIMT) on
+    the same inputs agree to the bf16 bar, and the sequential one to the oracle at 2e-4."""
+    inp, dy, dh = _problem(1, 4, 1, 128, 257, seed=63)
+    d = m3.Dims(1, 4, 1, 64, 128, 1, m3.M3_BF16)
+    tc = _gpu_bwd(inp, dy, dh, d, 257)
+    seq = _gpu_bwd(inp, dy, dh, d, 257, flags=m3.M3_FLAG_FORCE_SIMT)
+    ref = _oracle_bwd(inp, dy, dh)
+    for k in m3.GRAD_NAMES:
+        assert _rel(seq[k], ref[k]) <= 2e-4, k
+        assert _rel(tc[k], seq[k]) <= TOL, (k, _rel(tc[k], seq[k]))
+
+
+def test_tc_backward_all_heads_of_a_group():
+    """64 heads sharing one group (the 1.5B-scale head count): the group sums of dB, dC,
+    dtheta, dB_prev and dD over all 64 heads, 256 tokens."""
+    inp, dy, dh = _problem(1, 64, 1, 128, 256, seed=64)
+    d = m3.Dims(1, 64, 1, 64, 128, 1, m3.M3_BF16)
+    got = _gpu_bwd(inp, dy, dh, d, 256)
+    ref = _oracle_bwd(inp, dy, dh)
+    errs = {k: _rel(got[k], ref[k]) for k in m3.GRAD_NAMES}
+    assert all(e <= TOL for e in errs.values()), errs
+
+
+def test_tc_backward_fullsize_sampled_heads():
+    """The 1.5B-scale SISO prefill workload (b8 H64 T4096 P64 N128, bf16), backward at full
+    size on the chunked path; per-head gradients of heads 0 and 37 of batch row 0 against the
+    oracle on those two heads, the group-summed ones finite."""
+    w = inputs.WORKLOADS["siso_prefill_1p5b"]
+    b, H, G, P, N, R, T = w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank, w.seqlen
+    inp = inputs.make_scan_inputs(b, T, H, G, P, N, R, io_dtype=w.io_dtype, seed=7)
+    gen = torch.Generator().manual_seed(12)
+    dy = torch.randn((b, T, H, R, P), generator=gen).to(w.io_dtype)
+    d = m3.Dims(b, H, G, P, N, R, m3.M3_BF16)
+    got = _gpu_bwd(inp, dy, None, d, T)
+    heads = [0, 37]
+    sub = {k: inp[k][:1] for k in KEYS}
+    for k in ("x", "dt", "A", "lam"):
+        sub[k] = sub[k][:, :, heads]
+    ref = oracle.scan_bwd(*(f64(sub[k]) for k in KEYS), f64(dy[:1, :, heads]),
+                          D=f64(inp["D"][heads]), h0=f64(inp["h0"][:1, heads]),
+                          x_prev=f64(inp["x_prev"][:1, heads]), B_prev=f64(inp["B_prev"][:1]))
+    for k in ("dx", "ddt", "dA", "dlam"):
+        assert _rel(got[k][:1, :, heads], ref[k]) <= TOL, (k, _rel(got[k][:1, :, heads], ref[k]))
+    for k in ("dh0", "dx_prev"):
+        assert _rel(got[k][:1, heads], ref[k]) <= TOL, k
+    for k in ("dB", "dC", "dtheta", "dD", "dB_prev"):
+        assert np.all(np.isfinite(got[k])), k
