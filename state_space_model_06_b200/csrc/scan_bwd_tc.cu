@@ -201,7 +201,8 @@ struct VuCfg {
     static constexpr int OFF_XW = 2 * kQ * NST * 2;          // diag(e w) X [Q][64]
     static constexpr int OFF_DYF = OFF_XW + kQ * kPc * 2;    // diag(f) dY [Q][64]
     static constexpr int OFF_COEF = OFF_DYF + kQ * kPc * 2;
-    static constexpr int OFF_BAR = (OFF_COEF + Coefs::kFloats * 4 + 7) / 8 * 8;
+    static constexpr int OFF_SEG = OFF_COEF + Coefs::kFloats * 4;   // [128 / NH][NH] angle sums
+    static constexpr int OFF_BAR = (OFF_SEG + 128 * 4 + 7) / 8 * 8;
     static constexpr int OFF_MISC = OFF_BAR + 8;
     static constexpr int USED = OFF_MISC + 16 + 1024;
     // at least 50 KB, so that at most four CTAs (4 x 128 TMEM columns) share an SM
@@ -244,37 +245,55 @@ __global__ void __launch_bounds__(128) bwd_vu_kernel(const __grid_constant__ TcB
     const Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.status, p.limit_ns};
     if (tid == 0) p.ctot[cc] = k.cr[kQ - 1];
 
-    // B~, C~ in the chunk's frame: thread j (B) and NH + j (C) walk the chunk's tokens
-    if (tid < 2 * NH) {
-        const bool isC = tid >= NH;
-        const int j = isC ? tid - NH : tid;
-        const uint16_t* src = static_cast<const uint16_t*>(isC ? a.C : a.B);
-        uint8_t* tile = sm + (isC ? C::OFF_C : C::OFF_B);
+    // B~, C~ in the chunk's frame: thread (pair j, token segment sg) sums its segment's
+    // angles, the segments' totals are exchanged, and the thread rotates its segment's tokens
+    {
+        constexpr int SEGS = 128 / NH, TPS = kQ / SEGS;
+        const int j = tid % NH, sg = tid / NH;
+        float* segt = reinterpret_cast<float*>(sm + C::OFF_SEG);
         const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
-        float rho = 0.f;
-#pragma unroll 4
-        for (int u = 0; u < kQ; ++u) {
+        float rho[TPS];
+        float r = 0.f;
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) {
+            const int u = sg * TPS + i;
             const long long t = t0 + u;
-            float v0 = 0.f, v1 = 0.f, th = 0.f;
-            if (t < a.T) {
-                const size_t row = ((size_t)b * a.T + t) * a.G + g;
-                const uint32_t pr = *reinterpret_cast<const uint32_t*>(src + row * NST + 2 * j);
-                v0 = bf16lo(pr);
-                v1 = bf16hi(pr);
-                th = a.theta[row * NH + j];
-            }
-            rho += angle ? th : k.dd[u] * th;
-            float sn, cs;
-            __sincosf(wrap_angle(rho), &sn, &cs);
-            *reinterpret_cast<uint32_t*>(tile + tile_off(u, 2 * j, kQ)) =
-                pack_bf16x2(fmaf(cs, v0, sn * v1), fmaf(cs, v1, -sn * v0));
+            const float th = t < a.T ? a.theta[(((size_t)b * a.T + t) * a.G + g) * NH + j] : 0.f;
+            r += angle ? th : k.dd[u] * th;
+            rho[i] = r;
         }
-        if (!isC) p.atot[cc * NH + j] = rho;
+        segt[sg * NH + j] = r;
+        __syncthreads();
+        float off = 0.f;
+        for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + j];
+        if (sg == SEGS - 1) p.atot[cc * NH + j] = off + r;
+        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
+        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) {
+            const int u = sg * TPS + i;
+            const long long t = t0 + u;
+            uint32_t pb = 0u, pcv = 0u;
+            if (t < a.T) {
+                const size_t row = (((size_t)b * a.T + t) * a.G + g) * NST + 2 * j;
+                pb = *reinterpret_cast<const uint32_t*>(Bg + row);
+                pcv = *reinterpret_cast<const uint32_t*>(Cg + row);
+            }
+            float sn, cs;
+            __sincosf(wrap_angle(off + rho[i]), &sn, &cs);
+            const float b0 = bf16lo(pb), b1 = bf16hi(pb), c0 = bf16lo(pcv), c1 = bf16hi(pcv);
+            const uint32_t o = tile_off(u, 2 * j, kQ);
+            *reinterpret_cast<uint32_t*>(sm + C::OFF_B + o) =
+                pack_bf16x2(fmaf(cs, b0, sn * b1), fmaf(cs, b1, -sn * b0));
+            *reinterpret_cast<uint32_t*>(sm + C::OFF_C + o) =
+                pack_bf16x2(fmaf(cs, c0, sn * c1), fmaf(cs, c1, -sn * c0));
+        }
     }
     // diag(e w) X and diag(f) dY
     {
         const uint16_t* xg = static_cast<const uint16_t*>(a.x);
         const uint16_t* yg = static_cast<const uint16_t*>(a.dy);
+#pragma unroll 4
         for (int i = tid; i < 2 * kQ * 8; i += 128) {
             const bool isY = i >= kQ * 8;
             const int e = isY ? i - kQ * 8 : i;
@@ -499,6 +518,15 @@ __global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant
 
 // ------------------------------------------------------------------------------------
 // 3. chunk gradients
+//
+// Two CTAs share an SM: each allocates 256 TMEM columns after its loads, and keeps under
+// 113 KB of shared memory.  TMEM: columns [0, 64) hold S, then B~ dg, then dX; [64, 128)
+// dY X^T; [128, 128 + N) dY g^T, then dC~, then dB~.  Three MMA rounds:
+//   1. S = C~ B~^T, dY X^T, dY g^T;            epilogue: L o S, dS, the band and decay sums,
+//                                              <C~_t, (dY g^T)_t>, row scale f
+//   2. dC~ += dS B~, B~ dg;                    epilogue: dC~ rotated back (dC), angle terms;
+//                                              <X_s, (B~ dg)_s>, row scale e w; X <- e w X
+//   3. dX = (L o S)^T dY + ., dB~ = (e w X) dg^T + dS^T C~;   epilogue: dX, dB
 template <int NST>
 struct GrCfg {
     static constexpr int NH = NST / 2;
@@ -508,19 +536,20 @@ struct GrCfg {
     static constexpr int OFF_B = OFF_C + kQ * NST * 2;        // B~
     static constexpr int OFF_GIN = OFF_B + kQ * NST * 2;      // g_in [NST][64]
     static constexpr int OFF_DG = OFF_GIN + NST * kPc * 2;    // dg_out [NST][64]
-    static constexpr int PSI_LD = NH + 1;
-    static constexpr int OFF_PSI = OFF_DG + NST * kPc * 2;    // fp32 [Q][NH + 1]
-    static constexpr int OFF_SEG = OFF_PSI + kQ * PSI_LD * 4; // fp32 [256 / NH][NH]
+    static constexpr int OFF_SEG = OFF_DG + NST * kPc * 2;    // fp32 [256 / NH][NH]
     static constexpr int OFF_COEF = OFF_SEG + 256 * 4;
-    static constexpr int NACC = 9;
+    static constexpr int NACC = 10;
     static constexpr int OFF_ACC = OFF_COEF + Coefs::kFloats * 4;
     static constexpr int OFF_BAR = (OFF_ACC + (NACC * kQ + 4) * 4 + 7) / 8 * 8;
-    static constexpr int OFF_MISC = OFF_BAR + 3 * 8;
+    static constexpr int OFF_MISC = OFF_BAR + 4 * 8;
     static constexpr int USED = OFF_MISC + 16 + 1024;
-    // at least 120 KB: one CTA per SM (each allocates all 512 TMEM columns)
-    static constexpr int SMEM = USED > 122880 ? USED : 122880;
-    static_assert(SMEM <= 232448, "shared memory budget exceeded");
-    static constexpr uint32_t TM_S = 0, TM_GX = 64, TM_DX = 128, TM_DC = 192, TM_DB = 192 + NST;
+    // two CTAs per SM (2 x 256 TMEM columns), never three
+    static constexpr int SMEM = USED > 79872 ? USED : 79872;
+    static_assert(2 * (SMEM + 1024) <= 233472 && 3 * (SMEM + 1024) > 233472, "two CTAs per SM");
+    // the angle table [Q][NH] fp32 lives in the L o S / dS tiles until the first epilogue and
+    // in the g_in tile after it (both free at those times)
+    static_assert(kQ * NH * 4 <= 2 * T64 && kQ * NH * 4 <= NST * kPc * 2, "angle table");
+    static constexpr uint32_t TM_A = 0, TM_GX = 64, TM_C = 128;
     static constexpr uint32_t ID_QQ = idesc_bf16(kQ, kQ, false, false);    // S, dY X^T
     static constexpr uint32_t ID_BDG = idesc_bf16(kQ, kPc, false, true);   // B~ dg
     static constexpr uint32_t ID_KN = idesc_bf16(kQ, NST, false, false);   // dY g^T, X dg^T
@@ -528,6 +557,13 @@ struct GrCfg {
     static constexpr uint32_t ID_DSB = idesc_bf16(kQ, NST, false, true);   // dS B~
     static constexpr uint32_t ID_DSC = idesc_bf16(kQ, NST, true, true);    // dS^T C~
 };
+
+// angle table index: row u, pair j, XOR-swizzled so that a column read by the 16 rows of a
+// half warp hits 16 banks
+template <int NH>
+__device__ __forceinline__ int psi_idx(int u, int j) {
+    return u * NH + (j ^ (u & 31));
+}
 
 // TMEM access of an M = 64 accumulator by 8 warps: warp w reaches lane quadrant w % 4 (rows
 // 16 q .. 16 q + 15 at lanes 32 q .. 32 q + 15); 16-column blocks cb of the first half go to
@@ -558,9 +594,9 @@ __device__ __forceinline__ float colsum16(float (&v)[16], int lane) {
 }
 
 template <int NST>
-__global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant__ TcBwd p) {
+__global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant__ TcBwd p) {
     using C = GrCfg<NST>;
-    constexpr int NH = C::NH, PSI_LD = C::PSI_LD;
+    constexpr int NH = C::NH;
     const BwdArgs& a = p.a;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -576,8 +612,10 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
     float* qz = acc + 5 * kQ;     // <C~_t, (dY g^T)_t>
     float* dcm = acc + 6 * kQ;    // log-decay gradient, then its suffix sums
     float* dnx = acc + 7 * kQ;    // band-weight gradient owed to the next token
-    float* misc2 = acc + 8 * kQ;  // [0] dD partial, [1..2] warp sums
-    float* psi = reinterpret_cast<float*>(sm + C::OFF_PSI);
+    float* dpt = acc + 8 * kQ;    // dt gradient through the angles, per token
+    float* misc2 = acc + 9 * kQ;  // [0] dD partial, [1..2] warp sums, [3] suffix carry
+    float* psi0 = reinterpret_cast<float*>(sm + C::OFF_MS);    // angle table, first home
+    float* psi1 = reinterpret_cast<float*>(sm + C::OFF_GIN);   // and second
     float* segt = reinterpret_cast<float*>(sm + C::OFF_SEG);
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int c = (int)(blockIdx.x % p.nch);
@@ -590,7 +628,7 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
     const uint32_t tile_bytes = NST * kPc * 2;
 
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
         misc[1] = 0u;
         fence_mbar_init();
         mbar_arrive_expect_tx(&bar[0], 2 * tile_bytes);
@@ -599,14 +637,9 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
         bulk_load(sm + C::OFF_DG, reinterpret_cast<const uint8_t*>(p.dgo) + cc * tile_bytes,
                   tile_bytes, &bar[0]);
     }
-    if (w == 0) {
-        __syncwarp();
-        tmem_alloc(&misc[0], 512);
-        tmem_relinquish();
-    }
     if (w == 1) chunk_coefs(a, b, h, t0, k);
     for (int i = tid; i < C::NACC * kQ + 4; i += 256) acc[i] = 0.f;
-    // angles: thread (pair j, token segment sg) sums its segment's angles
+    // angles: thread (pair jj, token segment sg) sums its segment's angles
     constexpr int SEGS = 256 / NH, TPS = kQ / SEGS;
     const int jj = tid % NH, sg = tid / NH;
     float rho[TPS];
@@ -625,21 +658,11 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
         }
         segt[sg * NH + jj] = r;
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = misc[0];
-    const Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.status, p.limit_ns};
-    {
-        float off = p.P0[(bh * (p.nch + 1) + c) * NH + jj];
-        for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + jj];
-#pragma unroll
-        for (int i = 0; i < TPS; ++i) psi[(sg * TPS + i) * PSI_LD + jj] = wrap_angle(off + rho[i]);
-    }
     // X and dY tiles
     {
         const uint16_t* xg = static_cast<const uint16_t*>(a.x);
         const uint16_t* yg = static_cast<const uint16_t*>(a.dy);
+#pragma unroll
         for (int i = tid; i < 2 * kQ * 8; i += 256) {
             const bool isY = i >= kQ * 8;
             const int e = isY ? i - kQ * 8 : i;
@@ -652,12 +675,21 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
             *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DY : C::OFF_X) + sw128_off(u, ch * 8)) = v;
         }
     }
-    __syncthreads();   // psi complete
+    __syncthreads();
+    {
+        float off = p.P0[(bh * (p.nch + 1) + c) * NH + jj];
+        for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + jj];
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) psi0[psi_idx<NH>(sg * TPS + i, jj)] = wrap_angle(off + rho[i]);
+    }
+    __syncthreads();
     // B~, C~ in the call frame: thread (pair j, token u) for tasks i = tid + 256 m
     {
         const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
         const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
-        for (int i = tid; i < kQ * NH; i += 256) {
+#pragma unroll
+        for (int m = 0; m < kQ * NH / 256; ++m) {
+            const int i = tid + 256 * m;
             const int j = i % NH, u = i / NH;
             const long long t = t0 + u;
             uint32_t pb = 0u, pcv = 0u;
@@ -667,7 +699,7 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
                 pcv = *reinterpret_cast<const uint32_t*>(Cg + row);
             }
             float sn, cs2;
-            __sincosf(psi[u * PSI_LD + j], &sn, &cs2);
+            __sincosf(psi0[psi_idx<NH>(u, j)], &sn, &cs2);
             const float b0 = bf16lo(pb), b1 = bf16hi(pb), c0 = bf16lo(pcv), c1 = bf16hi(pcv);
             const uint32_t off = tile_off(u, 2 * j, kQ);
             *reinterpret_cast<uint32_t*>(sm + C::OFF_B + off) =
@@ -677,88 +709,99 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
         }
     }
     fence_proxy_async_smem();
+    if (w == 0) {
+        tmem_alloc(&misc[0], 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    const Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.status, p.limit_ns};
     const uint32_t sb = smem_u32(sm);
-    int issued = 0;   // thread 0: MMA batches issued
+    int issued = 0;   // thread 0: MMA rounds issued
     if (tid == 0) {
         if (mbar_wait(&bar[0], 0, ab)) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < NST / 16; ++kk)
-                mma_bf16(tmem + C::TM_S, bdesc_k(sb + C::OFF_C, kk, kQ), bdesc_k(sb + C::OFF_B, kk, kQ),
+                mma_bf16(tmem + C::TM_A, bdesc_k(sb + C::OFF_C, kk, kQ), bdesc_k(sb + C::OFF_B, kk, kQ),
                          C::ID_QQ, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < kPc / 16; ++kk)
                 mma_bf16(tmem + C::TM_GX, bdesc_k(sb + C::OFF_DY, kk, kQ), bdesc_k(sb + C::OFF_X, kk, kQ),
                          C::ID_QQ, kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < NST / 16; ++kk)
-                mma_bf16(tmem + C::TM_DX, bdesc_k(sb + C::OFF_B, kk, kQ),
-                         bdesc_mn(sb + C::OFF_DG, kk, tile_bytes), C::ID_BDG, kk > 0);
-#pragma unroll
             for (int kk = 0; kk < kPc / 16; ++kk)
-                mma_bf16(tmem + C::TM_DC, bdesc_k(sb + C::OFF_DY, kk, kQ),
+                mma_bf16(tmem + C::TM_C, bdesc_k(sb + C::OFF_DY, kk, kQ),
                          bdesc_k(sb + C::OFF_GIN, kk, NST), C::ID_KN, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < kPc / 16; ++kk)
-                mma_bf16(tmem + C::TM_DB, bdesc_k(sb + C::OFF_X, kk, kQ),
-                         bdesc_k(sb + C::OFF_DG, kk, NST), C::ID_KN, kk > 0);
             mma_commit(&bar[1]);
             issued = 1;
         } else {
-            // nothing issued: let the copies land before the CTA exits
-            drain(&bar[0], 0, 100000000ull);
+            drain(&bar[0], 0, 100000000ull);   // let the copies land before the CTA exits
         }
     }
 
-    // ---- first epilogue: masks, band and decay sums, state-term dot products, row scales
     const int q4 = w & 3, wg = w >> 2, hf = lane >> 4;
     const int t = 16 * q4 + (lane & 15);          // this thread's accumulator row
     const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
+    auto flag_ok = [&]() { return *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u; };
+
+    // ---- first epilogue: masks, band and decay sums, <C~_t, (dY g^T)_t>, row scale f
     bool ok = warp_wait_b(&bar[1], 0, ab);
     tc_fence_after();
+    if (ok) {   // the angle table moves to the g_in tile (read by round 1, now free)
+        constexpr int CP = kQ * NH * 4 / 16 / 256;
+        const uint4* src = reinterpret_cast<const uint4*>(psi0);
+        uint4* dst = reinterpret_cast<uint4*>(psi1);
+#pragma unroll
+        for (int i = 0; i < CP; ++i) dst[tid + 256 * i] = src[tid + 256 * i];
+    }
+    __syncthreads();
+    ok = ok && flag_ok();
     if (ok) {
         const float crt = k.cr[t];
-        // S and dY X^T: columns cb + 32 hf + i
         {
             const int cb = 16 * wg, col0 = cb + 32 * hf;
             uint32_t sv[16], gv[16];
-            ld_blk<64>(tq, C::TM_S, cb, sv);
+            ld_blk<64>(tq, C::TM_A, cb, sv);
             ld_blk<64>(tq, C::TM_GX, cb, gv);
             tmem_wait_ld();
             float ca[16], cbv[16], rsum = 0.f, ddiag = 0.f;
-            uint32_t ms[8], ds[8];
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                float mv[2], dvv[2];
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t ms[4], ds[4];
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int s = col0 + i + e;
-                    const bool in = s <= t;
-                    const float E = in ? ex2f((crt - k.cr[s]) * kLog2e) : 0.f;
-                    const float om = in ? k.gam[s] + (s < t ? k.nx[s] : 0.f) : 0.f;
-                    const float L = E * om;
-                    const float S = __uint_as_float(sv[i + e]), G = __uint_as_float(gv[i + e]);
-                    mv[e] = S * L;
-                    dvv[e] = G * L;
-                    const float dL = S * G;
-                    const float dom = dL * E;
-                    ca[i + e] = dom * om;
-                    cbv[i + e] = dom;
-                    rsum += dom * om;
-                    if (s == t) {
-                        dgd[t] = dom;
-                        ddiag = G;
+                for (int i2 = 0; i2 < 8; i2 += 2) {
+                    float mv[2], dvv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int i = 8 * hh + i2 + e;
+                        const int s = col0 + i;
+                        const bool in = s <= t;
+                        const float E = in ? ex2f((crt - k.cr[s]) * kLog2e) : 0.f;
+                        const float om = in ? k.gam[s] + (s < t ? k.nx[s] : 0.f) : 0.f;
+                        const float L = E * om;
+                        const float S = __uint_as_float(sv[i]), G = __uint_as_float(gv[i]);
+                        mv[e] = S * L;
+                        dvv[e] = G * L;
+                        const float dom = S * G * E;
+                        ca[i] = dom * om;
+                        cbv[i] = dom;
+                        rsum += dom * om;
+                        if (s == t) {
+                            dgd[t] = dom;
+                            ddiag = G;
+                        }
                     }
+                    ms[i2 / 2] = pack_bf16x2(mv[0], mv[1]);
+                    ds[i2 / 2] = pack_bf16x2(dvv[0], dvv[1]);
                 }
-                ms[i / 2] = pack_bf16x2(mv[0], mv[1]);
-                ds[i / 2] = pack_bf16x2(dvv[0], dvv[1]);
+                *reinterpret_cast<uint4*>(sm + C::OFF_MS + sw128_off(t, col0 + 8 * hh)) =
+                    make_uint4(ms[0], ms[1], ms[2], ms[3]);
+                *reinterpret_cast<uint4*>(sm + C::OFF_DS + sw128_off(t, col0 + 8 * hh)) =
+                    make_uint4(ds[0], ds[1], ds[2], ds[3]);
             }
-            *reinterpret_cast<uint4*>(sm + C::OFF_MS + sw128_off(t, col0)) = make_uint4(ms[0], ms[1], ms[2], ms[3]);
-            *reinterpret_cast<uint4*>(sm + C::OFF_MS + sw128_off(t, col0 + 8)) = make_uint4(ms[4], ms[5], ms[6], ms[7]);
-            *reinterpret_cast<uint4*>(sm + C::OFF_DS + sw128_off(t, col0)) = make_uint4(ds[0], ds[1], ds[2], ds[3]);
-            *reinterpret_cast<uint4*>(sm + C::OFF_DS + sw128_off(t, col0 + 8)) = make_uint4(ds[4], ds[5], ds[6], ds[7]);
             if (ddiag != 0.f) atomicAdd(&misc2[0], ddiag);
             const float csum = colsum16(ca, lane), gsum = colsum16(cbv, lane);
             atomicAdd(&cs[col0 + (lane & 15)], csum);
@@ -766,38 +809,14 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
             rsum += __shfl_xor_sync(0xffffffffu, rsum, 16);
             if (hf == 0) atomicAdd(&rs[t], rsum);
         }
-        // B~ dg: <X_s, .> for the state-update weight, then the row scale e_s w_s
-        {
-            const int cb = 16 * wg, col0 = cb + 32 * hf;
-            uint32_t v[16];
-            ld_blk<64>(tq, C::TM_DX, cb, v);
-            tmem_wait_ld();
-            const uint4 x0 = *reinterpret_cast<const uint4*>(sm + C::OFF_X + sw128_off(t, col0));
-            const uint4 x1 = *reinterpret_cast<const uint4*>(sm + C::OFF_X + sw128_off(t, col0 + 8));
-            const uint32_t xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            float d = 0.f;
-            const float sc = k.ew[t];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
-                d = fmaf(bf16lo(xs[i]), a0, fmaf(bf16hi(xs[i]), a1, d));
-                v[2 * i] = __float_as_uint(a0 * sc);
-                v[2 * i + 1] = __float_as_uint(a1 * sc);
-            }
-            st_blk<64>(tq, C::TM_DX, cb, v);
-            d += __shfl_xor_sync(0xffffffffu, d, 16);
-            if (hf == 0) atomicAdd(&dv[t], d);
-        }
-        // dY g^T: <C~_t, .> for the output term, then the row scale f_t; X dg^T: row scale e w
         {
             float d = 0.f;
-            const float sf = k.ff[t], se = k.ew[t];
+            const float sf = k.ff[t];
 #pragma unroll
             for (int m = 0; m < NST / 64; ++m) {
                 const int cb = 16 * (wg + 2 * m), col0 = cb + (NST / 2) * hf;
-                uint32_t v[16], u2[16];
-                ld_blk<NST>(tq, C::TM_DC, cb, v);
-                ld_blk<NST>(tq, C::TM_DB, cb, u2);
+                uint32_t v[16];
+                ld_blk<NST>(tq, C::TM_C, cb, v);
                 tmem_wait_ld();
                 const uint4 c0 = *reinterpret_cast<const uint4*>(sm + C::OFF_C + tile_off(t, col0, kQ));
                 const uint4 c1 = *reinterpret_cast<const uint4*>(sm + C::OFF_C + tile_off(t, col0 + 8, kQ));
@@ -809,10 +828,7 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
                     v[2 * i] = __float_as_uint(a0 * sf);
                     v[2 * i + 1] = __float_as_uint(a1 * sf);
                 }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) u2[i] = __float_as_uint(__uint_as_float(u2[i]) * se);
-                st_blk<NST>(tq, C::TM_DC, cb, v);
-                st_blk<NST>(tq, C::TM_DB, cb, u2);
+                st_blk<NST>(tq, C::TM_C, cb, v);
             }
             d += __shfl_xor_sync(0xffffffffu, d, 16);
             if (hf == 0) atomicAdd(&qz[t], d);
@@ -822,22 +838,18 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    ok = ok && *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u;
+    ok = ok && flag_ok();
     if (tid == 0 && issued == 1) {
         if (ok) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kQ / 16; ++kk)
-                mma_bf16(tmem + C::TM_DX, bdesc_mn(sb + C::OFF_MS, kk, kQ * 128),
-                         bdesc_mn(sb + C::OFF_DY, kk, kQ * 128), C::ID_MSDY, 1);
-#pragma unroll
-            for (int kk = 0; kk < kQ / 16; ++kk)
-                mma_bf16(tmem + C::TM_DC, bdesc_k(sb + C::OFF_DS, kk, kQ),
+                mma_bf16(tmem + C::TM_C, bdesc_k(sb + C::OFF_DS, kk, kQ),
                          bdesc_mn(sb + C::OFF_B, kk, kQ * 128), C::ID_DSB, 1);
 #pragma unroll
-            for (int kk = 0; kk < kQ / 16; ++kk)
-                mma_bf16(tmem + C::TM_DB, bdesc_mn(sb + C::OFF_DS, kk, kQ * 128),
-                         bdesc_mn(sb + C::OFF_C, kk, kQ * 128), C::ID_DSC, 1);
+            for (int kk = 0; kk < NST / 16; ++kk)
+                mma_bf16(tmem + C::TM_A, bdesc_k(sb + C::OFF_B, kk, kQ),
+                         bdesc_mn(sb + C::OFF_DG, kk, tile_bytes), C::ID_BDG, kk > 0);
             mma_commit(&bar[2]);
             issued = 2;
         } else {
@@ -845,16 +857,107 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
         }
     }
 
-    // ---- second epilogue: dX; dC~, dB~ rotated back, angle gradients per (token, pair)
+    // ---- second epilogue: <X_s, (B~ dg)_s>, row scale e w, X <- e w X; dC~ rotated back
+    const long long tg = t0 + t;
+    const bool live = t < nv;
+    const size_t grow = (((size_t)b * a.T + (live ? tg : 0)) * a.G + g) * NST;
+    constexpr int NB = NST / 64;          // 16-column blocks per thread in an N-wide tile
+    float dps[NB * 8];                    // this thread's angle gradients (from dC~)
     ok = ok && warp_wait_b(&bar[2], 0, ab);
     tc_fence_after();
     if (ok) {
-        const long long tg = t0 + t;
-        const bool live = t < nv;
         {
             const int cb = 16 * wg, col0 = cb + 32 * hf;
             uint32_t v[16];
-            ld_blk<64>(tq, C::TM_DX, cb, v);
+            ld_blk<64>(tq, C::TM_A, cb, v);
+            tmem_wait_ld();
+            uint4* xp0 = reinterpret_cast<uint4*>(sm + C::OFF_X + sw128_off(t, col0));
+            uint4* xp1 = reinterpret_cast<uint4*>(sm + C::OFF_X + sw128_off(t, col0 + 8));
+            const uint4 x0 = *xp0, x1 = *xp1;
+            const uint32_t xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            float d = 0.f;
+            const float sc = k.ew[t];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
+                d = fmaf(bf16lo(xs[i]), a0, fmaf(bf16hi(xs[i]), a1, d));
+                v[2 * i] = __float_as_uint(a0 * sc);
+                v[2 * i + 1] = __float_as_uint(a1 * sc);
+            }
+            st_blk<64>(tq, C::TM_A, cb, v);
+            *xp0 = make_uint4(scale2(x0.x, sc), scale2(x0.y, sc), scale2(x0.z, sc), scale2(x0.w, sc));
+            *xp1 = make_uint4(scale2(x1.x, sc), scale2(x1.y, sc), scale2(x1.z, sc), scale2(x1.w, sc));
+            d += __shfl_xor_sync(0xffffffffu, d, 16);
+            if (hf == 0) atomicAdd(&dv[t], d);
+        }
+        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
+#pragma unroll
+        for (int m = 0; m < NB; ++m) {
+            const int cb = 16 * (wg + 2 * m), col0 = cb + (NST / 2) * hf;
+            uint4 rc[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+            if (live) {
+                rc[0] = *reinterpret_cast<const uint4*>(Cg + grow + col0);
+                rc[1] = *reinterpret_cast<const uint4*>(Cg + grow + col0 + 8);
+            }
+            uint32_t vc[16];
+            ld_blk<NST>(tq, C::TM_C, cb, vc);
+            tmem_wait_ld();
+            const uint32_t cw[8] = {rc[0].x, rc[0].y, rc[0].z, rc[0].w, rc[1].x, rc[1].y, rc[1].z, rc[1].w};
+            float oc[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float sn, cs2;
+                __sincosf(psi1[psi_idx<NH>(t, col0 / 2 + i)], &sn, &cs2);
+                const float c0 = bf16lo(cw[i]), c1 = bf16hi(cw[i]);
+                const float ct0 = fmaf(cs2, c0, sn * c1), ct1 = fmaf(cs2, c1, -sn * c0);
+                const float dc0 = __uint_as_float(vc[2 * i]), dc1 = __uint_as_float(vc[2 * i + 1]);
+                dps[8 * m + i] = fmaf(dc0, ct1, -dc1 * ct0);
+                oc[2 * i] = fmaf(cs2, dc0, -sn * dc1);
+                oc[2 * i + 1] = fmaf(sn, dc0, cs2 * dc1);
+            }
+            if (live) {
+                float4* dC = reinterpret_cast<float4*>(a.dC + grow + col0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    atomicAdd(dC + i, make_float4(oc[4 * i], oc[4 * i + 1], oc[4 * i + 2], oc[4 * i + 3]));
+            }
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    ok = ok && flag_ok();
+    if (tid == 0 && issued == 2) {
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kQ / 16; ++kk)
+                mma_bf16(tmem + C::TM_A, bdesc_mn(sb + C::OFF_MS, kk, kQ * 128),
+                         bdesc_mn(sb + C::OFF_DY, kk, kQ * 128), C::ID_MSDY, 1);
+#pragma unroll
+            for (int kk = 0; kk < kPc / 16; ++kk)
+                mma_bf16(tmem + C::TM_C, bdesc_k(sb + C::OFF_X, kk, kQ),
+                         bdesc_k(sb + C::OFF_DG, kk, NST), C::ID_KN, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < kQ / 16; ++kk)
+                mma_bf16(tmem + C::TM_C, bdesc_mn(sb + C::OFF_DS, kk, kQ * 128),
+                         bdesc_mn(sb + C::OFF_C, kk, kQ * 128), C::ID_DSC, 1);
+            mma_commit(&bar[3]);
+            issued = 3;
+        } else {
+            drain(&bar[2], 0, 100000000ull);
+        }
+    }
+
+    // ---- third epilogue: dX; dB~ rotated back; the angle gradient of every (token, pair)
+    ok = ok && warp_wait_b(&bar[3], 0, ab);
+    tc_fence_after();
+    if (ok) {
+        {
+            const int cb = 16 * wg, col0 = cb + 32 * hf;
+            uint32_t v[16];
+            ld_blk<64>(tq, C::TM_A, cb, v);
             tmem_wait_ld();
             const float Dh = a.D ? a.D[h] : 0.f;
             const uint4 y0 = *reinterpret_cast<const uint4*>(sm + C::OFF_DY + sw128_off(t, col0));
@@ -870,76 +973,62 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
                                          fmaf(Dh, bf16hi(ys[2 * i + 1]), __uint_as_float(v[4 * i + 3])));
             }
         }
-        const size_t grow = (((size_t)b * a.T + (live ? tg : 0)) * a.G + g) * NST;
         const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
-        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
 #pragma unroll
-        for (int m = 0; m < NST / 64; ++m) {
+        for (int m = 0; m < NB; ++m) {
             const int cb = 16 * (wg + 2 * m), col0 = cb + (NST / 2) * hf;
-            uint32_t vc[16], vb[16];
-            ld_blk<NST>(tq, C::TM_DC, cb, vc);
-            ld_blk<NST>(tq, C::TM_DB, cb, vb);
-            tmem_wait_ld();
             uint4 rb[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-            uint4 rc[2] = {rb[0], rb[1]};
             if (live) {
                 rb[0] = *reinterpret_cast<const uint4*>(Bg + grow + col0);
                 rb[1] = *reinterpret_cast<const uint4*>(Bg + grow + col0 + 8);
-                rc[0] = *reinterpret_cast<const uint4*>(Cg + grow + col0);
-                rc[1] = *reinterpret_cast<const uint4*>(Cg + grow + col0 + 8);
             }
+            uint32_t vb[16];
+            ld_blk<NST>(tq, C::TM_C, cb, vb);
+            tmem_wait_ld();
             const uint32_t bw[8] = {rb[0].x, rb[0].y, rb[0].z, rb[0].w, rb[1].x, rb[1].y, rb[1].z, rb[1].w};
-            const uint32_t cw[8] = {rc[0].x, rc[0].y, rc[0].z, rc[0].w, rc[1].x, rc[1].y, rc[1].z, rc[1].w};
-            float oc[16], ob[16];
+            float ob[16];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int j = col0 / 2 + i;
                 float sn, cs2;
-                __sincosf(psi[t * PSI_LD + j], &sn, &cs2);
-                const float c0 = bf16lo(cw[i]), c1 = bf16hi(cw[i]);
+                __sincosf(psi1[psi_idx<NH>(t, j)], &sn, &cs2);
                 const float b0 = bf16lo(bw[i]), b1 = bf16hi(bw[i]);
-                const float ct0 = fmaf(cs2, c0, sn * c1), ct1 = fmaf(cs2, c1, -sn * c0);
                 const float bt0 = fmaf(cs2, b0, sn * b1), bt1 = fmaf(cs2, b1, -sn * b0);
-                const float dc0 = __uint_as_float(vc[2 * i]), dc1 = __uint_as_float(vc[2 * i + 1]);
                 const float db0 = __uint_as_float(vb[2 * i]), db1 = __uint_as_float(vb[2 * i + 1]);
-                psi[t * PSI_LD + j] = fmaf(dc0, ct1, -dc1 * ct0) + fmaf(db0, bt1, -db1 * bt0);
-                oc[2 * i] = fmaf(cs2, dc0, -sn * dc1);
-                oc[2 * i + 1] = fmaf(sn, dc0, cs2 * dc1);
+                psi1[psi_idx<NH>(t, j)] = dps[8 * m + i] + fmaf(db0, bt1, -db1 * bt0);
                 ob[2 * i] = fmaf(cs2, db0, -sn * db1);
                 ob[2 * i + 1] = fmaf(sn, db0, cs2 * db1);
             }
             if (live) {
-                float4* dC = reinterpret_cast<float4*>(a.dC + grow + col0);
                 float4* dB = reinterpret_cast<float4*>(a.dB + grow + col0);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    atomicAdd(dC + i, make_float4(oc[4 * i], oc[4 * i + 1], oc[4 * i + 2], oc[4 * i + 3]));
+                for (int i = 0; i < 4; ++i)
                     atomicAdd(dB + i, make_float4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]));
-                }
             }
         }
     }
+    // TMEM is no longer read: release it for the SM's other CTA
+    if (tid == 0 && issued > 0) drain(&bar[issued], 0, 100000000ull);
+    tc_fence_before();
     __syncthreads();
-    ok = ok && *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u;
+    if (w == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+    ok = ok && flag_ok();
+
+    // angles: suffix sums over the chunk's tokens per (pair, token segment), then the
+    // segments' totals; dtheta gets dang (x dt), the dt gradient dang . theta
+    float loc[TPS];
     if (ok) {
-        // angles: suffix sums over the chunk's tokens per pair; dtheta gets dang (x dt), the
-        // dt gradient dang . theta (summed over pairs below)
-        if (tid < NH) {
-            const int j = tid;
-            float sacc = 0.f;
-            for (int u = kQ - 1; u >= 0; --u) {
-                sacc += psi[u * PSI_LD + j];
-                float contrib = 0.f;
-                if (u < nv) {
-                    const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
-                    const float th = a.theta[row * NH + j];
-                    atomicAdd(&a.dtheta[row * NH + j], angle ? sacc : sacc * k.dd[u]);
-                    contrib = angle ? 0.f : sacc * th;
-                }
-                psi[u * PSI_LD + j] = contrib;
-            }
-            p.dtot[cc * NH + j] = sacc;
+        float r = 0.f;
+#pragma unroll
+        for (int i = TPS - 1; i >= 0; --i) {
+            r += psi1[psi_idx<NH>(sg * TPS + i, jj)];
+            loc[i] = r;
         }
+        segt[sg * NH + jj] = r;
         // the log-decay gradient of every token (chunk-local: its terms sum to zero over the
         // chunk, so the suffix sums that reach dA and dt stay inside the chunk)
         if (tid < kQ) {
@@ -953,6 +1042,34 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
         }
     }
     __syncthreads();
+    if (ok) {
+        float off = 0.f;
+        for (int s2 = sg + 1; s2 < SEGS; ++s2) off += segt[s2 * NH + jj];
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) {
+            const int u = sg * TPS + i;
+            const float dang = loc[i] + off;
+            float contrib = 0.f;
+            if (u < nv) {
+                const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
+                atomicAdd(&a.dtheta[row * NH + jj], angle ? dang : dang * k.dd[u]);
+                if (!angle) contrib = dang * a.theta[row * NH + jj];
+            }
+            psi1[psi_idx<NH>(u, jj)] = contrib;
+        }
+        if (sg == 0) p.dtot[cc * NH + jj] = loc[0] + off;
+    }
+    __syncthreads();
+    if (ok) {
+        // the dt gradient through the angles: four threads per token
+        const int u = tid >> 2, qq = tid & 3;
+        float sacc = 0.f;
+#pragma unroll
+        for (int i = 0; i < NH / 4; ++i) sacc += psi1[psi_idx<NH>(u, qq * (NH / 4) + i)];
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
+        if (qq == 0) dpt[u] = sacc;
+    }
     if (ok && tid < kQ) {
         const int u = tid;
         float v = dcm[u];
@@ -972,10 +1089,8 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
     if (ok && tid < kQ) {
         const int u = tid;
         const float dda = dcm[u] + (w == 0 ? misc2[3] : 0.f);
-        float dpt = 0.f;
-        for (int j = 0; j < NH; ++j) dpt += psi[u * PSI_LD + j];
         const float dga = k.ee[u] * dv[u] + ga[u];
-        float ddt = fmaf(dda, k.aa[u], fmaf(dga, k.ll[u], dpt));
+        float ddt = fmaf(dda, k.aa[u], fmaf(dga, k.ll[u], dpt[u]));
         float dlam = dga * k.dd[u];
         if (u > 0) {
             ddt = fmaf(dnx[u - 1], 1.f - k.ll[u], ddt);
@@ -995,16 +1110,6 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
         if (u == kQ - 1) p.spill[cc] = dnx[u];
         if (u == 0 && a.D && a.dD) atomicAdd(&a.dD[h], misc2[0]);
     }
-    if (tid == 0) {
-        if (issued == 2) drain(&bar[2], 0, 100000000ull);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (w == 0) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
 }
 
 // ------------------------------------------------------------------------------------
@@ -1013,7 +1118,8 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(const __grid_constant
 __global__ void __launch_bounds__(64) bwd_finish_kernel(const __grid_constant__ TcBwd p) {
     const BwdArgs& a = p.a;
     const int NH = a.N / 2;
-    __shared__ float car[64];
+    __shared__ float car[64], dts[64];
+    __shared__ float ths[kQ][65];
     const int tid = threadIdx.x;
     const int c = (int)(blockIdx.x % p.nch);
     const size_t bh = blockIdx.x / p.nch;
@@ -1021,29 +1127,38 @@ __global__ void __launch_bounds__(64) bwd_finish_kernel(const __grid_constant__ 
     const long long t0 = (long long)c * kQ;
     const int nv = (int)(a.T - t0 < kQ ? a.T - t0 : kQ);
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
+    if (tid < nv) dts[tid] = a.dt[((size_t)b * a.T + t0 + tid) * a.H + h];
     if (tid < NH) {
         float s = p.extra[bh * NH + tid];
+#pragma unroll 4
         for (int c2 = c + 1; c2 < p.nch; ++c2) s += p.dtot[(bh * p.nch + c2) * NH + tid];
         car[tid] = s;
-        for (int u = 0; u < nv; ++u) {
-            const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
-            const float d = a.dt[((size_t)b * a.T + t0 + u) * a.H + h];
-            atomicAdd(&a.dtheta[row * NH + tid], angle ? s : s * d);
+    }
+    if (!angle) {
+#pragma unroll 4
+        for (int i = tid; i < nv * NH; i += 64) {
+            const int u = i / NH, j = i - u * NH;
+            ths[u][j] = a.theta[(((size_t)b * a.T + t0 + u) * a.G + g) * NH + j];
         }
     }
     __syncthreads();
+    if (tid < NH) {
+        const float s = car[tid];
+        for (int u = 0; u < nv; ++u) {
+            const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
+            atomicAdd(&a.dtheta[row * NH + tid], angle ? s : s * dts[u]);
+        }
+    }
     if (tid < nv) {
         const size_t o = ((size_t)b * a.T + t0 + tid) * a.H + h;
         float add = 0.f;
-        if (!angle) {
-            const float* th = a.theta + (((size_t)b * a.T + t0 + tid) * a.G + g) * NH;
-            for (int j = 0; j < NH; ++j) add = fmaf(car[j], th[j], add);
-        }
+        if (!angle)
+            for (int j = 0; j < NH; ++j) add = fmaf(car[j], ths[tid][j], add);
         float dl = 0.f;
         if (tid == 0 && c > 0) {
             const float s = p.spill[bh * p.nch + c - 1];
             add = fmaf(s, 1.f - a.lam[o], add);
-            dl = -s * a.dt[o];
+            dl = -s * dts[0];
         }
         a.ddt[o] += add;
         if (dl != 0.f) a.dlam[o] += dl;
