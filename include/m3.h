@@ -347,6 +347,49 @@ m3_status m3_scan_bwd(const m3_dims* dims, int32_t seqlen, const void* x, const 
                       const void* dy, const float* dhT, const m3_grads* grads, void* workspace,
                       size_t workspace_bytes, uint32_t flags, void* stream);
 
+/* Backward pass of m3_scan_fwd_ex, the prefill with the fused extras, by the chain rule
+ * around the recurrence's backward ("Technical Approach": output gating, BC normalisation,
+ * BC biases; "MIMO Parameterization Choices": the lightweight expansion).  The forward is
+ * the recurrence on effective inputs X = x w_x, Z = z w_z, per-head B_h = B s(B) + B_bias[h]
+ * (s the BCNorm scale, 1 when off), C_h likewise, theta shared as before, followed by the
+ * gate y = y_pre SiLU(Z).  The backward
+ *   - forms the effective inputs (rounded to the io dtype, as the fused kernels use them);
+ *   - with the gate, reruns the forward without it for y_pre (from a copy of state0) and
+ *     takes dL/dy_pre = dy Z sig(Z), dL/dZ = dy y_pre sig(Z) (1 + Z (1 - sig(Z)));
+ *   - runs m3_scan_bwd's recurrence backward on the effective inputs, one group per head
+ *     when the BC map is on;
+ *   - maps back: dx = sum_r dX w_x, dw_x = sum_{b,t} dX x (z likewise), dB = J(sum over the
+ *     group's heads of dB_h) with the RMS scale's Jacobian J(du) = s du - (s^3/N) v <du, v>,
+ *     dB_bias[h] = sum_{b,t,r} dB_h (plus the carried B_prev's share), C likewise.
+ *   in : the forward call's inputs, state0 and extras (as given to m3_scan_fwd_ex), dy in the
+ *        layout of y, dhT or NULL.
+ *   out: grads as m3_scan_bwd (dx [b][T][H][P] with x_expand; dx_prev refers to the
+ *        expanded x_prev the state holds); m3_extra_grads below, fp32, caller-owned,
+ *        overwritten.  An extras pointer that is NULL or all zero runs m3_scan_bwd itself.
+ *   The parameter gradients (dx_expand, dz_expand, dB_bias, dC_bias) and, on the chunked
+ *   path, the group-shared ones are sums accumulated with atomics.  Supported: the shapes of
+ *   m3_scan_bwd (the SISO bf16 P 64 shapes run the chunked tensor-core backward).
+ *   Workspace: m3_scan_bwd_workspace_bytes_ex (the recurrence backward's own workspace
+ *   first, then the effective inputs, their gradients and, with the gate, the forward's
+ *   workspace, a state copy and y_pre). */
+typedef struct {
+    float* dz;         /* layout of z ([b][T][H][P] with z_expand); needed iff the gate is on */
+    float* dB_bias;    /* [H][N]; needed iff B_bias */
+    float* dC_bias;    /* [H][N]; needed iff C_bias */
+    float* dx_expand;  /* [H][R][P]; needed iff x_expand */
+    float* dz_expand;  /* [H][R][P]; needed iff z_expand */
+} m3_extra_grads;
+
+m3_status m3_scan_bwd_workspace_bytes_ex(const m3_dims* dims, int32_t seqlen,
+                                         const m3_extras* extras, size_t* bytes);
+
+m3_status m3_scan_bwd_ex(const m3_dims* dims, int32_t seqlen, const void* x, const void* B,
+                         const void* C, const float* dt, const float* A, const float* lam,
+                         const float* theta, const float* D, const m3_state* state0,
+                         const m3_extras* extras, const void* dy, const float* dhT,
+                         const m3_grads* grads, const m3_extra_grads* extra_grads,
+                         void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
+
 /* Synchronise `stream` and report the device-side status word in `workspace`:
  * M3_OK, M3_ERR_TIMEOUT when a bounded wait gave up, or M3_ERR_RANGE when the debug
  * scan of M3_FLAG_DEBUG_CHECKS found an input outside its range. */

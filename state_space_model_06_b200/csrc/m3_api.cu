@@ -499,6 +499,207 @@ m3_status m3_scan_bwd(const m3_dims* d, int32_t seqlen, const void* x, const voi
     return launch_status(launch_scan_bwd(a, R, d->io_dtype, s));
 }
 
+}  // extern "C"
+
+namespace {
+
+// the fused extras of a backward call: which parts are on and where their buffers sit in
+// the workspace (byte offsets; the recurrence backward's own workspace comes first, so that
+// its status word is the call's)
+struct ExLayout {
+    m3_dims de;   // effective dims: one group per head when the BC map is on
+    bool xe, bc, gate;
+    size_t inner, fwd, fwd_bytes, hS, xpS, bpS, ypre, dypre, dZ, X, dX, Bh, Ch, Bph, thh;
+    size_t dBh, dCh, dBph, dthh, bytes;
+};
+
+bool ex_any(const m3_extras* ex) {
+    return ex && (ex->z || ex->B_bias || ex->C_bias || ex->bc_norm_eps > 0.f || ex->x_expand ||
+                  ex->z_expand);
+}
+
+ExLayout ex_layout(const m3_dims* d, int32_t T, const m3_extras* ex) {
+    ExLayout L;
+    std::memset(&L, 0, sizeof(L));
+    L.xe = ex->x_expand != nullptr;
+    L.bc = ex->B_bias || ex->C_bias || ex->bc_norm_eps > 0.f;
+    L.gate = ex->z != nullptr;
+    L.de = *d;
+    if (L.bc) L.de.ngroups = d->nheads;
+    const size_t io = d->io_dtype == M3_BF16 ? 2 : 4;
+    const size_t b = d->batch, H = d->nheads, R = d->rank, P = d->headdim, N = d->dstate;
+    const size_t bt = b * (size_t)T, Ge = L.de.ngroups;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    size_t inner = 0;
+    m3_scan_bwd_workspace_bytes(&L.de, T, &inner);
+    L.inner = take(inner);
+    if (L.gate) {
+        m3_scan_workspace_bytes(&L.de, T, 64, &L.fwd_bytes);
+        L.fwd = take(L.fwd_bytes);
+        L.hS = take(b * H * N * P * 4);
+        L.xpS = take(b * H * R * P * io);
+        L.bpS = take(b * Ge * R * N * io);
+        L.ypre = take(bt * H * R * P * io);
+        L.dypre = take(bt * H * R * P * io);
+        if (ex->z_expand) L.dZ = take(bt * H * R * P * 4);
+    }
+    if (L.xe) {
+        L.X = take(bt * H * R * P * io);
+        L.dX = take(bt * H * R * P * 4);
+    }
+    if (L.bc) {
+        L.Bh = take(bt * H * R * N * io);
+        L.Ch = take(bt * H * R * N * io);
+        L.Bph = take(b * H * R * N * io);
+        L.thh = take(bt * H * (N / 2) * 4);
+        L.dBh = take(bt * H * R * N * 4);
+        L.dCh = take(bt * H * R * N * 4);
+        L.dBph = take(b * H * R * N * 4);
+        L.dthh = take(bt * H * (N / 2) * 4);
+    }
+    L.bytes = o;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+m3_status m3_scan_bwd_workspace_bytes_ex(const m3_dims* d, int32_t seqlen, const m3_extras* ex,
+                                         size_t* bytes) {
+    if (!ex_any(ex)) return m3_scan_bwd_workspace_bytes(d, seqlen, bytes);
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    if (!bytes) return M3_ERR_NULL;
+    if (seqlen < 0 || !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;
+    *bytes = ex_layout(d, seqlen, ex).bytes;
+    return M3_OK;
+}
+
+m3_status m3_scan_bwd_ex(const m3_dims* d, int32_t seqlen, const void* x, const void* B,
+                         const void* C, const float* dt, const float* A, const float* lam,
+                         const float* theta, const float* D, const m3_state* state0,
+                         const m3_extras* ex, const void* dy, const float* dhT,
+                         const m3_grads* gr, const m3_extra_grads* xg, void* workspace,
+                         size_t workspace_bytes, uint32_t flags, void* stream) {
+    if (!ex_any(ex))
+        return m3_scan_bwd(d, seqlen, x, B, C, dt, A, lam, theta, D, state0, dy, dhT, gr,
+                           workspace, workspace_bytes, flags, stream);
+    m3_status st = check_dims(d);
+    if (st != M3_OK) return st;
+    if (seqlen < 0 || !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;
+    if ((st = check_state(state0)) != M3_OK) return st;
+    if (!gr || !xg) return M3_ERR_NULL;
+    if (ex->z_expand && !ex->z) return M3_ERR_NULL;
+    if ((ex->z && !xg->dz) || (ex->B_bias && !xg->dB_bias) || (ex->C_bias && !xg->dC_bias) ||
+        (ex->x_expand && !xg->dx_expand) || (ex->z_expand && !xg->dz_expand))
+        return M3_ERR_NULL;
+    if ((ex->z && !aligned(ex->z, 16)) || (ex->x_expand && !aligned(ex->x_expand, 16)) ||
+        (ex->z_expand && !aligned(ex->z_expand, 16)) || (ex->B_bias && !aligned(ex->B_bias, 4)) ||
+        (ex->C_bias && !aligned(ex->C_bias, 4)) || (xg->dz && !aligned(xg->dz, 4)) ||
+        (xg->dB_bias && !aligned(xg->dB_bias, 4)) || (xg->dC_bias && !aligned(xg->dC_bias, 4)) ||
+        (xg->dx_expand && !aligned(xg->dx_expand, 4)) || (xg->dz_expand && !aligned(xg->dz_expand, 4)))
+        return M3_ERR_ALIGN;
+    if (seqlen == 0) return M3_OK;
+    if (!x || !B || !C || !dt || !A || !lam || !theta || !dy) return M3_ERR_NULL;
+    if (!gr->dx || !gr->dB || !gr->dC || !gr->ddt || !gr->dA || !gr->dlam || !gr->dtheta ||
+        !gr->dh0 || !gr->dx_prev || !gr->dB_prev)
+        return M3_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(dy, 16))
+        return M3_ERR_ALIGN;
+    if (!scan_bwd_shape_ok(d->dstate, d->headdim, d->rank)) return M3_ERR_UNSUPPORTED;
+    const ExLayout L = ex_layout(d, seqlen, ex);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.bytes) return M3_ERR_WORKSPACE;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(workspace);
+    const size_t io = d->io_dtype == M3_BF16 ? 2 : 4;
+    const size_t b = d->batch, H = d->nheads, R = d->rank, P = d->headdim, N = d->dstate;
+    ExBwdPlan pl;
+    std::memset(&pl, 0, sizeof(pl));
+    pl.batch = d->batch; pl.H = d->nheads; pl.G = d->ngroups; pl.R = R; pl.P = P; pl.N = N;
+    pl.T = seqlen; pl.eps = ex->bc_norm_eps;
+    pl.x = x; pl.B = B; pl.C = C; pl.B_prev = state0->B_prev; pl.theta = theta; pl.z = ex->z;
+    pl.B_bias = ex->B_bias; pl.C_bias = ex->C_bias; pl.x_expand = ex->x_expand;
+    pl.z_expand = ex->z_expand; pl.dy = dy;
+    pl.dx = gr->dx; pl.dB = gr->dB; pl.dC = gr->dC; pl.dB_prev = gr->dB_prev;
+    pl.dtheta = gr->dtheta; pl.dz = xg->dz; pl.dB_bias = xg->dB_bias; pl.dC_bias = xg->dC_bias;
+    pl.dx_expand = xg->dx_expand; pl.dz_expand = xg->dz_expand;
+    if (L.xe) {
+        pl.X = base + L.X;
+        pl.dX = reinterpret_cast<float*>(base + L.dX);
+    }
+    if (L.bc) {
+        pl.Bh = base + L.Bh; pl.Ch = base + L.Ch; pl.Bph = base + L.Bph;
+        pl.thh = reinterpret_cast<float*>(base + L.thh);
+        pl.dBh = reinterpret_cast<float*>(base + L.dBh);
+        pl.dCh = reinterpret_cast<float*>(base + L.dCh);
+        pl.dBph = reinterpret_cast<float*>(base + L.dBph);
+        pl.dthh = reinterpret_cast<float*>(base + L.dthh);
+    }
+    if (L.gate) {
+        pl.ypre = base + L.ypre;
+        pl.dy_pre = base + L.dypre;
+        pl.dZ = ex->z_expand ? reinterpret_cast<float*>(base + L.dZ) : xg->dz;
+    }
+    // the parameter gradients are sums accumulated with atomics
+    float* zero[] = {xg->dx_expand, xg->dz_expand, xg->dB_bias, xg->dC_bias};
+    const size_t zn[] = {H * R * P, H * R * P, H * N, H * N};
+    for (int i = 0; i < 4; ++i)
+        if (zero[i] && cudaMemsetAsync(zero[i], 0, zn[i] * sizeof(float), s) != cudaSuccess)
+            return M3_ERR_CUDA;
+    cudaError_t e = launch_ex_bwd_inputs(pl, d->io_dtype, s);
+    if (e != cudaSuccess) return launch_status(e);
+    const void* Xe = L.xe ? pl.X : x;
+    const void* Be = L.bc ? pl.Bh : B;
+    const void* Ce = L.bc ? pl.Ch : C;
+    const float* the = L.bc ? pl.thh : theta;
+    const void* Bpe = L.bc ? pl.Bph : state0->B_prev;
+    const uint32_t fwd_flags = flags & (M3_FLAG_THETA_IS_ANGLE | M3_FLAG_FORCE_SIMT);
+    if (L.gate) {
+        // the ungated output y_pre: the forward from a copy of the starting state
+        m3_state ss;
+        ss.h = reinterpret_cast<float*>(base + L.hS);
+        ss.x_prev = base + L.xpS;
+        ss.B_prev = base + L.bpS;
+        if (cudaMemcpyAsync(ss.h, state0->h, b * H * N * P * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(ss.x_prev, state0->x_prev, b * H * R * P * io, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(ss.B_prev, Bpe, b * L.de.ngroups * R * N * io, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return M3_ERR_CUDA;
+        st = m3_scan_fwd(&L.de, seqlen, 64, Xe, Be, Ce, dt, A, lam, the, D, &ss, pl.ypre,
+                         base + L.fwd, L.fwd_bytes, fwd_flags, stream);
+        if (st != M3_OK) return st;
+        if ((e = launch_ex_bwd_gate(pl, d->io_dtype, s)) != cudaSuccess) return launch_status(e);
+    }
+    m3_state s0;
+    s0.h = state0->h;
+    s0.x_prev = state0->x_prev;
+    s0.B_prev = const_cast<void*>(Bpe);
+    m3_grads ig = *gr;
+    if (L.xe) ig.dx = pl.dX;
+    if (L.bc) {
+        ig.dB = pl.dBh;
+        ig.dC = pl.dCh;
+        ig.dtheta = pl.dthh;
+        ig.dB_prev = pl.dBph;
+    }
+    size_t inner = 0;
+    m3_scan_bwd_workspace_bytes(&L.de, seqlen, &inner);
+    st = m3_scan_bwd(&L.de, seqlen, Xe, Be, Ce, dt, A, lam, the, D, &s0, L.gate ? pl.dy_pre : dy,
+                     dhT, &ig, base + L.inner, inner, flags, stream);
+    if (st != M3_OK) return st;
+    if (L.gate &&
+        (e = launch_status_or(static_cast<uint32_t*>(workspace),
+                              reinterpret_cast<const uint32_t*>(base + L.fwd), s)) != cudaSuccess)
+        return launch_status(e);
+    return launch_status(launch_ex_bwd_post(pl, d->io_dtype, s));
+}
+
 m3_status m3_query_status(const void* workspace, void* stream) {
     if (!workspace) return M3_ERR_NULL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -80,6 +80,62 @@ size_t scan_bwd_tc_workspace_bytes(int batch, int H, int N, long long T);
 cudaError_t launch_scan_bwd_tc(const BwdArgs& a, void* ws, uint32_t* status,
                                unsigned long long limit_ns, cudaStream_t s);
 
+// sum of per-head partials over the heads of each group (fixed order):
+// out[(o G + g) inner + k] = sum_j in[(o H + g hpg + j) inner + k]
+cudaError_t launch_group_sum(const float* in, float* out, long long outer, int G, int hpg,
+                             int inner, cudaStream_t s);
+
+// backward of the fused extras: the pointers of one call (null where a part is off)
+struct ExBwdPlan {
+    int batch, H, G, R, P, N;
+    long long T;
+    float eps;
+    // the call's inputs
+    const void* x;
+    const void* B;
+    const void* C;
+    const void* B_prev;
+    const float* theta;
+    const void* z;
+    const float* B_bias;
+    const float* C_bias;
+    const float* x_expand;
+    const float* z_expand;
+    const void* dy;
+    // effective inputs (workspace): expanded x, per-head mapped B / C / B_prev and theta,
+    // the ungated output, the gate's dL/dy_pre and dL/dZ
+    void* X;
+    void* Bh;
+    void* Ch;
+    void* Bph;
+    float* thh;
+    void* ypre;
+    void* dy_pre;
+    float* dZ;
+    // the recurrence's gradients of the effective inputs (workspace)
+    float* dX;
+    float* dBh;
+    float* dCh;
+    float* dBph;
+    float* dthh;
+    // outputs
+    float* dx;
+    float* dB;
+    float* dC;
+    float* dB_prev;
+    float* dtheta;
+    float* dz;
+    float* dB_bias;
+    float* dC_bias;
+    float* dx_expand;
+    float* dz_expand;
+};
+cudaError_t launch_ex_bwd_inputs(const ExBwdPlan& pl, int io_dtype, cudaStream_t s);
+cudaError_t launch_ex_bwd_gate(const ExBwdPlan& pl, int io_dtype, cudaStream_t s);
+cudaError_t launch_ex_bwd_post(const ExBwdPlan& pl, int io_dtype, cudaStream_t s);
+// *dst |= *src (device status words)
+cudaError_t launch_status_or(uint32_t* dst, const uint32_t* src, cudaStream_t s);
+
 // B_prev <- B[:, t] for every (batch, group): the previous-token input of the
 // next call, written after every head of the group has read the old value.
 cudaError_t launch_copy_prev(void* B_prev, const void* B, long long T, long long t, int batch,

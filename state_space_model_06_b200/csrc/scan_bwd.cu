@@ -476,15 +476,6 @@ __global__ void batch_sum_kernel(const float* __restrict__ in, float* __restrict
     }
 }
 
-cudaError_t launch_group_sum(const float* in, float* out, long long outer, int G, int hpg,
-                             int inner, cudaStream_t s) {
-    const long long n = outer * G * inner;
-    if (n == 0) return cudaSuccess;
-    const long long blocks = (n + 255) / 256;
-    group_sum_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, s>>>(
-        in, out, outer, G, hpg, inner);
-    return cudaGetLastError();
-}
 
 template <typename IO, int R, int CPM>
 cudaError_t launch_bwd_c(const BwdArgs& a, cudaStream_t s) {
@@ -518,6 +509,16 @@ cudaError_t launch_bwd_io(const BwdArgs& a, int R, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_group_sum(const float* in, float* out, long long outer, int G, int hpg,
+                             int inner, cudaStream_t s) {
+    const long long n = outer * G * inner;
+    if (n == 0) return cudaSuccess;
+    const long long blocks = (n + 255) / 256;
+    group_sum_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, s>>>(
+        in, out, outer, G, hpg, inner);
+    return cudaGetLastError();
+}
 
 bool scan_bwd_shape_ok(int N, int P, int R) {
     if (N < 2 || N > 256 || (N & 1) || P < 1 || P > 64) return false;

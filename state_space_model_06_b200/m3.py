@@ -29,7 +29,7 @@ EXPORTED = ("m3_state_bytes", "m3_state_init", "m3_scan_workspace_bytes", "m3_sc
             "m3_decode_step", "m3_query_status", "m3_scan_fwd_noalloc", "m3_scan_fwd_gated",
             "m3_decode_step_gated", "m3_scan_workspace_bytes_ex", "m3_scan_fwd_ex",
             "m3_decode_step_ex", "m3_scan_bwd_workspace_bytes", "m3_scan_bwd",
-            "m3_status_string")
+            "m3_scan_bwd_workspace_bytes_ex", "m3_scan_bwd_ex", "m3_status_string")
 
 
 class M3Error(RuntimeError):
@@ -52,6 +52,11 @@ class m3_state(ctypes.Structure):
 class m3_grads(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("dx", "dB", "dC", "ddt", "dA", "dlam", "dtheta",
                                                "dD", "dh0", "dx_prev", "dB_prev")]
+
+
+class m3_extra_grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dz", "dB_bias", "dC_bias", "dx_expand",
+                                                "dz_expand")]
 
 
 class m3_extras(ctypes.Structure):
@@ -94,6 +99,10 @@ def load_library(path: str = LIB_PATH):
         lib.m3_scan_bwd_workspace_bytes.argtypes = [dp, i32, szp]
         lib.m3_scan_bwd.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, vp, vp,
                                     ctypes.POINTER(m3_grads), vp, sz, u32, vp]
+        lib.m3_scan_bwd_workspace_bytes_ex.argtypes = [dp, i32, ep, szp]
+        lib.m3_scan_bwd_ex.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sp, ep, vp, vp,
+                                       ctypes.POINTER(m3_grads), ctypes.POINTER(m3_extra_grads),
+                                       vp, sz, u32, vp]
         lib.m3_query_status.argtypes = [vp, vp]
         lib.m3_status_string.argtypes = [ctypes.c_int]
         lib.m3_status_string.restype = ctypes.c_char_p
@@ -355,3 +364,53 @@ def m3_scan_bwd(dims: Dims, seqlen: int, x, B, C, dt, A, lam, theta, D, state0: 
         ctypes.byref(dims.c()), int(seqlen), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A),
         _ptr(lam), _ptr(theta), _ptr(D), ctypes.byref(st), _ptr(dy), _ptr(dhT), ctypes.byref(g),
         _ptr(workspace), ws_bytes, int(flags), _stream(stream)), "m3_scan_bwd")
+
+
+EXTRA_GRAD_NAMES = ("dz", "dB_bias", "dC_bias", "dx_expand", "dz_expand")
+
+
+def alloc_extra_grads(dims: Dims, seqlen: int, ex, device="cuda") -> dict:
+    """fp32 gradient tensors of the parts of ``ex`` (an Extras) that are on."""
+    b, H, P, N, R, T = dims.batch, dims.nheads, dims.headdim, dims.dstate, dims.rank, seqlen
+    f = dict(dtype=torch.float32, device=device)
+    out = {}
+    if ex.z is not None:
+        out["dz"] = torch.empty((b, T, H, P) if ex.z_expand is not None else (b, T, H, R, P), **f)
+    if ex.B_bias is not None:
+        out["dB_bias"] = torch.empty(H, N, **f)
+    if ex.C_bias is not None:
+        out["dC_bias"] = torch.empty(H, N, **f)
+    if ex.x_expand is not None:
+        out["dx_expand"] = torch.empty(H, R, P, **f)
+    if ex.z_expand is not None:
+        out["dz_expand"] = torch.empty(H, R, P, **f)
+    return out
+
+
+def m3_scan_bwd_workspace_bytes_ex(dims: Dims, seqlen: int, ex) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().m3_scan_bwd_workspace_bytes_ex(ctypes.byref(dims.c()), int(seqlen),
+                                                         _ex_ref(ex), ctypes.byref(n)),
+           "m3_scan_bwd_workspace_bytes_ex")
+    return n.value
+
+
+def alloc_bwd_workspace_ex(dims: Dims, seqlen: int, ex, device="cuda") -> torch.Tensor:
+    return torch.zeros(m3_scan_bwd_workspace_bytes_ex(dims, seqlen, ex), dtype=torch.uint8,
+                       device=device)
+
+
+def m3_scan_bwd_ex(dims: Dims, seqlen: int, x, B, C, dt, A, lam, theta, D, state0: State, ex,
+                   dy, dhT, grads: dict, extra_grads: dict, workspace, flags: int = 0,
+                   stream=None):
+    """Backward pass of m3_scan_fwd_ex: gradients into ``grads`` (alloc_grads; dx is
+    [b][T][H][P] with x_expand) and ``extra_grads`` (alloc_extra_grads)."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = state0.c()
+    g = m3_grads(*(_ptr(grads.get(k)) for k in GRAD_NAMES))
+    xg = m3_extra_grads(*(_ptr(extra_grads.get(k)) for k in EXTRA_GRAD_NAMES))
+    _check(load_library().m3_scan_bwd_ex(
+        ctypes.byref(dims.c()), int(seqlen), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A),
+        _ptr(lam), _ptr(theta), _ptr(D), ctypes.byref(st), _ex_ref(ex), _ptr(dy), _ptr(dhT),
+        ctypes.byref(g), ctypes.byref(xg), _ptr(workspace), ws_bytes, int(flags),
+        _stream(stream)), "m3_scan_bwd_ex")
