@@ -631,9 +631,10 @@ def ours(args):
         "clocks": clk.summary(),
     }
 
-    if args.prefill_only:
+    if args.prefill_only or args.bwd_only:
         args.no_decode = args.no_e2e = args.no_cpu = args.no_gate = args.no_mimo = True
         args.no_bwd = args.no_longctx = True
+        args.no_bwd = not args.bwd_only
     if not args.no_decode:
         line["decode"] = {}
         for name in (args.decode or DECODES):
@@ -777,6 +778,8 @@ def main():
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the sequence length (profiling only)")
     ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and CPU legs")
+    ap.add_argument("--bwd-only", action="store_true",
+                    help="the prefill line and the backward leg only (profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

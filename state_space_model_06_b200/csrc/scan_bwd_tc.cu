@@ -47,8 +47,8 @@ constexpr float kLog2e = 1.44269504088896340736f;
 struct TcBwd {
     BwdArgs a;
     int nch;                  // chunks of the call
-    float* V;                 // [BH][nch][N][P] chunk-frame state products
-    float* U;                 // [BH][nch][N][P] chunk-frame adjoint products
+    uint16_t* V;              // [BH][nch][N][P] bf16 chunk-frame state products
+    uint16_t* U;              // [BH][nch][N][P] bf16 chunk-frame adjoint products
     uint16_t* gin;            // [BH][nch] bf16 tile images [N][P] of the entering state
     uint16_t* dgo;            // [BH][nch] bf16 tile images [N][P] of the leaving adjoint
     float* ctot;              // [BH][nch] total log-decay of the chunk
@@ -329,11 +329,11 @@ __global__ void __launch_bounds__(128) bwd_vu_kernel(const __grid_constant__ TcB
     if (ok) {
         const int q = w & 3;
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-        float* Vo = p.V + cc * (size_t)NST * kPc;
-        float* Uo = p.U + cc * (size_t)NST * kPc;
+        uint16_t* Vo = p.V + cc * (size_t)NST * kPc;
+        uint16_t* Uo = p.U + cc * (size_t)NST * kPc;
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-            float* dst0 = m ? Uo : Vo;
+            uint16_t* dst0 = m ? Uo : Vo;
 #pragma unroll
             for (int cb = 0; cb < 32; cb += 16) {
                 uint32_t r[16], r2[16];
@@ -351,17 +351,21 @@ __global__ void __launch_bounds__(128) bwd_vu_kernel(const __grid_constant__ TcB
                     col2 = -1;
                 }
                 tmem_wait_ld();
-                float4* d = reinterpret_cast<float4*>(dst0 + (size_t)n * kPc + col);
+                uint4* d = reinterpret_cast<uint4*>(dst0 + (size_t)n * kPc + col);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    d[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                       __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                for (int i = 0; i < 2; ++i)
+                    d[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                                      pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                                      pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                                      pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
                 if (col2 >= 0) {
-                    float4* d2 = reinterpret_cast<float4*>(dst0 + (size_t)n * kPc + col2);
+                    uint4* d2 = reinterpret_cast<uint4*>(dst0 + (size_t)n * kPc + col2);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        d2[i] = make_float4(__uint_as_float(r2[4 * i]), __uint_as_float(r2[4 * i + 1]),
-                                            __uint_as_float(r2[4 * i + 2]), __uint_as_float(r2[4 * i + 3]));
+                    for (int i = 0; i < 2; ++i)
+                        d2[i] = make_uint4(pack_bf16x2(__uint_as_float(r2[8 * i]), __uint_as_float(r2[8 * i + 1])),
+                                           pack_bf16x2(__uint_as_float(r2[8 * i + 2]), __uint_as_float(r2[8 * i + 3])),
+                                           pack_bf16x2(__uint_as_float(r2[8 * i + 4]), __uint_as_float(r2[8 * i + 5])),
+                                           pack_bf16x2(__uint_as_float(r2[8 * i + 6]), __uint_as_float(r2[8 * i + 7])));
                 }
             }
         }
@@ -413,7 +417,7 @@ __global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant
     for (int c = 0; c < nch; ++c) {
         const size_t cc = bh * nch + c;
         uint8_t* gt = reinterpret_cast<uint8_t*>(p.gin) + cc * NP * 2;
-        const float* V = p.V + cc * NP;
+        const uint16_t* V = p.V + cc * NP;
         const float dec = ex2f(p.ctot[cc] * kLog2e);
 #pragma unroll
         for (int kx = 0; kx < 8; ++kx) {
@@ -421,7 +425,7 @@ __global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant
             if (pc == 0) p.P0[(bh * (nch + 1) + c) * NH + j] = P[kx];
             *reinterpret_cast<uint16_t*>(gt + sw128_off(2 * j, pc)) = to_bf(ge[kx]);
             *reinterpret_cast<uint16_t*>(gt + sw128_off(2 * j + 1, pc)) = to_bf(go[kx]);
-            const float v0 = V[(size_t)(2 * j) * kPc + pc], v1 = V[(size_t)(2 * j + 1) * kPc + pc];
+            const float v0 = bf_at(V, (size_t)(2 * j) * kPc + pc), v1 = bf_at(V, (size_t)(2 * j + 1) * kPc + pc);
             float sn, cs;
             __sincosf(P[kx], &sn, &cs);
             ge[kx] = fmaf(dec, ge[kx], fmaf(cs, v0, sn * v1));
@@ -457,7 +461,7 @@ __global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant
         const size_t cc = bh * nch + c;
         uint8_t* dt_ = reinterpret_cast<uint8_t*>(p.dgo) + cc * NP * 2;
         const uint8_t* gt = reinterpret_cast<const uint8_t*>(p.gin) + cc * NP * 2;
-        const float* Uc = p.U + cc * NP;
+        const uint16_t* Uc = p.U + cc * NP;
         const float dec = ex2f(p.ctot[cc] * kLog2e);
         float s = 0.f;
 #pragma unroll
@@ -468,7 +472,7 @@ __global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant
             const float g0 = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j, pc)) << 16);
             const float g1 = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j + 1, pc)) << 16);
             s = fmaf(de[kx], g0, fmaf(dq[kx], g1, s));
-            const float u0 = Uc[(size_t)(2 * j) * kPc + pc], u1 = Uc[(size_t)(2 * j + 1) * kPc + pc];
+            const float u0 = bf_at(Uc, (size_t)(2 * j) * kPc + pc), u1 = bf_at(Uc, (size_t)(2 * j + 1) * kPc + pc);
             float sn, cs;
             __sincosf(p.P0[(bh * (nch + 1) + c) * NH + j], &sn, &cs);
             de[kx] = fmaf(dec, de[kx], fmaf(cs, u0, sn * u1));
@@ -1179,8 +1183,8 @@ Layout layout(int batch, int H, int N, long long T) {
         o += (bytes + 255) / 256 * 256;
         return at;
     };
-    L.V = take(BH * nch * NP * 4);
-    L.U = take(BH * nch * NP * 4);
+    L.V = take(BH * nch * NP * 2);
+    L.U = take(BH * nch * NP * 2);
     L.gin = take(BH * nch * NP * 2);
     L.dgo = take(BH * nch * NP * 2);
     L.ctot = take(BH * nch * 4);
@@ -1226,8 +1230,8 @@ cudaError_t launch_scan_bwd_tc(const BwdArgs& a, void* ws, uint32_t* status, uns
     TcBwd p;
     p.a = a;
     p.nch = (int)((a.T + kQ - 1) / kQ);
-    p.V = reinterpret_cast<float*>(base + L.V);
-    p.U = reinterpret_cast<float*>(base + L.U);
+    p.V = reinterpret_cast<uint16_t*>(base + L.V);
+    p.U = reinterpret_cast<uint16_t*>(base + L.U);
     p.gin = reinterpret_cast<uint16_t*>(base + L.gin);
     p.dgo = reinterpret_cast<uint16_t*>(base + L.dgo);
     p.ctot = reinterpret_cast<float*>(base + L.ctot);
