@@ -643,74 +643,86 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     }
     if (w == 1) chunk_coefs(a, b, h, t0, k);
     for (int i = tid; i < C::NACC * kQ + 4; i += 256) acc[i] = 0.f;
-    // angles: thread (pair jj, token segment sg) sums its segment's angles
+    // Every global input of the chunk is requested before any of it is used: the angle
+    // prefix's theta and dt, the chunk-start angle, the X and dY rows; then, behind the first
+    // barrier, the B and C pairs of the rotation while the angle offsets are formed.
     constexpr int SEGS = 256 / NH, TPS = kQ / SEGS;
     const int jj = tid % NH, sg = tid / NH;
     float rho[TPS];
     {
-        float r = 0.f;
+        float thv[TPS], dtv[TPS];
 #pragma unroll
         for (int i = 0; i < TPS; ++i) {
             const long long t = t0 + sg * TPS + i;
-            float th = 0.f, d = 0.f;
-            if (t < a.T) {
-                th = a.theta[(((size_t)b * a.T + t) * a.G + g) * NH + jj];
-                d = a.dt[((size_t)b * a.T + t) * a.H + h];
-            }
-            r += angle ? th : d * th;
-            rho[i] = r;
+            const bool in = t < a.T;
+            const size_t bt = (size_t)b * a.T + (in ? t : 0);
+            thv[i] = in ? a.theta[(bt * a.G + g) * NH + jj] : 0.f;
+            dtv[i] = in ? a.dt[bt * a.H + h] : 0.f;
         }
-        segt[sg * NH + jj] = r;
-    }
-    // X and dY tiles
-    {
+        constexpr int XT = 2 * kQ * 8 / 256;   // X / dY 16-byte pieces per thread
+        uint4 xv[XT];
         const uint16_t* xg = static_cast<const uint16_t*>(a.x);
         const uint16_t* yg = static_cast<const uint16_t*>(a.dy);
 #pragma unroll
-        for (int i = tid; i < 2 * kQ * 8; i += 256) {
+        for (int m = 0; m < XT; ++m) {
+            const int i = tid + 256 * m;
             const bool isY = i >= kQ * 8;
             const int e = isY ? i - kQ * 8 : i;
-            const int u = e >> 3, ch = e & 7;
-            const long long t = t0 + u;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < a.T)
-                v = *reinterpret_cast<const uint4*>((isY ? yg : xg) +
-                                                    (((size_t)b * a.T + t) * a.H + h) * kPc + ch * 8);
-            *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DY : C::OFF_X) + sw128_off(u, ch * 8)) = v;
+            const long long t = t0 + (e >> 3);
+            xv[m] = t < a.T ? *reinterpret_cast<const uint4*>((isY ? yg : xg) +
+                                                             (((size_t)b * a.T + t) * a.H + h) * kPc + (e & 7) * 8)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float r = 0.f;
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) {
+            r += angle ? thv[i] : dtv[i] * thv[i];
+            rho[i] = r;
+        }
+        segt[sg * NH + jj] = r;
+#pragma unroll
+        for (int m = 0; m < XT; ++m) {
+            const int i = tid + 256 * m;
+            const bool isY = i >= kQ * 8;
+            const int e = isY ? i - kQ * 8 : i;
+            *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DY : C::OFF_X) + sw128_off(e >> 3, (e & 7) * 8)) = xv[m];
         }
     }
     __syncthreads();
+    // B~, C~ in the call frame: thread (pair jr, tokens ur + RS m) for m < KT
+    constexpr int KT = kQ * NH / 256, RS = 256 / NH;
+    const int jr = tid % NH, ur = tid / NH;
+    uint32_t pbv[KT], pcv[KT];
     {
+        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
+        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
+#pragma unroll
+        for (int m = 0; m < KT; ++m) {
+            const long long t = t0 + ur + RS * m;
+            pbv[m] = pcv[m] = 0u;
+            if (t < a.T) {
+                const size_t row = (((size_t)b * a.T + t) * a.G + g) * NST + 2 * jr;
+                pbv[m] = *reinterpret_cast<const uint32_t*>(Bg + row);
+                pcv[m] = *reinterpret_cast<const uint32_t*>(Cg + row);
+            }
+        }
         float off = p.P0[(bh * (p.nch + 1) + c) * NH + jj];
         for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + jj];
 #pragma unroll
         for (int i = 0; i < TPS; ++i) psi0[psi_idx<NH>(sg * TPS + i, jj)] = wrap_angle(off + rho[i]);
     }
     __syncthreads();
-    // B~, C~ in the call frame: thread (pair j, token u) for tasks i = tid + 256 m
-    {
-        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
-        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
 #pragma unroll
-        for (int m = 0; m < kQ * NH / 256; ++m) {
-            const int i = tid + 256 * m;
-            const int j = i % NH, u = i / NH;
-            const long long t = t0 + u;
-            uint32_t pb = 0u, pcv = 0u;
-            if (t < a.T) {
-                const size_t row = (((size_t)b * a.T + t) * a.G + g) * NST + 2 * j;
-                pb = *reinterpret_cast<const uint32_t*>(Bg + row);
-                pcv = *reinterpret_cast<const uint32_t*>(Cg + row);
-            }
-            float sn, cs2;
-            __sincosf(psi0[psi_idx<NH>(u, j)], &sn, &cs2);
-            const float b0 = bf16lo(pb), b1 = bf16hi(pb), c0 = bf16lo(pcv), c1 = bf16hi(pcv);
-            const uint32_t off = tile_off(u, 2 * j, kQ);
-            *reinterpret_cast<uint32_t*>(sm + C::OFF_B + off) =
-                pack_bf16x2(fmaf(cs2, b0, sn * b1), fmaf(cs2, b1, -sn * b0));
-            *reinterpret_cast<uint32_t*>(sm + C::OFF_C + off) =
-                pack_bf16x2(fmaf(cs2, c0, sn * c1), fmaf(cs2, c1, -sn * c0));
-        }
+    for (int m = 0; m < KT; ++m) {
+        const int u = ur + RS * m;
+        float sn, cs2;
+        __sincosf(psi0[psi_idx<NH>(u, jr)], &sn, &cs2);
+        const float b0 = bf16lo(pbv[m]), b1 = bf16hi(pbv[m]), c0 = bf16lo(pcv[m]), c1 = bf16hi(pcv[m]);
+        const uint32_t off = tile_off(u, 2 * jr, kQ);
+        *reinterpret_cast<uint32_t*>(sm + C::OFF_B + off) =
+            pack_bf16x2(fmaf(cs2, b0, sn * b1), fmaf(cs2, b1, -sn * b0));
+        *reinterpret_cast<uint32_t*>(sm + C::OFF_C + off) =
+            pack_bf16x2(fmaf(cs2, c0, sn * c1), fmaf(cs2, c1, -sn * c0));
     }
     fence_proxy_async_smem();
     if (w == 0) {
@@ -1024,8 +1036,13 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
 
     // angles: suffix sums over the chunk's tokens per (pair, token segment), then the
     // segments' totals; dtheta gets dang (x dt), the dt gradient dang . theta
-    float loc[TPS];
+    float loc[TPS], thl[TPS];
     if (ok) {
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) {   // theta of the segment's tokens, requested up front
+            const int u = sg * TPS + i;
+            thl[i] = (u < nv && !angle) ? a.theta[(((size_t)b * a.T + t0 + u) * a.G + g) * NH + jj] : 0.f;
+        }
         float r = 0.f;
 #pragma unroll
         for (int i = TPS - 1; i >= 0; --i) {
@@ -1057,7 +1074,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
             if (u < nv) {
                 const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
                 atomicAdd(&a.dtheta[row * NH + jj], angle ? dang : dang * k.dd[u]);
-                if (!angle) contrib = dang * a.theta[row * NH + jj];
+                contrib = dang * thl[i];
             }
             psi1[psi_idx<NH>(u, jj)] = contrib;
         }
