@@ -212,7 +212,7 @@ struct VuCfg {
 };
 
 template <int NST>
-__global__ void __launch_bounds__(128) bwd_vu_kernel(const __grid_constant__ TcBwd p) {
+__global__ void __launch_bounds__(128, 4) bwd_vu_kernel(const __grid_constant__ TcBwd p) {
     using C = VuCfg<NST>;
     constexpr int NH = C::NH;
     const BwdArgs& a = p.a;
@@ -228,6 +228,32 @@ __global__ void __launch_bounds__(128) bwd_vu_kernel(const __grid_constant__ TcB
     const long long t0 = (long long)c * kQ;
     const size_t cc = bh * p.nch + c;
 
+    // Every global input of the chunk is requested before any of it is used: X and dY rows
+    // and the thread's angles first; the B and C pairs once the angle prefix is formed.
+    constexpr int SEGS = 128 / NH, TPS = kQ / SEGS, XT = 2 * kQ * 8 / 128;
+    const int j = tid % NH, sg = tid / NH;
+    const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
+    uint4 xv[XT];
+    float thv[TPS];
+    {
+        const uint16_t* xg = static_cast<const uint16_t*>(a.x);
+        const uint16_t* yg = static_cast<const uint16_t*>(a.dy);
+#pragma unroll
+        for (int m = 0; m < XT; ++m) {
+            const int i = tid + 128 * m;
+            const bool isY = i >= kQ * 8;
+            const int e = isY ? i - kQ * 8 : i;
+            const long long t = t0 + (e >> 3);
+            xv[m] = t < a.T ? *reinterpret_cast<const uint4*>((isY ? yg : xg) +
+                                                             (((size_t)b * a.T + t) * a.H + h) * kPc + (e & 7) * 8)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) {
+            const long long t = t0 + sg * TPS + i;
+            thv[i] = t < a.T ? a.theta[(((size_t)b * a.T + t) * a.G + g) * NH + j] : 0.f;
+        }
+    }
     if (tid == 0) {
         mbar_init(&bar[0], 1);
         misc[1] = 0u;
@@ -245,67 +271,58 @@ __global__ void __launch_bounds__(128) bwd_vu_kernel(const __grid_constant__ TcB
     const Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.status, p.limit_ns};
     if (tid == 0) p.ctot[cc] = k.cr[kQ - 1];
 
+    // diag(e w) X and diag(f) dY
+#pragma unroll
+    for (int m = 0; m < XT; ++m) {
+        const int i = tid + 128 * m;
+        const bool isY = i >= kQ * 8;
+        const int e = isY ? i - kQ * 8 : i;
+        const int u = e >> 3;
+        const float sc = isY ? k.ff[u] : k.ew[u];
+        const uint4 v = xv[m];
+        *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DYF : C::OFF_XW) + sw128_off(u, (e & 7) * 8)) =
+            make_uint4(scale2(v.x, sc), scale2(v.y, sc), scale2(v.z, sc), scale2(v.w, sc));
+    }
     // B~, C~ in the chunk's frame: thread (pair j, token segment sg) sums its segment's
     // angles, the segments' totals are exchanged, and the thread rotates its segment's tokens
     {
-        constexpr int SEGS = 128 / NH, TPS = kQ / SEGS;
-        const int j = tid % NH, sg = tid / NH;
         float* segt = reinterpret_cast<float*>(sm + C::OFF_SEG);
-        const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
         float rho[TPS];
         float r = 0.f;
 #pragma unroll
         for (int i = 0; i < TPS; ++i) {
-            const int u = sg * TPS + i;
-            const long long t = t0 + u;
-            const float th = t < a.T ? a.theta[(((size_t)b * a.T + t) * a.G + g) * NH + j] : 0.f;
-            r += angle ? th : k.dd[u] * th;
+            r += angle ? thv[i] : k.dd[sg * TPS + i] * thv[i];
             rho[i] = r;
         }
         segt[sg * NH + j] = r;
+        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
+        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
+        uint32_t pbv[TPS], pcv[TPS];
+#pragma unroll
+        for (int i = 0; i < TPS; ++i) {
+            const long long t = t0 + sg * TPS + i;
+            pbv[i] = pcv[i] = 0u;
+            if (t < a.T) {
+                const size_t row = (((size_t)b * a.T + t) * a.G + g) * NST + 2 * j;
+                pbv[i] = *reinterpret_cast<const uint32_t*>(Bg + row);
+                pcv[i] = *reinterpret_cast<const uint32_t*>(Cg + row);
+            }
+        }
         __syncthreads();
         float off = 0.f;
         for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + j];
         if (sg == SEGS - 1) p.atot[cc * NH + j] = off + r;
-        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
-        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
 #pragma unroll
         for (int i = 0; i < TPS; ++i) {
             const int u = sg * TPS + i;
-            const long long t = t0 + u;
-            uint32_t pb = 0u, pcv = 0u;
-            if (t < a.T) {
-                const size_t row = (((size_t)b * a.T + t) * a.G + g) * NST + 2 * j;
-                pb = *reinterpret_cast<const uint32_t*>(Bg + row);
-                pcv = *reinterpret_cast<const uint32_t*>(Cg + row);
-            }
             float sn, cs;
             __sincosf(wrap_angle(off + rho[i]), &sn, &cs);
-            const float b0 = bf16lo(pb), b1 = bf16hi(pb), c0 = bf16lo(pcv), c1 = bf16hi(pcv);
+            const float b0 = bf16lo(pbv[i]), b1 = bf16hi(pbv[i]), c0 = bf16lo(pcv[i]), c1 = bf16hi(pcv[i]);
             const uint32_t o = tile_off(u, 2 * j, kQ);
             *reinterpret_cast<uint32_t*>(sm + C::OFF_B + o) =
                 pack_bf16x2(fmaf(cs, b0, sn * b1), fmaf(cs, b1, -sn * b0));
             *reinterpret_cast<uint32_t*>(sm + C::OFF_C + o) =
                 pack_bf16x2(fmaf(cs, c0, sn * c1), fmaf(cs, c1, -sn * c0));
-        }
-    }
-    // diag(e w) X and diag(f) dY
-    {
-        const uint16_t* xg = static_cast<const uint16_t*>(a.x);
-        const uint16_t* yg = static_cast<const uint16_t*>(a.dy);
-#pragma unroll 4
-        for (int i = tid; i < 2 * kQ * 8; i += 128) {
-            const bool isY = i >= kQ * 8;
-            const int e = isY ? i - kQ * 8 : i;
-            const int u = e >> 3, ch = e & 7;
-            const long long t = t0 + u;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < a.T)
-                v = *reinterpret_cast<const uint4*>((isY ? yg : xg) +
-                                                    (((size_t)b * a.T + t) * a.H + h) * kPc + ch * 8);
-            const float s = isY ? k.ff[u] : k.ew[u];
-            const uint4 o = make_uint4(scale2(v.x, s), scale2(v.y, s), scale2(v.z, s), scale2(v.w, s));
-            *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DYF : C::OFF_XW) + sw128_off(u, ch * 8)) = o;
         }
     }
     fence_proxy_async_smem();
@@ -384,7 +401,7 @@ __global__ void __launch_bounds__(128) bwd_vu_kernel(const __grid_constant__ TcB
 // 2. chunk scan: thread (channel p, pair group pg) holds state rows 2j, 2j+1 of column p for
 // the pairs j = pg + NPG k, k < 8.
 template <int NST>
-__global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant__ TcBwd p) {
+__global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(const __grid_constant__ TcBwd p) {
     constexpr int NH = NST / 2, NPG = NST / 16, NT = 4 * NST, NW = NT / 32;
     const BwdArgs& a = p.a;
     __shared__ float red[2][NW];
@@ -402,35 +419,56 @@ __global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant
     const size_t o0 = (size_t)b * a.T * a.H + h;
     const float k0 = (1.f - a.lam[o0]) * a.dt[o0];
     const float xp = bf_at(a.x_prev, bh * kPc + pc);
-    float ge[8], go[8], bpe[8], bpo[8], P[8];
+    const size_t bprow = ((size_t)b * a.G + g) * NST;
+    float ge[8], go[8], P[8];
 #pragma unroll
     for (int kx = 0; kx < 8; ++kx) {
         const int j = pg + NPG * kx;
-        const size_t bp = ((size_t)b * a.G + g) * NST + 2 * j;
-        bpe[kx] = bf_at(a.B_prev, bp);
-        bpo[kx] = bf_at(a.B_prev, bp + 1);
-        ge[kx] = fmaf(k0 * bpe[kx], xp, a.h0[bh * NP + (size_t)(2 * j) * kPc + pc]);
-        go[kx] = fmaf(k0 * bpo[kx], xp, a.h0[bh * NP + (size_t)(2 * j + 1) * kPc + pc]);
+        ge[kx] = fmaf(k0 * bf_at(a.B_prev, bprow + 2 * j), xp, a.h0[bh * NP + (size_t)(2 * j) * kPc + pc]);
+        go[kx] = fmaf(k0 * bf_at(a.B_prev, bprow + 2 * j + 1), xp, a.h0[bh * NP + (size_t)(2 * j + 1) * kPc + pc]);
         P[kx] = 0.f;
     }
-    // forward: the state entering every chunk, then the chunk's contribution in the call frame
+    // forward: the state entering every chunk, then the chunk's contribution in the call
+    // frame; the next chunk's V, decay and angles are requested one step ahead
+    uint16_t vn[16];
+    float atn[8], ctn;
+    auto fetch_fwd = [&](int c) {
+        const size_t cc = bh * nch + c;
+        const uint16_t* V = p.V + cc * NP;
+#pragma unroll
+        for (int kx = 0; kx < 8; ++kx) {
+            const int j = pg + NPG * kx;
+            vn[2 * kx] = V[(size_t)(2 * j) * kPc + pc];
+            vn[2 * kx + 1] = V[(size_t)(2 * j + 1) * kPc + pc];
+            atn[kx] = p.atot[cc * NH + j];
+        }
+        ctn = p.ctot[cc];
+    };
+    fetch_fwd(0);
     for (int c = 0; c < nch; ++c) {
         const size_t cc = bh * nch + c;
+        uint16_t vc[16];
+        float atc[8];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) vc[i] = vn[i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) atc[i] = atn[i];
+        const float dec = ex2f(ctn * kLog2e);
+        if (c + 1 < nch) fetch_fwd(c + 1);
         uint8_t* gt = reinterpret_cast<uint8_t*>(p.gin) + cc * NP * 2;
-        const uint16_t* V = p.V + cc * NP;
-        const float dec = ex2f(p.ctot[cc] * kLog2e);
 #pragma unroll
         for (int kx = 0; kx < 8; ++kx) {
             const int j = pg + NPG * kx;
             if (pc == 0) p.P0[(bh * (nch + 1) + c) * NH + j] = P[kx];
             *reinterpret_cast<uint16_t*>(gt + sw128_off(2 * j, pc)) = to_bf(ge[kx]);
             *reinterpret_cast<uint16_t*>(gt + sw128_off(2 * j + 1, pc)) = to_bf(go[kx]);
-            const float v0 = bf_at(V, (size_t)(2 * j) * kPc + pc), v1 = bf_at(V, (size_t)(2 * j + 1) * kPc + pc);
+            const float v0 = __uint_as_float((uint32_t)vc[2 * kx] << 16);
+            const float v1 = __uint_as_float((uint32_t)vc[2 * kx + 1] << 16);
             float sn, cs;
             __sincosf(P[kx], &sn, &cs);
             ge[kx] = fmaf(dec, ge[kx], fmaf(cs, v0, sn * v1));
             go[kx] = fmaf(dec, go[kx], fmaf(cs, v1, -sn * v0));
-            P[kx] = wrap_angle(P[kx] + p.atot[cc * NH + j]);
+            P[kx] = wrap_angle(P[kx] + atc[kx]);
         }
     }
     // the final state and dL/dh_T: dg = R(-psi_T) dH; the last token's angle gradient
@@ -456,25 +494,53 @@ __global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant
     }
     __syncthreads();   // the chunk-start angles (global) and exs are complete
     if (tid < NH) p.extra[bh * NH + tid] = exs[tid];
-    // reverse: the adjoint of the state leaving every chunk
+    // reverse: the adjoint of the state leaving every chunk; the next (earlier) chunk's U,
+    // stored entering state, angle and decay are requested one step ahead
+    uint16_t un[16], gn[16];
+    float pn[8], cn;
+    auto fetch_rev = [&](int c) {
+        const size_t cc = bh * nch + c;
+        const uint16_t* Uc = p.U + cc * NP;
+        const uint8_t* gt = reinterpret_cast<const uint8_t*>(p.gin) + cc * NP * 2;
+#pragma unroll
+        for (int kx = 0; kx < 8; ++kx) {
+            const int j = pg + NPG * kx;
+            un[2 * kx] = Uc[(size_t)(2 * j) * kPc + pc];
+            un[2 * kx + 1] = Uc[(size_t)(2 * j + 1) * kPc + pc];
+            gn[2 * kx] = *reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j, pc));
+            gn[2 * kx + 1] = *reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j + 1, pc));
+            pn[kx] = p.P0[(bh * (nch + 1) + c) * NH + j];
+        }
+        cn = p.ctot[cc];
+    };
+    fetch_rev(nch - 1);
     for (int c = nch - 1; c >= 0; --c) {
         const size_t cc = bh * nch + c;
+        uint16_t uc[16], gc[16];
+        float pcv[8];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            uc[i] = un[i];
+            gc[i] = gn[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pcv[i] = pn[i];
+        const float dec = ex2f(cn * kLog2e);
+        if (c > 0) fetch_rev(c - 1);
         uint8_t* dt_ = reinterpret_cast<uint8_t*>(p.dgo) + cc * NP * 2;
-        const uint8_t* gt = reinterpret_cast<const uint8_t*>(p.gin) + cc * NP * 2;
-        const uint16_t* Uc = p.U + cc * NP;
-        const float dec = ex2f(p.ctot[cc] * kLog2e);
         float s = 0.f;
 #pragma unroll
         for (int kx = 0; kx < 8; ++kx) {
             const int j = pg + NPG * kx;
             *reinterpret_cast<uint16_t*>(dt_ + sw128_off(2 * j, pc)) = to_bf(de[kx]);
             *reinterpret_cast<uint16_t*>(dt_ + sw128_off(2 * j + 1, pc)) = to_bf(dq[kx]);
-            const float g0 = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j, pc)) << 16);
-            const float g1 = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j + 1, pc)) << 16);
+            const float g0 = __uint_as_float((uint32_t)gc[2 * kx] << 16);
+            const float g1 = __uint_as_float((uint32_t)gc[2 * kx + 1] << 16);
             s = fmaf(de[kx], g0, fmaf(dq[kx], g1, s));
-            const float u0 = bf_at(Uc, (size_t)(2 * j) * kPc + pc), u1 = bf_at(Uc, (size_t)(2 * j + 1) * kPc + pc);
+            const float u0 = __uint_as_float((uint32_t)uc[2 * kx] << 16);
+            const float u1 = __uint_as_float((uint32_t)uc[2 * kx + 1] << 16);
             float sn, cs;
-            __sincosf(p.P0[(bh * (nch + 1) + c) * NH + j], &sn, &cs);
+            __sincosf(pcv[kx], &sn, &cs);
             de[kx] = fmaf(dec, de[kx], fmaf(cs, u0, sn * u1));
             dq[kx] = fmaf(dec, dq[kx], fmaf(cs, u1, -sn * u0));
         }
@@ -495,10 +561,10 @@ __global__ void __launch_bounds__(4 * NST) bwd_scan_kernel(const __grid_constant
         const int j = pg + NPG * kx;
         a.dh0[bh * NP + (size_t)(2 * j) * kPc + pc] = de[kx];
         a.dh0[bh * NP + (size_t)(2 * j + 1) * kPc + pc] = dq[kx];
-        pp = fmaf(de[kx], bpe[kx], fmaf(dq[kx], bpo[kx], pp));
+        pp = fmaf(de[kx], bf_at(a.B_prev, bprow + 2 * j), fmaf(dq[kx], bf_at(a.B_prev, bprow + 2 * j + 1), pp));
         const float se = warp_sum(de[kx] * xp), so = warp_sum(dq[kx] * xp);
         if (lane == 0) {
-            float* db = a.dB_prev + ((size_t)b * a.G + g) * NST + 2 * j;
+            float* db = a.dB_prev + bprow + 2 * j;
             atomicAdd(db, k0 * se);
             atomicAdd(db + 1, k0 * so);
         }
