@@ -572,6 +572,7 @@ extern "C" {
 
 m3_status m3_scan_bwd_workspace_bytes_ex(const m3_dims* d, int32_t seqlen, const m3_extras* ex,
                                          size_t* bytes) {
+    if (ex && !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;   // negative or NaN epsilon
     if (!ex_any(ex)) return m3_scan_bwd_workspace_bytes(d, seqlen, bytes);
     m3_status st = check_dims(d);
     if (st != M3_OK) return st;
@@ -587,6 +588,7 @@ m3_status m3_scan_bwd_ex(const m3_dims* d, int32_t seqlen, const void* x, const 
                          const m3_extras* ex, const void* dy, const float* dhT,
                          const m3_grads* gr, const m3_extra_grads* xg, void* workspace,
                          size_t workspace_bytes, uint32_t flags, void* stream) {
+    if (ex && !(ex->bc_norm_eps >= 0.f)) return M3_ERR_SHAPE;   // negative or NaN epsilon
     if (!ex_any(ex))
         return m3_scan_bwd(d, seqlen, x, B, C, dt, A, lam, theta, D, state0, dy, dhT, gr,
                            workspace, workspace_bytes, flags, stream);

@@ -224,6 +224,54 @@ def test_backward_validation_before_launch(lib):
                ws_bytes=1 << 30) == m3.M3_ERR_UNSUPPORTED      # headdim 128: no kernel
 
 
+def test_backward_ex_validation_before_launch(lib):
+    """m3_scan_bwd_ex checks the extras and their gradient pointers (needed exactly when the
+    part is on), alignment, epsilon and the workspace before anything is launched; an
+    all-zero extras block is the plain backward."""
+    d = m3.Dims(1, 2, 1, 16, 16, 2, m3.M3_F32)
+    st = m3.m3_state(0x2000, 0x3000, 0x4000)
+    p, ws = 0x1000, 0x100000
+    full = m3.m3_grads(*([p] * 11))
+
+    def ex_of(**kw):
+        e = m3.m3_extras()
+        for k, v in kw.items():
+            setattr(e, k, v)
+        return e
+
+    gate = ex_of(z=p, z_expand=p, x_expand=p, B_bias=p, bc_norm_eps=1e-5)
+    all_xg = m3.m3_extra_grads(p, p, None, p, p)
+    n = ctypes.c_size_t()
+    assert lib.m3_scan_bwd_workspace_bytes_ex(ctypes.byref(d.c()), 64, ctypes.byref(gate),
+                                              ctypes.byref(n)) == m3.M3_OK
+    need = n.value
+    assert need > m3.m3_scan_bwd_workspace_bytes(d, 64)       # effective inputs, y_pre, ...
+    bad = ex_of(bc_norm_eps=-1.0)
+    assert lib.m3_scan_bwd_workspace_bytes_ex(ctypes.byref(d.c()), 64, ctypes.byref(bad),
+                                              ctypes.byref(n)) == m3.M3_ERR_SHAPE
+
+    def bwd(ex=gate, xg=all_xg, ws_bytes=need, T=64, dims=d):
+        return lib.m3_scan_bwd_ex(ctypes.byref(dims.c()), T, p, p, p, p, p, p, p, None,
+                                  ctypes.byref(st), ctypes.byref(ex) if ex is not None else None,
+                                  p, None, ctypes.byref(full),
+                                  ctypes.byref(xg) if xg is not None else None, ws, ws_bytes, 0,
+                                  None)
+
+    assert bwd(T=0) == m3.M3_OK
+    assert bwd(T=-1) == m3.M3_ERR_SHAPE
+    assert bwd(xg=None) == m3.M3_ERR_NULL
+    assert bwd(xg=m3.m3_extra_grads(None, p, None, p, p)) == m3.M3_ERR_NULL        # dz
+    assert bwd(xg=m3.m3_extra_grads(p, None, None, p, p)) == m3.M3_ERR_NULL        # dB_bias
+    assert bwd(xg=m3.m3_extra_grads(p, p, None, None, p)) == m3.M3_ERR_NULL        # dx_expand
+    assert bwd(xg=m3.m3_extra_grads(p, p, None, p, None)) == m3.M3_ERR_NULL        # dz_expand
+    assert bwd(ex=ex_of(z_expand=p), xg=m3.m3_extra_grads(p, None, None, None, p)) == m3.M3_ERR_NULL
+    assert bwd(ex=ex_of(C_bias=p, bc_norm_eps=float("nan"))) == m3.M3_ERR_SHAPE
+    assert bwd(ex=ex_of(z=p + 2), xg=m3.m3_extra_grads(p, None, None, None, None)) == m3.M3_ERR_ALIGN
+    assert bwd(ex=ex_of(x_expand=p + 4), xg=m3.m3_extra_grads(None, None, None, p, None)) == m3.M3_ERR_ALIGN
+    assert bwd(ws_bytes=need - 256) == m3.M3_ERR_WORKSPACE
+    assert bwd(dims=m3.Dims(1, 2, 1, 128, 16, 2, m3.M3_F32), ws_bytes=1 << 34) == m3.M3_ERR_UNSUPPORTED
+
+
 def test_status_strings_cover_range_code(lib):
     assert "range" in m3.m3_status_string(m3.M3_ERR_RANGE)
 
