@@ -58,6 +58,8 @@ struct TcBwd {
     float* dtot;              // [BH][nch][N/2] sum of the chunk's angle gradients
     float* spill;             // [BH][nch] band-weight gradient owed to the next token
     float* extra;             // [BH][N/2] angle gradient of the last token from dL/dh_T
+    float* pang;              // [BH][T][N/2] chunk-local suffix sums of the angle gradients
+    float* carry;             // [BH][nch][N/2] angle gradient carried in from later chunks
     float* v0;                // [BH] <dg_0, B_prev x_prev^T>
     uint32_t* status;
     unsigned long long limit_ns;
@@ -682,7 +684,6 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     float* qz = acc + 5 * kQ;     // <C~_t, (dY g^T)_t>
     float* dcm = acc + 6 * kQ;    // log-decay gradient, then its suffix sums
     float* dnx = acc + 7 * kQ;    // band-weight gradient owed to the next token
-    float* dpt = acc + 8 * kQ;    // dt gradient through the angles, per token
     float* misc2 = acc + 9 * kQ;  // [0] dD partial, [1..2] warp sums, [3] suffix carry
     float* psi0 = reinterpret_cast<float*>(sm + C::OFF_MS);    // angle table, first home
     float* psi1 = reinterpret_cast<float*>(sm + C::OFF_GIN);   // and second
@@ -1101,14 +1102,10 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     ok = ok && flag_ok();
 
     // angles: suffix sums over the chunk's tokens per (pair, token segment), then the
-    // segments' totals; dtheta gets dang (x dt), the dt gradient dang . theta
-    float loc[TPS], thl[TPS];
+    // segments' totals; each head's chunk-local sums go to the workspace, where the finish
+    // step adds the carry from later chunks and sums over the group's heads
+    float loc[TPS];
     if (ok) {
-#pragma unroll
-        for (int i = 0; i < TPS; ++i) {   // theta of the segment's tokens, requested up front
-            const int u = sg * TPS + i;
-            thl[i] = (u < nv && !angle) ? a.theta[(((size_t)b * a.T + t0 + u) * a.G + g) * NH + jj] : 0.f;
-        }
         float r = 0.f;
 #pragma unroll
         for (int i = TPS - 1; i >= 0; --i) {
@@ -1132,30 +1129,13 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     if (ok) {
         float off = 0.f;
         for (int s2 = sg + 1; s2 < SEGS; ++s2) off += segt[s2 * NH + jj];
+        float* pg = p.pang + (bh * a.T + t0) * NH + jj;
 #pragma unroll
         for (int i = 0; i < TPS; ++i) {
             const int u = sg * TPS + i;
-            const float dang = loc[i] + off;
-            float contrib = 0.f;
-            if (u < nv) {
-                const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
-                atomicAdd(&a.dtheta[row * NH + jj], angle ? dang : dang * k.dd[u]);
-                contrib = dang * thl[i];
-            }
-            psi1[psi_idx<NH>(u, jj)] = contrib;
+            if (u < nv) pg[(size_t)u * NH] = loc[i] + off;
         }
         if (sg == 0) p.dtot[cc * NH + jj] = loc[0] + off;
-    }
-    __syncthreads();
-    if (ok) {
-        // the dt gradient through the angles: four threads per token
-        const int u = tid >> 2, qq = tid & 3;
-        float sacc = 0.f;
-#pragma unroll
-        for (int i = 0; i < NH / 4; ++i) sacc += psi1[psi_idx<NH>(u, qq * (NH / 4) + i)];
-        sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
-        sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
-        if (qq == 0) dpt[u] = sacc;
     }
     if (ok && tid < kQ) {
         const int u = tid;
@@ -1177,7 +1157,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
         const int u = tid;
         const float dda = dcm[u] + (w == 0 ? misc2[3] : 0.f);
         const float dga = k.ee[u] * dv[u] + ga[u];
-        float ddt = fmaf(dda, k.aa[u], fmaf(dga, k.ll[u], dpt[u]));
+        float ddt = fmaf(dda, k.aa[u], dga * k.ll[u]);
         float dlam = dga * k.dd[u];
         if (u > 0) {
             ddt = fmaf(dnx[u - 1], 1.f - k.ll[u], ddt);
@@ -1200,60 +1180,82 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
 }
 
 // ------------------------------------------------------------------------------------
-// 4. finish: the angle gradient carried in from later chunks (and from dL/dh_T) and the
-// next-token share of the previous chunk's last trapezoid weight
-__global__ void __launch_bounds__(64) bwd_finish_kernel(const __grid_constant__ TcBwd p) {
+// 4. finish.  The carry of every chunk: carry[c] = extra + sum over later chunks of their
+// angle-gradient totals (a suffix sum over chunks, one thread per (batch, head, pair)).
+__global__ void bwd_carry_kernel(const __grid_constant__ TcBwd p, int NH) {
+    const long long n = (long long)p.a.batch * p.a.H * NH;
+    const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (e >= n) return;
+    const long long bh = e / NH;
+    const int j = (int)(e % NH);
+    float run = p.extra[e];
+    for (int c = p.nch - 1; c >= 0; --c) {
+        const size_t o = ((size_t)bh * p.nch + c) * NH + j;
+        p.carry[o] = run;
+        run += p.dtot[o];
+    }
+}
+
+// Per (batch, chunk, group): dtheta of every token = sum over the group's heads of the full
+// angle gradient (chunk-local sums plus carry) times dt (1 with the angle flag), in a fixed
+// order; dt of every (token, head) gets the full angle gradient . theta, and the chunk's
+// first token the previous chunk's last-token share of the trapezoid weight.  Thread
+// (token u, pair quarter jq) holds NH / 4 pairs.
+template <int NH>
+__global__ void __launch_bounds__(256) bwd_finish_kernel(const __grid_constant__ TcBwd p) {
+    constexpr int JP = NH / 4;
     const BwdArgs& a = p.a;
-    const int NH = a.N / 2;
-    __shared__ float car[64], dts[64];
-    __shared__ float ths[kQ][65];
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, u = tid >> 2, jq = tid & 3;
     const int c = (int)(blockIdx.x % p.nch);
-    const size_t bh = blockIdx.x / p.nch;
-    const int b = (int)(bh / a.H), h = (int)(bh % a.H), g = h / (a.H / a.G);
-    const long long t0 = (long long)c * kQ;
-    const int nv = (int)(a.T - t0 < kQ ? a.T - t0 : kQ);
+    const long long bg = blockIdx.x / p.nch;
+    const int g = (int)(bg % a.G), b = (int)(bg / a.G);
+    const int hpg = a.H / a.G;
+    const long long t0 = (long long)c * kQ, t = t0 + u;
+    const bool live = t < a.T;
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
-    if (tid < nv) dts[tid] = a.dt[((size_t)b * a.T + t0 + tid) * a.H + h];
-    if (tid < NH) {
-        float s = p.extra[bh * NH + tid];
+    const size_t trow = ((size_t)b * a.T + (live ? t : 0)) * a.G + g;
+    float th[JP], acc[JP];
+#pragma unroll
+    for (int i = 0; i < JP; ++i) {
+        th[i] = (live && !angle) ? a.theta[trow * NH + jq * JP + i] : 0.f;
+        acc[i] = 0.f;
+    }
 #pragma unroll 4
-        for (int c2 = c + 1; c2 < p.nch; ++c2) s += p.dtot[(bh * p.nch + c2) * NH + tid];
-        car[tid] = s;
-    }
-    if (!angle) {
-#pragma unroll 4
-        for (int i = tid; i < nv * NH; i += 64) {
-            const int u = i / NH, j = i - u * NH;
-            ths[u][j] = a.theta[(((size_t)b * a.T + t0 + u) * a.G + g) * NH + j];
+    for (int hh = 0; hh < hpg; ++hh) {
+        const int h = g * hpg + hh;
+        const size_t bh = (size_t)b * a.H + h;
+        const float* pg = p.pang + (bh * a.T + (live ? t : 0)) * NH + jq * JP;
+        const float* cg = p.carry + (bh * p.nch + c) * NH + jq * JP;
+        const size_t o = ((size_t)b * a.T + (live ? t : 0)) * a.H + h;
+        const float d = live ? __ldg(a.dt + o) : 0.f;
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < JP; ++i) {
+            const float dang = live ? __ldg(pg + i) + __ldg(cg + i) : 0.f;
+            acc[i] = fmaf(dang, angle ? 1.f : d, acc[i]);
+            s = fmaf(dang, th[i], s);
+        }
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        if (jq == 0 && live) {
+            float add = s, dl = 0.f;
+            if (u == 0 && c > 0) {
+                const float sp = p.spill[bh * p.nch + c - 1];
+                add = fmaf(sp, 1.f - a.lam[o], add);
+                dl = -sp * d;
+            }
+            a.ddt[o] += add;
+            if (dl != 0.f) a.dlam[o] += dl;
         }
     }
-    __syncthreads();
-    if (tid < NH) {
-        const float s = car[tid];
-        for (int u = 0; u < nv; ++u) {
-            const size_t row = ((size_t)b * a.T + t0 + u) * a.G + g;
-            atomicAdd(&a.dtheta[row * NH + tid], angle ? s : s * dts[u]);
-        }
-    }
-    if (tid < nv) {
-        const size_t o = ((size_t)b * a.T + t0 + tid) * a.H + h;
-        float add = 0.f;
-        if (!angle)
-            for (int j = 0; j < NH; ++j) add = fmaf(car[j], ths[tid][j], add);
-        float dl = 0.f;
-        if (tid == 0 && c > 0) {
-            const float s = p.spill[bh * p.nch + c - 1];
-            add = fmaf(s, 1.f - a.lam[o], add);
-            dl = -s * dts[0];
-        }
-        a.ddt[o] += add;
-        if (dl != 0.f) a.dlam[o] += dl;
+    if (live) {
+#pragma unroll
+        for (int i = 0; i < JP; ++i) a.dtheta[trow * NH + jq * JP + i] = acc[i];
     }
 }
 
 struct Layout {
-    size_t V, U, gin, dgo, ctot, atot, P0, q, dtot, spill, extra, v0, bytes;
+    size_t V, U, gin, dgo, ctot, atot, P0, q, dtot, spill, extra, v0, pang, carry, bytes;
 };
 
 Layout layout(int batch, int H, int N, long long T) {
@@ -1278,6 +1280,8 @@ Layout layout(int batch, int H, int N, long long T) {
     L.spill = take(BH * nch * 4);
     L.extra = take(BH * NH * 4);
     L.v0 = take(BH * 4);
+    L.pang = take(BH * (size_t)T * NH * 4);
+    L.carry = take(BH * nch * NH * 4);
     L.bytes = o;
     return L;
 }
@@ -1292,7 +1296,9 @@ cudaError_t launch_n(const TcBwd& p, long long units, cudaStream_t s) {
     bwd_vu_kernel<NST><<<(unsigned)units, 128, smv, s>>>(p);
     bwd_scan_kernel<NST><<<(unsigned)((size_t)p.a.batch * p.a.H), 4 * NST, 0, s>>>(p);
     bwd_grads_kernel<NST><<<(unsigned)units, 256, smg, s>>>(p);
-    bwd_finish_kernel<<<(unsigned)units, 64, 0, s>>>(p);
+    const long long bhj = (long long)p.a.batch * p.a.H * (NST / 2);
+    bwd_carry_kernel<<<(unsigned)((bhj + 255) / 256), 256, 0, s>>>(p, NST / 2);
+    bwd_finish_kernel<NST / 2><<<(unsigned)((long long)p.a.batch * p.a.G * p.nch), 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -1325,6 +1331,8 @@ cudaError_t launch_scan_bwd_tc(const BwdArgs& a, void* ws, uint32_t* status, uns
     p.spill = reinterpret_cast<float*>(base + L.spill);
     p.extra = reinterpret_cast<float*>(base + L.extra);
     p.v0 = reinterpret_cast<float*>(base + L.v0);
+    p.pang = reinterpret_cast<float*>(base + L.pang);
+    p.carry = reinterpret_cast<float*>(base + L.carry);
     p.status = status;
     p.limit_ns = limit_ns;
     const long long units = (long long)a.batch * a.H * p.nch;
