@@ -1199,19 +1199,23 @@ __global__ void bwd_carry_kernel(const __grid_constant__ TcBwd p, int NH) {
 // Per (batch, chunk, group): dtheta of every token = sum over the group's heads of the full
 // angle gradient (chunk-local sums plus carry) times dt (1 with the angle flag), in a fixed
 // order; dt of every (token, head) gets the full angle gradient . theta, and the chunk's
-// first token the previous chunk's last-token share of the trapezoid weight.  Thread
-// (token u, pair quarter jq) holds NH / 4 pairs.
+// first token the previous chunk's last-token share of the trapezoid weight.  Heads go in
+// tiles of 64: thread (token u, pair quarter jq) accumulates dtheta over the tile's heads
+// (read-only loads only) and leaves each head's theta product in shared memory; then every
+// (token, head) of the tile updates its dt and lam.
 template <int NH>
-__global__ void __launch_bounds__(256) bwd_finish_kernel(const __grid_constant__ TcBwd p) {
-    constexpr int JP = NH / 4;
+__global__ void __launch_bounds__(256, 2) bwd_finish_kernel(const __grid_constant__ TcBwd p) {
+    constexpr int JP = NH / 4, HT = 64;
     const BwdArgs& a = p.a;
+    __shared__ float sdt[kQ][HT + 1];
     const int tid = threadIdx.x, u = tid >> 2, jq = tid & 3;
     const int c = (int)(blockIdx.x % p.nch);
     const long long bg = blockIdx.x / p.nch;
     const int g = (int)(bg % a.G), b = (int)(bg / a.G);
     const int hpg = a.H / a.G;
     const long long t0 = (long long)c * kQ, t = t0 + u;
-    const bool live = t < a.T;
+    const int nv = (int)(a.T - t0 < kQ ? a.T - t0 : kQ);
+    const bool live = u < nv;
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     const size_t trow = ((size_t)b * a.T + (live ? t : 0)) * a.G + g;
     float th[JP], acc[JP];
@@ -1220,33 +1224,50 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const __grid_constant__
         th[i] = (live && !angle) ? a.theta[trow * NH + jq * JP + i] : 0.f;
         acc[i] = 0.f;
     }
+    for (int h0 = 0; h0 < hpg; h0 += HT) {
+        const int nh = hpg - h0 < HT ? hpg - h0 : HT;
 #pragma unroll 4
-    for (int hh = 0; hh < hpg; ++hh) {
-        const int h = g * hpg + hh;
-        const size_t bh = (size_t)b * a.H + h;
-        const float* pg = p.pang + (bh * a.T + (live ? t : 0)) * NH + jq * JP;
-        const float* cg = p.carry + (bh * p.nch + c) * NH + jq * JP;
-        const size_t o = ((size_t)b * a.T + (live ? t : 0)) * a.H + h;
-        const float d = live ? __ldg(a.dt + o) : 0.f;
-        float s = 0.f;
+        for (int hh = 0; hh < nh; ++hh) {
+            const int h = g * hpg + h0 + hh;
+            const size_t bh = (size_t)b * a.H + h;
+            const float* pg = p.pang + (bh * a.T + (live ? t : 0)) * NH + jq * JP;
+            const float* cg = p.carry + (bh * p.nch + c) * NH + jq * JP;
+            const float d = live ? __ldg(a.dt + ((size_t)b * a.T + (live ? t : 0)) * a.H + h) : 0.f;
+            float s = 0.f;
 #pragma unroll
-        for (int i = 0; i < JP; ++i) {
-            const float dang = live ? __ldg(pg + i) + __ldg(cg + i) : 0.f;
-            acc[i] = fmaf(dang, angle ? 1.f : d, acc[i]);
-            s = fmaf(dang, th[i], s);
-        }
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        if (jq == 0 && live) {
-            float add = s, dl = 0.f;
-            if (u == 0 && c > 0) {
-                const float sp = p.spill[bh * p.nch + c - 1];
-                add = fmaf(sp, 1.f - a.lam[o], add);
-                dl = -sp * d;
+            for (int i = 0; i < JP; ++i) {
+                const float dang = live ? __ldg(pg + i) + __ldg(cg + i) : 0.f;
+                acc[i] = fmaf(dang, angle ? 1.f : d, acc[i]);
+                s = fmaf(dang, th[i], s);
             }
-            a.ddt[o] += add;
-            if (dl != 0.f) a.dlam[o] += dl;
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            if (jq == 0) sdt[u][hh] = s;
         }
+        __syncthreads();
+        // dt and lam of the tile's (token, head) pairs: 16 per thread, loads before stores
+        constexpr int PER = kQ * HT / 256;
+        float cur[PER];
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int e = tid + 256 * m, uu = e / HT, hh = e % HT;
+            cur[m] = (uu < nv && hh < nh) ? a.ddt[((size_t)b * a.T + t0 + uu) * a.H + g * hpg + h0 + hh] : 0.f;
+        }
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int e = tid + 256 * m, uu = e / HT, hh = e % HT;
+            if (uu >= nv || hh >= nh) continue;
+            const int h = g * hpg + h0 + hh;
+            const size_t o = ((size_t)b * a.T + t0 + uu) * a.H + h;
+            float add = sdt[uu][hh];
+            if (uu == 0 && c > 0) {
+                const float sp = p.spill[((size_t)b * a.H + h) * p.nch + c - 1];
+                add = fmaf(sp, 1.f - a.lam[o], add);
+                a.dlam[o] -= sp * a.dt[o];
+            }
+            a.ddt[o] = cur[m] + add;
+        }
+        __syncthreads();
     }
     if (live) {
 #pragma unroll
