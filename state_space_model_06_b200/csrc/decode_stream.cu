@@ -91,11 +91,14 @@ __device__ __forceinline__ float4 expand4(float4 v, float4 w) {
 // XE: x (and z with z_expand) hold one value per head channel, [b][H][P], and rank column r
 // is that value times the head's weight w[r][p], rounded to the io dtype ("Multi-Input,
 // Multi-Output (MIMO) Formulation", MIMO Parameterization Choices).
-template <typename IO, int R, bool BCM, bool XE>
+// HV = 2 (half-heads) with the BC map: the lane also holds the squares of the same pair of
+// the other half of N, so that each warp forms the column RMS over all N on its own.
+template <typename IO, int R, bool BCM, bool XE, int HV = 1>
 struct Small {
     float dt, A, lam, th, D;
     float2 bq[R], bp[R], cc[R];   // this lane's pair (rows 2 lane, 2 lane + 1) of B, B_prev, C
     float2 biasB, biasC;          // the head's BC biases of this lane's pair (BC map)
+    float oq[R], op[R], oc[R];    // HV = 2, BC map: squares of the other half's pair
     float4 x[R], xp[R], z[R];     // this lane's column chunk of x, x_prev, z (rank columns)
     // pb: the first state pair of this warp's rows
     __device__ void load(const DecodeArgs& a, int bh, int lane, int pb) {
@@ -128,6 +131,14 @@ struct Small {
             bq[r] = load2(Bg + r * N);
             bp[r] = load2(Bpg + r * N);
             cc[r] = load2(Cg + r * N);
+            if constexpr (BCM && HV == 2) {
+                const int other = 2 * (kNP - 2 * pb);   // element offset of the partner pair
+                const float2 q2 = load2(Bg + r * N + other), p2 = load2(Bpg + r * N + other),
+                             c2 = load2(Cg + r * N + other);
+                oq[r] = q2.x * q2.x + q2.y * q2.y;
+                op[r] = p2.x * p2.x + p2.y * p2.y;
+                oc[r] = c2.x * c2.x + c2.y * c2.y;
+            }
             x[r] = xe ? expand4<IO>(x1, load4(wx + r * P))
                       : load4(static_cast<const IO*>(a.x) + xofs + r * P);
             xp[r] = load4(xp0 + r * P);
@@ -150,7 +161,7 @@ template <typename IO, int R, bool BCM, bool XE, int HV>
 __global__ void __launch_bounds__((HV == 1 ? kSW1 : kSW2) * 32, 1)
     decode_stream_kernel(DecodeArgs a, int nbh) {
     using C = SCfg<R, HV>;
-    static_assert(HV == 1 || (HV == 2 && !BCM), "the BC map's column sums need the whole head");
+    static_assert(HV == 1 || (HV == 2 && !XE), "half-heads run SISO without the expansion");
     constexpr int R2 = 2 * R;
     extern __shared__ __align__(128) uint8_t sm_raw[];
     uint8_t* smb = sm_raw + ((128u - (smem_u32(sm_raw) & 127u)) & 127u);
@@ -189,7 +200,7 @@ __global__ void __launch_bounds__((HV == 1 ? kSW1 : kSW2) * 32, 1)
     };
     if (lane == 0)
         for (int i = 0; i < kSlots && i < nmine; ++i) issue(i);
-    Small<IO, R, BCM, XE> nx;
+    Small<IO, R, BCM, XE, HV> nx;
     if (nmine > 0) nx.load(a, gw, lane, hf * kNP);
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     int issued = nmine < kSlots ? nmine : kSlots;   // copies issued
@@ -197,7 +208,7 @@ __global__ void __launch_bounds__((HV == 1 ? kSW1 : kSW2) * 32, 1)
 
     for (int i = 0; i < nmine && ok; ++i) {
         const int bh = gw + i * NW;
-        Small<IO, R, BCM, XE> cur = nx;
+        Small<IO, R, BCM, XE, HV> cur = nx;
         if constexpr (BCM) {
             // BC map ("Technical Approach", BCNorm and BC biases): each rank column of B,
             // B_prev and C scaled to unit RMS over N (when bc_eps > 0; the lanes hold the
@@ -207,9 +218,15 @@ __global__ void __launch_bounds__((HV == 1 ? kSW1 : kSW2) * 32, 1)
                 float sq = 1.f, sp = 1.f, sc = 1.f;
                 if (a.bc_eps > 0.f) {
                     const float invn = 1.f / (float)a.N;
-                    sq = rsqrtf(warp_sum(cur.bq[r].x * cur.bq[r].x + cur.bq[r].y * cur.bq[r].y) * invn + a.bc_eps);
-                    sp = rsqrtf(warp_sum(cur.bp[r].x * cur.bp[r].x + cur.bp[r].y * cur.bp[r].y) * invn + a.bc_eps);
-                    sc = rsqrtf(warp_sum(cur.cc[r].x * cur.cc[r].x + cur.cc[r].y * cur.cc[r].y) * invn + a.bc_eps);
+                    float eq = 0.f, ep = 0.f, ec = 0.f;
+                    if constexpr (HV == 2) {
+                        eq = cur.oq[r];
+                        ep = cur.op[r];
+                        ec = cur.oc[r];
+                    }
+                    sq = rsqrtf(warp_sum(cur.bq[r].x * cur.bq[r].x + cur.bq[r].y * cur.bq[r].y + eq) * invn + a.bc_eps);
+                    sp = rsqrtf(warp_sum(cur.bp[r].x * cur.bp[r].x + cur.bp[r].y * cur.bp[r].y + ep) * invn + a.bc_eps);
+                    sc = rsqrtf(warp_sum(cur.cc[r].x * cur.cc[r].x + cur.cc[r].y * cur.cc[r].y + ec) * invn + a.bc_eps);
                 }
                 cur.bq[r] = make_float2(fmaf(cur.bq[r].x, sq, cur.biasB.x), fmaf(cur.bq[r].y, sq, cur.biasB.y));
                 cur.bp[r] = make_float2(fmaf(cur.bp[r].x, sp, cur.biasB.x), fmaf(cur.bp[r].y, sp, cur.biasB.y));
@@ -440,22 +457,26 @@ cudaError_t launch_stream_io(const DecodeArgs& a, int batch, int R, cudaStream_t
 
 }  // namespace
 
-// MIMO N = 64 (rank 2, 4; every fused part), and SISO N = 128 as half-heads (plain or
-// with the output gate: the BC map's column sums would need the whole head)
+// MIMO N = 64 (rank 2, 4; every fused part), and SISO N = 128 as half-heads (plain, with
+// the output gate and with the BC map; each half-head warp forms the column RMS over all N)
 bool decode_stream_ok(const DecodeArgs& a, int R) {
     if (a.P != kPc) return false;
     if (a.N == 2 * kNP) return R == 2 || R == 4;
-    const bool bcm = a.B_bias || a.C_bias || a.bc_eps > 0.f;
-    return a.N == 4 * kNP && R == 1 && !bcm && !a.x_expand && !a.z_expand;
+    return a.N == 4 * kNP && R == 1 && !a.x_expand && !a.z_expand;
 }
 
 // The BC map and the lightweight expansion are compile-time variants, so the plain
 // instantiations hold none of their code.
 cudaError_t launch_decode_stream(const DecodeArgs& a, int batch, int R, int io_dtype,
                                  cudaStream_t s) {
-    if (a.N == 4 * kNP)
+    if (a.N == 4 * kNP) {
+        const bool bcm = a.B_bias || a.C_bias || a.bc_eps > 0.f;
+        if (bcm)
+            return io_dtype == M3_BF16 ? launch_stream_t<__nv_bfloat16, 1, true, false, 2>(a, batch, s)
+                                       : launch_stream_t<float, 1, true, false, 2>(a, batch, s);
         return io_dtype == M3_BF16 ? launch_stream_t<__nv_bfloat16, 1, false, false, 2>(a, batch, s)
                                    : launch_stream_t<float, 1, false, false, 2>(a, batch, s);
+    }
     return io_dtype == M3_BF16 ? launch_stream_io<__nv_bfloat16>(a, batch, R, s)
                                : launch_stream_io<float>(a, batch, R, s);
 }

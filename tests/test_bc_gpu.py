@@ -115,7 +115,10 @@ def test_bc_call_split(chunk):
 
 
 @pytest.mark.parametrize("shape,io,tol,parts", [
-    ((4, 8, 1, 64, 128, 1), torch.bfloat16, 2e-2, "norm+bias"),
+    ((4, 8, 1, 64, 128, 1), torch.bfloat16, 2e-2, "norm+bias"),    # SISO half-heads
+    ((2, 4, 1, 64, 128, 1), torch.bfloat16, 2e-2, "bias"),
+    ((2, 4, 1, 64, 128, 1), torch.bfloat16, 2e-2, "norm+gate"),
+    ((2, 4, 2, 64, 128, 1), torch.float32, 1e-5, "norm+bias+gate"),
     ((4, 8, 2, 64, 64, 4), torch.bfloat16, 2e-2, "norm+bias+gate"),
     ((2, 6, 3, 8, 6, 3), torch.float32, 1e-5, "norm+bias+gate"),
     ((2, 4, 1, 16, 16, 2), torch.float32, 1e-5, "bias"),
