@@ -197,24 +197,28 @@ __device__ void chunk_coefs(const BwdArgs& a, int b, int h, long long t0, const 
 // 1. chunk products
 template <int NST>
 struct VuCfg {
+    static constexpr int NT = 256;                           // threads
     static constexpr int NH = NST / 2;
     static constexpr int OFF_B = 0;                          // B~ [NST/64][Q][64] bf16
     static constexpr int OFF_C = kQ * NST * 2;               // C~
     static constexpr int OFF_XW = 2 * kQ * NST * 2;          // diag(e w) X [Q][64]
     static constexpr int OFF_DYF = OFF_XW + kQ * kPc * 2;    // diag(f) dY [Q][64]
     static constexpr int OFF_COEF = OFF_DYF + kQ * kPc * 2;
-    static constexpr int OFF_SEG = OFF_COEF + Coefs::kFloats * 4;   // [128 / NH][NH] angle sums
-    static constexpr int OFF_BAR = (OFF_SEG + 128 * 4 + 7) / 8 * 8;
+    static constexpr int OFF_SEG = OFF_COEF + Coefs::kFloats * 4;   // [NT / NH][NH] angle sums
+    static constexpr int OFF_BAR = (OFF_SEG + NT * 4 + 7) / 8 * 8;
     static constexpr int OFF_MISC = OFF_BAR + 8;
     static constexpr int USED = OFF_MISC + 16 + 1024;
     // at least 50 KB, so that at most four CTAs (4 x 128 TMEM columns) share an SM
     static constexpr int SMEM = USED > 51200 ? USED : 51200;
     static constexpr uint32_t ID = idesc_bf16(NST, kPc, true, true);
-    static_assert(SMEM * 5 > 233472 && SMEM * 4 <= 233472 - 4096, "four CTAs per SM");
+    static_assert(SMEM * 5 > 233472 && SMEM * 4 <= 233472 - 4096, "at most four CTAs per SM");
 };
 
+// 256 threads: thread (pair j, token segment sg) holds KQ = Q / (256 / NH) tokens of one
+// pair, so that every global input of the chunk (X and dY rows, the angles, the B and C
+// pairs) is requested in one round before the first barrier.
 template <int NST>
-__global__ void __launch_bounds__(128, 4) bwd_vu_kernel(const __grid_constant__ TcBwd p) {
+__global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ TcBwd p) {
     using C = VuCfg<NST>;
     constexpr int NH = C::NH;
     const BwdArgs& a = p.a;
@@ -230,19 +234,20 @@ __global__ void __launch_bounds__(128, 4) bwd_vu_kernel(const __grid_constant__ 
     const long long t0 = (long long)c * kQ;
     const size_t cc = bh * p.nch + c;
 
-    // Every global input of the chunk is requested before any of it is used: X and dY rows
-    // and the thread's angles first; the B and C pairs once the angle prefix is formed.
-    constexpr int SEGS = 128 / NH, TPS = kQ / SEGS, XT = 2 * kQ * 8 / 128;
+    constexpr int SEGS = C::NT / NH, TPS = kQ / SEGS, XT = 2 * kQ * 8 / C::NT;
     const int j = tid % NH, sg = tid / NH;
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     uint4 xv[XT];
     float thv[TPS];
+    uint32_t pbv[TPS], pcv[TPS];
     {
         const uint16_t* xg = static_cast<const uint16_t*>(a.x);
         const uint16_t* yg = static_cast<const uint16_t*>(a.dy);
+        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
+        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
 #pragma unroll
         for (int m = 0; m < XT; ++m) {
-            const int i = tid + 128 * m;
+            const int i = tid + C::NT * m;
             const bool isY = i >= kQ * 8;
             const int e = isY ? i - kQ * 8 : i;
             const long long t = t0 + (e >> 3);
@@ -253,7 +258,14 @@ __global__ void __launch_bounds__(128, 4) bwd_vu_kernel(const __grid_constant__ 
 #pragma unroll
         for (int i = 0; i < TPS; ++i) {
             const long long t = t0 + sg * TPS + i;
-            thv[i] = t < a.T ? a.theta[(((size_t)b * a.T + t) * a.G + g) * NH + j] : 0.f;
+            thv[i] = 0.f;
+            pbv[i] = pcv[i] = 0u;
+            if (t < a.T) {
+                const size_t row = ((size_t)b * a.T + t) * a.G + g;
+                thv[i] = a.theta[row * NH + j];
+                pbv[i] = *reinterpret_cast<const uint32_t*>(Bg + row * NST + 2 * j);
+                pcv[i] = *reinterpret_cast<const uint32_t*>(Cg + row * NST + 2 * j);
+            }
         }
     }
     if (tid == 0) {
@@ -276,7 +288,7 @@ __global__ void __launch_bounds__(128, 4) bwd_vu_kernel(const __grid_constant__ 
     // diag(e w) X and diag(f) dY
 #pragma unroll
     for (int m = 0; m < XT; ++m) {
-        const int i = tid + 128 * m;
+        const int i = tid + C::NT * m;
         const bool isY = i >= kQ * 8;
         const int e = isY ? i - kQ * 8 : i;
         const int u = e >> 3;
@@ -285,8 +297,8 @@ __global__ void __launch_bounds__(128, 4) bwd_vu_kernel(const __grid_constant__ 
         *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DYF : C::OFF_XW) + sw128_off(u, (e & 7) * 8)) =
             make_uint4(scale2(v.x, sc), scale2(v.y, sc), scale2(v.z, sc), scale2(v.w, sc));
     }
-    // B~, C~ in the chunk's frame: thread (pair j, token segment sg) sums its segment's
-    // angles, the segments' totals are exchanged, and the thread rotates its segment's tokens
+    // B~, C~ in the chunk's frame: the segment's angle sums, the segments' totals exchanged,
+    // then the rotation of the segment's tokens
     {
         float* segt = reinterpret_cast<float*>(sm + C::OFF_SEG);
         float rho[TPS];
@@ -297,19 +309,6 @@ __global__ void __launch_bounds__(128, 4) bwd_vu_kernel(const __grid_constant__ 
             rho[i] = r;
         }
         segt[sg * NH + j] = r;
-        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
-        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
-        uint32_t pbv[TPS], pcv[TPS];
-#pragma unroll
-        for (int i = 0; i < TPS; ++i) {
-            const long long t = t0 + sg * TPS + i;
-            pbv[i] = pcv[i] = 0u;
-            if (t < a.T) {
-                const size_t row = (((size_t)b * a.T + t) * a.G + g) * NST + 2 * j;
-                pbv[i] = *reinterpret_cast<const uint32_t*>(Bg + row);
-                pcv[i] = *reinterpret_cast<const uint32_t*>(Cg + row);
-            }
-        }
         __syncthreads();
         float off = 0.f;
         for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + j];
@@ -346,46 +345,42 @@ __global__ void __launch_bounds__(128, 4) bwd_vu_kernel(const __grid_constant__ 
     const bool ok = warp_wait_b(&bar[0], 0, ab);
     tc_fence_after();
     if (ok) {
-        const int q = w & 3;
+        // warps 0-3 read V (columns 0-63), warps 4-7 read U (columns 64-127)
+        const int q = w & 3, m = w >> 2;
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-        uint16_t* Vo = p.V + cc * (size_t)NST * kPc;
-        uint16_t* Uo = p.U + cc * (size_t)NST * kPc;
+        uint16_t* dst0 = (m ? p.U : p.V) + cc * (size_t)NST * kPc;
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            uint16_t* dst0 = m ? Uo : Vo;
+        for (int cb = 0; cb < 32; cb += 16) {
+            uint32_t r[16], r2[16];
+            int n, col, col2;
+            if constexpr (NST == 128) {   // M = 128: row = lane of the quadrant
+                tmem_ld_32x32b_x16(tq + 64 * m + 2 * cb, r);
+                tmem_ld_32x32b_x16(tq + 64 * m + 2 * cb + 16, r2);
+                n = 32 * q + lane;
+                col = 2 * cb;
+                col2 = 2 * cb + 16;
+            } else {                      // M = 64: 16 rows per quadrant, column halves
+                tmem_ld_16x32bx2_x16<32>(tq + 64 * m + cb, r);
+                n = 16 * q + (lane & 15);
+                col = cb + 32 * (lane >> 4);
+                col2 = -1;
+            }
+            tmem_wait_ld();
+            uint4* d = reinterpret_cast<uint4*>(dst0 + (size_t)n * kPc + col);
 #pragma unroll
-            for (int cb = 0; cb < 32; cb += 16) {
-                uint32_t r[16], r2[16];
-                int n, col, col2;
-                if constexpr (NST == 128) {   // M = 128: row = lane of the quadrant
-                    tmem_ld_32x32b_x16(tq + 64 * m + 2 * cb, r);
-                    tmem_ld_32x32b_x16(tq + 64 * m + 2 * cb + 16, r2);
-                    n = 32 * q + lane;
-                    col = 2 * cb;
-                    col2 = 2 * cb + 16;
-                } else {                      // M = 64: 16 rows per quadrant, column halves
-                    tmem_ld_16x32bx2_x16<32>(tq + 64 * m + cb, r);
-                    n = 16 * q + (lane & 15);
-                    col = cb + 32 * (lane >> 4);
-                    col2 = -1;
-                }
-                tmem_wait_ld();
-                uint4* d = reinterpret_cast<uint4*>(dst0 + (size_t)n * kPc + col);
+            for (int i = 0; i < 2; ++i)
+                d[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                                  pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                                  pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                                  pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+            if (col2 >= 0) {
+                uint4* d2 = reinterpret_cast<uint4*>(dst0 + (size_t)n * kPc + col2);
 #pragma unroll
                 for (int i = 0; i < 2; ++i)
-                    d[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
-                                      pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
-                                      pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
-                                      pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
-                if (col2 >= 0) {
-                    uint4* d2 = reinterpret_cast<uint4*>(dst0 + (size_t)n * kPc + col2);
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        d2[i] = make_uint4(pack_bf16x2(__uint_as_float(r2[8 * i]), __uint_as_float(r2[8 * i + 1])),
-                                           pack_bf16x2(__uint_as_float(r2[8 * i + 2]), __uint_as_float(r2[8 * i + 3])),
-                                           pack_bf16x2(__uint_as_float(r2[8 * i + 4]), __uint_as_float(r2[8 * i + 5])),
-                                           pack_bf16x2(__uint_as_float(r2[8 * i + 6]), __uint_as_float(r2[8 * i + 7])));
-                }
+                    d2[i] = make_uint4(pack_bf16x2(__uint_as_float(r2[8 * i]), __uint_as_float(r2[8 * i + 1])),
+                                       pack_bf16x2(__uint_as_float(r2[8 * i + 2]), __uint_as_float(r2[8 * i + 3])),
+                                       pack_bf16x2(__uint_as_float(r2[8 * i + 4]), __uint_as_float(r2[8 * i + 5])),
+                                       pack_bf16x2(__uint_as_float(r2[8 * i + 6]), __uint_as_float(r2[8 * i + 7])));
             }
         }
     }
@@ -1314,7 +1309,7 @@ cudaError_t launch_n(const TcBwd& p, long long units, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_grads_kernel<NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smg);
     if (e != cudaSuccess) return e;
-    bwd_vu_kernel<NST><<<(unsigned)units, 128, smv, s>>>(p);
+    bwd_vu_kernel<NST><<<(unsigned)units, VuCfg<NST>::NT, smv, s>>>(p);
     bwd_scan_kernel<NST><<<(unsigned)((size_t)p.a.batch * p.a.H), 4 * NST, 0, s>>>(p);
     bwd_grads_kernel<NST><<<(unsigned)units, 256, smg, s>>>(p);
     const long long bhj = (long long)p.a.batch * p.a.H * (NST / 2);
