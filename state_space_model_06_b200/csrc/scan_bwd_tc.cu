@@ -1230,10 +1230,19 @@ __global__ void __launch_bounds__(256, 2) bwd_finish_kernel(const __grid_constan
             const float d = live ? __ldg(a.dt + ((size_t)b * a.T + (live ? t : 0)) * a.H + h) : 0.f;
             float s = 0.f;
 #pragma unroll
-            for (int i = 0; i < JP; ++i) {
-                const float dang = live ? __ldg(pg + i) + __ldg(cg + i) : 0.f;
-                acc[i] = fmaf(dang, angle ? 1.f : d, acc[i]);
-                s = fmaf(dang, th[i], s);
+            for (int i4 = 0; i4 < JP / 4; ++i4) {
+                float4 pv = make_float4(0.f, 0.f, 0.f, 0.f), cv = pv;
+                if (live) {
+                    pv = __ldg(reinterpret_cast<const float4*>(pg) + i4);
+                    cv = __ldg(reinterpret_cast<const float4*>(cg) + i4);
+                }
+                const float dv[4] = {pv.x + cv.x, pv.y + cv.y, pv.z + cv.z, pv.w + cv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 4 * i4 + e;
+                    acc[i] = fmaf(dv[e], angle ? 1.f : d, acc[i]);
+                    s = fmaf(dv[e], th[i], s);
+                }
             }
             s += __shfl_xor_sync(0xffffffffu, s, 1);
             s += __shfl_xor_sync(0xffffffffu, s, 2);
