@@ -41,6 +41,11 @@
  *     M3_ERR_TIMEOUT into the workspace status word (see m3_query_status).
  *   - Value ranges are the caller's contract: dt > 0, A <= 0, lam in [0, 1].
  *     M3_FLAG_DEBUG_CHECKS adds a non-trapping device scan of them.
+ *   - Tensor memory: the tensor-core kernels (bf16 prefill, chunked backward) size their
+ *     tensor-memory columns so that the CTAs one kernel places on an SM fit in its 512
+ *     columns together (prefill 512 x 1, backward 128 x 4 and 256 x 2).  Calls ordered on one
+ *     stream never share an SM's tensor memory.  Running them concurrently on several
+ *     streams, or beside other kernels that allocate tensor memory, is not supported.
  */
 #ifndef M3_H
 #define M3_H
