@@ -84,6 +84,8 @@ CASES = [
     (1, 2, 1, 128, 130, m3.M3_FLAG_THETA_IS_ANGLE, True, 0.1),
     (1, 3, 1, 128, 1, 0, True, 1.0),            # one token
     (1, 2, 1, 64, 65, 0, True, 1.0),            # one token past a chunk
+    (1, 4, 1, 64, 1000, 0, True, 1.0),          # N 64, 16 chunks, ragged tail
+    (2, 8, 2, 128, 700, 0, True, math.pi / 4),  # two groups of four heads, 11 chunks
 ]
 
 
