@@ -90,18 +90,18 @@ def source_hash(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def committed_traffic(kernel_src, workload):
-    """DRAM traffic per launch from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+def committed_counters(kernel_src, workload):
+    """The committed ncu figures of the workload's kernel (DRAM traffic per launch, tensor-pipe
+    utilisation), if they were taken on the current kernel source (else an empty dict)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
-        return None
+        return {}
     with open(path) as f:
         d = json.load(f)
     ent = d.get(workload)
     if not ent or ent.get("source_sha256_16") != source_hash(kernel_src):
-        return None
-    return ent.get("dram_bytes_per_launch")
+        return {}
+    return ent
 
 
 class ClockSampler:
@@ -570,6 +570,35 @@ def oracle_workload(w, inp, rows):
     return rows * w.seqlen / secs, threads, secs
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def oracle_one_thread(w, inp):
+    """The CPU oracle on one (batch, head) slice of the workload (batch row 0, head 0, all
+    tokens) on a single thread: tokens per second of one sequential recurrence."""
+    import oracle
+    keys = ("x", "B", "C", "dt", "A", "lam", "theta")
+    arr = {k: inp[k][:1].double().numpy() for k in keys}
+    for k in ("x", "dt", "A", "lam"):
+        arr[k] = arr[k][:, :, :1].copy()
+    for k in ("B", "C", "theta"):
+        arr[k] = arr[k][:, :, :1].copy()   # head 0 reads group 0
+    D = inp["D"][:1].double().numpy()
+    t0 = time.perf_counter()
+    oracle.scan(*(arr[k] for k in keys), D=D, nthreads=1)
+    secs = time.perf_counter() - t0
+    return w.seqlen / secs, secs
+
+
 def oracle_sample(w, seqlen, seed=0):
     """Time the CPU oracle on batch row 0, all heads, the first `seqlen` tokens."""
     import oracle
@@ -606,8 +635,9 @@ def ours(args):
     achieved = byts / (ms / 1e3) / 1e9
     tflops = flops / (ms / 1e3) / 1e12
     kernel_src = os.path.join(ROOT, "state_space_model_06_b200", "csrc", "scan_tc.cu")
-    # the committed DRAM counters describe the full workload only
-    traffic = None if (args.batch or args.seqlen) else committed_traffic(kernel_src, WORKLOAD)
+    # the committed counters describe the current kernel on the full workload only
+    counters = {} if (args.batch or args.seqlen) else committed_counters(kernel_src, WORKLOAD)
+    traffic = counters.get("dram_bytes_per_launch")
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_world,
@@ -626,7 +656,9 @@ def ours(args):
                      "alg_bytes_per_launch": byts,
                      "tensor": {"achieved_tflops": tflops, "peak_tflops": pk["bf16_tflops"],
                                 "frac": tflops / pk["bf16_tflops"],
-                                "alg_flops_per_launch": flops}},
+                                "alg_flops_per_launch": flops,
+                                "pipe_active_ncu_pct": counters.get("tensor_pipe_active_pct"),
+                                "pipe_active_ncu_how": counters.get("tensor_pipe_how")}},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
@@ -710,10 +742,15 @@ def ours(args):
     if rank == 0 and ws_world == 1 and not args.no_cpu:
         rows = max(1, min(args.cpu_rows, w.batch))
         tps, cores, secs = oracle_workload(w, inp, rows)
+        one_tps, one_secs = oracle_one_thread(w, inp)
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": f"the workload's own inputs, batch rows 0..{rows - 1} of "
                                           f"{w.batch}, all {w.nheads} heads and {w.seqlen} tokens "
-                                          f"({secs:.1f} s of fp64 CPU work)"}
+                                          f"({secs:.1f} s of fp64 CPU work)",
+                                "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+                                "one_thread": {"value": one_tps, "unit": "tokens/s per (batch, head)",
+                                               "sample": f"batch row 0, head 0, {w.seqlen} tokens, "
+                                                         f"1 thread ({one_secs:.2f} s)"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_world > 1:
