@@ -50,12 +50,26 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # ----------------------------------------------------------------------------- helpers
 def peaks():
+    """The measured peaks (HBM GB/s, bf16 TFLOP/s) of MEASURED_PEAKS.json where present, else
+    the fallback figures; a key that is missing or not a number falls back on its own."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
+    if not os.path.exists(path):
+        return FALLBACK_PEAKS, "fallback"
+    try:
         with open(path) as f:
             d = json.load(f)
-        return d, "measured"
-    return FALLBACK_PEAKS, "fallback"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+    out, kind = dict(FALLBACK_PEAKS), "measured"
+    for k in FALLBACK_PEAKS:
+        v = d.get(k) if isinstance(d, dict) else None
+        if isinstance(v, dict):
+            v = v.get("value")
+        if isinstance(v, (int, float)) and v > 0:
+            out[k] = float(v)
+        else:
+            kind = "measured (fallback for missing keys)"
+    return out, kind
 
 
 def scan_algorithmic(w):
