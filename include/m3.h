@@ -96,10 +96,11 @@ typedef struct {
 /* Flags (bitwise OR). */
 #define M3_FLAG_THETA_IS_ANGLE 1u  /* theta already holds the per-step angle: the dt multiply is skipped */
 #define M3_FLAG_FORCE_SIMT 2u      /* m3_scan_fwd: run the sequential fp32 CUDA-core kernel */
-/* Test hook for the failure path: the tensor-core prefill's MMA warp waits on a barrier
- * that nothing completes, with a 50 ms limit instead of 2 s.  The bounded wait gives
- * up, the kernel aborts cleanly (outputs are invalid), and m3_query_status reports
- * M3_ERR_TIMEOUT; the CUDA context stays usable. */
+/* Test hook for the failure path: the tensor-core prefill's MMA warp (and, in m3_scan_bwd's
+ * chunked tensor-core path, the chunk-gradient kernel's issuing thread, before it issues
+ * anything) waits on a barrier that nothing completes, with a 50 ms limit instead of 2 s.
+ * The bounded wait gives up, the kernel aborts cleanly (outputs are invalid), and
+ * m3_query_status reports M3_ERR_TIMEOUT; the CUDA context stays usable. */
 #define M3_FLAG_TEST_STALL 4u
 /* Debug scan of the caller's value ranges (m3_scan_fwd and its variants, m3_scan_bwd): one
  * extra kernel reads every input of the call once before the call runs and checks

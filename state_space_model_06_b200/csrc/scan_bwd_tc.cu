@@ -799,7 +799,11 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     const uint32_t sb = smem_u32(sm);
     int issued = 0;   // thread 0: MMA rounds issued
     if (tid == 0) {
-        if (mbar_wait(&bar[0], 0, ab)) {
+        // test hook of the failure path: a wait that nothing completes (bar[3] only follows
+        // round 3) gives up after the call's limit, raising the abort flag and the status
+        const bool stall = (a.flags & M3_FLAG_TEST_STALL) != 0;
+        if (stall) (void)mbar_wait(&bar[3], 0, ab);
+        if (!stall && mbar_wait(&bar[0], 0, ab)) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < NST / 16; ++kk)
