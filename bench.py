@@ -409,7 +409,8 @@ def time_decode(name, dev, stream, seed, tokens=DECODE_TOKENS, gated=False, bc=F
 def mimo_leg(args, dev, stream, rank, ws_world, pk):
     """The MIMO prefill workload (rank 4, N 64, 32-token tiles): plain, with the
     lightweight expansion of x (x read as [b][T][H][P]), and with the expansion of x and z
-    plus the fused gate.  Algorithmic bytes count each tensor as the call reads it."""
+    plus the fused gate; then its backward pass (16-token chunks of 64 (token, rank) rows).
+    Algorithmic bytes count each tensor as the call reads it."""
     w = inputs.WORKLOADS["mimo_prefill_r4"]
     inp, d, g, st, y, ws = prefill_setup(w, dev, seed=200 + rank)
     del inp
@@ -432,6 +433,8 @@ def mimo_leg(args, dev, stream, rank, ws_world, pk):
         gbs = nbytes / (ms / 1e3) / 1e9
         out[key] = {"tokens_per_s": val, "ms_per_step": ms_max, "alg_bytes_per_step": nbytes,
                     "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"]}
+    if not args.no_bwd:
+        out["backward"] = backward_leg(args, w, d, g, dev, stream, rank, ws_world, pk)
     out["config"] = {"workload": w.name, "batch": b, "heads": H, "seqlen": T, "headdim": P,
                      "dstate": w.dstate, "rank": R, "chunk": w.chunk}
     return out

@@ -411,7 +411,7 @@ m3_status m3_scan_bwd_workspace_bytes(const m3_dims* d, int32_t seqlen, size_t* 
                                          seqlen).floats;
     size_t need = ((fl * sizeof(float) + 255) / 256) * 256;
     if (scan_bwd_tc_ok(d->io_dtype, d->dstate, d->headdim, d->rank)) {
-        const size_t tc = scan_bwd_tc_workspace_bytes(d->batch, d->nheads, d->dstate, seqlen);
+        const size_t tc = scan_bwd_tc_workspace_bytes(d->batch, d->nheads, d->dstate, d->rank, seqlen);
         if (tc > need) need = tc;
     }
     *bytes = kStatusBytes + need;
@@ -483,14 +483,14 @@ m3_status m3_scan_bwd(const m3_dims* d, int32_t seqlen, const void* x, const voi
                     aligned(gr->dx, 16) && aligned(gr->dB, 16) && aligned(gr->dC, 16);
     if (tc) {
         // the group-shared gradients and dD are accumulated with atomics
-        const size_t b = d->batch, T = seqlen, G = d->ngroups;
-        if (cudaMemsetAsync(gr->dB, 0, b * T * G * N * sizeof(float), s) != cudaSuccess ||
-            cudaMemsetAsync(gr->dC, 0, b * T * G * N * sizeof(float), s) != cudaSuccess ||
+        const size_t b = d->batch, T = seqlen, G = d->ngroups, Rs = R;
+        if (cudaMemsetAsync(gr->dB, 0, b * T * G * Rs * N * sizeof(float), s) != cudaSuccess ||
+            cudaMemsetAsync(gr->dC, 0, b * T * G * Rs * N * sizeof(float), s) != cudaSuccess ||
             cudaMemsetAsync(gr->dtheta, 0, b * T * G * (N / 2) * sizeof(float), s) != cudaSuccess ||
-            cudaMemsetAsync(gr->dB_prev, 0, b * G * N * sizeof(float), s) != cudaSuccess ||
+            cudaMemsetAsync(gr->dB_prev, 0, b * G * Rs * N * sizeof(float), s) != cudaSuccess ||
             (D && gr->dD && cudaMemsetAsync(gr->dD, 0, d->nheads * sizeof(float), s) != cudaSuccess))
             return M3_ERR_CUDA;
-        return launch_status(launch_scan_bwd_tc(a, static_cast<char*>(workspace) + kStatusBytes,
+        return launch_status(launch_scan_bwd_tc(a, R, static_cast<char*>(workspace) + kStatusBytes,
                                                 static_cast<uint32_t*>(workspace),
                                                 (flags & M3_FLAG_TEST_STALL) ? 50000000ull
                                                                              : 2000000000ull,

@@ -76,8 +76,8 @@ cudaError_t launch_scan_bwd(const BwdArgs& a, int R, int io_dtype, cudaStream_t 
 // covers, its workspace bytes (after the status block) and the launch (four kernels; dB, dC,
 // dtheta, dB_prev and dD are accumulated with atomics and must be zero on entry)
 bool scan_bwd_tc_ok(int io_dtype, int N, int P, int R);
-size_t scan_bwd_tc_workspace_bytes(int batch, int H, int N, long long T);
-cudaError_t launch_scan_bwd_tc(const BwdArgs& a, void* ws, uint32_t* status,
+size_t scan_bwd_tc_workspace_bytes(int batch, int H, int N, int R, long long T);
+cudaError_t launch_scan_bwd_tc(const BwdArgs& a, int R, void* ws, uint32_t* status,
                                unsigned long long limit_ns, cudaStream_t s);
 
 // sum of per-head partials over the heads of each group (fixed order):

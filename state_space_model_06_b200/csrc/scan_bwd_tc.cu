@@ -1,8 +1,14 @@
 // scan_bwd_tc.cu -- chunked backward pass of the Mamba-3 recurrence on the tensor cores
-// (SISO, bf16 x / B / C / dy, P = 64, N in {64, 128}).
+// (bf16 x / B / C / dy, P = 64; SISO with N in {64, 128}, MIMO ranks 2 and 4 with N = 64).
+//
+// Every tile has 64 rows; a row is one (token, rank), row = R u + r, so a chunk holds 64 / R
+// tokens (the C_MIMO = C_SISO / R rule of "Expressing MIMO as Multiple SISO SSMs", "The
+// Chunked Training Optimization").  Sums over a token's rows stand where the SISO formulas
+// below have one row; every per-token factor (decay, weights, angle, causal mask) is looked up
+// by row / R.
 //
 // Reverse-mode gradients of the chunked form ("Parallel representation under SSD", with the
-// rotation of Propositions 3 and 4).  Per chunk [t0, t1) of Q = 64 tokens, with cum the prefix
+// rotation of Propositions 3 and 4).  Per chunk [t0, t1) of Q = 64 / R tokens, with cum the prefix
 // of the log-decays dt A, psi the prefix of the angles, B~ = R(-psi) B, C~ = R(-psi) C,
 //     gamma_s = lam_s dt_s,   w_s = gamma_s + (1 - lam_{s+1}) dt_{s+1},
 //     L[t, s] = e^{cum_t - cum_s} (gamma_s + [s < t] (1 - lam_{s+1}) dt_{s+1})    (s <= t),
@@ -47,6 +53,7 @@ constexpr float kLog2e = 1.44269504088896340736f;
 struct TcBwd {
     BwdArgs a;
     int nch;                  // chunks of the call
+    int qt;                   // tokens per chunk: 64 / R (a tile row is one (token, rank))
     uint16_t* V;              // [BH][nch][N][P] bf16 chunk-frame state products
     uint16_t* U;              // [BH][nch][N][P] bf16 chunk-frame adjoint products
     uint16_t* gin;            // [BH][nch] bf16 tile images [N][P] of the entering state
@@ -141,18 +148,22 @@ struct Coefs {
     static constexpr int kFloats = 2 * (kQ + 1) + 7 * kQ;
 };
 
+// Per-token coefficients of a chunk of QT tokens (QT = 64 / R), one warp, two tokens a lane.
+// Slots u >= QT hold zeros, except that slot QT holds the next token's dt and lam.
+template <int QT>
 __device__ void chunk_coefs(const BwdArgs& a, int b, int h, long long t0, const Coefs& k) {
     const int lane = threadIdx.x & 31;
     const long long T = a.T;
     float d2[2], l2[2], a2[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const long long t = t0 + 2 * lane + i;
-        const bool ok = t < T;
+        const int u = 2 * lane + i;
+        const long long t = t0 + u;
+        const bool ok = u <= QT && t < T;
         const size_t o = ((size_t)b * T + (ok ? t : 0)) * a.H + h;
         d2[i] = ok ? a.dt[o] : 0.f;
         l2[i] = ok ? a.lam[o] : 0.f;
-        a2[i] = ok ? a.A[o] : 0.f;
+        a2[i] = ok && u < QT ? a.A[o] : 0.f;
     }
     const float e0 = d2[0] * a2[0], e1 = d2[1] * a2[1];
     float s = e0 + e1;
@@ -167,15 +178,16 @@ __device__ void chunk_coefs(const BwdArgs& a, int b, int h, long long t0, const 
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const int u = 2 * lane + i;
+        const bool in = u < QT;
         k.dd[u] = d2[i];
         k.ll[u] = l2[i];
         k.aa[u] = a2[i];
-        k.cr[u] = cc[i];
-        k.gam[u] = l2[i] * d2[i];
-        k.ee[u] = ex2f((cend - cc[i]) * kLog2e);
-        k.ff[u] = ex2f(cc[i] * kLog2e);
+        k.cr[u] = in ? cc[i] : 0.f;
+        k.gam[u] = in ? l2[i] * d2[i] : 0.f;
+        k.ee[u] = in ? ex2f((cend - cc[i]) * kLog2e) : 0.f;
+        k.ff[u] = in ? ex2f(cc[i] * kLog2e) : 0.f;
     }
-    if (lane == 0) {
+    if (QT == kQ && lane == 0) {
         const long long t = t0 + kQ;
         const bool ok = t < T;
         const size_t o = ((size_t)b * T + (ok ? t : 0)) * a.H + h;
@@ -186,7 +198,7 @@ __device__ void chunk_coefs(const BwdArgs& a, int b, int h, long long t0, const 
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const int u = 2 * lane + i;
-        const float nx = (1.f - k.ll[u + 1]) * k.dd[u + 1];
+        const float nx = u < QT ? (1.f - k.ll[u + 1]) * k.dd[u + 1] : 0.f;
         k.nx[u] = nx;
         k.ew[u] = k.ee[u] * (k.gam[u] + nx);
     }
@@ -214,13 +226,14 @@ struct VuCfg {
     static_assert(SMEM * 5 > 233472 && SMEM * 4 <= 233472 - 4096, "at most four CTAs per SM");
 };
 
-// 256 threads: thread (pair j, token segment sg) holds KQ = Q / (256 / NH) tokens of one
-// pair, so that every global input of the chunk (X and dY rows, the angles, the B and C
-// pairs) is requested in one round before the first barrier.
-template <int NST>
+// 256 threads: thread (pair j, row segment sg) holds TPS = 64 / (256 / NH) tile rows of one
+// pair (TPS / R tokens), so that every global input of the chunk (X and dY rows, the angles,
+// the B and C pairs) is requested in one round before the first barrier.  A tile row is one
+// (token, rank): row = R u + r.
+template <int NST, int RK>
 __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ TcBwd p) {
     using C = VuCfg<NST>;
-    constexpr int NH = C::NH;
+    constexpr int NH = C::NH, QT = kQ / RK;
     const BwdArgs& a = p.a;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -231,14 +244,15 @@ __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ 
     const int c = (int)(blockIdx.x % p.nch);
     const size_t bh = blockIdx.x / p.nch;
     const int b = (int)(bh / a.H), h = (int)(bh % a.H), g = h / (a.H / a.G);
-    const long long t0 = (long long)c * kQ;
+    const long long t0 = (long long)c * QT;
     const size_t cc = bh * p.nch + c;
 
-    constexpr int SEGS = C::NT / NH, TPS = kQ / SEGS, XT = 2 * kQ * 8 / C::NT;
+    constexpr int SEGS = C::NT / NH, TPS = kQ / SEGS, TT = TPS / RK, XT = 2 * kQ * 8 / C::NT;
+    static_assert(TT * RK == TPS, "a segment holds whole tokens");
     const int j = tid % NH, sg = tid / NH;
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     uint4 xv[XT];
-    float thv[TPS];
+    float thv[TT];
     uint32_t pbv[TPS], pcv[TPS];
     {
         const uint16_t* xg = static_cast<const uint16_t*>(a.x);
@@ -250,21 +264,27 @@ __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ 
             const int i = tid + C::NT * m;
             const bool isY = i >= kQ * 8;
             const int e = isY ? i - kQ * 8 : i;
-            const long long t = t0 + (e >> 3);
-            xv[m] = t < a.T ? *reinterpret_cast<const uint4*>((isY ? yg : xg) +
-                                                             (((size_t)b * a.T + t) * a.H + h) * kPc + (e & 7) * 8)
+            const int row = e >> 3;
+            const long long t = t0 + row / RK;
+            xv[m] = t < a.T ? *reinterpret_cast<const uint4*>(
+                                  (isY ? yg : xg) +
+                                  ((((size_t)b * a.T + t) * a.H + h) * RK + row % RK) * kPc + (e & 7) * 8)
                             : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
+        for (int i = 0; i < TT; ++i) {
+            const long long t = t0 + sg * TT + i;
+            thv[i] = t < a.T ? a.theta[(((size_t)b * a.T + t) * a.G + g) * NH + j] : 0.f;
+        }
+#pragma unroll
         for (int i = 0; i < TPS; ++i) {
-            const long long t = t0 + sg * TPS + i;
-            thv[i] = 0.f;
+            const int row = sg * TPS + i;
+            const long long t = t0 + row / RK;
             pbv[i] = pcv[i] = 0u;
             if (t < a.T) {
-                const size_t row = ((size_t)b * a.T + t) * a.G + g;
-                thv[i] = a.theta[row * NH + j];
-                pbv[i] = *reinterpret_cast<const uint32_t*>(Bg + row * NST + 2 * j);
-                pcv[i] = *reinterpret_cast<const uint32_t*>(Cg + row * NST + 2 * j);
+                const size_t o = ((((size_t)b * a.T + t) * a.G + g) * RK + row % RK) * NST + 2 * j;
+                pbv[i] = *reinterpret_cast<const uint32_t*>(Bg + o);
+                pcv[i] = *reinterpret_cast<const uint32_t*>(Cg + o);
             }
         }
     }
@@ -277,13 +297,13 @@ __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ 
         tmem_alloc(&misc[0], 128);
         tmem_relinquish();
     }
-    if (w == 0) chunk_coefs(a, b, h, t0, k);
+    if (w == 0) chunk_coefs<QT>(a, b, h, t0, k);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
     const Abort ab{reinterpret_cast<volatile uint32_t*>(&misc[1]), p.status, p.limit_ns};
-    if (tid == 0) p.ctot[cc] = k.cr[kQ - 1];
+    if (tid == 0) p.ctot[cc] = k.cr[QT - 1];
 
     // diag(e w) X and diag(f) dY
 #pragma unroll
@@ -291,21 +311,21 @@ __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ 
         const int i = tid + C::NT * m;
         const bool isY = i >= kQ * 8;
         const int e = isY ? i - kQ * 8 : i;
-        const int u = e >> 3;
-        const float sc = isY ? k.ff[u] : k.ew[u];
+        const int row = e >> 3;
+        const float sc = isY ? k.ff[row / RK] : k.ew[row / RK];
         const uint4 v = xv[m];
-        *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DYF : C::OFF_XW) + sw128_off(u, (e & 7) * 8)) =
+        *reinterpret_cast<uint4*>(sm + (isY ? C::OFF_DYF : C::OFF_XW) + sw128_off(row, (e & 7) * 8)) =
             make_uint4(scale2(v.x, sc), scale2(v.y, sc), scale2(v.z, sc), scale2(v.w, sc));
     }
     // B~, C~ in the chunk's frame: the segment's angle sums, the segments' totals exchanged,
     // then the rotation of the segment's tokens
     {
         float* segt = reinterpret_cast<float*>(sm + C::OFF_SEG);
-        float rho[TPS];
+        float rho[TT];
         float r = 0.f;
 #pragma unroll
-        for (int i = 0; i < TPS; ++i) {
-            r += angle ? thv[i] : k.dd[sg * TPS + i] * thv[i];
+        for (int i = 0; i < TT; ++i) {
+            r += angle ? thv[i] : k.dd[sg * TT + i] * thv[i];
             rho[i] = r;
         }
         segt[sg * NH + j] = r;
@@ -315,9 +335,9 @@ __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ 
         if (sg == SEGS - 1) p.atot[cc * NH + j] = off + r;
 #pragma unroll
         for (int i = 0; i < TPS; ++i) {
-            const int u = sg * TPS + i;
+            const int u = sg * TPS + i;   // tile row
             float sn, cs;
-            __sincosf(wrap_angle(off + rho[i]), &sn, &cs);
+            __sincosf(wrap_angle(off + rho[i / RK]), &sn, &cs);
             const float b0 = bf16lo(pbv[i]), b1 = bf16hi(pbv[i]), c0 = bf16lo(pcv[i]), c1 = bf16hi(pcv[i]);
             const uint32_t o = tile_off(u, 2 * j, kQ);
             *reinterpret_cast<uint32_t*>(sm + C::OFF_B + o) =
@@ -397,12 +417,12 @@ __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ 
 // ------------------------------------------------------------------------------------
 // 2. chunk scan: thread (channel p, pair group pg) holds state rows 2j, 2j+1 of column p for
 // the pairs j = pg + NPG k, k < 8.
-template <int NST>
+template <int NST, int RK>
 __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(const __grid_constant__ TcBwd p) {
     constexpr int NH = NST / 2, NPG = NST / 16, NT = 4 * NST, NW = NT / 32;
     const BwdArgs& a = p.a;
     __shared__ float red[2][NW];
-    __shared__ float part[NPG][kPc];
+    __shared__ float part[RK][NPG][kPc];
     __shared__ float exs[NH];
     const int tid = threadIdx.x, pc = tid & 63, pg = tid >> 6, lane = tid & 31, w = tid >> 5;
     const size_t bh = blockIdx.x;
@@ -412,17 +432,25 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
     if (tid < NH) exs[tid] = 0.f;
     __syncthreads();
 
-    // starting state g0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T
+    // starting state g0 = h0 + (1 - lam_0) dt_0 sum_r B_prev,r x_prev,r^T
     const size_t o0 = (size_t)b * a.T * a.H + h;
     const float k0 = (1.f - a.lam[o0]) * a.dt[o0];
-    const float xp = bf_at(a.x_prev, bh * kPc + pc);
-    const size_t bprow = ((size_t)b * a.G + g) * NST;
+    float xp[RK];
+#pragma unroll
+    for (int r = 0; r < RK; ++r) xp[r] = bf_at(a.x_prev, (bh * RK + r) * kPc + pc);
+    const size_t bprow = ((size_t)b * a.G + g) * RK * NST;   // B_prev row of rank r: + r NST
     float ge[8], go[8], P[8];
 #pragma unroll
     for (int kx = 0; kx < 8; ++kx) {
         const int j = pg + NPG * kx;
-        ge[kx] = fmaf(k0 * bf_at(a.B_prev, bprow + 2 * j), xp, a.h0[bh * NP + (size_t)(2 * j) * kPc + pc]);
-        go[kx] = fmaf(k0 * bf_at(a.B_prev, bprow + 2 * j + 1), xp, a.h0[bh * NP + (size_t)(2 * j + 1) * kPc + pc]);
+        float se = 0.f, so = 0.f;
+#pragma unroll
+        for (int r = 0; r < RK; ++r) {
+            se = fmaf(bf_at(a.B_prev, bprow + r * NST + 2 * j), xp[r], se);
+            so = fmaf(bf_at(a.B_prev, bprow + r * NST + 2 * j + 1), xp[r], so);
+        }
+        ge[kx] = fmaf(k0, se, a.h0[bh * NP + (size_t)(2 * j) * kPc + pc]);
+        go[kx] = fmaf(k0, so, a.h0[bh * NP + (size_t)(2 * j + 1) * kPc + pc]);
         P[kx] = 0.f;
     }
     // forward: the state entering every chunk, then the chunk's contribution in the call
@@ -550,30 +578,41 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
             p.q[cc] = dec * t;
         }
     }
-    // the starting state: dh0 = dg; dx_prev = k0 B_prev^T dg; dB_prev += k0 dg x_prev;
-    // v0 = <dg, B_prev x_prev^T> (for dt_0 and lam_0)
-    float pp = 0.f;
+    // the starting state: dh0 = dg; dx_prev,r = k0 B_prev,r^T dg; dB_prev,r += k0 dg x_prev,r;
+    // v0 = sum_r <dg, B_prev,r x_prev,r^T> (for dt_0 and lam_0)
+    float pp[RK];
+#pragma unroll
+    for (int r = 0; r < RK; ++r) pp[r] = 0.f;
 #pragma unroll
     for (int kx = 0; kx < 8; ++kx) {
         const int j = pg + NPG * kx;
         a.dh0[bh * NP + (size_t)(2 * j) * kPc + pc] = de[kx];
         a.dh0[bh * NP + (size_t)(2 * j + 1) * kPc + pc] = dq[kx];
-        pp = fmaf(de[kx], bf_at(a.B_prev, bprow + 2 * j), fmaf(dq[kx], bf_at(a.B_prev, bprow + 2 * j + 1), pp));
-        const float se = warp_sum(de[kx] * xp), so = warp_sum(dq[kx] * xp);
-        if (lane == 0) {
-            float* db = a.dB_prev + bprow + 2 * j;
-            atomicAdd(db, k0 * se);
-            atomicAdd(db + 1, k0 * so);
+#pragma unroll
+        for (int r = 0; r < RK; ++r) {
+            const size_t br = bprow + r * NST + 2 * j;
+            pp[r] = fmaf(de[kx], bf_at(a.B_prev, br), fmaf(dq[kx], bf_at(a.B_prev, br + 1), pp[r]));
+            const float se = warp_sum(de[kx] * xp[r]), so = warp_sum(dq[kx] * xp[r]);
+            if (lane == 0) {
+                atomicAdd(a.dB_prev + br, k0 * se);
+                atomicAdd(a.dB_prev + br + 1, k0 * so);
+            }
         }
     }
-    part[pg][pc] = pp;
-    const float sv = warp_sum(pp * xp);
+    float sv = 0.f;
+#pragma unroll
+    for (int r = 0; r < RK; ++r) {
+        part[r][pg][pc] = pp[r];
+        sv = fmaf(pp[r], xp[r], sv);
+    }
+    sv = warp_sum(sv);
     __syncthreads();
     if (lane == 0) red[0][w] = sv;
-    if (tid < kPc) {
+    for (int e = tid; e < RK * kPc; e += NT) {
+        const int r = e / kPc, c2 = e % kPc;
         float t = 0.f;
-        for (int i = 0; i < NPG; ++i) t += part[i][tid];
-        a.dx_prev[bh * kPc + tid] = k0 * t;
+        for (int i = 0; i < NPG; ++i) t += part[r][i][c2];
+        a.dx_prev[(bh * RK + r) * kPc + c2] = k0 * t;
     }
     __syncthreads();
     if (tid == 0) {
@@ -594,7 +633,7 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
 //   2. dC~ += dS B~, B~ dg;                    epilogue: dC~ rotated back (dC), angle terms;
 //                                              <X_s, (B~ dg)_s>, row scale e w; X <- e w X
 //   3. dX = (L o S)^T dY + ., dB~ = (e w X) dg^T + dS^T C~;   epilogue: dX, dB
-template <int NST>
+template <int NST, int RK>
 struct GrCfg {
     static constexpr int NH = NST / 2;
     static constexpr int T64 = kQ * 128;                      // one [Q][64] bf16 tile
@@ -609,7 +648,10 @@ struct GrCfg {
     static constexpr int OFF_ACC = OFF_COEF + Coefs::kFloats * 4;
     static constexpr int OFF_BAR = (OFF_ACC + (NACC * kQ + 4) * 4 + 7) / 8 * 8;
     static constexpr int OFF_MISC = OFF_BAR + 4 * 8;
-    static constexpr int USED = OFF_MISC + 16 + 1024;
+    // with R > 1 the R rows of a token add their angle gradients into a table of their own
+    // [Q / R][NH] fp32 (the angle table is still read while they are formed)
+    static constexpr int OFF_DPS = OFF_MISC + 16;
+    static constexpr int USED = OFF_DPS + (RK > 1 ? (kQ / RK) * NH * 4 : 0) + 1024;
     // two CTAs per SM (2 x 256 TMEM columns), never three
     static constexpr int SMEM = USED > 79872 ? USED : 79872;
     static_assert(2 * (SMEM + 1024) <= 233472 && 3 * (SMEM + 1024) > 233472, "two CTAs per SM");
@@ -660,10 +702,10 @@ __device__ __forceinline__ float colsum16(float (&v)[16], int lane) {
     return v[0];
 }
 
-template <int NST>
+template <int NST, int RK>
 __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant__ TcBwd p) {
-    using C = GrCfg<NST>;
-    constexpr int NH = C::NH;
+    using C = GrCfg<NST, RK>;
+    constexpr int NH = C::NH, QT = kQ / RK;
     const BwdArgs& a = p.a;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -682,13 +724,14 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     float* misc2 = acc + 9 * kQ;  // [0] dD partial, [1..2] warp sums, [3] suffix carry
     float* psi0 = reinterpret_cast<float*>(sm + C::OFF_MS);    // angle table, first home
     float* psi1 = reinterpret_cast<float*>(sm + C::OFF_GIN);   // and second
+    float* dpsi = RK > 1 ? reinterpret_cast<float*>(sm + C::OFF_DPS) : psi1;   // angle gradients
     float* segt = reinterpret_cast<float*>(sm + C::OFF_SEG);
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int c = (int)(blockIdx.x % p.nch);
     const size_t bh = blockIdx.x / p.nch;
     const int b = (int)(bh / a.H), h = (int)(bh % a.H), g = h / (a.H / a.G);
-    const long long t0 = (long long)c * kQ;
-    const int nv = (int)(a.T - t0 < kQ ? a.T - t0 : kQ);
+    const long long t0 = (long long)c * QT;
+    const int nv = (int)(a.T - t0 < QT ? a.T - t0 : QT);   // tokens of the chunk
     const size_t cc = bh * p.nch + c;
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     const uint32_t tile_bytes = NST * kPc * 2;
@@ -703,12 +746,15 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
         bulk_load(sm + C::OFF_DG, reinterpret_cast<const uint8_t*>(p.dgo) + cc * tile_bytes,
                   tile_bytes, &bar[0]);
     }
-    if (w == 1) chunk_coefs(a, b, h, t0, k);
+    if (w == 1) chunk_coefs<QT>(a, b, h, t0, k);
     for (int i = tid; i < C::NACC * kQ + 4; i += 256) acc[i] = 0.f;
+    if constexpr (RK > 1)
+        for (int i = tid; i < QT * NH; i += 256) dpsi[i] = 0.f;
     // Every global input of the chunk is requested before any of it is used: the angle
     // prefix's theta and dt, the chunk-start angle, the X and dY rows; then, behind the first
     // barrier, the B and C pairs of the rotation while the angle offsets are formed.
-    constexpr int SEGS = 256 / NH, TPS = kQ / SEGS;
+    constexpr int SEGS = 256 / NH, TPS = QT / SEGS;   // tokens of a (pair, segment)
+    static_assert(TPS * SEGS == QT, "whole tokens per segment");
     const int jj = tid % NH, sg = tid / NH;
     float rho[TPS];
     {
@@ -730,9 +776,11 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
             const int i = tid + 256 * m;
             const bool isY = i >= kQ * 8;
             const int e = isY ? i - kQ * 8 : i;
-            const long long t = t0 + (e >> 3);
-            xv[m] = t < a.T ? *reinterpret_cast<const uint4*>((isY ? yg : xg) +
-                                                             (((size_t)b * a.T + t) * a.H + h) * kPc + (e & 7) * 8)
+            const int row = e >> 3;
+            const long long t = t0 + row / RK;
+            xv[m] = t < a.T ? *reinterpret_cast<const uint4*>(
+                                  (isY ? yg : xg) +
+                                  ((((size_t)b * a.T + t) * a.H + h) * RK + row % RK) * kPc + (e & 7) * 8)
                             : make_uint4(0u, 0u, 0u, 0u);
         }
         float r = 0.f;
@@ -751,7 +799,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
         }
     }
     __syncthreads();
-    // B~, C~ in the call frame: thread (pair jr, tokens ur + RS m) for m < KT
+    // B~, C~ in the call frame: thread (pair jr, tile rows ur + RS m) for m < KT
     constexpr int KT = kQ * NH / 256, RS = 256 / NH;
     const int jr = tid % NH, ur = tid / NH;
     uint32_t pbv[KT], pcv[KT];
@@ -760,12 +808,13 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
         const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
 #pragma unroll
         for (int m = 0; m < KT; ++m) {
-            const long long t = t0 + ur + RS * m;
+            const int rw = ur + RS * m;
+            const long long t = t0 + rw / RK;
             pbv[m] = pcv[m] = 0u;
             if (t < a.T) {
-                const size_t row = (((size_t)b * a.T + t) * a.G + g) * NST + 2 * jr;
-                pbv[m] = *reinterpret_cast<const uint32_t*>(Bg + row);
-                pcv[m] = *reinterpret_cast<const uint32_t*>(Cg + row);
+                const size_t o = ((((size_t)b * a.T + t) * a.G + g) * RK + rw % RK) * NST + 2 * jr;
+                pbv[m] = *reinterpret_cast<const uint32_t*>(Bg + o);
+                pcv[m] = *reinterpret_cast<const uint32_t*>(Cg + o);
             }
         }
         float off = p.P0[(bh * (p.nch + 1) + c) * NH + jj];
@@ -776,9 +825,9 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     __syncthreads();
 #pragma unroll
     for (int m = 0; m < KT; ++m) {
-        const int u = ur + RS * m;
+        const int u = ur + RS * m;   // tile row
         float sn, cs2;
-        __sincosf(psi0[psi_idx<NH>(u, jr)], &sn, &cs2);
+        __sincosf(psi0[psi_idx<NH>(u / RK, jr)], &sn, &cs2);
         const float b0 = bf16lo(pbv[m]), b1 = bf16hi(pbv[m]), c0 = bf16lo(pcv[m]), c1 = bf16hi(pcv[m]);
         const uint32_t off = tile_off(u, 2 * jr, kQ);
         *reinterpret_cast<uint32_t*>(sm + C::OFF_B + off) =
@@ -826,6 +875,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
 
     const int q4 = w & 3, wg = w >> 2, hf = lane >> 4;
     const int t = 16 * q4 + (lane & 15);          // this thread's accumulator row
+    const int tu = t / RK;                        // and its token
     const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
     auto flag_ok = [&]() { return *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u; };
 
@@ -842,14 +892,15 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     __syncthreads();
     ok = ok && flag_ok();
     if (ok) {
-        const float crt = k.cr[t];
+        const float crt = k.cr[tu];
         {
             const int cb = 16 * wg, col0 = cb + 32 * hf;
             uint32_t sv[16], gv[16];
             ld_blk<64>(tq, C::TM_A, cb, sv);
             ld_blk<64>(tq, C::TM_GX, cb, gv);
             tmem_wait_ld();
-            float ca[16], cbv[16], rsum = 0.f, ddiag = 0.f;
+            float ca[16], cbv[16], rsum = 0.f, ddiag = 0.f, dgl = 0.f;
+            bool dgh = false;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t ms[4], ds[4];
@@ -859,10 +910,10 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int i = 8 * hh + i2 + e;
-                        const int s = col0 + i;
-                        const bool in = s <= t;
-                        const float E = in ? ex2f((crt - k.cr[s]) * kLog2e) : 0.f;
-                        const float om = in ? k.gam[s] + (s < t ? k.nx[s] : 0.f) : 0.f;
+                        const int s = col0 + i, su = s / RK;
+                        const bool in = su <= tu;
+                        const float E = in ? ex2f((crt - k.cr[su]) * kLog2e) : 0.f;
+                        const float om = in ? k.gam[su] + (su < tu ? k.nx[su] : 0.f) : 0.f;
                         const float L = E * om;
                         const float S = __uint_as_float(sv[i]), G = __uint_as_float(gv[i]);
                         mv[e] = S * L;
@@ -871,10 +922,11 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
                         ca[i] = dom * om;
                         cbv[i] = dom;
                         rsum += dom * om;
-                        if (s == t) {
-                            dgd[t] = dom;
-                            ddiag = G;
+                        if (su == tu) {
+                            dgl += dom;
+                            dgh = true;
                         }
+                        if (s == t) ddiag = G;
                     }
                     ms[i2 / 2] = pack_bf16x2(mv[0], mv[1]);
                     ds[i2 / 2] = pack_bf16x2(dvv[0], dvv[1]);
@@ -885,15 +937,16 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
                     make_uint4(ds[0], ds[1], ds[2], ds[3]);
             }
             if (ddiag != 0.f) atomicAdd(&misc2[0], ddiag);
+            if (dgh) atomicAdd(&dgd[tu], dgl);
             const float csum = colsum16(ca, lane), gsum = colsum16(cbv, lane);
-            atomicAdd(&cs[col0 + (lane & 15)], csum);
-            atomicAdd(&ga[col0 + (lane & 15)], gsum);
+            atomicAdd(&cs[(col0 + (lane & 15)) / RK], csum);
+            atomicAdd(&ga[(col0 + (lane & 15)) / RK], gsum);
             rsum += __shfl_xor_sync(0xffffffffu, rsum, 16);
-            if (hf == 0) atomicAdd(&rs[t], rsum);
+            if (hf == 0) atomicAdd(&rs[tu], rsum);
         }
         {
             float d = 0.f;
-            const float sf = k.ff[t];
+            const float sf = k.ff[tu];
 #pragma unroll
             for (int m = 0; m < NST / 64; ++m) {
                 const int cb = 16 * (wg + 2 * m), col0 = cb + (NST / 2) * hf;
@@ -913,7 +966,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
                 st_blk<NST>(tq, C::TM_C, cb, v);
             }
             d += __shfl_xor_sync(0xffffffffu, d, 16);
-            if (hf == 0) atomicAdd(&qz[t], d);
+            if (hf == 0) atomicAdd(&qz[tu], d);
         }
         tmem_wait_st();
     }
@@ -940,9 +993,9 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     }
 
     // ---- second epilogue: <X_s, (B~ dg)_s>, row scale e w, X <- e w X; dC~ rotated back
-    const long long tg = t0 + t;
-    const bool live = t < nv;
-    const size_t grow = (((size_t)b * a.T + (live ? tg : 0)) * a.G + g) * NST;
+    const long long tg = t0 + tu;
+    const bool live = tu < nv;
+    const size_t grow = ((((size_t)b * a.T + (live ? tg : 0)) * a.G + g) * RK + t % RK) * NST;
     constexpr int NB = NST / 64;          // 16-column blocks per thread in an N-wide tile
     float dps[NB * 8];                    // this thread's angle gradients (from dC~)
     ok = ok && warp_wait_b(&bar[2], 0, ab);
@@ -958,7 +1011,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
             const uint4 x0 = *xp0, x1 = *xp1;
             const uint32_t xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
             float d = 0.f;
-            const float sc = k.ew[t];
+            const float sc = k.ew[tu];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
@@ -970,7 +1023,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
             *xp0 = make_uint4(scale2(x0.x, sc), scale2(x0.y, sc), scale2(x0.z, sc), scale2(x0.w, sc));
             *xp1 = make_uint4(scale2(x1.x, sc), scale2(x1.y, sc), scale2(x1.z, sc), scale2(x1.w, sc));
             d += __shfl_xor_sync(0xffffffffu, d, 16);
-            if (hf == 0) atomicAdd(&dv[t], d);
+            if (hf == 0) atomicAdd(&dv[tu], d);
         }
         const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
 #pragma unroll
@@ -989,7 +1042,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 float sn, cs2;
-                __sincosf(psi1[psi_idx<NH>(t, col0 / 2 + i)], &sn, &cs2);
+                __sincosf(psi1[psi_idx<NH>(tu, col0 / 2 + i)], &sn, &cs2);
                 const float c0 = bf16lo(cw[i]), c1 = bf16hi(cw[i]);
                 const float ct0 = fmaf(cs2, c0, sn * c1), ct1 = fmaf(cs2, c1, -sn * c0);
                 const float dc0 = __uint_as_float(vc[2 * i]), dc1 = __uint_as_float(vc[2 * i + 1]);
@@ -1046,7 +1099,8 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
             const uint4 y1 = *reinterpret_cast<const uint4*>(sm + C::OFF_DY + sw128_off(t, col0 + 8));
             const uint32_t ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
             if (live) {
-                float4* dst = reinterpret_cast<float4*>(a.dx + (((size_t)b * a.T + tg) * a.H + h) * kPc + col0);
+                float4* dst = reinterpret_cast<float4*>(
+                    a.dx + ((((size_t)b * a.T + tg) * a.H + h) * RK + t % RK) * kPc + col0);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     dst[i] = make_float4(fmaf(Dh, bf16lo(ys[2 * i]), __uint_as_float(v[4 * i])),
@@ -1073,11 +1127,15 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
             for (int i = 0; i < 8; ++i) {
                 const int j = col0 / 2 + i;
                 float sn, cs2;
-                __sincosf(psi1[psi_idx<NH>(t, j)], &sn, &cs2);
+                __sincosf(psi1[psi_idx<NH>(tu, j)], &sn, &cs2);
                 const float b0 = bf16lo(bw[i]), b1 = bf16hi(bw[i]);
                 const float bt0 = fmaf(cs2, b0, sn * b1), bt1 = fmaf(cs2, b1, -sn * b0);
                 const float db0 = __uint_as_float(vb[2 * i]), db1 = __uint_as_float(vb[2 * i + 1]);
-                psi1[psi_idx<NH>(t, j)] = dps[8 * m + i] + fmaf(db0, bt1, -db1 * bt0);
+                const float gp = dps[8 * m + i] + fmaf(db0, bt1, -db1 * bt0);
+                if constexpr (RK == 1)
+                    psi1[psi_idx<NH>(t, j)] = gp;   // the angle is read by this thread alone
+                else
+                    atomicAdd(&dpsi[psi_idx<NH>(tu, j)], gp);
                 ob[2 * i] = fmaf(cs2, db0, -sn * db1);
                 ob[2 * i + 1] = fmaf(sn, db0, cs2 * db1);
             }
@@ -1108,7 +1166,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
         float r = 0.f;
 #pragma unroll
         for (int i = TPS - 1; i >= 0; --i) {
-            r += psi1[psi_idx<NH>(sg * TPS + i, jj)];
+            r += dpsi[psi_idx<NH>(sg * TPS + i, jj)];
             loc[i] = r;
         }
         segt[sg * NH + jj] = r;
@@ -1173,7 +1231,7 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
             a.dA[o] = dda * k.dd[u];
             a.dlam[o] = dlam;
         }
-        if (u == kQ - 1) p.spill[cc] = dnx[u];
+        if (u == QT - 1) p.spill[cc] = dnx[u];
         if (u == 0 && a.D && a.dD) atomicAdd(&a.dD[h], misc2[0]);
     }
 }
@@ -1212,8 +1270,8 @@ __global__ void __launch_bounds__(256, 2) bwd_finish_kernel(const __grid_constan
     const long long bg = blockIdx.x / p.nch;
     const int g = (int)(bg % a.G), b = (int)(bg / a.G);
     const int hpg = a.H / a.G;
-    const long long t0 = (long long)c * kQ, t = t0 + u;
-    const int nv = (int)(a.T - t0 < kQ ? a.T - t0 : kQ);
+    const long long t0 = (long long)c * p.qt, t = t0 + u;
+    const int nv = (int)(a.T - t0 < p.qt ? a.T - t0 : p.qt);
     const bool live = u < nv;
     const bool angle = (a.flags & M3_FLAG_THETA_IS_ANGLE) != 0;
     const size_t trow = ((size_t)b * a.T + (live ? t : 0)) * a.G + g;
@@ -1287,8 +1345,9 @@ struct Layout {
     size_t V, U, gin, dgo, ctot, atot, P0, q, dtot, spill, extra, v0, pang, carry, bytes;
 };
 
-Layout layout(int batch, int H, int N, long long T) {
-    const size_t BH = (size_t)batch * H, nch = (size_t)((T + kQ - 1) / kQ), NP = (size_t)N * kPc;
+Layout layout(int batch, int H, int N, int R, long long T) {
+    const long long qt = kQ / R;
+    const size_t BH = (size_t)batch * H, nch = (size_t)((T + qt - 1) / qt), NP = (size_t)N * kPc;
     const size_t NH = N / 2;
     Layout L;
     size_t o = 0;
@@ -1315,16 +1374,16 @@ Layout layout(int batch, int H, int N, long long T) {
     return L;
 }
 
-template <int NST>
+template <int NST, int RK>
 cudaError_t launch_n(const TcBwd& p, long long units, cudaStream_t s) {
-    const int smv = VuCfg<NST>::SMEM, smg = GrCfg<NST>::SMEM;
-    cudaError_t e = cudaFuncSetAttribute(bwd_vu_kernel<NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smv);
+    const int smv = VuCfg<NST>::SMEM, smg = GrCfg<NST, RK>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(bwd_vu_kernel<NST, RK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smv);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_grads_kernel<NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smg);
+    e = cudaFuncSetAttribute(bwd_grads_kernel<NST, RK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smg);
     if (e != cudaSuccess) return e;
-    bwd_vu_kernel<NST><<<(unsigned)units, VuCfg<NST>::NT, smv, s>>>(p);
-    bwd_scan_kernel<NST><<<(unsigned)((size_t)p.a.batch * p.a.H), 4 * NST, 0, s>>>(p);
-    bwd_grads_kernel<NST><<<(unsigned)units, 256, smg, s>>>(p);
+    bwd_vu_kernel<NST, RK><<<(unsigned)units, VuCfg<NST>::NT, smv, s>>>(p);
+    bwd_scan_kernel<NST, RK><<<(unsigned)((size_t)p.a.batch * p.a.H), 4 * NST, 0, s>>>(p);
+    bwd_grads_kernel<NST, RK><<<(unsigned)units, 256, smg, s>>>(p);
     const long long bhj = (long long)p.a.batch * p.a.H * (NST / 2);
     bwd_carry_kernel<<<(unsigned)((bhj + 255) / 256), 256, 0, s>>>(p, NST / 2);
     bwd_finish_kernel<NST / 2><<<(unsigned)((long long)p.a.batch * p.a.G * p.nch), 256, 0, s>>>(p);
@@ -1334,20 +1393,22 @@ cudaError_t launch_n(const TcBwd& p, long long units, cudaStream_t s) {
 }  // namespace
 
 bool scan_bwd_tc_ok(int io_dtype, int N, int P, int R) {
-    return io_dtype == M3_BF16 && R == 1 && P == kPc && (N == 64 || N == 128);
+    return io_dtype == M3_BF16 && P == kPc &&
+           ((R == 1 && (N == 64 || N == 128)) || ((R == 2 || R == 4) && N == 64));
 }
 
-size_t scan_bwd_tc_workspace_bytes(int batch, int H, int N, long long T) {
-    return layout(batch, H, N, T).bytes;
+size_t scan_bwd_tc_workspace_bytes(int batch, int H, int N, int R, long long T) {
+    return layout(batch, H, N, R, T).bytes;
 }
 
-cudaError_t launch_scan_bwd_tc(const BwdArgs& a, void* ws, uint32_t* status, unsigned long long limit_ns,
-                               cudaStream_t s) {
-    const Layout L = layout(a.batch, a.H, a.N, a.T);
+cudaError_t launch_scan_bwd_tc(const BwdArgs& a, int R, void* ws, uint32_t* status,
+                               unsigned long long limit_ns, cudaStream_t s) {
+    const Layout L = layout(a.batch, a.H, a.N, R, a.T);
     uint8_t* base = static_cast<uint8_t*>(ws);
     TcBwd p;
     p.a = a;
-    p.nch = (int)((a.T + kQ - 1) / kQ);
+    p.qt = kQ / R;
+    p.nch = (int)((a.T + p.qt - 1) / p.qt);
     p.V = reinterpret_cast<uint16_t*>(base + L.V);
     p.U = reinterpret_cast<uint16_t*>(base + L.U);
     p.gin = reinterpret_cast<uint16_t*>(base + L.gin);
@@ -1365,7 +1426,10 @@ cudaError_t launch_scan_bwd_tc(const BwdArgs& a, void* ws, uint32_t* status, uns
     p.status = status;
     p.limit_ns = limit_ns;
     const long long units = (long long)a.batch * a.H * p.nch;
-    return a.N == 128 ? launch_n<128>(p, units, s) : launch_n<64>(p, units, s);
+    if (a.N == 128) return launch_n<128, 1>(p, units, s);
+    if (R == 2) return launch_n<64, 2>(p, units, s);
+    if (R == 4) return launch_n<64, 4>(p, units, s);
+    return launch_n<64, 1>(p, units, s);
 }
 
 }  // namespace m3

@@ -1,5 +1,5 @@
-"""Parity of the chunked tensor-core backward (m3_scan_bwd for SISO bf16, P 64, N 64 / 128)
-with the fp64 oracle's backward, through the C ABI.
+"""Parity of the chunked tensor-core backward (m3_scan_bwd for bf16, P 64: SISO with N 64 / 128,
+MIMO ranks 2 and 4 with N 64) with the fp64 oracle's backward, through the C ABI.
 
 The chunked backward multiplies bf16 operands on the tensor cores (the rotated B and C, the
 masked score tiles, the chunk states and their adjoints), so the bar is the bf16 one of the
@@ -41,11 +41,11 @@ def _rel(a, b):
     return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-30))
 
 
-def _problem(b, H, G, N, T, seed, dhT=True, theta_max=1.0):
-    inp = inputs.make_scan_inputs(b, T, H, G, 64, N, 1, io_dtype=torch.bfloat16,
+def _problem(b, H, G, N, T, seed, dhT=True, theta_max=1.0, R=1):
+    inp = inputs.make_scan_inputs(b, T, H, G, 64, N, R, io_dtype=torch.bfloat16,
                                   theta_max=theta_max, seed=seed, h0_random=True, carry_prev=True)
     gen = torch.Generator().manual_seed(seed + 5)
-    dy = torch.randn((b, T, H, 1, 64), generator=gen).to(torch.bfloat16)
+    dy = torch.randn((b, T, H, R, 64), generator=gen).to(torch.bfloat16)
     dh = torch.randn((b, H, N, 64), generator=gen) if dhT else None
     return inp, dy, dh
 
@@ -107,6 +107,47 @@ def test_tc_backward_matches_oracle(case):
     assert all(e <= TOL for e in errs.values()), errs
 
 
+MIMO_CASES = [
+    # (b, H, G, R, T, flags, dhT, theta_max): a chunk holds 64 / R tokens
+    (1, 2, 1, 2, 100, 0, True, 1.0),            # four chunks, ragged tail
+    (2, 4, 2, 4, 70, 0, True, 1.0),             # five chunks, two groups
+    (1, 2, 1, 4, 16, 0, True, 1.0),             # exactly one chunk
+    (1, 2, 1, 4, 17, 0, True, 1.0),             # one token past a chunk
+    (1, 3, 1, 2, 1, 0, True, 1.0),              # one token
+    (1, 2, 2, 4, 300, 0, False, math.pi),       # G = H, no dL/dh_T, fast rotation
+    (1, 2, 1, 2, 130, m3.M3_FLAG_THETA_IS_ANGLE, True, 0.1),
+    (1, 8, 1, 4, 500, 0, True, math.pi / 4),    # eight heads of one group, 32 chunks
+]
+
+
+def _mid(c):
+    return (f"b{c[0]}H{c[1]}G{c[2]}R{c[3]}T{c[4]}{'A' if c[5] else ''}"
+            f"{'' if c[6] else 'nodh'}")
+
+
+@pytest.mark.parametrize("case", MIMO_CASES, ids=[_mid(c) for c in MIMO_CASES])
+def test_tc_backward_mimo_matches_oracle(case):
+    b, H, G, R, T, flags, with_dh, tmax = case
+    inp, dy, dh = _problem(b, H, G, 64, T, seed=65, dhT=with_dh, theta_max=tmax, R=R)
+    d = m3.Dims(b, H, G, 64, 64, R, m3.M3_BF16)
+    got = _gpu_bwd(inp, dy, dh, d, T, flags)
+    ref = _oracle_bwd(inp, dy, dh, angle=bool(flags & m3.M3_FLAG_THETA_IS_ANGLE))
+    for k in m3.GRAD_NAMES:
+        assert np.all(np.isfinite(got[k])), k
+    errs = _slice_errors(got, ref)
+    assert all(e <= TOL for e in errs.values()), errs
+
+
+def test_tc_backward_mimo_against_sequential_kernel():
+    """Rank 4: the chunked path against the sequential fp32 kernel on the same inputs."""
+    inp, dy, dh = _problem(1, 4, 1, 64, 203, seed=66, R=4)
+    d = m3.Dims(1, 4, 1, 64, 64, 4, m3.M3_BF16)
+    tc = _gpu_bwd(inp, dy, dh, d, 203)
+    seq = _gpu_bwd(inp, dy, dh, d, 203, flags=m3.M3_FLAG_FORCE_SIMT)
+    errs = _slice_errors(tc, seq)
+    assert all(e <= TOL for e in errs.values()), errs
+
+
 def test_tc_backward_without_D():
     inp, dy, dh = _problem(1, 2, 1, 128, 150, seed=62)
     d = m3.Dims(1, 2, 1, 64, 128, 1, m3.M3_BF16)
@@ -142,11 +183,12 @@ def test_tc_backward_all_heads_of_a_group():
     assert all(e <= TOL for e in errs.values()), errs
 
 
-def test_tc_backward_fullsize_sampled_heads():
-    """The 1.5B-scale SISO prefill workload (b8 H64 T4096 P64 N128, bf16), backward at full
-    size on the chunked path; per-head gradients of heads 0 and 37 of batch row 0 against the
-    oracle on those two heads, the group-summed ones finite."""
-    w = inputs.WORKLOADS["siso_prefill_1p5b"]
+@pytest.mark.parametrize("name", ["siso_prefill_1p5b", "mimo_prefill_r4"])
+def test_tc_backward_fullsize_sampled_heads(name):
+    """The 1.5B-scale prefill workloads (b8 H64 T4096 P64: SISO N128, MIMO rank 4 N64; bf16),
+    backward at full size on the chunked path; per-head gradients of heads 0 and 37 of batch
+    row 0 against the oracle on those two heads, the group-summed ones finite."""
+    w = inputs.WORKLOADS[name]
     b, H, G, P, N, R, T = w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank, w.seqlen
     inp = inputs.make_scan_inputs(b, T, H, G, P, N, R, io_dtype=w.io_dtype, seed=7)
     gen = torch.Generator().manual_seed(12)
