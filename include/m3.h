@@ -320,13 +320,24 @@ m3_status m3_decode_step_gated(const m3_dims* dims, const void* x, const void* B
  *        dB_prev [b][G][R][N] (summed over the group's heads).
  *   The carried x_prev / B_prev outputs of the forward call (copies of its last token) get no
  *   gradient here: a caller chaining calls adds theirs to dx / dB of the last token.
- *   The states are recomputed inside (checkpoints every segment of up to 16 tokens, in the
- *   workspace); the call runs a sequential fp32 kernel, one CTA per (batch, head), then sums
- *   the per-head shares of the group gradients in a fixed order.  The sums over state pairs
- *   inside a head use shared-memory atomics, so dx, ddt, dA and dlam may differ in the last
- *   bits from run to run.  Supported: N even, N <= 256, P <= 64, R in {1, 2, 3, 4, 8}, within
- *   the kernel's thread and shared-memory limits (else M3_ERR_UNSUPPORTED).  seqlen 0 does
- *   nothing.
+ *   Two implementations, chosen by shape:
+ *   - bf16 io, P = 64, and either R = 1 with N in {64, 128} or R in {2, 4} with N = 64 (and
+ *     dx, dB, dC 16-byte aligned): the chunked backward on the tensor cores ("Parallel
+ *     representation under SSD"; chunks of 64 / R tokens, 64 (token, rank) rows).  Chunk
+ *     products, a scan over chunks for the entering states and leaving adjoints (stored in the
+ *     workspace as bf16), the chunk gradients from bf16 operands with fp32 accumulation, and
+ *     the angle carries.  dB, dC, dB_prev and dD are accumulated with atomics (last bits may
+ *     vary from run to run); dtheta is summed over the group's heads in a fixed order.
+ *     Accuracy: the bf16 bar of the prefill (about 1e-2 of each gradient's largest value).
+ *   - every other shape, and any shape with M3_FLAG_FORCE_SIMT: a sequential fp32 kernel,
+ *     one CTA per (batch, head), with the states recomputed from checkpoints every segment
+ *     of up to 16 tokens, then the per-head shares of the group gradients summed in a fixed
+ *     order.  The sums over state pairs inside a head use shared-memory atomics, so dx, ddt,
+ *     dA and dlam may differ in the last bits from run to run.
+ *   Supported: N even, N <= 256, P <= 64, R in {1, 2, 3, 4, 8}, within the sequential
+ *   kernel's thread and shared-memory limits (else M3_ERR_UNSUPPORTED).  seqlen 0 does
+ *   nothing.  A wait of the chunked path that runs out of time reports M3_ERR_TIMEOUT
+ *   through the workspace's status word (m3_query_status).
  */
 typedef struct {
     float* dx;
@@ -342,9 +353,12 @@ typedef struct {
     float* dB_prev;
 } m3_grads;
 
-/* Workspace bytes of m3_scan_bwd for (dims, seqlen): the status block; per (batch, head)
- * one N x P fp32 state per segment and one segment of states; and the per-head shares of
- * the group gradients (2 R N + N/2 floats per token and head). */
+/* Workspace bytes of m3_scan_bwd for (dims, seqlen): the status block, then the larger of
+ * the two implementations' needs.  Sequential: per (batch, head) one N x P fp32 state per
+ * segment and one segment of states, and the per-head shares of the group gradients
+ * (2 R N + N/2 floats per token and head).  Chunked (the shapes listed at m3_scan_bwd): per
+ * (batch, head, chunk) four N x P bf16 tiles and a few scalars per state pair, plus one
+ * fp32 angle gradient per (batch, head, token, pair). */
 m3_status m3_scan_bwd_workspace_bytes(const m3_dims* dims, int32_t seqlen, size_t* bytes);
 
 m3_status m3_scan_bwd(const m3_dims* dims, int32_t seqlen, const void* x, const void* B,
@@ -374,7 +388,7 @@ m3_status m3_scan_bwd(const m3_dims* dims, int32_t seqlen, const void* x, const 
  *        overwritten.  An extras pointer that is NULL or all zero runs m3_scan_bwd itself.
  *   The parameter gradients (dx_expand, dz_expand, dB_bias, dC_bias) and, on the chunked
  *   path, the group-shared ones are sums accumulated with atomics.  Supported: the shapes of
- *   m3_scan_bwd (the SISO bf16 P 64 shapes run the chunked tensor-core backward).
+ *   m3_scan_bwd (its chunked tensor-core shapes run the chunked backward).
  *   Workspace: m3_scan_bwd_workspace_bytes_ex (the recurrence backward's own workspace
  *   first, then the effective inputs, their gradients and, with the gate, the forward's
  *   workspace, a state copy and y_pre). */
