@@ -680,10 +680,11 @@ def ours(args):
         "clocks": clk.summary(),
     }
 
-    if args.prefill_only or args.bwd_only:
+    if args.prefill_only or args.bwd_only or args.mimo_only:
         args.no_decode = args.no_e2e = args.no_cpu = args.no_gate = args.no_mimo = True
         args.no_bwd = args.no_longctx = True
-        args.no_bwd = not args.bwd_only
+        args.no_bwd = not (args.bwd_only or args.mimo_only)
+        args.no_mimo = not args.mimo_only
     if not args.no_decode:
         line["decode"] = {}
         for name in (args.decode or DECODES):
@@ -743,7 +744,7 @@ def ours(args):
         line["longctx"] = longctx_leg(args, dev, stream, rank, ws_world, pk)
         line["small_f32"] = small_f32_leg(args, dev, stream, rank, ws_world)
 
-    if not args.no_bwd:
+    if not args.no_bwd and not args.mimo_only:
         line["backward"] = backward_leg(args, w, d, g, dev, stream, rank, ws_world, pk)
 
     if not args.no_e2e:
@@ -834,6 +835,8 @@ def main():
     ap.add_argument("--prefill-only", action="store_true", help="skip decode, e2e and CPU legs")
     ap.add_argument("--bwd-only", action="store_true",
                     help="the prefill line and the backward leg only (profiling)")
+    ap.add_argument("--mimo-only", action="store_true",
+                    help="the prefill line and the MIMO leg (prefill and backward) only (profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -1,7 +1,8 @@
 """Parity of the backward pass (m3_scan_bwd, reverse-mode gradients of the recurrence) with
 the fp64 oracle's backward, through the C ABI, on the same rounded inputs: the sequential fp32
-kernel (every shape it covers; SISO bf16 P 64 shapes through M3_FLAG_FORCE_SIMT, which would
-otherwise take the chunked tensor-core path checked in test_bwd_tc_gpu.py).
+kernel (every shape it covers; the bf16 P 64 shapes of the chunked tensor-core path, SISO
+N 64 / 128 and MIMO ranks 2 / 4 with N 64, through M3_FLAG_FORCE_SIMT, since they would
+otherwise take that path, checked in test_bwd_tc_gpu.py).
 
 The kernel computes in fp32 (checkpoints every 16 tokens, recomputed segments), so the
 bar is fp32 accumulation error: max |gpu - ref| / max |ref| per gradient tensor.  The full
@@ -69,7 +70,7 @@ CASES = [
     (1, 2, 1, 16, 16, 1, 50, torch.float32, m3.M3_FLAG_THETA_IS_ANGLE, True),
     (1, 4, 1, 64, 128, 1, 100, torch.bfloat16, m3.M3_FLAG_FORCE_SIMT, True),   # 1.5B-scale
     #                                   SISO head shape, on the sequential kernel
-    (1, 4, 2, 64, 64, 4, 70, torch.bfloat16, 0, True),     # MIMO R = 4
+    (1, 4, 2, 64, 64, 4, 70, torch.bfloat16, m3.M3_FLAG_FORCE_SIMT, True),   # MIMO R = 4
     (2, 2, 1, 40, 10, 2, 33, torch.float32, 0, True),      # two column blocks, partial warp
 ]
 
