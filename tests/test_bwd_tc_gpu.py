@@ -212,12 +212,13 @@ def test_tc_backward_fullsize_sampled_heads(name):
         assert np.all(np.isfinite(got[k])), k
 
 
-def test_tc_backward_fullsize_group_sums_vs_sequential():
-    """At the full 1.5B-scale size the group-summed gradients (dB, dC, dtheta over 64 heads,
-    dB_prev, dD over batch and tokens) of the chunked path against the sequential fp32
-    kernel on the same inputs (that kernel is held to the oracle at 2e-4 above and in
-    test_bwd_gpu.py), per (batch, group) slice."""
-    w = inputs.WORKLOADS["siso_prefill_1p5b"]
+@pytest.mark.parametrize("name", ["siso_prefill_1p5b", "mimo_prefill_r4"])
+def test_tc_backward_fullsize_group_sums_vs_sequential(name):
+    """At the full 1.5B-scale size (SISO N 128 and MIMO rank 4 N 64) the group-summed
+    gradients (dB, dC, dtheta over 64 heads, dB_prev, dD over batch and tokens) of the
+    chunked path against the sequential fp32 kernel on the same inputs (that kernel is held
+    to the oracle at 2e-4 above and in test_bwd_gpu.py), per (batch, group) slice."""
+    w = inputs.WORKLOADS[name]
     b, H, G, P, N, R, T = w.batch, w.nheads, w.ngroups, w.headdim, w.dstate, w.rank, w.seqlen
     inp = inputs.make_scan_inputs(b, T, H, G, P, N, R, io_dtype=w.io_dtype, seed=8,
                                   h0_random=True, carry_prev=True)
@@ -232,4 +233,13 @@ def test_tc_backward_fullsize_group_sums_vs_sequential():
     # <dg_0, B_prev x_prev^T>, whose adjoint dg_0 sums 64 chunks of bf16 products (measured
     # 2.2e-2 of its slice's largest value there, 0.3 % at the median slice)
     bars = {k: (3e-2 if k in ("ddt", "dA") else TOL) for k in errs}
+    if R > 1:
+        # dtheta_t is dt_t times a suffix sum, over every later token and the group's heads,
+        # of per-token angle gradients that cancel almost completely (a common rotation of
+        # all B~ and C~ leaves C~ B~^T unchanged), so the bf16 rounding of the chunk-boundary
+        # tiles (entering states, leaving adjoints) adds up over the suffix.  With 16-token
+        # chunks at rank 4 there are four times the boundaries of SISO: measured 3.3 % of the
+        # slice's largest value at the worst slice of 4096 tokens (3.2 % median, 1.3 % at
+        # 1024 tokens; SISO N 128: 0.9 %), largest at the first tokens
+        bars["dtheta"] = 5e-2
     assert all(errs[k] <= bars[k] for k in errs), errs
