@@ -416,11 +416,34 @@ __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ 
 
 // ------------------------------------------------------------------------------------
 // 2. chunk scan: thread (channel p, pair group pg) holds state rows 2j, 2j+1 of column p for
-// the pairs j = pg + NPG k, k < 8.
+// the pairs j = pg + NPG k, k < 8.  A chunk's inputs (its V or U tile, the stored entering
+// state, the angles and the decay) come through a ring of SCAN_KS shared-memory stages
+// filled by cp.async SCAN_KS - 1 chunks ahead, every thread copying 16-byte pieces.
+__device__ __forceinline__ void cpa16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cpa_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+constexpr int SCAN_KS = 3;
+template <int NST>
+struct ScanCfg {
+    static constexpr int TILE = NST * kPc * 2;                 // one [N][P] bf16 tile
+    static constexpr int VEC = NST / 2 * 4;                    // one fp32 value per pair
+    static constexpr int STAGE = 2 * TILE + VEC + 16;          // tile, tile, pairs, decay
+    static constexpr int SMEM = SCAN_KS * STAGE;
+};
+
 template <int NST, int RK>
 __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(const __grid_constant__ TcBwd p) {
     constexpr int NH = NST / 2, NPG = NST / 16, NT = 4 * NST, NW = NT / 32;
+    using SC = ScanCfg<NST>;
     const BwdArgs& a = p.a;
+    extern __shared__ __align__(128) uint8_t ring[];
     __shared__ float red[2][NW];
     __shared__ float part[RK][NPG][kPc];
     __shared__ float exs[NH];
@@ -454,32 +477,31 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
         P[kx] = 0.f;
     }
     // forward: the state entering every chunk, then the chunk's contribution in the call
-    // frame; the next chunk's V, decay and angles are requested one step ahead
-    uint16_t vn[16];
-    float atn[8], ctn;
-    auto fetch_fwd = [&](int c) {
+    // frame; stage c % KS holds chunk c's V tile, angles and decay
+    auto issue_fwd = [&](int c) {
         const size_t cc = bh * nch + c;
-        const uint16_t* V = p.V + cc * NP;
-#pragma unroll
-        for (int kx = 0; kx < 8; ++kx) {
-            const int j = pg + NPG * kx;
-            vn[2 * kx] = V[(size_t)(2 * j) * kPc + pc];
-            vn[2 * kx + 1] = V[(size_t)(2 * j + 1) * kPc + pc];
-            atn[kx] = p.atot[cc * NH + j];
-        }
-        ctn = p.ctot[cc];
+        uint8_t* d = ring + (c % SCAN_KS) * SC::STAGE;
+        const uint8_t* V = reinterpret_cast<const uint8_t*>(p.V + cc * NP);
+        for (int i = tid; i < SC::TILE / 16; i += NT) cpa16(d + 16 * i, V + 16 * i);
+        if (tid < SC::VEC / 16) cpa16(d + 2 * SC::TILE + 16 * tid, p.atot + cc * NH + 4 * tid);
+        if (tid == NT - 1) cpa4(d + 2 * SC::TILE + SC::VEC, p.ctot + cc);
     };
-    fetch_fwd(0);
+#pragma unroll
+    for (int i = 0; i < SCAN_KS - 1; ++i) {
+        if (i < nch) issue_fwd(i);
+        cpa_commit();
+    }
     for (int c = 0; c < nch; ++c) {
         const size_t cc = bh * nch + c;
-        uint16_t vc[16];
-        float atc[8];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) vc[i] = vn[i];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) atc[i] = atn[i];
-        const float dec = ex2f(ctn * kLog2e);
-        if (c + 1 < nch) fetch_fwd(c + 1);
+        __syncthreads();   // the stage read at c - 1 is free again
+        if (c + SCAN_KS - 1 < nch) issue_fwd(c + SCAN_KS - 1);
+        cpa_commit();
+        cpa_wait<SCAN_KS - 1>();
+        __syncthreads();   // chunk c's stage is complete
+        const uint8_t* st = ring + (c % SCAN_KS) * SC::STAGE;
+        const uint16_t* vt = reinterpret_cast<const uint16_t*>(st);
+        const float* at = reinterpret_cast<const float*>(st + 2 * SC::TILE);
+        const float dec = ex2f(at[NH] * kLog2e);
         uint8_t* gt = reinterpret_cast<uint8_t*>(p.gin) + cc * NP * 2;
 #pragma unroll
         for (int kx = 0; kx < 8; ++kx) {
@@ -487,13 +509,13 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
             if (pc == 0) p.P0[(bh * (nch + 1) + c) * NH + j] = P[kx];
             *reinterpret_cast<uint16_t*>(gt + sw128_off(2 * j, pc)) = to_bf(ge[kx]);
             *reinterpret_cast<uint16_t*>(gt + sw128_off(2 * j + 1, pc)) = to_bf(go[kx]);
-            const float v0 = __uint_as_float((uint32_t)vc[2 * kx] << 16);
-            const float v1 = __uint_as_float((uint32_t)vc[2 * kx + 1] << 16);
+            const float v0 = __uint_as_float((uint32_t)vt[(2 * j) * kPc + pc] << 16);
+            const float v1 = __uint_as_float((uint32_t)vt[(2 * j + 1) * kPc + pc] << 16);
             float sn, cs;
             __sincosf(P[kx], &sn, &cs);
             ge[kx] = fmaf(dec, ge[kx], fmaf(cs, v0, sn * v1));
             go[kx] = fmaf(dec, go[kx], fmaf(cs, v1, -sn * v0));
-            P[kx] = wrap_angle(P[kx] + atc[kx]);
+            P[kx] = wrap_angle(P[kx] + at[j]);
         }
     }
     // the final state and dL/dh_T: dg = R(-psi_T) dH; the last token's angle gradient
@@ -519,39 +541,43 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
     }
     __syncthreads();   // the chunk-start angles (global) and exs are complete
     if (tid < NH) p.extra[bh * NH + tid] = exs[tid];
-    // reverse: the adjoint of the state leaving every chunk; the next (earlier) chunk's U,
-    // stored entering state, angle and decay are requested one step ahead
-    uint16_t un[16], gn[16];
-    float pn[8], cn;
-    auto fetch_rev = [&](int c) {
+    // reverse: the adjoint of the state leaving every chunk; stage i % KS (i = nch - 1 - c)
+    // holds chunk c's U tile, its stored entering state, the angles before it and its decay.
+    // The entering states and angles were written by this CTA's forward sweep (ordered before
+    // these copies by the barrier above).
+    auto issue_rev = [&](int i) {
+        const int c = nch - 1 - i;
         const size_t cc = bh * nch + c;
-        const uint16_t* Uc = p.U + cc * NP;
+        uint8_t* d = ring + (i % SCAN_KS) * SC::STAGE;
+        const uint8_t* Uc = reinterpret_cast<const uint8_t*>(p.U + cc * NP);
         const uint8_t* gt = reinterpret_cast<const uint8_t*>(p.gin) + cc * NP * 2;
-#pragma unroll
-        for (int kx = 0; kx < 8; ++kx) {
-            const int j = pg + NPG * kx;
-            un[2 * kx] = Uc[(size_t)(2 * j) * kPc + pc];
-            un[2 * kx + 1] = Uc[(size_t)(2 * j + 1) * kPc + pc];
-            gn[2 * kx] = *reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j, pc));
-            gn[2 * kx + 1] = *reinterpret_cast<const uint16_t*>(gt + sw128_off(2 * j + 1, pc));
-            pn[kx] = p.P0[(bh * (nch + 1) + c) * NH + j];
+        for (int e = tid; e < SC::TILE / 16; e += NT) {
+            cpa16(d + 16 * e, Uc + 16 * e);
+            cpa16(d + SC::TILE + 16 * e, gt + 16 * e);
         }
-        cn = p.ctot[cc];
+        if (tid < SC::VEC / 16)
+            cpa16(d + 2 * SC::TILE + 16 * tid, p.P0 + (bh * (nch + 1) + c) * NH + 4 * tid);
+        if (tid == NT - 1) cpa4(d + 2 * SC::TILE + SC::VEC, p.ctot + cc);
     };
-    fetch_rev(nch - 1);
-    for (int c = nch - 1; c >= 0; --c) {
+    __syncthreads();   // every thread is past its last read of the forward stages
+#pragma unroll
+    for (int i = 0; i < SCAN_KS - 1; ++i) {
+        if (i < nch) issue_rev(i);
+        cpa_commit();
+    }
+    for (int i = 0; i < nch; ++i) {
+        const int c = nch - 1 - i;
         const size_t cc = bh * nch + c;
-        uint16_t uc[16], gc[16];
-        float pcv[8];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            uc[i] = un[i];
-            gc[i] = gn[i];
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) pcv[i] = pn[i];
-        const float dec = ex2f(cn * kLog2e);
-        if (c > 0) fetch_rev(c - 1);
+        if (i > 0) __syncthreads();   // the stage read at i - 1 is free again
+        if (i + SCAN_KS - 1 < nch) issue_rev(i + SCAN_KS - 1);
+        cpa_commit();
+        cpa_wait<SCAN_KS - 1>();
+        __syncthreads();   // chunk c's stage is complete
+        const uint8_t* st = ring + (i % SCAN_KS) * SC::STAGE;
+        const uint16_t* ut = reinterpret_cast<const uint16_t*>(st);
+        const uint8_t* gs = st + SC::TILE;
+        const float* pt = reinterpret_cast<const float*>(st + 2 * SC::TILE);
+        const float dec = ex2f(pt[NH] * kLog2e);
         uint8_t* dt_ = reinterpret_cast<uint8_t*>(p.dgo) + cc * NP * 2;
         float s = 0.f;
 #pragma unroll
@@ -559,13 +585,13 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
             const int j = pg + NPG * kx;
             *reinterpret_cast<uint16_t*>(dt_ + sw128_off(2 * j, pc)) = to_bf(de[kx]);
             *reinterpret_cast<uint16_t*>(dt_ + sw128_off(2 * j + 1, pc)) = to_bf(dq[kx]);
-            const float g0 = __uint_as_float((uint32_t)gc[2 * kx] << 16);
-            const float g1 = __uint_as_float((uint32_t)gc[2 * kx + 1] << 16);
+            const float g0 = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(gs + sw128_off(2 * j, pc)) << 16);
+            const float g1 = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(gs + sw128_off(2 * j + 1, pc)) << 16);
             s = fmaf(de[kx], g0, fmaf(dq[kx], g1, s));
-            const float u0 = __uint_as_float((uint32_t)uc[2 * kx] << 16);
-            const float u1 = __uint_as_float((uint32_t)uc[2 * kx + 1] << 16);
+            const float u0 = __uint_as_float((uint32_t)ut[(2 * j) * kPc + pc] << 16);
+            const float u1 = __uint_as_float((uint32_t)ut[(2 * j + 1) * kPc + pc] << 16);
             float sn, cs;
-            __sincosf(pcv[kx], &sn, &cs);
+            __sincosf(pt[j], &sn, &cs);
             de[kx] = fmaf(dec, de[kx], fmaf(cs, u0, sn * u1));
             dq[kx] = fmaf(dec, dq[kx], fmaf(cs, u1, -sn * u0));
         }
@@ -574,7 +600,7 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
         __syncthreads();
         if (tid == 0) {
             float t = 0.f;
-            for (int i = 0; i < NW; ++i) t += red[c & 1][i];
+            for (int k = 0; k < NW; ++k) t += red[c & 1][k];
             p.q[cc] = dec * t;
         }
     }
@@ -1381,8 +1407,11 @@ cudaError_t launch_n(const TcBwd& p, long long units, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_grads_kernel<NST, RK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smg);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_scan_kernel<NST, RK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ScanCfg<NST>::SMEM);
+    if (e != cudaSuccess) return e;
     bwd_vu_kernel<NST, RK><<<(unsigned)units, VuCfg<NST>::NT, smv, s>>>(p);
-    bwd_scan_kernel<NST, RK><<<(unsigned)((size_t)p.a.batch * p.a.H), 4 * NST, 0, s>>>(p);
+    bwd_scan_kernel<NST, RK><<<(unsigned)((size_t)p.a.batch * p.a.H), 4 * NST, ScanCfg<NST>::SMEM, s>>>(p);
     bwd_grads_kernel<NST, RK><<<(unsigned)units, 256, smg, s>>>(p);
     const long long bhj = (long long)p.a.batch * p.a.H * (NST / 2);
     bwd_carry_kernel<<<(unsigned)((bhj + 255) / 256), 256, 0, s>>>(p, NST / 2);
