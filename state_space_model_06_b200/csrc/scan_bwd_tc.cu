@@ -271,18 +271,17 @@ __global__ void __launch_bounds__(256, 2) bwd_vu_kernel(const __grid_constant__ 
                                   ((((size_t)b * a.T + t) * a.H + h) * RK + row % RK) * kPc + (e & 7) * 8)
                             : make_uint4(0u, 0u, 0u, 0u);
         }
-#pragma unroll
-        for (int i = 0; i < TT; ++i) {
-            const long long t = t0 + sg * TT + i;
-            thv[i] = t < a.T ? a.theta[(((size_t)b * a.T + t) * a.G + g) * NH + j] : 0.f;
-        }
+        // row sg TPS + i holds rank i % R of token (sg TPS + i) / R (TPS is a multiple of R);
+        // a token's angle is loaded with its first rank's B and C pair
 #pragma unroll
         for (int i = 0; i < TPS; ++i) {
-            const int row = sg * TPS + i;
-            const long long t = t0 + row / RK;
+            const long long t = t0 + (sg * TPS + i) / RK;
+            if (i % RK == 0) thv[i / RK] = 0.f;
             pbv[i] = pcv[i] = 0u;
             if (t < a.T) {
-                const size_t o = ((((size_t)b * a.T + t) * a.G + g) * RK + row % RK) * NST + 2 * j;
+                const size_t tr = ((size_t)b * a.T + t) * a.G + g;
+                if (i % RK == 0) thv[i / RK] = a.theta[tr * NH + j];
+                const size_t o = (tr * RK + i % RK) * NST + 2 * j;
                 pbv[i] = *reinterpret_cast<const uint32_t*>(Bg + o);
                 pcv[i] = *reinterpret_cast<const uint32_t*>(Cg + o);
             }
