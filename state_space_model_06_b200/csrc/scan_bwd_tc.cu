@@ -776,11 +776,34 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     if constexpr (RK > 1)
         for (int i = tid; i < QT * NH; i += 256) dpsi[i] = 0.f;
     // Every global input of the chunk is requested before any of it is used: the angle
-    // prefix's theta and dt, the chunk-start angle, the X and dY rows; then, behind the first
-    // barrier, the B and C pairs of the rotation while the angle offsets are formed.
+    // prefix's theta and dt, the chunk-start angle, the X and dY rows, and the B and C pairs
+    // of the rotation (with N = 128 those come behind the first barrier, while the angle
+    // offsets are formed, to keep the registers in flight under the budget of two CTAs).
     constexpr int SEGS = 256 / NH, TPS = QT / SEGS;   // tokens of a (pair, segment)
     static_assert(TPS * SEGS == QT, "whole tokens per segment");
     const int jj = tid % NH, sg = tid / NH;
+    // B~, C~ in the call frame: thread (pair jr, tile rows ur + RS m) for m < KT
+    constexpr int KT = kQ * NH / 256, RS = 256 / NH;
+    constexpr bool BC_EARLY = NST == 64;
+    const int jr = tid % NH, ur = tid / NH;
+    uint32_t pbv[KT], pcv[KT];
+    auto load_bc = [&]() {
+        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
+        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
+#pragma unroll
+        for (int m = 0; m < KT; ++m) {
+            const int rw = ur + RS * m;
+            const long long t = t0 + rw / RK;
+            pbv[m] = pcv[m] = 0u;
+            if (t < a.T) {
+                const size_t o = ((((size_t)b * a.T + t) * a.G + g) * RK + rw % RK) * NST + 2 * jr;
+                pbv[m] = *reinterpret_cast<const uint32_t*>(Bg + o);
+                pcv[m] = *reinterpret_cast<const uint32_t*>(Cg + o);
+            }
+        }
+    };
+    const float p0 = p.P0[(bh * (p.nch + 1) + c) * NH + jj];
+    if constexpr (BC_EARLY) load_bc();
     float rho[TPS];
     {
         float thv[TPS], dtv[TPS];
@@ -824,25 +847,9 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
         }
     }
     __syncthreads();
-    // B~, C~ in the call frame: thread (pair jr, tile rows ur + RS m) for m < KT
-    constexpr int KT = kQ * NH / 256, RS = 256 / NH;
-    const int jr = tid % NH, ur = tid / NH;
-    uint32_t pbv[KT], pcv[KT];
     {
-        const uint16_t* Bg = static_cast<const uint16_t*>(a.B);
-        const uint16_t* Cg = static_cast<const uint16_t*>(a.C);
-#pragma unroll
-        for (int m = 0; m < KT; ++m) {
-            const int rw = ur + RS * m;
-            const long long t = t0 + rw / RK;
-            pbv[m] = pcv[m] = 0u;
-            if (t < a.T) {
-                const size_t o = ((((size_t)b * a.T + t) * a.G + g) * RK + rw % RK) * NST + 2 * jr;
-                pbv[m] = *reinterpret_cast<const uint32_t*>(Bg + o);
-                pcv[m] = *reinterpret_cast<const uint32_t*>(Cg + o);
-            }
-        }
-        float off = p.P0[(bh * (p.nch + 1) + c) * NH + jj];
+        if constexpr (!BC_EARLY) load_bc();
+        float off = p0;
         for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + jj];
 #pragma unroll
         for (int i = 0; i < TPS; ++i) psi0[psi_idx<NH>(sg * TPS + i, jj)] = wrap_angle(off + rho[i]);
