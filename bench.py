@@ -412,6 +412,8 @@ def mimo_leg(args, dev, stream, rank, ws_world, pk):
     plus the fused gate; then its backward pass (16-token chunks of 64 (token, rank) rows).
     Algorithmic bytes count each tensor as the call reads it."""
     w = inputs.WORKLOADS["mimo_prefill_r4"]
+    if args.batch or args.seqlen:   # profiler captures only, as for the prefill line
+        w = dataclasses.replace(w, batch=args.batch or w.batch, seqlen=args.seqlen or w.seqlen)
     inp, d, g, st, y, ws = prefill_setup(w, dev, seed=200 + rank)
     del inp
     byts, _ = scan_algorithmic(w)
