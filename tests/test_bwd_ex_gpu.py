@@ -4,8 +4,9 @@ on the same rounded inputs.
 
 The GPU forms the effective inputs in the io dtype (as the fused forward kernels use them),
 reruns the ungated forward for the gate's derivative, runs the recurrence backward (the
-chunked tensor-core one for SISO bf16 P 64, the sequential fp32 one otherwise) and maps the
-gradients back.  Bars: 2e-2 of each gradient's largest value for bf16 inputs, 2e-4 for fp32.
+chunked tensor-core one for bf16 P 64 with SISO N 64 / 128 or MIMO R 2 / 4 N 64, the sequential
+fp32 one otherwise) and maps the gradients back.  Bars: 2e-2 of each gradient's largest value
+for bf16 inputs, 2e-4 for fp32.
 """
 import math
 
