@@ -492,11 +492,12 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
     }
     for (int c = 0; c < nch; ++c) {
         const size_t cc = bh * nch + c;
-        __syncthreads();   // the stage read at c - 1 is free again
+        cpa_wait<SCAN_KS - 2>();   // this thread's copies of chunk c have landed
+        // one barrier: chunk c's stage is complete, and every thread is done with the stage of
+        // chunk c - 1, which the next copies refill
+        __syncthreads();
         if (c + SCAN_KS - 1 < nch) issue_fwd(c + SCAN_KS - 1);
         cpa_commit();
-        cpa_wait<SCAN_KS - 1>();
-        __syncthreads();   // chunk c's stage is complete
         const uint8_t* st = ring + (c % SCAN_KS) * SC::STAGE;
         const uint16_t* vt = reinterpret_cast<const uint16_t*>(st);
         const float* at = reinterpret_cast<const float*>(st + 2 * SC::TILE);
@@ -564,14 +565,24 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
         if (i < nch) issue_rev(i);
         cpa_commit();
     }
+    // q of chunk c: the warps' partial sums in red[c & 1], added by thread 0 behind the next
+    // barrier (the next step writes the other half)
+    float dec_prev = 0.f;
+    auto finish_q = [&](int c) {
+        float t = 0.f;
+        for (int k = 0; k < NW; ++k) t += red[c & 1][k];
+        p.q[bh * nch + c] = dec_prev * t;
+    };
     for (int i = 0; i < nch; ++i) {
         const int c = nch - 1 - i;
         const size_t cc = bh * nch + c;
-        if (i > 0) __syncthreads();   // the stage read at i - 1 is free again
+        cpa_wait<SCAN_KS - 2>();   // this thread's copies of chunk c have landed
+        // one barrier: chunk c's stage is complete, every thread is done with the stage of
+        // step i - 1 (refilled next), and the partial sums of chunk c + 1 are in red
+        __syncthreads();
+        if (tid == 0 && i > 0) finish_q(c + 1);
         if (i + SCAN_KS - 1 < nch) issue_rev(i + SCAN_KS - 1);
         cpa_commit();
-        cpa_wait<SCAN_KS - 1>();
-        __syncthreads();   // chunk c's stage is complete
         const uint8_t* st = ring + (i % SCAN_KS) * SC::STAGE;
         const uint16_t* ut = reinterpret_cast<const uint16_t*>(st);
         const uint8_t* gs = st + SC::TILE;
@@ -596,13 +607,10 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
         }
         s = warp_sum(s);
         if (lane == 0) red[c & 1][w] = s;
-        __syncthreads();
-        if (tid == 0) {
-            float t = 0.f;
-            for (int k = 0; k < NW; ++k) t += red[c & 1][k];
-            p.q[cc] = dec * t;
-        }
+        dec_prev = dec;
     }
+    __syncthreads();
+    if (tid == 0) finish_q(0);   // before the starting-state sums below reuse red[0]
     // the starting state: dh0 = dg; dx_prev,r = k0 B_prev,r^T dg; dB_prev,r += k0 dg x_prev,r;
     // v0 = sum_r <dg, B_prev,r x_prev,r^T> (for dt_0 and lam_0)
     float pp[RK];
