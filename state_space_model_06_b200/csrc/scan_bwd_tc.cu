@@ -155,6 +155,13 @@ __device__ void chunk_coefs(const BwdArgs& a, int b, int h, long long t0, const 
     const int lane = threadIdx.x & 31;
     const long long T = a.T;
     float d2[2], l2[2], a2[2];
+    // with QT = 64 the next token has no slot of its own: lane 0 requests it with its tokens
+    float dn = 0.f, ln = 0.f;
+    if (QT == kQ && lane == 0 && t0 + kQ < T) {
+        const size_t o = ((size_t)b * T + t0 + kQ) * a.H + h;
+        dn = a.dt[o];
+        ln = a.lam[o];
+    }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const int u = 2 * lane + i;
@@ -188,11 +195,8 @@ __device__ void chunk_coefs(const BwdArgs& a, int b, int h, long long t0, const 
         k.ff[u] = in ? ex2f(cc[i] * kLog2e) : 0.f;
     }
     if (QT == kQ && lane == 0) {
-        const long long t = t0 + kQ;
-        const bool ok = t < T;
-        const size_t o = ((size_t)b * T + (ok ? t : 0)) * a.H + h;
-        k.dd[kQ] = ok ? a.dt[o] : 0.f;
-        k.ll[kQ] = ok ? a.lam[o] : 0.f;
+        k.dd[kQ] = dn;
+        k.ll[kQ] = ln;
     }
     __syncwarp();
 #pragma unroll
