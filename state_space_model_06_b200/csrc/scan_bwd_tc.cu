@@ -789,8 +789,8 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
         for (int i = tid; i < QT * NH; i += 256) dpsi[i] = 0.f;
     // Every global input of the chunk is requested before any of it is used: the angle
     // prefix's theta and dt, the chunk-start angle, the X and dY rows, and the B and C pairs
-    // of the rotation (with N = 128 those come behind the first barrier, while the angle
-    // offsets are formed, to keep the registers in flight under the budget of two CTAs).
+    // of the rotation (with N = 128 those follow once the angle prefix has consumed theta and
+    // dt, to keep the registers in flight under the budget of two CTAs).
     constexpr int SEGS = 256 / NH, TPS = QT / SEGS;   // tokens of a (pair, segment)
     static_assert(TPS * SEGS == QT, "whole tokens per segment");
     const int jj = tid % NH, sg = tid / NH;
@@ -850,6 +850,8 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
             rho[i] = r;
         }
         segt[sg * NH + jj] = r;
+        // theta and dt are consumed: their registers take the B and C pairs
+        if constexpr (!BC_EARLY) load_bc();
 #pragma unroll
         for (int m = 0; m < XT; ++m) {
             const int i = tid + 256 * m;
@@ -860,7 +862,6 @@ __global__ void __launch_bounds__(256, 2) bwd_grads_kernel(const __grid_constant
     }
     __syncthreads();
     {
-        if constexpr (!BC_EARLY) load_bc();
         float off = p0;
         for (int s2 = 0; s2 < sg; ++s2) off += segt[s2 * NH + jj];
 #pragma unroll
