@@ -104,7 +104,8 @@ def test_gradients_match_materialised_form_derivative(angle, R, G):
 
 
 @pytest.mark.parametrize("angle,R,G,chunk,T", [(False, 2, 1, 4, 13), (True, 1, 2, 5, 12),
-                                                (False, 3, 2, 3, 10), (False, 1, 1, 16, 9)])
+                                                (False, 3, 2, 3, 10), (False, 1, 1, 16, 9),
+                                                (False, 4, 1, 16, 37)])   # 64 (token, rank) rows
 def test_gradients_match_chunked_form_derivative(angle, R, G, chunk, T):
     """The chunked backward (adjoint state between chunks in the call's rotated frame,
     materialised-form derivative inside each chunk; tests/routes.py) equals the oracle's
