@@ -28,11 +28,13 @@
 //          dC~ = dS B~ + diag(f) dY g^T,      dB~ = dS^T C~ + diag(e w) X dg^T,
 //      rotated back by R(psi); the log-decay, band-weight and angle chains from row and
 //      column sums of the same tiles;
-//   4. finish, per (batch, head, chunk): the angle gradient carried from later chunks and the
-//      next token's share of the trapezoid weight w of the chunk's last token.
+//   4. carry, per (batch, head, pair): the angle gradient carried into every chunk from later
+//      chunks; finish, per (batch, chunk, group): dtheta summed over the group's heads in a
+//      fixed order, dt's angle term, and the next token's share of the trapezoid weight w of
+//      the previous chunk's last token.
 // Every reverse-mode term is the one the oracle's chunked route takes; the group-shared
-// gradients (B, C, theta, B_prev) and dD are added with atomics, so their last bits may vary
-// from run to run.  Every wait is bounded; a timeout writes M3_ERR_TIMEOUT to the status word.
+// gradients B, C, B_prev and dD are added with atomics, so their last bits may vary from run
+// to run.  Every wait is bounded; a timeout writes M3_ERR_TIMEOUT to the status word.
 #include <cuda_bf16.h>
 
 #include "m3_internal.h"
