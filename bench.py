@@ -6,12 +6,17 @@ i.e. every prefill step of the method.  Alongside, as sub-metrics: the batch-256
 workloads (SISO N 128 and MIMO R 4 N 64; 1000 sequential steps with fresh tokens, captured
 once as a CUDA graph and replayed), the same prefill and decode with the fused output gate
 ("gated") and with BCNorm + BC biases ("bc"), the MIMO rank-4 prefill plain and with the
-lightweight expansion of x and z ("mimo"), the long-context workload of 16 chained calls
+lightweight expansion of x and z, and its backward pass ("mimo"), the long-context workload of
+16 chained calls
 ("longctx") and the fp32 parity workload ("small_f32"), the backward pass of the prefill
 workload ("backward"), the end-to-end call through pinned host
 buffers ("e2e"), and the CPU oracle on the workload's inputs ("cpu_baseline").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Profiling subsets (their lines are not measurements of the full set): --prefill-only,
+--bwd-only (the prefill line and the SISO backward), --mimo-only (the prefill line and the
+MIMO leg); --batch / --seqlen shrink the workloads for short ncu captures.
 
 N > 1 runs one independent replica per GPU (the path has no cross-GPU exchange:
 every (batch, head) recurrence is independent), launched with torch.distributed.run;
