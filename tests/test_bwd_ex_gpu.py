@@ -33,6 +33,7 @@ CASES = [
     (1, 4, 1, 64, 128, 1, 130, torch.bfloat16, None, True, EPS, False, 2e-2),
     (1, 4, 2, 64, 128, 1, 90, torch.bfloat16, "exp", True, EPS, True, 2e-2),
     (1, 4, 1, 64, 64, 4, 70, torch.bfloat16, "exp", True, EPS, True, 2e-2),
+    (1, 4, 2, 64, 64, 2, 90, torch.bfloat16, "plain", True, EPS, False, 2e-2),
     (1, 4, 2, 8, 6, 2, 40, torch.float32, "exp", True, EPS, True, 2e-4),
     (2, 2, 1, 16, 16, 1, 33, torch.float32, "plain", True, 0.0, False, 2e-4),
 ]

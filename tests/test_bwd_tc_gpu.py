@@ -138,10 +138,11 @@ def test_tc_backward_mimo_matches_oracle(case):
     assert all(e <= TOL for e in errs.values()), errs
 
 
-def test_tc_backward_mimo_against_sequential_kernel():
-    """Rank 4: the chunked path against the sequential fp32 kernel on the same inputs."""
-    inp, dy, dh = _problem(1, 4, 1, 64, 203, seed=66, R=4)
-    d = m3.Dims(1, 4, 1, 64, 64, 4, m3.M3_BF16)
+@pytest.mark.parametrize("R", [2, 4])
+def test_tc_backward_mimo_against_sequential_kernel(R):
+    """Ranks 2 and 4: the chunked path against the sequential fp32 kernel on the same inputs."""
+    inp, dy, dh = _problem(1, 4, 1, 64, 203, seed=66, R=R)
+    d = m3.Dims(1, 4, 1, 64, 64, R, m3.M3_BF16)
     tc = _gpu_bwd(inp, dy, dh, d, 203)
     seq = _gpu_bwd(inp, dy, dh, d, 203, flags=m3.M3_FLAG_FORCE_SIMT)
     errs = _slice_errors(tc, seq)
