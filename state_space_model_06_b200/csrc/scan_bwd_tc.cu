@@ -672,6 +672,8 @@ __global__ void __launch_bounds__(4 * NST, NST == 128 ? 1 : 2) bwd_scan_kernel(c
 //   2. dC~ += dS B~, B~ dg;                    epilogue: dC~ rotated back (dC), angle terms;
 //                                              <X_s, (B~ dg)_s>, row scale e w; X <- e w X
 //   3. dX = (L o S)^T dY + ., dB~ = (e w X) dg^T + dS^T C~;   epilogue: dX, dB
+// Tile rows are (token, rank) pairs, 64 / R tokens of R ranks: the masks and scales are the
+// row's token's, and the per-token sums (band weights, log-decay, angles) gather its R rows.
 template <int NST, int RK>
 struct GrCfg {
     static constexpr int NH = NST / 2;
