@@ -85,6 +85,11 @@ def test_gradients_match_finite_differences(angle):
     assert _max_fd_error(3 + angle, angle) < 1e-7
 
 
+def test_gradients_match_finite_differences_rank4():
+    """R = 4 (the rank of the MIMO workloads), two groups of one head each."""
+    assert _max_fd_error(11, False, b=1, T=5, H=2, G=2, P=3, N=4, R=4) < 1e-7
+
+
 def test_gradients_match_finite_differences_siso_groups():
     """R = 1, two groups of two heads, odd headdim."""
     assert _max_fd_error(9, False, b=1, T=6, H=4, G=2, P=5, N=6, R=1) < 1e-7
